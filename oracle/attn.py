@@ -1,0 +1,77 @@
+"""Dequantization and exact decode attention in fp64 (oracle; test only).
+
+"RoPE-Aware Bit Allocation for KV-Cache Quantization", abstract: the
+packed-cache serving path runs decode attention over the packed K/V cache.
+Here that is written as its plain definition on the dequantized cache:
+
+    k_hat_i = n^K * a_hat_j * c_{b_j}[code_i]          (0 for b_j = 0)
+    v_hat   = n^V * (1/d) * s . (H c_{b_V}[codes])      (H H = d I)
+    o_h     = sum_t softmax_t(q_h . k_hat_t / sqrt d) v_hat_t
+
+over the L cached tokens (no mask: a decode query attends to every cached
+token). Query head h reads KV head floor(h / G), G = H_q / H_kv. A sequence
+with no cached token gives o = 0.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import lloydmax
+
+
+def hadamard(d: int = 128) -> np.ndarray:
+    """Sylvester Hadamard matrix, H[i, j] = (-1)^popcount(i & j)."""
+    i = np.arange(d)
+    x = i[:, None] & i[None, :]
+    pc = np.zeros_like(x)
+    while np.any(x):
+        pc += x & 1
+        x >>= 1
+    return np.where(pc % 2 == 0, 1.0, -1.0)
+
+
+def dequant_keys(codes, norms, plan) -> np.ndarray:
+    codes = np.asarray(codes)
+    T, d = codes.shape
+    half = d // 2
+    out = np.zeros((T, d), dtype=np.float64)
+    n = np.asarray(norms, dtype=np.float64)
+    for j in range(half):
+        w = int(plan.widths[j])
+        if w == 0:
+            continue
+        c = lloydmax.centroids(w)
+        for i in (j, j + half):
+            out[:, i] = n * float(plan.a_hat[j]) * c[codes[:, i]]
+    return out
+
+
+def dequant_values(codes, norms, plan) -> np.ndarray:
+    codes = np.asarray(codes)
+    d = codes.shape[1]
+    c = lloydmax.centroids(plan.bits_v)
+    y = c[codes] * np.asarray(norms, dtype=np.float64)[:, None]
+    return (y @ hadamard(d)) * plan.signs[None, :] / d
+
+
+def attention(q, k_hat, v_hat) -> np.ndarray:
+    """softmax(q k_hat^T / sqrt d) v_hat for one KV head; q[Hg, d]."""
+    q = np.asarray(q, dtype=np.float64)
+    if k_hat.shape[0] == 0:
+        return np.zeros_like(q)
+    s = q @ k_hat.T / np.sqrt(q.shape[-1])
+    s = s - s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    p /= p.sum(axis=1, keepdims=True)
+    return p @ v_hat
+
+
+def decode(q, k_hat_heads, v_hat_heads) -> np.ndarray:
+    """GQA decode for one sequence: q[Hq, d], per-KV-head dequantized caches."""
+    q = np.asarray(q, dtype=np.float64)
+    hkv = len(k_hat_heads)
+    G = q.shape[0] // hkv
+    out = np.zeros_like(q)
+    for h in range(hkv):
+        out[h * G:(h + 1) * G] = attention(q[h * G:(h + 1) * G], k_hat_heads[h], v_hat_heads[h])
+    return out

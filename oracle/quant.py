@@ -1,0 +1,133 @@
+"""TQ-MSE style quantizers for keys and values (oracle; test infrastructure).
+
+"RoPE-Aware Bit Allocation for KV-Cache Quantization", abstract: Block-GTQ is a
+bit allocator for key-cache quantization built on TurboQuant-MSE; keys get
+per-RoPE-block integer widths, values keep the uniform TQ-MSE quantizer at the
+matched value budget. TQ-MSE normalises a vector, rotates it so coordinates
+are near Gaussian, and applies an MSE-optimal scalar codebook per coordinate.
+The related-papers page ("Related papers: Quantization Dominates Rank
+Reduction for KV-Cache...", the KV/KQV/QKQV scheme summary) and the KVLinC
+summary (Hadamard rotation on values) support a Walsh-Hadamard rotation.
+
+Readings adopted:
+
+Keys (per token, per KV head). No rotation across blocks (it would mix the
+blocks whose widths differ). n = fp16 norm of the whole 128-vector; each
+coordinate i of block j is scaled to z_i = k_i * (1/n) * g_j and coded with
+the width-b_j Lloyd-Max thresholds.
+
+Values. y = H (s . v), H the unnormalised 128-point Sylvester Hadamard matrix,
+s the +-1 signs of the plan; n = fp16 norm of v; z_i = y_i * (1/n) (each y_i
+has variance |v|^2); coded with the uniform width b_V.
+
+Decision arithmetic (IEEE fp32, no fused multiply-add, fixed order):
+* the input is bf16/fp16/fp32; x*x is exact in fp32 for bf16 and fp16 inputs;
+* sumsq: with lane l = 0..31 holding coordinates l, l+32, l+64, l+96,
+  p_l = ((x_l^2 + x_{l+32}^2) + x_{l+64}^2) + x_{l+96}^2, then for
+  m = 16, 8, 4, 2, 1: p_l <- p_l + p_{l xor m}; the sum is p_0;
+* n = fp16_RNE(sqrt_RN(sumsq)); if that overflows, n = 65504 and the
+  NORM_SAT flag is raised; r = 1/n rounded to nearest;
+* keys: z_i = (k_i * r) * g_j; values: z_i = y_i * r;
+* code = number of thresholds t with t < z (strict), i.e. ties go low;
+* n = 0 gives all codes 0; a token with any non-finite coordinate is stored
+  as n = 0, codes 0, and raises NONFINITE;
+* FWHT: stages h = 1, 2, 4, ..., 64; for every i with (i & h) == 0 the pair
+  (a, b) = (x_i, x_{i+h}) becomes (a + b, a - b), in fp32.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import lloydmax
+
+FLAG_NONFINITE = 2
+FLAG_NORM_SAT = 4
+F16_MAX = 65504.0
+
+
+def sumsq_tree(x32: np.ndarray) -> np.ndarray:
+    """Fixed-order fp32 sum of squares over the last axis (length 128)."""
+    x32 = np.asarray(x32, dtype=np.float32)
+    sq = x32 * x32
+    p = ((sq[..., 0:32] + sq[..., 32:64]) + sq[..., 64:96]) + sq[..., 96:128]
+    lane = np.arange(32)
+    for m in (16, 8, 4, 2, 1):
+        p = p + p[..., lane ^ m]
+    return p[..., 0]
+
+
+def fp16_norm(sumsq: np.ndarray):
+    """(n as float32 holding an fp16 value, NORM_SAT mask)."""
+    s = np.sqrt(np.asarray(sumsq, dtype=np.float32))
+    with np.errstate(over="ignore"):
+        n16 = s.astype(np.float16)
+    sat = np.isinf(n16)
+    n16 = np.where(sat, np.float16(F16_MAX), n16)
+    return n16.astype(np.float32), sat
+
+
+def codes_from_z(z: np.ndarray, bits: int) -> np.ndarray:
+    """Number of width-``bits`` thresholds strictly below z (NaN -> 0)."""
+    thr = lloydmax.thresholds(bits)
+    c = np.searchsorted(thr, np.asarray(z, dtype=np.float32), side="left")
+    return np.where(np.isnan(z), 0, c).astype(np.int64)
+
+
+def fwht_f32(x: np.ndarray) -> np.ndarray:
+    """Unnormalised Walsh-Hadamard transform along the last axis, fp32 graph."""
+    y = np.array(x, dtype=np.float32, copy=True)
+    d = y.shape[-1]
+    h = 1
+    while h < d:
+        idx = np.array([i for i in range(d) if (i & h) == 0])
+        a = y[..., idx].copy()
+        b = y[..., idx + h].copy()
+        y[..., idx] = a + b
+        y[..., idx + h] = a - b
+        h *= 2
+    return y
+
+
+def _norm_and_recip(x32):
+    """Per-token n (fp16 value in float32), r = 1/n, and flags."""
+    fin = np.all(np.isfinite(x32), axis=-1)
+    x_safe = np.where(fin[..., None], x32, np.float32(0))
+    n, sat = fp16_norm(sumsq_tree(x_safe))
+    n = np.where(fin, n, np.float32(0))
+    with np.errstate(divide="ignore"):
+        r = np.float32(1.0) / n
+    flags = np.where(~fin, FLAG_NONFINITE, 0) | np.where(sat & fin, FLAG_NORM_SAT, 0)
+    return n, r, fin, flags
+
+
+def quantize_keys(k, plan):
+    """Key codes [T, 128] (canonical coords; unused for width-0 blocks), fp16
+    norms as float32 [T], per-token flags [T]."""
+    k32 = np.asarray(k, dtype=np.float32)
+    T, d = k32.shape
+    half = d // 2
+    n, r, fin, flags = _norm_and_recip(k32)
+    codes = np.zeros((T, d), dtype=np.int64)
+    live = fin & (n > 0)
+    with np.errstate(invalid="ignore", over="ignore"):
+        for j in range(half):
+            w = int(plan.widths[j])
+            if w == 0:
+                continue
+            for i in (j, j + half):
+                z = (k32[:, i] * r) * plan.g[j]
+                codes[:, i] = np.where(live, codes_from_z(z, w), 0)
+    return codes, n, flags
+
+
+def quantize_values(v, plan):
+    """Value codes [T, 128] (rotated coords), fp16 norms [T], flags [T]."""
+    v32 = np.asarray(v, dtype=np.float32)
+    n, r, fin, flags = _norm_and_recip(v32)
+    sv = np.where(plan.signs[None, :] < 0, -v32, v32).astype(np.float32)
+    y = fwht_f32(np.where(fin[:, None], sv, np.float32(0)))
+    with np.errstate(invalid="ignore", over="ignore"):
+        z = y * r[:, None]
+    live = fin & (n > 0)
+    codes = np.where(live[:, None], codes_from_z(z, plan.bits_v), 0)
+    return codes, n, flags
