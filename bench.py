@@ -1,0 +1,424 @@
+#!/usr/bin/env python
+"""Benchmark of the packed KV-cache decode path on B200.
+
+Workload (default): Qwen2.5-3B-shaped stack, 36 layers, 16 query / 2 KV
+heads, head size 128, RoPE theta 1e6, batch 1, 128K context, K3V3 Block-GTQ
+plans. Synthetic seeded inputs (synth.keys_values_torch); caches are built by
+the library itself (energy + greedy plans + bulk quantize-append) before the
+timed region.
+
+Step = one decode step of the whole stack: per layer, quantize-append the new
+token's key and value (1 token x 2 KV heads) and run packed decode attention
+over the layer's cache (decode + split combine). The step is captured in a
+CUDA graph. ``value`` = packed cache bytes read by decode attention per step
+/ step time (GB/s). The packed caches of the 36 layers (944 MB) exceed L2, and
+each layer's cache is read once per step, so no L2 flush is needed.
+
+Also reported: decode-kernel roofline (CUDA events around each layer's
+decode call, outside the graph), bulk quantize throughput (prefill), an e2e
+step through host buffers, SM clocks during the timed region, and the CPU
+oracle timed on a bounded sample of the same workload.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvq|reference]
+Under torchrun each rank runs the same per-GPU work (weak scaling, no
+data-path collective); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+BYTES_PER_TOKEN_HEAD = lambda bk, bv: 16 * (bk + bv) + 4  # noqa: E731  codes + 2 fp16 norms
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--workload", default="qwen3b_128k",
+                    choices=["qwen3b_128k", "llama8b", "qwen7b_serve"])
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ helpers
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def decode_source_hash():
+    h = hashlib.sha256()
+    for f in ("decode.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "bit_kv_cache_19_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """Per-launch DRAM bytes of the decode kernel from a committed ncu summary,
+    only if it was taken on the current decode source."""
+    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("source_hash") != decode_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------- CPU oracle
+def oracle_sample(wl, seconds_target=12.0, seed=0):
+    """Time the oracle's decode (unpack + dequantize + exact attention) on a
+    bounded sample: one layer, one KV head and its G query heads, over
+    contexts of 8K tokens, repeated until ~seconds_target of CPU work."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import oracle_pipeline as op  # noqa: F401
+    from oracle import alloc, attn, energy, layout, quant
+
+    T = 8192
+    G = wl.n_q_heads // wl.n_kv_heads
+    kb, vb = synth.keys_values(wl, seed, 0, 0, T)
+    k, v = synth.bf16_bits_to_f64(kb), synth.bf16_bits_to_f64(vb)
+    E, _ = energy.block_energy(k[:, None, :])
+    plan = alloc.make_plan(E[0], wl.bits_k, wl.bits_v, 1, 0, 0)
+    kc, kn, _ = quant.quantize_keys(k, plan)
+    vc, vn, _ = quant.quantize_values(v, plan)
+    rec = layout.pack(kc, vc, kn, vn, plan, T)
+    q = synth.bf16_bits_to_f64(synth.queries(wl, seed, 0, 0, T))[:G]
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        kc2, vc2, kn2, vn2 = layout.unpack(rec, plan, T)
+        kh = attn.dequant_keys(kc2, kn2, plan)
+        vh = attn.dequant_values(vc2, vn2, plan)
+        attn.attention(q, kh, vh)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds_target:
+            break
+    bytes_done = reps * T * BYTES_PER_TOKEN_HEAD(wl.bits_k, wl.bits_v)
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = 1
+    return {"value": bytes_done / el / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{reps} x (1 layer, 1 KV head + {G} query heads, {T} tokens, "
+                      f"K{wl.bits_k}V{wl.bits_v}): unpack + dequantize + exact fp64 attention",
+            "seconds": el}
+
+
+# --------------------------------------------------------------- main paths
+def run_reference(args, wl, rank, world):
+    if rank != 0:
+        return
+    steps, warmup = args.steps, args.warmup
+    times = []
+    per = max(1.0, min(10.0, 120.0 / max(1, steps + warmup)))
+    for i in range(warmup + steps):
+        r = oracle_sample(wl, seconds_target=per, seed=args.seed)
+        if i >= warmup:
+            times.append(r)
+    val = statistics.mean(r["value"] for r in times)
+    line = {
+        "impl": "reference", "metric": f"packed K{wl.bits_k}V{wl.bits_v} decode-attn HBM GB/s",
+        "value": val, "unit": "GB/s", "n_gpus": world, "steps": steps, "warmup": warmup,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "layers": wl.n_layers, "q_heads": wl.n_q_heads,
+                   "kv_heads": wl.n_kv_heads, "context": wl.context, "batch": wl.batch,
+                   "budget": f"K{wl.bits_k}V{wl.bits_v}"},
+        "cpu_baseline": {"value": val, "unit": "GB/s", "cores": times[0]["cores"],
+                         "kind": "oracle", "sample": times[0]["sample"]},
+        "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_kvq(args, wl, rank, world, dist):
+    import torch
+
+    from bit_kv_cache_19_b200 import kvq
+    from bit_kv_cache_19_b200.runtime import PackedLayer
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    n_layers, B, T = wl.n_layers, wl.batch, wl.context
+    steps, warmup = args.steps, args.warmup
+    cap = T + steps + warmup + 64
+    cfg = kvq.make_cfg(wl.n_kv_heads, wl.bits_k, wl.bits_v, v_seed=1234)
+    bpth = BYTES_PER_TOKEN_HEAD(wl.bits_k, wl.bits_v)
+
+    # ---- prefill: energies + greedy plans, bulk quantize-append (timed)
+    layers = []
+    t_alloc = t_quant = 0.0
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for li in range(n_layers):
+        L = PackedLayer(cfg, B, cap, device=dev, layer=li)
+        ks, vs = [], []
+        for b in range(B):
+            k, v = synth.keys_values_torch(wl, args.seed * 1000 + rank * 100 + b, li, T, dev)
+            ks.append(k)
+            vs.append(v)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        L.alloc_bits(ks[0])
+        t_alloc += time.perf_counter() - t0
+        kall = torch.stack(ks)
+        vall = torch.stack(vs)
+        del ks, vs
+        ev0.record()
+        L.append(kall, vall)
+        ev1.record()
+        torch.cuda.synchronize()
+        t_quant += ev0.elapsed_time(ev1) / 1e3
+        assert L.flags() == 0, f"layer {li}: status flags {L.flags()}"
+        del kall, vall
+        layers.append(L)
+    torch.cuda.empty_cache()
+
+    # ---- decode inputs (device resident) and static new-token buffers
+    qs = [synth.queries_torch(wl, args.seed, li, B, T, dev) for li in range(n_layers)]
+    knew = [torch.randn(B, 1, wl.n_kv_heads, 128, device=dev).to(torch.bfloat16)
+            for _ in range(n_layers)]
+    vnew = [torch.randn(B, 1, wl.n_kv_heads, 128, device=dev).to(torch.bfloat16)
+            for _ in range(n_layers)]
+    outs = [torch.empty(B, wl.n_q_heads, 128, dtype=torch.float32, device=dev)
+            for _ in range(n_layers)]
+    ws = layers[0].workspace(wl.n_q_heads, cap)
+
+    def step():
+        for li, L in enumerate(layers):
+            L.append(knew[li], vnew[li])
+            kvq.decode_attn(cfg, L.plan_ptrs, L.cache_ptrs, L.lens, cap, qs[li], outs[li], ws,
+                            L.status)
+
+    stream = torch.cuda.Stream(device=dev)
+    graph = None
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            step()
+        stream.synchronize()
+        if not args.no_graph:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                step()
+        len_before = int(layers[0].lens[0].item())
+        sampler = ClockSampler(dev.index)
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        sampler.start()
+        time.sleep(0.3)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            graph.replay() if graph is not None else step()
+        e1.record(stream)
+        e1.synchronize()
+        torch.cuda.synchronize()
+        clocks = sampler.stop()
+        ms = e0.elapsed_time(e1) / steps
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    # packed bytes read per step: length grows by 1 per step
+    lens_timed = [len_before + i + 1 for i in range(steps)]
+    bytes_step = n_layers * B * wl.n_kv_heads * bpth * statistics.mean(lens_timed)
+    flags = 0
+    for L in layers:
+        flags |= L.flags()
+    assert flags == 0, f"status flags {flags}"
+    value = world * bytes_step / (ms / 1e3) / 1e9
+
+    # ---- decode kernel alone: events around each layer's decode call
+    per_launch = []
+    with torch.cuda.stream(stream):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n_layers * 3)]
+        for r in range(3):
+            for li, L in enumerate(layers):
+                a, b = evs[r * n_layers + li]
+                a.record(stream)
+                kvq.decode_attn(cfg, L.plan_ptrs, L.cache_ptrs, L.lens, cap, qs[li], outs[li],
+                                ws, L.status)
+                b.record(stream)
+        stream.synchronize()
+        per_launch = [a.elapsed_time(b) for a, b in evs[n_layers:]]  # skip first pass
+    launch_ms = statistics.mean(per_launch)
+    cur_len = int(layers[0].lens[0].item())
+    bytes_launch = B * wl.n_kv_heads * bpth * cur_len
+    peak, peak_kind = measured_peaks()
+    achieved = bytes_launch / (launch_ms / 1e3) / 1e9
+
+    # ---- e2e: host buffers, H2D of the step's inputs and D2H of its outputs
+    q_host = [q.cpu().pin_memory() for q in qs]
+    k_host = [k.cpu().pin_memory() for k in knew]
+    v_host = [v.cpu().pin_memory() for v in vnew]
+    o_host = [torch.empty_like(o, device="cpu").pin_memory() for o in outs]
+    h2d = sum(q.numel() * q.element_size() + k.numel() * k.element_size() * 2
+              for q, k in zip(q_host, k_host))
+    d2h = sum(o.numel() * o.element_size() for o in o_host)
+    with torch.cuda.stream(stream):
+        def e2e_step():
+            for li in range(n_layers):
+                qs[li].copy_(q_host[li], non_blocking=True)
+                knew[li].copy_(k_host[li], non_blocking=True)
+                vnew[li].copy_(v_host[li], non_blocking=True)
+            graph.replay() if graph is not None else step()
+            for li in range(n_layers):
+                o_host[li].copy_(outs[li], non_blocking=True)
+        for _ in range(2):
+            e2e_step()
+        stream.synchronize()
+        e2e_steps = max(3, steps // 2)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        f1.record(stream)
+        f1.synchronize()
+        e2e_ms = f0.elapsed_time(f1) / e2e_steps
+    e2e_len = int(layers[0].lens[0].item())
+    e2e_bytes = n_layers * B * wl.n_kv_heads * bpth * (e2e_len - e2e_steps / 2)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_val = world * e2e_bytes / (e2e_ms / 1e3) / 1e9
+
+    if rank != 0:
+        return
+    cpu = oracle_sample(wl, seconds_target=12.0, seed=args.seed) if world == 1 else None
+    n_tok_quant = n_layers * B * T
+    line = {
+        "metric": f"packed K{wl.bits_k}V{wl.bits_v} decode-attn HBM GB/s",
+        "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps, "warmup": warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16 mma, f32 accumulate (codes u8/u32)", "data": "synthetic",
+        "config": {"workload": wl.name, "layers": n_layers, "q_heads": wl.n_q_heads,
+                   "kv_heads": wl.n_kv_heads, "head_dim": 128, "context": T, "batch": B,
+                   "budget": f"K{wl.bits_k}V{wl.bits_v}", "alloc": "Block-GTQ greedy",
+                   "step": "per layer: quantize-append 1 token + packed decode attention",
+                   "l2": f"inputs larger than L2 ({n_layers}-layer packed cache "
+                         f"{n_layers * B * wl.n_kv_heads * bpth * T / 1e6:.0f} MB, each layer "
+                         "read once per step)",
+                   "graph": graph is not None},
+        "pct_of_8TBs": value / 8000.0 * 100,
+        "tokens_per_s": world * B / (ms / 1e3),
+        "quantize_prefill": {"layer_tokens_per_s": n_tok_quant / t_quant,
+                             "token_heads_per_s": n_tok_quant * wl.n_kv_heads / t_quant,
+                             "seconds": t_quant, "alloc_bits_seconds": t_alloc},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "traffic": profiled_traffic(wl.name),
+                     "kernel": "decode_attn (decode_kernel + combine_kernel)",
+                     "bytes_per_launch": bytes_launch, "launch_us": launch_ms * 1e3},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": steps * n_layers * 4,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    wl = synth.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if args.impl == "reference":
+        run_reference(args, wl, rank, world)
+        return
+    import torch
+
+    if world > 1:
+        import torch.distributed as tdist
+        from datetime import timedelta
+
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        tdist.init_process_group("nccl", timeout=timedelta(seconds=120))
+        dist = tdist
+    else:
+        torch.cuda.set_device(0)
+    try:
+        run_kvq(args, wl, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,311 @@
+// Host side of the libkvq C ABI: argument checks, the greedy allocator and
+// plan builder, and the kernel launches. See kvq.h for the contract.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+
+namespace kvq {
+cudaError_t launch_energy(const void* k, int dtype, int64_t n_tokens, int n_kv,
+                          unsigned long long* acc, uint32_t* status, cudaStream_t st);
+struct QuantParams {
+  const Plan* const* plans;
+  const void* k;
+  const void* v;
+  int dtype;
+  int batch, n_new, n_kv;
+  uint8_t* const* caches;
+  const int32_t* len;
+  int64_t cap;
+  int tile_bytes;
+  uint32_t* status;
+};
+cudaError_t launch_quantize_append(const QuantParams& p, cudaStream_t st);
+int decode_splits(int64_t max_len);
+cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches, const int32_t* len,
+                          int batch, int64_t max_len, const void* q, int q_dtype, int n_q, int n_kv,
+                          int bits_k, int bits_v, float* out, float* part, uint32_t* status,
+                          cudaStream_t st);
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  std::vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+  return fail(KVQ_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+const double kD[9] = KVQ_CB_D;
+const uint16_t kC16[KVQ_CB_N_C16] = KVQ_CB_C16;
+const float kThr[KVQ_CB_N_THR] = KVQ_CB_THR;
+
+int check_cfg(const kvq_cfg* cfg) {
+  if (!cfg) return fail(KVQ_ERR_ARG, "cfg is NULL");
+  if (cfg->head_dim != kHeadDim) return fail(KVQ_ERR_UNSUPPORTED, "head_dim %d (only 128)", cfg->head_dim);
+  if (cfg->n_kv_heads < 1 || cfg->n_kv_heads > 4096) return fail(KVQ_ERR_ARG, "n_kv_heads %d", cfg->n_kv_heads);
+  if (cfg->bits_k < 1 || cfg->bits_k > 8) return fail(KVQ_ERR_ARG, "bits_k %d not in 1..8", cfg->bits_k);
+  if (cfg->bits_v < 1 || cfg->bits_v > 8) return fail(KVQ_ERR_ARG, "bits_v %d not in 1..8", cfg->bits_v);
+  if (cfg->b_max != 8) return fail(KVQ_ERR_ARG, "b_max %d (must be 8)", cfg->b_max);
+  if (cfg->alloc_mode != KVQ_ALLOC_GREEDY && cfg->alloc_mode != KVQ_ALLOC_UNIFORM)
+    return fail(KVQ_ERR_ARG, "alloc_mode %d", cfg->alloc_mode);
+  return KVQ_OK;
+}
+
+bool dtype_ok(int dt) { return dt == KVQ_BF16 || dt == KVQ_FP16 || dt == KVQ_FP32; }
+
+// SplitMix64: n-th output of the stream seeded with s.
+uint64_t splitmix64(uint64_t s, uint64_t n) {
+  uint64_t z = s + (n + 1) * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// Greedy marginal-gain widths: bits_k * 64 steps from zero, each +1 bit to the
+// block with the largest E_j (D(b_j) - D(b_j + 1)) below 8 (first index wins).
+void greedy_widths(const double* E, int bits_k, uint8_t* w) {
+  int b[kBlocks] = {0};
+  for (int step = 0; step < kBlocks * bits_k; ++step) {
+    int best = -1;
+    double best_gain = 0.0;
+    for (int j = 0; j < kBlocks; ++j) {
+      if (b[j] >= 8) continue;
+      const double gain = E[j] * (kD[b[j]] - kD[b[j] + 1]);
+      if (best < 0 || gain > best_gain) {
+        best = j;
+        best_gain = gain;
+      }
+    }
+    b[best] += 1;
+  }
+  for (int j = 0; j < kBlocks; ++j) w[j] = (uint8_t)b[j];
+}
+
+void build_plan(const kvq_cfg* cfg, int layer, int kv_head, const double* E, Plan* pl) {
+  std::memset(pl, 0, sizeof(Plan));
+  pl->magic = KVQ_PLAN_MAGIC;
+  pl->bits_k = cfg->bits_k;
+  pl->bits_v = cfg->bits_v;
+  pl->layer = layer;
+  pl->kv_head = kv_head;
+  pl->words_k = 128 * cfg->bits_k;
+  pl->words_v = 128 * cfg->bits_v;
+  if (cfg->alloc_mode == KVQ_ALLOC_UNIFORM) {
+    for (int j = 0; j < kBlocks; ++j) pl->width[j] = (uint8_t)cfg->bits_k;
+  } else {
+    greedy_widths(E, cfg->bits_k, pl->width);
+  }
+  double tot = 0.0;
+  for (int j = 0; j < kBlocks; ++j) tot += E[j];
+  pl->energy_sum = tot;
+  for (int j = 0; j < kBlocks; ++j) {
+    const double a = tot > 0.0 ? std::sqrt(E[j] / (2.0 * tot)) : 0.0;
+    pl->a_hat[j] = (float)a;
+    pl->g[j] = a > 0.0 ? (float)(1.0 / a) : 0.f;
+  }
+  // plan order: nonzero widths, width descending, block index ascending
+  int ranks = 0;
+  for (int w = 8; w >= 1; --w)
+    for (int j = 0; j < kBlocks; ++j)
+      if (pl->width[j] == w) pl->order[ranks++] = (uint8_t)j;
+  pl->n_ranks = ranks;
+  int off = 0;
+  for (int r = 0; r < ranks; ++r) {
+    pl->seg_off[r] = (uint16_t)off;
+    off += 2 * pl->width[pl->order[r]];
+  }
+  pl->seg_off[ranks] = (uint16_t)off;
+  // decode schedule: runs of equal width cut into groups of at most 4 ranks
+  int nh = 0;
+  for (int r = 0; r < ranks;) {
+    const int w = pl->width[pl->order[r]];
+    int n = 0;
+    while (r + n < ranks && n < 4 && pl->width[pl->order[r + n]] == w) ++n;
+    pl->hs_width[nh] = (uint8_t)w;
+    pl->hs_rank0[nh] = (uint8_t)r;
+    pl->hs_count[nh] = (uint8_t)n;
+    ++nh;
+    r += n;
+  }
+  pl->n_half = (uint8_t)nh;
+  const uint64_t key = splitmix64(cfg->v_seed, ((uint64_t)(uint32_t)layer << 32) + (uint32_t)kv_head);
+  for (int i = 0; i < kHeadDim; ++i)
+    if (splitmix64(key, (uint64_t)i) >> 63) pl->v_sign[i >> 5] |= 1u << (i & 31);
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+}  // namespace kvq
+
+using namespace kvq;
+
+extern "C" {
+
+const char* kvq_version(void) { return "kvq 0.1 (sm_100a)"; }
+
+const char* kvq_last_error(void) { return g_err.c_str(); }
+
+size_t kvq_plan_bytes(void) { return KVQ_PLAN_BYTES; }
+
+size_t kvq_tile_bytes(const kvq_cfg* cfg) {
+  if (check_cfg(cfg) != KVQ_OK) return 0;
+  return (size_t)tile_bytes(cfg->bits_k, cfg->bits_v);
+}
+
+size_t kvq_cache_bytes(const kvq_cfg* cfg, int64_t cap_tokens) {
+  if (check_cfg(cfg) != KVQ_OK || cap_tokens < 0) return 0;
+  const size_t tiles = (size_t)((cap_tokens + kTile - 1) / kTile);
+  return tiles * cfg->n_kv_heads * (size_t)tile_bytes(cfg->bits_k, cfg->bits_v);
+}
+
+size_t kvq_alloc_workspace_bytes(const kvq_cfg* cfg) {
+  if (check_cfg(cfg) != KVQ_OK) return 0;
+  return align_up((size_t)cfg->n_kv_heads * kBlocks * 16, 256);
+}
+
+size_t kvq_decode_workspace_bytes(const kvq_cfg* cfg, int batch, int n_q_heads, int64_t max_len) {
+  if (check_cfg(cfg) != KVQ_OK || batch < 1 || n_q_heads < 1 || max_len < 1 ||
+      max_len > 0x7FFFFFFF)
+    return 0;
+  return align_up((size_t)batch * n_q_heads * decode_splits(max_len) * 130 * sizeof(float), 256);
+}
+
+int kvq_codebook(int bits, float* centroids, float* thresholds, double* distortion) {
+  if (bits < 1 || bits > 8) return fail(KVQ_ERR_ARG, "bits %d not in 1..8", bits);
+  const int n = 1 << bits;
+  if (centroids)
+    for (int m = 0; m < n; ++m) {
+      __half h = __ushort_as_half(kC16[cb_c_off(bits) + m]);
+      centroids[m] = __half2float(h);
+    }
+  if (thresholds)
+    for (int m = 0; m < n - 1; ++m) thresholds[m] = kThr[cb_t_off(bits) + m];
+  if (distortion) *distortion = kD[bits];
+  return KVQ_OK;
+}
+
+int kvq_plan_build(const kvq_cfg* cfg, int layer, const double* E_host, int n_heads,
+                   void* plans_host) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (!E_host || !plans_host || n_heads < 1) return fail(KVQ_ERR_ARG, "null pointer or n_heads < 1");
+  for (int i = 0; i < n_heads * kBlocks; ++i)
+    if (!(E_host[i] >= 0.0) || !std::isfinite(E_host[i]))
+      return fail(KVQ_ERR_ARG, "energy %d is negative or not finite", i);
+  Plan* out = reinterpret_cast<Plan*>(plans_host);
+  for (int h = 0; h < n_heads; ++h) build_plan(cfg, layer, h, E_host + (size_t)h * kBlocks, out + h);
+  return KVQ_OK;
+}
+
+int kvq_alloc_bits(const kvq_cfg* cfg, int layer, const void* k_dev, int k_dtype, int64_t n_tokens,
+                   void* ws_dev, size_t ws_bytes, void* plans_dev, void* plans_host,
+                   double* energy_host, uint32_t* status_dev, kvq_stream_t stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (!k_dev || !ws_dev || !plans_dev) return fail(KVQ_ERR_ARG, "null device pointer");
+  if (!dtype_ok(k_dtype)) return fail(KVQ_ERR_ARG, "k_dtype %d", k_dtype);
+  if (n_tokens < 1) return fail(KVQ_ERR_ARG, "n_tokens %lld < 1", (long long)n_tokens);
+  if (ws_bytes < kvq_alloc_workspace_bytes(cfg)) return fail(KVQ_ERR_WORKSPACE, "alloc workspace too small");
+  const int n_kv = cfg->n_kv_heads;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  auto* acc = reinterpret_cast<unsigned long long*>(ws_dev);
+  cudaError_t e = launch_energy(k_dev, k_dtype, n_tokens, n_kv, acc, status_dev, st);
+  if (e != cudaSuccess) return cuda_fail(e, "energy kernel");
+  std::vector<unsigned long long> h_acc((size_t)n_kv * kBlocks * 2);
+  e = cudaMemcpyAsync(h_acc.data(), acc, h_acc.size() * 8, cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return cuda_fail(e, "energy copy");
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "energy sync");
+  std::vector<double> E((size_t)n_kv * kBlocks);
+  for (size_t i = 0; i < E.size(); ++i) {
+    const unsigned __int128 s = ((unsigned __int128)h_acc[2 * i + 1] << 64) | h_acc[2 * i];
+    E[i] = std::ldexp((double)s, -32) / (double)n_tokens;
+  }
+  std::vector<Plan> plans(n_kv);
+  for (int h = 0; h < n_kv; ++h) build_plan(cfg, layer, h, E.data() + (size_t)h * kBlocks, &plans[h]);
+  e = cudaMemcpyAsync(plans_dev, plans.data(), (size_t)n_kv * sizeof(Plan), cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return cuda_fail(e, "plan copy");
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "plan sync");
+  if (plans_host) std::memcpy(plans_host, plans.data(), (size_t)n_kv * sizeof(Plan));
+  if (energy_host) std::memcpy(energy_host, E.data(), E.size() * sizeof(double));
+  return KVQ_OK;
+}
+
+int kvq_quantize_append(const kvq_cfg* cfg, const void* const* plans_dev, const void* k_dev,
+                        const void* v_dev, int dtype, int batch, int n_new, void* const* cache_dev,
+                        int32_t* len_dev, int64_t cap_tokens, uint32_t* status_dev,
+                        kvq_stream_t stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (!plans_dev || !cache_dev || !len_dev || !status_dev)
+    return fail(KVQ_ERR_ARG, "null device pointer");
+  if (!dtype_ok(dtype)) return fail(KVQ_ERR_ARG, "dtype %d", dtype);
+  if (batch < 1 || batch > 65535) return fail(KVQ_ERR_ARG, "batch %d", batch);
+  if (n_new < 0 || cap_tokens < 0 || cap_tokens > 0x7FFFFFFF)
+    return fail(KVQ_ERR_ARG, "n_new %d / cap_tokens %lld", n_new, (long long)cap_tokens);
+  if (n_new == 0) return KVQ_OK;
+  if (!k_dev || !v_dev) return fail(KVQ_ERR_ARG, "null k/v pointer");
+  if (n_new > (1 << 24)) return fail(KVQ_ERR_ARG, "n_new %d too large", n_new);
+  QuantParams p;
+  p.plans = reinterpret_cast<const Plan* const*>(plans_dev);
+  p.k = k_dev;
+  p.v = v_dev;
+  p.dtype = dtype;
+  p.batch = batch;
+  p.n_new = n_new;
+  p.n_kv = cfg->n_kv_heads;
+  p.caches = reinterpret_cast<uint8_t* const*>(cache_dev);
+  p.len = len_dev;
+  p.cap = cap_tokens;
+  p.tile_bytes = tile_bytes(cfg->bits_k, cfg->bits_v);
+  p.status = status_dev;
+  cudaError_t e = launch_quantize_append(p, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "quantize_append");
+  return KVQ_OK;
+}
+
+int kvq_decode_attn(const kvq_cfg* cfg, const void* const* plans_dev, const void* const* cache_dev,
+                    const int32_t* len_dev, int batch, int64_t max_len, const void* q_dev,
+                    int q_dtype, int n_q_heads, float* out_dev, void* ws_dev, size_t ws_bytes,
+                    uint32_t* status_dev, kvq_stream_t stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (!plans_dev || !cache_dev || !len_dev || !q_dev || !out_dev || !ws_dev || !status_dev)
+    return fail(KVQ_ERR_ARG, "null device pointer");
+  if (!dtype_ok(q_dtype)) return fail(KVQ_ERR_ARG, "q_dtype %d", q_dtype);
+  if (batch < 1 || batch > 65535) return fail(KVQ_ERR_ARG, "batch %d", batch);
+  if (max_len < 1 || max_len > 0x7FFFFFFF) return fail(KVQ_ERR_ARG, "max_len %lld", (long long)max_len);
+  if (n_q_heads < 1 || n_q_heads % cfg->n_kv_heads != 0 || n_q_heads / cfg->n_kv_heads > 16)
+    return fail(KVQ_ERR_ARG, "n_q_heads %d vs n_kv_heads %d", n_q_heads, cfg->n_kv_heads);
+  if (ws_bytes < kvq_decode_workspace_bytes(cfg, batch, n_q_heads, max_len))
+    return fail(KVQ_ERR_WORKSPACE, "decode workspace %zu < %zu", ws_bytes,
+                kvq_decode_workspace_bytes(cfg, batch, n_q_heads, max_len));
+  cudaError_t e = launch_decode(reinterpret_cast<const Plan* const*>(plans_dev),
+                                reinterpret_cast<const uint8_t* const*>(cache_dev), len_dev, batch,
+                                max_len, q_dev, q_dtype, n_q_heads, cfg->n_kv_heads, cfg->bits_k,
+                                cfg->bits_v, out_dev, reinterpret_cast<float*>(ws_dev), status_dev,
+                                reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode_attn");
+  return KVQ_OK;
+}
+
+}  // extern "C"

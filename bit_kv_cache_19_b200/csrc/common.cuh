@@ -1,0 +1,151 @@
+// Shared device definitions of libkvq: plan record, codebook constants,
+// IEEE-exact helpers and the sm_100a inline-PTX primitives (bulk copies,
+// mbarriers, mma.sync, movmatrix).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "kvq.h"
+#include "kvq_codebooks_gen.h"
+
+namespace kvq {
+
+constexpr int kHeadDim = 128;
+constexpr int kBlocks = 64;
+constexpr int kTile = 32;
+constexpr int kMaxHalf = 32;
+
+// Plan record, byte layout documented in kvq.h.
+struct Plan {
+  uint32_t magic;
+  int32_t bits_k, bits_v, n_ranks, layer, kv_head, words_k, words_v;
+  float g[64];
+  float a_hat[64];
+  uint8_t width[64];
+  uint8_t order[64];
+  uint16_t seg_off[65];
+  uint8_t n_half;
+  uint8_t pad0;
+  uint8_t hs_width[32];
+  uint8_t hs_rank0[32];
+  uint8_t hs_count[32];
+  uint32_t v_sign[4];
+  uint32_t pad1;
+  double energy_sum;
+  uint8_t tail[KVQ_PLAN_BYTES - 928];
+};
+static_assert(sizeof(Plan) == KVQ_PLAN_BYTES, "plan size");
+static_assert(offsetof(Plan, g) == 32 && offsetof(Plan, a_hat) == 288, "plan layout");
+static_assert(offsetof(Plan, width) == 544 && offsetof(Plan, order) == 608, "plan layout");
+static_assert(offsetof(Plan, seg_off) == 672 && offsetof(Plan, n_half) == 802, "plan layout");
+static_assert(offsetof(Plan, hs_width) == 804 && offsetof(Plan, v_sign) == 900, "plan layout");
+static_assert(offsetof(Plan, energy_sum) == 920, "plan layout");
+
+// Codebook offsets: width w centroids at 2^w - 2, thresholds at 2^w - w - 1.
+__host__ __device__ constexpr int cb_c_off(int w) { return (1 << w) - 2; }
+__host__ __device__ constexpr int cb_t_off(int w) { return (1 << w) - w - 1; }
+
+__host__ __device__ inline int tile_bytes(int bits_k, int bits_v) { return 512 * (bits_k + bits_v) + 128; }
+
+// Token position t of a tile -> bit slot (K segments, V segments) and back.
+__host__ __device__ __forceinline__ int slot_k(int t) { return 4 * (t & 7) + (t >> 3); }
+__host__ __device__ __forceinline__ int slot_v(int t) {
+  return 8 * ((t & 7) >> 1) + 2 * (t >> 3) + (t & 1);
+}
+__host__ __device__ __forceinline__ int token_of_slot_k(int s) { return 8 * (s & 3) + (s >> 2); }
+__host__ __device__ __forceinline__ int token_of_slot_v(int s) {
+  return 8 * ((s & 7) >> 1) + 2 * (s >> 3) + (s & 1);
+}
+
+// ------------------------------------------------------------------ device
+#ifdef __CUDACC__
+
+__device__ __forceinline__ float load_as_float(const void* p, int dtype, size_t i) {
+  if (dtype == KVQ_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+  if (dtype == KVQ_FP16) return __half2float(reinterpret_cast<const __half*>(p)[i]);
+  return reinterpret_cast<const float*>(p)[i];
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(unsigned long long* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(unsigned long long* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// 1-D bulk copy global -> shared, completion counted on `bar` (no multicast).
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         unsigned long long* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(unsigned long long* bar, uint32_t phase) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(phase)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait: gives up after ~2^31 clock cycles (about a second).
+__device__ __forceinline__ bool mbar_wait_bounded(unsigned long long* bar, uint32_t phase) {
+  if (mbar_try_wait(bar, phase)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, phase)) {
+    if (clock64() - t0 > (1ll << 31)) return false;
+  }
+  return true;
+}
+
+// D = A(16x16 f16, row) * B(16x8 f16, col) + D, fp32 accumulate.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Transpose of an 8x8 b16 matrix held one row per 4 lanes (2 elements each).
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ uint32_t funnel_r(uint32_t lo, uint32_t hi, uint32_t sh) {
+  return __funnelshift_r(lo, hi, sh);
+}
+
+#endif  // __CUDACC__
+
+}  // namespace kvq

@@ -1,0 +1,193 @@
+"""ctypes binding of libkvq (C ABI in include/kvq.h).
+
+Argument marshalling only: every step of the quantize and decode path runs in
+the library's CUDA kernels. PyTorch supplies device memory and the current
+stream. There is no fallback: if ``libkvq.so`` is missing the import of the
+library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkvq.so")
+
+OK = 0
+ERR_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA = -1, -2, -3, -4
+FLAG_CAPACITY, FLAG_NONFINITE, FLAG_NORM_SAT, FLAG_TIMEOUT, FLAG_BAD_PLAN = 1, 2, 4, 8, 16
+BF16, FP16, FP32 = 0, 1, 2
+ALLOC_GREEDY, ALLOC_UNIFORM = 0, 1
+PLAN_BYTES = 1024
+PLAN_MAGIC = 0x5051564B
+
+# Plan record layout (kvq.h).
+PLAN_DTYPE = np.dtype([
+    ("magic", "<u4"), ("bits_k", "<i4"), ("bits_v", "<i4"), ("n_ranks", "<i4"),
+    ("layer", "<i4"), ("kv_head", "<i4"), ("words_k", "<i4"), ("words_v", "<i4"),
+    ("g", "<f4", 64), ("a_hat", "<f4", 64), ("width", "u1", 64), ("order", "u1", 64),
+    ("seg_off", "<u2", 65), ("n_half", "u1"), ("pad0", "u1"), ("hs_width", "u1", 32),
+    ("hs_rank0", "u1", 32), ("hs_count", "u1", 32), ("v_sign", "<u4", 4), ("pad1", "<u4"),
+    ("energy_sum", "<f8"), ("tail", "u1", PLAN_BYTES - 928),
+])
+assert PLAN_DTYPE.itemsize == PLAN_BYTES
+
+
+class KVQError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"kvq error {code}: {msg}")
+        self.code = code
+
+
+class Cfg(ctypes.Structure):
+    _fields_ = [("head_dim", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+                ("bits_k", ctypes.c_int32), ("bits_v", ctypes.c_int32), ("b_max", ctypes.c_int32),
+                ("alloc_mode", ctypes.c_int32), ("v_seed", ctypes.c_uint64)]
+
+
+def make_cfg(n_kv_heads, bits_k, bits_v, v_seed=0, alloc_mode=ALLOC_GREEDY, head_dim=128):
+    return Cfg(head_dim, n_kv_heads, bits_k, bits_v, 8, alloc_mode, v_seed)
+
+
+_vp, _sz, _i32, _i64, _u32p = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_int64, \
+    ctypes.c_void_p
+_SIGS = {
+    "kvq_version": (ctypes.c_char_p, []),
+    "kvq_last_error": (ctypes.c_char_p, []),
+    "kvq_plan_bytes": (_sz, []),
+    "kvq_tile_bytes": (_sz, [ctypes.POINTER(Cfg)]),
+    "kvq_cache_bytes": (_sz, [ctypes.POINTER(Cfg), _i64]),
+    "kvq_alloc_workspace_bytes": (_sz, [ctypes.POINTER(Cfg)]),
+    "kvq_decode_workspace_bytes": (_sz, [ctypes.POINTER(Cfg), _i32, _i32, _i64]),
+    "kvq_alloc_bits": (_i32, [ctypes.POINTER(Cfg), _i32, _vp, _i32, _i64, _vp, _sz, _vp, _vp,
+                              _vp, _vp, _vp]),
+    "kvq_plan_build": (_i32, [ctypes.POINTER(Cfg), _i32, _vp, _i32, _vp]),
+    "kvq_codebook": (_i32, [_i32, _vp, _vp, _vp]),
+    "kvq_quantize_append": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp,
+                                   _i64, _vp, _vp]),
+    "kvq_decode_attn": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i64, _vp, _i32, _i32,
+                               _vp, _vp, _sz, _vp, _vp]),
+}
+EXPORTS = tuple(_SIGS)
+
+_lib = None
+
+
+def lib():
+    """The loaded libkvq (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing; build it with "
+                              "`python -m bit_kv_cache_19_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(rc):
+    if rc != OK:
+        raise KVQError(rc, lib().kvq_last_error().decode())
+    return rc
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _dtype_code(t):
+    import torch
+    return {torch.bfloat16: BF16, torch.float16: FP16, torch.float32: FP32}[t.dtype]
+
+
+# ------------------------------------------------------------ sizes, host-only
+def version() -> str:
+    return lib().kvq_version().decode()
+
+
+def tile_bytes(cfg) -> int:
+    return lib().kvq_tile_bytes(ctypes.byref(cfg))
+
+
+def cache_bytes(cfg, cap_tokens) -> int:
+    return lib().kvq_cache_bytes(ctypes.byref(cfg), cap_tokens)
+
+
+def alloc_workspace_bytes(cfg) -> int:
+    return lib().kvq_alloc_workspace_bytes(ctypes.byref(cfg))
+
+
+def decode_workspace_bytes(cfg, batch, n_q_heads, max_len) -> int:
+    return lib().kvq_decode_workspace_bytes(ctypes.byref(cfg), batch, n_q_heads, max_len)
+
+
+def codebook(bits):
+    """(centroids float32 [2^b], thresholds float32 [2^b - 1], D) of the library."""
+    c = np.zeros(1 << bits, dtype=np.float32)
+    t = np.zeros((1 << bits) - 1, dtype=np.float32)
+    d = ctypes.c_double()
+    _check(lib().kvq_codebook(bits, c.ctypes.data, t.ctypes.data, ctypes.byref(d)))
+    return c, t, d.value
+
+
+def plan_build(cfg, layer, E) -> np.ndarray:
+    """Host plan records (PLAN_DTYPE array) from energies E[n_heads, 64]."""
+    E = np.ascontiguousarray(np.asarray(E, dtype=np.float64))
+    n = E.shape[0]
+    out = np.zeros(n, dtype=PLAN_DTYPE)
+    _check(lib().kvq_plan_build(ctypes.byref(cfg), layer, E.ctypes.data, n, out.ctypes.data))
+    return out
+
+
+def parse_plans(raw) -> np.ndarray:
+    return np.frombuffer(bytes(raw), dtype=PLAN_DTYPE)
+
+
+# ------------------------------------------------------------------ device
+def ptr_array(tensors, device):
+    """Device int64 tensor holding the data pointers of ``tensors``."""
+    import torch
+    return torch.tensor([t.data_ptr() for t in tensors], dtype=torch.int64, device=device)
+
+
+def alloc_bits(cfg, layer, k, plans_dev, status=None, ws=None):
+    """Energy + greedy plans of one layer. k: [T, n_kv, 128] on the device.
+
+    Writes plans_dev (uint8 [n_kv * 1024]); returns (host plans, energies)."""
+    import torch
+    n_kv = cfg.n_kv_heads
+    if ws is None:
+        ws = torch.empty(alloc_workspace_bytes(cfg), dtype=torch.uint8, device=k.device)
+    host = np.zeros(n_kv, dtype=PLAN_DTYPE)
+    E = np.zeros((n_kv, 64), dtype=np.float64)
+    _check(lib().kvq_alloc_bits(ctypes.byref(cfg), layer, _ptr(k), _dtype_code(k), k.shape[0],
+                                _ptr(ws), ws.numel(), _ptr(plans_dev), host.ctypes.data,
+                                E.ctypes.data, _ptr(status), _stream()))
+    return host, E
+
+
+def quantize_append(cfg, plan_ptrs, k, v, cache_ptrs, lens, cap_tokens, status):
+    """Append k, v [batch, n_new, n_kv, 128] to the packed caches."""
+    batch, n_new = k.shape[0], k.shape[1]
+    _check(lib().kvq_quantize_append(ctypes.byref(cfg), _ptr(plan_ptrs), _ptr(k), _ptr(v),
+                                     _dtype_code(k), batch, n_new, _ptr(cache_ptrs), _ptr(lens),
+                                     cap_tokens, _ptr(status), _stream()))
+
+
+def decode_attn(cfg, plan_ptrs, cache_ptrs, lens, max_len, q, out, ws, status):
+    """Packed-cache decode attention; q [batch, n_q, 128], out fp32 same shape."""
+    batch, n_q = q.shape[0], q.shape[1]
+    _check(lib().kvq_decode_attn(ctypes.byref(cfg), _ptr(plan_ptrs), _ptr(cache_ptrs), _ptr(lens),
+                                 batch, max_len, _ptr(q), _dtype_code(q), n_q, _ptr(out), _ptr(ws),
+                                 ws.numel() * ws.element_size(), _ptr(status), _stream()))

@@ -1,0 +1,76 @@
+"""Device-memory plumbing around libkvq (PyTorch tensors; no compute here).
+
+``PackedLayer`` owns, for one layer and a batch of sequences, the plan
+records, the packed caches, their pointer arrays, the lengths and the status
+word, and forwards to the three C-ABI calls.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import kvq
+
+
+class PackedLayer:
+    def __init__(self, cfg, batch: int, cap_tokens: int, device="cuda", layer: int = 0):
+        self.cfg = cfg
+        self.batch = batch
+        self.cap = cap_tokens
+        self.layer = layer
+        self.device = torch.device(device)
+        n_kv = cfg.n_kv_heads
+        self.plans = torch.zeros(n_kv * kvq.PLAN_BYTES, dtype=torch.uint8, device=self.device)
+        nbytes = kvq.cache_bytes(cfg, cap_tokens)
+        self.caches = [torch.zeros(nbytes, dtype=torch.uint8, device=self.device)
+                       for _ in range(batch)]
+        self.cache_ptrs = kvq.ptr_array(self.caches, self.device)
+        self.plan_ptrs = kvq.ptr_array([self.plans] * batch, self.device)
+        self.lens = torch.zeros(batch, dtype=torch.int32, device=self.device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self.plans_host = None
+        self.energy = None
+
+    # -------------------------------------------------------------- calls
+    def alloc_bits(self, k):
+        """Plans from keys k [T, n_kv, 128] (device)."""
+        self.plans_host, self.energy = kvq.alloc_bits(self.cfg, self.layer, k, self.plans,
+                                                      self.status)
+        return self.plans_host
+
+    def set_plans(self, plans_host: np.ndarray):
+        """Use host plan records (e.g. from kvq.plan_build)."""
+        raw = torch.from_numpy(np.frombuffer(plans_host.tobytes(), dtype=np.uint8).copy())
+        self.plans.copy_(raw.to(self.device))
+        self.plans_host = plans_host
+
+    def append(self, k, v):
+        """k, v [batch, n_new, n_kv, 128] (device) appended after each length."""
+        kvq.quantize_append(self.cfg, self.plan_ptrs, k, v, self.cache_ptrs, self.lens, self.cap,
+                            self.status)
+
+    def decode(self, q, out=None, ws=None, max_len=None):
+        """q [batch, n_q, 128] -> fp32 [batch, n_q, 128]."""
+        max_len = self.cap if max_len is None else max_len
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=self.device)
+        if ws is None:
+            ws = self.workspace(q.shape[1], max_len)
+        kvq.decode_attn(self.cfg, self.plan_ptrs, self.cache_ptrs, self.lens, max_len, q, out, ws,
+                        self.status)
+        return out
+
+    def workspace(self, n_q: int, max_len: int):
+        n = kvq.decode_workspace_bytes(self.cfg, self.batch, n_q, max_len)
+        return torch.empty(n, dtype=torch.uint8, device=self.device)
+
+    # ------------------------------------------------------------ inspect
+    def head_records(self, seq: int, head: int, n_tiles: int) -> np.ndarray:
+        """Tile records [n_tiles, tile_bytes / 4] (uint32) of one head, on the host."""
+        tb = kvq.tile_bytes(self.cfg)
+        raw = self.caches[seq][: n_tiles * self.cfg.n_kv_heads * tb].view(
+            n_tiles, self.cfg.n_kv_heads, tb)[:, head].contiguous().cpu().numpy()
+        return raw.view("<u4").reshape(n_tiles, tb // 4)
+
+    def flags(self) -> int:
+        return int(self.status.item()) & 0xFFFFFFFF

@@ -1,0 +1,266 @@
+/*
+ * kvq.h - C ABI of libkvq: RoPE-aware packed KV-cache quantization and
+ * packed-cache decode attention for NVIDIA B200 (sm_100a).
+ *
+ * Method: "RoPE-Aware Bit Allocation for KV-Cache Quantization" (Block-GTQ),
+ * abstract. Per (layer, KV head): a label-free energy score of each RoPE 2-D
+ * block, greedy integer bit widths by marginal gain under a matched K/V bit
+ * budget (KxVy), quantization built on TurboQuant-MSE (TQ-MSE), and a
+ * packed-cache serving path whose decode attention reads the packed cache.
+ * The abstract leaves the energy formula, the distortion model, the
+ * codebooks, the norm and the packing open; the readings adopted are stated
+ * at each entry point below.
+ *
+ * Conventions shared by every entry point
+ *   - Ownership: the caller allocates and frees every buffer (caches, plans,
+ *     workspace, lengths, status word). The library never allocates device
+ *     memory and keeps no pointer after a call returns.
+ *   - Pointers named *_dev are device pointers; *_host are host pointers.
+ *     "Device array of pointers" means a device buffer holding device
+ *     addresses (64-bit each).
+ *   - Asynchrony: calls enqueue work on `stream` and return once it is
+ *     launched. kvq_alloc_bits is the exception: it synchronizes `stream`
+ *     once (it needs the energies on the host).
+ *   - Errors: a negative return means nothing was launched;
+ *     kvq_last_error() gives a message (thread-local). Problems that only
+ *     the device can see set bits of *status_dev with an atomic OR
+ *     (KVQ_FLAG_*); kernels never trap and never wait without a bound.
+ *   - Supported shapes: head_dim = 128; bits_k and bits_v in 1..8; b_max = 8;
+ *     n_q_heads a multiple of n_kv_heads with G = n_q_heads / n_kv_heads <= 16.
+ *   - Thread safety: calls on different streams may run concurrently; the
+ *     library holds no mutable global state besides kvq_last_error().
+ */
+#ifndef KVQ_H_
+#define KVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported symbols (the library is built with hidden default visibility). */
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
+
+/* A cudaStream_t (the runtime's stream handle type). 0 = legacy stream. */
+typedef struct CUstream_st* kvq_stream_t;
+
+/* Return codes. */
+#define KVQ_OK 0
+#define KVQ_ERR_ARG (-1)          /* bad argument (null pointer, range, size) */
+#define KVQ_ERR_UNSUPPORTED (-2)  /* valid but unsupported shape (head_dim != 128) */
+#define KVQ_ERR_WORKSPACE (-3)    /* workspace smaller than required */
+#define KVQ_ERR_CUDA (-4)         /* a CUDA runtime call failed */
+
+/* Device status flags, OR-ed into *status_dev (a uint32 the caller zeroes). */
+#define KVQ_FLAG_CAPACITY 1u   /* append past cap_tokens (sequence skipped), or len > max_len */
+#define KVQ_FLAG_NONFINITE 2u  /* a token had a NaN/Inf coordinate: stored as norm 0, codes 0 */
+#define KVQ_FLAG_NORM_SAT 4u   /* a norm overflowed fp16: stored as 65504 */
+#define KVQ_FLAG_TIMEOUT 8u    /* a bounded wait for a tile copy ran out: output invalid */
+#define KVQ_FLAG_BAD_PLAN 16u  /* a plan record failed its magic/shape check */
+
+/* Input element types. */
+#define KVQ_BF16 0
+#define KVQ_FP16 1
+#define KVQ_FP32 2
+
+/* Allocation modes. */
+#define KVQ_ALLOC_GREEDY 0   /* Block-GTQ: greedy marginal-gain widths per RoPE block */
+#define KVQ_ALLOC_UNIFORM 1  /* every block gets bits_k (same bytes; comparator) */
+
+typedef struct {
+  int32_t head_dim;    /* must be 128 */
+  int32_t n_kv_heads;  /* KV heads per layer, >= 1 */
+  int32_t bits_k;      /* key budget, bits per dimension, 1..8 (K in KxVy) */
+  int32_t bits_v;      /* value width, bits per dimension, 1..8 (V in KxVy) */
+  int32_t b_max;       /* largest width of one block, must be 8 */
+  int32_t alloc_mode;  /* KVQ_ALLOC_GREEDY or KVQ_ALLOC_UNIFORM */
+  uint64_t v_seed;     /* seed of the value sign flips */
+} kvq_cfg;
+
+/*
+ * Plan record: one per (layer, KV head), KVQ_PLAN_BYTES bytes, plain data
+ * (copy it with memcpy; it holds no pointer). Little-endian layout:
+ *   off   0  uint32  magic = KVQ_PLAN_MAGIC
+ *   off   4  int32   bits_k
+ *   off   8  int32   bits_v
+ *   off  12  int32   n_ranks        stored (nonzero-width) blocks
+ *   off  16  int32   layer
+ *   off  20  int32   kv_head
+ *   off  24  int32   words_k        K code words per 32-token tile = 128 * bits_k
+ *   off  28  int32   words_v        V code words per 32-token tile = 128 * bits_v
+ *   off  32  float   g[64]          quantize scale of block j: fp32(1/a_j), 0 if a_j = 0
+ *   off 288  float   a_hat[64]      dequantize scale of block j: fp32(a_j)
+ *   off 544  uint8   width[64]      bits of block j (0..8)
+ *   off 608  uint8   order[64]      plan rank -> block index (ranks >= n_ranks unused)
+ *   off 672  uint16  seg_off[65]    rank -> first word of its K segment in a tile record
+ *   off 802  uint8   n_half         decode schedule: groups of <= 4 equal-width ranks
+ *   off 803  uint8   pad
+ *   off 804  uint8   hs_width[32]
+ *   off 836  uint8   hs_rank0[32]
+ *   off 868  uint8   hs_count[32]
+ *   off 900  uint32  v_sign[4]      bit i set <=> value sign s_i = -1
+ *   off 916  uint32  pad
+ *   off 920  double  energy_sum     sum of the 64 block energies, fp64 in block order
+ *   off 928  .. 1023 zero
+ */
+#define KVQ_PLAN_BYTES 1024
+#define KVQ_PLAN_MAGIC 0x5051564Bu /* "KVQP" */
+
+/* Library version string. */
+KVQ_API const char* kvq_version(void);
+
+/* Message of the last negative return on the calling thread ("" if none). */
+KVQ_API const char* kvq_last_error(void);
+
+/* Size of one plan record (KVQ_PLAN_BYTES). */
+KVQ_API size_t kvq_plan_bytes(void);
+
+/*
+ * Bytes of one 32-token tile record for the budget of `cfg`:
+ * 512 * (bits_k + bits_v) + 128. Layout (little-endian 32-bit words):
+ *   [K: 128 bits_k words][V: 128 bits_v words][K norms: 32 fp16][V norms: 32 fp16]
+ * K part: one segment of 2w words per stored block, in plan order
+ * (order[], seg_off[]); segment words hold 32 fields of 2w bits, token
+ * position t of the tile at bit (4 (t mod 8) + t div 8) * 2w, low w bits the
+ * code of coordinate j, high w bits the code of j + 64.
+ * V part: 128 segments of bits_v words (rotated coordinate p at word
+ * 128 bits_k + p bits_v), token position t at bit
+ * (8 ((t mod 8) div 2) + 2 (t div 8) + (t mod 2)) * bits_v.
+ * Code bits of positions holding no token are zero.
+ * This is the reading adopted for the pages' "packed K3V3" cache: exactly
+ * b_K + b_V bits per dimension plus two fp16 norms per token and head
+ * (K3V3: 100 bytes per token and KV head).
+ */
+KVQ_API size_t kvq_tile_bytes(const kvq_cfg* cfg);
+
+/*
+ * Bytes of the packed cache of one (sequence, layer) holding up to
+ * cap_tokens tokens: ceil(cap_tokens / 32) * n_kv_heads * kvq_tile_bytes.
+ * Tile tau (tokens 32 tau .. 32 tau + 31) of KV head h is the record at byte
+ * offset (tau * n_kv_heads + h) * tile_bytes. Returns 0 for an invalid cfg.
+ * The base address must be 16-byte aligned (kernels flag BAD_PLAN and skip
+ * a sequence whose cache is not).
+ */
+KVQ_API size_t kvq_cache_bytes(const kvq_cfg* cfg, int64_t cap_tokens);
+
+/* Workspace bytes kvq_alloc_bits needs: n_kv_heads * 64 * 16 (+ alignment). */
+KVQ_API size_t kvq_alloc_workspace_bytes(const kvq_cfg* cfg);
+
+/*
+ * Workspace bytes kvq_decode_attn needs for `batch` sequences of at most
+ * max_len tokens: split-K partials (m, l, o[128]) per (sequence, query head,
+ * split). Returns 0 for invalid arguments.
+ */
+KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cfg* cfg, int batch, int n_q_heads,
+                                  int64_t max_len);
+
+/*
+ * Block energies and bit allocation for one layer: Block-GTQ's label-free
+ * per-RoPE-block energy score and greedy marginal-gain integer widths
+ * ("RoPE-Aware Bit Allocation for KV-Cache Quantization", abstract).
+ * Readings adopted:
+ *   energy   E_j = (1/T) sum_t (k_{t,j}^2 + k_{t,j+64}^2) over the T given
+ *            keys, each square taken on a 2^-32 fixed-point grid
+ *            (floor(k^2 2^32), saturating at 2^64-1) and summed exactly as an
+ *            integer, so the result does not depend on summation order;
+ *   D(b)     Lloyd-Max MSE of a unit Gaussian with 2^b levels, D(0) = 1;
+ *   greedy   64 bits_k steps from all-zero widths; each adds 1 bit to the
+ *            block of largest E_j (D(b_j) - D(b_j + 1)) below b_max; ties to
+ *            the lowest index;
+ *   scales   a_j = sqrt(E_j / (2 sum_l E_l)); g_j = fp32(1/a_j), a_hat_j = fp32(a_j);
+ *   signs    value sign s_i = -1 iff bit 63 of SplitMix64(key, i) is set,
+ *            key = SplitMix64(v_seed, layer * 2^32 + kv_head) (n-th output of
+ *            the stream seeded with s: mix(s + (n + 1) 0x9E3779B97F4A7C15)).
+ * k_dev: keys [n_tokens][n_kv_heads][128] of type k_dtype (post-RoPE; the
+ *        energy is RoPE-invariant). n_tokens >= 1.
+ * ws_dev: >= kvq_alloc_workspace_bytes(cfg) bytes (contents overwritten).
+ * plans_dev: out, n_kv_heads plan records (contiguous).
+ * plans_host: optional out (may be NULL), same records on the host.
+ * energy_host: optional out (may be NULL), E[n_kv_heads][64] as fp64.
+ * status_dev: optional (may be NULL); NONFINITE if a key was not finite
+ *        (its square counts 0).
+ * Synchronizes `stream` once. Returns KVQ_OK or a negative code.
+ */
+KVQ_API int kvq_alloc_bits(const kvq_cfg* cfg, int layer, const void* k_dev, int k_dtype,
+                   int64_t n_tokens, void* ws_dev, size_t ws_bytes, void* plans_dev,
+                   void* plans_host, double* energy_host, uint32_t* status_dev,
+                   kvq_stream_t stream);
+
+/*
+ * Host-only plan builder from given energies (no GPU work): the greedy,
+ * scales and signs of kvq_alloc_bits for E_host[n_heads][64], writing
+ * n_heads plan records to plans_host (head h gets kv_head = h).
+ */
+KVQ_API int kvq_plan_build(const kvq_cfg* cfg, int layer, const double* E_host, int n_heads,
+                   void* plans_host);
+
+/*
+ * The library's own Gaussian Lloyd-Max tables for `bits` in 1..8 (host, no
+ * GPU): 2^bits fp16-exact centroids (as float), 2^bits - 1 fp32 thresholds
+ * (midpoints of the centroids), and D(bits). Any output may be NULL.
+ */
+KVQ_API int kvq_codebook(int bits, float* centroids, float* thresholds, double* distortion);
+
+/*
+ * Quantize and append n_new tokens per sequence to the packed cache
+ * (Block-GTQ keys on TQ-MSE, uniform TQ-MSE values). Per token and KV head:
+ *   keys:   n = fp16(sqrt(sum k_i^2)) (fixed fp32 order), r = 1/n,
+ *           z_i = (k_i r) g_j, code_i = #{thresholds of width b_j below z_i};
+ *   values: y = H (s . v) (Walsh-Hadamard, fp32 butterflies h = 1..64),
+ *           n = fp16 norm of v, z_i = y_i r, codes at width bits_v;
+ * all decisions in IEEE fp32 without fused multiply-add, so codes are
+ * reproducible bit for bit.
+ * plans_dev: device array of `batch` pointers, entry b -> the n_kv_heads
+ *        plan records used for sequence b (usually the same layer's plans).
+ * k_dev, v_dev: [batch][n_new][n_kv_heads][128] of type `dtype`.
+ * cache_dev: device array of `batch` pointers to each sequence's cache
+ *        (kvq_cache_bytes(cfg, cap_tokens) bytes, 16-byte aligned).
+ * len_dev: int32 [batch]; token positions len..len+n_new-1 are written and
+ *        len is then increased by n_new. A sequence with len + n_new >
+ *        cap_tokens is skipped (len unchanged) and CAPACITY is flagged.
+ * status_dev: required.
+ * Tokens already in a tile keep their bits; positions past the new length
+ * are zero. Returns KVQ_OK or a negative code.
+ */
+KVQ_API int kvq_quantize_append(const kvq_cfg* cfg, const void* const* plans_dev, const void* k_dev,
+                        const void* v_dev, int dtype, int batch, int n_new,
+                        void* const* cache_dev, int32_t* len_dev, int64_t cap_tokens,
+                        uint32_t* status_dev, kvq_stream_t stream);
+
+/*
+ * Decode attention straight from the packed cache: for sequence b and query
+ * head h (KV head h / G),
+ *   o_h = sum_t softmax_t(q_h . k_hat_t / sqrt(128)) v_hat_t
+ * over the len_dev[b] cached tokens, with k_hat and v_hat the dequantized
+ * keys and values (k_hat_i = n^K a_hat_j c_{b_j}[code_i];
+ * v_hat = n^V (1/128) s . (H c_{bits_v}[codes])). Split-K over the context:
+ * each CTA unpacks its tiles in registers, forms the logits of all G query
+ * heads of its KV head, keeps an online softmax and accumulates P V in the
+ * rotated value domain; a combine kernel merges the splits and applies the
+ * inverse rotation. fp32 accumulation.
+ * plans_dev, cache_dev: as for kvq_quantize_append.
+ * len_dev: int32 [batch], each <= max_len (a larger value is clamped to
+ *        max_len and flags CAPACITY). A sequence of length 0 gives o = 0.
+ * q_dev: [batch][n_q_heads][128] of type q_dtype (post-RoPE queries).
+ * out_dev: fp32 [batch][n_q_heads][128].
+ * ws_dev: >= kvq_decode_workspace_bytes(cfg, batch, n_q_heads, max_len).
+ * status_dev: required.
+ * Returns KVQ_OK or a negative code.
+ */
+KVQ_API int kvq_decode_attn(const kvq_cfg* cfg, const void* const* plans_dev,
+                    const void* const* cache_dev, const int32_t* len_dev, int batch,
+                    int64_t max_len, const void* q_dev, int q_dtype, int n_q_heads,
+                    float* out_dev, void* ws_dev, size_t ws_bytes, uint32_t* status_dev,
+                    kvq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H_ */

@@ -15,8 +15,9 @@ dimension on keys, y on values). Readings adopted where the abstract is silent:
   b_max = 8; ties go to the lowest block index; J * b_K steps, so the key
   budget (b_K bits per dimension, 2 J b_K bits per token) is met exactly.
   D is convex, so this is optimal for the separable objective.
-* Key scale: a_j = sqrt(E_j / (2 sum_l E_l)), the expected RMS of one
-  coordinate of block j after dividing the key by its norm; the quantizer
+* Key scale: a_j = sqrt(E_j / (2 sum_l E_l)) (the sum in fp64 in block
+  order), the expected RMS of one coordinate of block j after dividing the
+  key by its norm; the quantizer
   multiplies by g_j = fp32(1/a_j) (0 when a_j = 0) and reconstruction
   multiplies by a_hat_j = fp32(a_j).
 * Plan order: blocks with b_j > 0 sorted by width (descending), then block
@@ -74,7 +75,9 @@ def objective(E, widths, D=lloydmax.D) -> float:
 def key_scales(E):
     """(g, a_hat) as float32 arrays from energies ``E`` (length J)."""
     E = np.asarray(E, dtype=np.float64)
-    tot = float(np.sum(E))
+    tot = 0.0
+    for e in E:                 # fp64, block order 0, 1, 2, ...
+        tot += float(e)
     g = np.zeros(E.shape, dtype=np.float32)
     ah = np.zeros(E.shape, dtype=np.float32)
     for j, e in enumerate(E):

@@ -74,16 +74,20 @@ def codes_from_z(z: np.ndarray, bits: int) -> np.ndarray:
 
 
 def fwht_f32(x: np.ndarray) -> np.ndarray:
-    """Unnormalised Walsh-Hadamard transform along the last axis, fp32 graph."""
+    """Unnormalised Walsh-Hadamard transform along the last axis, fp32 graph.
+
+    Stage h views the last axis as (d / 2h, 2, h): the pair (a, b) of each
+    butterfly is (x_i, x_{i+h}) with (i & h) == 0, replaced by (a + b, a - b).
+    """
     y = np.array(x, dtype=np.float32, copy=True)
     d = y.shape[-1]
+    lead = y.shape[:-1]
     h = 1
     while h < d:
-        idx = np.array([i for i in range(d) if (i & h) == 0])
-        a = y[..., idx].copy()
-        b = y[..., idx + h].copy()
-        y[..., idx] = a + b
-        y[..., idx + h] = a - b
+        v = y.reshape(*lead, d // (2 * h), 2, h)
+        a = v[..., 0, :]
+        b = v[..., 1, :]
+        y = np.stack([a + b, a - b], axis=-2).reshape(*lead, d)
         h *= 2
     return y
 

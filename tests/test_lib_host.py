@@ -1,0 +1,123 @@
+"""Host-side checks of libkvq on the CPU: exports, codebooks, plans, errors."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from bit_kv_cache_19_b200 import kvq
+from oracle import alloc, lloydmax
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    return sorted(set(re.findall(r"KVQ_API\s+[\w\s\*]+?\b(kvq_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol():
+    names = _declared()
+    assert len(names) >= 12
+    L = kvq.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(kvq.EXPORTS)
+
+
+@pytest.mark.parametrize("b", range(1, 9))
+def test_library_codebook_equals_oracle(b):
+    c, t, d = kvq.codebook(b)
+    assert np.array_equal(c.astype(np.float64), lloydmax.centroids(b))
+    assert np.array_equal(t, lloydmax.thresholds(b))
+    assert abs(d - lloydmax.D(b)) <= 1e-10 * lloydmax.D(b)
+
+
+def _energies(rng, n, kind):
+    j = np.arange(64)
+    if kind == "decay":
+        return np.exp(-j / 6.0 + rng.standard_normal((n, 64)))
+    if kind == "flat":
+        return np.ones((n, 64))
+    if kind == "zeros":
+        E = np.exp(rng.standard_normal((n, 64)))
+        E[:, ::3] = 0.0
+        return E
+    return np.exp(3 * rng.standard_normal((n, 64)))
+
+
+@pytest.mark.parametrize("kind", ["decay", "flat", "zeros", "wild"])
+@pytest.mark.parametrize("bits", [(1, 1), (2, 2), (3, 2), (3, 3), (4, 8), (8, 1)])
+def test_plan_build_equals_oracle(kind, bits):
+    rng = np.random.default_rng(hash((kind, bits)) % 2 ** 32)
+    E = _energies(rng, 3, kind)
+    bk, bv = bits
+    for mode in (kvq.ALLOC_GREEDY, kvq.ALLOC_UNIFORM):
+        cfg = kvq.make_cfg(3, bk, bv, v_seed=987654321, alloc_mode=mode)
+        got = kvq.plan_build(cfg, 5, E)
+        for h in range(3):
+            ref = alloc.make_plan(E[h], bk, bv, 987654321, 5, h, uniform=mode == kvq.ALLOC_UNIFORM)
+            assert not ref.near_tie or mode == kvq.ALLOC_UNIFORM or kind == "flat"
+            p = got[h]
+            assert p["magic"] == kvq.PLAN_MAGIC and p["layer"] == 5 and p["kv_head"] == h
+            assert np.array_equal(p["width"].astype(int), ref.widths)
+            assert p["n_ranks"] == len(ref.order)
+            assert list(p["order"][:p["n_ranks"]]) == ref.order
+            assert np.array_equal(p["g"], ref.g) and np.array_equal(p["a_hat"], ref.a_hat)
+            signs = np.array([-1.0 if (p["v_sign"][i >> 5] >> (i & 31)) & 1 else 1.0
+                              for i in range(128)])
+            assert np.array_equal(signs, ref.signs)
+            # segment offsets and the half-step schedule are consistent
+            off = 0
+            for r in range(p["n_ranks"]):
+                assert p["seg_off"][r] == off
+                off += 2 * int(p["width"][p["order"][r]])
+            assert off == 128 * bk == p["seg_off"][p["n_ranks"]]
+            covered = []
+            for hs in range(p["n_half"]):
+                r0, n, w = p["hs_rank0"][hs], p["hs_count"][hs], p["hs_width"][hs]
+                assert 1 <= n <= 4
+                assert all(p["width"][p["order"][r]] == w for r in range(r0, r0 + n))
+                covered += list(range(r0, r0 + n))
+            assert covered == list(range(p["n_ranks"]))
+            assert p["n_half"] <= 24
+
+
+def test_sizes():
+    cfg = kvq.make_cfg(2, 3, 3)
+    assert kvq.tile_bytes(cfg) == 3200 == 32 * 100
+    assert kvq.cache_bytes(cfg, 131072) == 4096 * 2 * 3200
+    assert kvq.cache_bytes(cfg, 33) == 2 * 2 * 3200
+    assert kvq.alloc_workspace_bytes(cfg) >= 2 * 64 * 16
+    assert kvq.decode_workspace_bytes(cfg, 1, 16, 131072) > 0
+    assert kvq.lib().kvq_plan_bytes() == 1024
+
+
+def test_argument_errors_without_gpu():
+    L = kvq.lib()
+    bad = kvq.make_cfg(2, 3, 3, head_dim=64)
+    assert L.kvq_plan_build(ctypes.byref(bad), 0, None, 1, None) == kvq.ERR_UNSUPPORTED
+    cfg = kvq.make_cfg(2, 9, 3)
+    assert L.kvq_plan_build(ctypes.byref(cfg), 0, None, 1, None) == kvq.ERR_ARG
+    assert b"bits_k" in L.kvq_last_error()
+    cfg = kvq.make_cfg(2, 3, 3)
+    assert kvq.tile_bytes(kvq.make_cfg(2, 0, 3)) == 0
+    assert L.kvq_decode_attn(ctypes.byref(cfg), None, None, None, 1, 10, None, 0, 16, None, None,
+                             0, None, None) == kvq.ERR_ARG
+    E = -np.ones((1, 64))
+    assert L.kvq_plan_build(ctypes.byref(kvq.make_cfg(1, 2, 2)), 0, E.ctypes.data, 1,
+                            np.zeros(1, kvq.PLAN_DTYPE).ctypes.data) == kvq.ERR_ARG
+    # n_q not a multiple of n_kv, G > 16, workspace too small: rejected before launch
+    p = ctypes.c_void_p(16)
+    assert L.kvq_decode_attn(ctypes.byref(cfg), p, p, p, 1, 10, p, 0, 15, p, p, 1 << 30, p,
+                             None) == kvq.ERR_ARG
+    assert L.kvq_decode_attn(ctypes.byref(cfg), p, p, p, 1, 10, p, 0, 34, p, p, 1 << 30, p,
+                             None) == kvq.ERR_ARG
+    assert L.kvq_decode_attn(ctypes.byref(cfg), p, p, p, 1, 10, p, 0, 16, p, p, 8, p,
+                             None) == kvq.ERR_WORKSPACE
+    assert L.kvq_quantize_append(ctypes.byref(cfg), p, p, p, 7, 1, 1, p, p, 10, p,
+                                 None) == kvq.ERR_ARG
+    # zero new tokens is a no-op
+    assert L.kvq_quantize_append(ctypes.byref(cfg), p, None, None, 0, 1, 0, p, p, 10, p,
+                                 None) == kvq.OK
