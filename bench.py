@@ -54,6 +54,8 @@ def parse():
                     choices=["qwen3b_128k", "llama8b", "qwen7b_serve"])
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--layers", type=int, default=0,
+                    help="override the layer count (small cases for profiling)")
     return ap.parse_args()
 
 
@@ -212,7 +214,7 @@ def run_kvq(args, wl, rank, world, dist):
     from bit_kv_cache_19_b200.runtime import PackedLayer
 
     dev = torch.device("cuda", torch.cuda.current_device())
-    n_layers, B, T = wl.n_layers, wl.batch, wl.context
+    n_layers, B, T = args.layers or wl.n_layers, wl.batch, wl.context
     steps, warmup = args.steps, args.warmup
     cap = T + steps + warmup + 64
     cfg = kvq.make_cfg(wl.n_kv_heads, wl.bits_k, wl.bits_v, v_seed=1234)

@@ -430,30 +430,59 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(const DecodeParams 
 
 // Merge split partials and undo the value rotation:
 // o = (1 / (128 l)) s . (H sum_s 2^(m_s - m) o_s).
-__global__ void __launch_bounds__(128) combine_kernel(const float* __restrict__ part, int n_splits,
-                                                      int n_q, int G,
-                                                      const Plan* const* plans, float* out) {
+// One CTA of 512 threads per (sequence, query head): split weights in shared
+// memory, then 4 groups of 128 threads (one per coordinate) sum interleaved
+// splits with independent loads in flight.
+constexpr int kCombineThreads = 512;
+
+__device__ __forceinline__ float block_reduce(float v, bool is_max, float* red) {
+#pragma unroll
+  for (int m = 16; m; m >>= 1) {
+    const float o = __shfl_xor_sync(0xffffffffu, v, m);
+    v = is_max ? fmaxf(v, o) : v + o;
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  v = red[0];
+  for (int w = 1; w < kCombineThreads / 32; ++w) v = is_max ? fmaxf(v, red[w]) : v + red[w];
+  return v;
+}
+
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(
+    const float* __restrict__ part, int n_splits, int n_q, int G, const Plan* const* plans,
+    float* out) {
   const int bh = blockIdx.x, b = bh / n_q, head = bh % n_q;
   const int tid = threadIdx.x;
   const float* pp = part + (size_t)bh * n_splits * kPartStride;
-  float M = -INFINITY;
-  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, pp[(size_t)s * kPartStride]);
-  float Lsum = 0.f, O = 0.f;
-  if (M != -INFINITY) {
-    for (int s = 0; s < n_splits; ++s) {
-      const float* q = pp + (size_t)s * kPartStride;
-      const float sc = exp2f(q[0] - M);
-      Lsum += sc * q[1];
-      O += sc * q[2 + tid];
-    }
+  __shared__ float s_w[1024];
+  __shared__ float s_red[kCombineThreads / 32];
+  __shared__ float s_o[4][kHeadDim];
+  float m = -INFINITY;
+  for (int s = tid; s < n_splits; s += kCombineThreads) m = fmaxf(m, pp[(size_t)s * kPartStride]);
+  const float M = block_reduce(m, true, s_red);
+  float lsum = 0.f;
+  for (int s = tid; s < n_splits; s += kCombineThreads) {
+    const float w = M == -INFINITY ? 0.f : exp2f(pp[(size_t)s * kPartStride] - M);
+    s_w[s] = w;
+    lsum += w * pp[(size_t)s * kPartStride + 1];
   }
-  __shared__ float s_o[kHeadDim];
-  s_o[tid] = O;
+  const float Lsum = block_reduce(lsum, false, s_red);
+  __syncthreads();
+  const int coord = tid & (kHeadDim - 1), grp = tid >> 7;
+  float o = 0.f;
+#pragma unroll 8
+  for (int s = grp; s < n_splits; s += 4) o += s_w[s] * pp[(size_t)s * kPartStride + 2 + coord];
+  s_o[grp][coord] = o;
   __syncthreads();
   if (tid < 32) {
     float y[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) y[q] = s_o[tid + 32 * q];
+    for (int q = 0; q < 4; ++q) {
+      const int i = tid + 32 * q;
+      y[q] = (s_o[0][i] + s_o[1][i]) + (s_o[2][i] + s_o[3][i]);
+    }
 #pragma unroll
     for (int hh = 1; hh < 32; hh <<= 1) {
       const bool upper = (tid & hh) != 0;
@@ -551,7 +580,7 @@ cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches
   cudaError_t e = p.G <= 8 ? launch_decode_nt<1>(p, bits_v, batch, st)
                            : launch_decode_nt<2>(p, bits_v, batch, st);
   if (e != cudaSuccess) return e;
-  combine_kernel<<<batch * n_q, 128, 0, st>>>(part, p.n_splits, n_q, p.G, plans, out);
+  combine_kernel<<<batch * n_q, kCombineThreads, 0, st>>>(part, p.n_splits, n_q, p.G, plans, out);
   return cudaGetLastError();
 }
 
