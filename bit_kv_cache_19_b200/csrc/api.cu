@@ -153,6 +153,14 @@ void build_plan(const kvq_cfg* cfg, int layer, int kv_head, const double* E, Pla
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 }  // namespace
+
+// Lets the other translation units of the library report through
+// kvq_last_error().
+int set_last_error(int code, const char* msg) {
+  g_err = msg;
+  return code;
+}
+
 }  // namespace kvq
 
 using namespace kvq;

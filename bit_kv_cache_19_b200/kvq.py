@@ -69,6 +69,9 @@ _SIGS = {
                                    _i64, _vp, _vp]),
     "kvq_decode_attn": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i64, _vp, _i32, _i32,
                                _vp, _vp, _sz, _vp, _vp]),
+    "kvq_decode_attn_noalloc": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i64, _vp, _i32,
+                                       _i32, _vp, _vp, _vp]),
+    "kvq_decode_noalloc_scratch_bytes": (_sz, []),
 }
 EXPORTS = tuple(_SIGS)
 
@@ -191,3 +194,14 @@ def decode_attn(cfg, plan_ptrs, cache_ptrs, lens, max_len, q, out, ws, status):
     _check(lib().kvq_decode_attn(ctypes.byref(cfg), _ptr(plan_ptrs), _ptr(cache_ptrs), _ptr(lens),
                                  batch, max_len, _ptr(q), _dtype_code(q), n_q, _ptr(out), _ptr(ws),
                                  ws.numel() * ws.element_size(), _ptr(status), _stream()))
+
+
+def decode_attn_noalloc(cfg, plan_ptrs, cache_ptrs, lens, max_len, q, out, status):
+    """kvq_decode_attn without a caller workspace: the split partials go to
+    the library's fixed 4 MiB device scratch (for callers that cannot
+    allocate device memory where they decode). Calls must not overlap on the
+    GPU; the first call on a device must precede any stream capture."""
+    batch, n_q = q.shape[0], q.shape[1]
+    _check(lib().kvq_decode_attn_noalloc(ctypes.byref(cfg), _ptr(plan_ptrs), _ptr(cache_ptrs),
+                                         _ptr(lens), batch, max_len, _ptr(q), _dtype_code(q), n_q,
+                                         _ptr(out), _ptr(status), _stream()))

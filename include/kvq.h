@@ -259,6 +259,44 @@ KVQ_API int kvq_decode_attn(const kvq_cfg* cfg, const void* const* plans_dev,
                     float* out_dev, void* ws_dev, size_t ws_bytes, uint32_t* status_dev,
                     kvq_stream_t stream);
 
+/*
+ * Decode attention without a caller workspace. The paper has no counterpart:
+ * this is a library convenience. Same computation, arguments and results as
+ * kvq_decode_attn, minus ws_dev / ws_bytes.
+ *
+ * Who needs it: callers that cannot allocate device memory where they decode
+ * - a serving loop being recorded into a CUDA graph (cudaMalloc cannot be
+ * captured), an application whose device memory all belongs to a pool this
+ * library cannot reach, or code that must not risk the device-wide
+ * synchronization cudaMalloc / cudaFree can cause mid-step. The caller still
+ * passes every input and output buffer.
+ *
+ * Scratch: the split partials go to a fixed array of
+ * kvq_decode_noalloc_scratch_bytes() (4 MiB) in the library's own device
+ * memory, present on every GPU that loads the library until the process
+ * exits. A call whose partials would not fit (kvq_decode_workspace_bytes of
+ * the same arguments > 4 MiB) returns KVQ_ERR_WORKSPACE and launches nothing.
+ * The call allocates nothing: no cudaMalloc, cudaFree or allocating routine.
+ *
+ * Set-up: the first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture on the device.
+ *
+ * Sharing: every call uses the same array, which keeps the last call's
+ * contents (nothing in it needs clearing: each call writes every partial it
+ * reads). Calls that overlap on the GPU - on different streams, or from
+ * different host threads without ordering - race on the array and may give
+ * wrong outputs; order them on one stream.
+ */
+KVQ_API int kvq_decode_attn_noalloc(const kvq_cfg* cfg, const void* const* plans_dev,
+                                    const void* const* cache_dev, const int32_t* len_dev,
+                                    int batch, int64_t max_len, const void* q_dev, int q_dtype,
+                                    int n_q_heads, float* out_dev, uint32_t* status_dev,
+                                    kvq_stream_t stream);
+
+/* Size of the fixed scratch used by kvq_decode_attn_noalloc (4 MiB). */
+KVQ_API size_t kvq_decode_noalloc_scratch_bytes(void);
+
 #ifdef __cplusplus
 }
 #endif
