@@ -28,11 +28,12 @@ struct QuantParams {
   uint32_t* status;
 };
 cudaError_t launch_quantize_append(const QuantParams& p, cudaStream_t st);
-int decode_splits(int64_t max_len);
+size_t decode_workspace_bytes_for(int batch, int n_q, int n_kv, int bits_k, int bits_v,
+                                  int64_t max_len);
 cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches, const int32_t* len,
                           int batch, int64_t max_len, const void* q, int q_dtype, int n_q, int n_kv,
-                          int bits_k, int bits_v, float* out, float* part, uint32_t* status,
-                          cudaStream_t st);
+                          int bits_k, int bits_v, float* out, void* ws, size_t ws_bytes,
+                          uint32_t* status, cudaStream_t st);
 
 namespace {
 
@@ -191,9 +192,11 @@ size_t kvq_alloc_workspace_bytes(const kvq_cfg* cfg) {
 
 size_t kvq_decode_workspace_bytes(const kvq_cfg* cfg, int batch, int n_q_heads, int64_t max_len) {
   if (check_cfg(cfg) != KVQ_OK || batch < 1 || n_q_heads < 1 || max_len < 1 ||
-      max_len > 0x7FFFFFFF)
+      max_len > 0x7FFFFFFF || n_q_heads % cfg->n_kv_heads != 0 ||
+      n_q_heads / cfg->n_kv_heads > 16)
     return 0;
-  return align_up((size_t)batch * n_q_heads * decode_splits(max_len) * 130 * sizeof(float), 256);
+  return decode_workspace_bytes_for(batch, n_q_heads, cfg->n_kv_heads, cfg->bits_k, cfg->bits_v,
+                                    max_len);
 }
 
 int kvq_codebook(int bits, float* centroids, float* thresholds, double* distortion) {
@@ -310,7 +313,7 @@ int kvq_decode_attn(const kvq_cfg* cfg, const void* const* plans_dev, const void
   cudaError_t e = launch_decode(reinterpret_cast<const Plan* const*>(plans_dev),
                                 reinterpret_cast<const uint8_t* const*>(cache_dev), len_dev, batch,
                                 max_len, q_dev, q_dtype, n_q_heads, cfg->n_kv_heads, cfg->bits_k,
-                                cfg->bits_v, out_dev, reinterpret_cast<float*>(ws_dev), status_dev,
+                                cfg->bits_v, out_dev, ws_dev, ws_bytes, status_dev,
                                 reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode_attn");
   return KVQ_OK;

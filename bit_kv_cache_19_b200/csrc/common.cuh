@@ -16,7 +16,6 @@ namespace kvq {
 constexpr int kHeadDim = 128;
 constexpr int kBlocks = 64;
 constexpr int kTile = 32;
-constexpr int kMaxHalf = 32;
 
 // Plan record, byte layout documented in kvq.h.
 struct Plan {

@@ -1,30 +1,37 @@
-// Packed-cache decode attention (split-K) and the split combine.
+// Packed-cache decode attention: split-K over the context with an in-kernel
+// two-level merge of the splits.
 //
 // "RoPE-Aware Bit Allocation for KV-Cache Quantization", abstract: the
 // packed-cache serving path runs decode attention directly on the packed
 // K/V cache (the pages report it faster than fp16 FlashAttention2 at 128K on
 // H800). This is an sm_100a design of its own:
 //
-// * Work: CTA = (split, KV head, sequence), 4 warps; each warp owns every 4th
-//   32-token tile of the CTA's range and streams its tiles into a private
-//   3-stage shared-memory ring with 1-D bulk copies (cp.async.bulk +
-//   mbarrier, no multicast).
-// * Keys: the tile's codes are unpacked straight into the A fragments of
-//   mma.sync m16n8k16 (16 tokens x 16 plan-ordered coordinates): each 32-bit
-//   register is one RoPE block (codes of coordinates j and j + 64) of one
-//   token, looked up as an fp16 pair. The B operand is the query group
-//   (G <= 16 heads) pre-multiplied by the block scales a_hat_j, log2(e) and
-//   1/sqrt(128), split into hi + lo fp16 parts so the logits keep fp32
-//   accuracy. Width-uniform half k-steps (<= 4 blocks of one width) let the
-//   unpack use compile-time shifts.
+// * Work: CTA = (split, KV head, sequence), 8 warps, sized so the grid is one
+//   wave. Each warp owns every 8th 32-token tile of the CTA's range and
+//   streams its tiles into a private 3-stage shared-memory ring with 1-D bulk
+//   copies (cp.async.bulk + mbarrier, no multicast).
+// * Keys: the logits S[32 tokens x 8 heads] are mma.sync m16n8k8 products.
+//   One MMA covers one "half step" of the plan: <= 4 RoPE blocks of one width
+//   W. Each 32-bit A register is one block (codes of coordinates j and
+//   j + 64) of one token, looked up as an fp16 pair; the packed layout puts
+//   the 4 tokens a lane needs (g, g + 8, g + 16, g + 24) in 8W contiguous
+//   bits. Half steps of one width form a class, so the unpack of a class is
+//   compiled for its W and each lane's addresses are plain arithmetic. The B
+//   operand is the query group pre-multiplied by a_hat_j, log2(e) and
+//   1/sqrt(128), scaled by 2^sigma per head and split into hi + lo fp16, so
+//   the logits keep ~fp32 accuracy.
 // * Softmax: base-2 online softmax per head on the fp32 accumulators, scaled
-//   by the fp16 key norms; masked positions past the sequence length.
-// * Values: P' = p * n^V (fp16) is transposed in registers (movmatrix) into
-//   the B operand of O^T(128 x G) += Vhat^T(128 x 16 tokens) P'^T, where
-//   Vhat^T's fragments (one rotated coordinate, two tokens) come from the
-//   value tile's pair codes. Output stays in the rotated value domain.
-// * Combine: merges the (m, l, o) partials of all splits, applies the inverse
-//   randomised Hadamard transform and 1/l.
+//   by the fp16 key norms; positions past the sequence length are masked.
+// * Values: P' = p * n^V (fp16) goes from the accumulator layout to the B
+//   operand with movmatrix (register transpose); O^T(128 x G) += Vhat^T(128 x
+//   16 tokens) P'^T with A registers holding one rotated coordinate of two
+//   tokens (pair codes of adjacent value slots).
+// * Merge: the 8 warps merge in shared memory into one (m, l, o[128]) per
+//   head; the last CTA to finish in each group of 8 splits merges the group,
+//   and the last group merges the groups, undoes the value rotation
+//   (inverse Walsh-Hadamard, signs) and writes o / l. Arrivals are counted
+//   with atomics on counters that the last arriver resets, so a completed
+//   call leaves them at zero.
 #include <algorithm>
 #include <atomic>
 
@@ -34,11 +41,17 @@ namespace kvq {
 
 __constant__ uint16_t c_c16[KVQ_CB_N_C16] = KVQ_CB_C16;
 
-constexpr int kWarps = 4;
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
 constexpr int kStages = 3;
-constexpr int kMaxK = 12;       // k-steps of 16 coordinates (2 half-steps each)
+constexpr int kMaxHalf = 24;    // half steps of <= 4 blocks (<= 64/4 + 8)
+constexpr int kMaxClass = 8;    // widths 1..8
 constexpr int kPairLut = 340;   // pair tables of widths 1..4: 4 + 16 + 64 + 256
 constexpr int kPartStride = 130;
+constexpr int kGroup = 8;       // splits merged per first-level group
+constexpr int kMaxSplits = 1024;
+constexpr int kCntStride = 1 + kMaxSplits / kGroup;  // counters per (sequence, KV head)
+constexpr int kFallbackSlots = 1024;                  // CTA slots when no device answers
 
 __host__ __device__ constexpr int pair_off(int w) { return ((1 << (2 * w)) - 4) / 3; }
 
@@ -50,9 +63,12 @@ struct DecodeParams {
   int q_dtype;
   int n_q, n_kv, G;
   int max_len;
-  int n_splits, tiles_per_split;
+  int n_splits, tiles_per_split, n_groups;
   int tile_bytes;
-  float* part;  // [batch][n_q][n_splits][130] = m, l, o[128]
+  unsigned int* cnt_end;   // counters of pair k at cnt_end - (k + 1) * kCntStride
+  float* part;             // [batch][n_kv][n_splits][G][130] = m, l, o[128]
+  float* gpart;            // [batch][n_kv][n_groups][G][130]
+  float* out;              // [batch][n_q][128]
   uint32_t* status;
 };
 
@@ -61,10 +77,12 @@ struct alignas(128) Smem {
   uint32_t lut_pair[kPairLut];      // fp16 pairs (c[lo], c[hi]) for widths 1..4
   uint16_t lut1[KVQ_CB_N_C16];      // fp16 centroids, width w at 2^w - 2
   float inv_scale[16];              // 2^-sigma of each head's q' scaling
-  uint32_t flags;
-  uint4 qfrag[2][kMaxK][32];        // per (n-tile, k-step, lane): hi b0, hi b1, lo b0, lo b1
+  uint2 qfrag[2][kMaxHalf][32];     // per (n-tile, half step, lane): hi, lo
   unsigned long long bar[kWarps][kStages];
-  float qp[16][kHeadDim];           // q' (fp32) of the head group
+  int n_class;
+  int cls_w[kMaxClass], cls_hs0[kMaxClass], cls_nhs[kMaxClass], cls_seg0[kMaxClass],
+      cls_last[kMaxClass];
+  int is_last;
 };
 
 template <int W>
@@ -77,13 +95,10 @@ __device__ __forceinline__ uint32_t pair_lookup(const Smem& sm, uint32_t f) {
   }
 }
 
-// Four 2W-bit pair fields at bits [8Wq, 8Wq + 8W) of a segment, as fp16 pairs.
+// Four 2W-bit pair fields starting at bit `sh` of wp[0] (8W bits), as fp16 pairs.
 template <int W>
-__device__ __forceinline__ void fields4(const Smem& sm, const uint32_t* seg, int q,
+__device__ __forceinline__ void fields4(const Smem& sm, const uint32_t* wp, uint32_t sh,
                                         uint32_t (&out)[4]) {
-  const int bit = 8 * W * q;
-  const uint32_t* wp = seg + (bit >> 5);
-  const uint32_t sh = bit & 31;
   constexpr uint32_t mask = (1u << (2 * W)) - 1u;
   if constexpr (W <= 4) {
     const uint32_t v = funnel_r(wp[0], wp[1], sh);
@@ -97,69 +112,131 @@ __device__ __forceinline__ void fields4(const Smem& sm, const uint32_t* seg, int
   }
 }
 
-// Key fragments of one half k-step: block (rank0 + c) of width w, tokens
-// g, g + 8, g + 16, g + 24 (K slots 4g .. 4g + 3).
-__device__ __forceinline__ void key_half(const Smem& sm, const uint32_t* kw, int hs, int g, int c,
-                                         uint32_t (&o)[4]) {
-  o[0] = o[1] = o[2] = o[3] = 0u;
-  if (hs >= sm.plan.n_half || c >= sm.plan.hs_count[hs]) return;
-  const uint32_t* seg = kw + sm.plan.seg_off[sm.plan.hs_rank0[hs] + c];
-  switch (sm.plan.hs_width[hs]) {
-    case 1: fields4<1>(sm, seg, g, o); break;
-    case 2: fields4<2>(sm, seg, g, o); break;
-    case 3: fields4<3>(sm, seg, g, o); break;
-    case 4: fields4<4>(sm, seg, g, o); break;
-    case 5: fields4<5>(sm, seg, g, o); break;
-    case 6: fields4<6>(sm, seg, g, o); break;
-    case 7: fields4<7>(sm, seg, g, o); break;
-    default: fields4<8>(sm, seg, g, o); break;
+// D(16x8 f32) += A(16x8 f16, row) B(8x8 f16, col).
+__device__ __forceinline__ void mma_1688(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+
+// Logits of one width class: half steps hs0 .. hs0 + nhs - 1, each <= 4
+// blocks of width W (the last one has `last` blocks). Lane (g, c) takes block
+// c of every half step, tokens g, g + 8 (m-tile 0) and g + 16, g + 24 (m-tile 1).
+template <int W, int NT>
+__device__ __forceinline__ void key_class(const Smem& sm, const uint32_t* kw, int hs0, int nhs,
+                                          int seg0, int last, int g, int c, int lane,
+                                          float (&s)[2][NT][4]) {
+  const uint32_t* base = kw + seg0 + 2 * W * c + ((W * g) >> 2);
+  const uint32_t sh = (uint32_t)(8 * W * g) & 31u;
+  for (int i = 0; i < nhs; ++i) {
+    uint32_t A[4] = {0u, 0u, 0u, 0u};
+    if (i + 1 < nhs || c < last) fields4<W>(sm, base + 8 * W * i, sh, A);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const uint2 qf = sm.qfrag[nt][hs0 + i][lane];
+      mma_1688(s[0][nt], A[0], A[1], qf.x);
+      mma_1688(s[0][nt], A[0], A[1], qf.y);
+      mma_1688(s[1][nt], A[2], A[3], qf.x);
+      mma_1688(s[1][nt], A[2], A[3], qf.y);
+    }
   }
 }
 
-__device__ __forceinline__ void write_empty_partial(const DecodeParams& p, int b, int h, int split) {
-  for (int head = 0; head < p.G; ++head) {
-    float* dst = p.part + (((size_t)b * p.n_q + h * p.G + head) * p.n_splits + split) * kPartStride;
-    for (int i = threadIdx.x; i < kPartStride; i += blockDim.x)
-      dst[i] = i == 0 ? -INFINITY : 0.f;
+// Inverse value rotation of one head held by a warp (o[128] in `src`),
+// written as out[i] = s_i (H o)_i * inv.
+__device__ __forceinline__ void warp_unrotate_store(const float* src, const Plan& pl, float inv,
+                                                   float* out, int lane) {
+  float y[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) y[q] = src[lane + 32 * q];
+#pragma unroll
+  for (int hh = 1; hh < 32; hh <<= 1) {
+    const bool upper = (lane & hh) != 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float x = __shfl_xor_sync(0xffffffffu, y[q], hh);
+      y[q] = upper ? x - y[q] : y[q] + x;
+    }
+  }
+  const float a0 = y[0] + y[1], a1 = y[0] - y[1], a2 = y[2] + y[3], a3 = y[2] - y[3];
+  y[0] = a0 + a2;
+  y[2] = a0 - a2;
+  y[1] = a1 + a3;
+  y[3] = a1 - a3;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int i = lane + 32 * q;
+    const float sgn = ((pl.v_sign[i >> 5] >> (i & 31)) & 1u) ? -1.f : 1.f;
+    out[i] = sgn * y[q] * inv;
+  }
+}
+
+// Merge n records per head (record s of head h at src + s * rec_stride +
+// h * 130) into dst (record h at dst + h * 130), for G heads.
+__device__ __forceinline__ void merge_records(const float* src, int n, size_t rec_stride, int G,
+                                              float* dst) {
+  const int tid = threadIdx.x;
+  for (int head = tid >> 7; head < G; head += kThreads / 128) {
+    const int x = tid & 127;
+    const float* r = src + (size_t)head * kPartStride;
+    float M = -INFINITY;
+    for (int s = 0; s < n; ++s) M = fmaxf(M, r[s * rec_stride]);
+    float L = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll 4
+      for (int s = 0; s < n; ++s) {
+        const float* q = r + s * rec_stride;
+        const float w = exp2f(q[0] - M);
+        L += w * q[1];
+        O += w * q[2 + x];
+      }
+    }
+    float* d = dst + (size_t)head * kPartStride;
+    d[2 + x] = O;
+    if (x == 0) {
+      d[0] = M;
+      d[1] = L;
+    }
   }
 }
 
 template <int BV, int NT>
-__global__ void __launch_bounds__(kWarps * 32) decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
   uint8_t* const stage_base = smem_raw + sizeof(Smem);
 
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
+  const int G = p.G;
+  const size_t bh = (size_t)b * p.n_kv + h;
+  float* const my_part = p.part + (bh * p.n_splits + split) * G * kPartStride;
 
-  // ---- plan and lookup tables
+  // ---- plan, lookup tables
   {
     const uint4* src = reinterpret_cast<const uint4*>(p.plans[b] + h);
     uint4* dst = reinterpret_cast<uint4*>(&sm.plan);
-    for (int i = tid; i < KVQ_PLAN_BYTES / 16; i += blockDim.x) dst[i] = src[i];
-    for (int i = tid; i < KVQ_CB_N_C16; i += blockDim.x) sm.lut1[i] = c_c16[i];
-    for (int i = tid; i < kPairLut; i += blockDim.x) {
-      int w = 1;
-      while (w < 4 && i >= pair_off(w + 1)) ++w;
+    for (int i = tid; i < KVQ_PLAN_BYTES / 16; i += kThreads) dst[i] = src[i];
+    for (int i = tid; i < KVQ_CB_N_C16; i += kThreads) sm.lut1[i] = c_c16[i];
+    for (int i = tid; i < kPairLut; i += kThreads) {
+      const int w = i < 4 ? 1 : i < 20 ? 2 : i < 84 ? 3 : 4;
       const int f = i - pair_off(w);
       const uint32_t lo = c_c16[cb_c_off(w) + (f & ((1 << w) - 1))];
       const uint32_t hi = c_c16[cb_c_off(w) + (f >> w)];
       sm.lut_pair[i] = lo | (hi << 16);
     }
-    if (tid == 0) sm.flags = 0u;
   }
   __syncthreads();
   const uint8_t* cache = p.caches[b];
   const int bk = sm.plan.bits_k;
-  if (sm.plan.magic != KVQ_PLAN_MAGIC || sm.plan.bits_v != BV || bk < 1 || bk > 8 ||
-      p.tile_bytes != tile_bytes(bk, BV) || sm.plan.n_half > 2 * kMaxK ||
-      (reinterpret_cast<uintptr_t>(cache) & 15) != 0) {
-    if (tid == 0) atomicOr(p.status, KVQ_FLAG_BAD_PLAN);
-    write_empty_partial(p, b, h, split);
-    return;
-  }
-  int L = p.len[b];
+  const int n_half = sm.plan.n_half;
+  const bool bad = sm.plan.magic != KVQ_PLAN_MAGIC || sm.plan.bits_v != BV || bk < 1 || bk > 8 ||
+                   p.tile_bytes != tile_bytes(bk, BV) || n_half < 1 || n_half > kMaxHalf ||
+                   (reinterpret_cast<uintptr_t>(cache) & 15) != 0;
+  if (bad && tid == 0) atomicOr(p.status, KVQ_FLAG_BAD_PLAN);
+  int L = bad ? 0 : p.len[b];
   if (L > p.max_len) {
     if (tid == 0 && split == 0 && h == 0) atomicOr(p.status, KVQ_FLAG_CAPACITY);
     L = p.max_len;
@@ -168,76 +245,7 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(const DecodeParams 
   const int n_tiles = (L + kTile - 1) / kTile;
   const int tb = split * p.tiles_per_split;
   const int te = min(n_tiles, tb + p.tiles_per_split);
-  if (tb >= te) {
-    write_empty_partial(p, b, h, split);
-    return;
-  }
-
-  // ---- query prologue: q' = q a_hat_j log2(e) / sqrt(128), per-head 2^sigma
-  //      scaling into the fp16 range, hi/lo split into B fragments
-  const int G = p.G;
-  for (int i = tid; i < 16 * kHeadDim; i += blockDim.x) {
-    const int head = i >> 7, x = i & 127;
-    float v = 0.f;
-    if (head < G) {
-      const size_t qi = ((size_t)b * p.n_q + h * G + head) * kHeadDim + x;
-      v = load_as_float(p.q, p.q_dtype, qi) * sm.plan.a_hat[x & 63] * 0.12751743074f;
-    }
-    sm.qp[head][x] = v;  // 0.12751743 = log2(e) / sqrt(128)
-  }
-  __syncthreads();
-  for (int head = warp; head < 16; head += kWarps) {
-    float mx = 0.f;
-    for (int x = lane; x < kHeadDim; x += 32) mx = fmaxf(mx, fabsf(sm.qp[head][x]));
-#pragma unroll
-    for (int m = 16; m; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
-    const int sigma = (mx > 0.f && isfinite(mx)) ? 14 - ilogbf(mx) : 0;
-    const float sc = ldexpf(1.f, sigma);
-    for (int x = lane; x < kHeadDim; x += 32) sm.qp[head][x] *= sc;
-    if (lane == 0) sm.inv_scale[head] = ldexpf(1.f, -sigma);
-  }
-  __syncthreads();
-  const int n_half = sm.plan.n_half;
-  const int n_k = (n_half + 1) >> 1;
-  for (int e = tid; e < NT * n_k * 32; e += blockDim.x) {
-    const int ln = e & 31, ks = (e >> 5) % n_k, nt = (e >> 5) / n_k;
-    const int head = 8 * nt + (ln >> 2), cc = ln & 3;
-    float x[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int hs = 2 * ks + half;
-      if (hs < n_half && cc < sm.plan.hs_count[hs]) {
-        const int j = sm.plan.order[sm.plan.hs_rank0[hs] + cc];
-        x[2 * half] = sm.qp[head][j];
-        x[2 * half + 1] = sm.qp[head][j + 64];
-      }
-    }
-    const uint32_t hi0 = pack_half2(x[0], x[1]), hi1 = pack_half2(x[2], x[3]);
-    const __half2 h0 = *reinterpret_cast<const __half2*>(&hi0);
-    const __half2 h1 = *reinterpret_cast<const __half2*>(&hi1);
-    const uint32_t lo0 = pack_half2(x[0] - __low2float(h0), x[1] - __high2float(h0));
-    const uint32_t lo1 = pack_half2(x[2] - __low2float(h1), x[3] - __high2float(h1));
-    sm.qfrag[nt][ks][ln] = make_uint4(hi0, hi1, lo0, lo1);
-  }
-  if (tid < kWarps * kStages) mbar_init(&sm.bar[tid / kStages][tid % kStages], 1);
-  fence_proxy_async();
-  __syncthreads();
-
-  // ---- per-warp pipeline over the warp's tiles
-  const int tbytes = p.tile_bytes;
-  uint8_t* const my_stages = stage_base + (size_t)warp * kStages * tbytes;
-  const int n_mine = max(0, (te - tb - warp + kWarps - 1) / kWarps);
-  auto tile_of = [&](int i) { return tb + warp + i * kWarps; };
-  auto issue = [&](int i) {
-    const int s = i % kStages;
-    unsigned long long* bar = &sm.bar[warp][s];
-    mbar_expect_tx(bar, (uint32_t)tbytes);
-    bulk_g2s(my_stages + s * tbytes, cache + ((size_t)tile_of(i) * p.n_kv + h) * tbytes,
-             (uint32_t)tbytes, bar);
-  };
-  if (lane == 0)
-    for (int i = 0; i < min(kStages, n_mine); ++i) issue(i);
-  __syncwarp();
+  const bool has_work = tb < te;
 
   float o[8][NT][4];
   float m_run[NT][2], l_run[NT][2];
@@ -255,128 +263,210 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(const DecodeParams 
       l_run[nt][e] = 0.f;
     }
 
-  int consumed = 0;
-  bool timed_out = false;
-  for (int i = 0; i < n_mine; ++i) {
-    const int s = i % kStages;
-    const bool ok = mbar_wait_bounded(&sm.bar[warp][s], (uint32_t)((i / kStages) & 1));
-    if (!__all_sync(0xffffffffu, ok)) {
-      timed_out = true;
-      break;
+  if (has_work) {
+    // ---- classes of equal width over the half steps
+    if (tid == 0) {
+      int nc = 0;
+      for (int hs = 0; hs < n_half;) {
+        const int w = sm.plan.hs_width[hs];
+        int e = hs;
+        while (e < n_half && sm.plan.hs_width[e] == w) ++e;
+        sm.cls_w[nc] = w;
+        sm.cls_hs0[nc] = hs;
+        sm.cls_nhs[nc] = e - hs;
+        sm.cls_seg0[nc] = sm.plan.seg_off[sm.plan.hs_rank0[hs]];
+        sm.cls_last[nc] = sm.plan.hs_count[e - 1];
+        ++nc;
+        hs = e;
+      }
+      sm.n_class = nc;
     }
-    consumed = i + 1;
-    const int tile = tile_of(i);
-    const int nvalid = min(kTile, L - tile * kTile);
-    const uint32_t* kw = reinterpret_cast<const uint32_t*>(my_stages + s * tbytes);
-    const uint32_t* vw = kw + 128 * bk;
-    const __half* nrm = reinterpret_cast<const __half*>(vw + 128 * BV);
+    // ---- query prologue (q' staged in the tile ring, not in use yet):
+    //      q' = q a_hat_j log2(e) / sqrt(128); per-head 2^sigma scaling into
+    //      the fp16 range; hi/lo split into the B fragments of each half step
+    float* qp = reinterpret_cast<float*>(stage_base);  // [16][128]
+    for (int i = tid; i < 16 * kHeadDim; i += kThreads) {
+      const int head = i >> 7, x = i & 127;
+      float v = 0.f;
+      if (head < G) {
+        const size_t qi = ((size_t)b * p.n_q + h * G + head) * kHeadDim + x;
+        v = load_as_float(p.q, p.q_dtype, qi) * sm.plan.a_hat[x & 63] * 0.12751743074f;
+      }
+      qp[i] = v;  // 0.12751743 = log2(e) / sqrt(128)
+    }
+    __syncthreads();
+    for (int head = warp; head < 8 * NT; head += kWarps) {
+      float mx = 0.f;
+      for (int x = lane; x < kHeadDim; x += 32) mx = fmaxf(mx, fabsf(qp[head * kHeadDim + x]));
+#pragma unroll
+      for (int m = 16; m; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+      const int sigma = (mx > 0.f && isfinite(mx)) ? 14 - ilogbf(mx) : 0;
+      const float sc = ldexpf(1.f, sigma);
+      for (int x = lane; x < kHeadDim; x += 32) qp[head * kHeadDim + x] *= sc;
+      if (lane == 0) sm.inv_scale[head] = ldexpf(1.f, -sigma);
+    }
+    __syncthreads();
+    for (int e = tid; e < NT * n_half * 32; e += kThreads) {
+      const int ln = e & 31, hs = (e >> 5) % n_half, nt = (e >> 5) / n_half;
+      const int head = 8 * nt + (ln >> 2), cc = ln & 3;
+      float x0 = 0.f, x1 = 0.f;
+      if (cc < sm.plan.hs_count[hs]) {
+        const int j = sm.plan.order[sm.plan.hs_rank0[hs] + cc];
+        x0 = qp[head * kHeadDim + j];
+        x1 = qp[head * kHeadDim + j + 64];
+      }
+      const uint32_t hi = pack_half2(x0, x1);
+      const __half2 hh = *reinterpret_cast<const __half2*>(&hi);
+      const uint32_t lo = pack_half2(x0 - __low2float(hh), x1 - __high2float(hh));
+      sm.qfrag[nt][hs][ln] = make_uint2(hi, lo);
+    }
+    if (tid < kWarps * kStages) mbar_init(&sm.bar[tid / kStages][tid % kStages], 1);
+    fence_proxy_async();
+    __syncthreads();
 
-    // keys: S[32 tokens x 8 NT heads] on the tensor cores
-    float sacc[2][NT][4];
+    // ---- per-warp pipeline over the warp's tiles
+    const int tbytes = p.tile_bytes;
+    uint8_t* const my_stages = stage_base + (size_t)warp * kStages * tbytes;
+    const int n_mine = max(0, (te - tb - warp + kWarps - 1) / kWarps);
+    auto tile_of = [&](int i) { return tb + warp + i * kWarps; };
+    auto issue = [&](int i) {
+      const int s = i % kStages;
+      unsigned long long* bar = &sm.bar[warp][s];
+      mbar_expect_tx(bar, (uint32_t)tbytes);
+      bulk_g2s(my_stages + s * tbytes, cache + ((size_t)tile_of(i) * p.n_kv + h) * tbytes,
+               (uint32_t)tbytes, bar);
+    };
+    if (lane == 0)
+      for (int i = 0; i < min(kStages, n_mine); ++i) issue(i);
+    __syncwarp();
+
+    const int n_class = sm.n_class;
+    const uint32_t v_sh = (uint32_t)(8 * BV * c) & 31u;
+    const int v_off = (BV * c) >> 2;
+    int consumed = 0;
+    bool timed_out = false;
+    for (int i = 0; i < n_mine; ++i) {
+      const int s = i % kStages;
+      const bool ok = mbar_wait_bounded(&sm.bar[warp][s], (uint32_t)((i / kStages) & 1));
+      if (!__all_sync(0xffffffffu, ok)) {
+        timed_out = true;
+        break;
+      }
+      consumed = i + 1;
+      const int tile = tile_of(i);
+      const int nvalid = min(kTile, L - tile * kTile);
+      const uint32_t* kw = reinterpret_cast<const uint32_t*>(my_stages + s * tbytes);
+      const uint32_t* vw = kw + 128 * bk;
+      const __half* nrm = reinterpret_cast<const __half*>(vw + 128 * BV);
+
+      // keys: S[32 tokens x 8 NT heads] on the tensor cores
+      float sacc[2][NT][4];
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
+      for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int r = 0; r < 4; ++r) sacc[mt][nt][r] = 0.f;
-    for (int ks = 0; ks < n_k; ++ks) {
-      uint32_t A0[4], A1[4];
-      key_half(sm, kw, 2 * ks, g, c, A0);
-      key_half(sm, kw, 2 * ks + 1, g, c, A1);
+          for (int r = 0; r < 4; ++r) sacc[mt][nt][r] = 0.f;
+      for (int ci = 0; ci < n_class; ++ci) {
+        const int hs0 = sm.cls_hs0[ci], nhs = sm.cls_nhs[ci], seg0 = sm.cls_seg0[ci],
+                  last = sm.cls_last[ci];
+        switch (sm.cls_w[ci]) {
+          case 1: key_class<1, NT>(sm, kw, hs0, nhs, seg0, last, g, c, lane, sacc); break;
+          case 2: key_class<2, NT>(sm, kw, hs0, nhs, seg0, last, g, c, lane, sacc); break;
+          case 3: key_class<3, NT>(sm, kw, hs0, nhs, seg0, last, g, c, lane, sacc); break;
+          case 4: key_class<4, NT>(sm, kw, hs0, nhs, seg0, last, g, c, lane, sacc); break;
+          case 5: key_class<5, NT>(sm, kw, hs0, nhs, seg0, last, g, c, lane, sacc); break;
+          case 6: key_class<6, NT>(sm, kw, hs0, nhs, seg0, last, g, c, lane, sacc); break;
+          case 7: key_class<7, NT>(sm, kw, hs0, nhs, seg0, last, g, c, lane, sacc); break;
+          default: key_class<8, NT>(sm, kw, hs0, nhs, seg0, last, g, c, lane, sacc); break;
+        }
+      }
+
+      // online softmax (base 2); this thread's tokens are g + 8 r, r = 0..3
+      float nk[4], nv[4];
+      bool val[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int tok = g + 8 * r;
+        val[r] = tok < nvalid;
+        nk[r] = val[r] ? __half2float(nrm[tok]) : 0.f;
+        nv[r] = val[r] ? __half2float(nrm[kTile + tok]) : 0.f;
+      }
+      uint32_t pb0[2][NT], pb1[2][NT];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const uint4 qf = sm.qfrag[nt][ks][lane];
-        mma_16816(sacc[0][nt], A0[0], A0[1], A1[0], A1[1], qf.x, qf.y);
-        mma_16816(sacc[0][nt], A0[0], A0[1], A1[0], A1[1], qf.z, qf.w);
-        mma_16816(sacc[1][nt], A0[2], A0[3], A1[2], A1[3], qf.x, qf.y);
-        mma_16816(sacc[1][nt], A0[2], A0[3], A1[2], A1[3], qf.z, qf.w);
-      }
-    }
-
-    // online softmax (base 2); this thread's tokens are g + 8 r, r = 0..3
-    float nk[4], nv[4];
-    bool val[4];
+        float pe[2][4];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int tok = g + 8 * r;
-      val[r] = tok < nvalid;
-      nk[r] = val[r] ? __half2float(nrm[tok]) : 0.f;
-      nv[r] = val[r] ? __half2float(nrm[kTile + tok]) : 0.f;
-    }
-    uint32_t pb0[2][NT], pb1[2][NT];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      float pe[2][4];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float isc = sm.inv_scale[8 * nt + 2 * c + e];
-        float sv[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int mt = r >> 1, rr = r & 1;
-          sv[r] = val[r] ? sacc[mt][nt][2 * rr + e] * nk[r] * isc : -INFINITY;
-        }
-        float mx = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        const float m_new = fmaxf(m_run[nt][e], mx);
-        float alpha = 1.f, lsum = 0.f;
-        if (m_new != -INFINITY) {
-          alpha = exp2f(m_run[nt][e] - m_new);
+        for (int e = 0; e < 2; ++e) {
+          const float isc = sm.inv_scale[8 * nt + 2 * c + e];
+          float sv[4];
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
-            const float pr = exp2f(sv[r] - m_new);
-            lsum += pr;
-            pe[e][r] = val[r] ? pr * nv[r] : 0.f;
+            const int mt = r >> 1, rr = r & 1;
+            sv[r] = val[r] ? sacc[mt][nt][2 * rr + e] * nk[r] * isc : -INFINITY;
           }
-        } else {
+          float mx = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+          const float m_new = fmaxf(m_run[nt][e], mx);
+          float alpha = 1.f, lsum = 0.f;
+          if (m_new != -INFINITY) {
+            alpha = exp2f(m_run[nt][e] - m_new);
 #pragma unroll
-          for (int r = 0; r < 4; ++r) pe[e][r] = 0.f;
+            for (int r = 0; r < 4; ++r) {
+              const float pr = exp2f(sv[r] - m_new);
+              lsum += pr;
+              pe[e][r] = val[r] ? pr * nv[r] : 0.f;
+            }
+          } else {
+#pragma unroll
+            for (int r = 0; r < 4; ++r) pe[e][r] = 0.f;
+          }
+          l_run[nt][e] = l_run[nt][e] * alpha + lsum;
+          m_run[nt][e] = m_new;
+          if (alpha != 1.f) {
+#pragma unroll
+            for (int mu = 0; mu < 8; ++mu) {
+              o[mu][nt][e] *= alpha;
+              o[mu][nt][2 + e] *= alpha;
+            }
+          }
         }
-        l_run[nt][e] = l_run[nt][e] * alpha + lsum;
-        m_run[nt][e] = m_new;
-        if (alpha != 1.f) {
 #pragma unroll
-          for (int mu = 0; mu < 8; ++mu) {
-            o[mu][nt][e] *= alpha;
-            o[mu][nt][2 + e] *= alpha;
-          }
+        for (int mt = 0; mt < 2; ++mt) {
+          pb0[mt][nt] = movmatrix_trans(pack_half2(pe[0][2 * mt], pe[1][2 * mt]));
+          pb1[mt][nt] = movmatrix_trans(pack_half2(pe[0][2 * mt + 1], pe[1][2 * mt + 1]));
         }
       }
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-        pb0[mt][nt] = movmatrix_trans(pack_half2(pe[0][2 * mt], pe[1][2 * mt]));
-        pb1[mt][nt] = movmatrix_trans(pack_half2(pe[0][2 * mt + 1], pe[1][2 * mt + 1]));
-      }
-    }
 
-    // values: O^T[128 x 8 NT] += Vhat^T[128 x 32 tokens] P'^T
+      // values: O^T[128 x 8 NT] += Vhat^T[128 x 32 tokens] P'^T
 #pragma unroll
-    for (int mu = 0; mu < 8; ++mu) {
-      uint32_t F0[4], F1[4];
-      fields4<BV>(sm, vw + (16 * mu + g) * BV, c, F0);
-      fields4<BV>(sm, vw + (16 * mu + g + 8) * BV, c, F1);
+      for (int mu = 0; mu < 8; ++mu) {
+        uint32_t F0[4], F1[4];
+        fields4<BV>(sm, vw + (16 * mu + g) * BV + v_off, v_sh, F0);
+        fields4<BV>(sm, vw + (16 * mu + g + 8) * BV + v_off, v_sh, F1);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        mma_16816(o[mu][nt], F0[0], F1[0], F0[1], F1[1], pb0[0][nt], pb1[0][nt]);
-        mma_16816(o[mu][nt], F0[2], F1[2], F0[3], F1[3], pb0[1][nt], pb1[1][nt]);
+        for (int nt = 0; nt < NT; ++nt) {
+          mma_16816(o[mu][nt], F0[0], F1[0], F0[1], F1[1], pb0[0][nt], pb1[0][nt]);
+          mma_16816(o[mu][nt], F0[2], F1[2], F0[3], F1[3], pb0[1][nt], pb1[1][nt]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0 && i + kStages < n_mine) {
+        fence_proxy_async();
+        issue(i + kStages);
       }
     }
-    __syncwarp();
-    if (lane == 0 && i + kStages < n_mine) {
-      fence_proxy_async();
-      issue(i + kStages);
+    if (timed_out) {
+      if (lane == 0) atomicOr(p.status, KVQ_FLAG_TIMEOUT);
+      // let the copies this warp still has in flight land before leaving
+      for (int i = consumed; i < min(n_mine, consumed + kStages); ++i)
+        (void)mbar_wait_bounded(&sm.bar[warp][i % kStages], (uint32_t)((i / kStages) & 1));
     }
   }
-  if (timed_out) {
-    if (lane == 0) atomicOr(p.status, KVQ_FLAG_TIMEOUT);
-    // let the copies this warp still has in flight land before leaving
-    for (int i = consumed; i < min(n_mine, consumed + kStages); ++i)
-      (void)mbar_wait_bounded(&sm.bar[warp][i % kStages], (uint32_t)((i / kStages) & 1));
-  }
 
-  // ---- CTA merge of the 4 warps' (m, l, O), then one partial per head
+  // ---- warps -> one (m, l, o) per head in shared memory -> this split's record
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -405,140 +495,167 @@ __global__ void __launch_bounds__(kWarps * 32) decode_kernel(const DecodeParams 
       }
     }
   __syncthreads();
-  for (int head = 0; head < G; ++head) {
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mg[((size_t)w * 16 + head) * kPartStride]);
-    float Lsum = 0.f, O = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        const float* src = mg + ((size_t)w * 16 + head) * kPartStride;
-        const float sc = exp2f(src[0] - M);
-        Lsum += sc * src[1];
-        O += sc * src[2 + tid];
-      }
-    }
-    float* dst = p.part + (((size_t)b * p.n_q + h * G + head) * p.n_splits + split) * kPartStride;
-    dst[2 + tid] = O;
-    if (tid == 0) {
-      dst[0] = M;
-      dst[1] = Lsum;
-    }
-  }
-}
+  merge_records(mg, kWarps, (size_t)16 * kPartStride, G, my_part);
 
-// Merge split partials and undo the value rotation:
-// o = (1 / (128 l)) s . (H sum_s 2^(m_s - m) o_s).
-// One CTA of 512 threads per (sequence, query head): split weights in shared
-// memory, then 4 groups of 128 threads (one per coordinate) sum interleaved
-// splits with independent loads in flight.
-constexpr int kCombineThreads = 512;
-
-__device__ __forceinline__ float block_reduce(float v, bool is_max, float* red) {
-#pragma unroll
-  for (int m = 16; m; m >>= 1) {
-    const float o = __shfl_xor_sync(0xffffffffu, v, m);
-    v = is_max ? fmaxf(v, o) : v + o;
+  // ---- level 1: the last CTA of this group of splits merges the group
+  const int grp = split / kGroup;
+  const int g_lo = grp * kGroup, g_n = min(kGroup, p.n_splits - g_lo);
+  unsigned int* cnt = p.cnt_end - (bh + 1) * kCntStride;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const unsigned int prev = atomicAdd(&cnt[1 + grp], 1u);
+    sm.is_last = prev == (unsigned int)(g_n - 1);
+    if (sm.is_last) cnt[1 + grp] = 0u;
   }
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  v = red[0];
-  for (int w = 1; w < kCombineThreads / 32; ++w) v = is_max ? fmaxf(v, red[w]) : v + red[w];
-  return v;
-}
+  if (!sm.is_last) return;
+  __threadfence();
+  float* my_gpart = p.gpart + (bh * p.n_groups + grp) * G * kPartStride;
+  merge_records(p.part + (bh * p.n_splits + g_lo) * G * kPartStride, g_n,
+                (size_t)G * kPartStride, G, my_gpart);
 
-__global__ void __launch_bounds__(kCombineThreads) combine_kernel(
-    const float* __restrict__ part, int n_splits, int n_q, int G, const Plan* const* plans,
-    float* out) {
-  const int bh = blockIdx.x, b = bh / n_q, head = bh % n_q;
-  const int tid = threadIdx.x;
-  const float* pp = part + (size_t)bh * n_splits * kPartStride;
-  __shared__ float s_w[1024];
-  __shared__ float s_red[kCombineThreads / 32];
-  __shared__ float s_o[4][kHeadDim];
-  float m = -INFINITY;
-  for (int s = tid; s < n_splits; s += kCombineThreads) m = fmaxf(m, pp[(size_t)s * kPartStride]);
-  const float M = block_reduce(m, true, s_red);
-  float lsum = 0.f;
-  for (int s = tid; s < n_splits; s += kCombineThreads) {
-    const float w = M == -INFINITY ? 0.f : exp2f(pp[(size_t)s * kPartStride] - M);
-    s_w[s] = w;
-    lsum += w * pp[(size_t)s * kPartStride + 1];
+  // ---- level 2: the last group merges the groups and writes o / l
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const unsigned int prev = atomicAdd(&cnt[0], 1u);
+    sm.is_last = prev == (unsigned int)(p.n_groups - 1);
+    if (sm.is_last) cnt[0] = 0u;
   }
-  const float Lsum = block_reduce(lsum, false, s_red);
   __syncthreads();
-  const int coord = tid & (kHeadDim - 1), grp = tid >> 7;
-  float o = 0.f;
-#pragma unroll 8
-  for (int s = grp; s < n_splits; s += 4) o += s_w[s] * pp[(size_t)s * kPartStride + 2 + coord];
-  s_o[grp][coord] = o;
+  if (!sm.is_last) return;
+  __threadfence();
+  float* fin = reinterpret_cast<float*>(stage_base);  // [16][130]
+  merge_records(p.gpart + bh * p.n_groups * G * kPartStride, p.n_groups, (size_t)G * kPartStride,
+                G, fin);
   __syncthreads();
-  if (tid < 32) {
-    float y[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int i = tid + 32 * q;
-      y[q] = (s_o[0][i] + s_o[1][i]) + (s_o[2][i] + s_o[3][i]);
-    }
-#pragma unroll
-    for (int hh = 1; hh < 32; hh <<= 1) {
-      const bool upper = (tid & hh) != 0;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float x = __shfl_xor_sync(0xffffffffu, y[q], hh);
-        y[q] = upper ? x - y[q] : y[q] + x;
-      }
-    }
-    const float a0 = y[0] + y[1], a1 = y[0] - y[1], a2 = y[2] + y[3], a3 = y[2] - y[3];
-    y[0] = a0 + a2;
-    y[2] = a0 - a2;
-    y[1] = a1 + a3;
-    y[3] = a1 - a3;
-    const Plan* pl = plans[b] + head / G;
-    const float inv = Lsum > 0.f ? 1.f / (128.f * Lsum) : 0.f;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int i = tid + 32 * q;
-      const float sgn = ((pl->v_sign[i >> 5] >> (i & 31)) & 1u) ? -1.f : 1.f;
-      out[(size_t)bh * kHeadDim + i] = sgn * y[q] * inv;
-    }
+  for (int head = warp; head < G; head += kWarps) {
+    const float* r = fin + (size_t)head * kPartStride;
+    const float inv = r[1] > 0.f ? 1.f / (128.f * r[1]) : 0.f;
+    warp_unrotate_store(r + 2, sm.plan, inv,
+                        p.out + ((size_t)b * p.n_q + h * G + head) * kHeadDim, lane);
   }
 }
 
 // ------------------------------------------------------------- launchers
-int decode_splits(int64_t max_len) {
-  const int64_t tiles = (max_len + kTile - 1) / kTile;
-  const int64_t target = 6 * kWarps;  // tiles per CTA
-  int64_t s = (tiles + target - 1) / target;
-  return (int)std::max<int64_t>(1, std::min<int64_t>(s, 1024));
-}
-
 size_t decode_smem_bytes(int tile_bytes) {
   const size_t stages = (size_t)kWarps * kStages * tile_bytes;
   const size_t merge = (size_t)kWarps * 16 * kPartStride * sizeof(float);
   return sizeof(Smem) + std::max(stages, merge);
 }
 
-// The dynamic shared-memory cap is raised once per device and instantiation
-// (to the largest tile size), so calls made during stream capture only launch.
+// CTAs per SM of one instantiation for tiles of (bits_k, BV), queried once per
+// device and bits_k. The first query also raises the dynamic shared-memory cap
+// of the instantiation to its largest tile, so later calls (also under stream
+// capture) only launch.
 template <int BV, int NT>
-static cudaError_t launch_decode_t(const DecodeParams& p, int batch, cudaStream_t st) {
-  static std::atomic<unsigned long long> ready{0};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
+static int ctas_per_sm(int dev, int bits_k, cudaError_t* err) {
+  static std::atomic<int> cache[64][9];
+  static std::atomic<unsigned long long> cap_set{0};
+  std::atomic<int>& slot = cache[dev & 63][bits_k & 7 ? bits_k : 8];
+  int v = slot.load();
+  if (v > 0) return v;
+  cudaError_t e = cudaSuccess;
   const unsigned long long bit = 1ull << (dev & 63);
-  if (!(ready.load() & bit)) {
+  if (!(cap_set.load() & bit)) {
     e = cudaFuncSetAttribute(decode_kernel<BV, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)decode_smem_bytes(tile_bytes(8, BV)));
-    if (e != cudaSuccess) return e;
-    ready.fetch_or(bit);
+    if (e == cudaSuccess) cap_set.fetch_or(bit);
   }
+  if (e == cudaSuccess)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+        &v, decode_kernel<BV, NT>, kThreads, decode_smem_bytes(tile_bytes(bits_k, BV)));
+  if (e != cudaSuccess) {
+    *err = e;
+    return 0;
+  }
+  v = std::max(v, 1);
+  slot.store(v);
+  return v;
+}
+
+template <int NT>
+static int ctas_per_sm_bv(int dev, int bits_k, int bv, cudaError_t* err) {
+  switch (bv) {
+    case 1: return ctas_per_sm<1, NT>(dev, bits_k, err);
+    case 2: return ctas_per_sm<2, NT>(dev, bits_k, err);
+    case 3: return ctas_per_sm<3, NT>(dev, bits_k, err);
+    case 4: return ctas_per_sm<4, NT>(dev, bits_k, err);
+    case 5: return ctas_per_sm<5, NT>(dev, bits_k, err);
+    case 6: return ctas_per_sm<6, NT>(dev, bits_k, err);
+    case 7: return ctas_per_sm<7, NT>(dev, bits_k, err);
+    default: return ctas_per_sm<8, NT>(dev, bits_k, err);
+  }
+}
+
+struct SplitPlan {
+  int n_splits, tiles_per_split, n_groups;
+};
+
+// Splits per (sequence, KV head) so that the grid is about one wave of the
+// current device, with at least one tile per warp. Without a device (size
+// queries on a host without GPU) an upper bound of the CTA slots is used.
+static SplitPlan decode_split_plan(int batch, int n_kv, int G, int bits_k, int bits_v,
+                                   int64_t max_len, cudaError_t* err, bool allow_fallback) {
+  SplitPlan sp{1, 1, 1};
+  int64_t slots = kFallbackSlots;
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int per_sm = 0;
+  if (e == cudaSuccess)
+    per_sm = G <= 8 ? ctas_per_sm_bv<1>(dev, bits_k, bits_v, &e)
+                    : ctas_per_sm_bv<2>(dev, bits_k, bits_v, &e);
+  if (e == cudaSuccess) {
+    slots = (int64_t)sms * per_sm;
+  } else if (!allow_fallback) {
+    *err = e;
+    return sp;
+  } else {
+    (void)cudaGetLastError();
+  }
+  *err = cudaSuccess;
+  const int64_t tiles = std::max<int64_t>(1, (max_len + kTile - 1) / kTile);
+  const int64_t pairs = (int64_t)batch * n_kv;
+  int64_t s = std::max<int64_t>(1, slots / pairs);
+  s = std::min<int64_t>(s, std::max<int64_t>(1, (tiles + kWarps - 1) / kWarps));
+  s = std::min<int64_t>(s, kMaxSplits);
+  sp.tiles_per_split = (int)((tiles + s - 1) / s);
+  sp.n_splits = (int)((tiles + sp.tiles_per_split - 1) / sp.tiles_per_split);
+  sp.n_groups = (sp.n_splits + kGroup - 1) / kGroup;
+  return sp;
+}
+
+static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Workspace: split records | group records | ... | counters (at the end, pair
+// k at a fixed distance from the end so that calls of any shape sharing one
+// workspace never overwrite each other's counters).
+static size_t decode_workspace_layout(int batch, int n_kv, int G, const SplitPlan& sp,
+                                      size_t* gpart_off) {
+  const size_t pairs = (size_t)batch * n_kv;
+  const size_t part = align256(pairs * sp.n_splits * G * kPartStride * sizeof(float));
+  const size_t gpart = align256(pairs * sp.n_groups * G * kPartStride * sizeof(float));
+  const size_t counters = align256(pairs * kCntStride * sizeof(unsigned int));
+  if (gpart_off) *gpart_off = part;
+  return part + gpart + counters;
+}
+
+// Workspace bytes of a decode call on the current device (an upper bound if
+// no device answers).
+size_t decode_workspace_bytes_for(int batch, int n_q, int n_kv, int bits_k, int bits_v,
+                                  int64_t max_len) {
+  cudaError_t err = cudaSuccess;
+  const int G = n_q / n_kv;
+  const SplitPlan sp = decode_split_plan(batch, n_kv, G, bits_k, bits_v, max_len, &err, true);
+  return decode_workspace_layout(batch, n_kv, G, sp, nullptr);
+}
+
+template <int BV, int NT>
+static cudaError_t launch_decode_t(const DecodeParams& p, int batch, cudaStream_t st) {
   const size_t smem = decode_smem_bytes(p.tile_bytes);
-  decode_kernel<BV, NT><<<dim3(p.n_splits, p.n_kv, batch), kWarps * 32, smem, st>>>(p);
+  decode_kernel<BV, NT><<<dim3(p.n_splits, p.n_kv, batch), kThreads, smem, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -557,10 +674,19 @@ static cudaError_t launch_decode_nt(const DecodeParams& p, int bits_v, int batch
   return cudaErrorInvalidValue;
 }
 
+// ws: >= decode_workspace_bytes_for(...) bytes, zero-filled before its first
+// use; every completed call leaves its counters (at the end of ws) zero.
 cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches, const int32_t* len,
                           int batch, int64_t max_len, const void* q, int q_dtype, int n_q, int n_kv,
-                          int bits_k, int bits_v, float* out, float* part, uint32_t* status,
-                          cudaStream_t st) {
+                          int bits_k, int bits_v, float* out, void* ws, size_t ws_bytes,
+                          uint32_t* status, cudaStream_t st) {
+  cudaError_t err = cudaSuccess;
+  const int G = n_q / n_kv;
+  const SplitPlan sp = decode_split_plan(batch, n_kv, G, bits_k, bits_v, max_len, &err, false);
+  if (err != cudaSuccess) return err;
+  size_t gpart_off = 0;
+  if (decode_workspace_layout(batch, n_kv, G, sp, &gpart_off) > ws_bytes)
+    return cudaErrorInvalidValue;
   DecodeParams p;
   p.plans = plans;
   p.caches = caches;
@@ -569,19 +695,19 @@ cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches
   p.q_dtype = q_dtype;
   p.n_q = n_q;
   p.n_kv = n_kv;
-  p.G = n_q / n_kv;
+  p.G = G;
   p.max_len = (int)max_len;
-  p.n_splits = decode_splits(max_len);
-  const int tiles = (int)((max_len + kTile - 1) / kTile);
-  p.tiles_per_split = std::max(1, (tiles + p.n_splits - 1) / p.n_splits);
+  p.n_splits = sp.n_splits;
+  p.tiles_per_split = sp.tiles_per_split;
+  p.n_groups = sp.n_groups;
   p.tile_bytes = tile_bytes(bits_k, bits_v);
-  p.part = part;
+  p.part = reinterpret_cast<float*>(ws);
+  p.gpart = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + gpart_off);
+  p.cnt_end = reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(ws) + (ws_bytes & ~size_t(3)));
+  p.out = out;
   p.status = status;
-  cudaError_t e = p.G <= 8 ? launch_decode_nt<1>(p, bits_v, batch, st)
-                           : launch_decode_nt<2>(p, bits_v, batch, st);
-  if (e != cudaSuccess) return e;
-  combine_kernel<<<batch * n_q, kCombineThreads, 0, st>>>(part, p.n_splits, n_q, p.G, plans, out);
-  return cudaGetLastError();
+  return G <= 8 ? launch_decode_nt<1>(p, bits_v, batch, st)
+                : launch_decode_nt<2>(p, bits_v, batch, st);
 }
 
 }  // namespace kvq

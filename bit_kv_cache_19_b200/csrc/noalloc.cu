@@ -20,8 +20,8 @@
 namespace kvq {
 cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches, const int32_t* len,
                           int batch, int64_t max_len, const void* q, int q_dtype, int n_q, int n_kv,
-                          int bits_k, int bits_v, float* out, float* part, uint32_t* status,
-                          cudaStream_t st);
+                          int bits_k, int bits_v, float* out, void* ws, size_t ws_bytes,
+                          uint32_t* status, cudaStream_t st);
 int set_last_error(int code, const char* msg);
 }  // namespace kvq
 
@@ -87,12 +87,14 @@ extern "C" KVQ_API int kvq_decode_attn_noalloc(const kvq_cfg* cfg, const void* c
   cudaError_t e = scratch_address(&scratch);
   if (e != cudaSuccess)
     return kvq::set_last_error(KVQ_ERR_CUDA, cudaGetErrorString(e));
-  // Every split partial the combine reads is written by the decode kernel of
-  // the same call, so nothing in the scratch needs clearing first.
+  // The split records are written before they are read within each call. The
+  // arrival counters at the end of the scratch must be zero when a call
+  // starts: the array is zero when the library is loaded and every completed
+  // call resets the counters it used.
   e = kvq::launch_decode(reinterpret_cast<const kvq::Plan* const*>(plans_dev),
                          reinterpret_cast<const uint8_t* const*>(cache_dev), len_dev, batch,
                          max_len, q_dev, q_dtype, n_q_heads, cfg->n_kv_heads, cfg->bits_k,
-                         cfg->bits_v, out_dev, reinterpret_cast<float*>(scratch), status_dev,
+                         cfg->bits_v, out_dev, scratch, kScratchBytes, status_dev,
                          reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return kvq::set_last_error(KVQ_ERR_CUDA, cudaGetErrorString(e));
   return KVQ_OK;

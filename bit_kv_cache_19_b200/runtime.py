@@ -61,8 +61,9 @@ class PackedLayer:
         return out
 
     def workspace(self, n_q: int, max_len: int):
+        """Decode workspace, zero-filled (its arrival counters must start at 0)."""
         n = kvq.decode_workspace_bytes(self.cfg, self.batch, n_q, max_len)
-        return torch.empty(n, dtype=torch.uint8, device=self.device)
+        return torch.zeros(n, dtype=torch.uint8, device=self.device)
 
     # ------------------------------------------------------------ inspect
     def head_records(self, seq: int, head: int, n_tiles: int) -> np.ndarray:

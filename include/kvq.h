@@ -154,8 +154,10 @@ KVQ_API size_t kvq_alloc_workspace_bytes(const kvq_cfg* cfg);
 
 /*
  * Workspace bytes kvq_decode_attn needs for `batch` sequences of at most
- * max_len tokens: split-K partials (m, l, o[128]) per (sequence, query head,
- * split). Returns 0 for invalid arguments.
+ * max_len tokens on the current device: split-K records (m, l, o[128]) per
+ * (sequence, query head, split) and per group of 8 splits, and arrival
+ * counters at the end. Without a usable device it returns an upper bound.
+ * Returns 0 for invalid arguments.
  */
 KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cfg* cfg, int batch, int n_q_heads,
                                   int64_t max_len);
@@ -242,14 +244,20 @@ KVQ_API int kvq_quantize_append(const kvq_cfg* cfg, const void* const* plans_dev
  * v_hat = n^V (1/128) s . (H c_{bits_v}[codes])). Split-K over the context:
  * each CTA unpacks its tiles in registers, forms the logits of all G query
  * heads of its KV head, keeps an online softmax and accumulates P V in the
- * rotated value domain; a combine kernel merges the splits and applies the
- * inverse rotation. fp32 accumulation.
+ * rotated value domain; the last CTAs to finish merge the splits (two
+ * levels) and apply the inverse rotation. One kernel launch; fp32
+ * accumulation.
  * plans_dev, cache_dev: as for kvq_quantize_append.
  * len_dev: int32 [batch], each <= max_len (a larger value is clamped to
  *        max_len and flags CAPACITY). A sequence of length 0 gives o = 0.
  * q_dev: [batch][n_q_heads][128] of type q_dtype (post-RoPE queries).
  * out_dev: fp32 [batch][n_q_heads][128].
- * ws_dev: >= kvq_decode_workspace_bytes(cfg, batch, n_q_heads, max_len).
+ * ws_dev: >= kvq_decode_workspace_bytes(cfg, batch, n_q_heads, max_len)
+ *        bytes, zero-filled once before its first use. Every completed call
+ *        leaves the arrival counters it keeps at the end of the workspace at
+ *        zero, so one workspace can serve any sequence of calls (of any
+ *        shape that fits) on one stream; calls that overlap on the GPU must
+ *        use different workspaces.
  * status_dev: required.
  * Returns KVQ_OK or a negative code.
  */
@@ -283,10 +291,12 @@ KVQ_API int kvq_decode_attn(const kvq_cfg* cfg, const void* const* plans_dev,
  * first call before any stream capture on the device.
  *
  * Sharing: every call uses the same array, which keeps the last call's
- * contents (nothing in it needs clearing: each call writes every partial it
- * reads). Calls that overlap on the GPU - on different streams, or from
- * different host threads without ordering - race on the array and may give
- * wrong outputs; order them on one stream.
+ * contents. The split records are always written before they are read; the
+ * arrival counters kept at the end of the array must be zero when a call
+ * starts - the array is zero when the library is loaded, and every completed
+ * call resets the counters it used. Calls that overlap on the GPU - on
+ * different streams, or from different host threads without ordering - race
+ * on the array and may give wrong outputs; order them on one stream.
  */
 KVQ_API int kvq_decode_attn_noalloc(const kvq_cfg* cfg, const void* const* plans_dev,
                                     const void* const* cache_dev, const int32_t* len_dev,

@@ -71,9 +71,9 @@ def test_noalloc_matches_workspace_decode_twice():
 def test_noalloc_rejects_what_does_not_fit():
     cfg = kvq.make_cfg(4, 3, 2)
     limit = kvq.lib().kvq_decode_noalloc_scratch_bytes()
-    assert kvq.decode_workspace_bytes(cfg, 64, 28, 1 << 20) > limit
+    assert kvq.decode_workspace_bytes(cfg, 2048, 28, 1 << 20) > limit
     p = ctypes.c_void_p(256)
-    rc = kvq.lib().kvq_decode_attn_noalloc(ctypes.byref(cfg), p, p, p, 64, 1 << 20, p, kvq.BF16,
-                                           28, p, p, None)
+    rc = kvq.lib().kvq_decode_attn_noalloc(ctypes.byref(cfg), p, p, p, 2048, 1 << 20, p,
+                                           kvq.BF16, 28, p, p, None)
     assert rc == kvq.ERR_WORKSPACE
     assert b"4 MiB" in kvq.lib().kvq_last_error()
