@@ -7,10 +7,10 @@ plans. Synthetic seeded inputs (synth.keys_values_torch); caches are built by
 the library itself (energy + greedy plans + bulk quantize-append) before the
 timed region.
 
-Step = one decode step of the whole stack: per layer, quantize-append the new
-token's key and value (1 token x 2 KV heads) and run packed decode attention
-over the layer's cache (decode + split combine). The step is captured in a
-CUDA graph. ``value`` = packed cache bytes read by decode attention per step
+Step = one decode step of the whole stack: per layer, one kvq_append_decode
+launch quantize-appends the new token's key and value (1 token x 2 KV heads)
+and runs packed decode attention over the layer's cache, the split merge
+included. The step is captured in a CUDA graph. ``value`` = packed cache bytes read by decode attention per step
 / step time (GB/s). The packed caches of the 36 layers (944 MB) exceed L2, and
 each layer's cache is read once per step, so no L2 flush is needed.
 
@@ -259,10 +259,10 @@ def run_kvq(args, wl, rank, world, dist):
     ws = layers[0].workspace(wl.n_q_heads, cap)
 
     def step():
+        # one launch per layer: quantize-append the new token, then decode
         for li, L in enumerate(layers):
-            L.append(knew[li], vnew[li])
-            kvq.decode_attn(cfg, L.plan_ptrs, L.cache_ptrs, L.lens, cap, qs[li], outs[li], ws,
-                            L.status)
+            kvq.append_decode(cfg, L.plan_ptrs, knew[li], vnew[li], L.cache_ptrs, L.lens, cap,
+                              cap, qs[li], outs[li], ws, L.status)
 
     stream = torch.cuda.Stream(device=dev)
     graph = None
@@ -371,7 +371,8 @@ def run_kvq(args, wl, rank, world, dist):
         "config": {"workload": wl.name, "layers": n_layers, "q_heads": wl.n_q_heads,
                    "kv_heads": wl.n_kv_heads, "head_dim": 128, "context": T, "batch": B,
                    "budget": f"K{wl.bits_k}V{wl.bits_v}", "alloc": "Block-GTQ greedy",
-                   "step": "per layer: quantize-append 1 token + packed decode attention",
+                   "step": "per layer, one fused launch: quantize-append 1 token + packed "
+                           "decode attention",
                    "l2": f"inputs larger than L2 ({n_layers}-layer packed cache "
                          f"{n_layers * B * wl.n_kv_heads * bpth * T / 1e6:.0f} MB, each layer "
                          "read once per step)",
@@ -384,12 +385,12 @@ def run_kvq(args, wl, rank, world, dist):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "traffic": profiled_traffic(wl.name),
-                     "kernel": "decode_attn (decode_kernel + combine_kernel)",
+                     "kernel": "decode_kernel (kvq_decode_attn, one launch)",
                      "bytes_per_launch": bytes_launch, "launch_us": launch_ms * 1e3},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": steps * n_layers * 4,
+        "gpu_launches": steps * n_layers,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

@@ -30,10 +30,11 @@ struct QuantParams {
 cudaError_t launch_quantize_append(const QuantParams& p, cudaStream_t st);
 size_t decode_workspace_bytes_for(int batch, int n_q, int n_kv, int bits_k, int bits_v,
                                   int64_t max_len);
-cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches, const int32_t* len,
+cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches, int32_t* len,
                           int batch, int64_t max_len, const void* q, int q_dtype, int n_q, int n_kv,
                           int bits_k, int bits_v, float* out, void* ws, size_t ws_bytes,
-                          uint32_t* status, cudaStream_t st);
+                          uint32_t* status, cudaStream_t st, const void* k_new, const void* v_new,
+                          int kv_dtype, int n_new, int64_t cap);
 
 namespace {
 
@@ -146,6 +147,20 @@ void build_plan(const kvq_cfg* cfg, int layer, int kv_head, const double* E, Pla
     r += n;
   }
   pl->n_half = (uint8_t)nh;
+  // classes: maximal runs of half steps with one width
+  int nc = 0;
+  for (int hs = 0; hs < nh;) {
+    int e = hs;
+    while (e < nh && pl->hs_width[e] == pl->hs_width[hs]) ++e;
+    pl->cls_w[nc] = pl->hs_width[hs];
+    pl->cls_hs0[nc] = (uint8_t)hs;
+    pl->cls_nhs[nc] = (uint8_t)(e - hs);
+    pl->cls_last[nc] = pl->hs_count[e - 1];
+    pl->cls_seg0[nc] = pl->seg_off[pl->hs_rank0[hs]];
+    ++nc;
+    hs = e;
+  }
+  pl->n_class = (uint8_t)nc;
   const uint64_t key = splitmix64(cfg->v_seed, ((uint64_t)(uint32_t)layer << 32) + (uint32_t)kv_head);
   for (int i = 0; i < kHeadDim; ++i)
     if (splitmix64(key, (uint64_t)i) >> 63) pl->v_sign[i >> 5] |= 1u << (i & 31);
@@ -311,11 +326,43 @@ int kvq_decode_attn(const kvq_cfg* cfg, const void* const* plans_dev, const void
     return fail(KVQ_ERR_WORKSPACE, "decode workspace %zu < %zu", ws_bytes,
                 kvq_decode_workspace_bytes(cfg, batch, n_q_heads, max_len));
   cudaError_t e = launch_decode(reinterpret_cast<const Plan* const*>(plans_dev),
+                                reinterpret_cast<const uint8_t* const*>(cache_dev),
+                                const_cast<int32_t*>(len_dev), batch, max_len, q_dev, q_dtype,
+                                n_q_heads, cfg->n_kv_heads, cfg->bits_k, cfg->bits_v, out_dev,
+                                ws_dev, ws_bytes, status_dev, reinterpret_cast<cudaStream_t>(stream),
+                                nullptr, nullptr, 0, 0, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "decode_attn");
+  return KVQ_OK;
+}
+
+int kvq_append_decode(const kvq_cfg* cfg, const void* const* plans_dev, const void* k_dev,
+                      const void* v_dev, int kv_dtype, int n_new, void* const* cache_dev,
+                      int32_t* len_dev, int64_t cap_tokens, int batch, int64_t max_len,
+                      const void* q_dev, int q_dtype, int n_q_heads, float* out_dev, void* ws_dev,
+                      size_t ws_bytes, uint32_t* status_dev, kvq_stream_t stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (!plans_dev || !cache_dev || !len_dev || !q_dev || !out_dev || !ws_dev || !status_dev)
+    return fail(KVQ_ERR_ARG, "null device pointer");
+  if (n_new < 0 || n_new > 64) return fail(KVQ_ERR_ARG, "n_new %d not in 0..64", n_new);
+  if (n_new > 0 && (!k_dev || !v_dev)) return fail(KVQ_ERR_ARG, "null k/v pointer");
+  if (!dtype_ok(kv_dtype) || !dtype_ok(q_dtype)) return fail(KVQ_ERR_ARG, "bad dtype");
+  if (batch < 1 || batch > 65535) return fail(KVQ_ERR_ARG, "batch %d", batch);
+  if (max_len < 1 || max_len > 0x7FFFFFFF || cap_tokens < 0 || cap_tokens > 0x7FFFFFFF)
+    return fail(KVQ_ERR_ARG, "max_len %lld / cap_tokens %lld", (long long)max_len,
+                (long long)cap_tokens);
+  if (n_q_heads < 1 || n_q_heads % cfg->n_kv_heads != 0 || n_q_heads / cfg->n_kv_heads > 16)
+    return fail(KVQ_ERR_ARG, "n_q_heads %d vs n_kv_heads %d", n_q_heads, cfg->n_kv_heads);
+  if (ws_bytes < kvq_decode_workspace_bytes(cfg, batch, n_q_heads, max_len))
+    return fail(KVQ_ERR_WORKSPACE, "decode workspace %zu < %zu", ws_bytes,
+                kvq_decode_workspace_bytes(cfg, batch, n_q_heads, max_len));
+  cudaError_t e = launch_decode(reinterpret_cast<const Plan* const*>(plans_dev),
                                 reinterpret_cast<const uint8_t* const*>(cache_dev), len_dev, batch,
                                 max_len, q_dev, q_dtype, n_q_heads, cfg->n_kv_heads, cfg->bits_k,
                                 cfg->bits_v, out_dev, ws_dev, ws_bytes, status_dev,
-                                reinterpret_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "decode_attn");
+                                reinterpret_cast<cudaStream_t>(stream), k_dev, v_dev, kv_dtype,
+                                n_new, cap_tokens);
+  if (e != cudaSuccess) return cuda_fail(e, "append_decode");
   return KVQ_OK;
 }
 

@@ -34,7 +34,14 @@ struct Plan {
   uint32_t v_sign[4];
   uint32_t pad1;
   double energy_sum;
-  uint8_t tail[KVQ_PLAN_BYTES - 928];
+  uint8_t n_class;         // runs of half steps of one width
+  uint8_t pad2[7];
+  uint8_t cls_w[8];
+  uint8_t cls_hs0[8];
+  uint8_t cls_nhs[8];
+  uint8_t cls_last[8];     // blocks in the class's last half step
+  uint16_t cls_seg0[8];    // first K word of the class in a tile record
+  uint8_t tail[KVQ_PLAN_BYTES - 984];
 };
 static_assert(sizeof(Plan) == KVQ_PLAN_BYTES, "plan size");
 static_assert(offsetof(Plan, g) == 32 && offsetof(Plan, a_hat) == 288, "plan layout");
@@ -42,6 +49,8 @@ static_assert(offsetof(Plan, width) == 544 && offsetof(Plan, order) == 608, "pla
 static_assert(offsetof(Plan, seg_off) == 672 && offsetof(Plan, n_half) == 802, "plan layout");
 static_assert(offsetof(Plan, hs_width) == 804 && offsetof(Plan, v_sign) == 900, "plan layout");
 static_assert(offsetof(Plan, energy_sum) == 920, "plan layout");
+static_assert(offsetof(Plan, n_class) == 928 && offsetof(Plan, cls_w) == 936, "plan layout");
+static_assert(offsetof(Plan, cls_last) == 960 && offsetof(Plan, cls_seg0) == 968, "plan layout");
 
 // Codebook offsets: width w centroids at 2^w - 2, thresholds at 2^w - w - 1.
 __host__ __device__ constexpr int cb_c_off(int w) { return (1 << w) - 2; }

@@ -1,114 +1,164 @@
-// Packed-cache decode attention: split-K over the context with an in-kernel
-// two-level merge of the splits.
+// Packed-cache decode attention (optionally fused with the append of the
+// step's new tokens): split-K over the context with an in-kernel two-level
+// merge of the splits.
 //
 // "RoPE-Aware Bit Allocation for KV-Cache Quantization", abstract: the
 // packed-cache serving path runs decode attention directly on the packed
 // K/V cache (the pages report it faster than fp16 FlashAttention2 at 128K on
 // H800). This is an sm_100a design of its own:
 //
-// * Work: CTA = (split, KV head, sequence), 8 warps, sized so the grid is one
-//   wave. Each warp owns every 8th 32-token tile of the CTA's range and
-//   streams its tiles into a private 3-stage shared-memory ring with 1-D bulk
-//   copies (cp.async.bulk + mbarrier, no multicast).
-// * Keys: the logits S[32 tokens x 8 heads] are mma.sync m16n8k8 products.
-//   One MMA covers one "half step" of the plan: <= 4 RoPE blocks of one width
-//   W. Each 32-bit A register is one block (codes of coordinates j and
-//   j + 64) of one token, looked up as an fp16 pair; the packed layout puts
-//   the 4 tokens a lane needs (g, g + 8, g + 16, g + 24) in 8W contiguous
-//   bits. Half steps of one width form a class, so the unpack of a class is
-//   compiled for its W and each lane's addresses are plain arithmetic. The B
-//   operand is the query group pre-multiplied by a_hat_j, log2(e) and
-//   1/sqrt(128), scaled by 2^sigma per head and split into hi + lo fp16, so
-//   the logits keep ~fp32 accuracy.
+// * Work: CTA = (split, KV head, sequence), 8 warps, grid sized to one wave.
+//   Each warp owns every 8th 32-token tile of the CTA's range and streams its
+//   tiles into a private 2-stage shared-memory ring with 1-D bulk copies
+//   (cp.async.bulk + mbarrier, no multicast). The codebook lookup image
+//   (pair tables, replicated per lane for widths <= 3 so lookups are free of
+//   bank conflicts) and the plan also arrive by bulk copy. Launched with
+//   programmatic dependent launch: everything up to griddepcontrol.wait does
+//   not depend on the previous kernel.
+// * Append (fused calls): the CTA that owns the tile of a new token
+//   quantizes and packs it before streaming; the last CTA of the sequence to
+//   read its length writes the new length.
+// * Keys: logits S[32 tokens x 8 heads] by mma.sync m16n8k8, one MMA per
+//   "half step" of the plan (<= 4 RoPE blocks of one width W). Each 32-bit A
+//   register is one block (codes of coordinates j and j + 64) of one token,
+//   looked up as an fp16 pair; the packed layout puts the 4 tokens a lane
+//   needs (g, g + 8, g + 16, g + 24) in 8W contiguous bits. Half steps of one
+//   width form a class compiled for its W. B = the query group times a_hat_j,
+//   log2(e), 1/sqrt(128), scaled by 2^sigma per head and split hi + lo fp16.
 // * Softmax: base-2 online softmax per head on the fp32 accumulators, scaled
-//   by the fp16 key norms; positions past the sequence length are masked.
-// * Values: P' = p * n^V (fp16) goes from the accumulator layout to the B
-//   operand with movmatrix (register transpose); O^T(128 x G) += Vhat^T(128 x
-//   16 tokens) P'^T with A registers holding one rotated coordinate of two
-//   tokens (pair codes of adjacent value slots).
-// * Merge: the 8 warps merge in shared memory into one (m, l, o[128]) per
-//   head; the last CTA to finish in each group of 8 splits merges the group,
-//   and the last group merges the groups, undoes the value rotation
-//   (inverse Walsh-Hadamard, signs) and writes o / l. Arrivals are counted
-//   with atomics on counters that the last arriver resets, so a completed
-//   call leaves them at zero.
+//   by the fp16 key norms; positions past the sequence length masked.
+// * Values: P' = p * n^V (fp16) moves from the accumulator layout to the B
+//   operand with movmatrix; O^T(128 x G) += Vhat^T(128 x 16 tokens) P'^T with
+//   A registers holding one rotated coordinate of two tokens.
+// * Merge: the 8 warps merge in shared memory; the last CTA of each group of
+//   8 splits merges the group; the last group merges the groups, undoes the
+//   value rotation (inverse Walsh-Hadamard, signs) and writes o / l.
+//   Arrivals are counted on workspace counters that the last arriver resets.
 #include <algorithm>
 #include <atomic>
 
-#include "common.cuh"
+#include "quant_dev.cuh"
 
 namespace kvq {
 
-__constant__ uint16_t c_c16[KVQ_CB_N_C16] = KVQ_CB_C16;
+// Lookup image (generated with the codebooks): byte offsets of its tables.
+__device__ __align__(16) const uint32_t g_lut_image[KVQ_LUT_BYTES / 4] = KVQ_LUT_IMAGE;
+__device__ const float g_thr[KVQ_CB_N_THR] = KVQ_CB_THR;
+constexpr uint32_t kLutRep[4] = {0u, 0u, 512u, 2560u};  // widths 1..3, lane-replicated
+constexpr uint32_t kLutPair4 = 10752u, kLutPair5 = 11776u, kLutSingle = 15872u;
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kStages = 3;
-constexpr int kMaxHalf = 24;    // half steps of <= 4 blocks (<= 64/4 + 8)
-constexpr int kMaxClass = 8;    // widths 1..8
-constexpr int kPairLut = 340;   // pair tables of widths 1..4: 4 + 16 + 64 + 256
+constexpr int kStages = 2;
+constexpr int kMaxHalf = 24;  // half steps of <= 4 blocks (<= 64/4 + 8)
 constexpr int kPartStride = 130;
-constexpr int kGroup = 8;       // splits merged per first-level group
+constexpr int kGroup = 8;     // splits merged per first-level group
 constexpr int kMaxSplits = 1024;
-constexpr int kCntStride = 1 + kMaxSplits / kGroup;  // counters per (sequence, KV head)
+constexpr int kCntStride = 2 + kMaxSplits / kGroup;  // per (sequence, KV head); last = sequence
 constexpr int kFallbackSlots = 1024;                  // CTA slots when no device answers
-
-__host__ __device__ constexpr int pair_off(int w) { return ((1 << (2 * w)) - 4) / 3; }
+constexpr int kMaxNew = 64;                           // tokens appended by a fused call
 
 struct DecodeParams {
   const Plan* const* plans;
   const uint8_t* const* caches;
-  const int32_t* len;
+  int32_t* len;
   const void* q;
   int q_dtype;
   int n_q, n_kv, G;
   int max_len;
   int n_splits, tiles_per_split, n_groups;
   int tile_bytes;
-  unsigned int* cnt_end;   // counters of pair k at cnt_end - (k + 1) * kCntStride
-  float* part;             // [batch][n_kv][n_splits][G][130] = m, l, o[128]
-  float* gpart;            // [batch][n_kv][n_groups][G][130]
-  float* out;              // [batch][n_q][128]
+  // fused append (n_new > 0)
+  const void* k_new;
+  const void* v_new;
+  int kv_dtype, n_new;
+  int64_t cap;
+  unsigned int* cnt_end;  // counters of pair k at cnt_end - (k + 1) * kCntStride
+  float* part;            // [batch][n_kv][n_splits][G][130] = m, l, o[128]
+  float* gpart;           // [batch][n_kv][n_groups][G][130]
+  float* out;             // [batch][n_q][128]
   uint32_t* status;
 };
 
 struct alignas(128) Smem {
   Plan plan;
-  uint32_t lut_pair[kPairLut];      // fp16 pairs (c[lo], c[hi]) for widths 1..4
-  uint16_t lut1[KVQ_CB_N_C16];      // fp16 centroids, width w at 2^w - 2
-  float inv_scale[16];              // 2^-sigma of each head's q' scaling
-  uint2 qfrag[2][kMaxHalf][32];     // per (n-tile, half step, lane): hi, lo
+  uint8_t lut[KVQ_LUT_BYTES];
+  uint2 qfrag[2][kMaxHalf][32];  // per (n-tile, half step, lane): hi, lo
+  float inv_scale[16];           // 2^-sigma of each head's q' scaling
   unsigned long long bar[kWarps][kStages];
-  int n_class;
-  int cls_w[kMaxClass], cls_hs0[kMaxClass], cls_nhs[kMaxClass], cls_seg0[kMaxClass],
-      cls_last[kMaxClass];
-  int is_last;
+  unsigned long long setup_bar;
+  int len0, is_last;
+  uint32_t flags;
 };
 
-template <int W>
-__device__ __forceinline__ uint32_t pair_lookup(const Smem& sm, uint32_t f) {
-  if constexpr (W <= 4) {
-    return sm.lut_pair[pair_off(W) + f];
-  } else {
-    const uint16_t* t = sm.lut1 + cb_c_off(W);
-    return (uint32_t)t[f & ((1u << W) - 1u)] | ((uint32_t)t[f >> W] << 16);
-  }
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds16(uint32_t a) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// Four 2W-bit pair fields starting at bit `sh` of wp[0] (8W bits), as fp16 pairs.
+// Four fp16 pairs from the 4 pair fields (2W bits each) that start at bit
+// `sh` of the word at shared address `wa`. lut: shared address of the lookup
+// image; lane4 = 4 * lane.
 template <int W>
-__device__ __forceinline__ void fields4(const Smem& sm, const uint32_t* wp, uint32_t sh,
+__device__ __forceinline__ void fields4(uint32_t lut, uint32_t wa, uint32_t sh, uint32_t lane4,
                                         uint32_t (&out)[4]) {
-  constexpr uint32_t mask = (1u << (2 * W)) - 1u;
-  if constexpr (W <= 4) {
-    const uint32_t v = funnel_r(wp[0], wp[1], sh);
+  if constexpr (W <= 3) {
+    // replicated pair table: entry e of lane l at byte (e * 32 + l) * 4
+    constexpr uint32_t m7 = ((1u << (2 * W)) - 1u) << 7;
+    const uint32_t v7 = funnel_r(lds32(wa), lds32(wa + 4), sh) << 7;
+    const uint32_t base = lut + kLutRep[W];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) out[i] = pair_lookup<W>(sm, (v >> (2 * W * i)) & mask);
+    for (int i = 0; i < 4; ++i) out[i] = lds32(base + (((v7 >> (2 * W * i)) & m7) | lane4));
+  } else if constexpr (W == 4) {
+    const uint32_t v = funnel_r(lds32(wa), lds32(wa + 4), sh);
+    const uint32_t base = lut + kLutPair4;
+    out[0] = lds32(base + ((v << 2) & 0x3FCu));
+#pragma unroll
+    for (int i = 1; i < 4; ++i) out[i] = lds32(base + ((v >> (8 * i - 2)) & 0x3FCu));
+  } else if constexpr (W == 5) {
+    const uint32_t w0 = lds32(wa), w1 = lds32(wa + 4), w2 = lds32(wa + 8);
+    const uint32_t lo = funnel_r(w0, w1, sh), hi = funnel_r(w1, w2, sh);
+    const uint32_t base = lut + kLutPair5;
+    out[0] = lds32(base + ((lo << 2) & 0xFFCu));
+    out[1] = lds32(base + ((lo >> 8) & 0xFFCu));
+    out[2] = lds32(base + ((lo >> 18) & 0xFFCu));
+    out[3] = lds32(base + (funnel_r(lo, hi, 28) & 0xFFCu));
   } else {
-    const uint32_t lo = funnel_r(wp[0], wp[1], sh), hi = funnel_r(wp[1], wp[2], sh);
+    // widths 6..8: two single-code lookups per pair (fp16 table, 2 bytes each)
+    const uint32_t w0 = lds32(wa), w1 = lds32(wa + 4), w2 = lds32(wa + 8);
+    const uint32_t lo = funnel_r(w0, w1, sh), hi = funnel_r(w1, w2, sh);
     const unsigned long long v = ((unsigned long long)hi << 32) | lo;
+    constexpr uint32_t mw = ((1u << W) - 1u) << 1;
+    const uint32_t base = lut + kLutSingle + 2u * (uint32_t)cb_c_off(W);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) out[i] = pair_lookup<W>(sm, (uint32_t)(v >> (2 * W * i)) & mask);
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t a = (uint32_t)(v >> (2 * W * i)) << 1;
+      const uint32_t c0 = lds16(base + (a & mw));
+      const uint32_t c1 = lds16(base + ((a >> W) & mw));
+      out[i] = c0 | (c1 << 16);
+    }
   }
 }
 
@@ -121,27 +171,32 @@ __device__ __forceinline__ void mma_1688(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(b0));
 }
 
-// Logits of one width class: half steps hs0 .. hs0 + nhs - 1, each <= 4
-// blocks of width W (the last one has `last` blocks). Lane (g, c) takes block
-// c of every half step, tokens g, g + 8 (m-tile 0) and g + 16, g + 24 (m-tile 1).
+// Logits of one width class: half steps hs0 .. hs0 + nhs - 1, each 4 blocks
+// of width W (the last one `last` blocks). Lane (g, c) takes block c of every
+// half step, tokens g, g + 8 (m-tile 0) and g + 16, g + 24 (m-tile 1).
 template <int W, int NT>
-__device__ __forceinline__ void key_class(const Smem& sm, const uint32_t* kw, int hs0, int nhs,
-                                          int seg0, int last, int g, int c, int lane,
+__device__ __forceinline__ void key_class(uint32_t lut, uint32_t kw, uint32_t qf, int hs0, int nhs,
+                                          int seg0, int last, int g, int c, uint32_t lane4,
                                           float (&s)[2][NT][4]) {
-  const uint32_t* base = kw + seg0 + 2 * W * c + ((W * g) >> 2);
+  const uint32_t base = kw + 4u * (uint32_t)(seg0 + 2 * W * c + ((W * g) >> 2));
   const uint32_t sh = (uint32_t)(8 * W * g) & 31u;
-  for (int i = 0; i < nhs; ++i) {
+  const uint32_t qbase = qf + (uint32_t)hs0 * 256u + lane4 * 2u;
+  auto step = [&](int i, bool valid) {
     uint32_t A[4] = {0u, 0u, 0u, 0u};
-    if (i + 1 < nhs || c < last) fields4<W>(sm, base + 8 * W * i, sh, A);
+    if (valid) fields4<W>(lut, base + 32u * W * (uint32_t)i, sh, lane4, A);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      const uint2 qf = sm.qfrag[nt][hs0 + i][lane];
-      mma_1688(s[0][nt], A[0], A[1], qf.x);
-      mma_1688(s[0][nt], A[0], A[1], qf.y);
-      mma_1688(s[1][nt], A[2], A[3], qf.x);
-      mma_1688(s[1][nt], A[2], A[3], qf.y);
+      const uint2 b = lds64(qbase + (uint32_t)(nt * kMaxHalf + i) * 256u);
+      mma_1688(s[0][nt], A[0], A[1], b.x);
+      mma_1688(s[0][nt], A[0], A[1], b.y);
+      mma_1688(s[1][nt], A[2], A[3], b.x);
+      mma_1688(s[1][nt], A[2], A[3], b.y);
     }
-  }
+  };
+  for (int i = 0; i < nhs - 1; ++i) step(i, true);
+  // last half step: lanes past its last block feed zeros (their q' is 0);
+  // every lane still takes part in the warp-wide MMAs
+  step(nhs - 1, c < last);
 }
 
 // Inverse value rotation of one head held by a warp (o[128] in `src`),
@@ -188,7 +243,7 @@ __device__ __forceinline__ void merge_records(const float* src, int n, size_t re
 #pragma unroll 4
       for (int s = 0; s < n; ++s) {
         const float* q = r + s * rec_stride;
-        const float w = exp2f(q[0] - M);
+        const float w = ex2(q[0] - M);
         L += w * q[1];
         O += w * q[2 + x];
       }
@@ -212,31 +267,57 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
   const int G = p.G;
   const size_t bh = (size_t)b * p.n_kv + h;
-  float* const my_part = p.part + (bh * p.n_splits + split) * G * kPartStride;
+  unsigned int* const cnt = p.cnt_end - (bh + 1) * kCntStride;
+  unsigned int* const seq_cnt = p.cnt_end - ((size_t)b * p.n_kv + 1) * kCntStride + (kCntStride - 1);
 
-  // ---- plan, lookup tables
-  {
-    const uint4* src = reinterpret_cast<const uint4*>(p.plans[b] + h);
-    uint4* dst = reinterpret_cast<uint4*>(&sm.plan);
-    for (int i = tid; i < KVQ_PLAN_BYTES / 16; i += kThreads) dst[i] = src[i];
-    for (int i = tid; i < KVQ_CB_N_C16; i += kThreads) sm.lut1[i] = c_c16[i];
-    for (int i = tid; i < kPairLut; i += kThreads) {
-      const int w = i < 4 ? 1 : i < 20 ? 2 : i < 84 ? 3 : 4;
-      const int f = i - pair_off(w);
-      const uint32_t lo = c_c16[cb_c_off(w) + (f & ((1 << w) - 1))];
-      const uint32_t hi = c_c16[cb_c_off(w) + (f >> w)];
-      sm.lut_pair[i] = lo | (hi << 16);
+  // ---- independent of earlier kernels: barriers, plan and lookup image
+  if (tid == 0) {
+    mbar_init(&sm.setup_bar, 1);
+    for (int i = 0; i < kWarps * kStages; ++i) mbar_init(&sm.bar[i / kStages][i % kStages], 1);
+    fence_proxy_async();
+    mbar_expect_tx(&sm.setup_bar, KVQ_PLAN_BYTES + KVQ_LUT_BYTES);
+    bulk_g2s(&sm.plan, p.plans[b] + h, KVQ_PLAN_BYTES, &sm.setup_bar);
+    bulk_g2s(sm.lut, g_lut_image, KVQ_LUT_BYTES, &sm.setup_bar);
+    sm.flags = 0u;
+  }
+  // ---- everything below may read what the previous kernel wrote
+  grid_dep_wait();
+  if (tid == 0) {
+    const int l0 = p.len[b];
+    sm.len0 = l0;
+    if (p.n_new > 0) {
+      // the last CTA of the sequence to read its length writes the new one
+      __threadfence();
+      const unsigned int total = (unsigned int)(p.n_kv * p.n_splits);
+      if (atomicAdd(seq_cnt, 1u) == total - 1u) {
+        *seq_cnt = 0u;
+        const int64_t lim = min((int64_t)p.max_len, p.cap);
+        if (l0 >= 0 && (int64_t)l0 + p.n_new <= lim) p.len[b] = l0 + p.n_new;
+      }
     }
   }
   __syncthreads();
+  const bool ok_setup = mbar_wait_bounded(&sm.setup_bar, 0u);
+  grid_dep_launch();
   const uint8_t* cache = p.caches[b];
   const int bk = sm.plan.bits_k;
   const int n_half = sm.plan.n_half;
-  const bool bad = sm.plan.magic != KVQ_PLAN_MAGIC || sm.plan.bits_v != BV || bk < 1 || bk > 8 ||
-                   p.tile_bytes != tile_bytes(bk, BV) || n_half < 1 || n_half > kMaxHalf ||
+  const bool bad = !ok_setup || sm.plan.magic != KVQ_PLAN_MAGIC || sm.plan.bits_v != BV ||
+                   bk < 1 || bk > 8 || p.tile_bytes != tile_bytes(bk, BV) || n_half < 1 ||
+                   n_half > kMaxHalf || sm.plan.n_class < 1 || sm.plan.n_class > 8 ||
                    (reinterpret_cast<uintptr_t>(cache) & 15) != 0;
-  if (bad && tid == 0) atomicOr(p.status, KVQ_FLAG_BAD_PLAN);
-  int L = bad ? 0 : p.len[b];
+  if (bad && tid == 0) atomicOr(p.status, ok_setup ? KVQ_FLAG_BAD_PLAN : KVQ_FLAG_TIMEOUT);
+  const int len0 = sm.len0;
+  int n_add = 0;
+  if (p.n_new > 0) {
+    const int64_t lim = min((int64_t)p.max_len, p.cap);
+    if (len0 >= 0 && (int64_t)len0 + p.n_new <= lim) {
+      n_add = p.n_new;
+    } else if (tid == 0 && split == 0 && h == 0) {
+      atomicOr(p.status, KVQ_FLAG_CAPACITY);
+    }
+  }
+  int L = bad ? 0 : len0 + n_add;
   if (L > p.max_len) {
     if (tid == 0 && split == 0 && h == 0) atomicOr(p.status, KVQ_FLAG_CAPACITY);
     L = p.max_len;
@@ -246,6 +327,41 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
   const int tb = split * p.tiles_per_split;
   const int te = min(n_tiles, tb + p.tiles_per_split);
   const bool has_work = tb < te;
+
+  // ---- fused append: quantize and pack the new tokens whose tiles are ours
+  if (has_work && n_add > 0) {
+    const int t_first = len0 / kTile, t_last = (len0 + n_add - 1) / kTile;
+    uint8_t (*kc)[kHeadDim] = reinterpret_cast<uint8_t (*)[kHeadDim]>(stage_base);
+    uint8_t (*vc)[kHeadDim] = reinterpret_cast<uint8_t (*)[kHeadDim]>(stage_base + 32 * kHeadDim);
+    uint32_t flags = 0;
+    for (int tile = max(t_first, tb); tile <= min(t_last, te - 1); ++tile) {
+      const int t_lo = max(len0, tile * kTile), t_hi = min(len0 + n_add, tile * kTile + kTile);
+      uint8_t* rec = const_cast<uint8_t*>(cache) + ((size_t)tile * p.n_kv + h) * p.tile_bytes;
+      for (int t = t_lo + warp; t < t_hi; t += kWarps) {
+        const int tt = t - tile * kTile;
+        const size_t row = (((size_t)b * p.n_new + (t - len0)) * p.n_kv + h) * kHeadDim;
+        __half kn, vn;
+        warp_token_codes(sm.plan, g_thr, p.k_new, p.v_new, p.kv_dtype, row, lane, kc[tt], vc[tt],
+                         kn, vn, flags);
+        if (lane == 0) {
+          __half* norms = reinterpret_cast<__half*>(rec + 512 * (bk + BV));
+          norms[tt] = kn;
+          norms[kTile + tt] = vn;
+        }
+      }
+      __syncthreads();
+      assemble_tile_words(reinterpret_cast<uint32_t*>(rec), sm.plan, kc, vc,
+                          max(0, len0 - tile * kTile), t_lo - tile * kTile, t_hi - tile * kTile,
+                          tid, kThreads);
+      __syncthreads();
+    }
+    if (flags) atomicOr(&sm.flags, flags);
+    // the bulk copies below must see these writes
+    __threadfence();
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    __syncthreads();
+    if (tid == 0 && sm.flags) atomicOr(p.status, sm.flags);
+  }
 
   float o[8][NT][4];
   float m_run[NT][2], l_run[NT][2];
@@ -264,24 +380,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     }
 
   if (has_work) {
-    // ---- classes of equal width over the half steps
-    if (tid == 0) {
-      int nc = 0;
-      for (int hs = 0; hs < n_half;) {
-        const int w = sm.plan.hs_width[hs];
-        int e = hs;
-        while (e < n_half && sm.plan.hs_width[e] == w) ++e;
-        sm.cls_w[nc] = w;
-        sm.cls_hs0[nc] = hs;
-        sm.cls_nhs[nc] = e - hs;
-        sm.cls_seg0[nc] = sm.plan.seg_off[sm.plan.hs_rank0[hs]];
-        sm.cls_last[nc] = sm.plan.hs_count[e - 1];
-        ++nc;
-        hs = e;
-      }
-      sm.n_class = nc;
-    }
-    // ---- query prologue (q' staged in the tile ring, not in use yet):
+    // ---- query prologue (q' staged in the tile ring before it is used):
     //      q' = q a_hat_j log2(e) / sqrt(128); per-head 2^sigma scaling into
     //      the fp16 range; hi/lo split into the B fragments of each half step
     float* qp = reinterpret_cast<float*>(stage_base);  // [16][128]
@@ -320,8 +419,6 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
       const uint32_t lo = pack_half2(x0 - __low2float(hh), x1 - __high2float(hh));
       sm.qfrag[nt][hs][ln] = make_uint2(hi, lo);
     }
-    if (tid < kWarps * kStages) mbar_init(&sm.bar[tid / kStages][tid % kStages], 1);
-    fence_proxy_async();
     __syncthreads();
 
     // ---- per-warp pipeline over the warp's tiles
@@ -340,9 +437,12 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
       for (int i = 0; i < min(kStages, n_mine); ++i) issue(i);
     __syncwarp();
 
-    const int n_class = sm.n_class;
+    const uint32_t lut = smem_addr(sm.lut);
+    const uint32_t qf = smem_addr(&sm.qfrag[0][0][0]);
+    const uint32_t lane4 = (uint32_t)lane * 4u;
+    const int n_class = sm.plan.n_class;
     const uint32_t v_sh = (uint32_t)(8 * BV * c) & 31u;
-    const int v_off = (BV * c) >> 2;
+    const uint32_t v_off = 4u * (uint32_t)((BV * c) >> 2);
     int consumed = 0;
     bool timed_out = false;
     for (int i = 0; i < n_mine; ++i) {
@@ -355,9 +455,9 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
       consumed = i + 1;
       const int tile = tile_of(i);
       const int nvalid = min(kTile, L - tile * kTile);
-      const uint32_t* kw = reinterpret_cast<const uint32_t*>(my_stages + s * tbytes);
-      const uint32_t* vw = kw + 128 * bk;
-      const __half* nrm = reinterpret_cast<const __half*>(vw + 128 * BV);
+      const uint32_t kw = smem_addr(my_stages + s * tbytes);
+      const uint32_t vw = kw + 512u * (uint32_t)bk;
+      const __half* nrm = reinterpret_cast<const __half*>(my_stages + s * tbytes + 512 * (bk + BV));
 
       // keys: S[32 tokens x 8 NT heads] on the tensor cores
       float sacc[2][NT][4];
@@ -368,17 +468,17 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
 #pragma unroll
           for (int r = 0; r < 4; ++r) sacc[mt][nt][r] = 0.f;
       for (int ci = 0; ci < n_class; ++ci) {
-        const int hs0 = sm.cls_hs0[ci], nhs = sm.cls_nhs[ci], seg0 = sm.cls_seg0[ci],
-                  last = sm.cls_last[ci];
-        switch (sm.cls_w[ci]) {
-          case 1: key_class<1, NT>(sm, kw, hs0, nhs, seg0, last, g, c, lane, sacc); break;
-          case 2: key_class<2, NT>(sm, kw, hs0, nhs, seg0, last, g, c, lane, sacc); break;
-          case 3: key_class<3, NT>(sm, kw, hs0, nhs, seg0, last, g, c, lane, sacc); break;
-          case 4: key_class<4, NT>(sm, kw, hs0, nhs, seg0, last, g, c, lane, sacc); break;
-          case 5: key_class<5, NT>(sm, kw, hs0, nhs, seg0, last, g, c, lane, sacc); break;
-          case 6: key_class<6, NT>(sm, kw, hs0, nhs, seg0, last, g, c, lane, sacc); break;
-          case 7: key_class<7, NT>(sm, kw, hs0, nhs, seg0, last, g, c, lane, sacc); break;
-          default: key_class<8, NT>(sm, kw, hs0, nhs, seg0, last, g, c, lane, sacc); break;
+        const int hs0 = sm.plan.cls_hs0[ci], nhs = sm.plan.cls_nhs[ci],
+                  seg0 = sm.plan.cls_seg0[ci], last = sm.plan.cls_last[ci];
+        switch (sm.plan.cls_w[ci]) {
+          case 1: key_class<1, NT>(lut, kw, qf, hs0, nhs, seg0, last, g, c, lane4, sacc); break;
+          case 2: key_class<2, NT>(lut, kw, qf, hs0, nhs, seg0, last, g, c, lane4, sacc); break;
+          case 3: key_class<3, NT>(lut, kw, qf, hs0, nhs, seg0, last, g, c, lane4, sacc); break;
+          case 4: key_class<4, NT>(lut, kw, qf, hs0, nhs, seg0, last, g, c, lane4, sacc); break;
+          case 5: key_class<5, NT>(lut, kw, qf, hs0, nhs, seg0, last, g, c, lane4, sacc); break;
+          case 6: key_class<6, NT>(lut, kw, qf, hs0, nhs, seg0, last, g, c, lane4, sacc); break;
+          case 7: key_class<7, NT>(lut, kw, qf, hs0, nhs, seg0, last, g, c, lane4, sacc); break;
+          default: key_class<8, NT>(lut, kw, qf, hs0, nhs, seg0, last, g, c, lane4, sacc); break;
         }
       }
 
@@ -403,7 +503,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
             const int mt = r >> 1, rr = r & 1;
-            sv[r] = val[r] ? sacc[mt][nt][2 * rr + e] * nk[r] * isc : -INFINITY;
+            sv[r] = val[r] ? sacc[mt][nt][2 * rr + e] * (nk[r] * isc) : -INFINITY;
           }
           float mx = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
@@ -412,12 +512,12 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
           const float m_new = fmaxf(m_run[nt][e], mx);
           float alpha = 1.f, lsum = 0.f;
           if (m_new != -INFINITY) {
-            alpha = exp2f(m_run[nt][e] - m_new);
+            alpha = ex2(m_run[nt][e] - m_new);
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
-              const float pr = exp2f(sv[r] - m_new);
+              const float pr = ex2(sv[r] - m_new);
               lsum += pr;
-              pe[e][r] = val[r] ? pr * nv[r] : 0.f;
+              pe[e][r] = pr * nv[r];
             }
           } else {
 #pragma unroll
@@ -444,8 +544,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
 #pragma unroll
       for (int mu = 0; mu < 8; ++mu) {
         uint32_t F0[4], F1[4];
-        fields4<BV>(sm, vw + (16 * mu + g) * BV + v_off, v_sh, F0);
-        fields4<BV>(sm, vw + (16 * mu + g + 8) * BV + v_off, v_sh, F1);
+        fields4<BV>(lut, vw + 4u * (uint32_t)((16 * mu + g) * BV) + v_off, v_sh, lane4, F0);
+        fields4<BV>(lut, vw + 4u * (uint32_t)((16 * mu + g + 8) * BV) + v_off, v_sh, lane4, F1);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           mma_16816(o[mu][nt], F0[0], F1[0], F0[1], F1[1], pb0[0][nt], pb1[0][nt]);
@@ -495,12 +595,12 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
       }
     }
   __syncthreads();
+  float* const my_part = p.part + (bh * p.n_splits + split) * G * kPartStride;
   merge_records(mg, kWarps, (size_t)16 * kPartStride, G, my_part);
 
   // ---- level 1: the last CTA of this group of splits merges the group
   const int grp = split / kGroup;
   const int g_lo = grp * kGroup, g_n = min(kGroup, p.n_splits - g_lo);
-  unsigned int* cnt = p.cnt_end - (bh + 1) * kCntStride;
   __threadfence();
   __syncthreads();
   if (tid == 0) {
@@ -553,7 +653,7 @@ template <int BV, int NT>
 static int ctas_per_sm(int dev, int bits_k, cudaError_t* err) {
   static std::atomic<int> cache[64][9];
   static std::atomic<unsigned long long> cap_set{0};
-  std::atomic<int>& slot = cache[dev & 63][bits_k & 7 ? bits_k : 8];
+  std::atomic<int>& slot = cache[dev & 63][(bits_k & 7) ? bits_k : 8];
   int v = slot.load();
   if (v > 0) return v;
   cudaError_t e = cudaSuccess;
@@ -629,9 +729,9 @@ static SplitPlan decode_split_plan(int batch, int n_kv, int G, int bits_k, int b
 
 static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-// Workspace: split records | group records | ... | counters (at the end, pair
-// k at a fixed distance from the end so that calls of any shape sharing one
-// workspace never overwrite each other's counters).
+// Workspace: split records | group records | ... | counters (at the end: pair
+// k at a fixed distance from the end, so calls sharing one workspace, for one
+// n_kv_heads, never overwrite each other's counters).
 static size_t decode_workspace_layout(int batch, int n_kv, int G, const SplitPlan& sp,
                                       size_t* gpart_off) {
   const size_t pairs = (size_t)batch * n_kv;
@@ -654,9 +754,17 @@ size_t decode_workspace_bytes_for(int batch, int n_q, int n_kv, int bits_k, int 
 
 template <int BV, int NT>
 static cudaError_t launch_decode_t(const DecodeParams& p, int batch, cudaStream_t st) {
-  const size_t smem = decode_smem_bytes(p.tile_bytes);
-  decode_kernel<BV, NT><<<dim3(p.n_splits, p.n_kv, batch), kThreads, smem, st>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.n_splits, p.n_kv, batch);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = decode_smem_bytes(p.tile_bytes);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_kernel<BV, NT>, p);
 }
 
 template <int NT>
@@ -676,10 +784,13 @@ static cudaError_t launch_decode_nt(const DecodeParams& p, int bits_v, int batch
 
 // ws: >= decode_workspace_bytes_for(...) bytes, zero-filled before its first
 // use; every completed call leaves its counters (at the end of ws) zero.
-cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches, const int32_t* len,
+// n_new > 0 fuses the append of k_new / v_new ([batch][n_new][n_kv][128]).
+cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches, int32_t* len,
                           int batch, int64_t max_len, const void* q, int q_dtype, int n_q, int n_kv,
                           int bits_k, int bits_v, float* out, void* ws, size_t ws_bytes,
-                          uint32_t* status, cudaStream_t st) {
+                          uint32_t* status, cudaStream_t st, const void* k_new = nullptr,
+                          const void* v_new = nullptr, int kv_dtype = 0, int n_new = 0,
+                          int64_t cap = 0) {
   cudaError_t err = cudaSuccess;
   const int G = n_q / n_kv;
   const SplitPlan sp = decode_split_plan(batch, n_kv, G, bits_k, bits_v, max_len, &err, false);
@@ -687,6 +798,7 @@ cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches
   size_t gpart_off = 0;
   if (decode_workspace_layout(batch, n_kv, G, sp, &gpart_off) > ws_bytes)
     return cudaErrorInvalidValue;
+  if (n_new < 0 || n_new > kMaxNew) return cudaErrorInvalidValue;
   DecodeParams p;
   p.plans = plans;
   p.caches = caches;
@@ -701,9 +813,15 @@ cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches
   p.tiles_per_split = sp.tiles_per_split;
   p.n_groups = sp.n_groups;
   p.tile_bytes = tile_bytes(bits_k, bits_v);
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.kv_dtype = kv_dtype;
+  p.n_new = n_new;
+  p.cap = cap;
   p.part = reinterpret_cast<float*>(ws);
   p.gpart = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + gpart_off);
-  p.cnt_end = reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(ws) + (ws_bytes & ~size_t(3)));
+  p.cnt_end = reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(ws) +
+                                              (ws_bytes & ~size_t(3)));
   p.out = out;
   p.status = status;
   return G <= 8 ? launch_decode_nt<1>(p, bits_v, batch, st)

@@ -7,7 +7,7 @@
 // cache of the serving path. Readings adopted (energy on a 2^-32 integer
 // grid, fp16 norm, Gaussian Lloyd-Max codes, randomised Hadamard on values,
 // tile record layout) are stated in kvq.h.
-#include "common.cuh"
+#include "quant_dev.cuh"
 
 namespace kvq {
 
@@ -69,46 +69,6 @@ struct QuantParams {
   uint32_t* status;
 };
 
-// Number of width-w thresholds strictly below z (NaN -> 0): branch-free
-// binary search over the sorted 2^w - 1 thresholds.
-__device__ __forceinline__ int code_of(const float* thr, int w, float z) {
-  const float* t = thr + cb_t_off(w);
-  int c = 0;
-  for (int step = 1 << (w - 1); step; step >>= 1)
-    if (t[c + step - 1] < z) c += step;
-  return c;
-}
-
-// Fixed-order fp32 sum of squares of a 128-vector held as v[q] = x[lane + 32 q]:
-// p = ((v0^2 + v1^2) + v2^2) + v3^2, then p += p(lane ^ m) for m = 16..1.
-__device__ __forceinline__ float sumsq_tree(const float (&v)[4]) {
-  float p = __fadd_rn(__fadd_rn(__fadd_rn(__fmul_rn(v[0], v[0]), __fmul_rn(v[1], v[1])),
-                                __fmul_rn(v[2], v[2])),
-                      __fmul_rn(v[3], v[3]));
-#pragma unroll
-  for (int m = 16; m; m >>= 1) p = __fadd_rn(p, __shfl_xor_sync(0xffffffffu, p, m));
-  return p;
-}
-
-// Norm n (fp16 value), reciprocal r, flags, for a warp-held 128-vector.
-__device__ __forceinline__ void norm_and_recip(const float (&v)[4], bool finite, __half& n16,
-                                               float& r, uint32_t& flags) {
-  if (!finite) {
-    n16 = __float2half_rn(0.f);
-    r = 0.f;
-    flags |= KVQ_FLAG_NONFINITE;
-    return;
-  }
-  const float s = __fsqrt_rn(sumsq_tree(v));
-  n16 = __float2half_rn(s);
-  if (__hisinf(n16)) {
-    n16 = __ushort_as_half((unsigned short)0x7BFF);  // 65504
-    flags |= KVQ_FLAG_NORM_SAT;
-  }
-  const float n = __half2float(n16);
-  r = n > 0.f ? __frcp_rn(n) : 0.f;
-}
-
 // One CTA = the new tokens of one 32-token tile of one (sequence, KV head).
 __global__ void __launch_bounds__(256) quantize_append_kernel(QuantParams p) {
   const int b = blockIdx.z, h = blockIdx.y;
@@ -154,63 +114,8 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(QuantParams p) {
   for (int t = t_lo + warp; t < t_hi; t += blockDim.x >> 5) {
     const int tt = t - tile * kTile;
     const size_t row = (((size_t)b * p.n_new + (t - len0)) * p.n_kv + h) * kHeadDim;
-    float kx[4], vx[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      kx[q] = load_as_float(p.k, p.dtype, row + lane + 32 * q);
-      vx[q] = load_as_float(p.v, p.dtype, row + lane + 32 * q);
-    }
-    const bool kfin = __all_sync(0xffffffffu, isfinite(kx[0]) && isfinite(kx[1]) &&
-                                                  isfinite(kx[2]) && isfinite(kx[3]));
-    const bool vfin = __all_sync(0xffffffffu, isfinite(vx[0]) && isfinite(vx[1]) &&
-                                                  isfinite(vx[2]) && isfinite(vx[3]));
-    // keys: z_i = (k_i r) g_j, width b_j
-    __half kn;
-    float kr;
-    norm_and_recip(kx, kfin, kn, kr, flags);
-    const bool klive = kfin && __half2float(kn) > 0.f;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int i = lane + 32 * q, j = i & 63, w = pl.width[j];
-      int c = 0;
-      if (w > 0 && klive) c = code_of(s_thr, w, __fmul_rn(__fmul_rn(kx[q], kr), pl.g[j]));
-      s_kc[tt][i] = (uint8_t)c;
-    }
-    // values: y = H (s . v) by the fixed fp32 butterfly graph, z = y r
-    __half vn;
-    float vr;
-    norm_and_recip(vx, vfin, vn, vr, flags);
-    const bool vlive = vfin && __half2float(vn) > 0.f;
-    float y[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int i = lane + 32 * q;
-      const float x = vfin ? vx[q] : 0.f;
-      y[q] = ((pl.v_sign[i >> 5] >> (i & 31)) & 1u) ? -x : x;
-    }
-#pragma unroll
-    for (int hh = 1; hh < 32; hh <<= 1) {
-      const bool upper = (lane & hh) != 0;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float o = __shfl_xor_sync(0xffffffffu, y[q], hh);
-        y[q] = upper ? __fsub_rn(o, y[q]) : __fadd_rn(y[q], o);
-      }
-    }
-    {  // h = 32: (q0, q1), (q2, q3); h = 64: (q0, q2), (q1, q3)
-      float a0 = __fadd_rn(y[0], y[1]), a1 = __fsub_rn(y[0], y[1]);
-      float a2 = __fadd_rn(y[2], y[3]), a3 = __fsub_rn(y[2], y[3]);
-      y[0] = __fadd_rn(a0, a2);
-      y[2] = __fsub_rn(a0, a2);
-      y[1] = __fadd_rn(a1, a3);
-      y[3] = __fsub_rn(a1, a3);
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      int c = 0;
-      if (vlive) c = code_of(s_thr, bv, __fmul_rn(y[q], vr));
-      s_vc[tt][lane + 32 * q] = (uint8_t)c;
-    }
+    __half kn, vn;
+    warp_token_codes(pl, s_thr, p.k, p.v, p.dtype, row, lane, s_kc[tt], s_vc[tt], kn, vn, flags);
     if (lane == 0) {
       __half* norms = reinterpret_cast<__half*>(rec + 512 * (pl.bits_k + bv));
       norms[tt] = kn;
@@ -223,44 +128,8 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(QuantParams p) {
   // ---- assemble segment words: keep older tokens' bits, write the new ones,
   //      zero positions past the new length
   const int old_n = max(0, len0 - tile * kTile);  // positions holding older tokens
-  const int new_lo = t_lo - tile * kTile, new_hi = t_hi - tile * kTile;
-  uint32_t* words = reinterpret_cast<uint32_t*>(rec);
-  const int words_k = 128 * pl.bits_k;
-  for (int wi = threadIdx.x; wi < words_k + 128 * bv; wi += blockDim.x) {
-    int f, k, jj = 0, w = 0, pcoord = 0;
-    bool is_k = wi < words_k;
-    if (is_k) {
-      int lo = 0, hi = pl.n_ranks;  // largest rank r with seg_off[r] <= wi
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (pl.seg_off[mid] <= wi) lo = mid; else hi = mid;
-      }
-      jj = pl.order[lo];
-      w = pl.width[jj];
-      f = 2 * w;
-      k = wi - pl.seg_off[lo];
-    } else {
-      pcoord = (wi - words_k) / bv;
-      k = (wi - words_k) - pcoord * bv;
-      f = bv;
-    }
-    uint32_t nw = 0, keep = 0;
-    const int s0 = (32 * k) / f, s1 = (32 * k + 31) / f;
-    for (int s = s0; s <= s1 && s < kTile; ++s) {
-      const int tok = is_k ? token_of_slot_k(s) : token_of_slot_v(s);
-      const int fb = s * f - 32 * k + 32;  // bit position + 32, in (32 - f, 64)
-      uint32_t field;
-      if (tok >= new_lo && tok < new_hi) {
-        field = is_k ? (uint32_t)s_kc[tok][jj] | ((uint32_t)s_kc[tok][jj + 64] << w)
-                     : (uint32_t)s_vc[tok][pcoord];
-        nw |= (uint32_t)(((unsigned long long)field << fb) >> 32);
-      } else if (tok < old_n) {
-        field = (f == 32) ? 0xFFFFFFFFu : ((1u << f) - 1u);
-        keep |= (uint32_t)(((unsigned long long)field << fb) >> 32);
-      }
-    }
-    words[wi] = keep ? ((words[wi] & keep) | nw) : nw;
-  }
+  assemble_tile_words(reinterpret_cast<uint32_t*>(rec), pl, s_kc, s_vc, old_n,
+                      t_lo - tile * kTile, t_hi - tile * kTile, threadIdx.x, blockDim.x);
   if (threadIdx.x == 0 && s_flags) atomicOr(p.status, s_flags);
 }
 

@@ -30,7 +30,9 @@ PLAN_DTYPE = np.dtype([
     ("g", "<f4", 64), ("a_hat", "<f4", 64), ("width", "u1", 64), ("order", "u1", 64),
     ("seg_off", "<u2", 65), ("n_half", "u1"), ("pad0", "u1"), ("hs_width", "u1", 32),
     ("hs_rank0", "u1", 32), ("hs_count", "u1", 32), ("v_sign", "<u4", 4), ("pad1", "<u4"),
-    ("energy_sum", "<f8"), ("tail", "u1", PLAN_BYTES - 928),
+    ("energy_sum", "<f8"), ("n_class", "u1"), ("pad2", "u1", 7), ("cls_w", "u1", 8),
+    ("cls_hs0", "u1", 8), ("cls_nhs", "u1", 8), ("cls_last", "u1", 8), ("cls_seg0", "<u2", 8),
+    ("tail", "u1", PLAN_BYTES - 984),
 ])
 assert PLAN_DTYPE.itemsize == PLAN_BYTES
 
@@ -69,6 +71,8 @@ _SIGS = {
                                    _i64, _vp, _vp]),
     "kvq_decode_attn": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i64, _vp, _i32, _i32,
                                _vp, _vp, _sz, _vp, _vp]),
+    "kvq_append_decode": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i32, _vp, _vp, _i64,
+                                 _i32, _i64, _vp, _i32, _i32, _vp, _vp, _sz, _vp, _vp]),
     "kvq_decode_attn_noalloc": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i64, _vp, _i32,
                                        _i32, _vp, _vp, _vp]),
     "kvq_decode_noalloc_scratch_bytes": (_sz, []),
@@ -194,6 +198,18 @@ def decode_attn(cfg, plan_ptrs, cache_ptrs, lens, max_len, q, out, ws, status):
     _check(lib().kvq_decode_attn(ctypes.byref(cfg), _ptr(plan_ptrs), _ptr(cache_ptrs), _ptr(lens),
                                  batch, max_len, _ptr(q), _dtype_code(q), n_q, _ptr(out), _ptr(ws),
                                  ws.numel() * ws.element_size(), _ptr(status), _stream()))
+
+
+def append_decode(cfg, plan_ptrs, k, v, cache_ptrs, lens, cap_tokens, max_len, q, out, ws,
+                  status):
+    """Append k, v [batch, n_new, n_kv, 128] and decode q [batch, n_q, 128] in one launch."""
+    batch, n_q = q.shape[0], q.shape[1]
+    n_new = 0 if k is None else k.shape[1]
+    _check(lib().kvq_append_decode(ctypes.byref(cfg), _ptr(plan_ptrs), _ptr(k), _ptr(v),
+                                   _dtype_code(k) if k is not None else BF16, n_new,
+                                   _ptr(cache_ptrs), _ptr(lens), cap_tokens, batch, max_len,
+                                   _ptr(q), _dtype_code(q), n_q, _ptr(out), _ptr(ws),
+                                   ws.numel() * ws.element_size(), _ptr(status), _stream()))
 
 
 def decode_attn_noalloc(cfg, plan_ptrs, cache_ptrs, lens, max_len, q, out, status):

@@ -60,6 +60,17 @@ class PackedLayer:
                         self.status)
         return out
 
+    def append_decode(self, k, v, q, out=None, ws=None, max_len=None):
+        """Fused serving step: append k, v [batch, n_new, n_kv, 128], then decode q."""
+        max_len = self.cap if max_len is None else max_len
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=self.device)
+        if ws is None:
+            ws = self.workspace(q.shape[1], max_len)
+        kvq.append_decode(self.cfg, self.plan_ptrs, k, v, self.cache_ptrs, self.lens, self.cap,
+                          max_len, q, out, ws, self.status)
+        return out
+
     def workspace(self, n_q: int, max_len: int):
         """Decode workspace, zero-filled (its arrival counters must start at 0)."""
         n = kvq.decode_workspace_bytes(self.cfg, self.batch, n_q, max_len)

@@ -107,7 +107,13 @@ typedef struct {
  *   off 900  uint32  v_sign[4]      bit i set <=> value sign s_i = -1
  *   off 916  uint32  pad
  *   off 920  double  energy_sum     sum of the 64 block energies, fp64 in block order
- *   off 928  .. 1023 zero
+ *   off 928  uint8   n_class        decode schedule: runs of half steps of one width
+ *   off 936  uint8   cls_w[8]
+ *   off 944  uint8   cls_hs0[8]     first half step of the class
+ *   off 952  uint8   cls_nhs[8]     half steps in the class
+ *   off 960  uint8   cls_last[8]    blocks in the class's last half step
+ *   off 968  uint16  cls_seg0[8]    first K word of the class in a tile record
+ *   off 984  .. 1023 zero
  */
 #define KVQ_PLAN_BYTES 1024
 #define KVQ_PLAN_MAGIC 0x5051564Bu /* "KVQP" */
@@ -255,9 +261,9 @@ KVQ_API int kvq_quantize_append(const kvq_cfg* cfg, const void* const* plans_dev
  * ws_dev: >= kvq_decode_workspace_bytes(cfg, batch, n_q_heads, max_len)
  *        bytes, zero-filled once before its first use. Every completed call
  *        leaves the arrival counters it keeps at the end of the workspace at
- *        zero, so one workspace can serve any sequence of calls (of any
- *        shape that fits) on one stream; calls that overlap on the GPU must
- *        use different workspaces.
+ *        zero, so one workspace can serve any sequence of calls with the same
+ *        n_kv_heads (and shapes that fit) on one stream; calls that overlap
+ *        on the GPU must use different workspaces.
  * status_dev: required.
  * Returns KVQ_OK or a negative code.
  */
@@ -266,6 +272,27 @@ KVQ_API int kvq_decode_attn(const kvq_cfg* cfg, const void* const* plans_dev,
                     int64_t max_len, const void* q_dev, int q_dtype, int n_q_heads,
                     float* out_dev, void* ws_dev, size_t ws_bytes, uint32_t* status_dev,
                     kvq_stream_t stream);
+
+/*
+ * One serving step in one launch: kvq_quantize_append of n_new tokens per
+ * sequence followed by kvq_decode_attn over the grown caches (the pages'
+ * packed-cache serving path: append the step's keys and values, then decode).
+ * The CTA that owns a new token's tile quantizes and packs it before it
+ * streams the tile; every CTA decodes over len + n_new tokens; the last CTA
+ * of a sequence to read its length writes len + n_new.
+ * Arguments as for the two calls; n_new in 0..64 (k_dev, v_dev:
+ * [batch][n_new][n_kv_heads][128] of kv_dtype). A sequence with
+ * len + n_new > min(cap_tokens, max_len) gets no append (CAPACITY; len
+ * unchanged) and is decoded over its min(len, max_len) tokens. The workspace
+ * must be zero-filled once before first use and serve one n_kv_heads value.
+ * Returns KVQ_OK or a negative code.
+ */
+KVQ_API int kvq_append_decode(const kvq_cfg* cfg, const void* const* plans_dev, const void* k_dev,
+                              const void* v_dev, int kv_dtype, int n_new, void* const* cache_dev,
+                              int32_t* len_dev, int64_t cap_tokens, int batch, int64_t max_len,
+                              const void* q_dev, int q_dtype, int n_q_heads, float* out_dev,
+                              void* ws_dev, size_t ws_bytes, uint32_t* status_dev,
+                              kvq_stream_t stream);
 
 /*
  * Decode attention without a caller workspace. The paper has no counterpart:

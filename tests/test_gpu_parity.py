@@ -262,3 +262,52 @@ def test_serving_step_append_then_decode():
                               heads[h]["knorm"][tail], heads[h]["vnorm"][tail], plan, 64)
             check_records(got[-2:], ref, 64, wl.bits_k, wl.bits_v)
         assert op.rel_err(out[s], op.decode(host_f64(q[s]), heads)) <= TOL
+
+
+@pytest.mark.parametrize("n_new,bits", [(1, (3, 3)), (16, (3, 2)), (40, (2, 2)), (5, (6, 1))])
+def test_fused_append_decode(n_new, bits):
+    """kvq_append_decode (append n_new tokens and decode in one launch) against
+    the oracle: packed words and norms bit-exact, new lengths, outputs; one
+    sequence starts empty, one is refused for capacity (len unchanged, decoded
+    over its old tokens)."""
+    bk, bv = bits
+    rng = np.random.default_rng(100 + n_new)
+    n_kv, G, cap = 2, 8, 384
+    starts = [300, 31, 0, cap - n_new + 1]   # the last one overflows
+    cfg = kvq.make_cfg(n_kv, bk, bv, v_seed=6)
+    L = PackedLayer(cfg, len(starts), cap)
+    E, _, _ = _random_layer(rng, n_kv, 1, 1.2)
+    L.set_plans(kvq.plan_build(cfg, 2, E))
+    data = []
+    for s, T0 in enumerate(starts):
+        _, kb, vb = _random_layer(rng, n_kv, T0 + n_new, 1.2)
+        data.append((kb, vb))
+        if T0:
+            kvq.quantize_append(cfg, L.plan_ptrs[s:s + 1], dev_bf16(kb[:T0])[None],
+                                dev_bf16(vb[:T0])[None], L.cache_ptrs[s:s + 1],
+                                L.lens[s:s + 1], cap, L.status)
+    torch.cuda.synchronize()
+    assert L.flags() == 0
+    knew = torch.stack([dev_bf16(kb[T0:T0 + n_new]) for (kb, _), T0 in zip(data, starts)])
+    vnew = torch.stack([dev_bf16(vb[T0:T0 + n_new]) for (_, vb), T0 in zip(data, starts)])
+    qb = synth.to_bf16_bits(rng.standard_normal((len(starts), n_kv * G, 128)))
+    ws = L.workspace(n_kv * G, cap)
+    out = L.append_decode(knew, vnew, dev_bf16(qb), ws=ws).cpu().numpy()
+    torch.cuda.synchronize()
+    assert L.flags() == kvq.FLAG_CAPACITY
+    expect_len = [T0 + n_new for T0 in starts[:-1]] + [starts[-1]]
+    assert L.lens.cpu().tolist() == expect_len
+    for s, T in enumerate(expect_len):
+        kb, vb = data[s]
+        kh, vh = op.bf16_heads(kb[:T], vb[:T])
+        _, heads = op.layer(kh, vh, bk, bv, 6, 2, E=E)
+        for h in range(n_kv):
+            check_records(L.head_records(s, h, (T + 31) // 32), heads[h]["rec"], T, bk, bv)
+        q = synth.bf16_bits_to_f64(qb[s])
+        assert op.rel_err(out[s], op.decode(q, heads)) <= TOL, s
+    # the counters are back at zero: a second fused step on the same workspace
+    L.status.zero_()
+    k2 = torch.zeros((len(starts), 1, n_kv, 128), dtype=torch.bfloat16, device=DEV)
+    L.append_decode(k2, k2, dev_bf16(qb), ws=ws)
+    torch.cuda.synchronize()
+    assert L.lens.cpu().tolist()[:-1] == [x + 1 for x in expect_len[:-1]]

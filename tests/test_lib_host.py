@@ -82,6 +82,17 @@ def test_plan_build_equals_oracle(kind, bits):
                 covered += list(range(r0, r0 + n))
             assert covered == list(range(p["n_ranks"]))
             assert p["n_half"] <= 24
+            # classes: maximal runs of one width over the half steps
+            hs = 0
+            for ci in range(p["n_class"]):
+                w, h0, n = p["cls_w"][ci], p["cls_hs0"][ci], p["cls_nhs"][ci]
+                assert h0 == hs and n >= 1
+                assert all(p["hs_width"][x] == w for x in range(h0, h0 + n))
+                assert p["cls_last"][ci] == p["hs_count"][h0 + n - 1]
+                assert p["cls_seg0"][ci] == p["seg_off"][p["hs_rank0"][h0]]
+                hs += n
+            assert hs == p["n_half"]
+            assert len(set(p["cls_w"][:p["n_class"]])) == p["n_class"]
 
 
 def test_sizes():
