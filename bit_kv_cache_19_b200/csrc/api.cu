@@ -34,7 +34,7 @@ cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches
                           int batch, int64_t max_len, const void* q, int q_dtype, int n_q, int n_kv,
                           int bits_k, int bits_v, float* out, void* ws, size_t ws_bytes,
                           uint32_t* status, cudaStream_t st, const void* k_new, const void* v_new,
-                          int kv_dtype, int n_new, int64_t cap);
+                          int kv_dtype, int n_new, int64_t cap, int early);
 
 namespace {
 
@@ -330,7 +330,7 @@ int kvq_decode_attn(const kvq_cfg* cfg, const void* const* plans_dev, const void
                                 const_cast<int32_t*>(len_dev), batch, max_len, q_dev, q_dtype,
                                 n_q_heads, cfg->n_kv_heads, cfg->bits_k, cfg->bits_v, out_dev,
                                 ws_dev, ws_bytes, status_dev, reinterpret_cast<cudaStream_t>(stream),
-                                nullptr, nullptr, 0, 0, 0);
+                                nullptr, nullptr, 0, 0, 0, 0);
   if (e != cudaSuccess) return cuda_fail(e, "decode_attn");
   return KVQ_OK;
 }
@@ -339,13 +339,15 @@ int kvq_append_decode(const kvq_cfg* cfg, const void* const* plans_dev, const vo
                       const void* v_dev, int kv_dtype, int n_new, void* const* cache_dev,
                       int32_t* len_dev, int64_t cap_tokens, int batch, int64_t max_len,
                       const void* q_dev, int q_dtype, int n_q_heads, float* out_dev, void* ws_dev,
-                      size_t ws_bytes, uint32_t* status_dev, kvq_stream_t stream) {
+                      size_t ws_bytes, int step_flags, uint32_t* status_dev,
+                      kvq_stream_t stream) {
   int rc = check_cfg(cfg);
   if (rc) return rc;
   if (!plans_dev || !cache_dev || !len_dev || !q_dev || !out_dev || !ws_dev || !status_dev)
     return fail(KVQ_ERR_ARG, "null device pointer");
   if (n_new < 0 || n_new > 64) return fail(KVQ_ERR_ARG, "n_new %d not in 0..64", n_new);
   if (n_new > 0 && (!k_dev || !v_dev)) return fail(KVQ_ERR_ARG, "null k/v pointer");
+  if (step_flags & ~KVQ_STEP_EARLY) return fail(KVQ_ERR_ARG, "step_flags 0x%x", step_flags);
   if (!dtype_ok(kv_dtype) || !dtype_ok(q_dtype)) return fail(KVQ_ERR_ARG, "bad dtype");
   if (batch < 1 || batch > 65535) return fail(KVQ_ERR_ARG, "batch %d", batch);
   if (max_len < 1 || max_len > 0x7FFFFFFF || cap_tokens < 0 || cap_tokens > 0x7FFFFFFF)
@@ -361,7 +363,7 @@ int kvq_append_decode(const kvq_cfg* cfg, const void* const* plans_dev, const vo
                                 max_len, q_dev, q_dtype, n_q_heads, cfg->n_kv_heads, cfg->bits_k,
                                 cfg->bits_v, out_dev, ws_dev, ws_bytes, status_dev,
                                 reinterpret_cast<cudaStream_t>(stream), k_dev, v_dev, kv_dtype,
-                                n_new, cap_tokens);
+                                n_new, cap_tokens, (step_flags & KVQ_STEP_EARLY) ? 1 : 0);
   if (e != cudaSuccess) return cuda_fail(e, "append_decode");
   return KVQ_OK;
 }

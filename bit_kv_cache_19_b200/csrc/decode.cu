@@ -44,8 +44,10 @@ namespace kvq {
 // Lookup image (generated with the codebooks): byte offsets of its tables.
 __device__ __align__(16) const uint32_t g_lut_image[KVQ_LUT_BYTES / 4] = KVQ_LUT_IMAGE;
 __device__ const float g_thr[KVQ_CB_N_THR] = KVQ_CB_THR;
-constexpr uint32_t kLutRep[4] = {0u, 0u, 512u, 2560u};  // widths 1..3, lane-replicated
-constexpr uint32_t kLutPair4 = 10752u, kLutPair5 = 11776u, kLutSingle = 15872u;
+__host__ __device__ constexpr uint32_t lut_rep(int w) {  // widths 1..3, lane-replicated
+  return w == 1 ? 0x4000u : w == 2 ? 0x2000u : 0x0000u;
+}
+constexpr uint32_t kLutPair4 = 0x2800u, kLutPair5 = 0x2C00u, kLutSingle = 0x3C00u;
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
@@ -57,6 +59,7 @@ constexpr int kMaxSplits = 1024;
 constexpr int kCntStride = 2 + kMaxSplits / kGroup;  // per (sequence, KV head); last = sequence
 constexpr int kFallbackSlots = 1024;                  // CTA slots when no device answers
 constexpr int kMaxNew = 64;                           // tokens appended by a fused call
+constexpr int kScratch = 8192;                        // q' staging / append codes
 
 struct DecodeParams {
   const Plan* const* plans;
@@ -73,6 +76,7 @@ struct DecodeParams {
   const void* v_new;
   int kv_dtype, n_new;
   int64_t cap;
+  int early;  // read lengths and stream tiles before waiting for the previous kernel
   unsigned int* cnt_end;  // counters of pair k at cnt_end - (k + 1) * kCntStride
   float* part;            // [batch][n_kv][n_splits][G][130] = m, l, o[128]
   float* gpart;           // [batch][n_kv][n_groups][G][130]
@@ -87,25 +91,20 @@ struct alignas(128) Smem {
   float inv_scale[16];           // 2^-sigma of each head's q' scaling
   unsigned long long bar[kWarps][kStages];
   unsigned long long setup_bar;
+  uint32_t cls_lane[8][32];      // per (class, lane): first K word << 8 | bit shift
   int len0, is_last;
   uint32_t flags;
 };
 
-__device__ __forceinline__ uint32_t lds32(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
-  return v;
+// Loads from shared memory through pointers into the dynamic shared window,
+// so constant table offsets fold into the load instruction.
+__device__ __forceinline__ uint32_t ld32s(const uint8_t* p) {
+  return *reinterpret_cast<const uint32_t*>(p);
 }
-__device__ __forceinline__ uint32_t lds16(uint32_t a) {
-  unsigned short v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
-  return v;
+__device__ __forceinline__ uint32_t ld16s(const uint8_t* p) {
+  return *reinterpret_cast<const uint16_t*>(p);
 }
-__device__ __forceinline__ uint2 lds64(uint32_t a) {
-  uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
-  return v;
-}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -119,45 +118,41 @@ __device__ __forceinline__ void grid_dep_launch() {
 }
 
 // Four fp16 pairs from the 4 pair fields (2W bits each) that start at bit
-// `sh` of the word at shared address `wa`. lut: shared address of the lookup
-// image; lane4 = 4 * lane.
+// `sh` of the word at `wp` (shared memory). lut: the lookup image; lane4 = 4 *
+// lane. W is a compile-time width (the value width).
 template <int W>
-__device__ __forceinline__ void fields4(uint32_t lut, uint32_t wa, uint32_t sh, uint32_t lane4,
-                                        uint32_t (&out)[4]) {
+__device__ __forceinline__ void fields4(const uint8_t* lut, const uint8_t* wp, uint32_t sh,
+                                        uint32_t lane4, uint32_t (&out)[4]) {
   if constexpr (W <= 3) {
     // replicated pair table: entry e of lane l at byte (e * 32 + l) * 4
     constexpr uint32_t m7 = ((1u << (2 * W)) - 1u) << 7;
-    const uint32_t v7 = funnel_r(lds32(wa), lds32(wa + 4), sh) << 7;
-    const uint32_t base = lut + kLutRep[W];
+    const uint32_t v7 = funnel_r(ld32s(wp), ld32s(wp + 4), sh) << 7;
+    const uint32_t lb = lane4 | lut_rep(W);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) out[i] = lds32(base + (((v7 >> (2 * W * i)) & m7) | lane4));
+    for (int i = 0; i < 4; ++i) out[i] = ld32s(lut + (((v7 >> (2 * W * i)) & m7) | lb));
   } else if constexpr (W == 4) {
-    const uint32_t v = funnel_r(lds32(wa), lds32(wa + 4), sh);
-    const uint32_t base = lut + kLutPair4;
-    out[0] = lds32(base + ((v << 2) & 0x3FCu));
+    const uint32_t v = funnel_r(ld32s(wp), ld32s(wp + 4), sh);
+    out[0] = ld32s(lut + kLutPair4 + ((v << 2) & 0x3FCu));
 #pragma unroll
-    for (int i = 1; i < 4; ++i) out[i] = lds32(base + ((v >> (8 * i - 2)) & 0x3FCu));
+    for (int i = 1; i < 4; ++i) out[i] = ld32s(lut + kLutPair4 + ((v >> (8 * i - 2)) & 0x3FCu));
   } else if constexpr (W == 5) {
-    const uint32_t w0 = lds32(wa), w1 = lds32(wa + 4), w2 = lds32(wa + 8);
+    const uint32_t w0 = ld32s(wp), w1 = ld32s(wp + 4), w2 = ld32s(wp + 8);
     const uint32_t lo = funnel_r(w0, w1, sh), hi = funnel_r(w1, w2, sh);
-    const uint32_t base = lut + kLutPair5;
-    out[0] = lds32(base + ((lo << 2) & 0xFFCu));
-    out[1] = lds32(base + ((lo >> 8) & 0xFFCu));
-    out[2] = lds32(base + ((lo >> 18) & 0xFFCu));
-    out[3] = lds32(base + (funnel_r(lo, hi, 28) & 0xFFCu));
+    out[0] = ld32s(lut + kLutPair5 + ((lo << 2) & 0xFFCu));
+    out[1] = ld32s(lut + kLutPair5 + ((lo >> 8) & 0xFFCu));
+    out[2] = ld32s(lut + kLutPair5 + ((lo >> 18) & 0xFFCu));
+    out[3] = ld32s(lut + kLutPair5 + (funnel_r(lo, hi, 28) & 0xFFCu));
   } else {
     // widths 6..8: two single-code lookups per pair (fp16 table, 2 bytes each)
-    const uint32_t w0 = lds32(wa), w1 = lds32(wa + 4), w2 = lds32(wa + 8);
+    const uint32_t w0 = ld32s(wp), w1 = ld32s(wp + 4), w2 = ld32s(wp + 8);
     const uint32_t lo = funnel_r(w0, w1, sh), hi = funnel_r(w1, w2, sh);
     const unsigned long long v = ((unsigned long long)hi << 32) | lo;
     constexpr uint32_t mw = ((1u << W) - 1u) << 1;
-    const uint32_t base = lut + kLutSingle + 2u * (uint32_t)cb_c_off(W);
+    const uint8_t* tab = lut + kLutSingle + 2u * (uint32_t)cb_c_off(W);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const uint32_t a = (uint32_t)(v >> (2 * W * i)) << 1;
-      const uint32_t c0 = lds16(base + (a & mw));
-      const uint32_t c1 = lds16(base + ((a >> W) & mw));
-      out[i] = c0 | (c1 << 16);
+      out[i] = ld16s(tab + (a & mw)) | (ld16s(tab + ((a >> W) & mw)) << 16);
     }
   }
 }
@@ -171,32 +166,80 @@ __device__ __forceinline__ void mma_1688(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(b0));
 }
 
-// Logits of one width class: half steps hs0 .. hs0 + nhs - 1, each 4 blocks
-// of width W (the last one `last` blocks). Lane (g, c) takes block c of every
-// half step, tokens g, g + 8 (m-tile 0) and g + 16, g + 24 (m-tile 1).
-template <int W, int NT>
-__device__ __forceinline__ void key_class(uint32_t lut, uint32_t kw, uint32_t qf, int hs0, int nhs,
-                                          int seg0, int last, int g, int c, uint32_t lane4,
-                                          float (&s)[2][NT][4]) {
-  const uint32_t base = kw + 4u * (uint32_t)(seg0 + 2 * W * c + ((W * g) >> 2));
-  const uint32_t sh = (uint32_t)(8 * W * g) & 31u;
-  const uint32_t qbase = qf + (uint32_t)hs0 * 256u + lane4 * 2u;
-  auto step = [&](int i, bool valid) {
-    uint32_t A[4] = {0u, 0u, 0u, 0u};
-    if (valid) fields4<W>(lut, base + 32u * W * (uint32_t)i, sh, lane4, A);
+// Logits of one width class: its nhs half steps of <= 4 blocks of width W
+// (runtime, warp-uniform: one code path per lookup kind keeps the kernel
+// small). Lane (g, c) takes block c of every half step, tokens g, g + 8
+// (m-tile 0) and g + 16, g + 24 (m-tile 1). In a class's last half step the
+// lanes past its last block read other valid words of the tile: their q' is
+// exactly 0, so those finite fp16 values add nothing.
+template <int NT>
+__device__ __forceinline__ void key_mma(float (&s)[2][NT][4], const uint32_t (&A)[4],
+                                        const uint2* qp) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const uint2 b = lds64(qbase + (uint32_t)(nt * kMaxHalf + i) * 256u);
-      mma_1688(s[0][nt], A[0], A[1], b.x);
-      mma_1688(s[0][nt], A[0], A[1], b.y);
-      mma_1688(s[1][nt], A[2], A[3], b.x);
-      mma_1688(s[1][nt], A[2], A[3], b.y);
+  for (int nt = 0; nt < NT; ++nt) {
+    const uint2 b = qp[nt * kMaxHalf * 32];
+    mma_1688(s[0][nt], A[0], A[1], b.x);
+    mma_1688(s[0][nt], A[0], A[1], b.y);
+    mma_1688(s[1][nt], A[2], A[3], b.x);
+    mma_1688(s[1][nt], A[2], A[3], b.y);
+  }
+}
+
+template <int NT>
+__device__ __forceinline__ void key_class(const Smem& sm, const uint8_t* kw, int ci, int lane,
+                                          uint32_t lane4, float (&s)[2][NT][4]) {
+  const int W = sm.plan.cls_w[ci];
+  const int nhs = sm.plan.cls_nhs[ci];
+  const uint32_t pk = sm.cls_lane[ci][lane];
+  const uint8_t* wp = kw + 4u * (pk >> 8);
+  const uint32_t sh = pk & 31u;
+  const uint2* qp = &sm.qfrag[0][sm.plan.cls_hs0[ci]][lane];
+  const uint32_t stride = 32u * (uint32_t)W;  // bytes per half step (8W words)
+  const uint32_t w2 = 2u * (uint32_t)W;
+  const uint8_t* lut = sm.lut;
+  if (W <= 3) {
+    const uint32_t m7 = ((1u << w2) - 1u) << 7;
+    const uint32_t lb = lane4 | lut_rep(W);
+    for (int i = 0; i < nhs; ++i, wp += stride, qp += 32) {
+      const uint32_t v7 = funnel_r(ld32s(wp), ld32s(wp + 4), sh) << 7;
+      uint32_t A[4];
+      A[0] = ld32s(lut + ((v7 & m7) | lb));
+      A[1] = ld32s(lut + (((v7 >> w2) & m7) | lb));
+      A[2] = ld32s(lut + (((v7 >> (2u * w2)) & m7) | lb));
+      A[3] = ld32s(lut + (((v7 >> (3u * w2)) & m7) | lb));
+      key_mma<NT>(s, A, qp);
     }
-  };
-  for (int i = 0; i < nhs - 1; ++i) step(i, true);
-  // last half step: lanes past its last block feed zeros (their q' is 0);
-  // every lane still takes part in the warp-wide MMAs
-  step(nhs - 1, c < last);
+  } else if (W == 4) {
+    for (int i = 0; i < nhs; ++i, wp += stride, qp += 32) {
+      uint32_t A[4];
+      fields4<4>(lut, wp, sh, lane4, A);
+      key_mma<NT>(s, A, qp);
+    }
+  } else if (W == 5) {
+    for (int i = 0; i < nhs; ++i, wp += stride, qp += 32) {
+      uint32_t A[4];
+      fields4<5>(lut, wp, sh, lane4, A);
+      key_mma<NT>(s, A, qp);
+    }
+  } else {
+    // widths 6..8: two single-code lookups per pair (fp16 table, 2 bytes
+    // each); window a holds the codes of tokens g, g + 8, window b of g + 16,
+    // g + 24; code k of a window at byte 2 * code = (win >> (k W - 1)) & mw
+    const uint8_t* tab = lut + kLutSingle + 2u * (uint32_t)((1 << W) - 2);
+    const uint32_t mw = ((1u << W) - 1u) << 1;
+    const uint32_t offb = 4u * ((sh + 4u * W) >> 5), shb = (sh + 4u * W) & 31u;
+    const uint32_t s1 = (uint32_t)W - 1u, s2 = 2u * W - 1u, s3 = 3u * W - 1u;
+    for (int i = 0; i < nhs; ++i, wp += stride, qp += 32) {
+      const uint32_t ua = funnel_r(ld32s(wp), ld32s(wp + 4), sh);
+      const uint32_t ub = funnel_r(ld32s(wp + offb), ld32s(wp + offb + 4), shb);
+      uint32_t A[4];
+      A[0] = ld16s(tab + ((ua << 1) & mw)) | (ld16s(tab + ((ua >> s1) & mw)) << 16);
+      A[1] = ld16s(tab + ((ua >> s2) & mw)) | (ld16s(tab + ((ua >> s3) & mw)) << 16);
+      A[2] = ld16s(tab + ((ub << 1) & mw)) | (ld16s(tab + ((ub >> s1) & mw)) << 16);
+      A[3] = ld16s(tab + ((ub >> s2) & mw)) | (ld16s(tab + ((ub >> s3) & mw)) << 16);
+      key_mma<NT>(s, A, qp);
+    }
+  }
 }
 
 // Inverse value rotation of one head held by a warp (o[128] in `src`),
@@ -229,23 +272,41 @@ __device__ __forceinline__ void warp_unrotate_store(const float* src, const Plan
 }
 
 // Merge n records per head (record s of head h at src + s * rec_stride +
-// h * 130) into dst (record h at dst + h * 130), for G heads.
+// h * 130) into dst (record h at dst + h * 130), for G heads. One pass with
+// online rescaling over chunks of 8 records whose loads are issued together,
+// so a merge costs about n / 8 load round trips. Threads: 128 coordinates x
+// 2 heads at a time.
 __device__ __forceinline__ void merge_records(const float* src, int n, size_t rec_stride, int G,
                                               float* dst) {
   const int tid = threadIdx.x;
   for (int head = tid >> 7; head < G; head += kThreads / 128) {
     const int x = tid & 127;
     const float* r = src + (size_t)head * kPartStride;
-    float M = -INFINITY;
-    for (int s = 0; s < n; ++s) M = fmaxf(M, r[s * rec_stride]);
-    float L = 0.f, O = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll 4
-      for (int s = 0; s < n; ++s) {
-        const float* q = r + s * rec_stride;
-        const float w = ex2(q[0] - M);
-        L += w * q[1];
-        O += w * q[2 + x];
+    float M = -INFINITY, L = 0.f, O = 0.f;
+    for (int s0 = 0; s0 < n; s0 += 8) {
+      float mm[8], ll[8], oo[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const bool v = s0 + k < n;
+        const float* q = r + (size_t)(v ? s0 + k : 0) * rec_stride;
+        mm[k] = v ? q[0] : -INFINITY;
+        ll[k] = v ? q[1] : 0.f;
+        oo[k] = v ? q[2 + x] : 0.f;
+      }
+      float cm = M;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) cm = fmaxf(cm, mm[k]);
+      if (cm != -INFINITY) {
+        const float a = ex2(M - cm);
+        L *= a;
+        O *= a;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float w = ex2(mm[k] - cm);
+          L += w * ll[k];
+          O += w * oo[k];
+        }
+        M = cm;
       }
     }
     float* d = dst + (size_t)head * kPartStride;
@@ -258,10 +319,11 @@ __device__ __forceinline__ void merge_records(const float* src, int n, size_t re
 }
 
 template <int BV, int NT>
-__global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
-  uint8_t* const stage_base = smem_raw + sizeof(Smem);
+  uint8_t* const scratch = smem_raw + sizeof(Smem);  // q' staging / append codes
+  uint8_t* const stage_base = scratch + kScratch;
 
   const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
@@ -280,17 +342,20 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     bulk_g2s(sm.lut, g_lut_image, KVQ_LUT_BYTES, &sm.setup_bar);
     sm.flags = 0u;
   }
-  // ---- everything below may read what the previous kernel wrote
-  grid_dep_wait();
+  // ---- with `early` the caller guarantees that the previous kernel on the
+  //      stream writes neither these caches nor these lengths: the length is
+  //      read and the first tiles are streamed before waiting for it
+  if (!p.early) grid_dep_wait();
   if (tid == 0) {
     const int l0 = p.len[b];
     sm.len0 = l0;
     if (p.n_new > 0) {
-      // the last CTA of the sequence to read its length writes the new one
+      // the last CTA of the sequence to read its length writes the new one;
+      // the counter wraps to zero in the same atomic, so a kernel that starts
+      // before this one has ended finds it at zero
       __threadfence();
       const unsigned int total = (unsigned int)(p.n_kv * p.n_splits);
-      if (atomicAdd(seq_cnt, 1u) == total - 1u) {
-        *seq_cnt = 0u;
+      if (atomicInc(seq_cnt, total - 1u) == total - 1u) {
         const int64_t lim = min((int64_t)p.max_len, p.cap);
         if (l0 >= 0 && (int64_t)l0 + p.n_new <= lim) p.len[b] = l0 + p.n_new;
       }
@@ -298,7 +363,6 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
   }
   __syncthreads();
   const bool ok_setup = mbar_wait_bounded(&sm.setup_bar, 0u);
-  grid_dep_launch();
   const uint8_t* cache = p.caches[b];
   const int bk = sm.plan.bits_k;
   const int n_half = sm.plan.n_half;
@@ -328,11 +392,30 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
   const int te = min(n_tiles, tb + p.tiles_per_split);
   const bool has_work = tb < te;
 
+  // ---- start streaming the warp's first tiles (tiles the append writes wait)
+  const int tbytes = p.tile_bytes;
+  uint8_t* const my_stages = stage_base + (size_t)warp * kStages * tbytes;
+  const int n_mine = has_work ? max(0, (te - tb - warp + kWarps - 1) / kWarps) : 0;
+  auto tile_of = [&](int i) { return tb + warp + i * kWarps; };
+  auto issue = [&](int i) {
+    const int s = i % kStages;
+    unsigned long long* bar = &sm.bar[warp][s];
+    mbar_expect_tx(bar, (uint32_t)tbytes);
+    bulk_g2s(my_stages + s * tbytes, cache + ((size_t)tile_of(i) * p.n_kv + h) * tbytes,
+             (uint32_t)tbytes, bar);
+  };
+  const int t_app = n_add > 0 ? len0 / kTile : 0x7FFFFFFF;
+  if (lane == 0)
+    for (int i = 0; i < min(kStages, n_mine); ++i)
+      if (tile_of(i) < t_app) issue(i);
+  if (p.early) grid_dep_wait();
+  grid_dep_launch();
+
   // ---- fused append: quantize and pack the new tokens whose tiles are ours
   if (has_work && n_add > 0) {
     const int t_first = len0 / kTile, t_last = (len0 + n_add - 1) / kTile;
-    uint8_t (*kc)[kHeadDim] = reinterpret_cast<uint8_t (*)[kHeadDim]>(stage_base);
-    uint8_t (*vc)[kHeadDim] = reinterpret_cast<uint8_t (*)[kHeadDim]>(stage_base + 32 * kHeadDim);
+    uint8_t (*kc)[kHeadDim] = reinterpret_cast<uint8_t (*)[kHeadDim]>(scratch);
+    uint8_t (*vc)[kHeadDim] = reinterpret_cast<uint8_t (*)[kHeadDim]>(scratch + 32 * kHeadDim);
     uint32_t flags = 0;
     for (int tile = max(t_first, tb); tile <= min(t_last, te - 1); ++tile) {
       const int t_lo = max(len0, tile * kTile), t_hi = min(len0 + n_add, tile * kTile + kTile);
@@ -362,6 +445,9 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     __syncthreads();
     if (tid == 0 && sm.flags) atomicOr(p.status, sm.flags);
   }
+  if (lane == 0)
+    for (int i = 0; i < min(kStages, n_mine); ++i)
+      if (tile_of(i) >= t_app) issue(i);
 
   float o[8][NT][4];
   float m_run[NT][2], l_run[NT][2];
@@ -383,7 +469,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     // ---- query prologue (q' staged in the tile ring before it is used):
     //      q' = q a_hat_j log2(e) / sqrt(128); per-head 2^sigma scaling into
     //      the fp16 range; hi/lo split into the B fragments of each half step
-    float* qp = reinterpret_cast<float*>(stage_base);  // [16][128]
+    float* qp = reinterpret_cast<float*>(scratch);  // [16][128]
+#pragma unroll
     for (int i = tid; i < 16 * kHeadDim; i += kThreads) {
       const int head = i >> 7, x = i & 127;
       float v = 0.f;
@@ -419,30 +506,20 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
       const uint32_t lo = pack_half2(x0 - __low2float(hh), x1 - __high2float(hh));
       sm.qfrag[nt][hs][ln] = make_uint2(hi, lo);
     }
+    for (int e = tid; e < sm.plan.n_class * 32; e += kThreads) {
+      const int ci = e >> 5, ln = e & 31, W = sm.plan.cls_w[ci];
+      const int off = sm.plan.cls_seg0[ci] + 2 * W * (ln & 3) + ((W * (ln >> 2)) >> 2);
+      sm.cls_lane[ci][ln] = ((uint32_t)off << 8) | ((uint32_t)(8 * W * (ln >> 2)) & 31u);
+    }
     __syncthreads();
 
     // ---- per-warp pipeline over the warp's tiles
-    const int tbytes = p.tile_bytes;
-    uint8_t* const my_stages = stage_base + (size_t)warp * kStages * tbytes;
-    const int n_mine = max(0, (te - tb - warp + kWarps - 1) / kWarps);
-    auto tile_of = [&](int i) { return tb + warp + i * kWarps; };
-    auto issue = [&](int i) {
-      const int s = i % kStages;
-      unsigned long long* bar = &sm.bar[warp][s];
-      mbar_expect_tx(bar, (uint32_t)tbytes);
-      bulk_g2s(my_stages + s * tbytes, cache + ((size_t)tile_of(i) * p.n_kv + h) * tbytes,
-               (uint32_t)tbytes, bar);
-    };
-    if (lane == 0)
-      for (int i = 0; i < min(kStages, n_mine); ++i) issue(i);
     __syncwarp();
 
-    const uint32_t lut = smem_addr(sm.lut);
-    const uint32_t qf = smem_addr(&sm.qfrag[0][0][0]);
     const uint32_t lane4 = (uint32_t)lane * 4u;
     const int n_class = sm.plan.n_class;
     const uint32_t v_sh = (uint32_t)(8 * BV * c) & 31u;
-    const uint32_t v_off = 4u * (uint32_t)((BV * c) >> 2);
+    const int v_off = 4 * (g * BV + ((BV * c) >> 2));  // row g of each m-tile, lane's slots
     int consumed = 0;
     bool timed_out = false;
     for (int i = 0; i < n_mine; ++i) {
@@ -455,9 +532,9 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
       consumed = i + 1;
       const int tile = tile_of(i);
       const int nvalid = min(kTile, L - tile * kTile);
-      const uint32_t kw = smem_addr(my_stages + s * tbytes);
-      const uint32_t vw = kw + 512u * (uint32_t)bk;
-      const __half* nrm = reinterpret_cast<const __half*>(my_stages + s * tbytes + 512 * (bk + BV));
+      const uint8_t* kw = my_stages + s * tbytes;
+      const uint8_t* vw = kw + 512 * bk + v_off;
+      const __half* nrm = reinterpret_cast<const __half*>(kw + 512 * (bk + BV));
 
       // keys: S[32 tokens x 8 NT heads] on the tensor cores
       float sacc[2][NT][4];
@@ -467,20 +544,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
           for (int r = 0; r < 4; ++r) sacc[mt][nt][r] = 0.f;
-      for (int ci = 0; ci < n_class; ++ci) {
-        const int hs0 = sm.plan.cls_hs0[ci], nhs = sm.plan.cls_nhs[ci],
-                  seg0 = sm.plan.cls_seg0[ci], last = sm.plan.cls_last[ci];
-        switch (sm.plan.cls_w[ci]) {
-          case 1: key_class<1, NT>(lut, kw, qf, hs0, nhs, seg0, last, g, c, lane4, sacc); break;
-          case 2: key_class<2, NT>(lut, kw, qf, hs0, nhs, seg0, last, g, c, lane4, sacc); break;
-          case 3: key_class<3, NT>(lut, kw, qf, hs0, nhs, seg0, last, g, c, lane4, sacc); break;
-          case 4: key_class<4, NT>(lut, kw, qf, hs0, nhs, seg0, last, g, c, lane4, sacc); break;
-          case 5: key_class<5, NT>(lut, kw, qf, hs0, nhs, seg0, last, g, c, lane4, sacc); break;
-          case 6: key_class<6, NT>(lut, kw, qf, hs0, nhs, seg0, last, g, c, lane4, sacc); break;
-          case 7: key_class<7, NT>(lut, kw, qf, hs0, nhs, seg0, last, g, c, lane4, sacc); break;
-          default: key_class<8, NT>(lut, kw, qf, hs0, nhs, seg0, last, g, c, lane4, sacc); break;
-        }
-      }
+      for (int ci = 0; ci < n_class; ++ci) key_class<NT>(sm, kw, ci, lane, lane4, sacc);
 
       // online softmax (base 2); this thread's tokens are g + 8 r, r = 0..3
       float nk[4], nv[4];
@@ -544,8 +608,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
 #pragma unroll
       for (int mu = 0; mu < 8; ++mu) {
         uint32_t F0[4], F1[4];
-        fields4<BV>(lut, vw + 4u * (uint32_t)((16 * mu + g) * BV) + v_off, v_sh, lane4, F0);
-        fields4<BV>(lut, vw + 4u * (uint32_t)((16 * mu + g + 8) * BV) + v_off, v_sh, lane4, F1);
+        fields4<BV>(sm.lut, vw + 4 * (16 * mu * BV), v_sh, lane4, F0);
+        fields4<BV>(sm.lut, vw + 4 * ((16 * mu + 8) * BV), v_sh, lane4, F1);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           mma_16816(o[mu][nt], F0[0], F1[0], F0[1], F1[1], pb0[0][nt], pb1[0][nt]);
@@ -578,12 +642,12 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
       l_run[nt][e] = l;
     }
   __syncthreads();
-  float* mg = reinterpret_cast<float*>(stage_base);  // [warp][16 heads][130]
+  float* mg = reinterpret_cast<float*>(stage_base);  // [warp][8 NT heads][130]
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      float* dst = mg + ((size_t)warp * 16 + 8 * nt + 2 * c + e) * kPartStride;
+      float* dst = mg + ((size_t)warp * 8 * NT + 8 * nt + 2 * c + e) * kPartStride;
       if (g == 0) {
         dst[0] = m_run[nt][e];
         dst[1] = l_run[nt][e];
@@ -596,7 +660,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     }
   __syncthreads();
   float* const my_part = p.part + (bh * p.n_splits + split) * G * kPartStride;
-  merge_records(mg, kWarps, (size_t)16 * kPartStride, G, my_part);
+  merge_records(mg, kWarps, (size_t)8 * NT * kPartStride, G, my_part);
 
   // ---- level 1: the last CTA of this group of splits merges the group
   const int grp = split / kGroup;
@@ -639,10 +703,10 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
 }
 
 // ------------------------------------------------------------- launchers
-size_t decode_smem_bytes(int tile_bytes) {
+size_t decode_smem_bytes(int tile_bytes, int nt) {
   const size_t stages = (size_t)kWarps * kStages * tile_bytes;
-  const size_t merge = (size_t)kWarps * 16 * kPartStride * sizeof(float);
-  return sizeof(Smem) + std::max(stages, merge);
+  const size_t merge = (size_t)kWarps * 8 * nt * kPartStride * sizeof(float);
+  return sizeof(Smem) + kScratch + std::max(stages, merge);
 }
 
 // CTAs per SM of one instantiation for tiles of (bits_k, BV), queried once per
@@ -660,12 +724,12 @@ static int ctas_per_sm(int dev, int bits_k, cudaError_t* err) {
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(cap_set.load() & bit)) {
     e = cudaFuncSetAttribute(decode_kernel<BV, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)decode_smem_bytes(tile_bytes(8, BV)));
+                             (int)decode_smem_bytes(tile_bytes(8, BV), NT));
     if (e == cudaSuccess) cap_set.fetch_or(bit);
   }
   if (e == cudaSuccess)
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-        &v, decode_kernel<BV, NT>, kThreads, decode_smem_bytes(tile_bytes(bits_k, BV)));
+        &v, decode_kernel<BV, NT>, kThreads, decode_smem_bytes(tile_bytes(bits_k, BV), NT));
   if (e != cudaSuccess) {
     *err = e;
     return 0;
@@ -757,7 +821,7 @@ static cudaError_t launch_decode_t(const DecodeParams& p, int batch, cudaStream_
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.n_splits, p.n_kv, batch);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = decode_smem_bytes(p.tile_bytes);
+  cfg.dynamicSmemBytes = decode_smem_bytes(p.tile_bytes, NT);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -788,9 +852,8 @@ static cudaError_t launch_decode_nt(const DecodeParams& p, int bits_v, int batch
 cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches, int32_t* len,
                           int batch, int64_t max_len, const void* q, int q_dtype, int n_q, int n_kv,
                           int bits_k, int bits_v, float* out, void* ws, size_t ws_bytes,
-                          uint32_t* status, cudaStream_t st, const void* k_new = nullptr,
-                          const void* v_new = nullptr, int kv_dtype = 0, int n_new = 0,
-                          int64_t cap = 0) {
+                          uint32_t* status, cudaStream_t st, const void* k_new,
+                          const void* v_new, int kv_dtype, int n_new, int64_t cap, int early) {
   cudaError_t err = cudaSuccess;
   const int G = n_q / n_kv;
   const SplitPlan sp = decode_split_plan(batch, n_kv, G, bits_k, bits_v, max_len, &err, false);
@@ -818,6 +881,7 @@ cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches
   p.kv_dtype = kv_dtype;
   p.n_new = n_new;
   p.cap = cap;
+  p.early = early;
   p.part = reinterpret_cast<float*>(ws);
   p.gpart = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + gpart_off);
   p.cnt_end = reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(ws) +

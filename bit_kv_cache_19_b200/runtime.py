@@ -60,7 +60,7 @@ class PackedLayer:
                         self.status)
         return out
 
-    def append_decode(self, k, v, q, out=None, ws=None, max_len=None):
+    def append_decode(self, k, v, q, out=None, ws=None, max_len=None, step_flags=0):
         """Fused serving step: append k, v [batch, n_new, n_kv, 128], then decode q."""
         max_len = self.cap if max_len is None else max_len
         if out is None:
@@ -68,7 +68,7 @@ class PackedLayer:
         if ws is None:
             ws = self.workspace(q.shape[1], max_len)
         kvq.append_decode(self.cfg, self.plan_ptrs, k, v, self.cache_ptrs, self.lens, self.cap,
-                          max_len, q, out, ws, self.status)
+                          max_len, q, out, ws, self.status, step_flags)
         return out
 
     def workspace(self, n_q: int, max_len: int):

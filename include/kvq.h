@@ -69,6 +69,9 @@ typedef struct CUstream_st* kvq_stream_t;
 #define KVQ_FP16 1
 #define KVQ_FP32 2
 
+/* kvq_append_decode step flags. */
+#define KVQ_STEP_EARLY 1u  /* see kvq_append_decode */
+
 /* Allocation modes. */
 #define KVQ_ALLOC_GREEDY 0   /* Block-GTQ: greedy marginal-gain widths per RoPE block */
 #define KVQ_ALLOC_UNIFORM 1  /* every block gets bits_k (same bytes; comparator) */
@@ -285,13 +288,23 @@ KVQ_API int kvq_decode_attn(const kvq_cfg* cfg, const void* const* plans_dev,
  * len + n_new > min(cap_tokens, max_len) gets no append (CAPACITY; len
  * unchanged) and is decoded over its min(len, max_len) tokens. The workspace
  * must be zero-filled once before first use and serve one n_kv_heads value.
+ * The kernel uses programmatic dependent launch: work that reads nothing the
+ * previous kernel on the stream writes (the plan, the lookup tables) starts
+ * before that kernel ends. step_flags:
+ *   KVQ_STEP_EARLY  the lengths are read and the first cache tiles streamed
+ *                   before the previous kernel on the stream has finished.
+ *                   Only set it when that kernel writes neither these caches
+ *                   nor these lengths (e.g. in a loop over layers, where the
+ *                   previous kernel is another layer's step, which may share
+ *                   the workspace); q, k_dev, v_dev, out and the rest of the
+ *                   workspace are always accessed after it.
  * Returns KVQ_OK or a negative code.
  */
 KVQ_API int kvq_append_decode(const kvq_cfg* cfg, const void* const* plans_dev, const void* k_dev,
                               const void* v_dev, int kv_dtype, int n_new, void* const* cache_dev,
                               int32_t* len_dev, int64_t cap_tokens, int batch, int64_t max_len,
                               const void* q_dev, int q_dtype, int n_q_heads, float* out_dev,
-                              void* ws_dev, size_t ws_bytes, uint32_t* status_dev,
+                              void* ws_dev, size_t ws_bytes, int step_flags, uint32_t* status_dev,
                               kvq_stream_t stream);
 
 /*

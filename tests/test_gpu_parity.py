@@ -264,8 +264,9 @@ def test_serving_step_append_then_decode():
         assert op.rel_err(out[s], op.decode(host_f64(q[s]), heads)) <= TOL
 
 
-@pytest.mark.parametrize("n_new,bits", [(1, (3, 3)), (16, (3, 2)), (40, (2, 2)), (5, (6, 1))])
-def test_fused_append_decode(n_new, bits):
+@pytest.mark.parametrize("n_new,bits,flags", [(1, (3, 3), 0), (1, (3, 3), 1), (16, (3, 2), 1),
+                                              (40, (2, 2), 0), (5, (6, 1), 1)])
+def test_fused_append_decode(n_new, bits, flags):
     """kvq_append_decode (append n_new tokens and decode in one launch) against
     the oracle: packed words and norms bit-exact, new lengths, outputs; one
     sequence starts empty, one is refused for capacity (len unchanged, decoded
@@ -292,7 +293,7 @@ def test_fused_append_decode(n_new, bits):
     vnew = torch.stack([dev_bf16(vb[T0:T0 + n_new]) for (_, vb), T0 in zip(data, starts)])
     qb = synth.to_bf16_bits(rng.standard_normal((len(starts), n_kv * G, 128)))
     ws = L.workspace(n_kv * G, cap)
-    out = L.append_decode(knew, vnew, dev_bf16(qb), ws=ws).cpu().numpy()
+    out = L.append_decode(knew, vnew, dev_bf16(qb), ws=ws, step_flags=flags).cpu().numpy()
     torch.cuda.synchronize()
     assert L.flags() == kvq.FLAG_CAPACITY
     expect_len = [T0 + n_new for T0 in starts[:-1]] + [starts[-1]]
@@ -308,6 +309,55 @@ def test_fused_append_decode(n_new, bits):
     # the counters are back at zero: a second fused step on the same workspace
     L.status.zero_()
     k2 = torch.zeros((len(starts), 1, n_kv, 128), dtype=torch.bfloat16, device=DEV)
-    L.append_decode(k2, k2, dev_bf16(qb), ws=ws)
+    L.append_decode(k2, k2, dev_bf16(qb), ws=ws, step_flags=flags)
     torch.cuda.synchronize()
     assert L.lens.cpu().tolist()[:-1] == [x + 1 for x in expect_len[:-1]]
+
+
+def test_early_prefetch_layer_loop_matches_plain():
+    """A loop of fused steps over layers that share one workspace, launched
+    with STEP_EARLY (each layer's caches streamed before the previous layer's
+    kernel has ended), gives the same outputs, lengths and packed caches bit
+    for bit as the same loop without it."""
+    rng = np.random.default_rng(77)
+    n_kv, G, cap, n_layers, n_steps = 2, 8, 704, 3, 4
+    starts = [300, 31, 640]
+    cfg = kvq.make_cfg(n_kv, 3, 2, v_seed=12)
+    sets = []
+    for _ in range(2):
+        layers = [PackedLayer(cfg, len(starts), cap, layer=li) for li in range(n_layers)]
+        sets.append((layers, layers[0].workspace(n_kv * G, cap)))
+    for li in range(n_layers):
+        E, _, _ = _random_layer(rng, n_kv, 1, 1.2)
+        plans = kvq.plan_build(cfg, li, E)
+        for s, T0 in enumerate(starts):
+            _, kb, vb = _random_layer(rng, n_kv, T0, 1.2)
+            for layers, _ in sets:
+                L = layers[li]
+                L.set_plans(plans)
+                kvq.quantize_append(cfg, L.plan_ptrs[s:s + 1], dev_bf16(kb)[None],
+                                    dev_bf16(vb)[None], L.cache_ptrs[s:s + 1],
+                                    L.lens[s:s + 1], cap, L.status)
+    torch.cuda.synchronize()
+    shape = (len(starts), 1, n_kv, 128)
+    for step in range(n_steps):
+        ks = [dev_bf16(synth.to_bf16_bits(rng.standard_normal(shape))) for _ in range(n_layers)]
+        vs = [dev_bf16(synth.to_bf16_bits(rng.standard_normal(shape))) for _ in range(n_layers)]
+        qs = [dev_bf16(synth.to_bf16_bits(rng.standard_normal((len(starts), n_kv * G, 128))))
+              for _ in range(n_layers)]
+        outs = []
+        for (layers, ws), flags in zip(sets, (0, kvq.STEP_EARLY)):
+            o = [layers[li].append_decode(ks[li], vs[li], qs[li], ws=ws, step_flags=flags)
+                 for li in range(n_layers)]
+            outs.append(o)
+        torch.cuda.synchronize()
+        for li in range(n_layers):
+            assert torch.equal(outs[0][li], outs[1][li]), (step, li)
+            assert bool(torch.isfinite(outs[1][li]).all())
+    for li in range(n_layers):
+        a, b = sets[0][0][li], sets[1][0][li]
+        assert a.lens.cpu().tolist() == [T0 + n_steps for T0 in starts]
+        assert torch.equal(a.lens, b.lens)
+        for s in range(len(starts)):
+            assert torch.equal(a.caches[s], b.caches[s]), (li, s)
+        assert a.flags() == 0 and b.flags() == 0
