@@ -322,6 +322,8 @@ int kvq_decode_attn(const kvq_cfg* cfg, const void* const* plans_dev, const void
   if (max_len < 1 || max_len > 0x7FFFFFFF) return fail(KVQ_ERR_ARG, "max_len %lld", (long long)max_len);
   if (n_q_heads < 1 || n_q_heads % cfg->n_kv_heads != 0 || n_q_heads / cfg->n_kv_heads > 16)
     return fail(KVQ_ERR_ARG, "n_q_heads %d vs n_kv_heads %d", n_q_heads, cfg->n_kv_heads);
+  if (reinterpret_cast<uintptr_t>(ws_dev) & 15)
+    return fail(KVQ_ERR_ARG, "decode workspace not 16-byte aligned");
   if (ws_bytes < kvq_decode_workspace_bytes(cfg, batch, n_q_heads, max_len))
     return fail(KVQ_ERR_WORKSPACE, "decode workspace %zu < %zu", ws_bytes,
                 kvq_decode_workspace_bytes(cfg, batch, n_q_heads, max_len));
@@ -355,6 +357,8 @@ int kvq_append_decode(const kvq_cfg* cfg, const void* const* plans_dev, const vo
                 (long long)cap_tokens);
   if (n_q_heads < 1 || n_q_heads % cfg->n_kv_heads != 0 || n_q_heads / cfg->n_kv_heads > 16)
     return fail(KVQ_ERR_ARG, "n_q_heads %d vs n_kv_heads %d", n_q_heads, cfg->n_kv_heads);
+  if (reinterpret_cast<uintptr_t>(ws_dev) & 15)
+    return fail(KVQ_ERR_ARG, "decode workspace not 16-byte aligned");
   if (ws_bytes < kvq_decode_workspace_bytes(cfg, batch, n_q_heads, max_len))
     return fail(KVQ_ERR_WORKSPACE, "decode workspace %zu < %zu", ws_bytes,
                 kvq_decode_workspace_bytes(cfg, batch, n_q_heads, max_len));

@@ -31,10 +31,12 @@
 //   operand with movmatrix; O^T(128 x G) += Vhat^T(128 x 16 tokens) P'^T with
 //   A registers holding one rotated coordinate of two tokens.
 // * Merge: the 8 warps merge in shared memory; the last CTA of each group of
-//   8 splits merges the group; the last group merges the groups, undoes the
+//   16 splits merges the group; the last group merges the groups, undoes the
 //   value rotation (inverse Walsh-Hadamard, signs) and writes o / l.
-//   Arrivals are counted on workspace counters that the last arriver resets.
+//   Arrivals are counted on workspace counters (acquire-release atomics)
+//   that wrap to zero at the last arrival.
 #include <algorithm>
+#include <cstddef>
 #include <atomic>
 
 #include "quant_dev.cuh"
@@ -43,7 +45,8 @@ namespace kvq {
 
 // Lookup image (generated with the codebooks): byte offsets of its tables.
 __device__ __align__(16) const uint32_t g_lut_image[KVQ_LUT_BYTES / 4] = KVQ_LUT_IMAGE;
-__device__ const float g_thr[KVQ_CB_N_THR] = KVQ_CB_THR;
+constexpr int kThrPad = (KVQ_CB_N_THR + 3) & ~3;  // thresholds, padded to 16 bytes
+__device__ __align__(16) const float g_thr[kThrPad] = KVQ_CB_THR;
 __host__ __device__ constexpr uint32_t lut_rep(int w) {  // widths 1..3, lane-replicated
   return w == 1 ? 0x4000u : w == 2 ? 0x2000u : 0x0000u;
 }
@@ -53,13 +56,15 @@ constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kStages = 2;
 constexpr int kMaxHalf = 24;  // half steps of <= 4 blocks (<= 64/4 + 8)
-constexpr int kPartStride = 130;
-constexpr int kGroup = 8;     // splits merged per first-level group
+constexpr int kPartStride = 132;  // split record: m, l, 2 unused, o[128]
+constexpr int kRecO = 4;          // o at float 4 (16-byte aligned)
+constexpr int kGroup = 16;    // splits merged per first-level group
+constexpr int kMergeChunk = 16;  // records whose loads a merge issues together
 constexpr int kMaxSplits = 1024;
 constexpr int kCntStride = 2 + kMaxSplits / kGroup;  // per (sequence, KV head); last = sequence
 constexpr int kFallbackSlots = 1024;                  // CTA slots when no device answers
 constexpr int kMaxNew = 64;                           // tokens appended by a fused call
-constexpr int kScratch = 8192;                        // q' staging / append codes
+constexpr int kScratch = 8192 + 128;                  // q' staging / append codes + norms
 
 struct DecodeParams {
   const Plan* const* plans;
@@ -78,8 +83,8 @@ struct DecodeParams {
   int64_t cap;
   int early;  // read lengths and stream tiles before waiting for the previous kernel
   unsigned int* cnt_end;  // counters of pair k at cnt_end - (k + 1) * kCntStride
-  float* part;            // [batch][n_kv][n_splits][G][130] = m, l, o[128]
-  float* gpart;           // [batch][n_kv][n_groups][G][130]
+  float* part;            // [batch][n_kv][n_splits][G][132] = m, l, -, -, o[128]
+  float* gpart;           // [batch][n_kv][n_groups][G][132]
   float* out;             // [batch][n_q][128]
   uint32_t* status;
 };
@@ -92,9 +97,16 @@ struct alignas(128) Smem {
   unsigned long long bar[kWarps][kStages];
   unsigned long long setup_bar;
   uint32_t cls_lane[8][32];      // per (class, lane): first K word << 8 | bit shift
+  alignas(16) float thr[kThrPad];  // decision thresholds (fused append only)
+  int8_t qj[kMaxHalf][4];        // per half step: block of MMA column c, or -1
   int len0, is_last;
   uint32_t flags;
 };
+
+// Bulk-copy destinations start on 16-byte boundaries.
+static_assert(offsetof(Smem, plan) % 16 == 0 && offsetof(Smem, lut) % 16 == 0 &&
+                  offsetof(Smem, thr) % 16 == 0 && sizeof(Smem) % 128 == 0,
+              "shared-memory layout");
 
 // Loads from shared memory through pointers into the dynamic shared window,
 // so constant table offsets fold into the load instruction.
@@ -112,6 +124,25 @@ __device__ __forceinline__ float ex2(float x) {
 }
 __device__ __forceinline__ void grid_dep_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Arrival on a counter that wraps to zero after n arrivals, by one thread of
+// a CTA after a CTA barrier; true for the last arriver. The atomic is
+// acquire-release at GPU scope: the CTA's earlier writes (ordered before it
+// by the barrier) are visible to the last arriver, whose CTA reads after a
+// barrier that follows see the writes of every arriver.
+__device__ __forceinline__ bool arrive_last(unsigned int* c, unsigned int n) {
+  unsigned int old;
+  asm volatile("atom.acq_rel.gpu.global.inc.u32 %0, [%1], %2;"
+               : "=r"(old)
+               : "l"(c), "r"(n - 1u)
+               : "memory");
+  return old == n - 1u;
+}
+
+// L2 prefetch (a hint: no value is read, so it may precede the wait for the
+// kernel that writes the line).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 __device__ __forceinline__ void grid_dep_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -272,46 +303,53 @@ __device__ __forceinline__ void warp_unrotate_store(const float* src, const Plan
 }
 
 // Merge n records per head (record s of head h at src + s * rec_stride +
-// h * 130) into dst (record h at dst + h * 130), for G heads. One pass with
-// online rescaling over chunks of 8 records whose loads are issued together,
-// so a merge costs about n / 8 load round trips. Threads: 128 coordinates x
-// 2 heads at a time.
+// h * kPartStride) into dst (record h at dst + h * kPartStride), for G heads.
+// 32 threads per head, 4 coordinates each: one pass with online rescaling
+// over chunks of 16 records whose loads are issued together, so a merge of
+// all heads costs about n / 16 load round trips.
 __device__ __forceinline__ void merge_records(const float* src, int n, size_t rec_stride, int G,
                                               float* dst) {
-  const int tid = threadIdx.x;
-  for (int head = tid >> 7; head < G; head += kThreads / 128) {
-    const int x = tid & 127;
+  for (int item = threadIdx.x; item < G * 32; item += kThreads) {
+    const int head = item >> 5, x4 = (item & 31) * 4;
     const float* r = src + (size_t)head * kPartStride;
-    float M = -INFINITY, L = 0.f, O = 0.f;
-    for (int s0 = 0; s0 < n; s0 += 8) {
-      float mm[8], ll[8], oo[8];
+    float M = -INFINITY, L = 0.f;
+    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < n; s0 += kMergeChunk) {
+      float2 ml[kMergeChunk];
+      float4 oo[kMergeChunk];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
+      for (int k = 0; k < kMergeChunk; ++k) {
         const bool v = s0 + k < n;
         const float* q = r + (size_t)(v ? s0 + k : 0) * rec_stride;
-        mm[k] = v ? q[0] : -INFINITY;
-        ll[k] = v ? q[1] : 0.f;
-        oo[k] = v ? q[2 + x] : 0.f;
+        ml[k] = *reinterpret_cast<const float2*>(q);
+        oo[k] = *reinterpret_cast<const float4*>(q + kRecO + x4);
+        if (!v) ml[k].x = -INFINITY;
       }
       float cm = M;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) cm = fmaxf(cm, mm[k]);
+      for (int k = 0; k < kMergeChunk; ++k) cm = fmaxf(cm, ml[k].x);
       if (cm != -INFINITY) {
         const float a = ex2(M - cm);
         L *= a;
-        O *= a;
+        O.x *= a;
+        O.y *= a;
+        O.z *= a;
+        O.w *= a;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const float w = ex2(mm[k] - cm);
-          L += w * ll[k];
-          O += w * oo[k];
+        for (int k = 0; k < kMergeChunk; ++k) {
+          const float w = ex2(ml[k].x - cm);  // 0 for records past n
+          L += w * ml[k].y;
+          O.x += w * oo[k].x;
+          O.y += w * oo[k].y;
+          O.z += w * oo[k].z;
+          O.w += w * oo[k].w;
         }
         M = cm;
       }
     }
     float* d = dst + (size_t)head * kPartStride;
-    d[2 + x] = O;
-    if (x == 0) {
+    *reinterpret_cast<float4*>(d + kRecO + x4) = O;
+    if (x4 == 0) {
       d[0] = M;
       d[1] = L;
     }
@@ -337,10 +375,20 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
     mbar_init(&sm.setup_bar, 1);
     for (int i = 0; i < kWarps * kStages; ++i) mbar_init(&sm.bar[i / kStages][i % kStages], 1);
     fence_proxy_async();
-    mbar_expect_tx(&sm.setup_bar, KVQ_PLAN_BYTES + KVQ_LUT_BYTES);
+    const uint32_t thr_bytes = p.n_new > 0 ? (uint32_t)sizeof(g_thr) : 0u;
+    mbar_expect_tx(&sm.setup_bar, KVQ_PLAN_BYTES + KVQ_LUT_BYTES + thr_bytes);
     bulk_g2s(&sm.plan, p.plans[b] + h, KVQ_PLAN_BYTES, &sm.setup_bar);
     bulk_g2s(sm.lut, g_lut_image, KVQ_LUT_BYTES, &sm.setup_bar);
+    if (thr_bytes) bulk_g2s(sm.thr, g_thr, thr_bytes, &sm.setup_bar);
     sm.flags = 0u;
+  }
+  {  // this CTA's query rows into L2 while the previous kernel finishes
+    const size_t esz = (p.q_dtype == KVQ_BF16 || p.q_dtype == KVQ_FP16) ? 2 : 4;
+    const uintptr_t q0 =
+        reinterpret_cast<uintptr_t>(p.q) + ((size_t)b * p.n_q + (size_t)h * G) * kHeadDim * esz;
+    const uintptr_t q1 = q0 + (size_t)G * kHeadDim * esz;
+    for (uintptr_t a = (q0 & ~(uintptr_t)127) + (uintptr_t)tid * 128; a < q1; a += kThreads * 128)
+      prefetch_l2(reinterpret_cast<const void*>(a < q0 ? q0 : a));
   }
   // ---- with `early` the caller guarantees that the previous kernel on the
   //      stream writes neither these caches nor these lengths: the length is
@@ -392,11 +440,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   const int te = min(n_tiles, tb + p.tiles_per_split);
   const bool has_work = tb < te;
 
-  // ---- start streaming the warp's first tiles (tiles the append writes wait)
+  // ---- start streaming the warp's first tiles. Warp w takes tiles
+  //      te - 1 - w - 8 i, so the tiles a fused append writes (the last tiles
+  //      of the sequence) are the first tiles of warps 0..2.
   const int tbytes = p.tile_bytes;
   uint8_t* const my_stages = stage_base + (size_t)warp * kStages * tbytes;
   const int n_mine = has_work ? max(0, (te - tb - warp + kWarps - 1) / kWarps) : 0;
-  auto tile_of = [&](int i) { return tb + warp + i * kWarps; };
+  auto tile_of = [&](int i) { return te - 1 - warp - i * kWarps; };
   auto issue = [&](int i) {
     const int s = i % kStages;
     unsigned long long* bar = &sm.bar[warp][s];
@@ -404,50 +454,88 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
     bulk_g2s(my_stages + s * tbytes, cache + ((size_t)tile_of(i) * p.n_kv + h) * tbytes,
              (uint32_t)tbytes, bar);
   };
-  const int t_app = n_add > 0 ? len0 / kTile : 0x7FFFFFFF;
   if (lane == 0)
-    for (int i = 0; i < min(kStages, n_mine); ++i)
-      if (tile_of(i) < t_app) issue(i);
+    for (int i = 0; i < min(kStages, n_mine); ++i) issue(i);
+  // appended tiles of this CTA: [a_lo, a_hi] (CTA-uniform)
+  const int a_lo = n_add > 0 ? max(len0 / kTile, tb) : 1;
+  const int a_hi = n_add > 0 ? min((len0 + n_add - 1) / kTile, te - 1) : 0;
+  const bool appends = has_work && a_lo <= a_hi;
+  if (appends) {  // the new tokens' rows into L2 (no value read before the wait)
+    const size_t esz = (p.kv_dtype == KVQ_BF16 || p.kv_dtype == KVQ_FP16) ? 2 : 4;
+    const int lines = (int)(kHeadDim * esz / 128);
+    const int j0 = max(len0, a_lo * kTile) - len0, j1 = min(len0 + n_add, a_hi * kTile + kTile) - len0;
+    for (int e = tid; e < (j1 - j0) * lines * 2; e += kThreads) {
+      const int j = j0 + e / (2 * lines), l = e % lines;
+      const void* src = (e / lines) % 2 ? p.v_new : p.k_new;
+      prefetch_l2(reinterpret_cast<const uint8_t*>(src) +
+                  ((((size_t)b * p.n_new + j) * p.n_kv + h) * kHeadDim) * esz + (size_t)l * 128);
+    }
+  }
+  // plan-only part of the query prologue: MMA column -> RoPE block per half
+  // step, and each width class's first word and bit shift per lane
+  if (!bad) {
+    for (int e = tid; e < n_half * 4; e += kThreads) {
+      const int hs = e >> 2, cc = e & 3;
+      sm.qj[hs][cc] = cc < sm.plan.hs_count[hs]
+                          ? (int8_t)sm.plan.order[sm.plan.hs_rank0[hs] + cc] : (int8_t)-1;
+    }
+    for (int e = tid; e < sm.plan.n_class * 32; e += kThreads) {
+      const int ci = e >> 5, ln = e & 31, W = sm.plan.cls_w[ci];
+      const int off = sm.plan.cls_seg0[ci] + 2 * W * (ln & 3) + ((W * (ln >> 2)) >> 2);
+      sm.cls_lane[ci][ln] = ((uint32_t)off << 8) | ((uint32_t)(8 * W * (ln >> 2)) & 31u);
+    }
+  }
   if (p.early) grid_dep_wait();
   grid_dep_launch();
 
-  // ---- fused append: quantize and pack the new tokens whose tiles are ours
-  if (has_work && n_add > 0) {
-    const int t_first = len0 / kTile, t_last = (len0 + n_add - 1) / kTile;
+  // ---- fused append: quantize the new tokens of the appended tiles, then
+  //      patch them into the streamed copy of each tile (stage 0 of warp
+  //      te - 1 - tile) and into the cache
+  if (appends) {
     uint8_t (*kc)[kHeadDim] = reinterpret_cast<uint8_t (*)[kHeadDim]>(scratch);
     uint8_t (*vc)[kHeadDim] = reinterpret_cast<uint8_t (*)[kHeadDim]>(scratch + 32 * kHeadDim);
+    __half* nrm_new = reinterpret_cast<__half*>(scratch + 64 * kHeadDim);  // [2][32]
     uint32_t flags = 0;
-    for (int tile = max(t_first, tb); tile <= min(t_last, te - 1); ++tile) {
+    for (int tile = a_lo; tile <= a_hi; ++tile) {
       const int t_lo = max(len0, tile * kTile), t_hi = min(len0 + n_add, tile * kTile + kTile);
-      uint8_t* rec = const_cast<uint8_t*>(cache) + ((size_t)tile * p.n_kv + h) * p.tile_bytes;
+      const int w_own = te - 1 - tile;
+      uint8_t* rec = const_cast<uint8_t*>(cache) + ((size_t)tile * p.n_kv + h) * tbytes;
+      uint8_t* st = stage_base + (size_t)w_own * kStages * tbytes;
       for (int t = t_lo + warp; t < t_hi; t += kWarps) {
         const int tt = t - tile * kTile;
         const size_t row = (((size_t)b * p.n_new + (t - len0)) * p.n_kv + h) * kHeadDim;
         __half kn, vn;
-        warp_token_codes(sm.plan, g_thr, p.k_new, p.v_new, p.kv_dtype, row, lane, kc[tt], vc[tt],
+        warp_token_codes(sm.plan, sm.thr, p.k_new, p.v_new, p.kv_dtype, row, lane, kc[tt], vc[tt],
                          kn, vn, flags);
         if (lane == 0) {
-          __half* norms = reinterpret_cast<__half*>(rec + 512 * (bk + BV));
-          norms[tt] = kn;
-          norms[kTile + tt] = vn;
+          nrm_new[tt] = kn;
+          nrm_new[kTile + tt] = vn;
         }
       }
+      const bool ok = mbar_wait_bounded(&sm.bar[w_own][0], 0u);  // the old tile is in `st`
       __syncthreads();
-      assemble_tile_words(reinterpret_cast<uint32_t*>(rec), sm.plan, kc, vc,
-                          max(0, len0 - tile * kTile), t_lo - tile * kTile, t_hi - tile * kTile,
-                          tid, kThreads);
+      if (ok) {
+        assemble_tile_words(reinterpret_cast<uint32_t*>(rec), reinterpret_cast<uint32_t*>(st),
+                            reinterpret_cast<uint32_t*>(st), sm.plan, kc, vc,
+                            max(0, len0 - tile * kTile), t_lo - tile * kTile, t_hi - tile * kTile,
+                            tid, kThreads);
+        for (int t = t_lo + tid; t < t_hi; t += kThreads) {
+          const int tt = t - tile * kTile;
+          for (int e = 0; e < 2; ++e) {
+            reinterpret_cast<__half*>(rec + 512 * (bk + BV))[e * kTile + tt] = nrm_new[e * kTile + tt];
+            reinterpret_cast<__half*>(st + 512 * (bk + BV))[e * kTile + tt] = nrm_new[e * kTile + tt];
+          }
+        }
+      } else {
+        flags |= KVQ_FLAG_TIMEOUT;
+      }
       __syncthreads();
     }
     if (flags) atomicOr(&sm.flags, flags);
-    // the bulk copies below must see these writes
-    __threadfence();
-    asm volatile("fence.proxy.async.global;" ::: "memory");
+    fence_proxy_async();  // patched stages are later overwritten by bulk copies
     __syncthreads();
     if (tid == 0 && sm.flags) atomicOr(p.status, sm.flags);
   }
-  if (lane == 0)
-    for (int i = 0; i < min(kStages, n_mine); ++i)
-      if (tile_of(i) >= t_app) issue(i);
 
   float o[8][NT][4];
   float m_run[NT][2], l_run[NT][2];
@@ -469,35 +557,33 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
     // ---- query prologue (q' staged in the tile ring before it is used):
     //      q' = q a_hat_j log2(e) / sqrt(128); per-head 2^sigma scaling into
     //      the fp16 range; hi/lo split into the B fragments of each half step
-    float* qp = reinterpret_cast<float*>(scratch);  // [16][128]
-#pragma unroll
-    for (int i = tid; i < 16 * kHeadDim; i += kThreads) {
-      const int head = i >> 7, x = i & 127;
-      float v = 0.f;
-      if (head < G) {
-        const size_t qi = ((size_t)b * p.n_q + h * G + head) * kHeadDim + x;
-        v = load_as_float(p.q, p.q_dtype, qi) * sm.plan.a_hat[x & 63] * 0.12751743074f;
-      }
-      qp[i] = v;  // 0.12751743 = log2(e) / sqrt(128)
-    }
-    __syncthreads();
+    float* qp = reinterpret_cast<float*>(scratch);  // [8 NT][128]
     for (int head = warp; head < 8 * NT; head += kWarps) {
-      float mx = 0.f;
-      for (int x = lane; x < kHeadDim; x += 32) mx = fmaxf(mx, fabsf(qp[head * kHeadDim + x]));
+      float v[4], mx = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int x = lane + 32 * i;
+        v[i] = 0.f;
+        if (head < G) {
+          const size_t qi = ((size_t)b * p.n_q + h * G + head) * kHeadDim + x;
+          v[i] = load_as_float(p.q, p.q_dtype, qi) * sm.plan.a_hat[x & 63] * 0.12751743074f;
+        }  // 0.12751743 = log2(e) / sqrt(128)
+        mx = fmaxf(mx, fabsf(v[i]));
+      }
 #pragma unroll
       for (int m = 16; m; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
       const int sigma = (mx > 0.f && isfinite(mx)) ? 14 - ilogbf(mx) : 0;
       const float sc = ldexpf(1.f, sigma);
-      for (int x = lane; x < kHeadDim; x += 32) qp[head * kHeadDim + x] *= sc;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) qp[head * kHeadDim + lane + 32 * i] = v[i] * sc;
       if (lane == 0) sm.inv_scale[head] = ldexpf(1.f, -sigma);
     }
     __syncthreads();
     for (int e = tid; e < NT * n_half * 32; e += kThreads) {
       const int ln = e & 31, hs = (e >> 5) % n_half, nt = (e >> 5) / n_half;
-      const int head = 8 * nt + (ln >> 2), cc = ln & 3;
+      const int head = 8 * nt + (ln >> 2), j = sm.qj[hs][ln & 3];
       float x0 = 0.f, x1 = 0.f;
-      if (cc < sm.plan.hs_count[hs]) {
-        const int j = sm.plan.order[sm.plan.hs_rank0[hs] + cc];
+      if (j >= 0) {
         x0 = qp[head * kHeadDim + j];
         x1 = qp[head * kHeadDim + j + 64];
       }
@@ -505,11 +591,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
       const __half2 hh = *reinterpret_cast<const __half2*>(&hi);
       const uint32_t lo = pack_half2(x0 - __low2float(hh), x1 - __high2float(hh));
       sm.qfrag[nt][hs][ln] = make_uint2(hi, lo);
-    }
-    for (int e = tid; e < sm.plan.n_class * 32; e += kThreads) {
-      const int ci = e >> 5, ln = e & 31, W = sm.plan.cls_w[ci];
-      const int off = sm.plan.cls_seg0[ci] + 2 * W * (ln & 3) + ((W * (ln >> 2)) >> 2);
-      sm.cls_lane[ci][ln] = ((uint32_t)off << 8) | ((uint32_t)(8 * W * (ln >> 2)) & 31u);
     }
     __syncthreads();
 
@@ -642,7 +723,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
       l_run[nt][e] = l;
     }
   __syncthreads();
-  float* mg = reinterpret_cast<float*>(stage_base);  // [warp][8 NT heads][130]
+  float* mg = reinterpret_cast<float*>(stage_base);  // [warp][8 NT heads][132]
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -654,8 +735,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
       }
 #pragma unroll
       for (int mu = 0; mu < 8; ++mu) {
-        dst[2 + 16 * mu + g] = o[mu][nt][e];
-        dst[2 + 16 * mu + g + 8] = o[mu][nt][2 + e];
+        dst[kRecO + 16 * mu + g] = o[mu][nt][e];
+        dst[kRecO + 16 * mu + g + 8] = o[mu][nt][2 + e];
       }
     }
   __syncthreads();
@@ -665,39 +746,27 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   // ---- level 1: the last CTA of this group of splits merges the group
   const int grp = split / kGroup;
   const int g_lo = grp * kGroup, g_n = min(kGroup, p.n_splits - g_lo);
-  __threadfence();
   __syncthreads();
-  if (tid == 0) {
-    const unsigned int prev = atomicAdd(&cnt[1 + grp], 1u);
-    sm.is_last = prev == (unsigned int)(g_n - 1);
-    if (sm.is_last) cnt[1 + grp] = 0u;
-  }
+  if (tid == 0) sm.is_last = arrive_last(&cnt[1 + grp], (unsigned int)g_n);
   __syncthreads();
   if (!sm.is_last) return;
-  __threadfence();
   float* my_gpart = p.gpart + (bh * p.n_groups + grp) * G * kPartStride;
   merge_records(p.part + (bh * p.n_splits + g_lo) * G * kPartStride, g_n,
                 (size_t)G * kPartStride, G, my_gpart);
 
   // ---- level 2: the last group merges the groups and writes o / l
-  __threadfence();
   __syncthreads();
-  if (tid == 0) {
-    const unsigned int prev = atomicAdd(&cnt[0], 1u);
-    sm.is_last = prev == (unsigned int)(p.n_groups - 1);
-    if (sm.is_last) cnt[0] = 0u;
-  }
+  if (tid == 0) sm.is_last = arrive_last(&cnt[0], (unsigned int)p.n_groups);
   __syncthreads();
   if (!sm.is_last) return;
-  __threadfence();
-  float* fin = reinterpret_cast<float*>(stage_base);  // [16][130]
+  float* fin = reinterpret_cast<float*>(stage_base);  // [16][132]
   merge_records(p.gpart + bh * p.n_groups * G * kPartStride, p.n_groups, (size_t)G * kPartStride,
                 G, fin);
   __syncthreads();
   for (int head = warp; head < G; head += kWarps) {
     const float* r = fin + (size_t)head * kPartStride;
     const float inv = r[1] > 0.f ? 1.f / (128.f * r[1]) : 0.f;
-    warp_unrotate_store(r + 2, sm.plan, inv,
+    warp_unrotate_store(r + kRecO, sm.plan, inv,
                         p.out + ((size_t)b * p.n_q + h * G + head) * kHeadDim, lane);
   }
 }

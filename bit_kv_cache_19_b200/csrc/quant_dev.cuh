@@ -119,12 +119,16 @@ __device__ __forceinline__ void warp_token_codes(const Plan& pl, const float* th
   }
 }
 
-// Packed words of one tile record. Positions [0, old_n) hold older tokens
-// whose bits are kept; positions [new_lo, new_hi) get the codes in kc / vc
-// (rows indexed by position); all other positions are zero. When the tile
-// already holds tokens (old_n > 0) only words that carry bits of new
-// positions are rewritten. Threads tid, tid + nth, ... take one word each.
-__device__ __forceinline__ void assemble_tile_words(uint32_t* words, const Plan& pl,
+// Packed words of one tile record into `words` (and `copy`, if not null).
+// Positions [0, old_n) hold older tokens whose bits are kept from `old`;
+// positions [new_lo, new_hi) get the codes in kc / vc (rows indexed by
+// position); all other positions are zero. When the tile already holds
+// tokens (old_n > 0) only words that carry bits of new positions are
+// rewritten. Threads tid, tid + nth, ... take one word each (a word is read
+// from `old` and written by the same thread, so `old` may alias either
+// destination).
+__device__ __forceinline__ void assemble_tile_words(uint32_t* words, const uint32_t* old,
+                                                    uint32_t* copy, const Plan& pl,
                                                     const uint8_t (*kc)[kHeadDim],
                                                     const uint8_t (*vc)[kHeadDim], int old_n,
                                                     int new_lo, int new_hi, int tid, int nth) {
@@ -164,10 +168,10 @@ __device__ __forceinline__ void assemble_tile_words(uint32_t* words, const Plan&
         keep |= (uint32_t)(((unsigned long long)field << fb) >> 32);
       }
     }
-    if (old_n == 0) {
-      words[wi] = nw;
-    } else if (touched) {
-      words[wi] = (words[wi] & keep) | nw;
+    if (old_n == 0 || touched) {
+      const uint32_t w = old_n == 0 ? nw : (old[wi] & keep) | nw;
+      words[wi] = w;
+      if (copy) copy[wi] = w;
     }
   }
 }

@@ -128,7 +128,8 @@ __global__ void __launch_bounds__(256) quantize_append_kernel(QuantParams p) {
   // ---- assemble segment words: keep older tokens' bits, write the new ones,
   //      zero positions past the new length
   const int old_n = max(0, len0 - tile * kTile);  // positions holding older tokens
-  assemble_tile_words(reinterpret_cast<uint32_t*>(rec), pl, s_kc, s_vc, old_n,
+  assemble_tile_words(reinterpret_cast<uint32_t*>(rec), reinterpret_cast<const uint32_t*>(rec),
+                      nullptr, pl, s_kc, s_vc, old_n,
                       t_lo - tile * kTile, t_hi - tile * kTile, threadIdx.x, blockDim.x);
   if (threadIdx.x == 0 && s_flags) atomicOr(p.status, s_flags);
 }

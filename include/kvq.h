@@ -262,7 +262,8 @@ KVQ_API int kvq_quantize_append(const kvq_cfg* cfg, const void* const* plans_dev
  * q_dev: [batch][n_q_heads][128] of type q_dtype (post-RoPE queries).
  * out_dev: fp32 [batch][n_q_heads][128].
  * ws_dev: >= kvq_decode_workspace_bytes(cfg, batch, n_q_heads, max_len)
- *        bytes, zero-filled once before its first use. Every completed call
+ *        bytes, 16-byte aligned, zero-filled once before its first use
+ *        (KVQ_ERR_ARG if misaligned). Every completed call
  *        leaves the arrival counters it keeps at the end of the workspace at
  *        zero, so one workspace can serve any sequence of calls with the same
  *        n_kv_heads (and shapes that fit) on one stream; calls that overlap
@@ -297,7 +298,8 @@ KVQ_API int kvq_decode_attn(const kvq_cfg* cfg, const void* const* plans_dev,
  *                   nor these lengths (e.g. in a loop over layers, where the
  *                   previous kernel is another layer's step, which may share
  *                   the workspace); q, k_dev, v_dev, out and the rest of the
- *                   workspace are always accessed after it.
+ *                   workspace are always read and written after it (q is
+ *                   only prefetched into L2 before it, which reads no value).
  * Returns KVQ_OK or a negative code.
  */
 KVQ_API int kvq_append_decode(const kvq_cfg* cfg, const void* const* plans_dev, const void* k_dev,

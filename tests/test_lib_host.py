@@ -127,6 +127,16 @@ def test_argument_errors_without_gpu():
                              None) == kvq.ERR_ARG
     assert L.kvq_decode_attn(ctypes.byref(cfg), p, p, p, 1, 10, p, 0, 16, p, p, 8, p,
                              None) == kvq.ERR_WORKSPACE
+    # a workspace off a 16-byte boundary, and unknown step flags
+    p8 = ctypes.c_void_p(24)
+    assert L.kvq_decode_attn(ctypes.byref(cfg), p, p, p, 1, 10, p, 0, 16, p, p8, 1 << 30, p,
+                             None) == kvq.ERR_ARG
+    assert b"aligned" in L.kvq_last_error()
+    assert L.kvq_append_decode(ctypes.byref(cfg), p, p, p, 0, 1, p, p, 10, 1, 10, p, 0, 16, p,
+                               p8, 1 << 30, 0, p, None) == kvq.ERR_ARG
+    assert L.kvq_append_decode(ctypes.byref(cfg), p, p, p, 0, 1, p, p, 10, 1, 10, p, 0, 16, p,
+                               p, 1 << 30, 2, p, None) == kvq.ERR_ARG
+    assert b"step_flags" in L.kvq_last_error()
     assert L.kvq_quantize_append(ctypes.byref(cfg), p, p, p, 7, 1, 1, p, p, 10, p,
                                  None) == kvq.ERR_ARG
     # zero new tokens is a no-op
