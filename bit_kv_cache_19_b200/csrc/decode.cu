@@ -16,11 +16,14 @@
 //   programmatic dependent launch: everything up to griddepcontrol.wait does
 //   not depend on the previous kernel.
 // * Append (fused calls): the CTA that owns the tile of a new token
-//   quantizes and packs it before streaming; the last CTA of the sequence to
-//   read its length writes the new length.
-// * Keys: logits S[32 tokens x 8 heads] by mma.sync m16n8k8, one MMA per
-//   "half step" of the plan (<= 4 RoPE blocks of one width W). Each 32-bit A
-//   register is one block (codes of coordinates j and j + 64) of one token,
+//   quantizes it and patches it into the streamed copy of the tile (the
+//   first stage of one of its warps) and into the cache; the last CTA of the
+//   sequence to read its length writes the new length.
+// * Keys: logits S[32 tokens x 8 heads] by mma.sync m16n8k16, one MMA per
+//   m-tile and "half step" of the plan (<= 4 RoPE blocks of one width W),
+//   the A fragment repeated over k so that one MMA adds A q'_hi + A q'_lo
+//   (split below). Each 32-bit A register is one block (codes of
+//   coordinates j and j + 64) of one token,
 //   looked up as an fp16 pair; the packed layout puts the 4 tokens a lane
 //   needs (g, g + 8, g + 16, g + 24) in 8W contiguous bits. Half steps of one
 //   width form a class compiled for its W. B = the query group times a_hat_j,
@@ -188,15 +191,6 @@ __device__ __forceinline__ void fields4(const uint8_t* lut, const uint8_t* wp, u
   }
 }
 
-// D(16x8 f32) += A(16x8 f16, row) B(8x8 f16, col).
-__device__ __forceinline__ void mma_1688(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 "
-      "{%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(b0));
-}
-
 // Logits of one width class: its nhs half steps of <= 4 blocks of width W
 // (runtime, warp-uniform: one code path per lookup kind keeps the kernel
 // small). Lane (g, c) takes block c of every half step, tokens g, g + 8
@@ -208,11 +202,10 @@ __device__ __forceinline__ void key_mma(float (&s)[2][NT][4], const uint32_t (&A
                                         const uint2* qp) {
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
+    // k16 with the A fragment repeated: A q'_hi + A q'_lo in one MMA
     const uint2 b = qp[nt * kMaxHalf * 32];
-    mma_1688(s[0][nt], A[0], A[1], b.x);
-    mma_1688(s[0][nt], A[0], A[1], b.y);
-    mma_1688(s[1][nt], A[2], A[3], b.x);
-    mma_1688(s[1][nt], A[2], A[3], b.y);
+    mma_16816(s[0][nt], A[0], A[1], A[0], A[1], b.x, b.y);
+    mma_16816(s[1][nt], A[2], A[3], A[2], A[3], b.x, b.y);
   }
 }
 
@@ -231,6 +224,7 @@ __device__ __forceinline__ void key_class(const Smem& sm, const uint8_t* kw, int
   if (W <= 3) {
     const uint32_t m7 = ((1u << w2) - 1u) << 7;
     const uint32_t lb = lane4 | lut_rep(W);
+#pragma unroll 2
     for (int i = 0; i < nhs; ++i, wp += stride, qp += 32) {
       const uint32_t v7 = funnel_r(ld32s(wp), ld32s(wp + 4), sh) << 7;
       uint32_t A[4];
@@ -241,12 +235,14 @@ __device__ __forceinline__ void key_class(const Smem& sm, const uint8_t* kw, int
       key_mma<NT>(s, A, qp);
     }
   } else if (W == 4) {
+#pragma unroll 2
     for (int i = 0; i < nhs; ++i, wp += stride, qp += 32) {
       uint32_t A[4];
       fields4<4>(lut, wp, sh, lane4, A);
       key_mma<NT>(s, A, qp);
     }
   } else if (W == 5) {
+#pragma unroll 2
     for (int i = 0; i < nhs; ++i, wp += stride, qp += 32) {
       uint32_t A[4];
       fields4<5>(lut, wp, sh, lane4, A);
@@ -260,6 +256,7 @@ __device__ __forceinline__ void key_class(const Smem& sm, const uint8_t* kw, int
     const uint32_t mw = ((1u << W) - 1u) << 1;
     const uint32_t offb = 4u * ((sh + 4u * W) >> 5), shb = (sh + 4u * W) & 31u;
     const uint32_t s1 = (uint32_t)W - 1u, s2 = 2u * W - 1u, s3 = 3u * W - 1u;
+#pragma unroll 2
     for (int i = 0; i < nhs; ++i, wp += stride, qp += 32) {
       const uint32_t ua = funnel_r(ld32s(wp), ld32s(wp + 4), sh);
       const uint32_t ub = funnel_r(ld32s(wp + offb), ld32s(wp + offb + 4), shb);

@@ -61,7 +61,7 @@ typedef struct CUstream_st* kvq_stream_t;
 #define KVQ_FLAG_CAPACITY 1u   /* append past cap_tokens (sequence skipped), or len > max_len */
 #define KVQ_FLAG_NONFINITE 2u  /* a token had a NaN/Inf coordinate: stored as norm 0, codes 0 */
 #define KVQ_FLAG_NORM_SAT 4u   /* a norm overflowed fp16: stored as 65504 */
-#define KVQ_FLAG_TIMEOUT 8u    /* a bounded wait for a tile copy ran out: output invalid */
+#define KVQ_FLAG_TIMEOUT 8u    /* a bounded wait ran out: output invalid */
 #define KVQ_FLAG_BAD_PLAN 16u  /* a plan record failed its magic/shape check */
 
 /* Input element types. */
