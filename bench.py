@@ -250,13 +250,26 @@ def run_kvq(args, wl, rank, world, dist):
     torch.cuda.empty_cache()
 
     # ---- decode inputs (device resident) and static new-token buffers
-    qs = [synth.queries_torch(wl, args.seed, li, B, T, dev) for li in range(n_layers)]
-    knew = [torch.randn(B, 1, wl.n_kv_heads, 128, device=dev).to(torch.bfloat16)
-            for _ in range(n_layers)]
-    vnew = [torch.randn(B, 1, wl.n_kv_heads, 128, device=dev).to(torch.bfloat16)
-            for _ in range(n_layers)]
-    outs = [torch.empty(B, wl.n_q_heads, 128, dtype=torch.float32, device=dev)
-            for _ in range(n_layers)]
+    # the step's inputs (q, new k, new v of every layer) live in one device
+    # buffer and its outputs in another, so that an end-to-end step moves
+    # them with one host-to-device and one device-to-host copy
+    nq_el, nkv_el = B * wl.n_q_heads * 128, B * wl.n_kv_heads * 128
+    per_layer = nq_el + 2 * nkv_el
+    step_in = torch.empty(n_layers * per_layer, dtype=torch.bfloat16, device=dev)
+    step_out = torch.empty(n_layers, B, wl.n_q_heads, 128, dtype=torch.float32, device=dev)
+    qs, knew, vnew = [], [], []
+    for li in range(n_layers):
+        base = li * per_layer
+        q = step_in[base:base + nq_el].view(B, wl.n_q_heads, 128)
+        k = step_in[base + nq_el:base + nq_el + nkv_el].view(B, 1, wl.n_kv_heads, 128)
+        v = step_in[base + nq_el + nkv_el:base + per_layer].view(B, 1, wl.n_kv_heads, 128)
+        q.copy_(synth.queries_torch(wl, args.seed, li, B, T, dev))
+        k.copy_(torch.randn(B, 1, wl.n_kv_heads, 128, device=dev).to(torch.bfloat16))
+        v.copy_(torch.randn(B, 1, wl.n_kv_heads, 128, device=dev).to(torch.bfloat16))
+        qs.append(q)
+        knew.append(k)
+        vnew.append(v)
+    outs = [step_out[li] for li in range(n_layers)]
     ws = layers[0].workspace(wl.n_q_heads, cap)
 
     def step():
@@ -328,22 +341,15 @@ def run_kvq(args, wl, rank, world, dist):
     achieved = bytes_launch / (launch_ms / 1e3) / 1e9
 
     # ---- e2e: host buffers, H2D of the step's inputs and D2H of its outputs
-    q_host = [q.cpu().pin_memory() for q in qs]
-    k_host = [k.cpu().pin_memory() for k in knew]
-    v_host = [v.cpu().pin_memory() for v in vnew]
-    o_host = [torch.empty_like(o, device="cpu").pin_memory() for o in outs]
-    h2d = sum(q.numel() * q.element_size() + k.numel() * k.element_size() * 2
-              for q, k in zip(q_host, k_host))
-    d2h = sum(o.numel() * o.element_size() for o in o_host)
+    in_host = step_in.cpu().pin_memory()
+    out_host = torch.empty_like(step_out, device="cpu").pin_memory()
+    h2d = in_host.numel() * in_host.element_size()
+    d2h = out_host.numel() * out_host.element_size()
     with torch.cuda.stream(stream):
         def e2e_step():
-            for li in range(n_layers):
-                qs[li].copy_(q_host[li], non_blocking=True)
-                knew[li].copy_(k_host[li], non_blocking=True)
-                vnew[li].copy_(v_host[li], non_blocking=True)
+            step_in.copy_(in_host, non_blocking=True)
             graph.replay() if graph is not None else step()
-            for li in range(n_layers):
-                o_host[li].copy_(outs[li], non_blocking=True)
+            out_host.copy_(step_out, non_blocking=True)
         for _ in range(2):
             e2e_step()
         stream.synchronize()
