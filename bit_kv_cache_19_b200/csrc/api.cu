@@ -15,19 +15,7 @@
 namespace kvq {
 cudaError_t launch_energy(const void* k, int dtype, int64_t n_tokens, int n_kv,
                           unsigned long long* acc, uint32_t* status, cudaStream_t st);
-struct QuantParams {
-  const Plan* const* plans;
-  const void* k;
-  const void* v;
-  int dtype;
-  int batch, n_new, n_kv;
-  uint8_t* const* caches;
-  const int32_t* len;
-  int64_t cap;
-  int tile_bytes;
-  uint32_t* status;
-};
-cudaError_t launch_quantize_append(const QuantParams& p, cudaStream_t st);
+cudaError_t launch_quantize_append(const QuantParams& p, int bits_v, cudaStream_t st);
 size_t decode_workspace_bytes_for(int batch, int n_q, int n_kv, int bits_k, int bits_v,
                                   int64_t max_len);
 cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches, int32_t* len,
@@ -304,7 +292,7 @@ int kvq_quantize_append(const kvq_cfg* cfg, const void* const* plans_dev, const 
   p.cap = cap_tokens;
   p.tile_bytes = tile_bytes(cfg->bits_k, cfg->bits_v);
   p.status = status_dev;
-  cudaError_t e = launch_quantize_append(p, reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_quantize_append(p, cfg->bits_v, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "quantize_append");
   return KVQ_OK;
 }

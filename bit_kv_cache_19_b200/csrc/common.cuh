@@ -68,6 +68,21 @@ __host__ __device__ __forceinline__ int token_of_slot_v(int s) {
   return 8 * ((s & 7) >> 1) + 2 * (s >> 3) + (s & 1);
 }
 
+// Arguments of the quantize-append launch (host and device side).
+struct QuantParams {
+  const Plan* const* plans;  // [batch] -> [n_kv] plans
+  const void* k;
+  const void* v;
+  int dtype;
+  int batch, n_new, n_kv;
+  uint8_t* const* caches;  // [batch]
+  const int32_t* len;
+  int64_t cap;
+  int tile_bytes;
+  int tiles_max;  // work items per (sequence, KV head)
+  uint32_t* status;
+};
+
 // ------------------------------------------------------------------ device
 #ifdef __CUDACC__
 

@@ -176,4 +176,136 @@ __device__ __forceinline__ void assemble_tile_words(uint32_t* words, const uint3
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Tile quantizer in two passes (one CTA per tile record):
+//  1. one warp per new token: norms, kz[p][i] = k_i r (NaN for a token whose
+//     key codes are all zero), the value rotation and the value codes, which
+//     go straight into the packed words;
+//  2. one warp per stored key block, lane = position: z = kz * g_j and the
+//     codes of coordinates j and j + 64 with the block's width (uniform in
+//     the warp), packed as one 2W-bit field.
+// Fields enter the words by shared-memory atomics, so any number of warps
+// can write one word; with `clear` a field's old bits are cleared first.
+
+constexpr int kKzStride = kHeadDim + 1;  // padded rows: pass 2 reads a column
+
+// Branch-free: the word after the field's first word is always touched (an
+// OR of 0 / AND of all ones when the field does not reach it), so `words`
+// needs one word of slack past the packed words. nbits <= 16.
+__device__ __forceinline__ void put_field(uint32_t* words, int bit, uint32_t val, int nbits,
+                                          bool clear) {
+  const int wi = bit >> 5, off = bit & 31;
+  const uint32_t mask = (1u << nbits) - 1u;
+  // parts of the field in word wi and wi + 1 (64-bit shift: off may be 0)
+  const unsigned long long v2 = (unsigned long long)val << off;
+  const unsigned long long m2 = (unsigned long long)mask << off;
+  if (clear) {
+    atomicAnd(&words[wi], ~(uint32_t)m2);
+    atomicAnd(&words[wi + 1], ~(uint32_t)(m2 >> 32));
+  }
+  atomicOr(&words[wi], (uint32_t)v2);
+  atomicOr(&words[wi + 1], (uint32_t)(v2 >> 32));
+}
+
+// code_of for a compile-time width (all steps unrolled).
+template <int W>
+__device__ __forceinline__ int code_of_w(const float* thr, float z) {
+  const float* t = thr + cb_t_off(W);
+  int c = 0;
+#pragma unroll
+  for (int step = 1 << (W - 1); step; step >>= 1) c += (t[c + step - 1] < z) ? step : 0;
+  return c;
+}
+
+// Pass 1 for the token at tile position p (row: element offset of its key /
+// value in k / v), value width BV. Writes kz_row[128], the token's value
+// fields into `words` and returns the fp16 norms.
+template <int BV>
+__device__ __forceinline__ void warp_token_pass(const Plan& pl, const float* thr, const void* k,
+                                                const void* v, int dtype, size_t row, int lane,
+                                                int p, float* kz_row, uint32_t* words, bool clear,
+                                                __half& kn, __half& vn, uint32_t& flags) {
+  float kx[4], vx[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    kx[q] = load_as_float(k, dtype, row + lane + 32 * q);
+    vx[q] = load_as_float(v, dtype, row + lane + 32 * q);
+  }
+  const bool kfin = __all_sync(0xffffffffu, isfinite(kx[0]) && isfinite(kx[1]) &&
+                                                isfinite(kx[2]) && isfinite(kx[3]));
+  const bool vfin = __all_sync(0xffffffffu, isfinite(vx[0]) && isfinite(vx[1]) &&
+                                                isfinite(vx[2]) && isfinite(vx[3]));
+  float kr;
+  norm_and_recip(kx, kfin, kn, kr, flags);
+  const bool klive = kfin && __half2float(kn) > 0.f;
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    kz_row[lane + 32 * q] = klive ? __fmul_rn(kx[q], kr) : __int_as_float(0x7fc00000);
+  // values: y = H (s . v) by the fixed fp32 butterfly graph, z = y r
+  float vr;
+  norm_and_recip(vx, vfin, vn, vr, flags);
+  const bool vlive = vfin && __half2float(vn) > 0.f;
+  float y[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int i = lane + 32 * q;
+    const float x = vfin ? vx[q] : 0.f;
+    y[q] = ((pl.v_sign[i >> 5] >> (i & 31)) & 1u) ? -x : x;
+  }
+  // butterflies h = 1..16 across lanes: lower y + o, upper o - y, each one
+  // fma with a +-1 factor (exact product, one rounding: the same value)
+#pragma unroll
+  for (int hh = 1; hh < 32; hh <<= 1) {
+    const float sg = (lane & hh) ? -1.f : 1.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) y[q] = __fmaf_rn(y[q], sg, __shfl_xor_sync(0xffffffffu, y[q], hh));
+  }
+  {  // h = 32: (q0, q1), (q2, q3); h = 64: (q0, q2), (q1, q3)
+    const float a0 = __fadd_rn(y[0], y[1]), a1 = __fsub_rn(y[0], y[1]);
+    const float a2 = __fadd_rn(y[2], y[3]), a3 = __fsub_rn(y[2], y[3]);
+    y[0] = __fadd_rn(a0, a2);
+    y[2] = __fsub_rn(a0, a2);
+    y[1] = __fadd_rn(a1, a3);
+    y[3] = __fsub_rn(a1, a3);
+  }
+  uint32_t* vwords = words + kHeadDim * pl.bits_k;
+  const int sbit = slot_v(p) * BV;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int i = lane + 32 * q;
+    const uint32_t c = vlive ? (uint32_t)code_of_w<BV>(thr, __fmul_rn(y[q], vr)) : 0u;
+    put_field(vwords, 32 * BV * i + sbit, c, BV, clear);
+  }
+}
+
+// Pass 2 for stored block rank r, positions [p_lo, p_hi) (lane = position).
+template <int W>
+__device__ __forceinline__ void block_field(const Plan& pl, const float* thr, int r, int j,
+                                            const float* row, int lane, uint32_t* words,
+                                            bool clear) {
+  const float g = pl.g[j];
+  const uint32_t c0 = (uint32_t)code_of_w<W>(thr, __fmul_rn(row[j], g));
+  const uint32_t c1 = (uint32_t)code_of_w<W>(thr, __fmul_rn(row[j + 64], g));
+  put_field(words, 32 * pl.seg_off[r] + slot_k(lane) * 2 * W, c0 | (c1 << W), 2 * W, clear);
+}
+
+__device__ __forceinline__ void warp_block_pass(const Plan& pl, const float* thr, int r,
+                                                const float* kz, int p_lo, int p_hi, int lane,
+                                                uint32_t* words, bool clear) {
+  const int j = pl.order[r], w = pl.width[j];
+  if (lane < p_lo || lane >= p_hi) return;
+  const float* row = kz + lane * kKzStride;
+  switch (w) {  // uniform in the warp
+    case 1: block_field<1>(pl, thr, r, j, row, lane, words, clear); break;
+    case 2: block_field<2>(pl, thr, r, j, row, lane, words, clear); break;
+    case 3: block_field<3>(pl, thr, r, j, row, lane, words, clear); break;
+    case 4: block_field<4>(pl, thr, r, j, row, lane, words, clear); break;
+    case 5: block_field<5>(pl, thr, r, j, row, lane, words, clear); break;
+    case 6: block_field<6>(pl, thr, r, j, row, lane, words, clear); break;
+    case 7: block_field<7>(pl, thr, r, j, row, lane, words, clear); break;
+    default: block_field<8>(pl, thr, r, j, row, lane, words, clear); break;
+  }
+}
+
 }  // namespace kvq

@@ -7,6 +7,8 @@
 // cache of the serving path. Readings adopted (energy on a 2^-32 integer
 // grid, fp16 norm, Gaussian Lloyd-Max codes, randomised Hadamard on values,
 // tile record layout) are stated in kvq.h.
+#include <algorithm>
+
 #include "quant_dev.cuh"
 
 namespace kvq {
@@ -56,81 +58,87 @@ __global__ void __launch_bounds__(128) energy_kernel(const void* __restrict__ k,
 // --------------------------------------------------------------- quantize
 __constant__ float c_thr[KVQ_CB_N_THR] = KVQ_CB_THR;
 
-struct QuantParams {
-  const Plan* const* plans;  // [batch] -> [n_kv] plans
-  const void* k;
-  const void* v;
-  int dtype;
-  int batch, n_new, n_kv;
-  uint8_t* const* caches;  // [batch]
-  const int32_t* len;
-  int64_t cap;
-  int tile_bytes;
-  uint32_t* status;
-};
 
-// One CTA = the new tokens of one 32-token tile of one (sequence, KV head).
-__global__ void __launch_bounds__(256) quantize_append_kernel(QuantParams p) {
-  const int b = blockIdx.z, h = blockIdx.y;
-  const int len0 = p.len[b];
-  if (len0 < 0 || (int64_t)len0 + p.n_new > p.cap) {
-    if (threadIdx.x == 0 && blockIdx.x == 0 && h == 0) atomicOr(p.status, KVQ_FLAG_CAPACITY);
-    return;
-  }
-  const int tile = len0 / kTile + blockIdx.x;
-  const int t_lo = max(len0, tile * kTile), t_hi = min(len0 + p.n_new, tile * kTile + kTile);
-  if (t_lo >= t_hi) return;
-  uint8_t* rec = p.caches[b];
-  if ((reinterpret_cast<uintptr_t>(rec) & 15) != 0) {
-    if (threadIdx.x == 0) atomicOr(p.status, KVQ_FLAG_BAD_PLAN);
-    return;
-  }
-  rec += ((size_t)tile * p.n_kv + h) * p.tile_bytes;
-
+// Work item = the new tokens of one 32-token tile of one (sequence, KV head);
+// CTAs loop over items (item = (b n_kv + h) tiles_max + i, tile = len0 / 32
+// + i). A tile's words are assembled in shared memory (from zero for a fresh
+// tile, else from the record) by the two passes of quant_dev.cuh and written
+// back whole. The plan is reloaded only when (b, h) changes.
+template <int BV>
+__global__ void __launch_bounds__(256, 4) quantize_append_kernel(QuantParams p) {
   __shared__ Plan s_plan;
   __shared__ float s_thr[KVQ_CB_N_THR];
-  __shared__ uint8_t s_kc[kTile][kHeadDim];
-  __shared__ uint8_t s_vc[kTile][kHeadDim];
+  __shared__ float s_kz[kTile * kKzStride];
+  __shared__ uint32_t s_words[kHeadDim * 16 + 1];  // + slack word for put_field
   __shared__ uint32_t s_flags;
-  {
-    const uint32_t* src = reinterpret_cast<const uint32_t*>(p.plans[b] + h);
-    uint32_t* dst = reinterpret_cast<uint32_t*>(&s_plan);
-    for (int i = threadIdx.x; i < KVQ_PLAN_BYTES / 4; i += blockDim.x) dst[i] = src[i];
-    for (int i = threadIdx.x; i < KVQ_CB_N_THR; i += blockDim.x) s_thr[i] = c_thr[i];
-    if (threadIdx.x == 0) s_flags = 0;
-  }
-  __syncthreads();
-  const Plan& pl = s_plan;
-  const int bv = pl.bits_v;
-  if (pl.magic != KVQ_PLAN_MAGIC || pl.bits_k < 1 || pl.bits_k > 8 || bv < 1 || bv > 8 ||
-      p.tile_bytes != tile_bytes(pl.bits_k, bv)) {
-    if (threadIdx.x == 0) atomicOr(p.status, KVQ_FLAG_BAD_PLAN);
-    return;
-  }
-
-  // ---- codes of the new tokens: one warp per token
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint32_t flags = 0;
-  for (int t = t_lo + warp; t < t_hi; t += blockDim.x >> 5) {
-    const int tt = t - tile * kTile;
-    const size_t row = (((size_t)b * p.n_new + (t - len0)) * p.n_kv + h) * kHeadDim;
-    __half kn, vn;
-    warp_token_codes(pl, s_thr, p.k, p.v, p.dtype, row, lane, s_kc[tt], s_vc[tt], kn, vn, flags);
-    if (lane == 0) {
-      __half* norms = reinterpret_cast<__half*>(rec + 512 * (pl.bits_k + bv));
-      norms[tt] = kn;
-      norms[kTile + tt] = vn;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  for (int i = threadIdx.x; i < KVQ_CB_N_THR; i += blockDim.x) s_thr[i] = c_thr[i];
+  if (threadIdx.x == 0) s_flags = 0;
+  int cur = -1;  // (b, h) whose plan is in shared memory
+  bool plan_ok = false;
+  const int n_items = p.batch * p.n_kv * p.tiles_max;
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+    const int bh = item / p.tiles_max, ti = item - bh * p.tiles_max;
+    const int b = bh / p.n_kv, h = bh - b * p.n_kv;
+    const int len0 = p.len[b];
+    if (len0 < 0 || (int64_t)len0 + p.n_new > p.cap) {
+      if (threadIdx.x == 0 && ti == 0 && h == 0) atomicOr(p.status, KVQ_FLAG_CAPACITY);
+      continue;
     }
-  }
-  if (flags) atomicOr(&s_flags, flags);
-  __syncthreads();
+    const int tile = len0 / kTile + ti;
+    const int t_lo = max(len0, tile * kTile), t_hi = min(len0 + p.n_new, tile * kTile + kTile);
+    if (t_lo >= t_hi) continue;
+    uint8_t* rec = p.caches[b];
+    if ((reinterpret_cast<uintptr_t>(rec) & 15) != 0) {
+      if (threadIdx.x == 0) atomicOr(p.status, KVQ_FLAG_BAD_PLAN);
+      continue;
+    }
+    rec += ((size_t)tile * p.n_kv + h) * p.tile_bytes;
+    __syncthreads();  // the previous item is done with the shared buffers
+    if (bh != cur) {
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(p.plans[b] + h);
+      uint32_t* dst = reinterpret_cast<uint32_t*>(&s_plan);
+      for (int i = threadIdx.x; i < KVQ_PLAN_BYTES / 4; i += blockDim.x) dst[i] = src[i];
+      __syncthreads();
+      cur = bh;
+      plan_ok = s_plan.magic == KVQ_PLAN_MAGIC && s_plan.bits_k >= 1 && s_plan.bits_k <= 8 &&
+                s_plan.bits_v == BV && p.tile_bytes == tile_bytes(s_plan.bits_k, BV);
+    }
+    if (!plan_ok) {
+      if (threadIdx.x == 0) atomicOr(p.status, KVQ_FLAG_BAD_PLAN);
+      continue;
+    }
+    const Plan& pl = s_plan;
+    const int n_words = kHeadDim * (pl.bits_k + BV);
+    const bool clear = len0 > tile * kTile;  // the tile already holds tokens
+    uint32_t* gw = reinterpret_cast<uint32_t*>(rec);
+    for (int i = threadIdx.x; i < n_words; i += blockDim.x) s_words[i] = clear ? gw[i] : 0u;
+    __syncthreads();
 
-  // ---- assemble segment words: keep older tokens' bits, write the new ones,
-  //      zero positions past the new length
-  const int old_n = max(0, len0 - tile * kTile);  // positions holding older tokens
-  assemble_tile_words(reinterpret_cast<uint32_t*>(rec), reinterpret_cast<const uint32_t*>(rec),
-                      nullptr, pl, s_kc, s_vc, old_n,
-                      t_lo - tile * kTile, t_hi - tile * kTile, threadIdx.x, blockDim.x);
+    // ---- pass 1: one warp per new token
+    const int p_lo = t_lo - tile * kTile, p_hi = t_hi - tile * kTile;
+    uint32_t flags = 0;
+    __half* norms = reinterpret_cast<__half*>(rec + 512 * (pl.bits_k + BV));
+    for (int pp = p_lo + warp; pp < p_hi; pp += nw) {
+      const size_t row =
+          (((size_t)b * p.n_new + (tile * kTile + pp - len0)) * p.n_kv + h) * kHeadDim;
+      __half kn, vn;
+      warp_token_pass<BV>(pl, s_thr, p.k, p.v, p.dtype, row, lane, pp, s_kz + pp * kKzStride,
+                          s_words, clear, kn, vn, flags);
+      if (lane == 0) {
+        norms[pp] = kn;
+        norms[kTile + pp] = vn;
+      }
+    }
+    if (flags) atomicOr(&s_flags, flags);
+    __syncthreads();
+    // ---- pass 2: one warp per stored key block
+    for (int r = warp; r < pl.n_ranks; r += nw)
+      warp_block_pass(pl, s_thr, r, s_kz, p_lo, p_hi, lane, s_words, clear);
+    __syncthreads();
+    for (int i = threadIdx.x; i < n_words; i += blockDim.x) gw[i] = s_words[i];
+  }
+  __syncthreads();
   if (threadIdx.x == 0 && s_flags) atomicOr(p.status, s_flags);
 }
 
@@ -152,9 +160,27 @@ cudaError_t launch_energy(const void* k, int dtype, int64_t n_tokens, int n_kv,
   return cudaGetLastError();
 }
 
-cudaError_t launch_quantize_append(const QuantParams& p, cudaStream_t st) {
-  const int tiles = (p.n_new + kTile - 1) / kTile + 1;
-  quantize_append_kernel<<<dim3(tiles, p.n_kv, p.batch), 256, 0, st>>>(p);
+cudaError_t launch_quantize_append(const QuantParams& p_in, int bits_v, cudaStream_t st) {
+  QuantParams p = p_in;
+  p.tiles_max = (p.n_new + kTile - 1) / kTile + 1;
+  const int64_t n_items = (int64_t)p.batch * p.n_kv * p.tiles_max;
+  if (n_items > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    (void)cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  (void)cudaGetLastError();
+  const unsigned grid = (unsigned)std::min<int64_t>(n_items, (int64_t)4 * sms);  // resident
+  switch (bits_v) {
+    case 1: quantize_append_kernel<1><<<grid, 256, 0, st>>>(p); break;
+    case 2: quantize_append_kernel<2><<<grid, 256, 0, st>>>(p); break;
+    case 3: quantize_append_kernel<3><<<grid, 256, 0, st>>>(p); break;
+    case 4: quantize_append_kernel<4><<<grid, 256, 0, st>>>(p); break;
+    case 5: quantize_append_kernel<5><<<grid, 256, 0, st>>>(p); break;
+    case 6: quantize_append_kernel<6><<<grid, 256, 0, st>>>(p); break;
+    case 7: quantize_append_kernel<7><<<grid, 256, 0, st>>>(p); break;
+    case 8: quantize_append_kernel<8><<<grid, 256, 0, st>>>(p); break;
+    default: return cudaErrorInvalidValue;
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   bump_len_kernel<<<(p.batch + 255) / 256, 256, 0, st>>>(const_cast<int32_t*>(p.len), p.batch,
