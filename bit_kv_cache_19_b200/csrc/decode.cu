@@ -67,7 +67,7 @@ constexpr int kMaxSplits = 1024;
 constexpr int kCntStride = 2 + kMaxSplits / kGroup;  // per (sequence, KV head); last = sequence
 constexpr int kFallbackSlots = 1024;                  // CTA slots when no device answers
 constexpr int kMaxNew = 64;                           // tokens appended by a fused call
-constexpr int kScratch = 8192 + 128;                  // q' staging / append codes + norms
+constexpr int kScratch = 16640;  // q' staging; append: kz [32][129] fp32 + 64 fp16 norms
 
 struct DecodeParams {
   const Plan* const* plans;
@@ -489,39 +489,46 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   //      patch them into the streamed copy of each tile (stage 0 of warp
   //      te - 1 - tile) and into the cache
   if (appends) {
-    uint8_t (*kc)[kHeadDim] = reinterpret_cast<uint8_t (*)[kHeadDim]>(scratch);
-    uint8_t (*vc)[kHeadDim] = reinterpret_cast<uint8_t (*)[kHeadDim]>(scratch + 32 * kHeadDim);
-    __half* nrm_new = reinterpret_cast<__half*>(scratch + 64 * kHeadDim);  // [2][32]
+    float* kz = reinterpret_cast<float*>(scratch);                          // [32][129]
+    __half* nrm_new = reinterpret_cast<__half*>(scratch + kTile * kKzStride * 4);  // [2][32]
     uint32_t flags = 0;
     for (int tile = a_lo; tile <= a_hi; ++tile) {
       const int t_lo = max(len0, tile * kTile), t_hi = min(len0 + n_add, tile * kTile + kTile);
+      const int p_lo = t_lo - tile * kTile, p_hi = t_hi - tile * kTile;
       const int w_own = te - 1 - tile;
       uint8_t* rec = const_cast<uint8_t*>(cache) + ((size_t)tile * p.n_kv + h) * tbytes;
       uint8_t* st = stage_base + (size_t)w_own * kStages * tbytes;
-      for (int t = t_lo + warp; t < t_hi; t += kWarps) {
-        const int tt = t - tile * kTile;
-        const size_t row = (((size_t)b * p.n_new + (t - len0)) * p.n_kv + h) * kHeadDim;
+      uint32_t* sw = reinterpret_cast<uint32_t*>(st);
+      const int n_words = kHeadDim * (bk + BV);
+      const bool clear = len0 > tile * kTile;  // the tile already holds tokens
+      const bool ok = mbar_wait_bounded(&sm.bar[w_own][0], 0u);  // the old tile is in `st`
+      if (!clear)
+        for (int i = tid; i < n_words; i += kThreads) sw[i] = 0u;
+      __syncthreads();
+      // pass 1 (one warp per new token; the word after the packed words, the
+      // first norm word of the copy, takes only no-op atomics), then pass 2
+      for (int pp = p_lo + warp; pp < p_hi; pp += kWarps) {
+        const size_t row =
+            (((size_t)b * p.n_new + (tile * kTile + pp - len0)) * p.n_kv + h) * kHeadDim;
         __half kn, vn;
-        warp_token_codes(sm.plan, sm.thr, p.k_new, p.v_new, p.kv_dtype, row, lane, kc[tt], vc[tt],
-                         kn, vn, flags);
+        warp_token_pass<BV>(sm.plan, sm.thr, p.k_new, p.v_new, p.kv_dtype, row, lane, pp,
+                            kz + pp * kKzStride, sw, clear, kn, vn, flags);
         if (lane == 0) {
-          nrm_new[tt] = kn;
-          nrm_new[kTile + tt] = vn;
+          nrm_new[pp] = kn;
+          nrm_new[kTile + pp] = vn;
         }
       }
-      const bool ok = mbar_wait_bounded(&sm.bar[w_own][0], 0u);  // the old tile is in `st`
+      __syncthreads();
+      for (int r = warp; r < sm.plan.n_ranks; r += kWarps)
+        warp_block_pass(sm.plan, sm.thr, r, kz, p_lo, p_hi, lane, sw, clear);
       __syncthreads();
       if (ok) {
-        assemble_tile_words(reinterpret_cast<uint32_t*>(rec), reinterpret_cast<uint32_t*>(st),
-                            reinterpret_cast<uint32_t*>(st), sm.plan, kc, vc,
-                            max(0, len0 - tile * kTile), t_lo - tile * kTile, t_hi - tile * kTile,
-                            tid, kThreads);
-        for (int t = t_lo + tid; t < t_hi; t += kThreads) {
-          const int tt = t - tile * kTile;
-          for (int e = 0; e < 2; ++e) {
-            reinterpret_cast<__half*>(rec + 512 * (bk + BV))[e * kTile + tt] = nrm_new[e * kTile + tt];
-            reinterpret_cast<__half*>(st + 512 * (bk + BV))[e * kTile + tt] = nrm_new[e * kTile + tt];
-          }
+        uint32_t* gw = reinterpret_cast<uint32_t*>(rec);
+        for (int i = tid; i < n_words; i += kThreads) gw[i] = sw[i];
+        for (int e = tid; e < 2 * (p_hi - p_lo); e += kThreads) {
+          const int pp = p_lo + (e >> 1), off = (e & 1) * kTile + pp;
+          reinterpret_cast<__half*>(rec + 512 * (bk + BV))[off] = nrm_new[off];
+          reinterpret_cast<__half*>(st + 512 * (bk + BV))[off] = nrm_new[off];
         }
       } else {
         flags |= KVQ_FLAG_TIMEOUT;

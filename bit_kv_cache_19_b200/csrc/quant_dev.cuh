@@ -1,29 +1,19 @@
 // Device code shared by the quantize-append kernel and the fused
-// append + decode kernel: the TQ-MSE codes of one token (keys with per-block
-// widths, values with a randomised Hadamard rotation), and the assembly of
-// the packed words of one tile record.
+// append + decode kernel: the TQ-MSE codes of a tile's new tokens (keys with
+// per-block widths, values with a randomised Hadamard rotation) packed into
+// the words of its tile record.
 //
 // "RoPE-Aware Bit Allocation for KV-Cache Quantization", abstract: keys are
 // quantized with Block-GTQ's per-RoPE-block integer widths on top of
 // TurboQuant-MSE, values with uniform TQ-MSE. All decisions use IEEE fp32
-// without fused multiply-add in a fixed order (see kvq.h), so codes are the
-// same bit for bit on every run.
+// in a fixed order with no product contracted into a sum (see kvq.h; an fma
+// with a +-1 factor, whose product is exact, stands for an add or subtract),
+// so codes are the same bit for bit on every run.
 #pragma once
 
 #include "common.cuh"
 
 namespace kvq {
-
-// Number of width-w thresholds strictly below z (NaN -> 0): branch-free
-// binary search over the sorted 2^w - 1 thresholds (all widths at `thr`,
-// width w at cb_t_off(w)).
-__device__ __forceinline__ int code_of(const float* thr, int w, float z) {
-  const float* t = thr + cb_t_off(w);
-  int c = 0;
-  for (int step = 1 << (w - 1); step; step >>= 1)
-    if (t[c + step - 1] < z) c += step;
-  return c;
-}
 
 // Fixed-order fp32 sum of squares of a 128-vector held as v[q] = x[lane + 32 q]:
 // p = ((v0^2 + v1^2) + v2^2) + v3^2, then p += p(lane ^ m) for m = 16..1.
@@ -54,128 +44,6 @@ __device__ __forceinline__ void norm_and_recip(const float (&v)[4], bool finite,
   const float n = __half2float(n16);
   r = n > 0.f ? __frcp_rn(n) : 0.f;
 }
-
-// Codes of one token, computed by one warp. k_row / v_row: the token's key
-// and value (128 elements of `dtype`). Writes kc[128] (canonical coordinates)
-// and vc[128] (rotated coordinates) and returns the fp16 norms.
-__device__ __forceinline__ void warp_token_codes(const Plan& pl, const float* thr,
-                                                 const void* k, const void* v, int dtype,
-                                                 size_t row, int lane, uint8_t* kc, uint8_t* vc,
-                                                 __half& kn, __half& vn, uint32_t& flags) {
-  float kx[4], vx[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    kx[q] = load_as_float(k, dtype, row + lane + 32 * q);
-    vx[q] = load_as_float(v, dtype, row + lane + 32 * q);
-  }
-  const bool kfin = __all_sync(0xffffffffu, isfinite(kx[0]) && isfinite(kx[1]) &&
-                                                isfinite(kx[2]) && isfinite(kx[3]));
-  const bool vfin = __all_sync(0xffffffffu, isfinite(vx[0]) && isfinite(vx[1]) &&
-                                                isfinite(vx[2]) && isfinite(vx[3]));
-  // keys: z_i = (k_i r) g_j, width b_j
-  float kr;
-  norm_and_recip(kx, kfin, kn, kr, flags);
-  const bool klive = kfin && __half2float(kn) > 0.f;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int i = lane + 32 * q, j = i & 63, w = pl.width[j];
-    int c = 0;
-    if (w > 0 && klive) c = code_of(thr, w, __fmul_rn(__fmul_rn(kx[q], kr), pl.g[j]));
-    kc[i] = (uint8_t)c;
-  }
-  // values: y = H (s . v) by the fixed fp32 butterfly graph, z = y r
-  float vr;
-  norm_and_recip(vx, vfin, vn, vr, flags);
-  const bool vlive = vfin && __half2float(vn) > 0.f;
-  float y[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int i = lane + 32 * q;
-    const float x = vfin ? vx[q] : 0.f;
-    y[q] = ((pl.v_sign[i >> 5] >> (i & 31)) & 1u) ? -x : x;
-  }
-#pragma unroll
-  for (int hh = 1; hh < 32; hh <<= 1) {
-    const bool upper = (lane & hh) != 0;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float o = __shfl_xor_sync(0xffffffffu, y[q], hh);
-      y[q] = upper ? __fsub_rn(o, y[q]) : __fadd_rn(y[q], o);
-    }
-  }
-  {  // h = 32: (q0, q1), (q2, q3); h = 64: (q0, q2), (q1, q3)
-    const float a0 = __fadd_rn(y[0], y[1]), a1 = __fsub_rn(y[0], y[1]);
-    const float a2 = __fadd_rn(y[2], y[3]), a3 = __fsub_rn(y[2], y[3]);
-    y[0] = __fadd_rn(a0, a2);
-    y[2] = __fsub_rn(a0, a2);
-    y[1] = __fadd_rn(a1, a3);
-    y[3] = __fsub_rn(a1, a3);
-  }
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    int c = 0;
-    if (vlive) c = code_of(thr, pl.bits_v, __fmul_rn(y[q], vr));
-    vc[lane + 32 * q] = (uint8_t)c;
-  }
-}
-
-// Packed words of one tile record into `words` (and `copy`, if not null).
-// Positions [0, old_n) hold older tokens whose bits are kept from `old`;
-// positions [new_lo, new_hi) get the codes in kc / vc (rows indexed by
-// position); all other positions are zero. When the tile already holds
-// tokens (old_n > 0) only words that carry bits of new positions are
-// rewritten. Threads tid, tid + nth, ... take one word each (a word is read
-// from `old` and written by the same thread, so `old` may alias either
-// destination).
-__device__ __forceinline__ void assemble_tile_words(uint32_t* words, const uint32_t* old,
-                                                    uint32_t* copy, const Plan& pl,
-                                                    const uint8_t (*kc)[kHeadDim],
-                                                    const uint8_t (*vc)[kHeadDim], int old_n,
-                                                    int new_lo, int new_hi, int tid, int nth) {
-  const int bv = pl.bits_v;
-  const int words_k = 128 * pl.bits_k;
-  for (int wi = tid; wi < words_k + 128 * bv; wi += nth) {
-    int f, k, jj = 0, w = 0, pcoord = 0;
-    const bool is_k = wi < words_k;
-    if (is_k) {
-      int lo = 0, hi = pl.n_ranks;  // largest rank r with seg_off[r] <= wi
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (pl.seg_off[mid] <= wi) lo = mid; else hi = mid;
-      }
-      jj = pl.order[lo];
-      w = pl.width[jj];
-      f = 2 * w;
-      k = wi - pl.seg_off[lo];
-    } else {
-      pcoord = (wi - words_k) / bv;
-      k = (wi - words_k) - pcoord * bv;
-      f = bv;
-    }
-    uint32_t nw = 0, keep = 0;
-    bool touched = false;
-    const int s0 = (32 * k) / f, s1 = (32 * k + 31) / f;
-    for (int s = s0; s <= s1 && s < kTile; ++s) {
-      const int tok = is_k ? token_of_slot_k(s) : token_of_slot_v(s);
-      const int fb = s * f - 32 * k + 32;  // bit position + 32, in (32 - f, 64)
-      if (tok >= new_lo && tok < new_hi) {
-        const uint32_t field = is_k ? (uint32_t)kc[tok][jj] | ((uint32_t)kc[tok][jj + 64] << w)
-                                    : (uint32_t)vc[tok][pcoord];
-        nw |= (uint32_t)(((unsigned long long)field << fb) >> 32);
-        touched = true;
-      } else if (tok < old_n) {
-        const uint32_t field = (f == 32) ? 0xFFFFFFFFu : ((1u << f) - 1u);
-        keep |= (uint32_t)(((unsigned long long)field << fb) >> 32);
-      }
-    }
-    if (old_n == 0 || touched) {
-      const uint32_t w = old_n == 0 ? nw : (old[wi] & keep) | nw;
-      words[wi] = w;
-      if (copy) copy[wi] = w;
-    }
-  }
-}
-
 
 // ---------------------------------------------------------------------------
 // Tile quantizer in two passes (one CTA per tile record):
@@ -208,7 +76,9 @@ __device__ __forceinline__ void put_field(uint32_t* words, int bit, uint32_t val
   atomicOr(&words[wi + 1], (uint32_t)(v2 >> 32));
 }
 
-// code_of for a compile-time width (all steps unrolled).
+// Number of width-W thresholds strictly below z (NaN -> 0): branch-free
+// binary search over the sorted 2^W - 1 thresholds of width W (at
+// thr + cb_t_off(W)), all steps unrolled.
 template <int W>
 __device__ __forceinline__ int code_of_w(const float* thr, float z) {
   const float* t = thr + cb_t_off(W);
