@@ -139,13 +139,22 @@ __device__ __forceinline__ void warp_token_pass(const Plan& pl, const float* thr
     y[1] = __fadd_rn(a1, a3);
     y[3] = __fsub_rn(a1, a3);
   }
-  uint32_t* vwords = words + kHeadDim * pl.bits_k;
-  const int sbit = slot_v(p) * BV;
+  // value fields: coordinate i at bit slot_v(p) BV of its BV-word segment;
+  // the bit offset in the word is the same for every lane and q
+  uint32_t* vwords = words + kHeadDim * pl.bits_k + ((slot_v(p) * BV) >> 5);
+  const int off = (slot_v(p) * BV) & 31;
+  const bool spill = off + BV > 32;  // uniform
+  constexpr uint32_t mask = (1u << BV) - 1u;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    const int i = lane + 32 * q;
+    uint32_t* w = vwords + BV * (lane + 32 * q);
     const uint32_t c = vlive ? (uint32_t)code_of_w<BV>(thr, __fmul_rn(y[q], vr)) : 0u;
-    put_field(vwords, 32 * BV * i + sbit, c, BV, clear);
+    if (clear) atomicAnd(w, ~(mask << off));
+    atomicOr(w, c << off);
+    if (spill) {
+      if (clear) atomicAnd(w + 1, ~(mask >> (32 - off)));
+      atomicOr(w + 1, c >> (32 - off));
+    }
   }
 }
 

@@ -14,9 +14,30 @@
 namespace kvq {
 
 // ----------------------------------------------------------------- energy
+// Square term of one key element on the 2^-32 grid: floor(x^2 2^32),
+// saturating at 2^64 - 1; non-finite elements give 0 and set `bad`. For
+// 16-bit inputs x^2 2^32 is exact in fp32 (a square of <= 11 significant
+// bits, a power-of-two scale); fp32 inputs use fp64 (48-bit square).
+template <bool WIDE>
+__device__ __forceinline__ unsigned long long square_term(float x, bool& bad) {
+  if (!isfinite(x)) {
+    bad = true;
+    return 0ull;
+  }
+  if (!WIDE) {
+    const float s = x * x * 4294967296.0f;
+    return s >= 18446744073709551616.0f ? 0xFFFFFFFFFFFFFFFFull : (unsigned long long)s;
+  }
+  const double s = (double)x * (double)x * 4294967296.0;
+  return s >= 18446744073709551616.0 ? 0xFFFFFFFFFFFFFFFFull : (unsigned long long)s;
+}
+
 // acc[h][j] = (lo, hi) 128-bit sum over tokens and the two coordinates of
-// block j of min(floor(k^2 2^32), 2^64 - 1). Integer atomics: the total does
-// not depend on the order of the additions.
+// block j of the square terms. One thread per coordinate; 8 tokens' loads
+// in flight; the low and high 32-bit halves of the terms are summed apart
+// (no carries while streaming) and joined at the end. Integer sums: the
+// total does not depend on the order of the additions.
+template <bool WIDE>
 __global__ void __launch_bounds__(128) energy_kernel(const void* __restrict__ k, int dtype,
                                                     int64_t n_tokens, int n_kv, int chunk,
                                                     unsigned long long* __restrict__ acc,
@@ -25,20 +46,30 @@ __global__ void __launch_bounds__(128) energy_kernel(const void* __restrict__ k,
   const int i = threadIdx.x;  // coordinate
   const int64_t t0 = (int64_t)blockIdx.x * chunk;
   const int64_t t1 = min(n_tokens, t0 + chunk);
-  unsigned long long lo = 0, hi = 0;
+  unsigned long long slo = 0, shi = 0;  // sums of the terms' low / high 32-bit halves
   bool bad = false;
-  for (int64_t t = t0; t < t1; ++t) {
-    const float x = load_as_float(k, dtype, ((size_t)t * n_kv + h) * kHeadDim + i);
-    unsigned long long term = 0;
-    if (isfinite(x)) {
-      const double s = (double)x * (double)x * 4294967296.0;  // exact for <= 26-bit significands
-      term = s >= 18446744073709551616.0 ? 0xFFFFFFFFFFFFFFFFull : (unsigned long long)s;
-    } else {
-      bad = true;
+  const size_t stride = (size_t)n_kv * kHeadDim;
+  size_t e = ((size_t)t0 * n_kv + h) * kHeadDim + i;
+  int64_t t = t0;
+  for (; t + 8 <= t1; t += 8, e += 8 * stride) {
+    float x[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) x[u] = load_as_float(k, dtype, e + u * stride);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const unsigned long long term = square_term<WIDE>(x[u], bad);
+      slo += term & 0xFFFFFFFFull;
+      shi += term >> 32;
     }
-    lo += term;
-    hi += (lo < term);
   }
+  for (; t < t1; ++t, e += stride) {
+    const unsigned long long term = square_term<WIDE>(load_as_float(k, dtype, e), bad);
+    slo += term & 0xFFFFFFFFull;
+    shi += term >> 32;
+  }
+  // 128-bit value shi 2^32 + slo
+  const unsigned long long lo = slo + (shi << 32);
+  const unsigned long long hi = (shi >> 32) + (lo < slo ? 1ull : 0ull);
   __shared__ unsigned long long s_lo[kHeadDim], s_hi[kHeadDim];
   s_lo[i] = lo;
   s_hi[i] = hi;
@@ -155,8 +186,12 @@ cudaError_t launch_energy(const void* k, int dtype, int64_t n_tokens, int n_kv,
   if (nchunks > 0x7FFFFFFF) return cudaErrorInvalidValue;
   cudaError_t e = cudaMemsetAsync(acc, 0, (size_t)n_kv * kBlocks * 16, st);
   if (e != cudaSuccess) return e;
-  energy_kernel<<<dim3((unsigned)nchunks, n_kv), 128, 0, st>>>(k, dtype, n_tokens, n_kv, chunk,
-                                                                acc, status);
+  if (dtype == KVQ_BF16 || dtype == KVQ_FP16)
+    energy_kernel<false><<<dim3((unsigned)nchunks, n_kv), 128, 0, st>>>(k, dtype, n_tokens, n_kv,
+                                                                        chunk, acc, status);
+  else
+    energy_kernel<true><<<dim3((unsigned)nchunks, n_kv), 128, 0, st>>>(k, dtype, n_tokens, n_kv,
+                                                                       chunk, acc, status);
   return cudaGetLastError();
 }
 
