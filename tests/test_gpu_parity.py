@@ -361,3 +361,46 @@ def test_early_prefetch_layer_loop_matches_plain():
         for s in range(len(starts)):
             assert torch.equal(a.caches[s], b.caches[s]), (li, s)
         assert a.flags() == 0 and b.flags() == 0
+
+
+@pytest.mark.parametrize("bits", [(3, 3), (5, 2), (2, 7)])
+def test_chunked_appends_mixed_lengths(bits):
+    """Appends of 1, 5, 37, 64, 3 and 30 tokens to five sequences that start
+    at different lengths (fresh tiles, partly filled tiles, tile boundaries,
+    fields that straddle words): every record bit-exact against the oracle's
+    pack of the whole sequence, lengths and flags as expected."""
+    bk, bv = bits
+    rng = np.random.default_rng(500 + 10 * bk + bv)
+    n_kv = 2
+    starts = [0, 7, 31, 32, 100]
+    chunks = [1, 5, 37, 64, 3, 30]
+    total = sum(chunks)
+    cap = max(starts) + total + 32
+    cfg = kvq.make_cfg(n_kv, bk, bv, v_seed=21)
+    L = PackedLayer(cfg, len(starts), cap, layer=4)
+    E, _, _ = _random_layer(rng, n_kv, 1, 1.2)
+    L.set_plans(kvq.plan_build(cfg, 4, E))
+    data = []
+    for s, T0 in enumerate(starts):
+        _, kb, vb = _random_layer(rng, n_kv, T0 + total, 1.2)
+        data.append((kb, vb))
+        if T0:
+            kvq.quantize_append(cfg, L.plan_ptrs[s:s + 1], dev_bf16(kb[:T0])[None],
+                                dev_bf16(vb[:T0])[None], L.cache_ptrs[s:s + 1],
+                                L.lens[s:s + 1], cap, L.status)
+    off = 0
+    for n in chunks:
+        k = torch.stack([dev_bf16(kb[T0 + off:T0 + off + n]) for (kb, _), T0 in zip(data, starts)])
+        v = torch.stack([dev_bf16(vb[T0 + off:T0 + off + n]) for (_, vb), T0 in zip(data, starts)])
+        L.append(k, v)
+        off += n
+    torch.cuda.synchronize()
+    assert L.flags() == 0
+    assert L.lens.cpu().tolist() == [T0 + total for T0 in starts]
+    for s, T0 in enumerate(starts):
+        T = T0 + total
+        kb, vb = data[s]
+        kh, vh = op.bf16_heads(kb[:T], vb[:T])
+        _, heads = op.layer(kh, vh, bk, bv, 21, 4, E=E)
+        for h in range(n_kv):
+            check_records(L.head_records(s, h, (T + 31) // 32), heads[h]["rec"], T, bk, bv)
