@@ -23,6 +23,11 @@ cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches
                           int bits_k, int bits_v, float* out, void* ws, size_t ws_bytes,
                           uint32_t* status, cudaStream_t st, const void* k_new, const void* v_new,
                           int kv_dtype, int n_new, int64_t cap, int early);
+size_t dense_workspace_bytes_for(int batch, int n_kv, int n_q, int64_t max_len);
+cudaError_t launch_dense_decode(const void* k, const void* v, const int32_t* len, int batch,
+                                int n_kv, int64_t cap, int64_t max_len, const void* q, int n_q,
+                                float* out, void* ws, size_t ws_bytes, uint32_t* status,
+                                cudaStream_t st);
 
 namespace {
 
@@ -357,6 +362,44 @@ int kvq_append_decode(const kvq_cfg* cfg, const void* const* plans_dev, const vo
                                 reinterpret_cast<cudaStream_t>(stream), k_dev, v_dev, kv_dtype,
                                 n_new, cap_tokens, (step_flags & KVQ_STEP_EARLY) ? 1 : 0);
   if (e != cudaSuccess) return cuda_fail(e, "append_decode");
+  return KVQ_OK;
+}
+
+}  // extern "C"
+
+extern "C" {
+
+size_t kvq_bf16_decode_workspace_bytes(int batch, int n_kv_heads, int n_q_heads, int64_t max_len) {
+  if (batch < 1 || n_kv_heads < 1 || n_q_heads < 1 || n_q_heads % n_kv_heads != 0 ||
+      n_q_heads / n_kv_heads > 16 || max_len < 1)
+    return 0;
+  return dense_workspace_bytes_for(batch, n_kv_heads, n_q_heads, max_len);
+}
+
+int kvq_bf16_decode_attn(const void* k_dev, const void* v_dev, const int32_t* len_dev, int batch,
+                         int n_kv_heads, int64_t cap_tokens, int64_t max_len, const void* q_dev,
+                         int n_q_heads, float* out_dev, void* ws_dev, size_t ws_bytes,
+                         uint32_t* status_dev, kvq_stream_t stream) {
+  if (!k_dev || !v_dev || !len_dev || !q_dev || !out_dev || !ws_dev || !status_dev)
+    return fail(KVQ_ERR_ARG, "null device pointer");
+  if (batch < 1 || batch > 65535) return fail(KVQ_ERR_ARG, "batch %d", batch);
+  if (n_kv_heads < 1 || n_kv_heads > 65535) return fail(KVQ_ERR_ARG, "n_kv_heads %d", n_kv_heads);
+  if (n_q_heads < 1 || n_q_heads % n_kv_heads != 0 || n_q_heads / n_kv_heads > 16)
+    return fail(KVQ_ERR_ARG, "n_q_heads %d vs n_kv_heads %d", n_q_heads, n_kv_heads);
+  if (cap_tokens < 1 || max_len < 1 || max_len > 0x7FFFFFFF)
+    return fail(KVQ_ERR_ARG, "cap_tokens %lld max_len %lld", (long long)cap_tokens,
+                (long long)max_len);
+  if ((reinterpret_cast<uintptr_t>(k_dev) | reinterpret_cast<uintptr_t>(v_dev) |
+       reinterpret_cast<uintptr_t>(ws_dev)) & 15)
+    return fail(KVQ_ERR_ARG, "k, v and workspace must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(q_dev) & 3) return fail(KVQ_ERR_ARG, "q must be 4-byte aligned");
+  const size_t need = kvq_bf16_decode_workspace_bytes(batch, n_kv_heads, n_q_heads, max_len);
+  if (ws_bytes < need)
+    return fail(KVQ_ERR_WORKSPACE, "bf16 decode workspace %zu < %zu", ws_bytes, need);
+  cudaError_t e = launch_dense_decode(k_dev, v_dev, len_dev, batch, n_kv_heads, cap_tokens,
+                                      max_len, q_dev, n_q_heads, out_dev, ws_dev, ws_bytes,
+                                      status_dev, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "bf16_decode_attn");
   return KVQ_OK;
 }
 

@@ -43,6 +43,7 @@
 #include <atomic>
 
 #include "quant_dev.cuh"
+#include "splitk.cuh"
 
 namespace kvq {
 
@@ -59,12 +60,6 @@ constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kStages = 2;
 constexpr int kMaxHalf = 24;  // half steps of <= 4 blocks (<= 64/4 + 8)
-constexpr int kPartStride = 132;  // split record: m, l, 2 unused, o[128]
-constexpr int kRecO = 4;          // o at float 4 (16-byte aligned)
-constexpr int kGroup = 16;    // splits merged per first-level group
-constexpr int kMergeChunk = 16;  // records whose loads a merge issues together
-constexpr int kMaxSplits = 1024;
-constexpr int kCntStride = 2 + kMaxSplits / kGroup;  // per (sequence, KV head); last = sequence
 constexpr int kFallbackSlots = 1024;                  // CTA slots when no device answers
 constexpr int kMaxNew = 64;                           // tokens appended by a fused call
 constexpr int kScratch = 16640;  // q' staging; append: kz [32][129] fp32 + 64 fp16 norms
@@ -118,37 +113,6 @@ __device__ __forceinline__ uint32_t ld32s(const uint8_t* p) {
 }
 __device__ __forceinline__ uint32_t ld16s(const uint8_t* p) {
   return *reinterpret_cast<const uint16_t*>(p);
-}
-
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ void grid_dep_wait() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-}
-// Arrival on a counter that wraps to zero after n arrivals, by one thread of
-// a CTA after a CTA barrier; true for the last arriver. The atomic is
-// acquire-release at GPU scope: the CTA's earlier writes (ordered before it
-// by the barrier) are visible to the last arriver, whose CTA reads after a
-// barrier that follows see the writes of every arriver.
-__device__ __forceinline__ bool arrive_last(unsigned int* c, unsigned int n) {
-  unsigned int old;
-  asm volatile("atom.acq_rel.gpu.global.inc.u32 %0, [%1], %2;"
-               : "=r"(old)
-               : "l"(c), "r"(n - 1u)
-               : "memory");
-  return old == n - 1u;
-}
-
-// L2 prefetch (a hint: no value is read, so it may precede the wait for the
-// kernel that writes the line).
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
-__device__ __forceinline__ void grid_dep_launch() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // Four fp16 pairs from the 4 pair fields (2W bits each) that start at bit
@@ -296,60 +260,6 @@ __device__ __forceinline__ void warp_unrotate_store(const float* src, const Plan
     const int i = lane + 32 * q;
     const float sgn = ((pl.v_sign[i >> 5] >> (i & 31)) & 1u) ? -1.f : 1.f;
     out[i] = sgn * y[q] * inv;
-  }
-}
-
-// Merge n records per head (record s of head h at src + s * rec_stride +
-// h * kPartStride) into dst (record h at dst + h * kPartStride), for G heads.
-// 32 threads per head, 4 coordinates each: one pass with online rescaling
-// over chunks of 16 records whose loads are issued together, so a merge of
-// all heads costs about n / 16 load round trips.
-__device__ __forceinline__ void merge_records(const float* src, int n, size_t rec_stride, int G,
-                                              float* dst) {
-  for (int item = threadIdx.x; item < G * 32; item += kThreads) {
-    const int head = item >> 5, x4 = (item & 31) * 4;
-    const float* r = src + (size_t)head * kPartStride;
-    float M = -INFINITY, L = 0.f;
-    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s0 = 0; s0 < n; s0 += kMergeChunk) {
-      float2 ml[kMergeChunk];
-      float4 oo[kMergeChunk];
-#pragma unroll
-      for (int k = 0; k < kMergeChunk; ++k) {
-        const bool v = s0 + k < n;
-        const float* q = r + (size_t)(v ? s0 + k : 0) * rec_stride;
-        ml[k] = *reinterpret_cast<const float2*>(q);
-        oo[k] = *reinterpret_cast<const float4*>(q + kRecO + x4);
-        if (!v) ml[k].x = -INFINITY;
-      }
-      float cm = M;
-#pragma unroll
-      for (int k = 0; k < kMergeChunk; ++k) cm = fmaxf(cm, ml[k].x);
-      if (cm != -INFINITY) {
-        const float a = ex2(M - cm);
-        L *= a;
-        O.x *= a;
-        O.y *= a;
-        O.z *= a;
-        O.w *= a;
-#pragma unroll
-        for (int k = 0; k < kMergeChunk; ++k) {
-          const float w = ex2(ml[k].x - cm);  // 0 for records past n
-          L += w * ml[k].y;
-          O.x += w * oo[k].x;
-          O.y += w * oo[k].y;
-          O.z += w * oo[k].z;
-          O.w += w * oo[k].w;
-        }
-        M = cm;
-      }
-    }
-    float* d = dst + (size_t)head * kPartStride;
-    *reinterpret_cast<float4*>(d + kRecO + x4) = O;
-    if (x4 == 0) {
-      d[0] = M;
-      d[1] = L;
-    }
   }
 }
 
@@ -745,7 +655,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
     }
   __syncthreads();
   float* const my_part = p.part + (bh * p.n_splits + split) * G * kPartStride;
-  merge_records(mg, kWarps, (size_t)8 * NT * kPartStride, G, my_part);
+  merge_records<kThreads>(mg, kWarps, (size_t)8 * NT * kPartStride, G, my_part);
 
   // ---- level 1: the last CTA of this group of splits merges the group
   const int grp = split / kGroup;
@@ -755,7 +665,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   __syncthreads();
   if (!sm.is_last) return;
   float* my_gpart = p.gpart + (bh * p.n_groups + grp) * G * kPartStride;
-  merge_records(p.part + (bh * p.n_splits + g_lo) * G * kPartStride, g_n,
+  merge_records<kThreads>(p.part + (bh * p.n_splits + g_lo) * G * kPartStride, g_n,
                 (size_t)G * kPartStride, G, my_gpart);
 
   // ---- level 2: the last group merges the groups and writes o / l
@@ -764,7 +674,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   __syncthreads();
   if (!sm.is_last) return;
   float* fin = reinterpret_cast<float*>(stage_base);  // [16][132]
-  merge_records(p.gpart + bh * p.n_groups * G * kPartStride, p.n_groups, (size_t)G * kPartStride,
+  merge_records<kThreads>(p.gpart + bh * p.n_groups * G * kPartStride, p.n_groups, (size_t)G * kPartStride,
                 G, fin);
   __syncthreads();
   for (int head = warp; head < G; head += kWarps) {

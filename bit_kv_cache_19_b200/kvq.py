@@ -77,6 +77,9 @@ _SIGS = {
     "kvq_decode_attn_noalloc": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i64, _vp, _i32,
                                        _i32, _vp, _vp, _vp]),
     "kvq_decode_noalloc_scratch_bytes": (_sz, []),
+    "kvq_bf16_decode_workspace_bytes": (_sz, [_i32, _i32, _i32, _i64]),
+    "kvq_bf16_decode_attn": (_i32, [_vp, _vp, _vp, _i32, _i32, _i64, _i64, _vp, _i32, _vp, _vp, _sz,
+                                    _vp, _vp]),
 }
 EXPORTS = tuple(_SIGS)
 
@@ -226,3 +229,17 @@ def decode_attn_noalloc(cfg, plan_ptrs, cache_ptrs, lens, max_len, q, out, statu
     _check(lib().kvq_decode_attn_noalloc(ctypes.byref(cfg), _ptr(plan_ptrs), _ptr(cache_ptrs),
                                          _ptr(lens), batch, max_len, _ptr(q), _dtype_code(q), n_q,
                                          _ptr(out), _ptr(status), _stream()))
+
+
+def bf16_decode_workspace_bytes(batch, n_kv_heads, n_q_heads, max_len) -> int:
+    return lib().kvq_bf16_decode_workspace_bytes(batch, n_kv_heads, n_q_heads, max_len)
+
+
+def bf16_decode_attn(k, v, lens, max_len, q, out, ws, status):
+    """bf16 comparator (not the method): dense split-K decode attention over
+    k, v [batch, n_kv, cap, 128] bf16 with q [batch, n_q, 128] bf16 into out
+    [batch, n_q, 128] fp32."""
+    batch, n_kv, cap = k.shape[0], k.shape[1], k.shape[2]
+    _check(lib().kvq_bf16_decode_attn(_ptr(k), _ptr(v), _ptr(lens), batch, n_kv, cap, max_len,
+                                      _ptr(q), q.shape[1], _ptr(out), _ptr(ws),
+                                      ws.numel() * ws.element_size(), _ptr(status), _stream()))

@@ -310,6 +310,27 @@ KVQ_API int kvq_append_decode(const kvq_cfg* cfg, const void* const* plans_dev, 
                               kvq_stream_t stream);
 
 /*
+ * bf16 comparator (not part of the method): split-K decode attention over an
+ * unquantized bf16 cache, built like kvq_decode_attn, to measure the packed
+ * path against the dense one on the same shapes ("RoPE-Aware Bit Allocation
+ * for KV-Cache Quantization", abstract, compares with fp16 FlashAttention2).
+ * k_dev, v_dev: bf16 [batch][n_kv_heads][cap_tokens][128], 16-byte aligned.
+ * len_dev: int32 [batch], each <= min(max_len, cap_tokens) (larger values
+ *        are clamped and flag CAPACITY).
+ * q_dev: bf16 [batch][n_q_heads][128], 4-byte aligned; out_dev: fp32
+ *        [batch][n_q_heads][128] = softmax(q k^T / sqrt(128)) v per head.
+ * ws_dev: >= kvq_bf16_decode_workspace_bytes(...) bytes, 16-byte aligned,
+ *        zero-filled once; same reuse rules as kvq_decode_attn.
+ * Returns KVQ_OK or a negative code.
+ */
+KVQ_API size_t kvq_bf16_decode_workspace_bytes(int batch, int n_kv_heads, int n_q_heads,
+                                               int64_t max_len);
+KVQ_API int kvq_bf16_decode_attn(const void* k_dev, const void* v_dev, const int32_t* len_dev,
+                                 int batch, int n_kv_heads, int64_t cap_tokens, int64_t max_len,
+                                 const void* q_dev, int n_q_heads, float* out_dev, void* ws_dev,
+                                 size_t ws_bytes, uint32_t* status_dev, kvq_stream_t stream);
+
+/*
  * Decode attention without a caller workspace. The paper has no counterpart:
  * this is a library convenience. Same computation, arguments and results as
  * kvq_decode_attn, minus ws_dev / ws_bytes.
