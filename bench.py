@@ -57,6 +57,8 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--layers", type=int, default=0,
                     help="override the layer count (small cases for profiling)")
+    ap.add_argument("--no-bf16", action="store_true",
+                    help="skip the bf16 comparator (dense decode over an unquantized cache)")
     return ap.parse_args()
 
 
@@ -221,8 +223,11 @@ def run_kvq(args, wl, rank, world, dist):
     cfg = kvq.make_cfg(wl.n_kv_heads, wl.bits_k, wl.bits_v, v_seed=1234)
     bpth = BYTES_PER_TOKEN_HEAD(wl.bits_k, wl.bits_v)
 
-    # ---- prefill: energies + greedy plans, bulk quantize-append (timed)
+    # ---- prefill: energies + greedy plans, bulk quantize-append (timed);
+    #      the same keys / values also fill the bf16 comparator's caches
+    #      ([batch][n_kv][cap][128] per layer)
     layers = []
+    dense_k, dense_v = [], []
     t_alloc = t_quant = 0.0
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for li in range(n_layers):
@@ -239,6 +244,13 @@ def run_kvq(args, wl, rank, world, dist):
         kall = torch.stack(ks)
         vall = torch.stack(vs)
         del ks, vs
+        if not args.no_bf16:
+            dk = torch.zeros(B, wl.n_kv_heads, cap, 128, dtype=torch.bfloat16, device=dev)
+            dv = torch.zeros_like(dk)
+            dk[:, :, :T].copy_(kall.permute(0, 2, 1, 3))
+            dv[:, :, :T].copy_(vall.permute(0, 2, 1, 3))
+            dense_k.append(dk)
+            dense_v.append(dv)
         ev0.record()
         L.append(kall, vall)
         ev1.record()
@@ -316,6 +328,46 @@ def run_kvq(args, wl, rank, world, dist):
         flags |= L.flags()
     assert flags == 0, f"status flags {flags}"
     value = world * bytes_step / (ms / 1e3) / 1e9
+
+    # ---- bf16 comparator: the same decode over the unquantized caches (one
+    #      dense launch per layer, lengths as in the packed step, graph)
+    bf16 = None
+    if not args.no_bf16:
+        dlen = torch.full((B,), int(layers[0].lens[0].item()), dtype=torch.int32, device=dev)
+        dws = torch.zeros(kvq.bf16_decode_workspace_bytes(B, wl.n_kv_heads, wl.n_q_heads, cap),
+                          dtype=torch.uint8, device=dev)
+        dstatus = torch.zeros(1, dtype=torch.int32, device=dev)
+        dout = torch.empty(n_layers, B, wl.n_q_heads, 128, dtype=torch.float32, device=dev)
+
+        def dense_step():
+            for li in range(n_layers):
+                kvq.bf16_decode_attn(dense_k[li], dense_v[li], dlen, cap, qs[li], dout[li], dws,
+                                     dstatus)
+
+        with torch.cuda.stream(stream):
+            for _ in range(warmup):
+                dense_step()
+            stream.synchronize()
+            dgraph = None
+            if not args.no_graph:
+                dgraph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(dgraph, stream=stream):
+                    dense_step()
+            d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            d0.record(stream)
+            for _ in range(steps):
+                dgraph.replay() if dgraph is not None else dense_step()
+            d1.record(stream)
+            d1.synchronize()
+            dms = d0.elapsed_time(d1) / steps
+        assert int(dstatus.item()) == 0, "bf16 comparator status"
+        dbytes = n_layers * B * wl.n_kv_heads * 512 * int(dlen[0].item())
+        bf16 = {"kernel": "dense_decode_kernel (kvq_bf16_decode_attn, one launch per layer)",
+                "ms_per_step": dms, "value": world * dbytes / (dms / 1e3) / 1e9, "unit": "GB/s",
+                "bytes_per_step": dbytes, "cache_bytes": "512 B per token-head (bf16 K + V)",
+                "packed_step_speedup": dms / ms, "note": "decode only (no append)"}
+        del dense_k, dense_v
+        torch.cuda.empty_cache()
 
     # ---- decode kernel alone: events around each layer's decode call
     per_launch = []
@@ -402,6 +454,7 @@ def run_kvq(args, wl, rank, world, dist):
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "bf16_comparator": bf16,
         "gpu_launches": steps * n_layers,
         "clocks": clocks,
     }
