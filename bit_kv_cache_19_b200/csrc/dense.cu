@@ -19,7 +19,7 @@
 
 namespace kvq {
 
-constexpr int kDWarps = 4;
+constexpr int kDWarps = 6;
 constexpr int kDThreads = kDWarps * 32;
 constexpr int kDStages = 2;
 constexpr int kDRow = 272;                 // shared-memory row: 256 B of bf16 + 16 B pad
