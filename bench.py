@@ -63,6 +63,30 @@ def parse():
 
 
 # ------------------------------------------------------------------ helpers
+def rank_max(x, dist, device="cpu"):
+    """Max over ranks of a per-rank number (a job's time is its slowest
+    rank's); x itself without a process group."""
+    if dist is None:
+        return float(x)
+    import torch
+
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank, world, ms):
+    """Whole-job throughput: the units all ranks processed over the slowest
+    rank's time (weak scaling: every rank has the same per-GPU work)."""
+    return world * units_per_rank / (ms / 1e3)
+
+
+def rank_seed(seed, rank, b):
+    """Synthetic-data seed of sequence b on a rank: ranks hold different
+    sequences of the same shapes."""
+    return seed * 1000 + rank * 100 + b
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -234,7 +258,7 @@ def run_kvq(args, wl, rank, world, dist):
         L = PackedLayer(cfg, B, cap, device=dev, layer=li)
         ks, vs = [], []
         for b in range(B):
-            k, v = synth.keys_values_torch(wl, args.seed * 1000 + rank * 100 + b, li, T, dev)
+            k, v = synth.keys_values_torch(wl, rank_seed(args.seed, rank, b), li, T, dev)
             ks.append(k)
             vs.append(v)
         torch.cuda.synchronize()
@@ -316,10 +340,7 @@ def run_kvq(args, wl, rank, world, dist):
         torch.cuda.synchronize()
         clocks = sampler.stop()
         ms = e0.elapsed_time(e1) / steps
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = rank_max(ms, dist, dev)
     # packed bytes read per step: length grows by 1 per step
     lens_timed = [len_before + i + 1 for i in range(steps)]
     bytes_step = n_layers * B * wl.n_kv_heads * bpth * statistics.mean(lens_timed)
@@ -327,7 +348,7 @@ def run_kvq(args, wl, rank, world, dist):
     for L in layers:
         flags |= L.flags()
     assert flags == 0, f"status flags {flags}"
-    value = world * bytes_step / (ms / 1e3) / 1e9
+    value = job_rate(bytes_step, world, ms) / 1e9
 
     # ---- bf16 comparator: the same decode over the unquantized caches (one
     #      dense launch per layer, lengths as in the packed step, graph)
@@ -348,6 +369,8 @@ def run_kvq(args, wl, rank, world, dist):
             for _ in range(warmup):
                 dense_step()
             stream.synchronize()
+            if dist is not None:
+                dist.barrier()
             dgraph = None
             if not args.no_graph:
                 dgraph = torch.cuda.CUDAGraph()
@@ -360,10 +383,11 @@ def run_kvq(args, wl, rank, world, dist):
             d1.record(stream)
             d1.synchronize()
             dms = d0.elapsed_time(d1) / steps
+        dms = rank_max(dms, dist, dev)
         assert int(dstatus.item()) == 0, "bf16 comparator status"
         dbytes = n_layers * B * wl.n_kv_heads * 512 * int(dlen[0].item())
         bf16 = {"kernel": "dense_decode_kernel (kvq_bf16_decode_attn, one launch per layer)",
-                "ms_per_step": dms, "value": world * dbytes / (dms / 1e3) / 1e9, "unit": "GB/s",
+                "ms_per_step": dms, "value": job_rate(dbytes, world, dms) / 1e9, "unit": "GB/s",
                 "bytes_per_step": dbytes, "cache_bytes": "512 B per token-head (bf16 K + V)",
                 "packed_step_speedup": dms / ms, "note": "decode only (no append)"}
         del dense_k, dense_v
@@ -405,6 +429,8 @@ def run_kvq(args, wl, rank, world, dist):
         for _ in range(2):
             e2e_step()
         stream.synchronize()
+        if dist is not None:
+            dist.barrier()
         e2e_steps = max(3, steps // 2)
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         f0.record(stream)
@@ -415,11 +441,8 @@ def run_kvq(args, wl, rank, world, dist):
         e2e_ms = f0.elapsed_time(f1) / e2e_steps
     e2e_len = int(layers[0].lens[0].item())
     e2e_bytes = n_layers * B * wl.n_kv_heads * bpth * (e2e_len - e2e_steps / 2)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_val = world * e2e_bytes / (e2e_ms / 1e3) / 1e9
+    e2e_ms = rank_max(e2e_ms, dist, dev)
+    e2e_val = job_rate(e2e_bytes, world, e2e_ms) / 1e9
 
     if rank != 0:
         return
@@ -440,7 +463,7 @@ def run_kvq(args, wl, rank, world, dist):
                          "read once per step)",
                    "graph": graph is not None},
         "pct_of_8TBs": value / 8000.0 * 100,
-        "tokens_per_s": world * B / (ms / 1e3),
+        "tokens_per_s": job_rate(B, world, ms),
         "quantize_prefill": {"layer_tokens_per_s": n_tok_quant / t_quant,
                              "token_heads_per_s": n_tok_quant * wl.n_kv_heads / t_quant,
                              "seconds": t_quant, "alloc_bits_seconds": t_alloc},
