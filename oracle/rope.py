@@ -9,7 +9,13 @@ pairing), rotated by the angle pos * theta_j with theta_j = base^(-2j/d):
     (x_j, x_{j+64}) -> (x_j cos a - x_{j+64} sin a,  x_j sin a + x_{j+64} cos a)
 
 so that  RoPE(q, m) . RoPE(k, n) = sum_j q_j^T R(theta_j (n - m)) k_j,
-with q_j = (q_j, q_{j+64}). All arithmetic fp64.
+with q_j = (q_j, q_{j+64}). All arithmetic fp64, except rotate_f32, the
+recipe of the fused rotate-and-quantize path (pre-RoPE keys in, codes of the
+rotated keys out; a reading of ours, the pages give no RoPE arithmetic): the
+angles pos * theta_j in fp64, their cos and sin rounded once to fp32, then
+the 2-D rotation in fp32 with every product and sum rounded (no fused
+multiply-add), so the codes decided on the rotated values are exact on both
+sides.
 """
 import numpy as np
 
@@ -44,3 +50,19 @@ def block_terms(q, k, m, n, base: float) -> np.ndarray:
     k0 = k[:h] * c - k[h:] * s
     k1 = k[:h] * s + k[h:] * c
     return q[:h] * k0 + q[h:] * k1
+
+
+def rotate_f32(x, pos, base: float) -> np.ndarray:
+    """RoPE as the fused quantize path computes it (float32 result).
+
+    c = fp32(cos(pos theta_j)), s = fp32(sin(pos theta_j)) from fp64 angles;
+    a' = fp32(fp32(a c) - fp32(b s)), b' = fp32(fp32(a s) + fp32(b c)).
+    """
+    x32 = np.asarray(x, dtype=np.float32)
+    d = x32.shape[-1]
+    h = d // 2
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * thetas(base, d)
+    c = np.cos(ang).astype(np.float32)
+    s = np.sin(ang).astype(np.float32)
+    a, b = x32[..., :h], x32[..., h:]
+    return np.concatenate([a * c - b * s, a * s + b * c], axis=-1).astype(np.float32)

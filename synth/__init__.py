@@ -119,6 +119,19 @@ def keys_values(wl: Workload, seed: int, layer: int, kv_head: int, n_tokens: int
     return to_bf16_bits(k[start:]), to_bf16_bits(v[start:])
 
 
+def keys_pre_rope(wl: Workload, seed: int, layer: int, kv_head: int, n_tokens: int,
+                  start: int = 0) -> np.ndarray:
+    """bf16 bits of the same keys before RoPE (kappa of keys_values), positions
+    start..start+n-1: the input of the fused rotate-and-quantize path."""
+    total = start + n_tokens
+    rng = np.random.default_rng(_seq(wl.wid, seed, layer, kv_head))
+    sig = np.concatenate([block_sigmas(wl, seed, layer, kv_head)] * 2)
+    kappa = rng.standard_normal((total, D)) * sig[None, :]
+    out = rng.random((total, D)) < OUTLIER_P
+    kappa = np.where(out, kappa * OUTLIER_X, kappa)
+    return to_bf16_bits(kappa[start:])
+
+
 def queries(wl: Workload, seed: int, layer: int, seq: int, pos: int) -> np.ndarray:
     """bf16 bits q[n_q_heads, 128] rotated at position ``pos``."""
     rng = np.random.default_rng(_seq(wl.wid, seed, layer, 1000 + seq))

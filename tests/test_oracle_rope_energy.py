@@ -82,3 +82,32 @@ def test_energy_flags_and_saturation():
     assert fl == energy.FLAG_NONFINITE
     assert S[0][3] == 0
     assert S[0][4] == 2 ** 64 - 1
+
+
+# ---- the fp32 recipe of the fused rotate-and-quantize path
+@pytest.mark.parametrize("base", [1e4, 1e6])
+def test_rope_f32_close_to_fp64_and_blockwise(base):
+    rng = np.random.default_rng(9)
+    x = np.float32(rng.standard_normal((300, 128)) * 3).astype(np.float64)
+    pos = rng.integers(0, 600000, 300)
+    y32 = rope.rotate_f32(x, pos, base)
+    y64 = rope.rotate(x, pos, base)
+    assert y32.dtype == np.float32
+    # two fp32 products and one sum, each rounded, plus fp32 cos/sin: a few
+    # units of 2^-24 of the block magnitude
+    mag = np.sqrt(x[:, :64] ** 2 + x[:, 64:] ** 2)
+    err = np.maximum(np.abs(y32[:, :64] - y64[:, :64]), np.abs(y32[:, 64:] - y64[:, 64:]))
+    assert np.all(err <= 4 * 2.0 ** -24 * mag + 1e-30)
+    # block j only mixes coordinates j and j + 64
+    e = np.zeros(128)
+    e[7] = 1.0
+    z = rope.rotate_f32(e, 12345, base)
+    a = 12345 * float(base) ** (-2 * 7 / 128)
+    assert z[7] == np.float32(np.cos(a)) and z[71] == np.float32(np.sin(a))
+    assert np.count_nonzero(z) == 2
+
+
+def test_rope_f32_identity_at_position_zero():
+    rng = np.random.default_rng(10)
+    x = np.float32(rng.standard_normal((20, 128)))
+    assert np.array_equal(rope.rotate_f32(x, np.zeros(20), 5e5), x)
