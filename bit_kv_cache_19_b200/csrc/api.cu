@@ -22,7 +22,7 @@ cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches
                           int batch, int64_t max_len, const void* q, int q_dtype, int n_q, int n_kv,
                           int bits_k, int bits_v, float* out, void* ws, size_t ws_bytes,
                           uint32_t* status, cudaStream_t st, const void* k_new, const void* v_new,
-                          int kv_dtype, int n_new, int64_t cap, int early);
+                          int kv_dtype, int n_new, int64_t cap, int early, const double* theta);
 size_t dense_workspace_bytes_for(int batch, int n_kv, int n_q, int64_t max_len);
 cudaError_t launch_dense_decode(const void* k, const void* v, const int32_t* len, int batch,
                                 int n_kv, int64_t cap, int64_t max_len, const void* q, int n_q,
@@ -269,10 +269,11 @@ int kvq_alloc_bits(const kvq_cfg* cfg, int layer, const void* k_dev, int k_dtype
   return KVQ_OK;
 }
 
-int kvq_quantize_append(const kvq_cfg* cfg, const void* const* plans_dev, const void* k_dev,
-                        const void* v_dev, int dtype, int batch, int n_new, void* const* cache_dev,
-                        int32_t* len_dev, int64_t cap_tokens, uint32_t* status_dev,
-                        kvq_stream_t stream) {
+static int quantize_append_impl(const kvq_cfg* cfg, const void* const* plans_dev,
+                                const void* k_dev, const void* v_dev, int dtype, int batch,
+                                int n_new, void* const* cache_dev, int32_t* len_dev,
+                                int64_t cap_tokens, const double* theta, uint32_t* status_dev,
+                                kvq_stream_t stream) {
   int rc = check_cfg(cfg);
   if (rc) return rc;
   if (!plans_dev || !cache_dev || !len_dev || !status_dev)
@@ -297,9 +298,36 @@ int kvq_quantize_append(const kvq_cfg* cfg, const void* const* plans_dev, const 
   p.cap = cap_tokens;
   p.tile_bytes = tile_bytes(cfg->bits_k, cfg->bits_v);
   p.status = status_dev;
+  p.rope = theta ? 1 : 0;
+  for (int j = 0; j < 64; ++j) p.theta[j] = theta ? theta[j] : 0.0;
   cudaError_t e = launch_quantize_append(p, cfg->bits_v, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "quantize_append");
   return KVQ_OK;
+}
+
+// RoPE block frequencies theta_j = base^(-2j/128), fp64.
+static bool rope_thetas(double base, double* theta) {
+  if (!(base > 1.0) || !std::isfinite(base)) return false;
+  for (int j = 0; j < 64; ++j) theta[j] = std::pow(base, -2.0 * j / 128.0);
+  return true;
+}
+
+int kvq_quantize_append(const kvq_cfg* cfg, const void* const* plans_dev, const void* k_dev,
+                        const void* v_dev, int dtype, int batch, int n_new, void* const* cache_dev,
+                        int32_t* len_dev, int64_t cap_tokens, uint32_t* status_dev,
+                        kvq_stream_t stream) {
+  return quantize_append_impl(cfg, plans_dev, k_dev, v_dev, dtype, batch, n_new, cache_dev,
+                              len_dev, cap_tokens, nullptr, status_dev, stream);
+}
+
+int kvq_quantize_append_rope(const kvq_cfg* cfg, const void* const* plans_dev, const void* k_dev,
+                             const void* v_dev, int dtype, int batch, int n_new,
+                             void* const* cache_dev, int32_t* len_dev, int64_t cap_tokens,
+                             double rope_base, uint32_t* status_dev, kvq_stream_t stream) {
+  double theta[64];
+  if (!rope_thetas(rope_base, theta)) return fail(KVQ_ERR_ARG, "rope_base %g", rope_base);
+  return quantize_append_impl(cfg, plans_dev, k_dev, v_dev, dtype, batch, n_new, cache_dev,
+                              len_dev, cap_tokens, theta, status_dev, stream);
 }
 
 int kvq_decode_attn(const kvq_cfg* cfg, const void* const* plans_dev, const void* const* cache_dev,
@@ -325,7 +353,7 @@ int kvq_decode_attn(const kvq_cfg* cfg, const void* const* plans_dev, const void
                                 const_cast<int32_t*>(len_dev), batch, max_len, q_dev, q_dtype,
                                 n_q_heads, cfg->n_kv_heads, cfg->bits_k, cfg->bits_v, out_dev,
                                 ws_dev, ws_bytes, status_dev, reinterpret_cast<cudaStream_t>(stream),
-                                nullptr, nullptr, 0, 0, 0, 0);
+                                nullptr, nullptr, 0, 0, 0, 0, nullptr);
   if (e != cudaSuccess) return cuda_fail(e, "decode_attn");
   return KVQ_OK;
 }
@@ -334,7 +362,7 @@ int kvq_append_decode(const kvq_cfg* cfg, const void* const* plans_dev, const vo
                       const void* v_dev, int kv_dtype, int n_new, void* const* cache_dev,
                       int32_t* len_dev, int64_t cap_tokens, int batch, int64_t max_len,
                       const void* q_dev, int q_dtype, int n_q_heads, float* out_dev, void* ws_dev,
-                      size_t ws_bytes, int step_flags, uint32_t* status_dev,
+                      size_t ws_bytes, int step_flags, double rope_base, uint32_t* status_dev,
                       kvq_stream_t stream) {
   int rc = check_cfg(cfg);
   if (rc) return rc;
@@ -342,7 +370,11 @@ int kvq_append_decode(const kvq_cfg* cfg, const void* const* plans_dev, const vo
     return fail(KVQ_ERR_ARG, "null device pointer");
   if (n_new < 0 || n_new > 64) return fail(KVQ_ERR_ARG, "n_new %d not in 0..64", n_new);
   if (n_new > 0 && (!k_dev || !v_dev)) return fail(KVQ_ERR_ARG, "null k/v pointer");
-  if (step_flags & ~KVQ_STEP_EARLY) return fail(KVQ_ERR_ARG, "step_flags 0x%x", step_flags);
+  if (step_flags & ~(KVQ_STEP_EARLY | KVQ_STEP_ROPE))
+    return fail(KVQ_ERR_ARG, "step_flags 0x%x", step_flags);
+  double theta[64];
+  if ((step_flags & KVQ_STEP_ROPE) && !rope_thetas(rope_base, theta))
+    return fail(KVQ_ERR_ARG, "rope_base %g", rope_base);
   if (!dtype_ok(kv_dtype) || !dtype_ok(q_dtype)) return fail(KVQ_ERR_ARG, "bad dtype");
   if (batch < 1 || batch > 65535) return fail(KVQ_ERR_ARG, "batch %d", batch);
   if (max_len < 1 || max_len > 0x7FFFFFFF || cap_tokens < 0 || cap_tokens > 0x7FFFFFFF)
@@ -360,7 +392,8 @@ int kvq_append_decode(const kvq_cfg* cfg, const void* const* plans_dev, const vo
                                 max_len, q_dev, q_dtype, n_q_heads, cfg->n_kv_heads, cfg->bits_k,
                                 cfg->bits_v, out_dev, ws_dev, ws_bytes, status_dev,
                                 reinterpret_cast<cudaStream_t>(stream), k_dev, v_dev, kv_dtype,
-                                n_new, cap_tokens, (step_flags & KVQ_STEP_EARLY) ? 1 : 0);
+                                n_new, cap_tokens, (step_flags & KVQ_STEP_EARLY) ? 1 : 0,
+                                (step_flags & KVQ_STEP_ROPE) ? theta : nullptr);
   if (e != cudaSuccess) return cuda_fail(e, "append_decode");
   return KVQ_OK;
 }

@@ -81,6 +81,8 @@ struct QuantParams {
   int tile_bytes;
   int tiles_max;  // work items per (sequence, KV head)
   uint32_t* status;
+  int rope;           // keys are pre-RoPE: rotate each to its position first
+  double theta[64];   // RoPE block frequencies base^(-2j/128)
 };
 
 // ------------------------------------------------------------------ device

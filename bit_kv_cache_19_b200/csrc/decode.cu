@@ -80,6 +80,8 @@ struct DecodeParams {
   int kv_dtype, n_new;
   int64_t cap;
   int early;  // read lengths and stream tiles before waiting for the previous kernel
+  int rope;   // appended keys are pre-RoPE: rotate each to its position first
+  double theta[64];
   unsigned int* cnt_end;  // counters of pair k at cnt_end - (k + 1) * kCntStride
   float* part;            // [batch][n_kv][n_splits][G][132] = m, l, -, -, o[128]
   float* gpart;           // [batch][n_kv][n_groups][G][132]
@@ -96,6 +98,7 @@ struct alignas(128) Smem {
   unsigned long long setup_bar;
   uint32_t cls_lane[8][32];      // per (class, lane): first K word << 8 | bit shift
   alignas(16) float thr[kThrPad];  // decision thresholds (fused append only)
+  double theta[64];                // RoPE block frequencies (fused append of pre-RoPE keys)
   int8_t qj[kMaxHalf][4];        // per half step: block of MMA column c, or -1
   int len0, is_last;
   uint32_t flags;
@@ -289,6 +292,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
     if (thr_bytes) bulk_g2s(sm.thr, g_thr, thr_bytes, &sm.setup_bar);
     sm.flags = 0u;
   }
+  if (p.rope)
+    for (int i = tid; i < 64; i += kThreads) sm.theta[i] = p.theta[i];
   {  // this CTA's query rows into L2 while the previous kernel finishes
     const size_t esz = (p.q_dtype == KVQ_BF16 || p.q_dtype == KVQ_FP16) ? 2 : 4;
     const uintptr_t q0 =
@@ -422,7 +427,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
             (((size_t)b * p.n_new + (tile * kTile + pp - len0)) * p.n_kv + h) * kHeadDim;
         __half kn, vn;
         warp_token_pass<BV>(sm.plan, sm.thr, p.k_new, p.v_new, p.kv_dtype, row, lane, pp,
-                            kz + pp * kKzStride, sw, clear, kn, vn, flags);
+                            kz + pp * kKzStride, sw, clear, kn, vn, flags,
+                            p.rope ? sm.theta : nullptr, (int64_t)tile * kTile + pp);
         if (lane == 0) {
           nrm_new[pp] = kn;
           nrm_new[kTile + pp] = vn;
@@ -836,7 +842,8 @@ cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches
                           int batch, int64_t max_len, const void* q, int q_dtype, int n_q, int n_kv,
                           int bits_k, int bits_v, float* out, void* ws, size_t ws_bytes,
                           uint32_t* status, cudaStream_t st, const void* k_new,
-                          const void* v_new, int kv_dtype, int n_new, int64_t cap, int early) {
+                          const void* v_new, int kv_dtype, int n_new, int64_t cap, int early,
+                          const double* theta) {
   cudaError_t err = cudaSuccess;
   const int G = n_q / n_kv;
   const SplitPlan sp = decode_split_plan(batch, n_kv, G, bits_k, bits_v, max_len, &err, false);
@@ -865,6 +872,8 @@ cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches
   p.n_new = n_new;
   p.cap = cap;
   p.early = early;
+  p.rope = theta ? 1 : 0;
+  for (int j = 0; j < 64; ++j) p.theta[j] = theta ? theta[j] : 0.0;
   p.part = reinterpret_cast<float*>(ws);
   p.gpart = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + gpart_off);
   p.cnt_end = reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(ws) +

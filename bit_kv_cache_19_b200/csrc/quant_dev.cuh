@@ -88,20 +88,41 @@ __device__ __forceinline__ int code_of_w(const float* thr, float z) {
   return c;
 }
 
+// RoPE of the key held as kx[q] = k[lane + 32 q] at position pos (theta:
+// the 64 block frequencies, shared memory): angle pos theta_j in fp64, cos
+// and sin rounded once to fp32, the 2-D rotation of (k_j, k_{j+64}) in fp32
+// with every product and sum rounded. Block j = lane + 32 q pairs kx[q] with
+// kx[q + 2], both held by this lane.
+__device__ __forceinline__ void rope_f32(float (&kx)[4], const double* theta, int64_t pos,
+                                         int lane) {
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    double sd, cd;
+    sincos((double)pos * theta[lane + 32 * q], &sd, &cd);
+    const float c = (float)cd, s = (float)sd;
+    const float a = kx[q], b = kx[q + 2];
+    kx[q] = __fsub_rn(__fmul_rn(a, c), __fmul_rn(b, s));
+    kx[q + 2] = __fadd_rn(__fmul_rn(a, s), __fmul_rn(b, c));
+  }
+}
+
 // Pass 1 for the token at tile position p (row: element offset of its key /
-// value in k / v), value width BV. Writes kz_row[128], the token's value
+// value in k / v), value width BV. With theta (not null) the key is pre-RoPE
+// and is rotated to position pos first. Writes kz_row[128], the token's value
 // fields into `words` and returns the fp16 norms.
 template <int BV>
 __device__ __forceinline__ void warp_token_pass(const Plan& pl, const float* thr, const void* k,
                                                 const void* v, int dtype, size_t row, int lane,
                                                 int p, float* kz_row, uint32_t* words, bool clear,
-                                                __half& kn, __half& vn, uint32_t& flags) {
+                                                __half& kn, __half& vn, uint32_t& flags,
+                                                const double* theta = nullptr, int64_t pos = 0) {
   float kx[4], vx[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     kx[q] = load_as_float(k, dtype, row + lane + 32 * q);
     vx[q] = load_as_float(v, dtype, row + lane + 32 * q);
   }
+  if (theta) rope_f32(kx, theta, pos, lane);
   const bool kfin = __all_sync(0xffffffffu, isfinite(kx[0]) && isfinite(kx[1]) &&
                                                 isfinite(kx[2]) && isfinite(kx[3]));
   const bool vfin = __all_sync(0xffffffffu, isfinite(vx[0]) && isfinite(vx[1]) &&

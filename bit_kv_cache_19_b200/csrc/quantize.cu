@@ -102,8 +102,10 @@ __global__ void __launch_bounds__(256, 4) quantize_append_kernel(QuantParams p) 
   __shared__ float s_kz[kTile * kKzStride];
   __shared__ uint32_t s_words[kHeadDim * 16 + 1];  // + slack word for put_field
   __shared__ uint32_t s_flags;
+  __shared__ double s_theta[64];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   for (int i = threadIdx.x; i < KVQ_CB_N_THR; i += blockDim.x) s_thr[i] = c_thr[i];
+  for (int i = threadIdx.x; i < 64; i += blockDim.x) s_theta[i] = p.theta[i];
   if (threadIdx.x == 0) s_flags = 0;
   int cur = -1;  // (b, h) whose plan is in shared memory
   bool plan_ok = false;
@@ -155,7 +157,8 @@ __global__ void __launch_bounds__(256, 4) quantize_append_kernel(QuantParams p) 
           (((size_t)b * p.n_new + (tile * kTile + pp - len0)) * p.n_kv + h) * kHeadDim;
       __half kn, vn;
       warp_token_pass<BV>(pl, s_thr, p.k, p.v, p.dtype, row, lane, pp, s_kz + pp * kKzStride,
-                          s_words, clear, kn, vn, flags);
+                          s_words, clear, kn, vn, flags, p.rope ? s_theta : nullptr,
+                          (int64_t)tile * kTile + pp);
       if (lane == 0) {
         norms[pp] = kn;
         norms[kTile + pp] = vn;

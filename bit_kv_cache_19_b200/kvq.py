@@ -21,6 +21,7 @@ FLAG_CAPACITY, FLAG_NONFINITE, FLAG_NORM_SAT, FLAG_TIMEOUT, FLAG_BAD_PLAN = 1, 2
 BF16, FP16, FP32 = 0, 1, 2
 ALLOC_GREEDY, ALLOC_UNIFORM = 0, 1
 STEP_EARLY = 1
+STEP_ROPE = 2
 PLAN_BYTES = 1024
 PLAN_MAGIC = 0x5051564B
 
@@ -73,13 +74,16 @@ _SIGS = {
     "kvq_decode_attn": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i64, _vp, _i32, _i32,
                                _vp, _vp, _sz, _vp, _vp]),
     "kvq_append_decode": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i32, _vp, _vp, _i64,
-                                 _i32, _i64, _vp, _i32, _i32, _vp, _vp, _sz, _i32, _vp, _vp]),
+                                 _i32, _i64, _vp, _i32, _i32, _vp, _vp, _sz, _i32,
+                                 ctypes.c_double, _vp, _vp]),
     "kvq_decode_attn_noalloc": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i64, _vp, _i32,
                                        _i32, _vp, _vp, _vp]),
     "kvq_decode_noalloc_scratch_bytes": (_sz, []),
     "kvq_bf16_decode_workspace_bytes": (_sz, [_i32, _i32, _i32, _i64]),
     "kvq_bf16_decode_attn": (_i32, [_vp, _vp, _vp, _i32, _i32, _i64, _i64, _vp, _i32, _vp, _vp, _sz,
                                     _vp, _vp]),
+    "kvq_quantize_append_rope": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i32, _i32, _vp,
+                                        _vp, _i64, ctypes.c_double, _vp, _vp]),
 }
 EXPORTS = tuple(_SIGS)
 
@@ -196,6 +200,16 @@ def quantize_append(cfg, plan_ptrs, k, v, cache_ptrs, lens, cap_tokens, status):
                                      cap_tokens, _ptr(status), _stream()))
 
 
+def quantize_append_rope(cfg, plan_ptrs, k, v, cache_ptrs, lens, cap_tokens, rope_base, status):
+    """Fused RoPE + append: k [batch, n_new, n_kv, 128] holds pre-RoPE keys,
+    rotated to their cache positions before they are quantized."""
+    batch, n_new = k.shape[0], k.shape[1]
+    _check(lib().kvq_quantize_append_rope(ctypes.byref(cfg), _ptr(plan_ptrs), _ptr(k), _ptr(v),
+                                          _dtype_code(k), batch, n_new, _ptr(cache_ptrs),
+                                          _ptr(lens), cap_tokens, float(rope_base), _ptr(status),
+                                          _stream()))
+
+
 def decode_attn(cfg, plan_ptrs, cache_ptrs, lens, max_len, q, out, ws, status):
     """Packed-cache decode attention; q [batch, n_q, 128], out fp32 same shape."""
     batch, n_q = q.shape[0], q.shape[1]
@@ -205,19 +219,20 @@ def decode_attn(cfg, plan_ptrs, cache_ptrs, lens, max_len, q, out, ws, status):
 
 
 def append_decode(cfg, plan_ptrs, k, v, cache_ptrs, lens, cap_tokens, max_len, q, out, ws,
-                  status, step_flags=0):
+                  status, step_flags=0, rope_base=0.0):
     """Append k, v [batch, n_new, n_kv, 128] and decode q [batch, n_q, 128] in one launch.
 
     step_flags=STEP_EARLY: stream the caches before the previous kernel ends
-    (only when that kernel writes neither these caches nor these lengths)."""
+    (only when that kernel writes neither these caches nor these lengths);
+    STEP_ROPE: k holds pre-RoPE keys, rotated with base rope_base."""
     batch, n_q = q.shape[0], q.shape[1]
     n_new = 0 if k is None else k.shape[1]
     _check(lib().kvq_append_decode(ctypes.byref(cfg), _ptr(plan_ptrs), _ptr(k), _ptr(v),
                                    _dtype_code(k) if k is not None else BF16, n_new,
                                    _ptr(cache_ptrs), _ptr(lens), cap_tokens, batch, max_len,
                                    _ptr(q), _dtype_code(q), n_q, _ptr(out), _ptr(ws),
-                                   ws.numel() * ws.element_size(), step_flags, _ptr(status),
-                                   _stream()))
+                                   ws.numel() * ws.element_size(), step_flags,
+                                   float(rope_base), _ptr(status), _stream()))
 
 
 def decode_attn_noalloc(cfg, plan_ptrs, cache_ptrs, lens, max_len, q, out, status):

@@ -49,6 +49,12 @@ class PackedLayer:
         kvq.quantize_append(self.cfg, self.plan_ptrs, k, v, self.cache_ptrs, self.lens, self.cap,
                             self.status)
 
+    def append_rope(self, k_pre, v, rope_base):
+        """Pre-RoPE keys k_pre, values v [batch, n_new, n_kv, 128] (device):
+        each key is rotated to its cache position, then appended."""
+        kvq.quantize_append_rope(self.cfg, self.plan_ptrs, k_pre, v, self.cache_ptrs, self.lens,
+                                 self.cap, rope_base, self.status)
+
     def decode(self, q, out=None, ws=None, max_len=None):
         """q [batch, n_q, 128] -> fp32 [batch, n_q, 128]."""
         max_len = self.cap if max_len is None else max_len
@@ -60,7 +66,8 @@ class PackedLayer:
                         self.status)
         return out
 
-    def append_decode(self, k, v, q, out=None, ws=None, max_len=None, step_flags=0):
+    def append_decode(self, k, v, q, out=None, ws=None, max_len=None, step_flags=0,
+                      rope_base=0.0):
         """Fused serving step: append k, v [batch, n_new, n_kv, 128], then decode q."""
         max_len = self.cap if max_len is None else max_len
         if out is None:
@@ -68,7 +75,7 @@ class PackedLayer:
         if ws is None:
             ws = self.workspace(q.shape[1], max_len)
         kvq.append_decode(self.cfg, self.plan_ptrs, k, v, self.cache_ptrs, self.lens, self.cap,
-                          max_len, q, out, ws, self.status, step_flags)
+                          max_len, q, out, ws, self.status, step_flags, rope_base)
         return out
 
     def workspace(self, n_q: int, max_len: int):

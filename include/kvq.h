@@ -71,6 +71,7 @@ typedef struct CUstream_st* kvq_stream_t;
 
 /* kvq_append_decode step flags. */
 #define KVQ_STEP_EARLY 1u  /* see kvq_append_decode */
+#define KVQ_STEP_ROPE 2u   /* see kvq_append_decode */
 
 /* Allocation modes. */
 #define KVQ_ALLOC_GREEDY 0   /* Block-GTQ: greedy marginal-gain widths per RoPE block */
@@ -237,12 +238,31 @@ KVQ_API int kvq_codebook(int bits, float* centroids, float* thresholds, double* 
  *        cap_tokens is skipped (len unchanged) and CAPACITY is flagged.
  * status_dev: required.
  * Tokens already in a tile keep their bits; positions past the new length
- * are zero. Returns KVQ_OK or a negative code.
+ * are zero in a tile that held no tokens and otherwise keep their bits (zero
+ * in a cache that was zero-filled and only appended to). Returns KVQ_OK or
+ * a negative code.
  */
 KVQ_API int kvq_quantize_append(const kvq_cfg* cfg, const void* const* plans_dev, const void* k_dev,
                         const void* v_dev, int dtype, int batch, int n_new,
                         void* const* cache_dev, int32_t* len_dev, int64_t cap_tokens,
                         uint32_t* status_dev, kvq_stream_t stream);
+
+/*
+ * Fused RoPE + quantize-append: k_dev holds pre-RoPE keys;
+ * the key of the token at cache position t is first rotated by RoPE at
+ * position t with theta_j = rope_base^(-2j/128) (block j = coordinates j,
+ * j + 64): angles in fp64, cos and sin rounded once to fp32, the 2-D
+ * rotation in fp32 with every product and sum rounded. The rotated key is
+ * then quantized exactly as by kvq_quantize_append (the cache holds post-RoPE
+ * codes, so decode is unchanged). Same arguments otherwise; rope_base > 1.
+ * "RoPE-Aware Bit Allocation for KV-Cache Quantization", abstract: the keys
+ * enter the cache after RoPE; the rotation arithmetic is a reading of ours.
+ */
+KVQ_API int kvq_quantize_append_rope(const kvq_cfg* cfg, const void* const* plans_dev,
+                                     const void* k_dev, const void* v_dev, int dtype, int batch,
+                                     int n_new, void* const* cache_dev, int32_t* len_dev,
+                                     int64_t cap_tokens, double rope_base, uint32_t* status_dev,
+                                     kvq_stream_t stream);
 
 /*
  * Decode attention straight from the packed cache: for sequence b and query
@@ -300,14 +320,18 @@ KVQ_API int kvq_decode_attn(const kvq_cfg* cfg, const void* const* plans_dev,
  *                   the workspace); q, k_dev, v_dev, out and the rest of the
  *                   workspace are always read and written after it (q is
  *                   only prefetched into L2 before it, which reads no value).
+ *   KVQ_STEP_ROPE   k_dev holds pre-RoPE keys, rotated to their cache
+ *                   positions with base rope_base exactly as by
+ *                   kvq_quantize_append_rope (rope_base is ignored without
+ *                   this flag).
  * Returns KVQ_OK or a negative code.
  */
 KVQ_API int kvq_append_decode(const kvq_cfg* cfg, const void* const* plans_dev, const void* k_dev,
                               const void* v_dev, int kv_dtype, int n_new, void* const* cache_dev,
                               int32_t* len_dev, int64_t cap_tokens, int batch, int64_t max_len,
                               const void* q_dev, int q_dtype, int n_q_heads, float* out_dev,
-                              void* ws_dev, size_t ws_bytes, int step_flags, uint32_t* status_dev,
-                              kvq_stream_t stream);
+                              void* ws_dev, size_t ws_bytes, int step_flags, double rope_base,
+                              uint32_t* status_dev, kvq_stream_t stream);
 
 /*
  * bf16 comparator (not part of the method): split-K decode attention over an

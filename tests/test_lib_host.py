@@ -133,10 +133,16 @@ def test_argument_errors_without_gpu():
                              None) == kvq.ERR_ARG
     assert b"aligned" in L.kvq_last_error()
     assert L.kvq_append_decode(ctypes.byref(cfg), p, p, p, 0, 1, p, p, 10, 1, 10, p, 0, 16, p,
-                               p8, 1 << 30, 0, p, None) == kvq.ERR_ARG
+                               p8, 1 << 30, 0, 0.0, p, None) == kvq.ERR_ARG
     assert L.kvq_append_decode(ctypes.byref(cfg), p, p, p, 0, 1, p, p, 10, 1, 10, p, 0, 16, p,
-                               p, 1 << 30, 2, p, None) == kvq.ERR_ARG
+                               p, 1 << 30, 4, 0.0, p, None) == kvq.ERR_ARG
     assert b"step_flags" in L.kvq_last_error()
+    # RoPE: the base must exceed 1
+    assert L.kvq_append_decode(ctypes.byref(cfg), p, p, p, 0, 1, p, p, 10, 1, 10, p, 0, 16, p,
+                               p, 1 << 30, kvq.STEP_ROPE, 0.5, p, None) == kvq.ERR_ARG
+    assert b"rope_base" in L.kvq_last_error()
+    assert L.kvq_quantize_append_rope(ctypes.byref(cfg), p, p, p, 0, 1, 1, p, p, 10, 1.0, p,
+                                      None) == kvq.ERR_ARG
     assert L.kvq_quantize_append(ctypes.byref(cfg), p, p, p, 7, 1, 1, p, p, 10, p,
                                  None) == kvq.ERR_ARG
     # zero new tokens is a no-op
