@@ -52,11 +52,17 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--workload", default="qwen3b_128k",
-                    choices=["qwen3b_128k", "llama8b", "qwen7b_serve"])
+                    choices=["qwen3b_128k", "llama8b", "qwen7b_serve", "qwen3b_sweep"])
+    ap.add_argument("--context", type=int, default=0,
+                    help="override the context length (points of the qwen3b_sweep)")
+    ap.add_argument("--alloc", default="greedy", choices=["greedy", "uniform"],
+                    help="Block-GTQ greedy widths, or every block at the key budget")
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--layers", type=int, default=0,
                     help="override the layer count (small cases for profiling)")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the timed oracle sample (sweep points)")
     ap.add_argument("--no-bf16", action="store_true",
                     help="skip the bf16 comparator (dense decode over an unquantized cache)")
     return ap.parse_args()
@@ -241,10 +247,12 @@ def run_kvq(args, wl, rank, world, dist):
     from bit_kv_cache_19_b200.runtime import PackedLayer
 
     dev = torch.device("cuda", torch.cuda.current_device())
-    n_layers, B, T = args.layers or wl.n_layers, wl.batch, wl.context
+    n_layers, B, T = args.layers or wl.n_layers, wl.batch, args.context or wl.context
     steps, warmup = args.steps, args.warmup
-    cap = T + steps + warmup + 64
-    cfg = kvq.make_cfg(wl.n_kv_heads, wl.bits_k, wl.bits_v, v_seed=1234)
+    n_step = max(1, wl.n_new)  # tokens appended per sequence and layer in a step
+    cap = T + (steps + warmup + max(3, steps // 2) + 4) * n_step + 64
+    cfg = kvq.make_cfg(wl.n_kv_heads, wl.bits_k, wl.bits_v, v_seed=1234,
+                       alloc_mode=kvq.ALLOC_UNIFORM if args.alloc == "uniform" else kvq.ALLOC_GREEDY)
     bpth = BYTES_PER_TOKEN_HEAD(wl.bits_k, wl.bits_v)
 
     # ---- prefill: energies + greedy plans, bulk quantize-append (timed);
@@ -289,7 +297,7 @@ def run_kvq(args, wl, rank, world, dist):
     # the step's inputs (q, new k, new v of every layer) live in one device
     # buffer and its outputs in another, so that an end-to-end step moves
     # them with one host-to-device and one device-to-host copy
-    nq_el, nkv_el = B * wl.n_q_heads * 128, B * wl.n_kv_heads * 128
+    nq_el, nkv_el = B * wl.n_q_heads * 128, B * n_step * wl.n_kv_heads * 128
     per_layer = nq_el + 2 * nkv_el
     step_in = torch.empty(n_layers * per_layer, dtype=torch.bfloat16, device=dev)
     step_out = torch.empty(n_layers, B, wl.n_q_heads, 128, dtype=torch.float32, device=dev)
@@ -297,11 +305,11 @@ def run_kvq(args, wl, rank, world, dist):
     for li in range(n_layers):
         base = li * per_layer
         q = step_in[base:base + nq_el].view(B, wl.n_q_heads, 128)
-        k = step_in[base + nq_el:base + nq_el + nkv_el].view(B, 1, wl.n_kv_heads, 128)
-        v = step_in[base + nq_el + nkv_el:base + per_layer].view(B, 1, wl.n_kv_heads, 128)
+        k = step_in[base + nq_el:base + nq_el + nkv_el].view(B, n_step, wl.n_kv_heads, 128)
+        v = step_in[base + nq_el + nkv_el:base + per_layer].view(B, n_step, wl.n_kv_heads, 128)
         q.copy_(synth.queries_torch(wl, args.seed, li, B, T, dev))
-        k.copy_(torch.randn(B, 1, wl.n_kv_heads, 128, device=dev).to(torch.bfloat16))
-        v.copy_(torch.randn(B, 1, wl.n_kv_heads, 128, device=dev).to(torch.bfloat16))
+        k.copy_(torch.randn(B, n_step, wl.n_kv_heads, 128, device=dev).to(torch.bfloat16))
+        v.copy_(torch.randn(B, n_step, wl.n_kv_heads, 128, device=dev).to(torch.bfloat16))
         qs.append(q)
         knew.append(k)
         vnew.append(v)
@@ -325,24 +333,39 @@ def run_kvq(args, wl, rank, world, dist):
             with torch.cuda.graph(graph, stream=stream):
                 step()
         len_before = int(layers[0].lens[0].item())
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        stack_bytes = n_layers * B * wl.n_kv_heads * bpth * T
+        flush = (torch.zeros(2 * l2 // 4, dtype=torch.int32, device=dev)
+                 if stack_bytes < 4 * l2 else None)
         sampler = ClockSampler(dev.index)
         if dist is not None:
             dist.barrier()
         torch.cuda.synchronize()
         sampler.start()
         time.sleep(0.3)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(steps):
-            graph.replay() if graph is not None else step()
-        e1.record(stream)
-        e1.synchronize()
+        if flush is None:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(steps):
+                graph.replay() if graph is not None else step()
+            e1.record(stream)
+            e1.synchronize()
+            ms = e0.elapsed_time(e1) / steps
+        else:  # caches within 4x L2: flush it before each step, time the steps only
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(steps)]
+            for a, b_ in evs:
+                flush.add_(1)
+                a.record(stream)
+                graph.replay() if graph is not None else step()
+                b_.record(stream)
+            stream.synchronize()
+            ms = sum(a.elapsed_time(b_) for a, b_ in evs) / steps
         torch.cuda.synchronize()
         clocks = sampler.stop()
-        ms = e0.elapsed_time(e1) / steps
     ms = rank_max(ms, dist, dev)
     # packed bytes read per step: length grows by 1 per step
-    lens_timed = [len_before + i + 1 for i in range(steps)]
+    lens_timed = [len_before + (i + 1) * n_step for i in range(steps)]
     bytes_step = n_layers * B * wl.n_kv_heads * bpth * statistics.mean(lens_timed)
     flags = 0
     for L in layers:
@@ -440,13 +463,14 @@ def run_kvq(args, wl, rank, world, dist):
         f1.synchronize()
         e2e_ms = f0.elapsed_time(f1) / e2e_steps
     e2e_len = int(layers[0].lens[0].item())
-    e2e_bytes = n_layers * B * wl.n_kv_heads * bpth * (e2e_len - e2e_steps / 2)
+    e2e_bytes = n_layers * B * wl.n_kv_heads * bpth * (e2e_len - n_step * (e2e_steps - 1) / 2)
     e2e_ms = rank_max(e2e_ms, dist, dev)
     e2e_val = job_rate(e2e_bytes, world, e2e_ms) / 1e9
 
     if rank != 0:
         return
-    cpu = oracle_sample(wl, seconds_target=12.0, seed=args.seed) if world == 1 else None
+    cpu = (oracle_sample(wl, seconds_target=12.0, seed=args.seed)
+           if world == 1 and not args.no_cpu_baseline else None)
     n_tok_quant = n_layers * B * T
     line = {
         "metric": f"packed K{wl.bits_k}V{wl.bits_v} decode-attn HBM GB/s",
@@ -455,12 +479,16 @@ def run_kvq(args, wl, rank, world, dist):
         "dtype": "f16 mma, f32 accumulate (codes u8/u32)", "data": "synthetic",
         "config": {"workload": wl.name, "layers": n_layers, "q_heads": wl.n_q_heads,
                    "kv_heads": wl.n_kv_heads, "head_dim": 128, "context": T, "batch": B,
-                   "budget": f"K{wl.bits_k}V{wl.bits_v}", "alloc": "Block-GTQ greedy",
-                   "step": "per layer, one fused launch: quantize-append 1 token + packed "
-                           "decode attention",
-                   "l2": f"inputs larger than L2 ({n_layers}-layer packed cache "
-                         f"{n_layers * B * wl.n_kv_heads * bpth * T / 1e6:.0f} MB, each layer "
-                         "read once per step)",
+                   "budget": f"K{wl.bits_k}V{wl.bits_v}",
+                   "alloc": "Block-GTQ greedy" if args.alloc == "greedy" else "uniform",
+                   "appended_per_step": n_step,
+                   "step": f"per layer, one fused launch: quantize-append {n_step} token(s) "
+                           "per sequence + packed decode attention",
+                   "l2": (f"inputs larger than L2 ({n_layers}-layer packed cache "
+                          f"{stack_bytes / 1e6:.0f} MB, each layer read once per step)"
+                          if flush is None else
+                          f"L2 flushed before each timed step ({n_layers}-layer packed cache "
+                          f"{stack_bytes / 1e6:.0f} MB < 4x L2)"),
                    "graph": graph is not None},
         "pct_of_8TBs": value / 8000.0 * 100,
         "tokens_per_s": job_rate(B, world, ms),
