@@ -33,11 +33,15 @@
 // * Values: P' = p * n^V (fp16) moves from the accumulator layout to the B
 //   operand with movmatrix; O^T(128 x G) += Vhat^T(128 x 16 tokens) P'^T with
 //   A registers holding one rotated coordinate of two tokens.
-// * Merge: the 8 warps merge in shared memory; the last CTA of each group of
-//   16 splits merges the group; the last group merges the groups, undoes the
-//   value rotation (inverse Walsh-Hadamard, signs) and writes o / l.
-//   Arrivals are counted on workspace counters (acquire-release atomics)
-//   that wrap to zero at the last arrival.
+// * Merge: the 8 warps merge in shared memory into the split's record; per
+//   query head the split adds 2^(m - 32 k) (l, o), k = floor(m / 32), to
+//   exponent bucket k by L2 atomics (float, vector); the last of the pair's
+//   splits to arrive (one acquire-release counter) sums the few buckets in
+//   use with weights 2^(32 (k - k_max)), clears them, undoes the value
+//   rotation (inverse Walsh-Hadamard, signs) and writes o / l. A split max
+//   outside [-256, 256) makes the last split merge all records instead. The
+//   sum order of the atomics varies, so outputs agree run to run to fp32
+//   rounding, not bit for bit.
 #include <algorithm>
 #include <cstddef>
 #include <atomic>
@@ -60,6 +64,7 @@ constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kStages = 2;
 constexpr int kMaxHalf = 24;  // half steps of <= 4 blocks (<= 64/4 + 8)
+constexpr int kBuckets = 16;  // split maxima m in [32 (k - 8), 32 (k - 7)), k = 0..15
 constexpr int kFallbackSlots = 1024;                  // CTA slots when no device answers
 constexpr int kMaxNew = 64;                           // tokens appended by a fused call
 constexpr int kScratch = 16640;  // q' staging; append: kz [32][129] fp32 + 64 fp16 norms
@@ -84,7 +89,7 @@ struct DecodeParams {
   double theta[64];
   unsigned int* cnt_end;  // counters of pair k at cnt_end - (k + 1) * kCntStride
   float* part;            // [batch][n_kv][n_splits][G][132] = m, l, -, -, o[128]
-  float* gpart;           // [batch][n_kv][n_groups][G][132]
+  float* bkt;             // [batch][n_kv][G][kBuckets][132]: exponent buckets
   float* out;             // [batch][n_q][128]
   uint32_t* status;
 };
@@ -116,6 +121,13 @@ __device__ __forceinline__ uint32_t ld32s(const uint8_t* p) {
 }
 __device__ __forceinline__ uint32_t ld16s(const uint8_t* p) {
   return *reinterpret_cast<const uint16_t*>(p);
+}
+
+// Vector float reduction in L2 (no return value).
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
 }
 
 // Four fp16 pairs from the 4 pair fields (2W bits each) that start at bit
@@ -660,29 +672,93 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
       }
     }
   __syncthreads();
+  // ---- this split's record, then its contribution to the exponent buckets:
+  //      head hd with max m adds 2^(m - 32 kk) (l, o), kk = floor(m / 32), to
+  //      bucket kk by L2 atomics, so the splits are summed in L2 without a
+  //      merge tree; a max outside [-256, 256) flags the pair for a merge of
+  //      all records instead
   float* const my_part = p.part + (bh * p.n_splits + split) * G * kPartStride;
-  merge_records<kThreads>(mg, kWarps, (size_t)8 * NT * kPartStride, G, my_part);
-
-  // ---- level 1: the last CTA of this group of splits merges the group
-  const int grp = split / kGroup;
-  const int g_lo = grp * kGroup, g_n = min(kGroup, p.n_splits - g_lo);
+  float* const crec = reinterpret_cast<float*>(scratch);  // [G][132]
+  merge_records<kThreads>(mg, kWarps, (size_t)8 * NT * kPartStride, G, crec);
   __syncthreads();
-  if (tid == 0) sm.is_last = arrive_last(&cnt[1 + grp], (unsigned int)g_n);
+  unsigned int* const ovf = cnt + 1;
+  unsigned int* const bmask = cnt + 2;  // [G]: buckets in use
+  float* const bkt = p.bkt + bh * (size_t)G * kBuckets * kPartStride;
+  for (int item = tid; item < G * 32; item += kThreads) {
+    const int hd = item >> 5, x4 = (item & 31) * 4;
+    const float* r = crec + hd * kPartStride;
+    const float4 ov = *reinterpret_cast<const float4*>(r + kRecO + x4);
+    const float m = r[0], l = r[1];
+    *reinterpret_cast<float4*>(my_part + hd * kPartStride + kRecO + x4) = ov;
+    if (x4 == 0) {
+      my_part[hd * kPartStride] = m;
+      my_part[hd * kPartStride + 1] = l;
+    }
+    if (m == -INFINITY) continue;  // no tokens in this split
+    const float kf = floorf(m * (1.f / 32.f));
+    if (!(kf >= -8.f && kf < 8.f)) {
+      if (x4 == 0) atomicOr(ovf, 1u);
+      continue;
+    }
+    const int kk = (int)kf + 8;
+    const float sc = ex2(m - 32.f * kf);  // in [1, 2^32)
+    float* dst = bkt + (hd * kBuckets + kk) * kPartStride;
+    red_add_v4(dst + kRecO + x4, ov.x * sc, ov.y * sc, ov.z * sc, ov.w * sc);
+    if (x4 == 0) {
+      atomicAdd(dst + 1, l * sc);
+      atomicOr(bmask + hd, 1u << kk);
+    }
+  }
+  __syncthreads();
+  if (tid == 0) sm.is_last = arrive_last(&cnt[0], (unsigned int)p.n_splits);
   __syncthreads();
   if (!sm.is_last) return;
-  float* my_gpart = p.gpart + (bh * p.n_groups + grp) * G * kPartStride;
-  merge_records<kThreads>(p.part + (bh * p.n_splits + g_lo) * G * kPartStride, g_n,
-                (size_t)G * kPartStride, G, my_gpart);
 
-  // ---- level 2: the last group merges the groups and writes o / l
+  // ---- the last split of the pair: sum the buckets (or merge all records),
+  //      clear what this call used, undo the value rotation, write o / l.
+  //      Reads go to L2 (ld.cg): the atomics were performed there.
+  float* fin = reinterpret_cast<float*>(stage_base);  // [G][132]
+  const bool overflow = __ldcg(ovf) != 0u;
+  if (!overflow) {
+    for (int item = tid; item < G * 32; item += kThreads) {
+      const int hd = item >> 5, x4 = (item & 31) * 4;
+      const unsigned int mask = __ldcg(bmask + hd);
+      float L = 0.f;
+      float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (mask) {
+        const int kmax = 31 - __clz(mask);
+        for (unsigned int mm = mask; mm; mm &= mm - 1u) {
+          const int kk = __ffs(mm) - 1;
+          const float w = ex2(32.f * (float)(kk - kmax));  // 2^(-32 j), exact
+          const float* src = bkt + (hd * kBuckets + kk) * kPartStride;
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(src + kRecO + x4));
+          O.x += w * v.x;
+          O.y += w * v.y;
+          O.z += w * v.z;
+          O.w += w * v.w;
+          if (x4 == 0) L += w * __ldcg(src + 1);
+        }
+      }
+      *reinterpret_cast<float4*>(fin + hd * kPartStride + kRecO + x4) = O;
+      if (x4 == 0) fin[hd * kPartStride + 1] = L;
+    }
+  } else {
+    merge_records<kThreads>(p.part + bh * p.n_splits * G * kPartStride, p.n_splits,
+                            (size_t)G * kPartStride, G, fin);
+  }
   __syncthreads();
-  if (tid == 0) sm.is_last = arrive_last(&cnt[0], (unsigned int)p.n_groups);
+  for (int item = tid; item < G * 32; item += kThreads) {
+    const int hd = item >> 5, x4 = (item & 31) * 4;
+    const unsigned int mask = __ldcg(bmask + hd);
+    for (unsigned int mm = mask; mm; mm &= mm - 1u) {
+      float* dst = bkt + (hd * kBuckets + __ffs(mm) - 1) * kPartStride;
+      *reinterpret_cast<float4*>(dst + kRecO + x4) = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (x4 == 0) dst[1] = 0.f;
+    }
+  }
   __syncthreads();
-  if (!sm.is_last) return;
-  float* fin = reinterpret_cast<float*>(stage_base);  // [16][132]
-  merge_records<kThreads>(p.gpart + bh * p.n_groups * G * kPartStride, p.n_groups, (size_t)G * kPartStride,
-                G, fin);
-  __syncthreads();
+  if (tid < G) bmask[tid] = 0u;
+  if (tid == 0) *ovf = 0u;
   for (int head = warp; head < G; head += kWarps) {
     const float* r = fin + (size_t)head * kPartStride;
     const float inv = r[1] > 0.f ? 1.f / (128.f * r[1]) : 0.f;
@@ -782,14 +858,14 @@ static SplitPlan decode_split_plan(int batch, int n_kv, int G, int bits_k, int b
 
 static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-// Workspace: split records | group records | ... | counters (at the end: pair
+// Workspace: split records | exponent buckets | ... | counters (at the end: pair
 // k at a fixed distance from the end, so calls sharing one workspace, for one
 // n_kv_heads, never overwrite each other's counters).
 static size_t decode_workspace_layout(int batch, int n_kv, int G, const SplitPlan& sp,
                                       size_t* gpart_off) {
   const size_t pairs = (size_t)batch * n_kv;
   const size_t part = align256(pairs * sp.n_splits * G * kPartStride * sizeof(float));
-  const size_t gpart = align256(pairs * sp.n_groups * G * kPartStride * sizeof(float));
+  const size_t gpart = align256(pairs * G * kBuckets * kPartStride * sizeof(float));
   const size_t counters = align256(pairs * kCntStride * sizeof(unsigned int));
   if (gpart_off) *gpart_off = part;
   return part + gpart + counters;
@@ -875,7 +951,7 @@ cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches
   p.rope = theta ? 1 : 0;
   for (int j = 0; j < 64; ++j) p.theta[j] = theta ? theta[j] : 0.0;
   p.part = reinterpret_cast<float*>(ws);
-  p.gpart = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + gpart_off);
+  p.bkt = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + gpart_off);
   p.cnt_end = reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(ws) +
                                               (ws_bytes & ~size_t(3)));
   p.out = out;

@@ -317,8 +317,8 @@ def test_fused_append_decode(n_new, bits, flags):
 def test_early_prefetch_layer_loop_matches_plain():
     """A loop of fused steps over layers that share one workspace, launched
     with STEP_EARLY (each layer's caches streamed before the previous layer's
-    kernel has ended), gives the same outputs, lengths and packed caches bit
-    for bit as the same loop without it."""
+    kernel has ended), gives the same lengths and packed caches bit for bit,
+    and the same outputs to fp32 rounding, as the same loop without it."""
     rng = np.random.default_rng(77)
     n_kv, G, cap, n_layers, n_steps = 2, 8, 704, 3, 4
     starts = [300, 31, 640]
@@ -352,7 +352,11 @@ def test_early_prefetch_layer_loop_matches_plain():
             outs.append(o)
         torch.cuda.synchronize()
         for li in range(n_layers):
-            assert torch.equal(outs[0][li], outs[1][li]), (step, li)
+            # the split sums run through L2 atomics in arrival order: equal
+            # to fp32 rounding (the packed caches below are bit-exact)
+            a_, b_ = outs[0][li].double(), outs[1][li].double()
+            den = a_.abs().amax(dim=-1).clamp_min(1e-30)
+            assert float(((a_ - b_).abs().amax(dim=-1) / den).max()) <= 1e-5, (step, li)
             assert bool(torch.isfinite(outs[1][li]).all())
     for li in range(n_layers):
         a, b = sets[0][0][li], sets[1][0][li]
@@ -404,3 +408,27 @@ def test_chunked_appends_mixed_lengths(bits):
         _, heads = op.layer(kh, vh, bk, bv, 21, 4, E=E)
         for h in range(n_kv):
             check_records(L.head_records(s, h, (T + 31) // 32), heads[h]["rec"], T, bk, bv)
+
+
+def test_split_maxima_outside_bucket_range_take_the_record_merge():
+    """Queries large enough that split maxima leave the exponent-bucket range
+    [-256, 256) (base-2 logits): the last split merges all split records
+    instead; the output still matches the oracle, and the next call on the
+    same workspace (buckets and flags cleared) is right again."""
+    rng = np.random.default_rng(31)
+    n_kv, G, T = 2, 8, 3000
+    cfg = kvq.make_cfg(n_kv, 3, 3, v_seed=4)
+    L = PackedLayer(cfg, 1, 3072)
+    E, kb, vb = _random_layer(rng, n_kv, T, 1.0)
+    L.set_plans(kvq.plan_build(cfg, 0, E))
+    L.append(dev_bf16(kb)[None], dev_bf16(vb)[None])
+    kh, vh = op.bf16_heads(kb, vb)
+    _, heads = op.layer(kh, vh, 3, 3, 4, 0, E=E, pack=False)
+    ws = L.workspace(n_kv * G, 3072)
+    for scale in (400.0, 1.0, -400.0, 1.0):
+        qb = synth.to_bf16_bits(rng.standard_normal((1, n_kv * G, 128)) * scale)
+        out = L.decode(dev_bf16(qb), ws=ws).cpu().numpy()[0]
+        ref = op.decode(synth.bf16_bits_to_f64(qb[0]), heads)
+        assert np.isfinite(out).all(), scale
+        assert op.rel_err(out, ref) <= TOL, scale
+    assert L.flags() == 0
