@@ -104,7 +104,7 @@ def measured_peaks():
 
 def decode_source_hash():
     h = hashlib.sha256()
-    for f in ("decode.cu", "common.cuh"):
+    for f in ("decode.cu", "common.cuh", "splitk.cuh", "quant_dev.cuh"):
         with open(os.path.join(ROOT, "bit_kv_cache_19_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
