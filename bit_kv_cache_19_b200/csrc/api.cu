@@ -22,12 +22,15 @@ cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches
                           int batch, int64_t max_len, const void* q, int q_dtype, int n_q, int n_kv,
                           int bits_k, int bits_v, float* out, void* ws, size_t ws_bytes,
                           uint32_t* status, cudaStream_t st, const void* k_new, const void* v_new,
-                          int kv_dtype, int n_new, int64_t cap, int early, const double* theta);
+                          int kv_dtype, int n_new, int64_t cap, int early, const double* theta,
+                          float* rec_out);
 size_t dense_workspace_bytes_for(int batch, int n_kv, int n_q, int64_t max_len);
 cudaError_t launch_dense_decode(const void* k, const void* v, const int32_t* len, int batch,
                                 int n_kv, int64_t cap, int64_t max_len, const void* q, int n_q,
                                 float* out, void* ws, size_t ws_bytes, uint32_t* status,
                                 cudaStream_t st);
+cudaError_t launch_combine(const Plan* const* plans, const float* recs, int n_parts, int batch,
+                           int n_q, int n_kv, float* out, cudaStream_t st);
 
 namespace {
 
@@ -330,17 +333,27 @@ int kvq_quantize_append_rope(const kvq_cfg* cfg, const void* const* plans_dev, c
                               len_dev, cap_tokens, theta, status_dev, stream);
 }
 
-int kvq_decode_attn(const kvq_cfg* cfg, const void* const* plans_dev, const void* const* cache_dev,
-                    const int32_t* len_dev, int batch, int64_t max_len, const void* q_dev,
-                    int q_dtype, int n_q_heads, float* out_dev, void* ws_dev, size_t ws_bytes,
-                    uint32_t* status_dev, kvq_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// kvq_decode_attn and kvq_decode_attn_partial: exactly one of out_dev (final
+// outputs) and rec_out (merged records of this context shard) is set.
+int decode_impl(const kvq_cfg* cfg, const void* const* plans_dev, const void* const* cache_dev,
+                const int32_t* len_dev, int batch, int64_t max_len, const void* q_dev, int q_dtype,
+                int n_q_heads, float* out_dev, float* rec_out, void* ws_dev, size_t ws_bytes,
+                uint32_t* status_dev, kvq_stream_t stream) {
   int rc = check_cfg(cfg);
   if (rc) return rc;
-  if (!plans_dev || !cache_dev || !len_dev || !q_dev || !out_dev || !ws_dev || !status_dev)
+  if (!plans_dev || !cache_dev || !len_dev || !q_dev || !(out_dev || rec_out) || !ws_dev ||
+      !status_dev)
     return fail(KVQ_ERR_ARG, "null device pointer");
+  if (rec_out && (reinterpret_cast<uintptr_t>(rec_out) & 15))
+    return fail(KVQ_ERR_ARG, "records not 16-byte aligned");
   if (!dtype_ok(q_dtype)) return fail(KVQ_ERR_ARG, "q_dtype %d", q_dtype);
   if (batch < 1 || batch > 65535) return fail(KVQ_ERR_ARG, "batch %d", batch);
-  if (max_len < 1 || max_len > 0x7FFFFFFF) return fail(KVQ_ERR_ARG, "max_len %lld", (long long)max_len);
+  if (max_len < 1 || max_len > 0x7FFFFFFF)
+    return fail(KVQ_ERR_ARG, "max_len %lld", (long long)max_len);
   if (n_q_heads < 1 || n_q_heads % cfg->n_kv_heads != 0 || n_q_heads / cfg->n_kv_heads > 16)
     return fail(KVQ_ERR_ARG, "n_q_heads %d vs n_kv_heads %d", n_q_heads, cfg->n_kv_heads);
   if (reinterpret_cast<uintptr_t>(ws_dev) & 15)
@@ -353,8 +366,50 @@ int kvq_decode_attn(const kvq_cfg* cfg, const void* const* plans_dev, const void
                                 const_cast<int32_t*>(len_dev), batch, max_len, q_dev, q_dtype,
                                 n_q_heads, cfg->n_kv_heads, cfg->bits_k, cfg->bits_v, out_dev,
                                 ws_dev, ws_bytes, status_dev, reinterpret_cast<cudaStream_t>(stream),
-                                nullptr, nullptr, 0, 0, 0, 0, nullptr);
-  if (e != cudaSuccess) return cuda_fail(e, "decode_attn");
+                                nullptr, nullptr, 0, 0, 0, 0, nullptr, rec_out);
+  if (e != cudaSuccess) return cuda_fail(e, rec_out ? "decode_attn_partial" : "decode_attn");
+  return KVQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kvq_decode_attn(const kvq_cfg* cfg, const void* const* plans_dev, const void* const* cache_dev,
+                    const int32_t* len_dev, int batch, int64_t max_len, const void* q_dev,
+                    int q_dtype, int n_q_heads, float* out_dev, void* ws_dev, size_t ws_bytes,
+                    uint32_t* status_dev, kvq_stream_t stream) {
+  if (!out_dev) return fail(KVQ_ERR_ARG, "null device pointer");
+  return decode_impl(cfg, plans_dev, cache_dev, len_dev, batch, max_len, q_dev, q_dtype, n_q_heads,
+                     out_dev, nullptr, ws_dev, ws_bytes, status_dev, stream);
+}
+
+int kvq_decode_attn_partial(const kvq_cfg* cfg, const void* const* plans_dev,
+                            const void* const* cache_dev, const int32_t* len_dev, int batch,
+                            int64_t max_len, const void* q_dev, int q_dtype, int n_q_heads,
+                            float* rec_dev, void* ws_dev, size_t ws_bytes, uint32_t* status_dev,
+                            kvq_stream_t stream) {
+  if (!rec_dev) return fail(KVQ_ERR_ARG, "null device pointer");
+  return decode_impl(cfg, plans_dev, cache_dev, len_dev, batch, max_len, q_dev, q_dtype, n_q_heads,
+                     nullptr, rec_dev, ws_dev, ws_bytes, status_dev, stream);
+}
+
+int kvq_combine_partials(const kvq_cfg* cfg, const void* const* plans_dev, int n_parts,
+                         const float* recs_dev, int batch, int n_q_heads, float* out_dev,
+                         kvq_stream_t stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (!plans_dev || !recs_dev || !out_dev) return fail(KVQ_ERR_ARG, "null device pointer");
+  if (reinterpret_cast<uintptr_t>(recs_dev) & 15)
+    return fail(KVQ_ERR_ARG, "records not 16-byte aligned");
+  if (n_parts < 1 || n_parts > 65535) return fail(KVQ_ERR_ARG, "n_parts %d", n_parts);
+  if (batch < 1 || batch > 65535) return fail(KVQ_ERR_ARG, "batch %d", batch);
+  if (n_q_heads < 1 || n_q_heads % cfg->n_kv_heads != 0 || n_q_heads / cfg->n_kv_heads > 16)
+    return fail(KVQ_ERR_ARG, "n_q_heads %d vs n_kv_heads %d", n_q_heads, cfg->n_kv_heads);
+  cudaError_t e = launch_combine(reinterpret_cast<const Plan* const*>(plans_dev), recs_dev,
+                                 n_parts, batch, n_q_heads, cfg->n_kv_heads, out_dev,
+                                 reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "combine_partials");
   return KVQ_OK;
 }
 
@@ -393,7 +448,7 @@ int kvq_append_decode(const kvq_cfg* cfg, const void* const* plans_dev, const vo
                                 cfg->bits_v, out_dev, ws_dev, ws_bytes, status_dev,
                                 reinterpret_cast<cudaStream_t>(stream), k_dev, v_dev, kv_dtype,
                                 n_new, cap_tokens, (step_flags & KVQ_STEP_EARLY) ? 1 : 0,
-                                (step_flags & KVQ_STEP_ROPE) ? theta : nullptr);
+                                (step_flags & KVQ_STEP_ROPE) ? theta : nullptr, nullptr);
   if (e != cudaSuccess) return cuda_fail(e, "append_decode");
   return KVQ_OK;
 }

@@ -91,6 +91,7 @@ struct DecodeParams {
   float* part;            // [batch][n_kv][n_splits][G][132] = m, l, -, -, o[128]
   float* bkt;             // [batch][n_kv][G][kBuckets][132]: exponent buckets
   float* out;             // [batch][n_q][128]
+  float* rec_out;         // partial decode: merged records [batch][n_q][132], no out
   uint32_t* status;
 };
 
@@ -740,7 +741,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
         }
       }
       *reinterpret_cast<float4*>(fin + hd * kPartStride + kRecO + x4) = O;
-      if (x4 == 0) fin[hd * kPartStride + 1] = L;
+      if (x4 == 0) {  // (L, O) are 2^-(32 (kmax - 8)) times the split sums
+        fin[hd * kPartStride] = mask ? 32.f * (float)(31 - __clz(mask) - 8) : -INFINITY;
+        fin[hd * kPartStride + 1] = L;
+      }
     }
   } else {
     merge_records<kThreads>(p.part + bh * p.n_splits * G * kPartStride, p.n_splits,
@@ -759,11 +763,40 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   __syncthreads();
   if (tid < G) bmask[tid] = 0u;
   if (tid == 0) *ovf = 0u;
+  if (p.rec_out) {  // partial decode: the merged record, still rotated
+    float* dst = p.rec_out + ((size_t)b * p.n_q + (size_t)h * G) * kPartStride;
+    for (int i = tid; i < G * kPartStride / 4; i += kThreads)
+      reinterpret_cast<float4*>(dst)[i] = reinterpret_cast<const float4*>(fin)[i];
+    return;
+  }
   for (int head = warp; head < G; head += kWarps) {
     const float* r = fin + (size_t)head * kPartStride;
     const float inv = r[1] > 0.f ? 1.f / (128.f * r[1]) : 0.f;
     warp_unrotate_store(r + kRecO, sm.plan, inv,
                         p.out + ((size_t)b * p.n_q + h * G + head) * kHeadDim, lane);
+  }
+}
+
+// Merge of the records of n_parts partial decodes (context shards of the same
+// sequences: part r's record of query head i at recs + (r * batch * n_q + i)
+// * 132) and the inverse value rotation, o = s . H o_rot / (128 l). One CTA per
+// (KV head, sequence).
+__global__ void __launch_bounds__(kThreads) combine_kernel(const Plan* const* plans,
+                                                           const float* recs, int n_parts,
+                                                           int batch, int n_q, int n_kv,
+                                                           float* out) {
+  __shared__ __align__(16) float fin[16 * kPartStride];
+  const int h = blockIdx.x, b = blockIdx.y, G = n_q / n_kv;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t head0 = (size_t)b * n_q + (size_t)h * G;
+  merge_records<kThreads>(recs + head0 * kPartStride, n_parts,
+                          (size_t)batch * n_q * kPartStride, G, fin);
+  __syncthreads();
+  const Plan& pl = plans[b][h];
+  for (int head = warp; head < G; head += kWarps) {
+    const float* r = fin + (size_t)head * kPartStride;
+    const float inv = r[1] > 0.f ? 1.f / (128.f * r[1]) : 0.f;
+    warp_unrotate_store(r + kRecO, pl, inv, out + (head0 + head) * kHeadDim, lane);
   }
 }
 
@@ -919,7 +952,7 @@ cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches
                           int bits_k, int bits_v, float* out, void* ws, size_t ws_bytes,
                           uint32_t* status, cudaStream_t st, const void* k_new,
                           const void* v_new, int kv_dtype, int n_new, int64_t cap, int early,
-                          const double* theta) {
+                          const double* theta, float* rec_out) {
   cudaError_t err = cudaSuccess;
   const int G = n_q / n_kv;
   const SplitPlan sp = decode_split_plan(batch, n_kv, G, bits_k, bits_v, max_len, &err, false);
@@ -955,9 +988,17 @@ cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches
   p.cnt_end = reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(ws) +
                                               (ws_bytes & ~size_t(3)));
   p.out = out;
+  p.rec_out = rec_out;
   p.status = status;
   return G <= 8 ? launch_decode_nt<1>(p, bits_v, batch, st)
                 : launch_decode_nt<2>(p, bits_v, batch, st);
+}
+
+cudaError_t launch_combine(const Plan* const* plans, const float* recs, int n_parts, int batch,
+                           int n_q, int n_kv, float* out, cudaStream_t st) {
+  combine_kernel<<<dim3(n_kv, batch), kThreads, 0, st>>>(plans, recs, n_parts, batch, n_q, n_kv,
+                                                         out);
+  return cudaGetLastError();
 }
 
 }  // namespace kvq

@@ -22,7 +22,8 @@ cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches
                           int batch, int64_t max_len, const void* q, int q_dtype, int n_q, int n_kv,
                           int bits_k, int bits_v, float* out, void* ws, size_t ws_bytes,
                           uint32_t* status, cudaStream_t st, const void* k_new, const void* v_new,
-                          int kv_dtype, int n_new, int64_t cap, int early, const double* theta);
+                          int kv_dtype, int n_new, int64_t cap, int early, const double* theta,
+                          float* rec_out);
 int set_last_error(int code, const char* msg);
 }  // namespace kvq
 
@@ -97,7 +98,7 @@ extern "C" KVQ_API int kvq_decode_attn_noalloc(const kvq_cfg* cfg, const void* c
                          const_cast<int32_t*>(len_dev), batch, max_len, q_dev, q_dtype, n_q_heads,
                          cfg->n_kv_heads, cfg->bits_k, cfg->bits_v, out_dev, scratch,
                          kScratchBytes, status_dev, reinterpret_cast<cudaStream_t>(stream),
-                         nullptr, nullptr, 0, 0, 0, 0, nullptr);
+                         nullptr, nullptr, 0, 0, 0, 0, nullptr, nullptr);
   if (e != cudaSuccess) return kvq::set_last_error(KVQ_ERR_CUDA, cudaGetErrorString(e));
   return KVQ_OK;
 }

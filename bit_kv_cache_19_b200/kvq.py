@@ -84,6 +84,9 @@ _SIGS = {
                                     _vp, _vp]),
     "kvq_quantize_append_rope": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i32, _i32, _vp,
                                         _vp, _i64, ctypes.c_double, _vp, _vp]),
+    "kvq_decode_attn_partial": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i64, _vp, _i32,
+                                       _i32, _vp, _vp, _sz, _vp, _vp]),
+    "kvq_combine_partials": (_i32, [ctypes.POINTER(Cfg), _vp, _i32, _vp, _i32, _i32, _vp, _vp]),
 }
 EXPORTS = tuple(_SIGS)
 
@@ -216,6 +219,29 @@ def decode_attn(cfg, plan_ptrs, cache_ptrs, lens, max_len, q, out, ws, status):
     _check(lib().kvq_decode_attn(ctypes.byref(cfg), _ptr(plan_ptrs), _ptr(cache_ptrs), _ptr(lens),
                                  batch, max_len, _ptr(q), _dtype_code(q), n_q, _ptr(out), _ptr(ws),
                                  ws.numel() * ws.element_size(), _ptr(status), _stream()))
+
+
+REC_FLOATS = 132  # partial-decode record: m, l, 2 unused, o_rot[128]
+
+
+def decode_attn_partial(cfg, plan_ptrs, cache_ptrs, lens, max_len, q, rec, ws, status):
+    """Decode over one context shard (caches holding a token range of each
+    sequence) into merged records rec fp32 [batch, n_q, 132]: (m, l, -, -,
+    o_rot) with 2^m l = sum_t 2^s_t and 2^m o_rot = sum_t 2^s_t v_rot_t."""
+    batch, n_q = q.shape[0], q.shape[1]
+    _check(lib().kvq_decode_attn_partial(ctypes.byref(cfg), _ptr(plan_ptrs), _ptr(cache_ptrs),
+                                         _ptr(lens), batch, max_len, _ptr(q), _dtype_code(q), n_q,
+                                         _ptr(rec), _ptr(ws), ws.numel() * ws.element_size(),
+                                         _ptr(status), _stream()))
+
+
+def combine_partials(cfg, plan_ptrs, recs, out):
+    """Merge the stacked records recs fp32 [n_parts, batch, n_q, 132] of the
+    shards of the same sequences and undo the value rotation into out fp32
+    [batch, n_q, 128]."""
+    n_parts, batch, n_q = recs.shape[0], recs.shape[1], recs.shape[2]
+    _check(lib().kvq_combine_partials(ctypes.byref(cfg), _ptr(plan_ptrs), n_parts, _ptr(recs),
+                                      batch, n_q, _ptr(out), _stream()))
 
 
 def append_decode(cfg, plan_ptrs, k, v, cache_ptrs, lens, cap_tokens, max_len, q, out, ws,

@@ -2,7 +2,8 @@
 
 ``PackedLayer`` owns, for one layer and a batch of sequences, the plan
 records, the packed caches, their pointer arrays, the lengths and the status
-word, and forwards to the three C-ABI calls.
+word, and forwards to the C-ABI calls; ``sharded_decode`` is the one
+exchange step of a decode whose context is split over ranks.
 """
 from __future__ import annotations
 
@@ -78,6 +79,32 @@ class PackedLayer:
                           max_len, q, out, ws, self.status, step_flags, rope_base)
         return out
 
+    def decode_partial(self, q, rec=None, ws=None, max_len=None):
+        """Decode over this layer's caches as one context shard: merged
+        records fp32 [batch, n_q, 132] (m, l, -, -, o_rot) for combine()."""
+        max_len = self.cap if max_len is None else max_len
+        if rec is None:
+            rec = torch.empty((q.shape[0], q.shape[1], kvq.REC_FLOATS), dtype=torch.float32,
+                              device=self.device)
+        if ws is None:
+            ws = self.workspace(q.shape[1], max_len)
+        kvq.decode_attn_partial(self.cfg, self.plan_ptrs, self.cache_ptrs, self.lens, max_len, q,
+                                rec, ws, self.status)
+        return rec
+
+    def combine(self, recs, out=None):
+        """Outputs fp32 [batch, n_q, 128] from the stacked records
+        [n_parts, batch, n_q, 132] of the shards of these sequences."""
+        if out is None:
+            out = torch.empty(recs.shape[1:3] + (128,), dtype=torch.float32, device=self.device)
+        kvq.combine_partials(self.cfg, self.plan_ptrs, recs, out)
+        return out
+
+    def decode_sharded(self, q, group=None, max_len=None):
+        """Context-sharded decode: this rank's caches hold one token range of
+        each sequence (ranks in sequence order); one all-gather of records."""
+        return sharded_decode(lambda: self.decode_partial(q, max_len=max_len), self.combine, group)
+
     def workspace(self, n_q: int, max_len: int):
         """Decode workspace, zero-filled (its arrival counters must start at 0)."""
         n = kvq.decode_workspace_bytes(self.cfg, self.batch, n_q, max_len)
@@ -93,3 +120,18 @@ class PackedLayer:
 
     def flags(self) -> int:
         return int(self.status.item()) & 0xFFFFFFFF
+
+
+def sharded_decode(partial, combine, group=None):
+    """One exchange step of a context-sharded decode.
+
+    partial() returns this rank's records [batch, n_q, 132] for its token
+    range; the records of all ranks are gathered in rank order (one
+    all-gather, a few KB per sequence) and combine(stacked) turns them into
+    the outputs over the whole context, identical on every rank."""
+    import torch.distributed as dist
+    rec = partial()
+    world = dist.get_world_size(group)
+    recs = torch.empty((world,) + tuple(rec.shape), dtype=rec.dtype, device=rec.device)
+    dist.all_gather(list(recs.unbind(0)), rec.contiguous(), group=group)
+    return combine(recs)

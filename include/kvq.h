@@ -165,8 +165,9 @@ KVQ_API size_t kvq_alloc_workspace_bytes(const kvq_cfg* cfg);
 /*
  * Workspace bytes kvq_decode_attn needs for `batch` sequences of at most
  * max_len tokens on the current device: split-K records (m, l, o[128]) per
- * (sequence, query head, split) and per group of 8 splits, and arrival
- * counters at the end. Without a usable device it returns an upper bound.
+ * (sequence, query head, split), 16 exponent buckets of the same shape per
+ * (sequence, query head), and arrival counters at the end. Without a usable
+ * device it returns an upper bound.
  * Returns 0 for invalid arguments.
  */
 KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cfg* cfg, int batch, int n_q_heads,
@@ -273,9 +274,11 @@ KVQ_API int kvq_quantize_append_rope(const kvq_cfg* cfg, const void* const* plan
  * v_hat = n^V (1/128) s . (H c_{bits_v}[codes])). Split-K over the context:
  * each CTA unpacks its tiles in registers, forms the logits of all G query
  * heads of its KV head, keeps an online softmax and accumulates P V in the
- * rotated value domain; the last CTAs to finish merge the splits (two
- * levels) and apply the inverse rotation. One kernel launch; fp32
- * accumulation.
+ * rotated value domain; each split adds its rescaled sums into exponent
+ * buckets in L2 and the last split of a (sequence, KV head) sums the
+ * buckets and applies the inverse rotation. One kernel launch; fp32
+ * accumulation; the atomic sum order varies, so repeated calls agree to fp32
+ * rounding, not bit for bit.
  * plans_dev, cache_dev: as for kvq_quantize_append.
  * len_dev: int32 [batch], each <= max_len (a larger value is clamped to
  *        max_len and flags CAPACITY). A sequence of length 0 gives o = 0.
@@ -296,6 +299,43 @@ KVQ_API int kvq_decode_attn(const kvq_cfg* cfg, const void* const* plans_dev,
                     int64_t max_len, const void* q_dev, int q_dtype, int n_q_heads,
                     float* out_dev, void* ws_dev, size_t ws_bytes, uint32_t* status_dev,
                     kvq_stream_t stream);
+
+/*
+ * Context-sharded decode (no counterpart in the pages, whose serving path
+ * runs on one GPU): a sequence whose cache is split by token ranges over
+ * several caches (e.g. one per GPU) is decoded by one kvq_decode_attn_partial
+ * per range and one kvq_combine_partials over their records. Softmax over
+ * the union of ranges is the log-sum-exp-weighted mix of the per-range
+ * results, so the combined output is the kvq_decode_attn output over all
+ * tokens (to fp32 rounding). Each range's cache is an ordinary cache
+ * holding that range's tokens (post-RoPE keys keep their global positions);
+ * len_dev holds the range lengths.
+ *
+ * kvq_decode_attn_partial: arguments as kvq_decode_attn, but instead of
+ *   outputs it writes one record per (sequence, query head) to rec_dev
+ *   (fp32 [batch][n_q_heads][132], 16-byte aligned): rec[0] = m,
+ *   rec[1] = l, rec[2..3] unused, rec[4..131] = o_rot, meaning
+ *   sum_t 2^(s_t - m) = l and sum_t 2^(s_t - m) n^V_t c[vcode_t] = o_rot over
+ *   the range's tokens, s_t the base-2 logit q.k_hat_t log2(e) / sqrt(128),
+ *   o_rot still in the rotated value domain. An empty range gives
+ *   m = -inf, l = 0, o_rot = 0. m is any reference exponent (not
+ *   necessarily the range's max); only 2^m (l, o_rot) is defined.
+ * kvq_combine_partials: recs_dev = the n_parts record arrays stacked
+ *   (fp32 [n_parts][batch][n_q_heads][132], 16-byte aligned, e.g. the result
+ *   of an all-gather); plans_dev as for kvq_decode_attn (the value signs);
+ *   out_dev fp32 [batch][n_q_heads][128] = s . H o_rot_total / (128 l_total)
+ *   after merging the records like split results; 0 where every range was
+ *   empty. One launch, no workspace.
+ * Both return KVQ_OK or a negative code.
+ */
+KVQ_API int kvq_decode_attn_partial(const kvq_cfg* cfg, const void* const* plans_dev,
+                                    const void* const* cache_dev, const int32_t* len_dev,
+                                    int batch, int64_t max_len, const void* q_dev, int q_dtype,
+                                    int n_q_heads, float* rec_dev, void* ws_dev, size_t ws_bytes,
+                                    uint32_t* status_dev, kvq_stream_t stream);
+KVQ_API int kvq_combine_partials(const kvq_cfg* cfg, const void* const* plans_dev, int n_parts,
+                                 const float* recs_dev, int batch, int n_q_heads, float* out_dev,
+                                 kvq_stream_t stream);
 
 /*
  * One serving step in one launch: kvq_quantize_append of n_new tokens per

@@ -75,3 +75,40 @@ def decode(q, k_hat_heads, v_hat_heads) -> np.ndarray:
     for h in range(hkv):
         out[h * G:(h + 1) * G] = attention(q[h * G:(h + 1) * G], k_hat_heads[h], v_hat_heads[h])
     return out
+
+
+# Context shards. Softmax over a sequence split into disjoint token ranges is
+# the log-sum-exp-weighted mix of the ranges' own softmax outputs; this is the
+# plain identity, written out in base 2 (the library keeps base-2 logits).
+def range_record(q, k_hat, v_hat):
+    """Statistics of one token range for one KV head; q[Hg, d].
+
+    lse2_h = log2 sum_t 2^{s_t}, s_t = q_h . k_hat_t log2(e) / sqrt d, and the
+    range's own output o_h = sum_t 2^{s_t - lse2_h} v_hat_t. An empty range
+    gives lse2 = -inf and o = 0."""
+    q = np.asarray(q, dtype=np.float64)
+    if k_hat.shape[0] == 0:
+        return np.full(q.shape[0], -np.inf), np.zeros_like(q)
+    s = q @ k_hat.T / np.sqrt(q.shape[-1]) * np.log2(np.e)
+    m = s.max(axis=1, keepdims=True)
+    w = np.exp2(s - m)
+    lse2 = m[:, 0] + np.log2(w.sum(axis=1))
+    return lse2, np.exp2(s - lse2[:, None]) @ v_hat
+
+
+def combine_ranges(lse2, o):
+    """Output over the union of disjoint ranges from their records.
+
+    lse2[R, Hg], o[R, Hg, d]: o = sum_r 2^{lse2_r - LSE} o_r with
+    LSE = log2 sum_r 2^{lse2_r}; ranges with lse2 = -inf add nothing, and if
+    every range is empty the output is 0."""
+    lse2 = np.asarray(lse2, dtype=np.float64)
+    o = np.asarray(o, dtype=np.float64)
+    m = lse2.max(axis=0)
+    out = np.zeros(o.shape[1:])
+    for h in range(lse2.shape[1]):
+        if m[h] == -np.inf:
+            continue
+        w = np.exp2(lse2[:, h] - m[h])
+        out[h] = (w[:, None] * o[:, h]).sum(axis=0) / w.sum()
+    return out

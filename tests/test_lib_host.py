@@ -145,6 +145,18 @@ def test_argument_errors_without_gpu():
                                       None) == kvq.ERR_ARG
     assert L.kvq_quantize_append(ctypes.byref(cfg), p, p, p, 7, 1, 1, p, p, 10, p,
                                  None) == kvq.ERR_ARG
+    # context shards: records must be given and 16-byte aligned; n_parts >= 1
+    assert L.kvq_decode_attn_partial(ctypes.byref(cfg), p, p, p, 1, 10, p, 0, 16, None, p,
+                                     1 << 30, p, None) == kvq.ERR_ARG
+    assert L.kvq_decode_attn_partial(ctypes.byref(cfg), p, p, p, 1, 10, p, 0, 16, p8, p,
+                                     1 << 30, p, None) == kvq.ERR_ARG
+    assert b"aligned" in L.kvq_last_error()
+    assert L.kvq_decode_attn_partial(ctypes.byref(cfg), p, p, p, 1, 10, p, 0, 16, p, p, 8, p,
+                                     None) == kvq.ERR_WORKSPACE
+    assert L.kvq_combine_partials(ctypes.byref(cfg), p, 0, p, 1, 16, p, None) == kvq.ERR_ARG
+    assert b"n_parts" in L.kvq_last_error()
+    assert L.kvq_combine_partials(ctypes.byref(cfg), p, 2, p8, 1, 16, p, None) == kvq.ERR_ARG
+    assert L.kvq_combine_partials(ctypes.byref(cfg), p, 2, p, 1, 15, p, None) == kvq.ERR_ARG
     # zero new tokens is a no-op
     assert L.kvq_quantize_append(ctypes.byref(cfg), p, None, None, 0, 1, 0, p, p, 10, p,
                                  None) == kvq.OK

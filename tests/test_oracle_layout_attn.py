@@ -130,3 +130,34 @@ def test_gqa_mapping():
     o = attn.decode(q, ks, vs)
     assert np.allclose(o[4], attn.attention(q[4:5], ks[1], vs[1])[0])
     assert np.allclose(o[2], attn.attention(q[2:3], ks[0], vs[0])[0])
+
+
+def test_range_records_combine_to_attention_over_all_tokens():
+    """Context shards: the combine of the ranges' records equals softmax
+    attention over every token (pinned to the textbook form above), for cut
+    points that leave empty and one-token ranges."""
+    from scipy.special import logsumexp
+    rng = np.random.default_rng(5)
+    T, Hg = 300, 4
+    q = rng.standard_normal((Hg, 128)) * 2.0
+    k = rng.standard_normal((T, 128))
+    v = rng.standard_normal((T, 128))
+    full = attn.attention(q, k, v)
+    for cuts in ([0, 0, 150, 300, 300], [0, 1, 2, 299, 300], [0, 77, 133, 134, 300]):
+        recs = [attn.range_record(q, k[a:b], v[a:b]) for a, b in zip(cuts[:-1], cuts[1:])]
+        lse = np.stack([r[0] for r in recs])
+        o = np.stack([r[1] for r in recs])
+        assert np.max(np.abs(attn.combine_ranges(lse, o) - full)) < 1e-12
+        for (a, b), l in zip(zip(cuts[:-1], cuts[1:]), lse):
+            if b > a:  # log2 sum 2^s from the library's natural-log logsumexp
+                s = q @ k[a:b].T / np.sqrt(128.0)
+                assert np.allclose(l, logsumexp(s, axis=1) / np.log(2.0), rtol=0, atol=1e-12)
+            else:
+                assert np.all(l == -np.inf)
+    # one token: lse2 is its own base-2 logit and the output its value
+    l1, o1 = attn.range_record(q, k[:1], v[:1])
+    assert np.allclose(l1, (q @ k[0]) / np.sqrt(128.0) * np.log2(np.e), rtol=0, atol=1e-12)
+    assert np.allclose(o1, np.broadcast_to(v[0], o1.shape), rtol=0, atol=1e-12)
+    # every range empty: output 0
+    le, oe = attn.range_record(q, k[:0], v[:0])
+    assert np.all(attn.combine_ranges(np.stack([le, le]), np.stack([oe, oe])) == 0.0)
