@@ -680,7 +680,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   //      all records instead
   float* const my_part = p.part + (bh * p.n_splits + split) * G * kPartStride;
   float* const crec = reinterpret_cast<float*>(scratch);  // [G][132]
-  merge_records<kThreads>(mg, kWarps, (size_t)8 * NT * kPartStride, G, crec);
+  merge_records<kThreads, kWarps>(mg, kWarps, (size_t)8 * NT * kPartStride, G, crec);
   __syncthreads();
   unsigned int* const ovf = cnt + 1;
   unsigned int* const bmask = cnt + 2;  // [G]: buckets in use
@@ -723,21 +723,42 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   if (!overflow) {
     for (int item = tid; item < G * 32; item += kThreads) {
       const int hd = item >> 5, x4 = (item & 31) * 4;
+      // the buckets around this split's own (the usual ones) are loaded
+      // together with the mask, saving a dependent round trip to L2
+      const float m_own = crec[hd * kPartStride];
+      const int k_own = m_own == -INFINITY ? 8 : (int)floorf(m_own * (1.f / 32.f)) + 8;
+      const int k0 = min(max(k_own - 1, 0), kBuckets - 3);
+      float4 pre[3];
+      float pl[3];
+#pragma unroll
+      for (int j = 0; j < 3; ++j) {
+        const float* src = bkt + (hd * kBuckets + k0 + j) * kPartStride;
+        pre[j] = __ldcg(reinterpret_cast<const float4*>(src + kRecO + x4));
+        pl[j] = x4 == 0 ? __ldcg(src + 1) : 0.f;
+      }
       const unsigned int mask = __ldcg(bmask + hd);
       float L = 0.f;
       float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
       if (mask) {
         const int kmax = 31 - __clz(mask);
         for (unsigned int mm = mask; mm; mm &= mm - 1u) {
-          const int kk = __ffs(mm) - 1;
+          const int kk = __ffs(mm) - 1, d = kk - k0;
           const float w = ex2(32.f * (float)(kk - kmax));  // 2^(-32 j), exact
-          const float* src = bkt + (hd * kBuckets + kk) * kPartStride;
-          const float4 v = __ldcg(reinterpret_cast<const float4*>(src + kRecO + x4));
+          float4 v;
+          float lv;
+          if (d >= 0 && d < 3) {
+            v = d == 0 ? pre[0] : d == 1 ? pre[1] : pre[2];
+            lv = d == 0 ? pl[0] : d == 1 ? pl[1] : pl[2];
+          } else {
+            const float* src = bkt + (hd * kBuckets + kk) * kPartStride;
+            v = __ldcg(reinterpret_cast<const float4*>(src + kRecO + x4));
+            lv = x4 == 0 ? __ldcg(src + 1) : 0.f;
+          }
           O.x += w * v.x;
           O.y += w * v.y;
           O.z += w * v.z;
           O.w += w * v.w;
-          if (x4 == 0) L += w * __ldcg(src + 1);
+          L += w * lv;
         }
       }
       *reinterpret_cast<float4*>(fin + hd * kPartStride + kRecO + x4) = O;

@@ -297,7 +297,7 @@ __global__ void __launch_bounds__(kDThreads, 1) dense_decode_kernel(const DenseP
     }
   __syncthreads();
   float* const my_part = p.part + (bh * p.n_splits + split) * G * kPartStride;
-  merge_records<kDThreads>(mg, kDWarps, (size_t)8 * NT * kPartStride, G, my_part);
+  merge_records<kDThreads, 8>(mg, kDWarps, (size_t)8 * NT * kPartStride, G, my_part);
 
   const int grp = split / kGroup;
   const int g_lo = grp * kGroup, g_n = min(kGroup, p.n_splits - g_lo);

@@ -54,9 +54,9 @@ __device__ __forceinline__ void grid_dep_launch() {
 // Merge n records per head (record s of head h at src + s * rec_stride +
 // h * kPartStride) into dst (record h at dst + h * kPartStride), for G heads.
 // 32 threads per head, 4 coordinates each: one pass with online rescaling
-// over chunks of 16 records whose loads are issued together, so a merge of
-// all heads costs about n / 16 load round trips.
-template <int NTHREADS>
+// over chunks of CHUNK records whose loads are issued together, so a merge of
+// all heads costs about n / CHUNK load round trips.
+template <int NTHREADS, int CHUNK = kMergeChunk>
 __device__ __forceinline__ void merge_records(const float* src, int n, size_t rec_stride, int G,
                                               float* dst) {
   for (int item = threadIdx.x; item < G * 32; item += NTHREADS) {
@@ -64,11 +64,11 @@ __device__ __forceinline__ void merge_records(const float* src, int n, size_t re
     const float* r = src + (size_t)head * kPartStride;
     float M = -INFINITY, L = 0.f;
     float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s0 = 0; s0 < n; s0 += kMergeChunk) {
-      float2 ml[kMergeChunk];
-      float4 oo[kMergeChunk];
+    for (int s0 = 0; s0 < n; s0 += CHUNK) {
+      float2 ml[CHUNK];
+      float4 oo[CHUNK];
 #pragma unroll
-      for (int k = 0; k < kMergeChunk; ++k) {
+      for (int k = 0; k < CHUNK; ++k) {
         const bool v = s0 + k < n;
         const float* q = r + (size_t)(v ? s0 + k : 0) * rec_stride;
         ml[k] = *reinterpret_cast<const float2*>(q);
@@ -77,7 +77,7 @@ __device__ __forceinline__ void merge_records(const float* src, int n, size_t re
       }
       float cm = M;
 #pragma unroll
-      for (int k = 0; k < kMergeChunk; ++k) cm = fmaxf(cm, ml[k].x);
+      for (int k = 0; k < CHUNK; ++k) cm = fmaxf(cm, ml[k].x);
       if (cm != -INFINITY) {
         const float a = ex2(M - cm);
         L *= a;
@@ -86,7 +86,7 @@ __device__ __forceinline__ void merge_records(const float* src, int n, size_t re
         O.z *= a;
         O.w *= a;
 #pragma unroll
-        for (int k = 0; k < kMergeChunk; ++k) {
+        for (int k = 0; k < CHUNK; ++k) {
           const float w = ex2(ml[k].x - cm);  // 0 for records past n
           L += w * ml[k].y;
           O.x += w * oo[k].x;
