@@ -719,36 +719,53 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   //      clear what this call used, undo the value rotation, write o / l.
   //      Reads go to L2 (ld.cg): the atomics were performed there.
   float* fin = reinterpret_cast<float*>(stage_base);  // [G][132]
-  const bool overflow = __ldcg(ovf) != 0u;
-  if (!overflow) {
-    for (int item = tid; item < G * 32; item += kThreads) {
+  // one round of L2 loads (ld.cg: the atomics were performed there): the
+  // overflow flag, each item's bucket mask, and the three buckets around this
+  // split's own for the item's head (the usual ones)
+  constexpr int kItems = (16 * 32 + kThreads - 1) / kThreads;  // items per thread
+  const unsigned int ovf_v = __ldcg(ovf);
+  unsigned int msk[kItems];
+  int k0[kItems];
+  float4 pre[kItems][3];
+  float pl[kItems][3];
+#pragma unroll
+  for (int it = 0; it < kItems; ++it) {
+    const int item = tid + it * kThreads;
+    msk[it] = 0u;
+    k0[it] = 0;
+    if (item < G * 32) {
       const int hd = item >> 5, x4 = (item & 31) * 4;
-      // the buckets around this split's own (the usual ones) are loaded
-      // together with the mask, saving a dependent round trip to L2
       const float m_own = crec[hd * kPartStride];
       const int k_own = m_own == -INFINITY ? 8 : (int)floorf(m_own * (1.f / 32.f)) + 8;
-      const int k0 = min(max(k_own - 1, 0), kBuckets - 3);
-      float4 pre[3];
-      float pl[3];
+      k0[it] = min(max(k_own - 1, 0), kBuckets - 3);
 #pragma unroll
       for (int j = 0; j < 3; ++j) {
-        const float* src = bkt + (hd * kBuckets + k0 + j) * kPartStride;
-        pre[j] = __ldcg(reinterpret_cast<const float4*>(src + kRecO + x4));
-        pl[j] = x4 == 0 ? __ldcg(src + 1) : 0.f;
+        const float* src = bkt + (hd * kBuckets + k0[it] + j) * kPartStride;
+        pre[it][j] = __ldcg(reinterpret_cast<const float4*>(src + kRecO + x4));
+        pl[it][j] = x4 == 0 ? __ldcg(src + 1) : 0.f;
       }
-      const unsigned int mask = __ldcg(bmask + hd);
+      msk[it] = __ldcg(bmask + hd);
+    }
+  }
+  if (ovf_v == 0u) {
+#pragma unroll
+    for (int it = 0; it < kItems; ++it) {
+      const int item = tid + it * kThreads;
+      if (item >= G * 32) continue;
+      const int hd = item >> 5, x4 = (item & 31) * 4;
+      const unsigned int mask = msk[it];
       float L = 0.f;
       float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
       if (mask) {
         const int kmax = 31 - __clz(mask);
         for (unsigned int mm = mask; mm; mm &= mm - 1u) {
-          const int kk = __ffs(mm) - 1, d = kk - k0;
+          const int kk = __ffs(mm) - 1, d = kk - k0[it];
           const float w = ex2(32.f * (float)(kk - kmax));  // 2^(-32 j), exact
           float4 v;
           float lv;
           if (d >= 0 && d < 3) {
-            v = d == 0 ? pre[0] : d == 1 ? pre[1] : pre[2];
-            lv = d == 0 ? pl[0] : d == 1 ? pl[1] : pl[2];
+            v = d == 0 ? pre[it][0] : d == 1 ? pre[it][1] : pre[it][2];
+            lv = d == 0 ? pl[it][0] : d == 1 ? pl[it][1] : pl[it][2];
           } else {
             const float* src = bkt + (hd * kBuckets + kk) * kPartStride;
             v = __ldcg(reinterpret_cast<const float4*>(src + kRecO + x4));
@@ -772,10 +789,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
                             (size_t)G * kPartStride, G, fin);
   }
   __syncthreads();
-  for (int item = tid; item < G * 32; item += kThreads) {
+  // clear the buckets this call used (the masks were read with the sums)
+#pragma unroll
+  for (int it = 0; it < kItems; ++it) {
+    const int item = tid + it * kThreads;
+    if (item >= G * 32) continue;
     const int hd = item >> 5, x4 = (item & 31) * 4;
-    const unsigned int mask = __ldcg(bmask + hd);
-    for (unsigned int mm = mask; mm; mm &= mm - 1u) {
+    for (unsigned int mm = msk[it]; mm; mm &= mm - 1u) {
       float* dst = bkt + (hd * kBuckets + __ffs(mm) - 1) * kPartStride;
       *reinterpret_cast<float4*>(dst + kRecO + x4) = make_float4(0.f, 0.f, 0.f, 0.f);
       if (x4 == 0) dst[1] = 0.f;
