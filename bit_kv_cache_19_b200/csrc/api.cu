@@ -18,7 +18,7 @@ cudaError_t launch_energy(const void* k, int dtype, int64_t n_tokens, int n_kv,
 cudaError_t launch_quantize_append(const QuantParams& p, int bits_v, cudaStream_t st);
 size_t decode_workspace_bytes_for(int batch, int n_q, int n_kv, int bits_k, int bits_v,
                                   int64_t max_len);
-cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches, int32_t* len,
+cudaError_t launch_decode(const Plan* const* plans, const CacheMap& cm, int32_t* len,
                           int batch, int64_t max_len, const void* q, int q_dtype, int n_q, int n_kv,
                           int bits_k, int bits_v, float* out, void* ws, size_t ws_bytes,
                           uint32_t* status, cudaStream_t st, const void* k_new, const void* v_new,
@@ -274,12 +274,12 @@ int kvq_alloc_bits(const kvq_cfg* cfg, int layer, const void* k_dev, int k_dtype
 
 static int quantize_append_impl(const kvq_cfg* cfg, const void* const* plans_dev,
                                 const void* k_dev, const void* v_dev, int dtype, int batch,
-                                int n_new, void* const* cache_dev, int32_t* len_dev,
+                                int n_new, const CacheMap& cm, int32_t* len_dev,
                                 int64_t cap_tokens, const double* theta, uint32_t* status_dev,
                                 kvq_stream_t stream) {
   int rc = check_cfg(cfg);
   if (rc) return rc;
-  if (!plans_dev || !cache_dev || !len_dev || !status_dev)
+  if (!plans_dev || !(cm.caches || cm.table) || !len_dev || !status_dev)
     return fail(KVQ_ERR_ARG, "null device pointer");
   if (!dtype_ok(dtype)) return fail(KVQ_ERR_ARG, "dtype %d", dtype);
   if (batch < 1 || batch > 65535) return fail(KVQ_ERR_ARG, "batch %d", batch);
@@ -296,7 +296,7 @@ static int quantize_append_impl(const kvq_cfg* cfg, const void* const* plans_dev
   p.batch = batch;
   p.n_new = n_new;
   p.n_kv = cfg->n_kv_heads;
-  p.caches = reinterpret_cast<uint8_t* const*>(cache_dev);
+  p.cm = cm;
   p.len = len_dev;
   p.cap = cap_tokens;
   p.tile_bytes = tile_bytes(cfg->bits_k, cfg->bits_v);
@@ -319,8 +319,9 @@ int kvq_quantize_append(const kvq_cfg* cfg, const void* const* plans_dev, const 
                         const void* v_dev, int dtype, int batch, int n_new, void* const* cache_dev,
                         int32_t* len_dev, int64_t cap_tokens, uint32_t* status_dev,
                         kvq_stream_t stream) {
-  return quantize_append_impl(cfg, plans_dev, k_dev, v_dev, dtype, batch, n_new, cache_dev,
-                              len_dev, cap_tokens, nullptr, status_dev, stream);
+  return quantize_append_impl(cfg, plans_dev, k_dev, v_dev, dtype, batch, n_new,
+                              contiguous_map(cache_dev), len_dev, cap_tokens, nullptr, status_dev,
+                              stream);
 }
 
 int kvq_quantize_append_rope(const kvq_cfg* cfg, const void* const* plans_dev, const void* k_dev,
@@ -329,8 +330,9 @@ int kvq_quantize_append_rope(const kvq_cfg* cfg, const void* const* plans_dev, c
                              double rope_base, uint32_t* status_dev, kvq_stream_t stream) {
   double theta[64];
   if (!rope_thetas(rope_base, theta)) return fail(KVQ_ERR_ARG, "rope_base %g", rope_base);
-  return quantize_append_impl(cfg, plans_dev, k_dev, v_dev, dtype, batch, n_new, cache_dev,
-                              len_dev, cap_tokens, theta, status_dev, stream);
+  return quantize_append_impl(cfg, plans_dev, k_dev, v_dev, dtype, batch, n_new,
+                              contiguous_map(cache_dev), len_dev, cap_tokens, theta, status_dev,
+                              stream);
 }
 
 }  // extern "C"
@@ -339,14 +341,14 @@ namespace {
 
 // kvq_decode_attn and kvq_decode_attn_partial: exactly one of out_dev (final
 // outputs) and rec_out (merged records of this context shard) is set.
-int decode_impl(const kvq_cfg* cfg, const void* const* plans_dev, const void* const* cache_dev,
+int decode_impl(const kvq_cfg* cfg, const void* const* plans_dev, const CacheMap& cm,
                 const int32_t* len_dev, int batch, int64_t max_len, const void* q_dev, int q_dtype,
                 int n_q_heads, float* out_dev, float* rec_out, void* ws_dev, size_t ws_bytes,
                 uint32_t* status_dev, kvq_stream_t stream) {
   int rc = check_cfg(cfg);
   if (rc) return rc;
-  if (!plans_dev || !cache_dev || !len_dev || !q_dev || !(out_dev || rec_out) || !ws_dev ||
-      !status_dev)
+  if (!plans_dev || !(cm.caches || cm.table) || !len_dev || !q_dev || !(out_dev || rec_out) ||
+      !ws_dev || !status_dev)
     return fail(KVQ_ERR_ARG, "null device pointer");
   if (rec_out && (reinterpret_cast<uintptr_t>(rec_out) & 15))
     return fail(KVQ_ERR_ARG, "records not 16-byte aligned");
@@ -361,13 +363,79 @@ int decode_impl(const kvq_cfg* cfg, const void* const* plans_dev, const void* co
   if (ws_bytes < kvq_decode_workspace_bytes(cfg, batch, n_q_heads, max_len))
     return fail(KVQ_ERR_WORKSPACE, "decode workspace %zu < %zu", ws_bytes,
                 kvq_decode_workspace_bytes(cfg, batch, n_q_heads, max_len));
-  cudaError_t e = launch_decode(reinterpret_cast<const Plan* const*>(plans_dev),
-                                reinterpret_cast<const uint8_t* const*>(cache_dev),
+  cudaError_t e = launch_decode(reinterpret_cast<const Plan* const*>(plans_dev), cm,
                                 const_cast<int32_t*>(len_dev), batch, max_len, q_dev, q_dtype,
                                 n_q_heads, cfg->n_kv_heads, cfg->bits_k, cfg->bits_v, out_dev,
                                 ws_dev, ws_bytes, status_dev, reinterpret_cast<cudaStream_t>(stream),
                                 nullptr, nullptr, 0, 0, 0, 0, nullptr, rec_out);
   if (e != cudaSuccess) return cuda_fail(e, rec_out ? "decode_attn_partial" : "decode_attn");
+  return KVQ_OK;
+}
+
+int append_decode_impl(const kvq_cfg* cfg, const void* const* plans_dev, const void* k_dev,
+                       const void* v_dev, int kv_dtype, int n_new, const CacheMap& cm,
+                       int32_t* len_dev, int64_t cap_tokens, int batch, int64_t max_len,
+                       const void* q_dev, int q_dtype, int n_q_heads, float* out_dev, void* ws_dev,
+                       size_t ws_bytes, int step_flags, double rope_base, uint32_t* status_dev,
+                       kvq_stream_t stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (!plans_dev || !len_dev || !q_dev || !out_dev || !ws_dev || !status_dev)
+    return fail(KVQ_ERR_ARG, "null device pointer");
+  if (n_new < 0 || n_new > 64) return fail(KVQ_ERR_ARG, "n_new %d not in 0..64", n_new);
+  if (n_new > 0 && (!k_dev || !v_dev)) return fail(KVQ_ERR_ARG, "null k/v pointer");
+  if (step_flags & ~(KVQ_STEP_EARLY | KVQ_STEP_ROPE))
+    return fail(KVQ_ERR_ARG, "step_flags 0x%x", step_flags);
+  double theta[64];
+  if ((step_flags & KVQ_STEP_ROPE) && !rope_thetas(rope_base, theta))
+    return fail(KVQ_ERR_ARG, "rope_base %g", rope_base);
+  if (!dtype_ok(kv_dtype) || !dtype_ok(q_dtype)) return fail(KVQ_ERR_ARG, "bad dtype");
+  if (batch < 1 || batch > 65535) return fail(KVQ_ERR_ARG, "batch %d", batch);
+  if (max_len < 1 || max_len > 0x7FFFFFFF || cap_tokens < 0 || cap_tokens > 0x7FFFFFFF)
+    return fail(KVQ_ERR_ARG, "max_len %lld / cap_tokens %lld", (long long)max_len,
+                (long long)cap_tokens);
+  if (n_q_heads < 1 || n_q_heads % cfg->n_kv_heads != 0 || n_q_heads / cfg->n_kv_heads > 16)
+    return fail(KVQ_ERR_ARG, "n_q_heads %d vs n_kv_heads %d", n_q_heads, cfg->n_kv_heads);
+  if (reinterpret_cast<uintptr_t>(ws_dev) & 15)
+    return fail(KVQ_ERR_ARG, "decode workspace not 16-byte aligned");
+  if (ws_bytes < kvq_decode_workspace_bytes(cfg, batch, n_q_heads, max_len))
+    return fail(KVQ_ERR_WORKSPACE, "decode workspace %zu < %zu", ws_bytes,
+                kvq_decode_workspace_bytes(cfg, batch, n_q_heads, max_len));
+  cudaError_t e = launch_decode(reinterpret_cast<const Plan* const*>(plans_dev), cm, len_dev,
+                                batch, max_len, q_dev, q_dtype, n_q_heads, cfg->n_kv_heads,
+                                cfg->bits_k, cfg->bits_v, out_dev, ws_dev, ws_bytes, status_dev,
+                                reinterpret_cast<cudaStream_t>(stream), k_dev, v_dev, kv_dtype,
+                                n_new, cap_tokens, (step_flags & KVQ_STEP_EARLY) ? 1 : 0,
+                                (step_flags & KVQ_STEP_ROPE) ? theta : nullptr, nullptr);
+  if (e != cudaSuccess) return cuda_fail(e, "append_decode");
+  return KVQ_OK;
+}
+
+// Checks a page description and turns it into the kernels' cache map; the
+// capacity of a sequence is its block-table row.
+int paged_map(const kvq_cfg* cfg, const kvq_pages* pg, CacheMap* cm, int64_t* cap_tokens) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (!pg || !pg->pool || !pg->block_table) return fail(KVQ_ERR_ARG, "null page description");
+  if (reinterpret_cast<uintptr_t>(pg->pool) & 15)
+    return fail(KVQ_ERR_ARG, "page pool not 16-byte aligned");
+  const size_t pb = kvq_page_bytes(cfg, pg->page_tiles);
+  if (pb == 0) return fail(KVQ_ERR_ARG, "page_tiles %d (a power of two, 1..2^20)", pg->page_tiles);
+  if (pg->max_pages < 1 || pg->n_pages < 1)
+    return fail(KVQ_ERR_ARG, "max_pages %d / n_pages %lld", pg->max_pages,
+                (long long)pg->n_pages);
+  const int64_t cap = (int64_t)pg->max_pages * pg->page_tiles * 32;
+  if (cap > 0x7FFFFFFF) return fail(KVQ_ERR_ARG, "block-table capacity %lld tokens", (long long)cap);
+  int shift = 0;
+  while ((1 << shift) < pg->page_tiles) ++shift;
+  *cm = CacheMap{};
+  cm->pool = reinterpret_cast<uint8_t*>(pg->pool);
+  cm->table = pg->block_table;
+  cm->n_pages = pg->n_pages;
+  cm->page_bytes = (int64_t)pb;
+  cm->max_pages = pg->max_pages;
+  cm->page_shift = shift;
+  *cap_tokens = cap;
   return KVQ_OK;
 }
 
@@ -380,8 +448,8 @@ int kvq_decode_attn(const kvq_cfg* cfg, const void* const* plans_dev, const void
                     int q_dtype, int n_q_heads, float* out_dev, void* ws_dev, size_t ws_bytes,
                     uint32_t* status_dev, kvq_stream_t stream) {
   if (!out_dev) return fail(KVQ_ERR_ARG, "null device pointer");
-  return decode_impl(cfg, plans_dev, cache_dev, len_dev, batch, max_len, q_dev, q_dtype, n_q_heads,
-                     out_dev, nullptr, ws_dev, ws_bytes, status_dev, stream);
+  return decode_impl(cfg, plans_dev, contiguous_map(cache_dev), len_dev, batch, max_len, q_dev,
+                     q_dtype, n_q_heads, out_dev, nullptr, ws_dev, ws_bytes, status_dev, stream);
 }
 
 int kvq_decode_attn_partial(const kvq_cfg* cfg, const void* const* plans_dev,
@@ -390,8 +458,8 @@ int kvq_decode_attn_partial(const kvq_cfg* cfg, const void* const* plans_dev,
                             float* rec_dev, void* ws_dev, size_t ws_bytes, uint32_t* status_dev,
                             kvq_stream_t stream) {
   if (!rec_dev) return fail(KVQ_ERR_ARG, "null device pointer");
-  return decode_impl(cfg, plans_dev, cache_dev, len_dev, batch, max_len, q_dev, q_dtype, n_q_heads,
-                     nullptr, rec_dev, ws_dev, ws_bytes, status_dev, stream);
+  return decode_impl(cfg, plans_dev, contiguous_map(cache_dev), len_dev, batch, max_len, q_dev,
+                     q_dtype, n_q_heads, nullptr, rec_dev, ws_dev, ws_bytes, status_dev, stream);
 }
 
 int kvq_combine_partials(const kvq_cfg* cfg, const void* const* plans_dev, int n_parts,
@@ -419,38 +487,61 @@ int kvq_append_decode(const kvq_cfg* cfg, const void* const* plans_dev, const vo
                       const void* q_dev, int q_dtype, int n_q_heads, float* out_dev, void* ws_dev,
                       size_t ws_bytes, int step_flags, double rope_base, uint32_t* status_dev,
                       kvq_stream_t stream) {
-  int rc = check_cfg(cfg);
+  if (!cache_dev) return fail(KVQ_ERR_ARG, "null device pointer");
+  return append_decode_impl(cfg, plans_dev, k_dev, v_dev, kv_dtype, n_new,
+                            contiguous_map(cache_dev), len_dev, cap_tokens, batch, max_len, q_dev,
+                            q_dtype, n_q_heads, out_dev, ws_dev, ws_bytes, step_flags, rope_base,
+                            status_dev, stream);
+}
+
+size_t kvq_page_bytes(const kvq_cfg* cfg, int32_t page_tiles) {
+  if (check_cfg(cfg) || page_tiles < 1 || page_tiles > (1 << 20) ||
+      (page_tiles & (page_tiles - 1)))
+    return 0;
+  return (size_t)page_tiles * cfg->n_kv_heads * tile_bytes(cfg->bits_k, cfg->bits_v);
+}
+
+int kvq_paged_quantize_append(const kvq_cfg* cfg, const void* const* plans_dev, const void* k_dev,
+                              const void* v_dev, int dtype, int batch, int n_new,
+                              const kvq_pages* pages, int32_t* len_dev, double rope_base,
+                              uint32_t* status_dev, kvq_stream_t stream) {
+  CacheMap cm;
+  int64_t cap = 0;
+  int rc = paged_map(cfg, pages, &cm, &cap);
   if (rc) return rc;
-  if (!plans_dev || !cache_dev || !len_dev || !q_dev || !out_dev || !ws_dev || !status_dev)
-    return fail(KVQ_ERR_ARG, "null device pointer");
-  if (n_new < 0 || n_new > 64) return fail(KVQ_ERR_ARG, "n_new %d not in 0..64", n_new);
-  if (n_new > 0 && (!k_dev || !v_dev)) return fail(KVQ_ERR_ARG, "null k/v pointer");
-  if (step_flags & ~(KVQ_STEP_EARLY | KVQ_STEP_ROPE))
-    return fail(KVQ_ERR_ARG, "step_flags 0x%x", step_flags);
   double theta[64];
-  if ((step_flags & KVQ_STEP_ROPE) && !rope_thetas(rope_base, theta))
+  if (rope_base != 0.0 && !rope_thetas(rope_base, theta))
     return fail(KVQ_ERR_ARG, "rope_base %g", rope_base);
-  if (!dtype_ok(kv_dtype) || !dtype_ok(q_dtype)) return fail(KVQ_ERR_ARG, "bad dtype");
-  if (batch < 1 || batch > 65535) return fail(KVQ_ERR_ARG, "batch %d", batch);
-  if (max_len < 1 || max_len > 0x7FFFFFFF || cap_tokens < 0 || cap_tokens > 0x7FFFFFFF)
-    return fail(KVQ_ERR_ARG, "max_len %lld / cap_tokens %lld", (long long)max_len,
-                (long long)cap_tokens);
-  if (n_q_heads < 1 || n_q_heads % cfg->n_kv_heads != 0 || n_q_heads / cfg->n_kv_heads > 16)
-    return fail(KVQ_ERR_ARG, "n_q_heads %d vs n_kv_heads %d", n_q_heads, cfg->n_kv_heads);
-  if (reinterpret_cast<uintptr_t>(ws_dev) & 15)
-    return fail(KVQ_ERR_ARG, "decode workspace not 16-byte aligned");
-  if (ws_bytes < kvq_decode_workspace_bytes(cfg, batch, n_q_heads, max_len))
-    return fail(KVQ_ERR_WORKSPACE, "decode workspace %zu < %zu", ws_bytes,
-                kvq_decode_workspace_bytes(cfg, batch, n_q_heads, max_len));
-  cudaError_t e = launch_decode(reinterpret_cast<const Plan* const*>(plans_dev),
-                                reinterpret_cast<const uint8_t* const*>(cache_dev), len_dev, batch,
-                                max_len, q_dev, q_dtype, n_q_heads, cfg->n_kv_heads, cfg->bits_k,
-                                cfg->bits_v, out_dev, ws_dev, ws_bytes, status_dev,
-                                reinterpret_cast<cudaStream_t>(stream), k_dev, v_dev, kv_dtype,
-                                n_new, cap_tokens, (step_flags & KVQ_STEP_EARLY) ? 1 : 0,
-                                (step_flags & KVQ_STEP_ROPE) ? theta : nullptr, nullptr);
-  if (e != cudaSuccess) return cuda_fail(e, "append_decode");
-  return KVQ_OK;
+  return quantize_append_impl(cfg, plans_dev, k_dev, v_dev, dtype, batch, n_new, cm, len_dev, cap,
+                              rope_base != 0.0 ? theta : nullptr, status_dev, stream);
+}
+
+int kvq_paged_decode_attn(const kvq_cfg* cfg, const void* const* plans_dev, const kvq_pages* pages,
+                          const int32_t* len_dev, int batch, int64_t max_len, const void* q_dev,
+                          int q_dtype, int n_q_heads, float* out_dev, void* ws_dev,
+                          size_t ws_bytes, uint32_t* status_dev, kvq_stream_t stream) {
+  CacheMap cm;
+  int64_t cap = 0;
+  int rc = paged_map(cfg, pages, &cm, &cap);
+  if (rc) return rc;
+  if (!out_dev) return fail(KVQ_ERR_ARG, "null device pointer");
+  return decode_impl(cfg, plans_dev, cm, len_dev, batch, max_len, q_dev, q_dtype, n_q_heads,
+                     out_dev, nullptr, ws_dev, ws_bytes, status_dev, stream);
+}
+
+int kvq_paged_append_decode(const kvq_cfg* cfg, const void* const* plans_dev, const void* k_dev,
+                            const void* v_dev, int kv_dtype, int n_new, const kvq_pages* pages,
+                            int32_t* len_dev, int batch, int64_t max_len, const void* q_dev,
+                            int q_dtype, int n_q_heads, float* out_dev, void* ws_dev,
+                            size_t ws_bytes, int step_flags, double rope_base,
+                            uint32_t* status_dev, kvq_stream_t stream) {
+  CacheMap cm;
+  int64_t cap = 0;
+  int rc = paged_map(cfg, pages, &cm, &cap);
+  if (rc) return rc;
+  return append_decode_impl(cfg, plans_dev, k_dev, v_dev, kv_dtype, n_new, cm, len_dev, cap,
+                            batch, max_len, q_dev, q_dtype, n_q_heads, out_dev, ws_dev, ws_bytes,
+                            step_flags, rope_base, status_dev, stream);
 }
 
 }  // extern "C"

@@ -68,6 +68,28 @@ __host__ __device__ __forceinline__ int token_of_slot_v(int s) {
   return 8 * ((s & 7) >> 1) + 2 * (s >> 3) + (s & 1);
 }
 
+// Where the tiles of each sequence live (host and device side).
+// Contiguous (table == nullptr): record of tile t, KV head h of sequence b at
+// caches[b] + (t n_kv + h) tile_bytes. Paged: tile t is tile t mod P of page
+// table[b][t / P] of the pool (P = 2^page_shift tiles per page, each page laid
+// out like a contiguous cache of P tiles, page_bytes = P n_kv tile_bytes).
+struct CacheMap {
+  uint8_t* const* caches;  // contiguous: [batch] bases
+  uint8_t* pool;           // paged: page g at pool + g page_bytes
+  const int32_t* table;    // paged: [batch][max_pages] page ids
+  int64_t n_pages;         // paged: ids outside [0, n_pages) are refused
+  int64_t page_bytes;
+  int max_pages;
+  int page_shift;          // contiguous: 31 (one page)
+};
+
+inline CacheMap contiguous_map(const void* const* caches) {
+  CacheMap m{};
+  m.caches = reinterpret_cast<uint8_t* const*>(const_cast<void* const*>(caches));
+  m.page_shift = 31;
+  return m;
+}
+
 // Arguments of the quantize-append launch (host and device side).
 struct QuantParams {
   const Plan* const* plans;  // [batch] -> [n_kv] plans
@@ -75,7 +97,7 @@ struct QuantParams {
   const void* v;
   int dtype;
   int batch, n_new, n_kv;
-  uint8_t* const* caches;  // [batch]
+  CacheMap cm;
   const int32_t* len;
   int64_t cap;
   int tile_bytes;
@@ -87,6 +109,22 @@ struct QuantParams {
 
 // ------------------------------------------------------------------ device
 #ifdef __CUDACC__
+
+// Base of the page holding tile `tile` of sequence b (for a contiguous cache
+// the sequence's base), or nullptr for a tile past the block table or a page
+// id outside the pool. The record of (tile, h) is at base + tile_in_page
+// offset: ((tile & page_mask(m)) n_kv + h) tile_bytes.
+__device__ __forceinline__ const uint8_t* page_base(const CacheMap& m, int b, int tile) {
+  if (!m.table) return m.caches[b];
+  const int j = tile >> m.page_shift;
+  if (j < 0 || j >= m.max_pages) return nullptr;
+  const int g = m.table[(size_t)b * m.max_pages + j];
+  if (g < 0 || (int64_t)g >= m.n_pages) return nullptr;
+  return m.pool + (int64_t)g * m.page_bytes;
+}
+__device__ __forceinline__ int page_mask(const CacheMap& m) {
+  return m.page_shift >= 31 ? 0x7FFFFFFF : (1 << m.page_shift) - 1;
+}
 
 __device__ __forceinline__ float load_as_float(const void* p, int dtype, size_t i) {
   if (dtype == KVQ_BF16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);

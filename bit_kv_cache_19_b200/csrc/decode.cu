@@ -53,6 +53,7 @@ namespace kvq {
 
 // Lookup image (generated with the codebooks): byte offsets of its tables.
 __device__ __align__(16) const uint32_t g_lut_image[KVQ_LUT_BYTES / 4] = KVQ_LUT_IMAGE;
+static_assert(KVQ_LUT_BYTES >= 512 * 16 + 128, "placeholder source of a refused page's tile");
 constexpr int kThrPad = (KVQ_CB_N_THR + 3) & ~3;  // thresholds, padded to 16 bytes
 __device__ __align__(16) const float g_thr[kThrPad] = KVQ_CB_THR;
 __host__ __device__ constexpr uint32_t lut_rep(int w) {  // widths 1..3, lane-replicated
@@ -71,7 +72,7 @@ constexpr int kScratch = 16640;  // q' staging; append: kz [32][129] fp32 + 64 f
 
 struct DecodeParams {
   const Plan* const* plans;
-  const uint8_t* const* caches;
+  CacheMap cm;
   int32_t* len;
   const void* q;
   int q_dtype;
@@ -336,13 +337,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   }
   __syncthreads();
   const bool ok_setup = mbar_wait_bounded(&sm.setup_bar, 0u);
-  const uint8_t* cache = p.caches[b];
+  const uint8_t* const cache0 = p.cm.table ? nullptr : p.cm.caches[b];  // contiguous base
   const int bk = sm.plan.bits_k;
   const int n_half = sm.plan.n_half;
   const bool bad = !ok_setup || sm.plan.magic != KVQ_PLAN_MAGIC || sm.plan.bits_v != BV ||
                    bk < 1 || bk > 8 || p.tile_bytes != tile_bytes(bk, BV) || n_half < 1 ||
                    n_half > kMaxHalf || sm.plan.n_class < 1 || sm.plan.n_class > 8 ||
-                   (reinterpret_cast<uintptr_t>(cache) & 15) != 0;
+                   (reinterpret_cast<uintptr_t>(cache0) & 15) != 0;
   if (bad && tid == 0) atomicOr(p.status, ok_setup ? KVQ_FLAG_BAD_PLAN : KVQ_FLAG_TIMEOUT);
   const int len0 = sm.len0;
   int n_add = 0;
@@ -371,16 +372,27 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   const int tbytes = p.tile_bytes;
   uint8_t* const my_stages = stage_base + (size_t)warp * kStages * tbytes;
   const int n_mine = has_work ? max(0, (te - tb - warp + kWarps - 1) / kWarps) : 0;
+  const int pmask = page_mask(p.cm);
   auto tile_of = [&](int i) { return te - 1 - warp - i * kWarps; };
-  auto issue = [&](int i) {
+  // page base of the warp's i-th tile (a paged cache looks it up in the block
+  // table; lane 0 does so one tile ahead of the copy that needs it)
+  auto base_of = [&](int i) { return p.cm.table ? page_base(p.cm, b, tile_of(i)) : cache0; };
+  auto issue = [&](int i, const uint8_t* base) {
     const int s = i % kStages;
     unsigned long long* bar = &sm.bar[warp][s];
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(g_lut_image);
+    if (base)
+      src = base + ((size_t)(tile_of(i) & pmask) * p.n_kv + h) * tbytes;
+    else  // refused page: placeholder bytes are streamed, the output is flagged
+      atomicOr(p.status, KVQ_FLAG_BAD_PAGE);
     mbar_expect_tx(bar, (uint32_t)tbytes);
-    bulk_g2s(my_stages + s * tbytes, cache + ((size_t)tile_of(i) * p.n_kv + h) * tbytes,
-             (uint32_t)tbytes, bar);
+    bulk_g2s(my_stages + s * tbytes, src, (uint32_t)tbytes, bar);
   };
-  if (lane == 0)
-    for (int i = 0; i < min(kStages, n_mine); ++i) issue(i);
+  const uint8_t* next_base = nullptr;  // lane 0: base of tile kStages, kStages + 1, ...
+  if (lane == 0) {
+    for (int i = 0; i < min(kStages, n_mine); ++i) issue(i, base_of(i));
+    if (kStages < n_mine) next_base = base_of(kStages);
+  }
   // appended tiles of this CTA: [a_lo, a_hi] (CTA-uniform)
   const int a_lo = n_add > 0 ? max(len0 / kTile, tb) : 1;
   const int a_hi = n_add > 0 ? min((len0 + n_add - 1) / kTile, te - 1) : 0;
@@ -424,7 +436,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
       const int t_lo = max(len0, tile * kTile), t_hi = min(len0 + n_add, tile * kTile + kTile);
       const int p_lo = t_lo - tile * kTile, p_hi = t_hi - tile * kTile;
       const int w_own = te - 1 - tile;
-      uint8_t* rec = const_cast<uint8_t*>(cache) + ((size_t)tile * p.n_kv + h) * tbytes;
+      const uint8_t* pb = page_base(p.cm, b, tile);
+      uint8_t* rec = pb ? const_cast<uint8_t*>(pb) + ((size_t)(tile & pmask) * p.n_kv + h) * tbytes
+                        : nullptr;
       uint8_t* st = stage_base + (size_t)w_own * kStages * tbytes;
       uint32_t* sw = reinterpret_cast<uint32_t*>(st);
       const int n_words = kHeadDim * (bk + BV);
@@ -451,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
       for (int r = warp; r < sm.plan.n_ranks; r += kWarps)
         warp_block_pass(sm.plan, sm.thr, r, kz, p_lo, p_hi, lane, sw, clear);
       __syncthreads();
-      if (ok) {
+      if (ok && rec) {
         uint32_t* gw = reinterpret_cast<uint32_t*>(rec);
         for (int i = tid; i < n_words; i += kThreads) gw[i] = sw[i];
         for (int e = tid; e < 2 * (p_hi - p_lo); e += kThreads) {
@@ -460,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
           reinterpret_cast<__half*>(st + 512 * (bk + BV))[off] = nrm_new[off];
         }
       } else {
-        flags |= KVQ_FLAG_TIMEOUT;
+        flags |= ok ? KVQ_FLAG_BAD_PAGE : KVQ_FLAG_TIMEOUT;
       }
       __syncthreads();
     }
@@ -633,7 +647,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
       __syncwarp();
       if (lane == 0 && i + kStages < n_mine) {
         fence_proxy_async();
-        issue(i + kStages);
+        issue(i + kStages, next_base);
+        if (i + kStages + 1 < n_mine) next_base = base_of(i + kStages + 1);
       }
     }
     if (timed_out) {
@@ -988,7 +1003,7 @@ static cudaError_t launch_decode_nt(const DecodeParams& p, int bits_v, int batch
 // ws: >= decode_workspace_bytes_for(...) bytes, zero-filled before its first
 // use; every completed call leaves its counters (at the end of ws) zero.
 // n_new > 0 fuses the append of k_new / v_new ([batch][n_new][n_kv][128]).
-cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches, int32_t* len,
+cudaError_t launch_decode(const Plan* const* plans, const CacheMap& cm, int32_t* len,
                           int batch, int64_t max_len, const void* q, int q_dtype, int n_q, int n_kv,
                           int bits_k, int bits_v, float* out, void* ws, size_t ws_bytes,
                           uint32_t* status, cudaStream_t st, const void* k_new,
@@ -1004,7 +1019,7 @@ cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches
   if (n_new < 0 || n_new > kMaxNew) return cudaErrorInvalidValue;
   DecodeParams p;
   p.plans = plans;
-  p.caches = caches;
+  p.cm = cm;
   p.len = len;
   p.q = q;
   p.q_dtype = q_dtype;

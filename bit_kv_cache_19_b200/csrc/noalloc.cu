@@ -18,7 +18,7 @@
 #include "common.cuh"
 
 namespace kvq {
-cudaError_t launch_decode(const Plan* const* plans, const uint8_t* const* caches, int32_t* len,
+cudaError_t launch_decode(const Plan* const* plans, const CacheMap& cm, int32_t* len,
                           int batch, int64_t max_len, const void* q, int q_dtype, int n_q, int n_kv,
                           int bits_k, int bits_v, float* out, void* ws, size_t ws_bytes,
                           uint32_t* status, cudaStream_t st, const void* k_new, const void* v_new,
@@ -94,8 +94,7 @@ extern "C" KVQ_API int kvq_decode_attn_noalloc(const kvq_cfg* cfg, const void* c
   // starts: the array is zero when the library is loaded and every completed
   // call resets the counters it used.
   e = kvq::launch_decode(reinterpret_cast<const kvq::Plan* const*>(plans_dev),
-                         reinterpret_cast<const uint8_t* const*>(cache_dev),
-                         const_cast<int32_t*>(len_dev), batch, max_len, q_dev, q_dtype, n_q_heads,
+                         kvq::contiguous_map(cache_dev), const_cast<int32_t*>(len_dev), batch, max_len, q_dev, q_dtype, n_q_heads,
                          cfg->n_kv_heads, cfg->bits_k, cfg->bits_v, out_dev, scratch,
                          kScratchBytes, status_dev, reinterpret_cast<cudaStream_t>(stream),
                          nullptr, nullptr, 0, 0, 0, 0, nullptr, nullptr);

@@ -121,12 +121,16 @@ __global__ void __launch_bounds__(256, 4) quantize_append_kernel(QuantParams p) 
     const int tile = len0 / kTile + ti;
     const int t_lo = max(len0, tile * kTile), t_hi = min(len0 + p.n_new, tile * kTile + kTile);
     if (t_lo >= t_hi) continue;
-    uint8_t* rec = p.caches[b];
+    uint8_t* rec = const_cast<uint8_t*>(page_base(p.cm, b, tile));
+    if (!rec) {
+      if (threadIdx.x == 0) atomicOr(p.status, KVQ_FLAG_BAD_PAGE);
+      continue;
+    }
     if ((reinterpret_cast<uintptr_t>(rec) & 15) != 0) {
       if (threadIdx.x == 0) atomicOr(p.status, KVQ_FLAG_BAD_PLAN);
       continue;
     }
-    rec += ((size_t)tile * p.n_kv + h) * p.tile_bytes;
+    rec += ((size_t)(tile & page_mask(p.cm)) * p.n_kv + h) * p.tile_bytes;
     __syncthreads();  // the previous item is done with the shared buffers
     if (bh != cur) {
       const uint32_t* src = reinterpret_cast<const uint32_t*>(p.plans[b] + h);

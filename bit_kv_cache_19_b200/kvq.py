@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libkvq.so")
 OK = 0
 ERR_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA = -1, -2, -3, -4
 FLAG_CAPACITY, FLAG_NONFINITE, FLAG_NORM_SAT, FLAG_TIMEOUT, FLAG_BAD_PLAN = 1, 2, 4, 8, 16
+FLAG_BAD_PAGE = 32
 BF16, FP16, FP32 = 0, 1, 2
 ALLOC_GREEDY, ALLOC_UNIFORM = 0, 1
 STEP_EARLY = 1
@@ -55,6 +56,14 @@ def make_cfg(n_kv_heads, bits_k, bits_v, v_seed=0, alloc_mode=ALLOC_GREEDY, head
     return Cfg(head_dim, n_kv_heads, bits_k, bits_v, 8, alloc_mode, v_seed)
 
 
+class Pages(ctypes.Structure):
+    """kvq_pages: pool, block table [batch][max_pages] (int32 page ids),
+    pages in the pool, 32-token tiles per page, block-table row length."""
+    _fields_ = [("pool", ctypes.c_void_p), ("block_table", ctypes.c_void_p),
+                ("n_pages", ctypes.c_int64), ("page_tiles", ctypes.c_int32),
+                ("max_pages", ctypes.c_int32)]
+
+
 _vp, _sz, _i32, _i64, _u32p = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_int64, \
     ctypes.c_void_p
 _SIGS = {
@@ -87,6 +96,14 @@ _SIGS = {
     "kvq_decode_attn_partial": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i64, _vp, _i32,
                                        _i32, _vp, _vp, _sz, _vp, _vp]),
     "kvq_combine_partials": (_i32, [ctypes.POINTER(Cfg), _vp, _i32, _vp, _i32, _i32, _vp, _vp]),
+    "kvq_page_bytes": (_sz, [ctypes.POINTER(Cfg), _i32]),
+    "kvq_paged_quantize_append": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i32, _i32,
+                                         ctypes.POINTER(Pages), _vp, ctypes.c_double, _vp, _vp]),
+    "kvq_paged_decode_attn": (_i32, [ctypes.POINTER(Cfg), _vp, ctypes.POINTER(Pages), _vp, _i32,
+                                     _i64, _vp, _i32, _i32, _vp, _vp, _sz, _vp, _vp]),
+    "kvq_paged_append_decode": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i32,
+                                       ctypes.POINTER(Pages), _vp, _i32, _i64, _vp, _i32, _i32,
+                                       _vp, _vp, _sz, _i32, ctypes.c_double, _vp, _vp]),
 }
 EXPORTS = tuple(_SIGS)
 
@@ -242,6 +259,48 @@ def combine_partials(cfg, plan_ptrs, recs, out):
     n_parts, batch, n_q = recs.shape[0], recs.shape[1], recs.shape[2]
     _check(lib().kvq_combine_partials(ctypes.byref(cfg), _ptr(plan_ptrs), n_parts, _ptr(recs),
                                       batch, n_q, _ptr(out), _stream()))
+
+
+def page_bytes(cfg, page_tiles) -> int:
+    return lib().kvq_page_bytes(ctypes.byref(cfg), page_tiles)
+
+
+def make_pages(pool, block_table, n_pages, page_tiles):
+    """kvq_pages over a device pool (n_pages pages of page_bytes) and a device
+    block table int32 [batch, max_pages]."""
+    return Pages(pool.data_ptr(), block_table.data_ptr(), n_pages, page_tiles,
+                 block_table.shape[1])
+
+
+def paged_quantize_append(cfg, plan_ptrs, k, v, pages, lens, status, rope_base=0.0):
+    """kvq_quantize_append into paged caches (rope_base > 1: pre-RoPE keys)."""
+    batch, n_new = k.shape[0], k.shape[1]
+    _check(lib().kvq_paged_quantize_append(ctypes.byref(cfg), _ptr(plan_ptrs), _ptr(k), _ptr(v),
+                                           _dtype_code(k), batch, n_new, ctypes.byref(pages),
+                                           _ptr(lens), float(rope_base), _ptr(status),
+                                           _stream()))
+
+
+def paged_decode_attn(cfg, plan_ptrs, pages, lens, max_len, q, out, ws, status):
+    """kvq_decode_attn over paged caches."""
+    batch, n_q = q.shape[0], q.shape[1]
+    _check(lib().kvq_paged_decode_attn(ctypes.byref(cfg), _ptr(plan_ptrs), ctypes.byref(pages),
+                                       _ptr(lens), batch, max_len, _ptr(q), _dtype_code(q), n_q,
+                                       _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
+                                       _ptr(status), _stream()))
+
+
+def paged_append_decode(cfg, plan_ptrs, k, v, pages, lens, max_len, q, out, ws, status,
+                        step_flags=0, rope_base=0.0):
+    """kvq_append_decode over paged caches."""
+    batch, n_q = q.shape[0], q.shape[1]
+    n_new = 0 if k is None else k.shape[1]
+    _check(lib().kvq_paged_append_decode(ctypes.byref(cfg), _ptr(plan_ptrs), _ptr(k), _ptr(v),
+                                         _dtype_code(k) if k is not None else BF16, n_new,
+                                         ctypes.byref(pages), _ptr(lens), batch, max_len,
+                                         _ptr(q), _dtype_code(q), n_q, _ptr(out), _ptr(ws),
+                                         ws.numel() * ws.element_size(), step_flags,
+                                         float(rope_base), _ptr(status), _stream()))
 
 
 def append_decode(cfg, plan_ptrs, k, v, cache_ptrs, lens, cap_tokens, max_len, q, out, ws,

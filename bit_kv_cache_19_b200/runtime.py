@@ -135,3 +135,116 @@ def sharded_decode(partial, combine, group=None):
     recs = torch.empty((world,) + tuple(rec.shape), dtype=rec.dtype, device=rec.device)
     dist.all_gather(list(recs.unbind(0)), rec.contiguous(), group=group)
     return combine(recs)
+
+
+class PagedLayer:
+    """One layer's packed caches for a batch of sequences in pages of a shared
+    pool: the pool, the block table (device) and a host-side page allocator.
+    Pages are handed out in order from a free list as sequences grow
+    (``reserve``) and returned by ``release``; the kernels only follow the
+    block table."""
+
+    def __init__(self, cfg, batch: int, n_pages: int, page_tiles: int, max_pages: int,
+                 device="cuda", layer: int = 0):
+        self.cfg = cfg
+        self.batch = batch
+        self.layer = layer
+        self.device = torch.device(device)
+        self.page_tiles = page_tiles
+        self.n_pages = n_pages
+        nb = kvq.page_bytes(cfg, page_tiles)
+        if nb == 0:
+            raise ValueError(f"page_tiles {page_tiles}: a power of two, 1..2^20")
+        self.pool = torch.zeros(n_pages * nb, dtype=torch.uint8, device=self.device)
+        self.table_host = np.full((batch, max_pages), -1, dtype=np.int32)
+        self.table = torch.from_numpy(self.table_host.copy()).to(self.device)
+        self.pages = kvq.make_pages(self.pool, self.table, n_pages, page_tiles)
+        self.free = list(range(n_pages))
+        self.n_held = [0] * batch
+        self.plans = torch.zeros(cfg.n_kv_heads * kvq.PLAN_BYTES, dtype=torch.uint8,
+                                 device=self.device)
+        self.plan_ptrs = kvq.ptr_array([self.plans] * batch, self.device)
+        self.lens = torch.zeros(batch, dtype=torch.int32, device=self.device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self.plans_host = None
+
+    @property
+    def cap(self) -> int:
+        return self.table_host.shape[1] * self.page_tiles * 32
+
+    # ---------------------------------------------------------- pages
+    def reserve(self, seq: int, n_tokens: int, order=None):
+        """Give sequence `seq` pages for its first n_tokens tokens (from the
+        free list, or in the given page order) and upload the block table."""
+        need = -(-n_tokens // (32 * self.page_tiles))
+        if need > self.table_host.shape[1]:
+            raise ValueError(f"{n_tokens} tokens exceed the block-table row")
+        while self.n_held[seq] < need:
+            if not self.free:
+                raise MemoryError("page pool exhausted")
+            g = self.free.pop(0) if order is None else order.pop(0)
+            if order is not None:
+                self.free.remove(g)
+            self.table_host[seq, self.n_held[seq]] = g
+            self.n_held[seq] += 1
+        self.table.copy_(torch.from_numpy(self.table_host))
+
+    def release(self, seq: int):
+        """Return a sequence's pages to the free list and empty it."""
+        held = self.table_host[seq, :self.n_held[seq]].tolist()
+        self.free.extend(held)
+        self.table_host[seq, :] = -1
+        self.n_held[seq] = 0
+        self.table.copy_(torch.from_numpy(self.table_host))
+        self.lens[seq] = 0
+
+    # ---------------------------------------------------------- calls
+    def set_plans(self, plans_host: np.ndarray):
+        raw = torch.from_numpy(np.frombuffer(plans_host.tobytes(), dtype=np.uint8).copy())
+        self.plans.copy_(raw.to(self.device))
+        self.plans_host = plans_host
+
+    def append(self, k, v, rope_base=0.0):
+        """k, v [batch, n_new, n_kv, 128]; the pages must have been reserved."""
+        kvq.paged_quantize_append(self.cfg, self.plan_ptrs, k, v, self.pages, self.lens,
+                                  self.status, rope_base)
+
+    def decode(self, q, out=None, ws=None, max_len=None):
+        max_len = self.cap if max_len is None else max_len
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=self.device)
+        if ws is None:
+            ws = self.workspace(q.shape[1], max_len)
+        kvq.paged_decode_attn(self.cfg, self.plan_ptrs, self.pages, self.lens, max_len, q, out,
+                              ws, self.status)
+        return out
+
+    def append_decode(self, k, v, q, out=None, ws=None, max_len=None, step_flags=0,
+                      rope_base=0.0):
+        max_len = self.cap if max_len is None else max_len
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=self.device)
+        if ws is None:
+            ws = self.workspace(q.shape[1], max_len)
+        kvq.paged_append_decode(self.cfg, self.plan_ptrs, k, v, self.pages, self.lens, max_len,
+                                q, out, ws, self.status, step_flags, rope_base)
+        return out
+
+    def workspace(self, n_q: int, max_len: int):
+        n = kvq.decode_workspace_bytes(self.cfg, self.batch, n_q, max_len)
+        return torch.zeros(n, dtype=torch.uint8, device=self.device)
+
+    def head_records(self, seq: int, head: int, n_tiles: int) -> np.ndarray:
+        """Tile records [n_tiles, tile_bytes / 4] of one head, gathered
+        through the block table (host)."""
+        tb = kvq.tile_bytes(self.cfg)
+        n_kv = self.cfg.n_kv_heads
+        pool = self.pool.cpu().numpy().reshape(self.n_pages, self.page_tiles, n_kv, tb)
+        out = np.empty((n_tiles, tb), dtype=np.uint8)
+        for t in range(n_tiles):
+            g = self.table_host[seq, t // self.page_tiles]
+            out[t] = pool[g, t % self.page_tiles, head]
+        return out.view("<u4").reshape(n_tiles, tb // 4)
+
+    def flags(self) -> int:
+        return int(self.status.item()) & 0xFFFFFFFF

@@ -63,6 +63,8 @@ typedef struct CUstream_st* kvq_stream_t;
 #define KVQ_FLAG_NORM_SAT 4u   /* a norm overflowed fp16: stored as 65504 */
 #define KVQ_FLAG_TIMEOUT 8u    /* a bounded wait ran out: output invalid */
 #define KVQ_FLAG_BAD_PLAN 16u  /* a plan record failed its magic/shape check */
+#define KVQ_FLAG_BAD_PAGE 32u  /* paged cache: a tile past the block table or a page id outside
+                                  the pool (appends skip it; decode output is invalid) */
 
 /* Input element types. */
 #define KVQ_BF16 0
@@ -372,6 +374,65 @@ KVQ_API int kvq_append_decode(const kvq_cfg* cfg, const void* const* plans_dev, 
                               const void* q_dev, int q_dtype, int n_q_heads, float* out_dev,
                               void* ws_dev, size_t ws_bytes, int step_flags, double rope_base,
                               uint32_t* status_dev, kvq_stream_t stream);
+
+/*
+ * Paged caches (no counterpart in the pages, which keep one cache per
+ * sequence): the tiles of all sequences live in pages of one pool and a
+ * block table says which page holds which span of each sequence, so
+ * sequences grow page by page without reserving their full capacity.
+ * A page holds page_tiles consecutive 32-token tiles of one sequence for all
+ * KV heads, laid out exactly like a contiguous cache of page_tiles tiles
+ * (record of tile t, head h of the page at (t n_kv_heads + h) tile_bytes);
+ * tile t of sequence b is tile t mod page_tiles of page
+ * block_table[b][t / page_tiles]. Codes, norms and decode results are those
+ * of a contiguous cache holding the same tokens.
+ *
+ * pool:        device, 16-byte aligned; page g at pool + g kvq_page_bytes.
+ * block_table: device int32 [batch][max_pages]; entries that a call reaches
+ *              (tiles below len + n_new) must be page ids in [0, n_pages);
+ *              others are never read. An id outside the pool, or a tile past
+ *              the row, flags BAD_PAGE: appends skip that tile, decode
+ *              streams placeholder bytes instead and its output is invalid.
+ *              Pages of different sequences must not overlap.
+ * n_pages:     pages in the pool. page_tiles: a power of two, 1..2^20.
+ * max_pages:   row length; a sequence holds at most
+ *              max_pages * page_tiles * 32 tokens (the capacity that
+ *              cap_tokens gives for contiguous caches; at most 2^31 - 1).
+ * The block table is read by the kernels as the lengths are: with
+ * KVQ_STEP_EARLY it must not be written by the previous kernel on the stream.
+ */
+typedef struct kvq_pages {
+  void* pool;
+  const int32_t* block_table;
+  int64_t n_pages;
+  int32_t page_tiles;
+  int32_t max_pages;
+} kvq_pages;
+
+/* Bytes of one page (page_tiles * n_kv_heads * kvq_tile_bytes); 0 if invalid. */
+KVQ_API size_t kvq_page_bytes(const kvq_cfg* cfg, int32_t page_tiles);
+
+/* kvq_quantize_append into paged caches. rope_base = 0: k_dev holds post-RoPE
+ * keys; rope_base > 1: pre-RoPE keys rotated as by kvq_quantize_append_rope. */
+KVQ_API int kvq_paged_quantize_append(const kvq_cfg* cfg, const void* const* plans_dev,
+                                      const void* k_dev, const void* v_dev, int dtype, int batch,
+                                      int n_new, const kvq_pages* pages, int32_t* len_dev,
+                                      double rope_base, uint32_t* status_dev,
+                                      kvq_stream_t stream);
+/* kvq_decode_attn over paged caches (same workspace rules). */
+KVQ_API int kvq_paged_decode_attn(const kvq_cfg* cfg, const void* const* plans_dev,
+                                  const kvq_pages* pages, const int32_t* len_dev, int batch,
+                                  int64_t max_len, const void* q_dev, int q_dtype, int n_q_heads,
+                                  float* out_dev, void* ws_dev, size_t ws_bytes,
+                                  uint32_t* status_dev, kvq_stream_t stream);
+/* kvq_append_decode over paged caches (capacity from the block table). */
+KVQ_API int kvq_paged_append_decode(const kvq_cfg* cfg, const void* const* plans_dev,
+                                    const void* k_dev, const void* v_dev, int kv_dtype, int n_new,
+                                    const kvq_pages* pages, int32_t* len_dev, int batch,
+                                    int64_t max_len, const void* q_dev, int q_dtype,
+                                    int n_q_heads, float* out_dev, void* ws_dev, size_t ws_bytes,
+                                    int step_flags, double rope_base, uint32_t* status_dev,
+                                    kvq_stream_t stream);
 
 /*
  * bf16 comparator (not part of the method): split-K decode attention over an

@@ -157,6 +157,28 @@ def test_argument_errors_without_gpu():
     assert b"n_parts" in L.kvq_last_error()
     assert L.kvq_combine_partials(ctypes.byref(cfg), p, 2, p8, 1, 16, p, None) == kvq.ERR_ARG
     assert L.kvq_combine_partials(ctypes.byref(cfg), p, 2, p, 1, 15, p, None) == kvq.ERR_ARG
+    # paged caches: page_tiles a power of two, pool aligned, capacity < 2^31 tokens
+    assert kvq.page_bytes(cfg, 4) == 4 * 2 * kvq.tile_bytes(cfg)
+    assert kvq.page_bytes(cfg, 3) == 0 and kvq.page_bytes(cfg, 0) == 0
+    pg = kvq.Pages(16, 16, 10, 3, 8)
+    assert L.kvq_paged_decode_attn(ctypes.byref(cfg), p, ctypes.byref(pg), p, 1, 10, p, 0, 16, p,
+                                   p, 1 << 30, p, None) == kvq.ERR_ARG
+    assert b"page_tiles" in L.kvq_last_error()
+    pg = kvq.Pages(24, 16, 10, 4, 8)
+    assert L.kvq_paged_quantize_append(ctypes.byref(cfg), p, p, p, 0, 1, 1, ctypes.byref(pg), p,
+                                       0.0, p, None) == kvq.ERR_ARG
+    assert b"aligned" in L.kvq_last_error()
+    pg = kvq.Pages(16, 16, 10, 1 << 20, 1 << 10)
+    assert L.kvq_paged_append_decode(ctypes.byref(cfg), p, p, p, 0, 1, ctypes.byref(pg), p, 1,
+                                     10, p, 0, 16, p, p, 1 << 30, 0, 0.0, p, None) == kvq.ERR_ARG
+    assert b"capacity" in L.kvq_last_error()
+    pg = kvq.Pages(16, None, 10, 4, 8)
+    assert L.kvq_paged_decode_attn(ctypes.byref(cfg), p, ctypes.byref(pg), p, 1, 10, p, 0, 16, p,
+                                   p, 1 << 30, p, None) == kvq.ERR_ARG
+    pg = kvq.Pages(16, 16, 10, 4, 8)
+    assert L.kvq_paged_quantize_append(ctypes.byref(cfg), p, p, p, 0, 1, 1, ctypes.byref(pg), p,
+                                       0.5, p, None) == kvq.ERR_ARG
+    assert b"rope_base" in L.kvq_last_error()
     # zero new tokens is a no-op
     assert L.kvq_quantize_append(ctypes.byref(cfg), p, None, None, 0, 1, 0, p, p, 10, p,
                                  None) == kvq.OK
