@@ -96,7 +96,10 @@ void greedy_widths(const double* E, int bits_k, uint8_t* w) {
   for (int j = 0; j < kBlocks; ++j) w[j] = (uint8_t)b[j];
 }
 
-void build_plan(const kvq_cfg* cfg, int layer, int kv_head, const double* E, Plan* pl) {
+// W (optional): query block energies of the query-weighted variant; the
+// widths then come from the products E_j W_j, the key scales still from E.
+void build_plan(const kvq_cfg* cfg, int layer, int kv_head, const double* E, Plan* pl,
+                const double* W = nullptr) {
   std::memset(pl, 0, sizeof(Plan));
   pl->magic = KVQ_PLAN_MAGIC;
   pl->bits_k = cfg->bits_k;
@@ -107,6 +110,10 @@ void build_plan(const kvq_cfg* cfg, int layer, int kv_head, const double* E, Pla
   pl->words_v = 128 * cfg->bits_v;
   if (cfg->alloc_mode == KVQ_ALLOC_UNIFORM) {
     for (int j = 0; j < kBlocks; ++j) pl->width[j] = (uint8_t)cfg->bits_k;
+  } else if (W) {
+    double EW[kBlocks];
+    for (int j = 0; j < kBlocks; ++j) EW[j] = E[j] * W[j];
+    greedy_widths(EW, cfg->bits_k, pl->width);
   } else {
     greedy_widths(E, cfg->bits_k, pl->width);
   }
@@ -234,6 +241,64 @@ int kvq_plan_build(const kvq_cfg* cfg, int layer, const double* E_host, int n_he
       return fail(KVQ_ERR_ARG, "energy %d is negative or not finite", i);
   Plan* out = reinterpret_cast<Plan*>(plans_host);
   for (int h = 0; h < n_heads; ++h) build_plan(cfg, layer, h, E_host + (size_t)h * kBlocks, out + h);
+  return KVQ_OK;
+}
+
+int kvq_plan_build_weighted(const kvq_cfg* cfg, int layer, const double* E_host,
+                            const double* Eq_host, int n_q_heads, void* plans_host) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  const int n_kv = cfg->n_kv_heads;
+  if (!E_host || !Eq_host || !plans_host) return fail(KVQ_ERR_ARG, "null pointer");
+  if (n_q_heads < 1 || n_q_heads % n_kv != 0)
+    return fail(KVQ_ERR_ARG, "n_q_heads %d vs n_kv_heads %d", n_q_heads, n_kv);
+  for (int i = 0; i < n_kv * kBlocks; ++i)
+    if (!(E_host[i] >= 0.0) || !std::isfinite(E_host[i]))
+      return fail(KVQ_ERR_ARG, "energy %d is negative or not finite", i);
+  for (int i = 0; i < n_q_heads * kBlocks; ++i)
+    if (!(Eq_host[i] >= 0.0) || !std::isfinite(Eq_host[i]))
+      return fail(KVQ_ERR_ARG, "query energy %d is negative or not finite", i);
+  const int G = n_q_heads / n_kv;
+  Plan* out = reinterpret_cast<Plan*>(plans_host);
+  for (int h = 0; h < n_kv; ++h) {
+    double W[kBlocks];  // the group's mean query energy, summed in increasing g
+    for (int j = 0; j < kBlocks; ++j) {
+      double acc = 0.0;
+      for (int g = 0; g < G; ++g) acc += Eq_host[(size_t)(h * G + g) * kBlocks + j];
+      W[j] = acc / G;
+    }
+    build_plan(cfg, layer, h, E_host + (size_t)h * kBlocks, out + h, W);
+  }
+  return KVQ_OK;
+}
+
+size_t kvq_energy_workspace_bytes(int n_heads) {
+  if (n_heads < 1 || n_heads > 65535) return 0;
+  return align_up((size_t)n_heads * kBlocks * 16, 256);
+}
+
+int kvq_block_energy(const void* x_dev, int dtype, int64_t n_tokens, int n_heads, void* ws_dev,
+                     size_t ws_bytes, double* energy_host, uint32_t* status_dev,
+                     kvq_stream_t stream) {
+  if (!x_dev || !ws_dev || !energy_host) return fail(KVQ_ERR_ARG, "null pointer");
+  if (!dtype_ok(dtype)) return fail(KVQ_ERR_ARG, "dtype %d", dtype);
+  if (n_tokens < 1) return fail(KVQ_ERR_ARG, "n_tokens %lld < 1", (long long)n_tokens);
+  if (n_heads < 1 || n_heads > 65535) return fail(KVQ_ERR_ARG, "n_heads %d", n_heads);
+  if (ws_bytes < kvq_energy_workspace_bytes(n_heads))
+    return fail(KVQ_ERR_WORKSPACE, "energy workspace too small");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  auto* acc = reinterpret_cast<unsigned long long*>(ws_dev);
+  cudaError_t e = launch_energy(x_dev, dtype, n_tokens, n_heads, acc, status_dev, st);
+  if (e != cudaSuccess) return cuda_fail(e, "energy kernel");
+  std::vector<unsigned long long> h_acc((size_t)n_heads * kBlocks * 2);
+  e = cudaMemcpyAsync(h_acc.data(), acc, h_acc.size() * 8, cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return cuda_fail(e, "energy copy");
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "energy sync");
+  for (size_t i = 0; i < (size_t)n_heads * kBlocks; ++i) {
+    const unsigned __int128 s = ((unsigned __int128)h_acc[2 * i + 1] << 64) | h_acc[2 * i];
+    energy_host[i] = std::ldexp((double)s, -32) / (double)n_tokens;
+  }
   return KVQ_OK;
 }
 

@@ -505,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
     //      q' = q a_hat_j log2(e) / sqrt(128); per-head 2^sigma scaling into
     //      the fp16 range; hi/lo split into the B fragments of each half step
     float* qp = reinterpret_cast<float*>(scratch);  // [8 NT][128]
-    for (int head = warp; head < 8 * NT; head += kWarps) {
+    for (int head = warp; head < 8 * NT; head += kWarps) {  // warp-local: one head each
       float v[4], mx = 0.f;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -524,20 +524,21 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
 #pragma unroll
       for (int i = 0; i < 4; ++i) qp[head * kHeadDim + lane + 32 * i] = v[i] * sc;
       if (lane == 0) sm.inv_scale[head] = ldexpf(1.f, -sigma);
-    }
-    __syncthreads();
-    for (int e = tid; e < NT * n_half * 32; e += kThreads) {
-      const int ln = e & 31, hs = (e >> 5) % n_half, nt = (e >> 5) / n_half;
-      const int head = 8 * nt + (ln >> 2), j = sm.qj[hs][ln & 3];
-      float x0 = 0.f, x1 = 0.f;
-      if (j >= 0) {
-        x0 = qp[head * kHeadDim + j];
-        x1 = qp[head * kHeadDim + j + 64];
+      __syncwarp();
+      // this head's B-fragment entries: lane 4 (head mod 8) + c of each half step
+      const int nt = head >> 3, g8 = head & 7;
+      for (int e = lane; e < n_half * 4; e += 32) {
+        const int hs = e >> 2, cc = e & 3, j = sm.qj[hs][cc];
+        float x0 = 0.f, x1 = 0.f;
+        if (j >= 0) {
+          x0 = qp[head * kHeadDim + j];
+          x1 = qp[head * kHeadDim + j + 64];
+        }
+        const uint32_t hi = pack_half2(x0, x1);
+        const __half2 hh = *reinterpret_cast<const __half2*>(&hi);
+        const uint32_t lo = pack_half2(x0 - __low2float(hh), x1 - __high2float(hh));
+        sm.qfrag[nt][hs][4 * g8 + cc] = make_uint2(hi, lo);
       }
-      const uint32_t hi = pack_half2(x0, x1);
-      const __half2 hh = *reinterpret_cast<const __half2*>(&hi);
-      const uint32_t lo = pack_half2(x0 - __low2float(hh), x1 - __high2float(hh));
-      sm.qfrag[nt][hs][ln] = make_uint2(hi, lo);
     }
     __syncthreads();
 
@@ -695,18 +696,19 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   //      all records instead
   float* const my_part = p.part + (bh * p.n_splits + split) * G * kPartStride;
   float* const crec = reinterpret_cast<float*>(scratch);  // [G][132]
-  merge_records<kThreads, kWarps>(mg, kWarps, (size_t)8 * NT * kPartStride, G, crec);
-  __syncthreads();
   unsigned int* const ovf = cnt + 1;
   unsigned int* const bmask = cnt + 2;  // [G]: buckets in use
   float* const bkt = p.bkt + bh * (size_t)G * kBuckets * kPartStride;
   for (int item = tid; item < G * 32; item += kThreads) {
     const int hd = item >> 5, x4 = (item & 31) * 4;
-    const float* r = crec + hd * kPartStride;
-    const float4 ov = *reinterpret_cast<const float4*>(r + kRecO + x4);
-    const float m = r[0], l = r[1];
+    float m, l;
+    float4 ov;
+    merge_item<kWarps>(mg + hd * kPartStride, kWarps, (size_t)8 * NT * kPartStride, x4, m, l, ov);
+    *reinterpret_cast<float4*>(crec + hd * kPartStride + kRecO + x4) = ov;
     *reinterpret_cast<float4*>(my_part + hd * kPartStride + kRecO + x4) = ov;
     if (x4 == 0) {
+      crec[hd * kPartStride] = m;
+      crec[hd * kPartStride + 1] = l;
       my_part[hd * kPartStride] = m;
       my_part[hd * kPartStride + 1] = l;
     }

@@ -51,52 +51,62 @@ __device__ __forceinline__ void grid_dep_launch() {
 }
 
 
+// Merge of n records of one head at coordinates x4..x4+3 (record s at
+// r + s * rec_stride): one pass with online rescaling over chunks of CHUNK
+// records whose loads are issued together (about n / CHUNK load round trips).
+// Every thread of the head gets the same M and L.
+template <int CHUNK>
+__device__ __forceinline__ void merge_item(const float* r, int n, size_t rec_stride, int x4,
+                                           float& M, float& L, float4& O) {
+  M = -INFINITY;
+  L = 0.f;
+  O = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < n; s0 += CHUNK) {
+    float2 ml[CHUNK];
+    float4 oo[CHUNK];
+#pragma unroll
+    for (int k = 0; k < CHUNK; ++k) {
+      const bool v = s0 + k < n;
+      const float* q = r + (size_t)(v ? s0 + k : 0) * rec_stride;
+      ml[k] = *reinterpret_cast<const float2*>(q);
+      oo[k] = *reinterpret_cast<const float4*>(q + kRecO + x4);
+      if (!v) ml[k].x = -INFINITY;
+    }
+    float cm = M;
+#pragma unroll
+    for (int k = 0; k < CHUNK; ++k) cm = fmaxf(cm, ml[k].x);
+    if (cm != -INFINITY) {
+      const float a = ex2(M - cm);
+      L *= a;
+      O.x *= a;
+      O.y *= a;
+      O.z *= a;
+      O.w *= a;
+#pragma unroll
+      for (int k = 0; k < CHUNK; ++k) {
+        const float w = ex2(ml[k].x - cm);  // 0 for records past n
+        L += w * ml[k].y;
+        O.x += w * oo[k].x;
+        O.y += w * oo[k].y;
+        O.z += w * oo[k].z;
+        O.w += w * oo[k].w;
+      }
+      M = cm;
+    }
+  }
+}
+
 // Merge n records per head (record s of head h at src + s * rec_stride +
-// h * kPartStride) into dst (record h at dst + h * kPartStride), for G heads.
-// 32 threads per head, 4 coordinates each: one pass with online rescaling
-// over chunks of CHUNK records whose loads are issued together, so a merge of
-// all heads costs about n / CHUNK load round trips.
+// h * kPartStride) into dst (record h at dst + h * kPartStride), for G heads,
+// 32 threads per head, 4 coordinates each.
 template <int NTHREADS, int CHUNK = kMergeChunk>
 __device__ __forceinline__ void merge_records(const float* src, int n, size_t rec_stride, int G,
                                               float* dst) {
   for (int item = threadIdx.x; item < G * 32; item += NTHREADS) {
     const int head = item >> 5, x4 = (item & 31) * 4;
-    const float* r = src + (size_t)head * kPartStride;
-    float M = -INFINITY, L = 0.f;
-    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s0 = 0; s0 < n; s0 += CHUNK) {
-      float2 ml[CHUNK];
-      float4 oo[CHUNK];
-#pragma unroll
-      for (int k = 0; k < CHUNK; ++k) {
-        const bool v = s0 + k < n;
-        const float* q = r + (size_t)(v ? s0 + k : 0) * rec_stride;
-        ml[k] = *reinterpret_cast<const float2*>(q);
-        oo[k] = *reinterpret_cast<const float4*>(q + kRecO + x4);
-        if (!v) ml[k].x = -INFINITY;
-      }
-      float cm = M;
-#pragma unroll
-      for (int k = 0; k < CHUNK; ++k) cm = fmaxf(cm, ml[k].x);
-      if (cm != -INFINITY) {
-        const float a = ex2(M - cm);
-        L *= a;
-        O.x *= a;
-        O.y *= a;
-        O.z *= a;
-        O.w *= a;
-#pragma unroll
-        for (int k = 0; k < CHUNK; ++k) {
-          const float w = ex2(ml[k].x - cm);  // 0 for records past n
-          L += w * ml[k].y;
-          O.x += w * oo[k].x;
-          O.y += w * oo[k].y;
-          O.z += w * oo[k].z;
-          O.w += w * oo[k].w;
-        }
-        M = cm;
-      }
-    }
+    float M, L;
+    float4 O;
+    merge_item<CHUNK>(src + (size_t)head * kPartStride, n, rec_stride, x4, M, L, O);
     float* d = dst + (size_t)head * kPartStride;
     *reinterpret_cast<float4*>(d + kRecO + x4) = O;
     if (x4 == 0) {

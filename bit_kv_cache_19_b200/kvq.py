@@ -97,6 +97,9 @@ _SIGS = {
                                        _i32, _vp, _vp, _sz, _vp, _vp]),
     "kvq_combine_partials": (_i32, [ctypes.POINTER(Cfg), _vp, _i32, _vp, _i32, _i32, _vp, _vp]),
     "kvq_page_bytes": (_sz, [ctypes.POINTER(Cfg), _i32]),
+    "kvq_energy_workspace_bytes": (_sz, [_i32]),
+    "kvq_block_energy": (_i32, [_vp, _i32, _i64, _i32, _vp, _sz, _vp, _vp, _vp]),
+    "kvq_plan_build_weighted": (_i32, [ctypes.POINTER(Cfg), _i32, _vp, _vp, _i32, _vp]),
     "kvq_paged_quantize_append": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i32, _i32,
                                          ctypes.POINTER(Pages), _vp, ctypes.c_double, _vp, _vp]),
     "kvq_paged_decode_attn": (_i32, [ctypes.POINTER(Cfg), _vp, ctypes.POINTER(Pages), _vp, _i32,
@@ -183,6 +186,32 @@ def plan_build(cfg, layer, E) -> np.ndarray:
     out = np.zeros(n, dtype=PLAN_DTYPE)
     _check(lib().kvq_plan_build(ctypes.byref(cfg), layer, E.ctypes.data, n, out.ctypes.data))
     return out
+
+
+def plan_build_weighted(cfg, layer, E, Eq) -> np.ndarray:
+    """Host plans of the query-weighted variant: widths from the greedy on
+    E * W, W the query energies Eq [n_q_heads, 64] averaged over each KV
+    head's group (in the library); key scales from E [n_kv_heads, 64]."""
+    E = np.ascontiguousarray(E, dtype=np.float64)
+    Eq = np.ascontiguousarray(Eq, dtype=np.float64)
+    out = np.zeros(E.shape[0], dtype=PLAN_DTYPE)
+    _check(lib().kvq_plan_build_weighted(ctypes.byref(cfg), layer, E.ctypes.data, Eq.ctypes.data,
+                                         Eq.shape[0], out.ctypes.data))
+    return out
+
+
+def block_energy(x, status=None, ws=None) -> np.ndarray:
+    """Exact block energies fp64 [n_heads, 64] of a device tensor
+    x [n_tokens, n_heads, 128] (e.g. calibration queries)."""
+    import torch
+    n_heads = x.shape[1]
+    if ws is None:
+        ws = torch.zeros(lib().kvq_energy_workspace_bytes(n_heads), dtype=torch.uint8,
+                         device=x.device)
+    E = np.zeros((n_heads, 64), dtype=np.float64)
+    _check(lib().kvq_block_energy(_ptr(x), _dtype_code(x), x.shape[0], n_heads, _ptr(ws),
+                                  ws.numel(), E.ctypes.data, _ptr(status), _stream()))
+    return E
 
 
 def parse_plans(raw) -> np.ndarray:

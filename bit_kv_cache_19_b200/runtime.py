@@ -39,6 +39,18 @@ class PackedLayer:
                                                       self.status)
         return self.plans_host
 
+    def alloc_bits_query_weighted(self, k, q_calib):
+        """Query-weighted variant: key energies of k [T, n_kv, 128] and query
+        energies of calibration queries q_calib [Tq, n_q, 128] (both device
+        tensors, both by the library's energy kernel); the library averages
+        the query energies over each KV head's group and runs the greedy on
+        the products."""
+        E = kvq.block_energy(k, self.status)
+        Eq = kvq.block_energy(q_calib, self.status)
+        self.set_plans(kvq.plan_build_weighted(self.cfg, self.layer, E, Eq))
+        self.energy = E
+        return self.plans_host
+
     def set_plans(self, plans_host: np.ndarray):
         """Use host plan records (e.g. from kvq.plan_build)."""
         raw = torch.from_numpy(np.frombuffer(plans_host.tobytes(), dtype=np.uint8).copy())

@@ -223,6 +223,34 @@ KVQ_API int kvq_plan_build(const kvq_cfg* cfg, int layer, const double* E_host, 
 KVQ_API int kvq_codebook(int bits, float* centroids, float* thresholds, double* distortion);
 
 /*
+ * Query-weighted allocation (a variant; the pages' score is key-only and
+ * label-free). The logit q . k is a sum of 2-D RoPE block terms q_j . k_j, so
+ * the error of key block j reaches the logit scaled by the query's block
+ * energy; weighting the greedy by calibration queries minimises
+ * sum_j W_j E_j D(b_j), the expected squared logit error, instead of
+ * sum_j E_j D(b_j).
+ *
+ * kvq_block_energy: the exact block energy E[h][j] (as in kvq_alloc_bits) of
+ *   any x_dev [n_tokens][n_heads][128] of type dtype, e.g. calibration
+ *   queries; energy_host: out, fp64 [n_heads][64]; ws_dev >=
+ *   kvq_energy_workspace_bytes(n_heads) bytes (overwritten); status_dev
+ *   optional (NONFINITE). Synchronizes `stream` once.
+ * kvq_plan_build_weighted: kvq_plan_build for the n_kv_heads KV heads with
+ *   the widths of the greedy on E_j W_j (fp64 products) and the key scales
+ *   of E. E_host: key energies [n_kv_heads][64]; Eq_host: query energies
+ *   [n_q_heads][64] (kvq_block_energy of calibration queries); W[h] is the
+ *   mean over KV head h's query group, (1/G) sum_{g<G} Eq[h G + g] summed
+ *   in increasing g, G = n_q_heads / n_kv_heads.
+ * Return KVQ_OK or a negative code (size query: 0 if invalid).
+ */
+KVQ_API size_t kvq_energy_workspace_bytes(int n_heads);
+KVQ_API int kvq_block_energy(const void* x_dev, int dtype, int64_t n_tokens, int n_heads,
+                             void* ws_dev, size_t ws_bytes, double* energy_host,
+                             uint32_t* status_dev, kvq_stream_t stream);
+KVQ_API int kvq_plan_build_weighted(const kvq_cfg* cfg, int layer, const double* E_host,
+                                    const double* Eq_host, int n_q_heads, void* plans_host);
+
+/*
  * Quantize and append n_new tokens per sequence to the packed cache
  * (Block-GTQ keys on TQ-MSE, uniform TQ-MSE values). Per token and KV head:
  *   keys:   n = fp16(sqrt(sum k_i^2)) (fixed fp32 order), r = 1/n,

@@ -115,15 +115,21 @@ class Plan:
 
 
 def make_plan(E, bits_k: int, bits_v: int, v_seed: int, layer: int, kv_head: int,
-              uniform: bool = False) -> Plan:
+              uniform: bool = False, weights=None) -> Plan:
     """Plan of one (layer, KV head) from its block energies ``E[64]``.
 
     ``uniform=True`` gives every block the width ``bits_k`` (the same key
     bytes as the greedy plan), the uniform-allocation comparator.
+    ``weights`` (query-weighted variant): the greedy runs on the products
+    E_j * W_j (fp64), i.e. minimises sum_j W_j E_j D(b_j), the expected
+    squared logit error when block j's error reaches the logit scaled by the
+    query's block energy W_j; the key scales stay those of E.
     """
     E = np.asarray(E, dtype=np.float64)
     if uniform:
         w, tie = np.full(E.shape, bits_k, dtype=np.int64), False
+    elif weights is not None:
+        w, tie = greedy(E * np.asarray(weights, dtype=np.float64), bits_k)
     else:
         w, tie = greedy(E, bits_k)
     g, ah = key_scales(E)

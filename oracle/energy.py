@@ -67,3 +67,25 @@ def block_energy(k):
     S, flags = block_energy_int(k)
     E = np.array([[float(s) / _TWO32 / T for s in row] for row in S], dtype=np.float64)
     return E, flags
+
+
+def query_weights(q, n_kv: int):
+    """Query block energies averaged over each KV head's query group.
+
+    Variant of the allocation (not the pages' label-free score): the logit
+    q . k decomposes into 2-D RoPE block terms q_j . k_j, so a quantization
+    error in block j reaches the logit scaled by the query's block-j energy.
+    For calibration queries ``q[T, Hq, 128]`` (post-RoPE; the energy is
+    RoPE-invariant) this returns Q[h][j] = (1/G) sum_{g < G} E^q_{hG+g, j}
+    (sum over g in increasing order, fp64), E^q the same exact block energy
+    as for keys, G = Hq / n_kv."""
+    Eq, flags = block_energy(q)
+    Hq = Eq.shape[0]
+    G = Hq // n_kv
+    Q = np.zeros((n_kv, Eq.shape[1]))
+    for h in range(n_kv):
+        acc = np.zeros(Eq.shape[1])
+        for g in range(G):
+            acc = acc + Eq[h * G + g]
+        Q[h] = acc / G
+    return Q, flags

@@ -139,6 +139,22 @@ def queries(wl: Workload, seed: int, layer: int, seq: int, pos: int) -> np.ndarr
     return to_bf16_bits(_rope(q, np.full(wl.n_q_heads, pos), wl.rope_base))
 
 
+def queries_anisotropic(wl: Workload, seed: int, layer: int, kv_head: int, n: int, G: int,
+                        start_pos: int) -> np.ndarray:
+    """bf16 bits q[n, G, 128] of one KV head's query group at positions
+    start_pos..start_pos+n-1, with uneven block energy: coordinates of block j
+    scaled by exp(0.75 e_j), e_j ~ N(0, 1) drawn once per (layer, KV head)
+    and shared by the group and by every seed (the seed draws the samples). A
+    query family for the query-weighted allocation study (the workloads' own
+    queries are isotropic)."""
+    sc = np.exp(0.75 * np.random.default_rng(_seq(wl.wid, layer, 2000 + kv_head)).standard_normal(HALF))
+    sc = np.concatenate([sc, sc])
+    rng = np.random.default_rng(_seq(wl.wid, seed, layer, 3000 + kv_head))
+    q = rng.standard_normal((n, G, D)) * sc[None, None, :]
+    pos = np.repeat(np.arange(start_pos, start_pos + n), G)
+    return to_bf16_bits(_rope(q.reshape(n * G, D), pos, wl.rope_base).reshape(n, G, D))
+
+
 # ---------------------------------------------------------------- torch draws
 def _torch_seed(*key) -> int:
     return int(_seq(*key).generate_state(1, np.uint64)[0] & np.uint64((1 << 63) - 1))

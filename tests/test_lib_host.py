@@ -95,6 +95,39 @@ def test_plan_build_equals_oracle(kind, bits):
             assert len(set(p["cls_w"][:p["n_class"]])) == p["n_class"]
 
 
+@pytest.mark.parametrize("bits", [(2, 2), (3, 3), (4, 2)])
+def test_plan_build_weighted_equals_oracle(bits):
+    """Query-weighted plans: the library averages the query heads' energies
+    over each group and runs the greedy on E * W; widths, order and scales
+    equal the oracle's (group mean in increasing head order, fp64)."""
+    from oracle import energy
+    rng = np.random.default_rng(sum(bits))
+    bk, bv = bits
+    n_kv, G = 2, 4
+    q = rng.standard_normal((64, n_kv * G, 128)) * np.exp(rng.standard_normal(128))[None, None]
+    Eq, _ = energy.block_energy(q)
+    W, _ = energy.query_weights(q, n_kv)
+    E = np.exp(1.5 * rng.standard_normal((n_kv, 64)) - np.arange(64) / 8.0)
+    cfg = kvq.make_cfg(n_kv, bk, bv, v_seed=3)
+    got = kvq.plan_build_weighted(cfg, 1, E, Eq)
+    plain = kvq.plan_build(cfg, 1, E)
+    for h in range(n_kv):
+        ref = alloc.make_plan(E[h], bk, bv, 3, 1, h, weights=W[h])
+        assert not ref.near_tie
+        assert np.array_equal(got[h]["width"].astype(int), ref.widths)
+        assert list(got[h]["order"][:got[h]["n_ranks"]]) == ref.order
+        assert np.array_equal(got[h]["g"], ref.g) and np.array_equal(got[h]["a_hat"], ref.a_hat)
+        assert np.array_equal(got[h]["g"], plain[h]["g"])
+    L = kvq.lib()
+    assert L.kvq_plan_build_weighted(ctypes.byref(cfg), 0, E.ctypes.data, Eq.ctypes.data, 7,
+                                     got.ctypes.data) == kvq.ERR_ARG
+    bad = Eq.copy()
+    bad[0, 0] = -1.0
+    assert L.kvq_plan_build_weighted(ctypes.byref(cfg), 0, E.ctypes.data, bad.ctypes.data, 8,
+                                     got.ctypes.data) == kvq.ERR_ARG
+    assert kvq.lib().kvq_energy_workspace_bytes(16) >= 16 * 64 * 16
+
+
 def test_sizes():
     cfg = kvq.make_cfg(2, 3, 3)
     assert kvq.tile_bytes(cfg) == 3200 == 32 * 100

@@ -102,3 +102,47 @@ def test_v_signs():
     assert s == v_signs(12345, 3, 1)
     assert s != v_signs(12345, 3, 0) and s != v_signs(12345, 2, 1)
     assert 40 < sum(1 for x in s if x > 0) < 88
+
+
+def test_query_weighted_greedy():
+    """Query-weighted variant: the widths minimise sum_j W_j E_j D(b_j)
+    (exhaustive search at 4 blocks), constant weights change nothing, and the
+    key scales stay those of E."""
+    rng = np.random.default_rng(3)
+    for seed in range(60):
+        E = np.exp(rng.standard_normal(4) * 2.0)
+        W = np.exp(rng.standard_normal(4) * 1.5)
+        for bits in (1, 2, 3, 5):
+            J = 4
+            w = alloc.greedy(E * W, bits)[0]
+            best, arg, n_best = _brute(E * W, bits)
+            f = float((_DTAB[w] * E * W).sum())
+            assert f <= best * (1 + 1e-12)
+            if n_best == 1:
+                assert tuple(w) == arg
+            assert int(w.sum()) == J * bits
+    E = np.exp(rng.standard_normal(64))
+    W = np.exp(rng.standard_normal(64))
+    base = alloc.make_plan(E, 3, 3, 1, 0, 0)
+    for c in (1.0, 2.0, 0.125):           # powers of two: E * c is exact
+        p = alloc.make_plan(E, 3, 3, 1, 0, 0, weights=np.full(64, c))
+        assert np.array_equal(p.widths, base.widths)
+    pw = alloc.make_plan(E, 3, 3, 1, 0, 0, weights=W)
+    assert np.array_equal(pw.g, base.g) and np.array_equal(pw.a_hat, base.a_hat)
+    assert int(pw.widths.sum()) == 64 * 3 and not np.array_equal(pw.widths, base.widths)
+
+
+def test_query_weights_group_mean():
+    """W[h] is the mean block energy of KV head h's query group: identical
+    query heads give their own energy; two heads give the average."""
+    from oracle import energy
+    rng = np.random.default_rng(4)
+    q = rng.standard_normal((50, 4, 128))
+    q[:, 1] = q[:, 0]
+    W, _ = energy.query_weights(q, 2)
+    Eq, _ = energy.block_energy(q)
+    assert np.array_equal(W[0], Eq[0])          # (a + a) / 2 = a exactly
+    assert np.allclose(W[1], (Eq[2] + Eq[3]) / 2, rtol=1e-15, atol=0)
+    # and each block energy is the textbook mean of the block's squared length
+    ref = (q[:, 2, :64] ** 2 + q[:, 2, 64:] ** 2).mean(axis=0)
+    assert np.allclose(Eq[2], ref, rtol=1e-9, atol=0)

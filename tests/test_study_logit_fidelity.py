@@ -71,3 +71,37 @@ def test_block_gtq_lowers_logit_error_vs_uniform_tqmse(bits):
               f"        {r['tqmse']:.5f}       {100 * red:5.1f} %")
         assert r["greedy"] < r["tqmse"]
         assert r["greedy"] <= r["uniform"] * 1.0001
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+def test_query_weighted_allocation_on_anisotropic_queries(bits):
+    """Query-weighted variant (not the pages' key-only score): with queries
+    whose block energies are uneven (synth.queries_anisotropic), widths from
+    the greedy on E_j W_j, W the calibration queries' group-mean block
+    energy, lower the key-logit error on held-out queries of the same family
+    against the key-only Block-GTQ plan. 256 calibration positions, 64
+    evaluation positions after them; mean |q.(k - k_hat)| / sqrt(128)."""
+    rows = []
+    for wname in ("llama8b", "qwen3b_128k"):
+        wl = synth.WORKLOADS[wname]
+        G = wl.n_q_heads // wl.n_kv_heads
+        for layer, h in ((0, 0), (5, 1)):
+            kb, _ = synth.keys_values(wl, 11, layer, h, T)
+            k = synth.bf16_bits_to_f64(kb)
+            qc = synth.bf16_bits_to_f64(synth.queries_anisotropic(wl, 11, layer, h, 256, G, T))
+            qe = synth.bf16_bits_to_f64(
+                synth.queries_anisotropic(wl, 12, layer, h, 64, G, T + 256)).reshape(-1, 128)
+            E, _ = energy.block_energy(k[:, None, :])
+            W, _ = energy.query_weights(qc, 1)
+            res = {}
+            for mode, wts in (("key-only", None), ("query-weighted", W[0])):
+                plan = alloc.make_plan(E[0], bits, 2, 5, layer, h, weights=wts)
+                kc, kn, _ = quant.quantize_keys(k, plan)
+                res[mode] = _mae(qe, k, attn.dequant_keys(kc, kn, plan))
+            rows.append((wname, layer, h, res))
+    print(f"\nK{bits}: mean |logit error|, anisotropic queries   key-only   query-weighted   reduction")
+    for wname, layer, h, r in rows:
+        red = 1.0 - r["query-weighted"] / r["key-only"]
+        print(f"  {wname:12s} L{layer} h{h}   {r['key-only']:.5f}   {r['query-weighted']:.5f}"
+              f"   {100 * red:5.1f} %")
+        assert r["query-weighted"] < r["key-only"]
