@@ -61,7 +61,8 @@ int check_cfg(const kvq_cfg* cfg) {
   if (cfg->bits_k < 1 || cfg->bits_k > 8) return fail(KVQ_ERR_ARG, "bits_k %d not in 1..8", cfg->bits_k);
   if (cfg->bits_v < 1 || cfg->bits_v > 8) return fail(KVQ_ERR_ARG, "bits_v %d not in 1..8", cfg->bits_v);
   if (cfg->b_max != 8) return fail(KVQ_ERR_ARG, "b_max %d (must be 8)", cfg->b_max);
-  if (cfg->alloc_mode != KVQ_ALLOC_GREEDY && cfg->alloc_mode != KVQ_ALLOC_UNIFORM)
+  const int mode = cfg->alloc_mode & ~KVQ_ALLOC_ROTATE_KEYS;
+  if (mode != KVQ_ALLOC_GREEDY && mode != KVQ_ALLOC_UNIFORM)
     return fail(KVQ_ERR_ARG, "alloc_mode %d", cfg->alloc_mode);
   return KVQ_OK;
 }
@@ -108,7 +109,7 @@ void build_plan(const kvq_cfg* cfg, int layer, int kv_head, const double* E, Pla
   pl->kv_head = kv_head;
   pl->words_k = 128 * cfg->bits_k;
   pl->words_v = 128 * cfg->bits_v;
-  if (cfg->alloc_mode == KVQ_ALLOC_UNIFORM) {
+  if ((cfg->alloc_mode & ~KVQ_ALLOC_ROTATE_KEYS) == KVQ_ALLOC_UNIFORM) {
     for (int j = 0; j < kBlocks; ++j) pl->width[j] = (uint8_t)cfg->bits_k;
   } else if (W) {
     double EW[kBlocks];
@@ -167,6 +168,11 @@ void build_plan(const kvq_cfg* cfg, int layer, int kv_head, const double* E, Pla
   const uint64_t key = splitmix64(cfg->v_seed, ((uint64_t)(uint32_t)layer << 32) + (uint32_t)kv_head);
   for (int i = 0; i < kHeadDim; ++i)
     if (splitmix64(key, (uint64_t)i) >> 63) pl->v_sign[i >> 5] |= 1u << (i & 31);
+  if (cfg->alloc_mode & KVQ_ALLOC_ROTATE_KEYS) {  // key rotation signs: outputs 128 + P
+    pl->k_rot = 1;
+    for (int P = 0; P < kHeadDim; ++P)
+      if (splitmix64(key, (uint64_t)(kHeadDim + P)) >> 63) pl->k_sign[P >> 5] |= 1u << (P & 31);
+  }
 }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }

@@ -41,7 +41,10 @@ struct Plan {
   uint8_t cls_nhs[8];
   uint8_t cls_last[8];     // blocks in the class's last half step
   uint16_t cls_seg0[8];    // first K word of the class in a tile record
-  uint8_t tail[KVQ_PLAN_BYTES - 984];
+  uint32_t k_sign[4];      // key rotation: bit P set <=> sign of plan position P is -1
+  uint8_t k_rot;           // 1: keys rotated inside each width group
+  uint8_t pad3[3];
+  uint8_t tail[KVQ_PLAN_BYTES - 1004];
 };
 static_assert(sizeof(Plan) == KVQ_PLAN_BYTES, "plan size");
 static_assert(offsetof(Plan, g) == 32 && offsetof(Plan, a_hat) == 288, "plan layout");
@@ -51,6 +54,7 @@ static_assert(offsetof(Plan, hs_width) == 804 && offsetof(Plan, v_sign) == 900, 
 static_assert(offsetof(Plan, energy_sum) == 920, "plan layout");
 static_assert(offsetof(Plan, n_class) == 928 && offsetof(Plan, cls_w) == 936, "plan layout");
 static_assert(offsetof(Plan, cls_last) == 960 && offsetof(Plan, cls_seg0) == 968, "plan layout");
+static_assert(offsetof(Plan, k_sign) == 984 && offsetof(Plan, k_rot) == 1000, "plan layout");
 
 // Codebook offsets: width w centroids at 2^w - 2, thresholds at 2^w - w - 1.
 __host__ __device__ constexpr int cb_c_off(int w) { return (1 << w) - 2; }

@@ -109,6 +109,7 @@ struct alignas(128) Smem {
   int8_t qj[kMaxHalf][4];        // per half step: block of MMA column c, or -1
   int len0, is_last;
   uint32_t flags;
+  RotTables rot;                   // key rotation tables (plans with k_rot)
 };
 
 // Bulk-copy destinations start on 16-byte boundaries.
@@ -343,6 +344,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   const bool bad = !ok_setup || sm.plan.magic != KVQ_PLAN_MAGIC || sm.plan.bits_v != BV ||
                    bk < 1 || bk > 8 || p.tile_bytes != tile_bytes(bk, BV) || n_half < 1 ||
                    n_half > kMaxHalf || sm.plan.n_class < 1 || sm.plan.n_class > 8 ||
+                   sm.plan.n_ranks < 1 || sm.plan.n_ranks > 64 ||
                    (reinterpret_cast<uintptr_t>(cache0) & 15) != 0;
   if (bad && tid == 0) atomicOr(p.status, ok_setup ? KVQ_FLAG_BAD_PLAN : KVQ_FLAG_TIMEOUT);
   const int len0 = sm.len0;
@@ -421,7 +423,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
       const int off = sm.plan.cls_seg0[ci] + 2 * W * (ln & 3) + ((W * (ln >> 2)) >> 2);
       sm.cls_lane[ci][ln] = ((uint32_t)off << 8) | ((uint32_t)(8 * W * (ln >> 2)) & 31u);
     }
+    if (sm.plan.k_rot && tid == kThreads - 1) rot_tables(sm.plan, sm.rot);
   }
+  __syncthreads();  // the tables above are read by every warp
   if (p.early) grid_dep_wait();
   grid_dep_launch();
 
@@ -462,6 +466,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
         }
       }
       __syncthreads();
+      if (sm.plan.k_rot) {  // key rotation inside width groups, one warp per new token
+        for (int pp = p_lo + warp; pp < p_hi; pp += kWarps)
+          warp_rotate_row(kz + pp * kKzStride, sm.plan, sm.rot, sm.plan.g, lane);
+        __syncthreads();
+      }
       for (int r = warp; r < sm.plan.n_ranks; r += kWarps)
         warp_block_pass(sm.plan, sm.thr, r, kz, p_lo, p_hi, lane, sw, clear);
       __syncthreads();
@@ -505,34 +514,41 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
     //      q' = q a_hat_j log2(e) / sqrt(128); per-head 2^sigma scaling into
     //      the fp16 range; hi/lo split into the B fragments of each half step
     float* qp = reinterpret_cast<float*>(scratch);  // [8 NT][128]
+    const bool krot = sm.plan.k_rot != 0;
     for (int head = warp; head < 8 * NT; head += kWarps) {  // warp-local: one head each
-      float v[4], mx = 0.f;
+      float* row = qp + head * kHeadDim;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int x = lane + 32 * i;
-        v[i] = 0.f;
+        float v = 0.f;
         if (head < G) {
           const size_t qi = ((size_t)b * p.n_q + h * G + head) * kHeadDim + x;
-          v[i] = load_as_float(p.q, p.q_dtype, qi) * sm.plan.a_hat[x & 63] * 0.12751743074f;
+          v = load_as_float(p.q, p.q_dtype, qi) * sm.plan.a_hat[x & 63] * 0.12751743074f;
         }  // 0.12751743 = log2(e) / sqrt(128)
-        mx = fmaxf(mx, fabsf(v[i]));
+        row[x] = v;
       }
+      __syncwarp();
+      // rotated plans: the same per-chunk rotation as the keys, so that
+      // q'~ . y_hat = q' . z_hat; the row is then indexed by plan position
+      if (krot) warp_rotate_row(row, sm.plan, sm.rot, nullptr, lane);
+      float mx = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (!krot || lane + 32 * i < sm.rot.npos) mx = fmaxf(mx, fabsf(row[lane + 32 * i]));
 #pragma unroll
       for (int m = 16; m; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
       const int sigma = (mx > 0.f && isfinite(mx)) ? 14 - ilogbf(mx) : 0;
       const float sc = ldexpf(1.f, sigma);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) qp[head * kHeadDim + lane + 32 * i] = v[i] * sc;
       if (lane == 0) sm.inv_scale[head] = ldexpf(1.f, -sigma);
-      __syncwarp();
       // this head's B-fragment entries: lane 4 (head mod 8) + c of each half step
       const int nt = head >> 3, g8 = head & 7;
       for (int e = lane; e < n_half * 4; e += 32) {
         const int hs = e >> 2, cc = e & 3, j = sm.qj[hs][cc];
         float x0 = 0.f, x1 = 0.f;
         if (j >= 0) {
-          x0 = qp[head * kHeadDim + j];
-          x1 = qp[head * kHeadDim + j + 64];
+          const int i0 = krot ? 2 * (sm.plan.hs_rank0[hs] + cc) : j;
+          x0 = row[i0] * sc;
+          x1 = row[krot ? i0 + 1 : j + 64] * sc;
         }
         const uint32_t hi = pack_half2(x0, x1);
         const __half2 hh = *reinterpret_cast<const __half2*>(&hi);

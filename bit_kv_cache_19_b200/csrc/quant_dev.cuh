@@ -179,14 +179,99 @@ __device__ __forceinline__ void warp_token_pass(const Plan& pl, const float* thr
   }
 }
 
+// ---- key rotation inside width groups (plan.k_rot)
+// Plan position P = 2 r + e is coordinate order[r] + 64 e. A width group (the
+// ranks of one width) holds 2 n positions, cut into chunks by the binary
+// expansion of 2 n, largest first. Tables (shared memory): rank of each block
+// (0xFF for width 0); first position and log2 size of each position's chunk.
+struct RotTables {
+  uint8_t rank_of[64];
+  uint8_t base[128];
+  uint8_t lg[128];
+  int npos;
+};
+
+__device__ __forceinline__ void rot_tables(const Plan& pl, RotTables& t) {  // one thread
+  for (int j = 0; j < 64; ++j) t.rank_of[j] = 0xFF;
+  for (int r = 0; r < pl.n_ranks; ++r) t.rank_of[pl.order[r] & 63] = (uint8_t)r;
+  for (int r = 0; r < pl.n_ranks;) {
+    const int w = pl.width[pl.order[r]];
+    int n = 1;
+    while (r + n < pl.n_ranks && pl.width[pl.order[r + n]] == w) ++n;
+    int P = 2 * r;
+    for (int e = 7; e >= 0; --e)
+      if ((2 * n) & (1 << e)) {
+        for (int q = 0; q < (1 << e); ++q) {
+          t.base[P + q] = (uint8_t)P;
+          t.lg[P + q] = (uint8_t)e;
+        }
+        P += 1 << e;
+      }
+    r += n;
+  }
+  t.npos = 2 * pl.n_ranks;
+}
+
+// Chunk factor c(2^e) = 2^-floor(e/2), times fp32(sqrt(1/2)) for odd e.
+__device__ __forceinline__ float rot_scale(int e) {
+  const float base = (e & 1) ? 0.70710678118654752f : 1.f;
+  return __fmul_rn(base, __int_as_float((127 - (e >> 1)) << 23));
+}
+
+// One warp rotates one row in place: in, 128 values in coordinate order (times
+// gs[j] when gs is given, one fp32 product); out, positions [0, npos):
+// u_P = s_P x, the fp32 butterflies h = 1, 2, ... inside each chunk, then
+// y_P = fp32(h_P c(size)).
+__device__ __forceinline__ void warp_rotate_row(float* row, const Plan& pl, const RotTables& t,
+                                                const float* gs, int lane) {
+  float v[4];
+  int P[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int i = lane + 32 * q, j = i & 63, rk = t.rank_of[j];
+    P[q] = rk == 0xFF ? -1 : 2 * rk + (i >> 6);
+    float x = row[i];
+    if (gs) x = __fmul_rn(x, gs[j]);
+    if (P[q] >= 0 && ((pl.k_sign[P[q] >> 5] >> (P[q] & 31)) & 1u)) x = -x;
+    v[q] = x;
+  }
+  __syncwarp();
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    if (P[q] >= 0) row[P[q]] = v[q];
+  __syncwarp();
+  for (int h = 1; h < 128; h <<= 1) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int p = lane + 32 * q;
+      if (p < t.npos && (1 << t.lg[p]) > h && ((p - t.base[p]) & h) == 0) {
+        const float a = row[p], b = row[p + h];
+        row[p] = __fadd_rn(a, b);
+        row[p + h] = __fsub_rn(a, b);
+      }
+    }
+    __syncwarp();
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int p = lane + 32 * q;
+    if (p < t.npos) row[p] = __fmul_rn(row[p], rot_scale(t.lg[p]));
+  }
+  __syncwarp();
+}
+
 // Pass 2 for stored block rank r, positions [p_lo, p_hi) (lane = position).
+// Without rotation the row holds k r by coordinate (z = (k r) g_j); with it,
+// the rotated y by plan position (2 r, 2 r + 1).
 template <int W>
 __device__ __forceinline__ void block_field(const Plan& pl, const float* thr, int r, int j,
                                             const float* row, int lane, uint32_t* words,
-                                            bool clear) {
+                                            bool clear, bool rot) {
   const float g = pl.g[j];
-  const uint32_t c0 = (uint32_t)code_of_w<W>(thr, __fmul_rn(row[j], g));
-  const uint32_t c1 = (uint32_t)code_of_w<W>(thr, __fmul_rn(row[j + 64], g));
+  const float z0 = rot ? row[2 * r] : __fmul_rn(row[j], g);
+  const float z1 = rot ? row[2 * r + 1] : __fmul_rn(row[j + 64], g);
+  const uint32_t c0 = (uint32_t)code_of_w<W>(thr, z0);
+  const uint32_t c1 = (uint32_t)code_of_w<W>(thr, z1);
   put_field(words, 32 * pl.seg_off[r] + slot_k(lane) * 2 * W, c0 | (c1 << W), 2 * W, clear);
 }
 
@@ -194,17 +279,18 @@ __device__ __forceinline__ void warp_block_pass(const Plan& pl, const float* thr
                                                 const float* kz, int p_lo, int p_hi, int lane,
                                                 uint32_t* words, bool clear) {
   const int j = pl.order[r], w = pl.width[j];
+  const bool rot = pl.k_rot != 0;
   if (lane < p_lo || lane >= p_hi) return;
   const float* row = kz + lane * kKzStride;
   switch (w) {  // uniform in the warp
-    case 1: block_field<1>(pl, thr, r, j, row, lane, words, clear); break;
-    case 2: block_field<2>(pl, thr, r, j, row, lane, words, clear); break;
-    case 3: block_field<3>(pl, thr, r, j, row, lane, words, clear); break;
-    case 4: block_field<4>(pl, thr, r, j, row, lane, words, clear); break;
-    case 5: block_field<5>(pl, thr, r, j, row, lane, words, clear); break;
-    case 6: block_field<6>(pl, thr, r, j, row, lane, words, clear); break;
-    case 7: block_field<7>(pl, thr, r, j, row, lane, words, clear); break;
-    default: block_field<8>(pl, thr, r, j, row, lane, words, clear); break;
+    case 1: block_field<1>(pl, thr, r, j, row, lane, words, clear, rot); break;
+    case 2: block_field<2>(pl, thr, r, j, row, lane, words, clear, rot); break;
+    case 3: block_field<3>(pl, thr, r, j, row, lane, words, clear, rot); break;
+    case 4: block_field<4>(pl, thr, r, j, row, lane, words, clear, rot); break;
+    case 5: block_field<5>(pl, thr, r, j, row, lane, words, clear, rot); break;
+    case 6: block_field<6>(pl, thr, r, j, row, lane, words, clear, rot); break;
+    case 7: block_field<7>(pl, thr, r, j, row, lane, words, clear, rot); break;
+    default: block_field<8>(pl, thr, r, j, row, lane, words, clear, rot); break;
   }
 }
 

@@ -103,6 +103,7 @@ __global__ void __launch_bounds__(256, 4) quantize_append_kernel(QuantParams p) 
   __shared__ uint32_t s_words[kHeadDim * 16 + 1];  // + slack word for put_field
   __shared__ uint32_t s_flags;
   __shared__ double s_theta[64];
+  __shared__ RotTables s_rot;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   for (int i = threadIdx.x; i < KVQ_CB_N_THR; i += blockDim.x) s_thr[i] = c_thr[i];
   for (int i = threadIdx.x; i < 64; i += blockDim.x) s_theta[i] = p.theta[i];
@@ -139,7 +140,10 @@ __global__ void __launch_bounds__(256, 4) quantize_append_kernel(QuantParams p) 
       __syncthreads();
       cur = bh;
       plan_ok = s_plan.magic == KVQ_PLAN_MAGIC && s_plan.bits_k >= 1 && s_plan.bits_k <= 8 &&
-                s_plan.bits_v == BV && p.tile_bytes == tile_bytes(s_plan.bits_k, BV);
+                s_plan.bits_v == BV && p.tile_bytes == tile_bytes(s_plan.bits_k, BV) &&
+                s_plan.n_ranks >= 1 && s_plan.n_ranks <= 64;
+      if (plan_ok && s_plan.k_rot && threadIdx.x == 0) rot_tables(s_plan, s_rot);
+      __syncthreads();
     }
     if (!plan_ok) {
       if (threadIdx.x == 0) atomicOr(p.status, KVQ_FLAG_BAD_PLAN);
@@ -170,6 +174,11 @@ __global__ void __launch_bounds__(256, 4) quantize_append_kernel(QuantParams p) 
     }
     if (flags) atomicOr(&s_flags, flags);
     __syncthreads();
+    if (pl.k_rot) {  // ---- key rotation inside width groups, one warp per new token
+      for (int pp = p_lo + warp; pp < p_hi; pp += nw)
+        warp_rotate_row(s_kz + pp * kKzStride, pl, s_rot, pl.g, lane);
+      __syncthreads();
+    }
     // ---- pass 2: one warp per stored key block
     for (int r = warp; r < pl.n_ranks; r += nw)
       warp_block_pass(pl, s_thr, r, s_kz, p_lo, p_hi, lane, s_words, clear);

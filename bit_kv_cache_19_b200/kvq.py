@@ -21,6 +21,7 @@ FLAG_CAPACITY, FLAG_NONFINITE, FLAG_NORM_SAT, FLAG_TIMEOUT, FLAG_BAD_PLAN = 1, 2
 FLAG_BAD_PAGE = 32
 BF16, FP16, FP32 = 0, 1, 2
 ALLOC_GREEDY, ALLOC_UNIFORM = 0, 1
+ALLOC_ROTATE_KEYS = 0x100
 STEP_EARLY = 1
 STEP_ROPE = 2
 PLAN_BYTES = 1024
@@ -35,7 +36,8 @@ PLAN_DTYPE = np.dtype([
     ("hs_rank0", "u1", 32), ("hs_count", "u1", 32), ("v_sign", "<u4", 4), ("pad1", "<u4"),
     ("energy_sum", "<f8"), ("n_class", "u1"), ("pad2", "u1", 7), ("cls_w", "u1", 8),
     ("cls_hs0", "u1", 8), ("cls_nhs", "u1", 8), ("cls_last", "u1", 8), ("cls_seg0", "<u2", 8),
-    ("tail", "u1", PLAN_BYTES - 984),
+    ("k_sign", "<u4", 4), ("k_rot", "u1"), ("pad3", "u1", 3),
+    ("tail", "u1", PLAN_BYTES - 1004),
 ])
 assert PLAN_DTYPE.itemsize == PLAN_BYTES
 

@@ -78,6 +78,8 @@ typedef struct CUstream_st* kvq_stream_t;
 /* Allocation modes. */
 #define KVQ_ALLOC_GREEDY 0   /* Block-GTQ: greedy marginal-gain widths per RoPE block */
 #define KVQ_ALLOC_UNIFORM 1  /* every block gets bits_k (same bytes; comparator) */
+#define KVQ_ALLOC_ROTATE_KEYS 0x100 /* OR-ed into alloc_mode: rotate keys inside each group of
+                                       blocks of one width before coding (plan field k_rot) */
 
 typedef struct {
   int32_t head_dim;    /* must be 128 */
@@ -85,7 +87,7 @@ typedef struct {
   int32_t bits_k;      /* key budget, bits per dimension, 1..8 (K in KxVy) */
   int32_t bits_v;      /* value width, bits per dimension, 1..8 (V in KxVy) */
   int32_t b_max;       /* largest width of one block, must be 8 */
-  int32_t alloc_mode;  /* KVQ_ALLOC_GREEDY or KVQ_ALLOC_UNIFORM */
+  int32_t alloc_mode;  /* KVQ_ALLOC_GREEDY or KVQ_ALLOC_UNIFORM, optionally | KVQ_ALLOC_ROTATE_KEYS */
   uint64_t v_seed;     /* seed of the value sign flips */
 } kvq_cfg;
 
@@ -119,7 +121,23 @@ typedef struct {
  *   off 952  uint8   cls_nhs[8]     half steps in the class
  *   off 960  uint8   cls_last[8]    blocks in the class's last half step
  *   off 968  uint16  cls_seg0[8]    first K word of the class in a tile record
- *   off 984  .. 1023 zero
+ *   off 984  uint32  k_sign[4]      key rotation: bit P set <=> sign of plan position P is -1
+ *   off 1000 uint8   k_rot          1: keys rotated inside each width group (see below)
+ *   off 1001 .. 1023 zero
+ *
+ * Key rotation (KVQ_ALLOC_ROTATE_KEYS; the alternative reading of "built on
+ * TQ-MSE" for keys, which spreads outlier coordinates before coding). Plan
+ * position P = 2 r + e is coordinate order[r] + 64 e. A width group (the
+ * ranks of one class) holds 2 n positions, cut into chunks by the binary
+ * expansion of 2 n (largest first). Per token, after z_i = (k_i * r) * g_j
+ * as without rotation: u_P = s_P z_P, the fp32 FWHT graph over each chunk
+ * (stages h = 1, 2, ... < size, pairs (P, P + h) with (P - chunk start) & h
+ * == 0 become (a + b, a - b)), y_P = fp32(h_P * c(size)), c(2^e) =
+ * 2^-floor(e/2) times fp32(sqrt(1/2)) for odd e; y_P is coded at the group's
+ * width into the slot of coordinate order[r] + 64 e. Signs: s_P = -1 iff bit
+ * 63 of SplitMix64(key, 128 + P) is set (key as for the value signs).
+ * Decode rotates the query the same way (q~ = c H (s . q') per chunk), so
+ * q . k_hat needs no inverse transform per token.
  */
 #define KVQ_PLAN_BYTES 1024
 #define KVQ_PLAN_MAGIC 0x5051564Bu /* "KVQP" */

@@ -23,6 +23,8 @@ dimension on keys, y on values). Readings adopted where the abstract is silent:
 * Plan order: blocks with b_j > 0 sorted by width (descending), then block
   index (ascending). Zero-width blocks are not stored.
 * Values use the uniform width b_V on every coordinate.
+* Per-width-group key rotation (optional, the alternative reading of "built
+  on TQ-MSE" for keys): see ``rot_chunks`` and ``quant.quantize_keys``.
 """
 from __future__ import annotations
 
@@ -31,7 +33,7 @@ from dataclasses import dataclass, field
 import numpy as np
 
 from . import lloydmax
-from .splitmix import v_signs
+from .splitmix import k_signs, v_signs
 
 B_MAX = 8
 NEAR_TIE_REL = 1e-9
@@ -104,6 +106,8 @@ class Plan:
     signs: np.ndarray           # [128] +-1 (float64)
     energy: np.ndarray = field(default=None)
     near_tie: bool = False
+    k_rot: bool = False         # per-width-group key rotation (reading D22)
+    k_signs: np.ndarray = field(default=None)  # [128] +-1 by plan position
 
     @property
     def words_k(self) -> int:
@@ -114,8 +118,29 @@ class Plan:
         return 4 * self.bits_v
 
 
+def rot_chunks(widths, order):
+    """Chunks of the per-width-group key rotation, as (first position, size,
+    width). Plan position P = 2 r + e is coordinate order[r] + 64 e of rank r.
+    A width group is a maximal run of equal-width ranks (2 n positions); it is
+    cut into chunks by the binary expansion of 2 n, largest first."""
+    out = []
+    r = 0
+    while r < len(order):
+        w = int(widths[order[r]])
+        n = 1
+        while r + n < len(order) and int(widths[order[r + n]]) == w:
+            n += 1
+        P, m = 2 * r, 2 * n
+        for e in range(7, -1, -1):
+            if m & (1 << e):
+                out.append((P, 1 << e, w))
+                P += 1 << e
+        r += n
+    return out
+
+
 def make_plan(E, bits_k: int, bits_v: int, v_seed: int, layer: int, kv_head: int,
-              uniform: bool = False, weights=None) -> Plan:
+              uniform: bool = False, weights=None, rotate_keys: bool = False) -> Plan:
     """Plan of one (layer, KV head) from its block energies ``E[64]``.
 
     ``uniform=True`` gives every block the width ``bits_k`` (the same key
@@ -134,5 +159,6 @@ def make_plan(E, bits_k: int, bits_v: int, v_seed: int, layer: int, kv_head: int
         w, tie = greedy(E, bits_k)
     g, ah = key_scales(E)
     s = np.array(v_signs(v_seed, layer, kv_head, 2 * len(E)), dtype=np.float64)
+    ks = np.array(k_signs(v_seed, layer, kv_head), dtype=np.float64) if rotate_keys else None
     return Plan(bits_k=bits_k, bits_v=bits_v, widths=w, order=plan_order(w), g=g,
-                a_hat=ah, signs=s, energy=E, near_tie=tie)
+                a_hat=ah, signs=s, energy=E, near_tie=tie, k_rot=rotate_keys, k_signs=ks)

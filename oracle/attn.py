@@ -36,6 +36,19 @@ def dequant_keys(codes, norms, plan) -> np.ndarray:
     half = d // 2
     out = np.zeros((T, d), dtype=np.float64)
     n = np.asarray(norms, dtype=np.float64)
+    if getattr(plan, "k_rot", False):
+        # per chunk: z = s . (H y_hat) / sqrt(size) (the orthonormal inverse)
+        from .alloc import rot_chunks
+        order = list(plan.order)
+        coord = [order[P // 2] + half * (P % 2) for P in range(2 * len(order))]
+        for P0, sz, w in rot_chunks(plan.widths, order):
+            c = lloydmax.centroids(w)
+            yh = np.stack([c[codes[:, coord[P0 + q]]] for q in range(sz)], axis=1)
+            zh = (yh @ hadamard(sz)) / np.sqrt(sz) * plan.k_signs[P0:P0 + sz][None, :]
+            for q in range(sz):
+                i = coord[P0 + q]
+                out[:, i] = n * float(plan.a_hat[i % half]) * zh[:, q]
+        return out
     for j in range(half):
         w = int(plan.widths[j])
         if w == 0:

@@ -11,8 +11,9 @@ summary (Hadamard rotation on values) support a Walsh-Hadamard rotation.
 
 Readings adopted:
 
-Keys (per token, per KV head). No rotation across blocks (it would mix the
-blocks whose widths differ). n = fp16 norm of the whole 128-vector; each
+Keys (per token, per KV head). No rotation across blocks of different widths
+(it would mix the blocks whose widths differ); optionally a rotation inside
+each group of equal width (``quantize_keys``). n = fp16 norm of the whole 128-vector; each
 coordinate i of block j is scaled to z_i = k_i * (1/n) * g_j and coded with
 the width-b_j Lloyd-Max thresholds.
 
@@ -104,15 +105,43 @@ def _norm_and_recip(x32):
     return n, r, fin, flags
 
 
+def rot_scale(size: int) -> np.float32:
+    """fp32 factor of a rotation chunk of 2^e positions: 2^-floor(e/2), times
+    fp32(sqrt(1/2)) for odd e (an exact power-of-two scaling of one fp32)."""
+    e = int(size).bit_length() - 1
+    base = np.float32(np.sqrt(0.5)) if e % 2 else np.float32(1.0)
+    return np.float32(np.ldexp(base, -(e // 2)))
+
+
 def quantize_keys(k, plan):
     """Key codes [T, 128] (canonical coords; unused for width-0 blocks), fp16
-    norms as float32 [T], per-token flags [T]."""
+    norms as float32 [T], per-token flags [T].
+
+    With plan.k_rot (per-width-group rotation): z is formed as without it;
+    then per plan position P = 2 r + e (coordinate order[r] + 64 e),
+    u_P = s_P z_P; each chunk of ``alloc.rot_chunks`` takes the fp32 FWHT
+    graph over its positions and y_P = fp32(h_P * rot_scale(size)); the code
+    of position P (width of its group) is stored at coordinate order[r] + 64 e."""
     k32 = np.asarray(k, dtype=np.float32)
     T, d = k32.shape
     half = d // 2
     n, r, fin, flags = _norm_and_recip(k32)
     codes = np.zeros((T, d), dtype=np.int64)
     live = fin & (n > 0)
+    if getattr(plan, "k_rot", False):
+        from .alloc import rot_chunks
+        order = list(plan.order)
+        coord = [order[P // 2] + half * (P % 2) for P in range(2 * len(order))]
+        with np.errstate(invalid="ignore", over="ignore"):
+            u = np.zeros((T, 2 * len(order)), dtype=np.float32)
+            for P, i in enumerate(coord):
+                z = (k32[:, i] * r) * plan.g[i % half]
+                u[:, P] = -z if plan.k_signs[P] < 0 else z
+            for P0, sz, w in rot_chunks(plan.widths, order):
+                y = fwht_f32(u[:, P0:P0 + sz]) * rot_scale(sz)
+                for q in range(sz):
+                    codes[:, coord[P0 + q]] = np.where(live, codes_from_z(y[:, q], w), 0)
+        return codes, n, flags
     with np.errstate(invalid="ignore", over="ignore"):
         for j in range(half):
             w = int(plan.widths[j])

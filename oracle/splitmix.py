@@ -35,3 +35,11 @@ def v_signs(v_seed: int, layer: int, kv_head: int, d: int = 128):
     """Sign vector (list of +-1) of the value rotation of one (layer, KV head)."""
     key = splitmix64(v_seed, (layer << 32) + kv_head)
     return [-1 if (splitmix64(key, i) >> 63) else 1 for i in range(d)]
+
+
+def k_signs(v_seed: int, layer: int, kv_head: int, n: int = 128):
+    """Signs of the per-width-group key rotation (when it is on): plan position
+    P = 0..n-1 takes output 128 + P of the same stream as the value signs,
+    -1 if its bit 63 is set."""
+    key = splitmix64(v_seed, (layer << 32) + kv_head)
+    return [-1 if (splitmix64(key, 128 + P) >> 63) else 1 for P in range(n)]

@@ -14,7 +14,7 @@ def energies(k_heads):
 
 
 def layer(k_heads, v_heads, bits_k, bits_v, v_seed, layer_idx, uniform=False, E=None,
-          window=None, pack=True):
+          window=None, pack=True, rotate_keys=False):
     """Oracle plans, tile records, dequantized caches for one layer.
 
     k_heads / v_heads: per KV head float arrays [T, 128] holding bf16 values.
@@ -27,7 +27,8 @@ def layer(k_heads, v_heads, bits_k, bits_v, v_seed, layer_idx, uniform=False, E=
         E, _ = energies([k[:w] for k in k_heads])
     out = []
     for h, (k, v) in enumerate(zip(k_heads, v_heads)):
-        plan = alloc.make_plan(E[h], bits_k, bits_v, v_seed, layer_idx, h, uniform=uniform)
+        plan = alloc.make_plan(E[h], bits_k, bits_v, v_seed, layer_idx, h, uniform=uniform,
+                               rotate_keys=rotate_keys)
         kc, kn, kf = quant.quantize_keys(k, plan)
         vc, vn, vf = quant.quantize_values(v, plan)
         rec = layout.pack(kc, vc, kn, vn, plan, T) if pack else None

@@ -128,6 +128,32 @@ def test_plan_build_weighted_equals_oracle(bits):
     assert kvq.lib().kvq_energy_workspace_bytes(16) >= 16 * 64 * 16
 
 
+@pytest.mark.parametrize("bits", [(1, 1), (3, 3), (8, 2)])
+def test_plan_build_rotate_keys_equals_oracle(bits):
+    """KVQ_ALLOC_ROTATE_KEYS: same widths, order and scales as without it;
+    k_rot set and the key signs of the oracle's SplitMix64 positions."""
+    from oracle.splitmix import k_signs
+    rng = np.random.default_rng(bits[0] * 9 + bits[1])
+    E = np.exp(1.5 * rng.standard_normal((2, 64)) - np.arange(64) / 8.0)
+    bk, bv = bits
+    for mode in (kvq.ALLOC_GREEDY, kvq.ALLOC_UNIFORM):
+        cfg0 = kvq.make_cfg(2, bk, bv, v_seed=55, alloc_mode=mode)
+        cfg1 = kvq.make_cfg(2, bk, bv, v_seed=55, alloc_mode=mode | kvq.ALLOC_ROTATE_KEYS)
+        p0 = kvq.plan_build(cfg0, 4, E)
+        p1 = kvq.plan_build(cfg1, 4, E)
+        for h in range(2):
+            ref = alloc.make_plan(E[h], bk, bv, 55, 4, h, uniform=mode == kvq.ALLOC_UNIFORM,
+                                  rotate_keys=True)
+            assert p0[h]["k_rot"] == 0 and p1[h]["k_rot"] == 1
+            assert np.array_equal(p1[h]["width"], p0[h]["width"])
+            assert np.array_equal(p1[h]["g"], p0[h]["g"])
+            sg = [-1 if (p1[h]["k_sign"][P >> 5] >> (P & 31)) & 1 else 1 for P in range(128)]
+            assert sg == k_signs(55, 4, h) == ref.k_signs.tolist()
+    bad = kvq.make_cfg(2, 3, 3, alloc_mode=0x200)
+    assert kvq.lib().kvq_plan_build(ctypes.byref(bad), 0, E.ctypes.data, 1,
+                                    np.zeros(1, kvq.PLAN_DTYPE).ctypes.data) == kvq.ERR_ARG
+
+
 def test_sizes():
     cfg = kvq.make_cfg(2, 3, 3)
     assert kvq.tile_bytes(cfg) == 3200 == 32 * 100
