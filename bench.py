@@ -57,6 +57,8 @@ def parse():
                     help="override the context length (points of the qwen3b_sweep)")
     ap.add_argument("--alloc", default="greedy", choices=["greedy", "uniform"],
                     help="Block-GTQ greedy widths, or every block at the key budget")
+    ap.add_argument("--rotate-keys", action="store_true",
+                    help="plans with the per-width-group key rotation (KVQ_ALLOC_ROTATE_KEYS)")
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--layers", type=int, default=0,
@@ -251,8 +253,10 @@ def run_kvq(args, wl, rank, world, dist):
     steps, warmup = args.steps, args.warmup
     n_step = max(1, wl.n_new)  # tokens appended per sequence and layer in a step
     cap = T + (steps + warmup + max(3, steps // 2) + 4) * n_step + 64
-    cfg = kvq.make_cfg(wl.n_kv_heads, wl.bits_k, wl.bits_v, v_seed=1234,
-                       alloc_mode=kvq.ALLOC_UNIFORM if args.alloc == "uniform" else kvq.ALLOC_GREEDY)
+    mode = kvq.ALLOC_UNIFORM if args.alloc == "uniform" else kvq.ALLOC_GREEDY
+    if args.rotate_keys:
+        mode |= kvq.ALLOC_ROTATE_KEYS
+    cfg = kvq.make_cfg(wl.n_kv_heads, wl.bits_k, wl.bits_v, v_seed=1234, alloc_mode=mode)
     bpth = BYTES_PER_TOKEN_HEAD(wl.bits_k, wl.bits_v)
 
     # ---- prefill: energies + greedy plans, bulk quantize-append (timed);
@@ -480,7 +484,8 @@ def run_kvq(args, wl, rank, world, dist):
         "config": {"workload": wl.name, "layers": n_layers, "q_heads": wl.n_q_heads,
                    "kv_heads": wl.n_kv_heads, "head_dim": 128, "context": T, "batch": B,
                    "budget": f"K{wl.bits_k}V{wl.bits_v}",
-                   "alloc": "Block-GTQ greedy" if args.alloc == "greedy" else "uniform",
+                   "alloc": ("Block-GTQ greedy" if args.alloc == "greedy" else "uniform")
+                            + (", width-group key rotation" if args.rotate_keys else ""),
                    "appended_per_step": n_step,
                    "step": f"per layer, one fused launch: quantize-append {n_step} token(s) "
                            "per sequence + packed decode attention",

@@ -423,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
       const int off = sm.plan.cls_seg0[ci] + 2 * W * (ln & 3) + ((W * (ln >> 2)) >> 2);
       sm.cls_lane[ci][ln] = ((uint32_t)off << 8) | ((uint32_t)(8 * W * (ln >> 2)) & 31u);
     }
-    if (sm.plan.k_rot && tid == kThreads - 1) rot_tables(sm.plan, sm.rot);
+    if (sm.plan.k_rot) rot_tables(sm.plan, sm.rot, tid);
   }
   __syncthreads();  // the tables above are read by every warp
   if (p.early) grid_dep_wait();

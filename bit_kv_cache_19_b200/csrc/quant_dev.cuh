@@ -191,25 +191,32 @@ struct RotTables {
   int npos;
 };
 
-__device__ __forceinline__ void rot_tables(const Plan& pl, RotTables& t) {  // one thread
-  for (int j = 0; j < 64; ++j) t.rank_of[j] = 0xFF;
-  for (int r = 0; r < pl.n_ranks; ++r) t.rank_of[pl.order[r] & 63] = (uint8_t)r;
-  for (int r = 0; r < pl.n_ranks;) {
-    const int w = pl.width[pl.order[r]];
-    int n = 1;
-    while (r + n < pl.n_ranks && pl.width[pl.order[r + n]] == w) ++n;
-    int P = 2 * r;
-    for (int e = 7; e >= 0; --e)
-      if ((2 * n) & (1 << e)) {
-        for (int q = 0; q < (1 << e); ++q) {
-          t.base[P + q] = (uint8_t)P;
-          t.lg[P + q] = (uint8_t)e;
-        }
-        P += 1 << e;
-      }
-    r += n;
+// Built by the threads of a CTA in one parallel step (a barrier must follow):
+// thread x < 128 fills position x from the plan's classes (a class is the
+// run of ranks of one width), thread x < 64 block x's rank entry.
+__device__ __forceinline__ void rot_tables(const Plan& pl, RotTables& t, int x) {
+  if (x < 64) {
+    if (pl.width[x] == 0) t.rank_of[x] = 0xFF;          // not stored
+    if (x < pl.n_ranks) t.rank_of[pl.order[x] & 63] = (uint8_t)x;  // blocks of width > 0
   }
-  t.npos = 2 * pl.n_ranks;
+  if (x == 0) t.npos = 2 * pl.n_ranks;
+  if (x >= 2 * pl.n_ranks || x >= 128) return;
+  const int r = x >> 1;
+  int ci = 0;
+  while (ci + 1 < pl.n_class && ci + 1 < 8 && pl.hs_rank0[pl.cls_hs0[ci + 1] & 31] <= r) ++ci;
+  const int r0 = pl.hs_rank0[pl.cls_hs0[ci] & 31];
+  const int m = 2 * (4 * (pl.cls_nhs[ci] - 1) + pl.cls_last[ci]);  // positions of the group
+  const int local = x - 2 * r0;
+  int off = 0;
+  for (int e = 7; e >= 0; --e)
+    if (m & (1 << e)) {
+      if (local < off + (1 << e)) {
+        t.base[x] = (uint8_t)(2 * r0 + off);
+        t.lg[x] = (uint8_t)e;
+        return;
+      }
+      off += 1 << e;
+    }
 }
 
 // Chunk factor c(2^e) = 2^-floor(e/2), times fp32(sqrt(1/2)) for odd e.
@@ -225,7 +232,7 @@ __device__ __forceinline__ float rot_scale(int e) {
 __device__ __forceinline__ void warp_rotate_row(float* row, const Plan& pl, const RotTables& t,
                                                 const float* gs, int lane) {
   float v[4];
-  int P[4];
+  int P[4], sz[4], loc[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const int i = lane + 32 * q, j = i & 63, rk = t.rank_of[j];
@@ -234,17 +241,22 @@ __device__ __forceinline__ void warp_rotate_row(float* row, const Plan& pl, cons
     if (gs) x = __fmul_rn(x, gs[j]);
     if (P[q] >= 0 && ((pl.k_sign[P[q] >> 5] >> (P[q] & 31)) & 1u)) x = -x;
     v[q] = x;
+    // this lane's butterfly positions p = lane + 32 q: chunk size and offset
+    const int p = lane + 32 * q;
+    sz[q] = p < t.npos ? 1 << (t.lg[p] & 7) : 0;
+    loc[q] = p < t.npos ? p - t.base[p] : 0;
   }
   __syncwarp();
 #pragma unroll
   for (int q = 0; q < 4; ++q)
     if (P[q] >= 0) row[P[q]] = v[q];
   __syncwarp();
+#pragma unroll
   for (int h = 1; h < 128; h <<= 1) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int p = lane + 32 * q;
-      if (p < t.npos && (1 << t.lg[p]) > h && ((p - t.base[p]) & h) == 0) {
+      if (sz[q] > h && (loc[q] & h) == 0 && p + h < t.npos) {
         const float a = row[p], b = row[p + h];
         row[p] = __fadd_rn(a, b);
         row[p + h] = __fsub_rn(a, b);
@@ -255,7 +267,7 @@ __device__ __forceinline__ void warp_rotate_row(float* row, const Plan& pl, cons
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const int p = lane + 32 * q;
-    if (p < t.npos) row[p] = __fmul_rn(row[p], rot_scale(t.lg[p]));
+    if (sz[q]) row[p] = __fmul_rn(row[p], rot_scale(31 - __clz(sz[q])));
   }
   __syncwarp();
 }

@@ -151,3 +151,43 @@ def test_rotated_full_size_qwen3b_layer():
     out = L.decode(dev_bf16(qb)[None], max_len=T).cpu().numpy()[0]
     _, heads = op.layer(kh, vh, wl.bits_k, wl.bits_v, 99, 9, E=E, pack=False, rotate_keys=True)
     assert op.rel_err(out, op.decode(synth.bf16_bits_to_f64(qb), heads)) <= TOL
+
+
+def test_rotated_edge_tokens_and_paged_cache():
+    """Rotated plans with a non-finite key, a non-finite value, a zero key and
+    a key whose norm saturates fp16: codes and norms bit-exact against the
+    oracle; the same tokens in a paged cache (shuffled 1-tile pages) give the
+    same records and the same decode output."""
+    from bit_kv_cache_19_b200.runtime import PagedLayer
+    rng = np.random.default_rng(8)
+    n_kv, T = 1, 90
+    cfg = kvq.make_cfg(n_kv, 3, 3, v_seed=2, alloc_mode=ROT)
+    E = np.exp(rng.standard_normal((n_kv, 64)))
+    kb, vb = _random_kv(rng, n_kv, T, E)
+    k = synth.bf16_bits_to_f64(kb)
+    v = synth.bf16_bits_to_f64(vb)
+    k[5, 0, 17] = np.nan
+    v[9, 0, 3] = np.inf
+    k[11, 0, :] = 0.0
+    k[12, 0, :] = 3e38
+    kb, vb = synth.to_bf16_bits(k), synth.to_bf16_bits(v)
+    plans = kvq.plan_build(cfg, 0, E)
+    L = PackedLayer(cfg, 1, 96)
+    L.set_plans(plans)
+    L.append(dev_bf16(kb)[None], dev_bf16(vb)[None])
+    P = PagedLayer(cfg, 1, 5, 1, 3)
+    P.set_plans(plans)
+    P.reserve(0, T, order=[4, 1, 3])
+    P.append(dev_bf16(kb)[None], dev_bf16(vb)[None])
+    torch.cuda.synchronize()
+    fl = L.flags()
+    assert fl & kvq.FLAG_NONFINITE and fl & kvq.FLAG_NORM_SAT and P.flags() == fl
+    kh, vh = op.bf16_heads(kb, vb)
+    _, heads = op.layer(kh, vh, 3, 3, 2, 0, E=E, rotate_keys=True)
+    check_records(L.head_records(0, 0, 3), heads[0]["rec"], T, 3, 3)
+    assert np.array_equal(P.head_records(0, 0, 3), L.head_records(0, 0, 3))
+    qb = synth.to_bf16_bits(rng.standard_normal((1, 8, 128)))
+    out = L.decode(dev_bf16(qb), max_len=96).cpu().numpy()
+    out_p = P.decode(dev_bf16(qb), max_len=96).cpu().numpy()
+    assert op.rel_err(out[0], op.decode(synth.bf16_bits_to_f64(qb[0]), heads)) <= TOL
+    assert op.rel_err(out_p[0], out[0]) <= 1e-5
