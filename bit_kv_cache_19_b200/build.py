@@ -45,7 +45,8 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
         with open(header, "w") as f:
             f.write(out)
     srcs = [os.path.join(CSRC, s) for s in SOURCES]
-    deps = srcs + [header, os.path.join(CSRC, "common.cuh"), os.path.join(ROOT, "include", "kvq.h")]
+    headers = sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h")))
+    deps = srcs + headers + [header, os.path.join(ROOT, "include", "kvq.h")]
     if force or _stale(LIB, deps):
         objs = []
         for s in srcs:

@@ -252,23 +252,50 @@ __device__ __forceinline__ void warp_rotate_row(float* row, const Plan& pl, cons
     if (P[q] >= 0) row[P[q]] = v[q];
   __syncwarp();
 #pragma unroll
-  for (int h = 1; h < 128; h <<= 1) {
+  for (int q = 0; q < 4; ++q) v[q] = row[lane + 32 * q];  // position order
+  // butterflies h < 32 across lanes: the partner of position p is p + h
+  // (lower element) or p - h (upper), in this or the neighbouring register
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
+    float nv[4];
+    const int s_lo = (lane + h) & 31, s_up = (lane - h) & 31;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const int p = lane + 32 * q;
-      if (sz[q] > h && (loc[q] & h) == 0 && p + h < t.npos) {
-        const float a = row[p], b = row[p + h];
-        row[p] = __fadd_rn(a, b);
-        row[p + h] = __fsub_rn(a, b);
+      const float a0 = __shfl_sync(0xffffffffu, v[q], s_lo);
+      const float a1 = __shfl_sync(0xffffffffu, v[q < 3 ? q + 1 : q], s_lo);
+      const float b0 = __shfl_sync(0xffffffffu, v[q], s_up);
+      const float b1 = __shfl_sync(0xffffffffu, v[q > 0 ? q - 1 : q], s_up);
+      const float lo_partner = lane + h < 32 ? a0 : a1;
+      const float up_partner = lane >= h ? b0 : b1;
+      nv[q] = v[q];
+      if (sz[q] > h)
+        nv[q] = (loc[q] & h) == 0 ? __fadd_rn(v[q], lo_partner) : __fsub_rn(up_partner, v[q]);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) v[q] = nv[q];
+  }
+  // h = 32, 64: the partner is in this lane, register q +- h / 32
+#pragma unroll
+  for (int k = 1; k <= 2; k <<= 1) {
+    const int h = 32 * k;
+    float nv[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      nv[q] = v[q];
+      if (sz[q] > h) {
+        if ((loc[q] & h) == 0) {
+          if (q + k < 4) nv[q] = __fadd_rn(v[q], v[q + k]);
+        } else {
+          if (q - k >= 0) nv[q] = __fsub_rn(v[q - k], v[q]);
+        }
       }
     }
-    __syncwarp();
+#pragma unroll
+    for (int q = 0; q < 4; ++q) v[q] = nv[q];
   }
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int p = lane + 32 * q;
-    if (sz[q]) row[p] = __fmul_rn(row[p], rot_scale(31 - __clz(sz[q])));
-  }
+  for (int q = 0; q < 4; ++q)
+    if (sz[q]) row[lane + 32 * q] = __fmul_rn(v[q], rot_scale(31 - __clz(sz[q])));
   __syncwarp();
 }
 
