@@ -600,6 +600,20 @@ int kvq_paged_decode_attn(const kvq_cfg* cfg, const void* const* plans_dev, cons
                      out_dev, nullptr, ws_dev, ws_bytes, status_dev, stream);
 }
 
+int kvq_paged_decode_attn_partial(const kvq_cfg* cfg, const void* const* plans_dev,
+                                  const kvq_pages* pages, const int32_t* len_dev, int batch,
+                                  int64_t max_len, const void* q_dev, int q_dtype,
+                                  int n_q_heads, float* rec_dev, void* ws_dev, size_t ws_bytes,
+                                  uint32_t* status_dev, kvq_stream_t stream) {
+  CacheMap cm;
+  int64_t cap = 0;
+  int rc = paged_map(cfg, pages, &cm, &cap);
+  if (rc) return rc;
+  if (!rec_dev) return fail(KVQ_ERR_ARG, "null device pointer");
+  return decode_impl(cfg, plans_dev, cm, len_dev, batch, max_len, q_dev, q_dtype, n_q_heads,
+                     nullptr, rec_dev, ws_dev, ws_bytes, status_dev, stream);
+}
+
 int kvq_paged_append_decode(const kvq_cfg* cfg, const void* const* plans_dev, const void* k_dev,
                             const void* v_dev, int kv_dtype, int n_new, const kvq_pages* pages,
                             int32_t* len_dev, int batch, int64_t max_len, const void* q_dev,

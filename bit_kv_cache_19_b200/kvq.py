@@ -106,6 +106,9 @@ _SIGS = {
                                          ctypes.POINTER(Pages), _vp, ctypes.c_double, _vp, _vp]),
     "kvq_paged_decode_attn": (_i32, [ctypes.POINTER(Cfg), _vp, ctypes.POINTER(Pages), _vp, _i32,
                                      _i64, _vp, _i32, _i32, _vp, _vp, _sz, _vp, _vp]),
+    "kvq_paged_decode_attn_partial": (_i32, [ctypes.POINTER(Cfg), _vp, ctypes.POINTER(Pages),
+                                             _vp, _i32, _i64, _vp, _i32, _i32, _vp, _vp, _sz,
+                                             _vp, _vp]),
     "kvq_paged_append_decode": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i32,
                                        ctypes.POINTER(Pages), _vp, _i32, _i64, _vp, _i32, _i32,
                                        _vp, _vp, _sz, _i32, ctypes.c_double, _vp, _vp]),
@@ -319,6 +322,16 @@ def paged_decode_attn(cfg, plan_ptrs, pages, lens, max_len, q, out, ws, status):
                                        _ptr(lens), batch, max_len, _ptr(q), _dtype_code(q), n_q,
                                        _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
                                        _ptr(status), _stream()))
+
+
+def paged_decode_attn_partial(cfg, plan_ptrs, pages, lens, max_len, q, rec, ws, status):
+    """kvq_decode_attn_partial over paged caches: records fp32 [batch, n_q, 132]."""
+    batch, n_q = q.shape[0], q.shape[1]
+    _check(lib().kvq_paged_decode_attn_partial(ctypes.byref(cfg), _ptr(plan_ptrs),
+                                               ctypes.byref(pages), _ptr(lens), batch, max_len,
+                                               _ptr(q), _dtype_code(q), n_q, _ptr(rec), _ptr(ws),
+                                               ws.numel() * ws.element_size(), _ptr(status),
+                                               _stream()))
 
 
 def paged_append_decode(cfg, plan_ptrs, k, v, pages, lens, max_len, q, out, ws, status,

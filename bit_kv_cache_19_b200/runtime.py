@@ -231,6 +231,29 @@ class PagedLayer:
                               ws, self.status)
         return out
 
+    def decode_partial(self, q, rec=None, ws=None, max_len=None):
+        """This pool's sequences as one context shard: records [batch, n_q, 132]."""
+        max_len = self.cap if max_len is None else max_len
+        if rec is None:
+            rec = torch.empty((q.shape[0], q.shape[1], kvq.REC_FLOATS), dtype=torch.float32,
+                              device=self.device)
+        if ws is None:
+            ws = self.workspace(q.shape[1], max_len)
+        kvq.paged_decode_attn_partial(self.cfg, self.plan_ptrs, self.pages, self.lens, max_len,
+                                      q, rec, ws, self.status)
+        return rec
+
+    def combine(self, recs, out=None):
+        """Outputs [batch, n_q, 128] from stacked shard records [n_parts, batch, n_q, 132]."""
+        if out is None:
+            out = torch.empty(recs.shape[1:3] + (128,), dtype=torch.float32, device=self.device)
+        kvq.combine_partials(self.cfg, self.plan_ptrs, recs, out)
+        return out
+
+    def decode_sharded(self, q, group=None, max_len=None):
+        """Context-sharded decode over ranks (this rank's pool holds its range)."""
+        return sharded_decode(lambda: self.decode_partial(q, max_len=max_len), self.combine, group)
+
     def append_decode(self, k, v, q, out=None, ws=None, max_len=None, step_flags=0,
                       rope_base=0.0):
         max_len = self.cap if max_len is None else max_len

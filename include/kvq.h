@@ -471,6 +471,13 @@ KVQ_API int kvq_paged_decode_attn(const kvq_cfg* cfg, const void* const* plans_d
                                   int64_t max_len, const void* q_dev, int q_dtype, int n_q_heads,
                                   float* out_dev, void* ws_dev, size_t ws_bytes,
                                   uint32_t* status_dev, kvq_stream_t stream);
+/* kvq_decode_attn_partial over paged caches (one context shard's records). */
+KVQ_API int kvq_paged_decode_attn_partial(const kvq_cfg* cfg, const void* const* plans_dev,
+                                          const kvq_pages* pages, const int32_t* len_dev,
+                                          int batch, int64_t max_len, const void* q_dev,
+                                          int q_dtype, int n_q_heads, float* rec_dev,
+                                          void* ws_dev, size_t ws_bytes, uint32_t* status_dev,
+                                          kvq_stream_t stream);
 /* kvq_append_decode over paged caches (capacity from the block table). */
 KVQ_API int kvq_paged_append_decode(const kvq_cfg* cfg, const void* const* plans_dev,
                                     const void* k_dev, const void* v_dev, int kv_dtype, int n_new,

@@ -190,3 +190,35 @@ def test_paged_qwen3b_64k():
     assert P.flags() == 0
     _, heads = op.layer(kh, vh, wl.bits_k, wl.bits_v, 6, 3, E=E, pack=False)
     assert op.rel_err(out, op.decode(synth.bf16_bits_to_f64(qb), heads)) <= TOL
+
+
+def test_paged_context_shards_combine():
+    """A sequence split into a paged shard and a contiguous shard: the combine
+    of the paged partial records and the contiguous ones equals the decode of
+    one cache holding every token."""
+    rng = np.random.default_rng(21)
+    n_kv, G, T, cut = 2, 8, 900, 420
+    cfg = kvq.make_cfg(n_kv, 3, 3, v_seed=9)
+    E = np.exp(rng.standard_normal((n_kv, 64)) - np.arange(64) / 9.0)
+    plans = kvq.plan_build(cfg, 1, E)
+    kb, vb = _random_kv(rng, n_kv, T, E)
+    P = PagedLayer(cfg, 1, 20, 2, 10)
+    P.set_plans(plans)
+    P.reserve(0, cut, order=list(rng.permutation(20)))
+    P.append(dev_bf16(kb[:cut])[None], dev_bf16(vb[:cut])[None])
+    C = PackedLayer(cfg, 1, T - cut)
+    C.set_plans(plans)
+    C.append(dev_bf16(kb[cut:])[None], dev_bf16(vb[cut:])[None])
+    F = PackedLayer(cfg, 1, T)
+    F.set_plans(plans)
+    F.append(dev_bf16(kb)[None], dev_bf16(vb)[None])
+    qb = synth.to_bf16_bits(rng.standard_normal((1, n_kv * G, 128)))
+    q = dev_bf16(qb)
+    recs = torch.stack([P.decode_partial(q), C.decode_partial(q, max_len=T)])
+    out = P.combine(recs).cpu().numpy()
+    ref = F.decode(q).cpu().numpy()
+    assert P.flags() == 0 and C.flags() == 0
+    assert op.rel_err(out, ref) <= 1e-3
+    kh, vh = op.bf16_heads(kb, vb)
+    heads = op.layer(kh, vh, 3, 3, 9, 1, E=E, pack=False)[1]
+    assert op.rel_err(out[0], op.decode(synth.bf16_bits_to_f64(qb[0]), heads)) <= TOL
