@@ -1,6 +1,6 @@
 // Packed-cache decode attention (optionally fused with the append of the
-// step's new tokens): split-K over the context with an in-kernel two-level
-// merge of the splits.
+// step's new tokens): split-K over the context, the splits summed inside the
+// same kernel (exponent buckets in L2, read by the last split).
 //
 // "RoPE-Aware Bit Allocation for KV-Cache Quantization", abstract: the
 // packed-cache serving path runs decode attention directly on the packed
@@ -78,7 +78,7 @@ struct DecodeParams {
   int q_dtype;
   int n_q, n_kv, G;
   int max_len;
-  int n_splits, tiles_per_split, n_groups;
+  int n_splits, tiles_per_split;
   int tile_bytes;
   // fused append (n_new > 0)
   const void* k_new;
@@ -926,7 +926,7 @@ static int ctas_per_sm_bv(int dev, int bits_k, int bv, cudaError_t* err) {
 }
 
 struct SplitPlan {
-  int n_splits, tiles_per_split, n_groups;
+  int n_splits, tiles_per_split;
 };
 
 // Splits per (sequence, KV head) so that the grid is about one wave of the
@@ -934,7 +934,7 @@ struct SplitPlan {
 // queries on a host without GPU) an upper bound of the CTA slots is used.
 static SplitPlan decode_split_plan(int batch, int n_kv, int G, int bits_k, int bits_v,
                                    int64_t max_len, cudaError_t* err, bool allow_fallback) {
-  SplitPlan sp{1, 1, 1};
+  SplitPlan sp{1, 1};
   int64_t slots = kFallbackSlots;
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -959,7 +959,6 @@ static SplitPlan decode_split_plan(int batch, int n_kv, int G, int bits_k, int b
   s = std::min<int64_t>(s, kMaxSplits);
   sp.tiles_per_split = (int)((tiles + s - 1) / s);
   sp.n_splits = (int)((tiles + sp.tiles_per_split - 1) / sp.tiles_per_split);
-  sp.n_groups = (sp.n_splits + kGroup - 1) / kGroup;
   return sp;
 }
 
@@ -969,13 +968,13 @@ static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 // k at a fixed distance from the end, so calls sharing one workspace, for one
 // n_kv_heads, never overwrite each other's counters).
 static size_t decode_workspace_layout(int batch, int n_kv, int G, const SplitPlan& sp,
-                                      size_t* gpart_off) {
+                                      size_t* bkt_off) {
   const size_t pairs = (size_t)batch * n_kv;
   const size_t part = align256(pairs * sp.n_splits * G * kPartStride * sizeof(float));
-  const size_t gpart = align256(pairs * G * kBuckets * kPartStride * sizeof(float));
+  const size_t bkt = align256(pairs * G * kBuckets * kPartStride * sizeof(float));
   const size_t counters = align256(pairs * kCntStride * sizeof(unsigned int));
-  if (gpart_off) *gpart_off = part;
-  return part + gpart + counters;
+  if (bkt_off) *bkt_off = part;
+  return part + bkt + counters;
 }
 
 // Workspace bytes of a decode call on the current device (an upper bound if
@@ -1031,8 +1030,8 @@ cudaError_t launch_decode(const Plan* const* plans, const CacheMap& cm, int32_t*
   const int G = n_q / n_kv;
   const SplitPlan sp = decode_split_plan(batch, n_kv, G, bits_k, bits_v, max_len, &err, false);
   if (err != cudaSuccess) return err;
-  size_t gpart_off = 0;
-  if (decode_workspace_layout(batch, n_kv, G, sp, &gpart_off) > ws_bytes)
+  size_t bkt_off = 0;
+  if (decode_workspace_layout(batch, n_kv, G, sp, &bkt_off) > ws_bytes)
     return cudaErrorInvalidValue;
   if (n_new < 0 || n_new > kMaxNew) return cudaErrorInvalidValue;
   DecodeParams p;
@@ -1047,7 +1046,6 @@ cudaError_t launch_decode(const Plan* const* plans, const CacheMap& cm, int32_t*
   p.max_len = (int)max_len;
   p.n_splits = sp.n_splits;
   p.tiles_per_split = sp.tiles_per_split;
-  p.n_groups = sp.n_groups;
   p.tile_bytes = tile_bytes(bits_k, bits_v);
   p.k_new = k_new;
   p.v_new = v_new;
@@ -1058,7 +1056,7 @@ cudaError_t launch_decode(const Plan* const* plans, const CacheMap& cm, int32_t*
   p.rope = theta ? 1 : 0;
   for (int j = 0; j < 64; ++j) p.theta[j] = theta ? theta[j] : 0.0;
   p.part = reinterpret_cast<float*>(ws);
-  p.bkt = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + gpart_off);
+  p.bkt = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + bkt_off);
   p.cnt_end = reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(ws) +
                                               (ws_bytes & ~size_t(3)));
   p.out = out;
