@@ -134,3 +134,29 @@ def test_width_group_rotation_lowers_logit_error(bits):
         print(f"  {wname:12s} L{layer} h{h}   {r[False]:.5f}     {r[True]:.5f}            "
               f"{100 * red:5.1f} %")
         assert r[True] < r[False]
+
+
+def test_rotation_and_query_weighting_combine():
+    """The two variants act on different things (the quantizer, the widths):
+    with anisotropic queries, rotated keys under query-weighted widths give the
+    lowest key-logit error of the four combinations (K3, both workloads)."""
+    bits = 3
+    print("\nK3, anisotropic queries: key-only | +rotation | +query weights | both")
+    for wname in ("llama8b", "qwen3b_128k"):
+        wl = synth.WORKLOADS[wname]
+        G = wl.n_q_heads // wl.n_kv_heads
+        layer, h = 5, 1
+        kb, _ = synth.keys_values(wl, 11, layer, h, T)
+        k = synth.bf16_bits_to_f64(kb)
+        qc = synth.bf16_bits_to_f64(synth.queries_anisotropic(wl, 11, layer, h, 256, G, T))
+        qe = synth.bf16_bits_to_f64(
+            synth.queries_anisotropic(wl, 12, layer, h, 64, G, T + 256)).reshape(-1, 128)
+        E, _ = energy.block_energy(k[:, None, :])
+        W, _ = energy.query_weights(qc, 1)
+        res = []
+        for rot, wts in ((False, None), (True, None), (False, W[0]), (True, W[0])):
+            plan = alloc.make_plan(E[0], bits, 2, 5, layer, h, weights=wts, rotate_keys=rot)
+            kc, kn, _ = quant.quantize_keys(k, plan)
+            res.append(_mae(qe, k, attn.dequant_keys(kc, kn, plan)))
+        print(f"  {wname:12s} " + "  ".join(f"{x:.5f}" for x in res))
+        assert res[3] == min(res)
