@@ -112,9 +112,10 @@ def decode_source_hash():
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload):
-    """Per-launch DRAM bytes of the decode kernel from a committed ncu summary,
-    only if it was taken on the current decode source."""
+def profiled(workload, key):
+    """A per-launch counter of the decode kernel (DRAM bytes, warp
+    instructions) from a committed ncu summary, only if it was taken on the
+    current decode source."""
     p = os.path.join(ROOT, "profiles", "decode_traffic.json")
     if not os.path.exists(p):
         return None
@@ -123,7 +124,11 @@ def profiled_traffic(workload):
     e = d.get(workload)
     if not e or e.get("source_hash") != decode_source_hash():
         return None
-    return e.get("dram_bytes_per_launch")
+    return e.get(key)
+
+
+def profiled_traffic(workload):
+    return profiled(workload, "dram_bytes_per_launch")
 
 
 class ClockSampler:
@@ -507,6 +512,7 @@ def run_kvq(args, wl, rank, world, dist):
                      "bytes_per_launch": bytes_launch, "launch_us": launch_ms * 1e3,
                      "launch_timing": "timed region / launches in it",
                      "isolated_launch_us": iso_launch_ms * 1e3},
+        "issue_roofline": issue_roofline(wl.name, launch_ms, clocks),
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
@@ -515,6 +521,23 @@ def run_kvq(args, wl, rank, world, dist):
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
+
+
+def issue_roofline(workload, launch_ms, clocks):
+    """The decode kernel against the instruction-issue ceiling (it is bound by
+    issue, not by HBM): warp instructions per launch (ncu, same source) over
+    the launch time, against 148 SMs x 4 schedulers x 1 warp instruction per
+    cycle at the SM clock sampled during the timed region."""
+    import torch
+    inst = profiled(workload, "warp_inst_per_launch")
+    if inst is None or not clocks or not clocks.get("sm_mhz"):
+        return None
+    n_sm = torch.cuda.get_device_properties(0).multi_processor_count
+    peak = n_sm * 4 * clocks["sm_mhz"] * 1e6 / 1e9
+    achieved = inst / (launch_ms * 1e-3) / 1e9
+    return {"bound": "issue", "achieved": achieved, "peak": peak, "unit": "G warp-inst/s",
+            "frac": achieved / peak, "warp_inst_per_launch": inst,
+            "peak_basis": f"{n_sm} SMs x 4 schedulers x 1 inst/cycle x {clocks['sm_mhz']:.0f} MHz"}
 
 
 def main():
