@@ -238,6 +238,10 @@ def test_argument_errors_without_gpu():
     assert L.kvq_paged_quantize_append(ctypes.byref(cfg), p, p, p, 0, 1, 1, ctypes.byref(pg), p,
                                        0.5, p, None) == kvq.ERR_ARG
     assert b"rope_base" in L.kvq_last_error()
+    assert L.kvq_paged_decode_attn_partial(ctypes.byref(cfg), p, ctypes.byref(pg), p, 1, 10, p,
+                                           0, 16, None, p, 1 << 30, p, None) == kvq.ERR_ARG
+    assert L.kvq_paged_decode_attn_partial(ctypes.byref(cfg), p, ctypes.byref(pg), p, 1, 10, p,
+                                           0, 16, p, p, 8, p, None) == kvq.ERR_WORKSPACE
     # zero new tokens is a no-op
     assert L.kvq_quantize_append(ctypes.byref(cfg), p, None, None, 0, 1, 0, p, p, 10, p,
                                  None) == kvq.OK
