@@ -57,6 +57,9 @@ def parse():
                     help="override the context length (points of the qwen3b_sweep)")
     ap.add_argument("--alloc", default="greedy", choices=["greedy", "uniform"],
                     help="Block-GTQ greedy widths, or every block at the key budget")
+    ap.add_argument("--paged", type=int, default=0,
+                    help="paged caches with this many 32-token tiles per page (pages handed "
+                         "out in a shuffled order); 0: one contiguous cache per sequence")
     ap.add_argument("--rotate-keys", action="store_true",
                     help="plans with the per-width-group key rotation (KVQ_ALLOC_ROTATE_KEYS)")
     ap.add_argument("--no-graph", action="store_true")
@@ -251,7 +254,7 @@ def run_kvq(args, wl, rank, world, dist):
     import torch
 
     from bit_kv_cache_19_b200 import kvq
-    from bit_kv_cache_19_b200.runtime import PackedLayer
+    from bit_kv_cache_19_b200.runtime import PackedLayer, PagedLayer
 
     dev = torch.device("cuda", torch.cuda.current_device())
     n_layers, B, T = args.layers or wl.n_layers, wl.batch, args.context or wl.context
@@ -272,7 +275,14 @@ def run_kvq(args, wl, rank, world, dist):
     t_alloc = t_quant = 0.0
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for li in range(n_layers):
-        L = PackedLayer(cfg, B, cap, device=dev, layer=li)
+        if args.paged:
+            per_seq = -(-cap // (32 * args.paged))
+            L = PagedLayer(cfg, B, B * per_seq, args.paged, per_seq, device=dev, layer=li)
+            order = [int(x) for x in np.random.default_rng(li).permutation(B * per_seq)]
+            for b in range(B):
+                L.reserve(b, cap, order=order)
+        else:
+            L = PackedLayer(cfg, B, cap, device=dev, layer=li)
         ks, vs = [], []
         for b in range(B):
             k, v = synth.keys_values_torch(wl, rank_seed(args.seed, rank, b), li, T, dev)
@@ -328,8 +338,12 @@ def run_kvq(args, wl, rank, world, dist):
     def step():
         # one launch per layer: quantize-append the new token, then decode
         for li, L in enumerate(layers):
-            kvq.append_decode(cfg, L.plan_ptrs, knew[li], vnew[li], L.cache_ptrs, L.lens, cap,
-                              cap, qs[li], outs[li], ws, L.status, kvq.STEP_EARLY)
+            if args.paged:
+                kvq.paged_append_decode(cfg, L.plan_ptrs, knew[li], vnew[li], L.pages, L.lens,
+                                        cap, qs[li], outs[li], ws, L.status, kvq.STEP_EARLY)
+            else:
+                kvq.append_decode(cfg, L.plan_ptrs, knew[li], vnew[li], L.cache_ptrs, L.lens,
+                                  cap, cap, qs[li], outs[li], ws, L.status, kvq.STEP_EARLY)
 
     stream = torch.cuda.Stream(device=dev)
     graph = None
@@ -434,8 +448,12 @@ def run_kvq(args, wl, rank, world, dist):
             for li, L in enumerate(layers):
                 a, b = evs[r * n_layers + li]
                 a.record(stream)
-                kvq.decode_attn(cfg, L.plan_ptrs, L.cache_ptrs, L.lens, cap, qs[li], outs[li],
-                                ws, L.status)
+                if args.paged:
+                    kvq.paged_decode_attn(cfg, L.plan_ptrs, L.pages, L.lens, cap, qs[li],
+                                          outs[li], ws, L.status)
+                else:
+                    kvq.decode_attn(cfg, L.plan_ptrs, L.cache_ptrs, L.lens, cap, qs[li],
+                                    outs[li], ws, L.status)
                 b.record(stream)
         stream.synchronize()
         per_launch = [a.elapsed_time(b) for a, b in evs[n_layers:]]  # skip first pass
@@ -492,6 +510,9 @@ def run_kvq(args, wl, rank, world, dist):
                    "alloc": ("Block-GTQ greedy" if args.alloc == "greedy" else "uniform")
                             + (", width-group key rotation" if args.rotate_keys else ""),
                    "appended_per_step": n_step,
+                   "cache": (f"paged: {args.paged} tiles ({32 * args.paged} tokens) per page, "
+                             "pages in shuffled order" if args.paged
+                             else "one contiguous cache per sequence"),
                    "step": f"per layer, one fused launch: quantize-append {n_step} token(s) "
                            "per sequence + packed decode attention",
                    "l2": (f"inputs larger than L2 ({n_layers}-layer packed cache "

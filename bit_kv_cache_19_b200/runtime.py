@@ -211,6 +211,12 @@ class PagedLayer:
         self.lens[seq] = 0
 
     # ---------------------------------------------------------- calls
+    def alloc_bits(self, k):
+        """Plans from keys k [T, n_kv, 128] (device), as PackedLayer.alloc_bits."""
+        self.plans_host, self.energy = kvq.alloc_bits(self.cfg, self.layer, k, self.plans,
+                                                      self.status)
+        return self.plans_host
+
     def set_plans(self, plans_host: np.ndarray):
         raw = torch.from_numpy(np.frombuffer(plans_host.tobytes(), dtype=np.uint8).copy())
         self.plans.copy_(raw.to(self.device))
