@@ -48,7 +48,8 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     headers = sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h")))
     deps = srcs + headers + [header, os.path.join(ROOT, "include", "kvq.h")]
     if force or _stale(LIB, deps):
-        objs = []
+        from concurrent.futures import ThreadPoolExecutor
+        objs, cmds = [], []
         for s in srcs:
             o = os.path.join(BUILD, os.path.basename(s) + ".o")
             cmd = [NVCC, *ARCH, "-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC",
@@ -56,8 +57,11 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
                    "-I", BUILD, "-c", s, "-o", o]
             if verbose_ptxas:
                 cmd.insert(1, "-Xptxas=-v")
-            _run(cmd)
+            cmds.append(cmd)
             objs.append(o)
+        # the translation units compile independently (decode.cu takes longest)
+        with ThreadPoolExecutor(max_workers=min(len(cmds), os.cpu_count() or 1)) as ex:
+            list(ex.map(_run, cmds))
         _run([NVCC, *ARCH, "-shared", "-o", LIB, *objs, "-cudart", "static"])
     return LIB
 
