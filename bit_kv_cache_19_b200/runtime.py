@@ -7,6 +7,8 @@ exchange step of a decode whose context is split over ranks.
 """
 from __future__ import annotations
 
+import collections
+
 import numpy as np
 import torch
 
@@ -149,6 +151,54 @@ def sharded_decode(partial, combine, group=None):
     return combine(recs)
 
 
+class PageAllocator:
+    """Host-side page bookkeeping of a paged cache: the block table
+    [batch][max_pages] (int32 page ids, -1 = none) and a free list. Pages are
+    handed out in order (or in a caller's order) as sequences grow and come
+    back when a sequence is released."""
+
+    def __init__(self, n_pages: int, page_tiles: int, batch: int, max_pages: int):
+        self.n_pages = n_pages
+        self.page_tiles = page_tiles
+        self.table = np.full((batch, max_pages), -1, dtype=np.int32)
+        self.free = collections.deque(range(n_pages))
+        self.used = set()
+        self.n_held = [0] * batch
+
+    def reserve(self, seq: int, n_tokens: int, order=None):
+        """Pages for the first n_tokens tokens of sequence seq (from the free
+        list, or taken from `order`, a list consumed from the front; pages in
+        use are skipped)."""
+        need = -(-n_tokens // (32 * self.page_tiles))
+        if need > self.table.shape[1]:
+            raise ValueError(f"{n_tokens} tokens exceed the block-table row")
+        while self.n_held[seq] < need:
+            g = None
+            while g is None:
+                if order is not None:
+                    if not order:
+                        break
+                    c = int(order.pop(0))
+                else:
+                    if not self.free:
+                        break
+                    c = self.free.popleft()
+                if c not in self.used:
+                    g = c
+            if g is None:
+                raise MemoryError("page pool exhausted")
+            self.used.add(g)
+            self.table[seq, self.n_held[seq]] = g
+            self.n_held[seq] += 1
+
+    def release(self, seq: int):
+        held = self.table[seq, :self.n_held[seq]].tolist()
+        self.used.difference_update(held)
+        self.free.extend(held)
+        self.table[seq, :] = -1
+        self.n_held[seq] = 0
+
+
 class PagedLayer:
     """One layer's packed caches for a batch of sequences in pages of a shared
     pool: the pool, the block table (device) and a host-side page allocator.
@@ -168,11 +218,9 @@ class PagedLayer:
         if nb == 0:
             raise ValueError(f"page_tiles {page_tiles}: a power of two, 1..2^20")
         self.pool = torch.zeros(n_pages * nb, dtype=torch.uint8, device=self.device)
-        self.table_host = np.full((batch, max_pages), -1, dtype=np.int32)
-        self.table = torch.from_numpy(self.table_host.copy()).to(self.device)
+        self.alloc = PageAllocator(n_pages, page_tiles, batch, max_pages)
+        self.table = torch.from_numpy(self.alloc.table.copy()).to(self.device)
         self.pages = kvq.make_pages(self.pool, self.table, n_pages, page_tiles)
-        self.free = list(range(n_pages))
-        self.n_held = [0] * batch
         self.plans = torch.zeros(cfg.n_kv_heads * kvq.PLAN_BYTES, dtype=torch.uint8,
                                  device=self.device)
         self.plan_ptrs = kvq.ptr_array([self.plans] * batch, self.device)
@@ -181,33 +229,23 @@ class PagedLayer:
         self.plans_host = None
 
     @property
+    def table_host(self):
+        return self.alloc.table
+
+    @property
     def cap(self) -> int:
-        return self.table_host.shape[1] * self.page_tiles * 32
+        return self.alloc.table.shape[1] * self.page_tiles * 32
 
     # ---------------------------------------------------------- pages
     def reserve(self, seq: int, n_tokens: int, order=None):
-        """Give sequence `seq` pages for its first n_tokens tokens (from the
-        free list, or in the given page order) and upload the block table."""
-        need = -(-n_tokens // (32 * self.page_tiles))
-        if need > self.table_host.shape[1]:
-            raise ValueError(f"{n_tokens} tokens exceed the block-table row")
-        while self.n_held[seq] < need:
-            if not self.free:
-                raise MemoryError("page pool exhausted")
-            g = self.free.pop(0) if order is None else order.pop(0)
-            if order is not None:
-                self.free.remove(g)
-            self.table_host[seq, self.n_held[seq]] = g
-            self.n_held[seq] += 1
-        self.table.copy_(torch.from_numpy(self.table_host))
+        """Pages for the first n_tokens tokens of sequence seq; uploads the table."""
+        self.alloc.reserve(seq, n_tokens, order)
+        self.table.copy_(torch.from_numpy(self.alloc.table))
 
     def release(self, seq: int):
         """Return a sequence's pages to the free list and empty it."""
-        held = self.table_host[seq, :self.n_held[seq]].tolist()
-        self.free.extend(held)
-        self.table_host[seq, :] = -1
-        self.n_held[seq] = 0
-        self.table.copy_(torch.from_numpy(self.table_host))
+        self.alloc.release(seq)
+        self.table.copy_(torch.from_numpy(self.alloc.table))
         self.lens[seq] = 0
 
     # ---------------------------------------------------------- calls
