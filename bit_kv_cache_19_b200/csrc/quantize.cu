@@ -6,7 +6,9 @@
 // top of TurboQuant-MSE and values with uniform TQ-MSE, into the packed
 // cache of the serving path. Readings adopted (energy on a 2^-32 integer
 // grid, fp16 norm, Gaussian Lloyd-Max codes, randomised Hadamard on values,
-// tile record layout) are stated in kvq.h.
+// tile record layout, the optional rotation of keys inside each width group)
+// are stated in kvq.h. Tile records are found through the cache map, so the
+// same kernel fills contiguous and paged caches.
 #include <algorithm>
 
 #include "quant_dev.cuh"
