@@ -84,6 +84,7 @@ def _check(cfg, E, kb, vb, qb, cuts, layer_idx, v_seed):
     (3, 3, 8, [0, 1000, 1000, 2017, 3000]),   # an empty range, ragged ends
     (2, 2, 4, [0, 1, 33, 3000]),              # one-token and partial-tile ranges
     (4, 2, 7, [0, 1500, 3000]),
+    (3, 3, 16, [0, 700, 1800, 1800, 3000]),  # two query groups per CTA (G = 16)
 ])
 def test_shards_combine_to_whole_context(bits_k, bits_v, G, cuts):
     rng = np.random.default_rng(bits_k * 10 + G)
