@@ -297,7 +297,7 @@ KVQ_API int kvq_quantize_append(const kvq_cfg* cfg, const void* const* plans_dev
                         uint32_t* status_dev, kvq_stream_t stream);
 
 /*
- * Fused RoPE + quantize-append (SURVEY NEXT-1): k_dev holds pre-RoPE keys;
+ * Fused RoPE + quantize-append: k_dev holds pre-RoPE keys;
  * the key of the token at cache position t is first rotated by RoPE at
  * position t with theta_j = rope_base^(-2j/128) (block j = coordinates j,
  * j + 64): angles in fp64, cos and sin rounded once to fp32, the 2-D
