@@ -245,3 +245,22 @@ def test_argument_errors_without_gpu():
     # zero new tokens is a no-op
     assert L.kvq_quantize_append(ctypes.byref(cfg), p, None, None, 0, 1, 0, p, p, 10, p,
                                  None) == kvq.OK
+
+
+@pytest.mark.parametrize("kind", ["zero", "one_block", "tiny"])
+def test_plan_build_degenerate_energies(kind):
+    """Degenerate energy vectors (all zero, one nonzero block, denormal-small)
+    give the oracle's plans: widths by the tie rule, zero scales where the
+    energy is zero."""
+    E = np.zeros((1, 64))
+    if kind == "one_block":
+        E[0, 17] = 3.0
+    elif kind == "tiny":
+        E[0] = np.ldexp(1.0, -1060) * (1 + np.arange(64))
+    for bits in (1, 3, 8):
+        cfg = kvq.make_cfg(1, bits, 2, v_seed=4)
+        got = kvq.plan_build(cfg, 0, E)[0]
+        ref = alloc.make_plan(E[0], bits, 2, 4, 0, 0)
+        assert np.array_equal(got["width"].astype(int), ref.widths)
+        assert np.array_equal(got["g"], ref.g) and np.array_equal(got["a_hat"], ref.a_hat)
+        assert int(got["width"].sum()) == 64 * bits
