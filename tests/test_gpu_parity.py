@@ -432,3 +432,32 @@ def test_split_maxima_outside_bucket_range_take_the_record_merge():
         assert np.isfinite(out).all(), scale
         assert op.rel_err(out, ref) <= TOL, scale
     assert L.flags() == 0
+
+
+@pytest.mark.parametrize("rot", [0, kvq.ALLOC_ROTATE_KEYS])
+def test_degenerate_plans_zero_and_single_block_energy(rot):
+    """Plans from degenerate energies (all zero: every key scale 0, so every
+    dequantized key is 0 and attention is uniform; one nonzero block) with
+    and without key rotation: records bit-exact, outputs against the oracle."""
+    rng = np.random.default_rng(12)
+    n_kv, G, T = 2, 8, 200
+    E = np.zeros((n_kv, 64))
+    E[1, 9] = 2.5
+    cfg = kvq.make_cfg(n_kv, 3, 2, v_seed=3, alloc_mode=rot)
+    L = PackedLayer(cfg, 1, 256)
+    L.set_plans(kvq.plan_build(cfg, 1, E))
+    kb = synth.to_bf16_bits(rng.standard_normal((T, n_kv, 128)))
+    vb = synth.to_bf16_bits(rng.standard_normal((T, n_kv, 128)))
+    L.append(dev_bf16(kb)[None], dev_bf16(vb)[None])
+    qb = synth.to_bf16_bits(rng.standard_normal((1, n_kv * G, 128)))
+    out = L.decode(dev_bf16(qb), max_len=256).cpu().numpy()[0]
+    torch.cuda.synchronize()
+    assert L.flags() == 0
+    kh, vh = op.bf16_heads(kb, vb)
+    _, heads = op.layer(kh, vh, 3, 2, 3, 1, E=E, rotate_keys=bool(rot))
+    for h in range(n_kv):
+        check_records(L.head_records(0, h, (T + 31) // 32), heads[h]["rec"], T, 3, 2)
+    ref = op.decode(synth.bf16_bits_to_f64(qb[0]), heads)
+    assert op.rel_err(out, ref) <= TOL
+    # head 0 has all-zero scales: its keys dequantize to 0, attention is the mean of V
+    assert np.allclose(ref[:G], heads[0]["vhat"].mean(axis=0)[None], rtol=0, atol=1e-12)
