@@ -446,6 +446,13 @@ KVQ_API int kvq_append_decode(const kvq_cfg* cfg, const void* const* plans_dev, 
  *              cap_tokens gives for contiguous caches; at most 2^31 - 1).
  * The block table is read by the kernels as the lengths are: with
  * KVQ_STEP_EARLY it must not be written by the previous kernel on the stream.
+ * The library only reads the pool through the table and never allocates or
+ * frees pages; the caller owns the pool, the table and the page bookkeeping.
+ * Errors (before any launch): KVQ_ERR_ARG for a null page description, pool
+ * or block table, a pool off a 16-byte boundary, page_tiles not a power of
+ * two in 1..2^20, max_pages or n_pages < 1, or a row capacity above
+ * 2^31 - 1 tokens; the other arguments are checked as for the contiguous
+ * calls.
  */
 typedef struct kvq_pages {
   void* pool;
