@@ -97,36 +97,23 @@ void greedy_widths(const double* E, int bits_k, uint8_t* w) {
   for (int j = 0; j < kBlocks; ++j) w[j] = (uint8_t)b[j];
 }
 
-// W (optional): query block energies of the query-weighted variant; the
-// widths then come from the products E_j W_j, the key scales still from E.
-void build_plan(const kvq_cfg* cfg, int layer, int kv_head, const double* E, Plan* pl,
-                const double* W = nullptr) {
-  std::memset(pl, 0, sizeof(Plan));
-  pl->magic = KVQ_PLAN_MAGIC;
-  pl->bits_k = cfg->bits_k;
-  pl->bits_v = cfg->bits_v;
-  pl->layer = layer;
-  pl->kv_head = kv_head;
-  pl->words_k = 128 * cfg->bits_k;
-  pl->words_v = 128 * cfg->bits_v;
-  if ((cfg->alloc_mode & ~KVQ_ALLOC_ROTATE_KEYS) == KVQ_ALLOC_UNIFORM) {
-    for (int j = 0; j < kBlocks; ++j) pl->width[j] = (uint8_t)cfg->bits_k;
-  } else if (W) {
-    double EW[kBlocks];
-    for (int j = 0; j < kBlocks; ++j) EW[j] = E[j] * W[j];
-    greedy_widths(EW, cfg->bits_k, pl->width);
-  } else {
-    greedy_widths(E, cfg->bits_k, pl->width);
-  }
-  double tot = 0.0;
-  for (int j = 0; j < kBlocks; ++j) tot += E[j];
-  pl->energy_sum = tot;
-  for (int j = 0; j < kBlocks; ++j) {
-    const double a = tot > 0.0 ? std::sqrt(E[j] / (2.0 * tot)) : 0.0;
-    pl->a_hat[j] = (float)a;
-    pl->g[j] = a > 0.0 ? (float)(1.0 / a) : 0.f;
-  }
-  // plan order: nonzero widths, width descending, block index ascending
+// Everything of a plan that follows from its widths: plan order (nonzero
+// widths, width descending, block index ascending), K segment offsets, the
+// decode schedule (half steps, classes). Zeroes those fields first.
+void fill_schedule(Plan* pl) {
+  pl->n_ranks = 0;
+  std::memset(pl->order, 0, sizeof pl->order);
+  std::memset(pl->seg_off, 0, sizeof pl->seg_off);
+  pl->n_half = 0;
+  std::memset(pl->hs_width, 0, sizeof pl->hs_width);
+  std::memset(pl->hs_rank0, 0, sizeof pl->hs_rank0);
+  std::memset(pl->hs_count, 0, sizeof pl->hs_count);
+  pl->n_class = 0;
+  std::memset(pl->cls_w, 0, sizeof pl->cls_w);
+  std::memset(pl->cls_hs0, 0, sizeof pl->cls_hs0);
+  std::memset(pl->cls_nhs, 0, sizeof pl->cls_nhs);
+  std::memset(pl->cls_last, 0, sizeof pl->cls_last);
+  std::memset(pl->cls_seg0, 0, sizeof pl->cls_seg0);
   int ranks = 0;
   for (int w = 8; w >= 1; --w)
     for (int j = 0; j < kBlocks; ++j)
@@ -165,6 +152,38 @@ void build_plan(const kvq_cfg* cfg, int layer, int kv_head, const double* E, Pla
     hs = e;
   }
   pl->n_class = (uint8_t)nc;
+}
+
+// W (optional): query block energies of the query-weighted variant; the
+// widths then come from the products E_j W_j, the key scales still from E.
+void build_plan(const kvq_cfg* cfg, int layer, int kv_head, const double* E, Plan* pl,
+                const double* W = nullptr) {
+  std::memset(pl, 0, sizeof(Plan));
+  pl->magic = KVQ_PLAN_MAGIC;
+  pl->bits_k = cfg->bits_k;
+  pl->bits_v = cfg->bits_v;
+  pl->layer = layer;
+  pl->kv_head = kv_head;
+  pl->words_k = 128 * cfg->bits_k;
+  pl->words_v = 128 * cfg->bits_v;
+  if ((cfg->alloc_mode & ~KVQ_ALLOC_ROTATE_KEYS) == KVQ_ALLOC_UNIFORM) {
+    for (int j = 0; j < kBlocks; ++j) pl->width[j] = (uint8_t)cfg->bits_k;
+  } else if (W) {
+    double EW[kBlocks];
+    for (int j = 0; j < kBlocks; ++j) EW[j] = E[j] * W[j];
+    greedy_widths(EW, cfg->bits_k, pl->width);
+  } else {
+    greedy_widths(E, cfg->bits_k, pl->width);
+  }
+  double tot = 0.0;
+  for (int j = 0; j < kBlocks; ++j) tot += E[j];
+  pl->energy_sum = tot;
+  for (int j = 0; j < kBlocks; ++j) {
+    const double a = tot > 0.0 ? std::sqrt(E[j] / (2.0 * tot)) : 0.0;
+    pl->a_hat[j] = (float)a;
+    pl->g[j] = a > 0.0 ? (float)(1.0 / a) : 0.f;
+  }
+  fill_schedule(pl);
   const uint64_t key = splitmix64(cfg->v_seed, ((uint64_t)(uint32_t)layer << 32) + (uint32_t)kv_head);
   for (int i = 0; i < kHeadDim; ++i)
     if (splitmix64(key, (uint64_t)i) >> 63) pl->v_sign[i >> 5] |= 1u << (i & 31);
@@ -247,6 +266,46 @@ int kvq_plan_build(const kvq_cfg* cfg, int layer, const double* E_host, int n_he
       return fail(KVQ_ERR_ARG, "energy %d is negative or not finite", i);
   Plan* out = reinterpret_cast<Plan*>(plans_host);
   for (int h = 0; h < n_heads; ++h) build_plan(cfg, layer, h, E_host + (size_t)h * kBlocks, out + h);
+  return KVQ_OK;
+}
+
+int kvq_plan_check(const kvq_cfg* cfg, const void* plan_host) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (!plan_host) return fail(KVQ_ERR_ARG, "null plan");
+  const Plan& p = *reinterpret_cast<const Plan*>(plan_host);
+  if (p.magic != KVQ_PLAN_MAGIC) return fail(KVQ_ERR_ARG, "plan magic 0x%08x", p.magic);
+  if (p.bits_k != cfg->bits_k || p.bits_v != cfg->bits_v)
+    return fail(KVQ_ERR_ARG, "plan K%dV%d vs cfg K%dV%d", p.bits_k, p.bits_v, cfg->bits_k,
+                cfg->bits_v);
+  if (p.words_k != 128 * p.bits_k || p.words_v != 128 * p.bits_v)
+    return fail(KVQ_ERR_ARG, "plan word counts");
+  int sum = 0;
+  for (int j = 0; j < kBlocks; ++j) {
+    if (p.width[j] > 8) return fail(KVQ_ERR_ARG, "width of block %d is %d", j, p.width[j]);
+    sum += p.width[j];
+    if (!(p.g[j] >= 0.f) || !std::isfinite(p.g[j]) || !(p.a_hat[j] >= 0.f) ||
+        !std::isfinite(p.a_hat[j]))
+      return fail(KVQ_ERR_ARG, "scales of block %d", j);
+  }
+  if (sum != kBlocks * p.bits_k)
+    return fail(KVQ_ERR_ARG, "widths sum to %d bits per block pair, not %d", sum,
+                kBlocks * p.bits_k);
+  if (p.k_rot > 1) return fail(KVQ_ERR_ARG, "k_rot %d", p.k_rot);
+  Plan q = p;
+  fill_schedule(&q);
+  const bool same =
+      q.n_ranks == p.n_ranks && !std::memcmp(q.order, p.order, sizeof q.order) &&
+      !std::memcmp(q.seg_off, p.seg_off, sizeof q.seg_off) && q.n_half == p.n_half &&
+      !std::memcmp(q.hs_width, p.hs_width, sizeof q.hs_width) &&
+      !std::memcmp(q.hs_rank0, p.hs_rank0, sizeof q.hs_rank0) &&
+      !std::memcmp(q.hs_count, p.hs_count, sizeof q.hs_count) && q.n_class == p.n_class &&
+      !std::memcmp(q.cls_w, p.cls_w, sizeof q.cls_w) &&
+      !std::memcmp(q.cls_hs0, p.cls_hs0, sizeof q.cls_hs0) &&
+      !std::memcmp(q.cls_nhs, p.cls_nhs, sizeof q.cls_nhs) &&
+      !std::memcmp(q.cls_last, p.cls_last, sizeof q.cls_last) &&
+      !std::memcmp(q.cls_seg0, p.cls_seg0, sizeof q.cls_seg0);
+  if (!same) return fail(KVQ_ERR_ARG, "plan order or decode schedule inconsistent with the widths");
   return KVQ_OK;
 }
 

@@ -99,6 +99,7 @@ _SIGS = {
                                        _i32, _vp, _vp, _sz, _vp, _vp]),
     "kvq_combine_partials": (_i32, [ctypes.POINTER(Cfg), _vp, _i32, _vp, _i32, _i32, _vp, _vp]),
     "kvq_page_bytes": (_sz, [ctypes.POINTER(Cfg), _i32]),
+    "kvq_plan_check": (_i32, [ctypes.POINTER(Cfg), _vp]),
     "kvq_energy_workspace_bytes": (_sz, [_i32]),
     "kvq_block_energy": (_i32, [_vp, _i32, _i64, _i32, _vp, _sz, _vp, _vp, _vp]),
     "kvq_plan_build_weighted": (_i32, [ctypes.POINTER(Cfg), _i32, _vp, _vp, _i32, _vp]),
@@ -217,6 +218,14 @@ def block_energy(x, status=None, ws=None) -> np.ndarray:
     _check(lib().kvq_block_energy(_ptr(x), _dtype_code(x), x.shape[0], n_heads, _ptr(ws),
                                   ws.numel(), E.ctypes.data, _ptr(status), _stream()))
     return E
+
+
+def plan_check(cfg, plans):
+    """Raise KVQError unless every host plan record (PLAN_DTYPE array) is
+    consistent (kvq_plan_check)."""
+    plans = np.ascontiguousarray(plans)
+    for i in range(plans.shape[0]):
+        _check(lib().kvq_plan_check(ctypes.byref(cfg), plans[i:i + 1].ctypes.data))
 
 
 def parse_plans(raw) -> np.ndarray:

@@ -53,8 +53,11 @@ class PackedLayer:
         self.energy = E
         return self.plans_host
 
-    def set_plans(self, plans_host: np.ndarray):
-        """Use host plan records (e.g. from kvq.plan_build)."""
+    def set_plans(self, plans_host: np.ndarray, check: bool = True):
+        """Use host plan records (e.g. from kvq.plan_build); checked on the
+        host first (kvq_plan_check) unless check=False."""
+        if check:
+            kvq.plan_check(self.cfg, plans_host)
         raw = torch.from_numpy(np.frombuffer(plans_host.tobytes(), dtype=np.uint8).copy())
         self.plans.copy_(raw.to(self.device))
         self.plans_host = plans_host
@@ -255,7 +258,9 @@ class PagedLayer:
                                                       self.status)
         return self.plans_host
 
-    def set_plans(self, plans_host: np.ndarray):
+    def set_plans(self, plans_host: np.ndarray, check: bool = True):
+        if check:
+            kvq.plan_check(self.cfg, plans_host)
         raw = torch.from_numpy(np.frombuffer(plans_host.tobytes(), dtype=np.uint8).copy())
         self.plans.copy_(raw.to(self.device))
         self.plans_host = plans_host

@@ -241,6 +241,18 @@ KVQ_API int kvq_plan_build(const kvq_cfg* cfg, int layer, const double* E_host, 
 KVQ_API int kvq_codebook(int bits, float* centroids, float* thresholds, double* distortion);
 
 /*
+ * Host check of one plan record before it is uploaded (host memory): magic,
+ * bits against cfg, word counts, widths in 0..8 summing to 64 bits_k, finite
+ * non-negative scales, k_rot in {0, 1}, and every field that follows from
+ * the widths (plan order, segment offsets, half steps, classes) equal to what
+ * the widths give. The kernels check only the magic and the shape fields, so
+ * a plan that was not built by this library should pass here first.
+ * Returns KVQ_OK, or KVQ_ERR_ARG with the first inconsistency in
+ * kvq_last_error().
+ */
+KVQ_API int kvq_plan_check(const kvq_cfg* cfg, const void* plan_host);
+
+/*
  * Query-weighted allocation (a variant; the pages' score is key-only and
  * label-free). The logit q . k is a sum of 2-D RoPE block terms q_j . k_j, so
  * the error of key block j reaches the logit scaled by the query's block

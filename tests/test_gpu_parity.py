@@ -158,7 +158,7 @@ def test_edge_flags():
     # a plan record with a bad magic is refused on the device
     bad = kvq.plan_build(cfg, 0, E)
     bad["magic"] = 0
-    L.set_plans(bad)
+    L.set_plans(bad, check=False)  # the device check is under test
     L.status.zero_()
     L.decode(dev_bf16(qb), max_len=96)
     torch.cuda.synchronize()

@@ -264,3 +264,59 @@ def test_plan_build_degenerate_energies(kind):
         assert np.array_equal(got["width"].astype(int), ref.widths)
         assert np.array_equal(got["g"], ref.g) and np.array_equal(got["a_hat"], ref.a_hat)
         assert int(got["width"].sum()) == 64 * bits
+
+
+def test_plan_check_accepts_built_plans_and_refuses_inconsistent_ones():
+    rng = np.random.default_rng(31)
+    E = np.exp(1.5 * rng.standard_normal((2, 64)) - np.arange(64) / 8.0)
+    for mode in (kvq.ALLOC_GREEDY, kvq.ALLOC_UNIFORM, kvq.ALLOC_GREEDY | kvq.ALLOC_ROTATE_KEYS):
+        for bits in ((1, 1), (3, 3), (8, 2)):
+            cfg = kvq.make_cfg(2, *bits, v_seed=1, alloc_mode=mode)
+            kvq.plan_check(cfg, kvq.plan_build(cfg, 0, E))
+    cfg = kvq.make_cfg(2, 3, 3, v_seed=1)
+    good = kvq.plan_build(cfg, 0, E)
+
+    def refused(mutate, what):
+        p = good.copy()
+        mutate(p)
+        with pytest.raises(kvq.KVQError) as ei:
+            kvq.plan_check(cfg, p)
+        assert what in str(ei.value)
+
+    def bad_magic(p):
+        p["magic"] = 0
+
+    def wide_block(p):
+        p["width"][0, 0] = 9
+
+    refused(bad_magic, "magic")
+    refused(wide_block, "width")
+    j0, j1 = int(good["order"][0][0]), int(good["order"][0][1])
+
+    def swap_order(p):
+        p["order"][0][0], p["order"][0][1] = j1, j0
+    if good["width"][0][j0] != good["width"][0][j1]:
+        refused(swap_order, "inconsistent")
+
+    def move_bit(p):  # one bit moved between blocks: widths still sum right
+        w = p["width"][0]
+        a = int(np.argmax(w))
+        b = int(np.argmin(np.where(w < 8, w, 99)))
+        w[a] -= 1
+        w[b] += 1
+    refused(move_bit, "inconsistent")
+    def shift_segment(p):
+        p["seg_off"][0, 3] += 1
+
+    def bad_rot(p):
+        p["k_rot"] = 2
+
+    def nan_scale(p):
+        p["g"][0, 5] = np.float32(np.nan)
+
+    refused(shift_segment, "inconsistent")
+    refused(bad_rot, "k_rot")
+    refused(nan_scale, "scales")
+    other = kvq.make_cfg(2, 2, 3, v_seed=1)
+    with pytest.raises(kvq.KVQError):
+        kvq.plan_check(other, good)
