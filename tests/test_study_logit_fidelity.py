@@ -160,3 +160,28 @@ def test_rotation_and_query_weighting_combine():
             res.append(_mae(qe, k, attn.dequant_keys(kc, kn, plan)))
         print(f"  {wname:12s} " + "  ".join(f"{x:.5f}" for x in res))
         assert res[3] == min(res)
+
+
+def test_logit_error_against_key_budget():
+    """Key-logit error from K1 to K5 (qwen3b L5 h1, isotropic queries) for
+    uniform allocation, Block-GTQ, and both with the width-group rotation:
+    Block-GTQ is below uniform allocation at every budget, and the rotation
+    lowers Block-GTQ's error at every budget."""
+    wl = synth.WORKLOADS["qwen3b_128k"]
+    G, layer, h = 8, 5, 1
+    kb, _ = synth.keys_values(wl, 11, layer, h, T)
+    k = synth.bf16_bits_to_f64(kb)
+    q = synth.bf16_bits_to_f64(synth.queries(wl, 11, layer, 0, T))[h * G:(h + 1) * G]
+    E, _ = energy.block_energy(k[:, None, :])
+
+    def err(bits, uniform, rot):
+        plan = alloc.make_plan(E[0], bits, 2, 5, layer, h, uniform=uniform, rotate_keys=rot)
+        kc, kn, _ = quant.quantize_keys(k, plan)
+        return _mae(q, k, attn.dequant_keys(kc, kn, plan))
+
+    print("\nK bits: uniform | Block-GTQ | uniform + rotation | Block-GTQ + rotation")
+    for bits in range(1, 6):
+        r = [err(bits, u, rot) for u, rot in ((True, False), (False, False), (True, True),
+                                               (False, True))]
+        print(f"  K{bits}: " + "  ".join(f"{x:.5f}" for x in r))
+        assert r[1] < r[0] and r[3] < r[1]
