@@ -66,6 +66,16 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kStages = 2;
 constexpr int kMaxHalf = 24;  // half steps of <= 4 blocks (<= 64/4 + 8)
 constexpr int kBuckets = 16;  // split maxima m in [32 (k - 8), 32 (k - 7)), k = 0..15
+// Per (sequence, KV head) "pair block" of the workspace, at a fixed distance
+// from its end: 32 counter words (0: arrivals, 1: range flag, 2..17: bucket
+// masks of the query heads, 31: sequence counter of KV head 0), then the
+// exponent buckets of up to 16 query heads. Every completed call leaves the
+// words and buckets it used at zero, and a pair block never overlaps the
+// split records of any call whose batch x n_kv fits the workspace.
+constexpr int kPairCntWords = 32;
+constexpr size_t kPairBlockBytes =
+    kPairCntWords * 4 + (size_t)16 * kBuckets * kPartStride * sizeof(float);
+static_assert(kPairBlockBytes % 128 == 0, "pair blocks keep the buckets 16-byte aligned");
 constexpr int kFallbackSlots = 1024;                  // CTA slots when no device answers
 constexpr int kMaxNew = 64;                           // tokens appended by a fused call
 constexpr int kScratch = 16640;  // q' staging; append: kz [32][129] fp32 + 64 fp16 norms
@@ -88,9 +98,8 @@ struct DecodeParams {
   int early;  // read lengths and stream tiles before waiting for the previous kernel
   int rope;   // appended keys are pre-RoPE: rotate each to its position first
   double theta[64];
-  unsigned int* cnt_end;  // counters of pair k at cnt_end - (k + 1) * kCntStride
+  uint8_t* pb_end;        // pair block of pair k at pb_end - (k + 1) * kPairBlockBytes
   float* part;            // [batch][n_kv][n_splits][G][132] = m, l, -, -, o[128]
-  float* bkt;             // [batch][n_kv][G][kBuckets][132]: exponent buckets
   float* out;             // [batch][n_q][128]
   float* rec_out;         // partial decode: merged records [batch][n_q][132], no out
   uint32_t* status;
@@ -292,8 +301,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
   const int G = p.G;
   const size_t bh = (size_t)b * p.n_kv + h;
-  unsigned int* const cnt = p.cnt_end - (bh + 1) * kCntStride;
-  unsigned int* const seq_cnt = p.cnt_end - ((size_t)b * p.n_kv + 1) * kCntStride + (kCntStride - 1);
+  unsigned int* const cnt = reinterpret_cast<unsigned int*>(p.pb_end - (bh + 1) * kPairBlockBytes);
+  unsigned int* const seq_cnt =
+      reinterpret_cast<unsigned int*>(p.pb_end - ((size_t)b * p.n_kv + 1) * kPairBlockBytes) +
+      (kPairCntWords - 1);
+
 
   // ---- independent of earlier kernels: barriers, plan and lookup image
   if (tid == 0) {
@@ -714,7 +726,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   float* const crec = reinterpret_cast<float*>(scratch);  // [G][132]
   unsigned int* const ovf = cnt + 1;
   unsigned int* const bmask = cnt + 2;  // [G]: buckets in use
-  float* const bkt = p.bkt + bh * (size_t)G * kBuckets * kPartStride;
+  float* const bkt = reinterpret_cast<float*>(cnt + kPairCntWords);  // [G][kBuckets][132]
   for (int item = tid; item < G * 32; item += kThreads) {
     const int hd = item >> 5, x4 = (item & 31) * 4;
     float m, l;
@@ -927,14 +939,17 @@ static int ctas_per_sm_bv(int dev, int bits_k, int bv, cudaError_t* err) {
 
 struct SplitPlan {
   int n_splits, tiles_per_split;
+  int64_t slots;  // bound on the CTA slots of any decode launch on the device
 };
+
+constexpr int kMaxCtasPerSm = 2;  // the launch bounds' residency, also the grid's cap
 
 // Splits per (sequence, KV head) so that the grid is about one wave of the
 // current device, with at least one tile per warp. Without a device (size
 // queries on a host without GPU) an upper bound of the CTA slots is used.
 static SplitPlan decode_split_plan(int batch, int n_kv, int G, int bits_k, int bits_v,
                                    int64_t max_len, cudaError_t* err, bool allow_fallback) {
-  SplitPlan sp{1, 1};
+  SplitPlan sp{1, 1, kFallbackSlots};
   int64_t slots = kFallbackSlots;
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -944,7 +959,8 @@ static SplitPlan decode_split_plan(int batch, int n_kv, int G, int bits_k, int b
     per_sm = G <= 8 ? ctas_per_sm_bv<1>(dev, bits_k, bits_v, &e)
                     : ctas_per_sm_bv<2>(dev, bits_k, bits_v, &e);
   if (e == cudaSuccess) {
-    slots = (int64_t)sms * per_sm;
+    slots = (int64_t)sms * std::min(per_sm, kMaxCtasPerSm);
+    sp.slots = (int64_t)sms * kMaxCtasPerSm;  // the same for every bit budget
   } else if (!allow_fallback) {
     *err = e;
     return sp;
@@ -964,17 +980,18 @@ static SplitPlan decode_split_plan(int batch, int n_kv, int G, int bits_k, int b
 
 static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-// Workspace: split records | exponent buckets | ... | counters (at the end: pair
-// k at a fixed distance from the end, so calls sharing one workspace, for one
-// n_kv_heads, never overwrite each other's counters).
-static size_t decode_workspace_layout(int batch, int n_kv, int G, const SplitPlan& sp,
-                                      size_t* bkt_off) {
-  const size_t pairs = (size_t)batch * n_kv;
-  const size_t part = align256(pairs * sp.n_splits * G * kPartStride * sizeof(float));
-  const size_t bkt = align256(pairs * G * kBuckets * kPartStride * sizeof(float));
-  const size_t counters = align256(pairs * kCntStride * sizeof(unsigned int));
-  if (bkt_off) *bkt_off = part;
-  return part + bkt + counters;
+// Workspace: split records from the start | ... | pair blocks at fixed
+// distances from the end (pair k at end - (k + 1) * kPairBlockBytes, the end
+// rounded down to 128 bytes). The split records of a call are bounded by one
+// record per CTA slot of the device (or per pair, if there are more pairs)
+// and 16 query heads, independently of max_len and G, so the records of any
+// call with batch x n_kv <= that of the sizing call end before the pair
+// blocks of any such call: one zero-filled workspace serves every sequence of
+// calls of those shapes, whatever their max_len or query-head count.
+static size_t decode_workspace_layout(size_t pairs, int64_t slots) {
+  const size_t recs = (size_t)std::max<int64_t>(slots, (int64_t)pairs);
+  const size_t part = align256(recs * 16 * kPartStride * sizeof(float));
+  return part + pairs * kPairBlockBytes + 128;
 }
 
 // Workspace bytes of a decode call on the current device (an upper bound if
@@ -984,7 +1001,7 @@ size_t decode_workspace_bytes_for(int batch, int n_q, int n_kv, int bits_k, int 
   cudaError_t err = cudaSuccess;
   const int G = n_q / n_kv;
   const SplitPlan sp = decode_split_plan(batch, n_kv, G, bits_k, bits_v, max_len, &err, true);
-  return decode_workspace_layout(batch, n_kv, G, sp, nullptr);
+  return decode_workspace_layout((size_t)batch * n_kv, sp.slots);
 }
 
 template <int BV, int NT>
@@ -1018,7 +1035,7 @@ static cudaError_t launch_decode_nt(const DecodeParams& p, int bits_v, int batch
 }
 
 // ws: >= decode_workspace_bytes_for(...) bytes, zero-filled before its first
-// use; every completed call leaves its counters (at the end of ws) zero.
+// use; every completed call leaves its pair blocks (at the end of ws) zero.
 // n_new > 0 fuses the append of k_new / v_new ([batch][n_new][n_kv][128]).
 cudaError_t launch_decode(const Plan* const* plans, const CacheMap& cm, int32_t* len,
                           int batch, int64_t max_len, const void* q, int q_dtype, int n_q, int n_kv,
@@ -1030,8 +1047,7 @@ cudaError_t launch_decode(const Plan* const* plans, const CacheMap& cm, int32_t*
   const int G = n_q / n_kv;
   const SplitPlan sp = decode_split_plan(batch, n_kv, G, bits_k, bits_v, max_len, &err, false);
   if (err != cudaSuccess) return err;
-  size_t bkt_off = 0;
-  if (decode_workspace_layout(batch, n_kv, G, sp, &bkt_off) > ws_bytes)
+  if (decode_workspace_layout((size_t)batch * n_kv, sp.slots) > ws_bytes)
     return cudaErrorInvalidValue;
   if (n_new < 0 || n_new > kMaxNew) return cudaErrorInvalidValue;
   DecodeParams p;
@@ -1056,9 +1072,8 @@ cudaError_t launch_decode(const Plan* const* plans, const CacheMap& cm, int32_t*
   p.rope = theta ? 1 : 0;
   for (int j = 0; j < 64; ++j) p.theta[j] = theta ? theta[j] : 0.0;
   p.part = reinterpret_cast<float*>(ws);
-  p.bkt = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + bkt_off);
-  p.cnt_end = reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(ws) +
-                                              (ws_bytes & ~size_t(3)));
+  p.pb_end = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(ws) + ws_bytes) & ~static_cast<uintptr_t>(127));
   p.out = out;
   p.rec_out = rec_out;
   p.status = status;

@@ -353,11 +353,12 @@ static int dense_ctas_per_sm(int dev, cudaError_t* err) {
 
 struct DenseSplit {
   int n_splits, tiles_per_split, n_groups;
+  int64_t slots;  // CTA slots the split count was sized for
 };
 
 static DenseSplit dense_split_plan(int batch, int n_kv, int G, int64_t max_len, bool allow_fallback,
                                    cudaError_t* err) {
-  DenseSplit sp{1, 1, 1};
+  DenseSplit sp{1, 1, 1, 1024};
   int64_t slots = 1024;
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -374,6 +375,7 @@ static DenseSplit dense_split_plan(int batch, int n_kv, int G, int64_t max_len, 
     (void)cudaGetLastError();
   }
   *err = cudaSuccess;
+  sp.slots = slots;
   const int64_t tiles = std::max<int64_t>(1, (max_len + kTile - 1) / kTile);
   int64_t s = std::max<int64_t>(1, slots / ((int64_t)batch * n_kv));
   s = std::min<int64_t>(s, std::max<int64_t>(1, (tiles + kDWarps - 1) / kDWarps));
@@ -386,21 +388,28 @@ static DenseSplit dense_split_plan(int batch, int n_kv, int G, int64_t max_len, 
 
 static size_t dense_align256(size_t x) { return (x + 255) / 256 * 256; }
 
-static size_t dense_workspace_layout(int batch, int n_kv, int G, const DenseSplit& sp,
-                                     size_t* gpart_off) {
-  const size_t pairs = (size_t)batch * n_kv;
-  const size_t part = dense_align256(pairs * sp.n_splits * G * kPartStride * sizeof(float));
-  const size_t gpart = dense_align256(pairs * sp.n_groups * G * kPartStride * sizeof(float));
+// Workspace: split records | group records | ... | counters of pair k at a
+// fixed distance from the end (k + 1) * kCntStride words. The record regions
+// are bounded by one record per CTA slot (or per pair, if there are more
+// pairs) and 16 query heads, independently of max_len and G, so the records
+// of any call with batch x n_kv <= that of the sizing call end before the
+// counters of any such call (the counters are the only words that must be
+// zero when a call starts; every completed call leaves them at zero).
+static size_t dense_workspace_layout(size_t pairs, int64_t slots, size_t* gpart_off) {
+  const size_t recs = (size_t)std::max<int64_t>(slots, (int64_t)pairs);
+  const size_t rec_bytes = 16 * kPartStride * sizeof(float);
+  const size_t part = dense_align256(recs * rec_bytes);
+  const size_t gpart = dense_align256((recs / kGroup + pairs + 1) * rec_bytes);
   const size_t counters = dense_align256(pairs * kCntStride * sizeof(unsigned int));
   if (gpart_off) *gpart_off = part;
-  return part + gpart + counters;
+  return part + gpart + counters + 16;
 }
 
 size_t dense_workspace_bytes_for(int batch, int n_kv, int n_q, int64_t max_len) {
   cudaError_t err = cudaSuccess;
   const int G = n_q / n_kv;
   const DenseSplit sp = dense_split_plan(batch, n_kv, G, max_len, true, &err);
-  return dense_workspace_layout(batch, n_kv, G, sp, nullptr);
+  return dense_workspace_layout((size_t)batch * n_kv, sp.slots, nullptr);
 }
 
 template <int NT>
@@ -427,7 +436,7 @@ cudaError_t launch_dense_decode(const void* k, const void* v, const int32_t* len
   const DenseSplit sp = dense_split_plan(batch, n_kv, G, max_len, false, &err);
   if (err != cudaSuccess) return err;
   size_t gpart_off = 0;
-  if (dense_workspace_layout(batch, n_kv, G, sp, &gpart_off) > ws_bytes)
+  if (dense_workspace_layout((size_t)batch * n_kv, sp.slots, &gpart_off) > ws_bytes)
     return cudaErrorInvalidValue;
   DenseParams p;
   p.k = reinterpret_cast<const __nv_bfloat16*>(k);
@@ -444,8 +453,8 @@ cudaError_t launch_dense_decode(const void* k, const void* v, const int32_t* len
   p.n_groups = sp.n_groups;
   p.part = reinterpret_cast<float*>(ws);
   p.gpart = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + gpart_off);
-  p.cnt_end = reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(ws) +
-                                              (ws_bytes & ~size_t(3)));
+  p.cnt_end = reinterpret_cast<unsigned int*>(
+      (reinterpret_cast<uintptr_t>(ws) + ws_bytes) & ~static_cast<uintptr_t>(15));
   p.out = out;
   p.status = status;
   return G <= 8 ? launch_dense_t<1>(p, batch, st) : launch_dense_t<2>(p, batch, st);

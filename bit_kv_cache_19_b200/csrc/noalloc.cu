@@ -29,7 +29,7 @@ int set_last_error(int code, const char* msg);
 
 namespace {
 
-constexpr size_t kScratchBytes = size_t(4) << 20;  // 4 MiB per device
+constexpr size_t kScratchBytes = size_t(16) << 20;  // 16 MiB per device
 constexpr int kMaxDevices = 64;
 
 // The scratch itself. In host code this name is only a stand-in for the
@@ -76,7 +76,7 @@ extern "C" KVQ_API int kvq_decode_attn_noalloc(const kvq_cfg* cfg, const void* c
   if (need > kScratchBytes)
     return kvq::set_last_error(KVQ_ERR_WORKSPACE,
                                "kvq_decode_attn_noalloc: this call needs more split-partial "
-                               "scratch than the fixed 4 MiB (use kvq_decode_attn with a "
+                               "scratch than the fixed 16 MiB (use kvq_decode_attn with a "
                                "workspace, or fewer sequences / query heads / a smaller max_len)");
   if (!plans_dev || !cache_dev || !len_dev || !q_dev || !out_dev || !status_dev)
     return kvq::set_last_error(KVQ_ERR_ARG, "kvq_decode_attn_noalloc: null device pointer");
@@ -89,10 +89,12 @@ extern "C" KVQ_API int kvq_decode_attn_noalloc(const kvq_cfg* cfg, const void* c
   cudaError_t e = scratch_address(&scratch);
   if (e != cudaSuccess)
     return kvq::set_last_error(KVQ_ERR_CUDA, cudaGetErrorString(e));
-  // The split records are written before they are read within each call. The
-  // arrival counters at the end of the scratch must be zero when a call
-  // starts: the array is zero when the library is loaded and every completed
-  // call resets the counters it used.
+  // The scratch is laid out like a workspace: split records (written before
+  // they are read) from its start, and the per-(sequence, KV head) counter and
+  // bucket blocks, which must be zero when a call starts, at fixed distances
+  // from its end. The array is zero when the library is loaded, every
+  // completed call clears the blocks it used, and no call's records reach the
+  // blocks of another call that fits (kvq.h, kvq_decode_attn).
   e = kvq::launch_decode(reinterpret_cast<const kvq::Plan* const*>(plans_dev),
                          kvq::contiguous_map(cache_dev), const_cast<int32_t*>(len_dev), batch, max_len, q_dev, q_dtype, n_q_heads,
                          cfg->n_kv_heads, cfg->bits_k, cfg->bits_v, out_dev, scratch,

@@ -17,7 +17,7 @@ constexpr int kRecO = 4;          // o at float 4 (16-byte aligned)
 constexpr int kGroup = 16;        // splits merged per first-level group
 constexpr int kMergeChunk = 16;   // records whose loads a merge issues together
 constexpr int kMaxSplits = 1024;
-constexpr int kCntStride = 2 + kMaxSplits / kGroup;  // per (sequence, KV head); last = sequence
+constexpr int kCntStride = 2 + kMaxSplits / kGroup;  // merge-tree counters per (sequence, KV head)
 
 __device__ __forceinline__ float ex2(float x) {
   float y;

@@ -375,7 +375,7 @@ def append_decode(cfg, plan_ptrs, k, v, cache_ptrs, lens, cap_tokens, max_len, q
 
 def decode_attn_noalloc(cfg, plan_ptrs, cache_ptrs, lens, max_len, q, out, status):
     """kvq_decode_attn without a caller workspace: the split partials go to
-    the library's fixed 4 MiB device scratch (for callers that cannot
+    the library's fixed 16 MiB device scratch (for callers that cannot
     allocate device memory where they decode). Calls must not overlap on the
     GPU; the first call on a device must precede any stream capture."""
     batch, n_q = q.shape[0], q.shape[1]

@@ -183,11 +183,14 @@ KVQ_API size_t kvq_cache_bytes(const kvq_cfg* cfg, int64_t cap_tokens);
 KVQ_API size_t kvq_alloc_workspace_bytes(const kvq_cfg* cfg);
 
 /*
- * Workspace bytes kvq_decode_attn needs for `batch` sequences of at most
- * max_len tokens on the current device: split-K records (m, l, o[128]) per
- * (sequence, query head, split), 16 exponent buckets of the same shape per
- * (sequence, query head), and arrival counters at the end. Without a usable
- * device it returns an upper bound.
+ * Workspace bytes kvq_decode_attn needs for `batch` sequences on the current
+ * device: a region of split-K records (m, l, o[128]) bounded by one record
+ * set per CTA slot of the device (or per sequence x KV head, if there are
+ * more) for up to 16 query heads, then, at fixed distances from the end of
+ * the workspace, one block per (sequence, KV head) of arrival counters and
+ * 16 exponent buckets per query head (135,296 bytes). The size depends on
+ * batch x n_kv_heads only, not on max_len or n_q_heads (kept as arguments).
+ * Without a usable device it returns an upper bound.
  * Returns 0 for invalid arguments.
  */
 KVQ_API size_t kvq_decode_workspace_bytes(const kvq_cfg* cfg, int batch, int n_q_heads,
@@ -346,11 +349,15 @@ KVQ_API int kvq_quantize_append_rope(const kvq_cfg* cfg, const void* const* plan
  * out_dev: fp32 [batch][n_q_heads][128].
  * ws_dev: >= kvq_decode_workspace_bytes(cfg, batch, n_q_heads, max_len)
  *        bytes, 16-byte aligned, zero-filled once before its first use
- *        (KVQ_ERR_ARG if misaligned). Every completed call
- *        leaves the arrival counters it keeps at the end of the workspace at
- *        zero, so one workspace can serve any sequence of calls with the same
- *        n_kv_heads (and shapes that fit) on one stream; calls that overlap
- *        on the GPU must use different workspaces.
+ *        (KVQ_ERR_ARG if misaligned). Only the per-(sequence, KV head)
+ *        blocks at the end of the workspace must be zero when a call starts;
+ *        every completed call leaves the blocks it used at zero, and the
+ *        split records (written before they are read) never reach into the
+ *        blocks of a call with at most as many sequences x KV heads. So one
+ *        workspace, sized for the largest batch x n_kv_heads, serves any
+ *        sequence of calls on one stream whatever their max_len, query
+ *        heads or bit budget; calls that overlap on the GPU must use
+ *        different workspaces.
  * status_dev: required.
  * Returns KVQ_OK or a negative code.
  */
@@ -408,7 +415,7 @@ KVQ_API int kvq_combine_partials(const kvq_cfg* cfg, const void* const* plans_de
  * [batch][n_new][n_kv_heads][128] of kv_dtype). A sequence with
  * len + n_new > min(cap_tokens, max_len) gets no append (CAPACITY; len
  * unchanged) and is decoded over its min(len, max_len) tokens. The workspace
- * must be zero-filled once before first use and serve one n_kv_heads value.
+ * follows the rules of kvq_decode_attn.
  * The kernel uses programmatic dependent launch: work that reads nothing the
  * previous kernel on the stream writes (the plan, the lookup tables) starts
  * before that kernel ends. step_flags:
@@ -517,7 +524,8 @@ KVQ_API int kvq_paged_append_decode(const kvq_cfg* cfg, const void* const* plans
  * q_dev: bf16 [batch][n_q_heads][128], 4-byte aligned; out_dev: fp32
  *        [batch][n_q_heads][128] = softmax(q k^T / sqrt(128)) v per head.
  * ws_dev: >= kvq_bf16_decode_workspace_bytes(...) bytes, 16-byte aligned,
- *        zero-filled once; same reuse rules as kvq_decode_attn.
+ *        zero-filled once; same reuse rules as kvq_decode_attn (here only
+ *        the merge counters at the end must start at zero).
  * Returns KVQ_OK or a negative code.
  */
 KVQ_API size_t kvq_bf16_decode_workspace_bytes(int batch, int n_kv_heads, int n_q_heads,
@@ -540,23 +548,31 @@ KVQ_API int kvq_bf16_decode_attn(const void* k_dev, const void* v_dev, const int
  * passes every input and output buffer.
  *
  * Scratch: the split partials go to a fixed array of
- * kvq_decode_noalloc_scratch_bytes() (4 MiB) in the library's own device
+ * kvq_decode_noalloc_scratch_bytes() (16 MiB) in the library's own device
  * memory, present on every GPU that loads the library until the process
- * exits. A call whose partials would not fit (kvq_decode_workspace_bytes of
- * the same arguments > 4 MiB) returns KVQ_ERR_WORKSPACE and launches nothing.
+ * exits. A call whose workspace would not fit (kvq_decode_workspace_bytes of
+ * the same arguments > 16 MiB; on a B200 that is more than about 100
+ * sequences x KV heads) returns KVQ_ERR_WORKSPACE and launches nothing.
  * The call allocates nothing: no cudaMalloc, cudaFree or allocating routine.
  *
  * Set-up: the first call on a device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current) and caches it; make that
- * first call before any stream capture on the device.
+ * first call before any stream capture on the device. The cached address
+ * belongs to the device's current primary context: after cudaDeviceReset
+ * (or anything else that destroys that context) it is stale, and the call
+ * must not be used again in the process.
  *
  * Sharing: every call uses the same array, which keeps the last call's
- * contents. The split records are always written before they are read; the
- * arrival counters kept at the end of the array must be zero when a call
- * starts - the array is zero when the library is loaded, and every completed
- * call resets the counters it used. Calls that overlap on the GPU - on
- * different streams, or from different host threads without ordering - race
- * on the array and may give wrong outputs; order them on one stream.
+ * contents. The array is laid out like a kvq_decode_attn workspace: split
+ * records from its start (always written before they are read) and, at
+ * fixed distances from its end, one block per (sequence, KV head) of arrival
+ * counters and exponent buckets that must be zero when a call starts. The
+ * array is zero when the library is loaded, every completed call clears the
+ * blocks it used, and no call's records reach the blocks of another call
+ * that fits, so calls of any shapes that fit may follow one another. Calls
+ * that overlap on the GPU - on different streams, or from different host
+ * threads without ordering - race on the array and may give wrong outputs;
+ * order them on one stream.
  */
 KVQ_API int kvq_decode_attn_noalloc(const kvq_cfg* cfg, const void* const* plans_dev,
                                     const void* const* cache_dev, const int32_t* len_dev,
@@ -564,7 +580,7 @@ KVQ_API int kvq_decode_attn_noalloc(const kvq_cfg* cfg, const void* const* plans
                                     int n_q_heads, float* out_dev, uint32_t* status_dev,
                                     kvq_stream_t stream);
 
-/* Size of the fixed scratch used by kvq_decode_attn_noalloc (4 MiB). */
+/* Size of the fixed scratch used by kvq_decode_attn_noalloc (16 MiB). */
 KVQ_API size_t kvq_decode_noalloc_scratch_bytes(void);
 
 #ifdef __cplusplus

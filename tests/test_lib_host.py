@@ -161,6 +161,12 @@ def test_sizes():
     assert kvq.cache_bytes(cfg, 33) == 2 * 2 * 3200
     assert kvq.alloc_workspace_bytes(cfg) >= 2 * 64 * 16
     assert kvq.decode_workspace_bytes(cfg, 1, 16, 131072) > 0
+    # decode workspace: sized by batch x n_kv only (records bounded by one
+    # wave; per-pair counter/bucket blocks at fixed distances from the end)
+    w = kvq.decode_workspace_bytes(cfg, 4, 16, 1 << 10)
+    assert w == kvq.decode_workspace_bytes(cfg, 4, 4, 1 << 20)
+    assert w == kvq.decode_workspace_bytes(kvq.make_cfg(cfg.n_kv_heads, 1, 8), 4, 8, 77)
+    assert kvq.decode_workspace_bytes(cfg, 8, 16, 1 << 10) - w == 4 * cfg.n_kv_heads * 135296
     assert kvq.lib().kvq_plan_bytes() == 1024
 
 
