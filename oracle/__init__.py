@@ -26,6 +26,8 @@ Modules (each function cites the passage it follows):
                  decision arithmetic written out step by step.
 * ``layout``   - the packed tile record: pack and unpack.
 * ``attn``     - dequantization and exact softmax attention in fp64.
+* ``window``   - the recent-token window: which tokens stay exact, decode
+                 over the packed and the exact tokens together.
 
 Floating point is fp64 except where a quantization decision is taken: there
 the arithmetic is IEEE fp32 in a fixed order so that codes are reproducible
