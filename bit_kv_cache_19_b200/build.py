@@ -15,7 +15,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libkvq.so")
-SOURCES = ["api.cu", "quantize.cu", "decode.cu", "dense.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "quantize.cu", "decode.cu", "dense.cu", "noalloc.cu", "window.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -31,6 +31,14 @@ cudaError_t launch_dense_decode(const void* k, const void* v, const int32_t* len
                                 cudaStream_t st);
 cudaError_t launch_combine(const Plan* const* plans, const float* recs, int n_parts, int batch,
                            int n_q, int n_kv, float* out, cudaStream_t st);
+void set_decode_stall(long long cycles);
+cudaError_t launch_window_push(const void* k, const void* v, int dtype, int n_new, int n_kv,
+                               int32_t* len, int32_t* wlen, float* const* wins, int R,
+                               int64_t cap, int batch, cudaStream_t st);
+cudaError_t launch_window_record(const Plan* const* plans, const float* const* wins,
+                                 const int32_t* len, const int32_t* wlen, int R, const void* q,
+                                 int q_dtype, int n_q, int n_kv, int batch, float* recs,
+                                 cudaStream_t st);
 
 namespace {
 
@@ -433,6 +441,9 @@ static int quantize_append_impl(const kvq_cfg* cfg, const void* const* plans_dev
   p.status = status_dev;
   p.rope = theta ? 1 : 0;
   for (int j = 0; j < 64; ++j) p.theta[j] = theta ? theta[j] : 0.0;
+  p.wins = nullptr;
+  p.wlen = nullptr;
+  p.R = 0;
   cudaError_t e = launch_quantize_append(p, cfg->bits_v, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "quantize_append");
   return KVQ_OK;
@@ -608,6 +619,115 @@ int kvq_combine_partials(const kvq_cfg* cfg, const void* const* plans_dev, int n
                                  n_parts, batch, n_q_heads, cfg->n_kv_heads, out_dev,
                                  reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "combine_partials");
+  return KVQ_OK;
+}
+
+int kvq_debug_decode_stall(long long cycles) {
+  if (cycles < 0 || cycles > (1ll << 40)) return fail(KVQ_ERR_ARG, "stall cycles %lld", cycles);
+  set_decode_stall(cycles);
+  return KVQ_OK;
+}
+
+// ---------------------------------------------------------- recent window
+constexpr int kRecFloats = 132;  // merged record: m, l, 2 unused, o[128]
+
+size_t kvq_window_bytes(const kvq_cfg* cfg, int R) {
+  if (check_cfg(cfg) != KVQ_OK || R < 0 || R > (1 << 20)) return 0;
+  return (size_t)2 * R * cfg->n_kv_heads * kHeadDim * sizeof(float);
+}
+
+int kvq_window_append(const kvq_cfg* cfg, const void* const* plans_dev, const void* k_dev,
+                      const void* v_dev, int kv_dtype, int n_new, void* const* cache_dev,
+                      int32_t* len_dev, int64_t cap_tokens, void* const* win_dev,
+                      int32_t* wlen_dev, int R, int batch, uint32_t* status_dev,
+                      kvq_stream_t stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (R < 0 || R > (1 << 20)) return fail(KVQ_ERR_ARG, "window R %d", R);
+  if (!wlen_dev || (R > 0 && !win_dev)) return fail(KVQ_ERR_ARG, "null window pointer");
+  if (R == 0)  // no window: every token is quantized at once
+    return quantize_append_impl(cfg, plans_dev, k_dev, v_dev, kv_dtype, batch, n_new,
+                                contiguous_map(cache_dev), len_dev, cap_tokens, nullptr,
+                                status_dev, stream);
+  if (!plans_dev || !cache_dev || !len_dev || !status_dev)
+    return fail(KVQ_ERR_ARG, "null device pointer");
+  if (!dtype_ok(kv_dtype)) return fail(KVQ_ERR_ARG, "dtype %d", kv_dtype);
+  if (batch < 1 || batch > 65535) return fail(KVQ_ERR_ARG, "batch %d", batch);
+  if (n_new < 0 || n_new > (1 << 24) || cap_tokens < 0 || cap_tokens > 0x7FFFFFFF)
+    return fail(KVQ_ERR_ARG, "n_new %d / cap_tokens %lld", n_new, (long long)cap_tokens);
+  if (n_new == 0) return KVQ_OK;
+  if (!k_dev || !v_dev) return fail(KVQ_ERR_ARG, "null k/v pointer");
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  QuantParams p;
+  p.plans = reinterpret_cast<const Plan* const*>(plans_dev);
+  p.k = k_dev;
+  p.v = v_dev;
+  p.dtype = kv_dtype;
+  p.batch = batch;
+  p.n_new = n_new;
+  p.n_kv = cfg->n_kv_heads;
+  p.cm = contiguous_map(cache_dev);
+  p.len = len_dev;
+  p.cap = cap_tokens;
+  p.tile_bytes = tile_bytes(cfg->bits_k, cfg->bits_v);
+  p.status = status_dev;
+  p.rope = 0;
+  for (int j = 0; j < 64; ++j) p.theta[j] = 0.0;
+  p.wins = reinterpret_cast<const float* const*>(win_dev);
+  p.wlen = wlen_dev;
+  p.R = R;
+  cudaError_t e = launch_quantize_append(p, cfg->bits_v, st);
+  if (e != cudaSuccess) return cuda_fail(e, "window_append (evictions)");
+  e = launch_window_push(k_dev, v_dev, kv_dtype, n_new, cfg->n_kv_heads, len_dev, wlen_dev,
+                         reinterpret_cast<float* const*>(win_dev), R, cap_tokens, batch, st);
+  if (e != cudaSuccess) return cuda_fail(e, "window_append (ring)");
+  return KVQ_OK;
+}
+
+static size_t window_records_bytes(int batch, int n_q_heads) {
+  return ((size_t)2 * batch * n_q_heads * kRecFloats * sizeof(float) + 255) / 256 * 256;
+}
+
+size_t kvq_window_decode_workspace_bytes(const kvq_cfg* cfg, int batch, int n_q_heads,
+                                         int64_t max_len) {
+  const size_t d = kvq_decode_workspace_bytes(cfg, batch, n_q_heads, max_len);
+  return d ? d + window_records_bytes(batch, n_q_heads) : 0;
+}
+
+int kvq_decode_attn_window(const kvq_cfg* cfg, const void* const* plans_dev,
+                           const void* const* cache_dev, const int32_t* len_dev,
+                           const void* const* win_dev, const int32_t* wlen_dev, int R, int batch,
+                           int64_t max_len, const void* q_dev, int q_dtype, int n_q_heads,
+                           float* out_dev, void* ws_dev, size_t ws_bytes, uint32_t* status_dev,
+                           kvq_stream_t stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (R < 0 || R > (1 << 20)) return fail(KVQ_ERR_ARG, "window R %d", R);
+  if (!wlen_dev || (R > 0 && !win_dev) || !out_dev || !ws_dev)
+    return fail(KVQ_ERR_ARG, "null device pointer");
+  if (batch < 1 || batch > 65535) return fail(KVQ_ERR_ARG, "batch %d", batch);
+  if (n_q_heads < 1 || n_q_heads % cfg->n_kv_heads != 0 || n_q_heads / cfg->n_kv_heads > 16)
+    return fail(KVQ_ERR_ARG, "n_q_heads %d vs n_kv_heads %d", n_q_heads, cfg->n_kv_heads);
+  const size_t rb = window_records_bytes(batch, n_q_heads);
+  if (ws_bytes < kvq_window_decode_workspace_bytes(cfg, batch, n_q_heads, max_len))
+    return fail(KVQ_ERR_WORKSPACE, "window decode workspace %zu < %zu", ws_bytes,
+                kvq_window_decode_workspace_bytes(cfg, batch, n_q_heads, max_len));
+  float* recs = reinterpret_cast<float*>(ws_dev);
+  float* rec_win = recs + (size_t)batch * n_q_heads * kRecFloats;
+  // the packed tokens: one merged record per query head (part 0)
+  rc = decode_impl(cfg, plans_dev, contiguous_map(cache_dev), len_dev, batch, max_len, q_dev,
+                   q_dtype, n_q_heads, nullptr, recs, reinterpret_cast<uint8_t*>(ws_dev) + rb,
+                   ws_bytes - rb, status_dev, stream);
+  if (rc) return rc;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_window_record(reinterpret_cast<const Plan* const*>(plans_dev),
+                                       reinterpret_cast<const float* const*>(win_dev), len_dev,
+                                       wlen_dev, R, q_dev, q_dtype, n_q_heads, cfg->n_kv_heads,
+                                       batch, rec_win, st);
+  if (e != cudaSuccess) return cuda_fail(e, "decode_attn_window (window)");
+  e = launch_combine(reinterpret_cast<const Plan* const*>(plans_dev), recs, 2, batch, n_q_heads,
+                     cfg->n_kv_heads, out_dev, st);
+  if (e != cudaSuccess) return cuda_fail(e, "decode_attn_window (combine)");
   return KVQ_OK;
 }
 

@@ -109,6 +109,13 @@ struct QuantParams {
   uint32_t* status;
   int rope;           // keys are pre-RoPE: rotate each to its position first
   double theta[64];   // RoPE block frequencies base^(-2j/128)
+  // recent-token window (wins != nullptr): per sequence, the oldest
+  // max(0, wlen + n_new - R) tokens of window + new tokens are quantized
+  // (window token at position t: fp32 rows in ring slot t mod R, keys then
+  // values), and the lengths are left to the ring kernel
+  const float* const* wins;
+  const int32_t* wlen;
+  int R;
 };
 
 // ------------------------------------------------------------------ device
@@ -177,12 +184,15 @@ __device__ __forceinline__ bool mbar_try_wait(unsigned long long* bar, uint32_t 
   return ok != 0;
 }
 
-// Bounded wait: gives up after ~2^31 clock cycles (about a second).
-__device__ __forceinline__ bool mbar_wait_bounded(unsigned long long* bar, uint32_t phase) {
+// Bounded wait: gives up after `limit` clock cycles (default 2^31, about a
+// second) and returns false.
+constexpr long long kWaitCycles = 1ll << 31;
+__device__ __forceinline__ bool mbar_wait_bounded(unsigned long long* bar, uint32_t phase,
+                                                  long long limit = kWaitCycles) {
   if (mbar_try_wait(bar, phase)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, phase)) {
-    if (clock64() - t0 > (1ll << 31)) return false;
+    if (clock64() - t0 > limit) return false;
   }
   return true;
 }

@@ -92,12 +92,62 @@ __global__ void __launch_bounds__(128) energy_kernel(const void* __restrict__ k,
 __constant__ float c_thr[KVQ_CB_N_THR] = KVQ_CB_THR;
 
 
-// Work item = the new tokens of one 32-token tile of one (sequence, KV head);
-// CTAs loop over items (item = (b n_kv + h) tiles_max + i, tile = len0 / 32
-// + i). A tile's words are assembled in shared memory (from zero for a fresh
-// tile, else from the record) by the two passes of quant_dev.cuh and written
-// back whole. The plan is reloaded only when (b, h) changes.
-template <int BV>
+// Work item = the new tokens of one 32-token tile of one (sequence, KV head):
+// item = (b n_kv + h) tiles_max + i, tile = len0 / 32 + i.
+struct Item {
+  int b, h, tile, len0, t_lo, t_hi;
+  int n_add, w0;  // tokens quantized for the sequence; window tokens among them
+  bool fits;      // capacity allows the append
+  bool live;      // and the item has tokens to quantize
+};
+
+template <bool WIN>
+__device__ __forceinline__ Item item_of(const QuantParams& p, int item) {
+  Item it;
+  const int bh = item / p.tiles_max, ti = item - bh * p.tiles_max;
+  it.b = bh / p.n_kv;
+  it.h = bh - it.b * p.n_kv;
+  it.len0 = p.len[it.b];
+  it.w0 = 0;
+  it.n_add = p.n_new;
+  if (WIN) {
+    it.w0 = min(max(p.wlen[it.b], 0), p.R);
+    it.n_add = max(0, it.w0 + p.n_new - p.R);
+  }
+  it.tile = it.len0 / kTile + ti;
+  it.t_lo = max(it.len0, it.tile * kTile);
+  it.t_hi = min(it.len0 + it.n_add, it.tile * kTile + kTile);
+  it.fits = it.len0 >= 0 && (int64_t)it.len0 + it.n_add <= p.cap;
+  it.live = it.fits && it.t_lo < it.t_hi;
+  return it;
+}
+
+// Source rows of the token at position t (>= len0) of an item: the window
+// ring (fp32) for the first w0 tokens of a window append, else the new
+// tokens' rows (element offsets; returns the dtype).
+__device__ __forceinline__ int token_source(const QuantParams& p, const Item& it, int t,
+                                            const void*& k, const void*& v, size_t& row) {
+  const int i = t - it.len0;
+  if (i < it.w0) {
+    const int slot = t % p.R;
+    const float* w = p.wins[it.b];
+    k = w;
+    v = w + (size_t)p.R * p.n_kv * kHeadDim;
+    row = ((size_t)slot * p.n_kv + it.h) * kHeadDim;
+    return KVQ_FP32;
+  }
+  k = p.k;
+  v = p.v;
+  row = (((size_t)it.b * p.n_new + (i - it.w0)) * p.n_kv + it.h) * kHeadDim;
+  return p.dtype;
+}
+
+// CTAs loop over the work items. A tile's words are assembled in shared
+// memory (from zero for a fresh tile, else from the record) by the two passes
+// of quant_dev.cuh and written back whole. The plan is reloaded only when
+// (b, h) changes. WIN: a window append (rows from the ring or the new tokens,
+// token by token); otherwise every row comes from the new tokens.
+template <int BV, bool WIN>
 __global__ void __launch_bounds__(256, 4) quantize_append_kernel(QuantParams p) {
   __shared__ Plan s_plan;
   __shared__ float s_thr[KVQ_CB_N_THR];
@@ -114,16 +164,14 @@ __global__ void __launch_bounds__(256, 4) quantize_append_kernel(QuantParams p) 
   bool plan_ok = false;
   const int n_items = p.batch * p.n_kv * p.tiles_max;
   for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-    const int bh = item / p.tiles_max, ti = item - bh * p.tiles_max;
-    const int b = bh / p.n_kv, h = bh - b * p.n_kv;
-    const int len0 = p.len[b];
-    if (len0 < 0 || (int64_t)len0 + p.n_new > p.cap) {
-      if (threadIdx.x == 0 && ti == 0 && h == 0) atomicOr(p.status, KVQ_FLAG_CAPACITY);
+    const Item it = item_of<WIN>(p, item);
+    const int b = it.b, h = it.h, bh = b * p.n_kv + h, tile = it.tile, len0 = it.len0;
+    if (!it.fits) {
+      if (threadIdx.x == 0 && item % p.tiles_max == 0 && h == 0)
+        atomicOr(p.status, KVQ_FLAG_CAPACITY);
       continue;
     }
-    const int tile = len0 / kTile + ti;
-    const int t_lo = max(len0, tile * kTile), t_hi = min(len0 + p.n_new, tile * kTile + kTile);
-    if (t_lo >= t_hi) continue;
+    if (!it.live) continue;
     uint8_t* rec = const_cast<uint8_t*>(page_base(p.cm, b, tile));
     if (!rec) {
       if (threadIdx.x == 0) atomicOr(p.status, KVQ_FLAG_BAD_PAGE);
@@ -160,16 +208,24 @@ __global__ void __launch_bounds__(256, 4) quantize_append_kernel(QuantParams p) 
     __syncthreads();
 
     // ---- pass 1: one warp per new token
-    const int p_lo = t_lo - tile * kTile, p_hi = t_hi - tile * kTile;
+    const int p_lo = it.t_lo - tile * kTile, p_hi = it.t_hi - tile * kTile;
     uint32_t flags = 0;
     __half* norms = reinterpret_cast<__half*>(rec + 512 * (pl.bits_k + BV));
     for (int pp = p_lo + warp; pp < p_hi; pp += nw) {
-      const size_t row =
-          (((size_t)b * p.n_new + (tile * kTile + pp - len0)) * p.n_kv + h) * kHeadDim;
       __half kn, vn;
-      warp_token_pass<BV>(pl, s_thr, p.k, p.v, p.dtype, row, lane, pp, s_kz + pp * kKzStride,
-                          s_words, clear, kn, vn, flags, p.rope ? s_theta : nullptr,
-                          (int64_t)tile * kTile + pp);
+      if (WIN) {
+        const void *ks, *vs;
+        size_t row;
+        const int dt = token_source(p, it, tile * kTile + pp, ks, vs, row);
+        warp_token_pass<BV>(pl, s_thr, ks, vs, dt, row, lane, pp, s_kz + pp * kKzStride,
+                            s_words, clear, kn, vn, flags);
+      } else {
+        const size_t row =
+            (((size_t)b * p.n_new + (tile * kTile + pp - len0)) * p.n_kv + h) * kHeadDim;
+        warp_token_pass<BV>(pl, s_thr, p.k, p.v, p.dtype, row, lane, pp, s_kz + pp * kKzStride,
+                            s_words, clear, kn, vn, flags, p.rope ? s_theta : nullptr,
+                            (int64_t)tile * kTile + pp);
+      }
       if (lane == 0) {
         norms[pp] = kn;
         norms[kTile + pp] = vn;
@@ -214,6 +270,12 @@ cudaError_t launch_energy(const void* k, int dtype, int64_t n_tokens, int n_kv,
   return cudaGetLastError();
 }
 
+template <int BV>
+static void launch_quant_t(const QuantParams& p, bool win, unsigned grid, cudaStream_t st) {
+  if (win) quantize_append_kernel<BV, true><<<grid, 256, 0, st>>>(p);
+  else quantize_append_kernel<BV, false><<<grid, 256, 0, st>>>(p);
+}
+
 cudaError_t launch_quantize_append(const QuantParams& p_in, int bits_v, cudaStream_t st) {
   QuantParams p = p_in;
   p.tiles_max = (p.n_new + kTile - 1) / kTile + 1;
@@ -224,19 +286,21 @@ cudaError_t launch_quantize_append(const QuantParams& p_in, int bits_v, cudaStre
     (void)cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   (void)cudaGetLastError();
   const unsigned grid = (unsigned)std::min<int64_t>(n_items, (int64_t)4 * sms);  // resident
+  const bool win = p.wins != nullptr;
   switch (bits_v) {
-    case 1: quantize_append_kernel<1><<<grid, 256, 0, st>>>(p); break;
-    case 2: quantize_append_kernel<2><<<grid, 256, 0, st>>>(p); break;
-    case 3: quantize_append_kernel<3><<<grid, 256, 0, st>>>(p); break;
-    case 4: quantize_append_kernel<4><<<grid, 256, 0, st>>>(p); break;
-    case 5: quantize_append_kernel<5><<<grid, 256, 0, st>>>(p); break;
-    case 6: quantize_append_kernel<6><<<grid, 256, 0, st>>>(p); break;
-    case 7: quantize_append_kernel<7><<<grid, 256, 0, st>>>(p); break;
-    case 8: quantize_append_kernel<8><<<grid, 256, 0, st>>>(p); break;
+    case 1: launch_quant_t<1>(p, win, grid, st); break;
+    case 2: launch_quant_t<2>(p, win, grid, st); break;
+    case 3: launch_quant_t<3>(p, win, grid, st); break;
+    case 4: launch_quant_t<4>(p, win, grid, st); break;
+    case 5: launch_quant_t<5>(p, win, grid, st); break;
+    case 6: launch_quant_t<6>(p, win, grid, st); break;
+    case 7: launch_quant_t<7>(p, win, grid, st); break;
+    case 8: launch_quant_t<8>(p, win, grid, st); break;
     default: return cudaErrorInvalidValue;
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (p.wins) return cudaSuccess;  // the window's ring kernel updates the lengths
   bump_len_kernel<<<(p.batch + 255) / 256, 256, 0, st>>>(const_cast<int32_t*>(p.len), p.batch,
                                                           p.n_new, p.cap);
   return cudaGetLastError();

@@ -113,6 +113,13 @@ _SIGS = {
     "kvq_paged_append_decode": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i32,
                                        ctypes.POINTER(Pages), _vp, _i32, _i64, _vp, _i32, _i32,
                                        _vp, _vp, _sz, _i32, ctypes.c_double, _vp, _vp]),
+    "kvq_debug_decode_stall": (_i32, [ctypes.c_longlong]),
+    "kvq_window_bytes": (_sz, [ctypes.POINTER(Cfg), _i32]),
+    "kvq_window_append": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i32, _vp, _vp, _i64,
+                                 _vp, _vp, _i32, _i32, _vp, _vp]),
+    "kvq_window_decode_workspace_bytes": (_sz, [ctypes.POINTER(Cfg), _i32, _i32, _i64]),
+    "kvq_decode_attn_window": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _vp, _vp, _i32, _i32,
+                                      _i64, _vp, _i32, _i32, _vp, _vp, _sz, _vp, _vp]),
 }
 EXPORTS = tuple(_SIGS)
 
@@ -396,3 +403,34 @@ def bf16_decode_attn(k, v, lens, max_len, q, out, ws, status):
     _check(lib().kvq_bf16_decode_attn(_ptr(k), _ptr(v), _ptr(lens), batch, n_kv, cap, max_len,
                                       _ptr(q), q.shape[1], _ptr(out), _ptr(ws),
                                       ws.numel() * ws.element_size(), _ptr(status), _stream()))
+
+
+def window_bytes(cfg, R) -> int:
+    """Bytes of one sequence's recent-token window of R slots."""
+    return lib().kvq_window_bytes(ctypes.byref(cfg), R)
+
+
+def window_decode_workspace_bytes(cfg, batch, n_q_heads, max_len) -> int:
+    return lib().kvq_window_decode_workspace_bytes(ctypes.byref(cfg), batch, n_q_heads, max_len)
+
+
+def window_append(cfg, plan_ptrs, k, v, cache_ptrs, lens, cap_tokens, win_ptrs, wlens, R,
+                  status):
+    """Append k, v [batch, n_new, n_kv, 128]: the oldest tokens beyond the
+    R-token window are quantize-appended, the rest enter the window ring."""
+    batch, n_new = k.shape[0], k.shape[1]
+    _check(lib().kvq_window_append(ctypes.byref(cfg), _ptr(plan_ptrs), _ptr(k), _ptr(v),
+                                   _dtype_code(k), n_new, _ptr(cache_ptrs), _ptr(lens),
+                                   cap_tokens, _ptr(win_ptrs), _ptr(wlens), R, batch,
+                                   _ptr(status), _stream()))
+
+
+def decode_attn_window(cfg, plan_ptrs, cache_ptrs, lens, win_ptrs, wlens, R, max_len, q, out,
+                       ws, status):
+    """Decode q [batch, n_q, 128] over the packed tokens and the window tokens."""
+    batch, n_q = q.shape[0], q.shape[1]
+    _check(lib().kvq_decode_attn_window(ctypes.byref(cfg), _ptr(plan_ptrs), _ptr(cache_ptrs),
+                                        _ptr(lens), _ptr(win_ptrs), _ptr(wlens), R, batch,
+                                        max_len, _ptr(q), _dtype_code(q), n_q, _ptr(out),
+                                        _ptr(ws), ws.numel() * ws.element_size(), _ptr(status),
+                                        _stream()))

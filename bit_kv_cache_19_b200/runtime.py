@@ -16,7 +16,13 @@ from . import kvq
 
 
 class PackedLayer:
-    def __init__(self, cfg, batch: int, cap_tokens: int, device="cuda", layer: int = 0):
+    """One layer's packed caches for a batch of sequences. ``window=R > 0``
+    adds a recent-token window per sequence: the R most recent tokens stay
+    exact (appended with ``append_window``, decoded with ``decode_window``);
+    ``lens`` then counts the packed tokens and ``wlens`` the window's."""
+
+    def __init__(self, cfg, batch: int, cap_tokens: int, device="cuda", layer: int = 0,
+                 window: int = 0):
         self.cfg = cfg
         self.batch = batch
         self.cap = cap_tokens
@@ -33,6 +39,14 @@ class PackedLayer:
         self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
         self.plans_host = None
         self.energy = None
+        self.window = window
+        self.wlens = torch.zeros(batch, dtype=torch.int32, device=self.device)
+        self.wins, self.win_ptrs = [], None
+        if window > 0:
+            wb = kvq.window_bytes(cfg, window)
+            self.wins = [torch.zeros(wb // 4, dtype=torch.float32, device=self.device)
+                         for _ in range(batch)]
+            self.win_ptrs = kvq.ptr_array(self.wins, self.device)
 
     # -------------------------------------------------------------- calls
     def alloc_bits(self, k):
@@ -72,6 +86,33 @@ class PackedLayer:
         each key is rotated to its cache position, then appended."""
         kvq.quantize_append_rope(self.cfg, self.plan_ptrs, k_pre, v, self.cache_ptrs, self.lens,
                                  self.cap, rope_base, self.status)
+
+    def append_window(self, k, v):
+        """k, v [batch, n_new, n_kv, 128] (device) through the recent-token
+        window: tokens older than the window's R are quantize-appended."""
+        kvq.window_append(self.cfg, self.plan_ptrs, k, v, self.cache_ptrs, self.lens, self.cap,
+                          self.win_ptrs, self.wlens, self.window, self.status)
+
+    def decode_window(self, q, out=None, ws=None, max_len=None):
+        """q [batch, n_q, 128] -> fp32 [batch, n_q, 128] over the packed and
+        the window tokens."""
+        max_len = self.cap if max_len is None else max_len
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=self.device)
+        if ws is None:
+            n = kvq.window_decode_workspace_bytes(self.cfg, self.batch, q.shape[1], max_len)
+            ws = torch.zeros(n, dtype=torch.uint8, device=self.device)
+        kvq.decode_attn_window(self.cfg, self.plan_ptrs, self.cache_ptrs, self.lens,
+                               self.win_ptrs, self.wlens, self.window, max_len, q, out, ws,
+                               self.status)
+        return out
+
+    def window_rows(self, seq: int):
+        """The window ring of one sequence on the host: keys, values fp32
+        [R, n_kv, 128] (slot t mod R holds token t)."""
+        R, n_kv = self.window, self.cfg.n_kv_heads
+        w = self.wins[seq].cpu().numpy().reshape(2, R, n_kv, 128)
+        return w[0], w[1]
 
     def decode(self, q, out=None, ws=None, max_len=None):
         """q [batch, n_q, 128] -> fp32 [batch, n_q, 128]."""

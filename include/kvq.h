@@ -405,6 +405,71 @@ KVQ_API int kvq_combine_partials(const kvq_cfg* cfg, const void* const* plans_de
                                  kvq_stream_t stream);
 
 /*
+ * Test hook (no counterpart in the paper): with cycles > 0, every later
+ * packed decode launch (kvq_decode_attn and the calls built on it) first
+ * waits `cycles` clock cycles on a shared-memory barrier that nothing
+ * arrives on. The wait runs out, the launch sets KVQ_FLAG_TIMEOUT in
+ * *status_dev, lets the tile copies it already issued land, skips its tiles
+ * and completes normally (its outputs are then meaningless), which exercises
+ * the path every bounded wait of the kernels takes when it gives up. 0
+ * restores normal launches. Process-wide; for tests only. Returns KVQ_OK or
+ * KVQ_ERR_ARG.
+ */
+KVQ_API int kvq_debug_decode_stall(long long cycles);
+
+/*
+ * Recent-token window ("RoPE-Aware Bit Allocation for KV-Cache
+ * Quantization", abstract: the paper's K3V2 result is stated for a packed
+ * cache without an fp16 recent-key buffer, which names such a buffer as an
+ * option of the serving path). Reading adopted: the keys and values of the R
+ * most recent tokens of a sequence stay exactly as appended; a token is
+ * quantized with the layer's plan, exactly as without a window, once R newer
+ * tokens follow it (tokens leave in order). After T appended tokens the
+ * packed cache holds tokens [0, T - w) and the window tokens [T - w, T),
+ * w = min(R, T), whatever the sizes of the appends. Decode attends over the
+ * packed and the window tokens together.
+ *
+ * Window buffer (one per sequence, caller-owned, >= kvq_window_bytes(cfg, R)
+ * bytes, 16-byte aligned): a ring of R slots, token t in slot t mod R; keys
+ * fp32 [R][n_kv_heads][128], then values fp32 [R][n_kv_heads][128] (the
+ * appended 16-bit values held exactly in fp32). wlen_dev: int32 [batch],
+ * tokens in each window, zero-filled with the buffers; len_dev counts the
+ * packed tokens only.
+ *
+ * kvq_window_append: appends n_new tokens per sequence (k_dev, v_dev as for
+ *   kvq_quantize_append). The oldest max(0, wlen + n_new - R) of the window
+ *   and new tokens are quantize-appended to the packed cache at len..., the
+ *   others enter the ring; then len += evicted, wlen = min(R, wlen + n_new).
+ *   A sequence whose evictions do not fit min(cap_tokens) flags CAPACITY and
+ *   is left unchanged. R = 0 is kvq_quantize_append (every token quantized,
+ *   wlen untouched). Two launches; no workspace.
+ * kvq_decode_attn_window: kvq_decode_attn over the packed tokens (len_dev,
+ *   max_len >= every len) and the window tokens (wlen_dev) together: one
+ *   partial decode of the packed tokens, one record of the window tokens
+ *   (fp32 logits q.k log2(e)/sqrt(128) and values rotated like the packed
+ *   ones), one combine; three launches. ws_dev: >=
+ *   kvq_window_decode_workspace_bytes(...) bytes, 16-byte aligned,
+ *   zero-filled once, reuse rules of kvq_decode_attn; its first
+ *   2 batch n_q_heads 132 floats (rounded up to 256 bytes) hold the two
+ *   records, the rest serves the partial decode.
+ * Both return KVQ_OK or a negative code.
+ */
+KVQ_API size_t kvq_window_bytes(const kvq_cfg* cfg, int R);
+KVQ_API int kvq_window_append(const kvq_cfg* cfg, const void* const* plans_dev, const void* k_dev,
+                              const void* v_dev, int kv_dtype, int n_new, void* const* cache_dev,
+                              int32_t* len_dev, int64_t cap_tokens, void* const* win_dev,
+                              int32_t* wlen_dev, int R, int batch, uint32_t* status_dev,
+                              kvq_stream_t stream);
+KVQ_API size_t kvq_window_decode_workspace_bytes(const kvq_cfg* cfg, int batch, int n_q_heads,
+                                                 int64_t max_len);
+KVQ_API int kvq_decode_attn_window(const kvq_cfg* cfg, const void* const* plans_dev,
+                                   const void* const* cache_dev, const int32_t* len_dev,
+                                   const void* const* win_dev, const int32_t* wlen_dev, int R,
+                                   int batch, int64_t max_len, const void* q_dev, int q_dtype,
+                                   int n_q_heads, float* out_dev, void* ws_dev, size_t ws_bytes,
+                                   uint32_t* status_dev, kvq_stream_t stream);
+
+/*
  * One serving step in one launch: kvq_quantize_append of n_new tokens per
  * sequence followed by kvq_decode_attn over the grown caches (the pages'
  * packed-cache serving path: append the step's keys and values, then decode).

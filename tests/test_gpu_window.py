@@ -1,0 +1,133 @@
+"""GPU parity of the recent-token window (kvq_window_append,
+kvq_decode_attn_window) against the oracle's window reading.
+
+After any sequence of appends, the packed cache must hold exactly the oracle
+records of the tokens that left the window (bit for bit), the ring must hold
+the window tokens exactly (token t in slot t mod R), and decode must be the
+fp64 attention over the dequantized packed tokens and the exact window tokens
+within 2e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle_pipeline as op
+import synth
+from bit_kv_cache_19_b200 import kvq
+from bit_kv_cache_19_b200.runtime import PackedLayer
+from oracle import window
+from test_gpu_parity import check_records, dev_bf16
+
+pytestmark = pytest.mark.gpu
+TOL = 2e-3
+V_SEED = 6
+
+
+def _inputs(rng, batch, T, n_kv):
+    k = synth.to_bf16_bits(rng.standard_normal((batch, T, n_kv, 128)))
+    v = synth.to_bf16_bits(rng.standard_normal((batch, T, n_kv, 128)))
+    return k, v
+
+
+def _check_state(L, kb, vb, T, E, bits_k, bits_v, R, rng, G):
+    n_kv = L.cfg.n_kv_heads
+    sp = window.split_point(T, R)
+    assert L.lens.cpu().tolist() == [sp] * L.batch
+    assert L.wlens.cpu().tolist() == [min(R, T) if R else 0] * L.batch
+    assert L.flags() == 0
+    qb = synth.to_bf16_bits(rng.standard_normal((L.batch, n_kv * G, 128)))
+    out = L.decode_window(dev_bf16(qb)).cpu().numpy()
+    for s in range(L.batch):
+        kh, vh = op.bf16_heads(kb[s, :T], vb[s, :T])
+        heads = op.layer([x[:sp] for x in kh], [x[:sp] for x in vh], bits_k, bits_v, V_SEED, 0,
+                         E=E, pack=sp > 0)[1] if sp else None
+        if sp:
+            for h in range(n_kv):
+                check_records(L.head_records(s, h, (sp + 31) // 32), heads[h]["rec"], sp,
+                              bits_k, bits_v)
+        if R:
+            wk, wv = L.window_rows(s)
+            for t, slot in window.ring_slots(T, R):
+                assert np.array_equal(wk[slot], synth.bf16_bits_to_f64(kb[s, t])), (t, slot)
+                assert np.array_equal(wv[slot], synth.bf16_bits_to_f64(vb[s, t])), (t, slot)
+        empty = [np.zeros((0, 128))] * n_kv
+        ref = window.decode(synth.bf16_bits_to_f64(qb[s]),
+                            [x["khat"] for x in heads] if sp else empty,
+                            [x["vhat"] for x in heads] if sp else empty,
+                            [x[sp:] for x in kh], [x[sp:] for x in vh])
+        assert op.rel_err(out[s], ref) <= TOL, (s, T, sp)
+
+
+@pytest.mark.parametrize("R,bits_k,bits_v,G", [(48, 3, 2, 4), (32, 2, 3, 8), (100, 4, 4, 16),
+                                               (1, 3, 3, 7)])
+def test_window_appends_and_decode(R, bits_k, bits_v, G):
+    rng = np.random.default_rng(R * 7 + bits_k)
+    n_kv, batch = 2, 2
+    steps = [300, 1, 5, 17, 1, 64, 2, 40]
+    T = sum(steps)
+    cfg = kvq.make_cfg(n_kv, bits_k, bits_v, v_seed=V_SEED)
+    L = PackedLayer(cfg, batch, T + 32, window=R)
+    E = np.exp(rng.standard_normal((n_kv, 64)) - np.arange(64) / 8.0)
+    L.set_plans(kvq.plan_build(cfg, 0, E))
+    kb, vb = _inputs(rng, batch, T, n_kv)
+    t = 0
+    for i, n in enumerate(steps):
+        L.append_window(dev_bf16(kb[:, t:t + n]), dev_bf16(vb[:, t:t + n]))
+        t += n
+        torch.cuda.synchronize()
+        if i in (0, 1, 3, len(steps) - 1):
+            _check_state(L, kb, vb, t, E, bits_k, bits_v, R, rng, G)
+
+
+def test_window_holds_everything_short_sequences():
+    # fewer tokens than the window: nothing is quantized, decode is exact attention
+    rng = np.random.default_rng(5)
+    n_kv, batch, R = 2, 3, 128
+    cfg = kvq.make_cfg(n_kv, 3, 3, v_seed=V_SEED)
+    L = PackedLayer(cfg, batch, 256, window=R)
+    E = np.exp(rng.standard_normal((n_kv, 64)))
+    L.set_plans(kvq.plan_build(cfg, 0, E))
+    kb, vb = _inputs(rng, batch, 90, n_kv)
+    L.append_window(dev_bf16(kb[:, :60]), dev_bf16(vb[:, :60]))
+    L.append_window(dev_bf16(kb[:, 60:]), dev_bf16(vb[:, 60:]))
+    torch.cuda.synchronize()
+    _check_state(L, kb, vb, 90, E, 3, 3, R, rng, 8)
+
+
+def test_no_window_is_the_plain_append_and_decode():
+    rng = np.random.default_rng(6)
+    n_kv, batch, T = 2, 2, 200
+    cfg = kvq.make_cfg(n_kv, 3, 2, v_seed=V_SEED)
+    E = np.exp(rng.standard_normal((n_kv, 64)))
+    La = PackedLayer(cfg, batch, 256, window=0)
+    Lb = PackedLayer(cfg, batch, 256)
+    for L in (La, Lb):
+        L.set_plans(kvq.plan_build(cfg, 0, E))
+    kb, vb = _inputs(rng, batch, T, n_kv)
+    La.append_window(dev_bf16(kb), dev_bf16(vb))
+    Lb.append(dev_bf16(kb), dev_bf16(vb))
+    torch.cuda.synchronize()
+    for s in range(batch):
+        assert torch.equal(La.caches[s], Lb.caches[s])
+    assert La.lens.cpu().tolist() == [T, T]
+    _check_state(La, kb, vb, T, E, 3, 2, 0, rng, 4)
+    q = dev_bf16(synth.to_bf16_bits(rng.standard_normal((batch, n_kv * 4, 128))))
+    a = La.decode_window(q).cpu().numpy()
+    b = Lb.decode(q).cpu().numpy()
+    assert op.rel_err(a, b) <= 1e-5
+
+
+def test_window_evictions_past_capacity_flag_and_leave_state():
+    rng = np.random.default_rng(8)
+    n_kv, R, cap = 1, 16, 64
+    cfg = kvq.make_cfg(n_kv, 2, 2, v_seed=V_SEED)
+    L = PackedLayer(cfg, 1, cap, window=R)
+    L.set_plans(kvq.plan_build(cfg, 0, np.exp(rng.standard_normal((n_kv, 64)))))
+    kb, vb = _inputs(rng, 1, 120, n_kv)
+    L.append_window(dev_bf16(kb[:, :70]), dev_bf16(vb[:, :70]))  # 54 packed, 16 in the window
+    torch.cuda.synchronize()
+    assert L.lens.item() == 54 and L.wlens.item() == 16 and L.flags() == 0
+    L.append_window(dev_bf16(kb[:, 70:]), dev_bf16(vb[:, 70:]))  # would pack 104 > 64
+    torch.cuda.synchronize()
+    assert L.flags() & kvq.FLAG_CAPACITY
+    assert L.lens.item() == 54 and L.wlens.item() == 16

@@ -170,6 +170,29 @@ def test_sizes():
     assert kvq.lib().kvq_plan_bytes() == 1024
 
 
+def test_window_sizes_and_argument_errors_without_gpu():
+    L = kvq.lib()
+    cfg = kvq.make_cfg(2, 3, 2)
+    assert kvq.window_bytes(cfg, 48) == 2 * 48 * 2 * 128 * 4
+    assert kvq.window_bytes(cfg, 0) == 0 and kvq.window_bytes(cfg, -1) == 0
+    d = kvq.decode_workspace_bytes(cfg, 3, 8, 1000)
+    assert kvq.window_decode_workspace_bytes(cfg, 3, 8, 1000) == d + (2 * 3 * 8 * 528 + 255) // 256 * 256
+    p = ctypes.c_void_p(256)
+    # negative R, a null length array, a window call without its ring
+    assert L.kvq_window_append(ctypes.byref(cfg), p, p, p, 0, 1, p, p, 100, p, p, -1, 1, p,
+                               None) == kvq.ERR_ARG
+    assert L.kvq_window_append(ctypes.byref(cfg), p, p, p, 0, 1, p, p, 100, p, None, 8, 1, p,
+                               None) == kvq.ERR_ARG
+    assert L.kvq_window_append(ctypes.byref(cfg), p, p, p, 0, 1, p, p, 100, None, p, 8, 1, p,
+                               None) == kvq.ERR_ARG
+    assert L.kvq_decode_attn_window(ctypes.byref(cfg), p, p, p, None, p, 8, 1, 100, p, 0, 8, p,
+                                    p, 1 << 30, p, None) == kvq.ERR_ARG
+    # workspace too small (the records come on top of the decode workspace)
+    assert L.kvq_decode_attn_window(ctypes.byref(cfg), p, p, p, p, p, 8, 1, 100, p, 0, 8, p, p,
+                                    kvq.decode_workspace_bytes(cfg, 1, 8, 100), p,
+                                    None) == kvq.ERR_WORKSPACE
+
+
 def test_argument_errors_without_gpu():
     L = kvq.lib()
     bad = kvq.make_cfg(2, 3, 3, head_dim=64)
