@@ -29,7 +29,10 @@
 //   width form a class compiled for its W. B = the query group times a_hat_j,
 //   log2(e), 1/sqrt(128), scaled by 2^sigma per head and split hi + lo fp16.
 // * Softmax: base-2 online softmax per head on the fp32 accumulators, scaled
-//   by the fp16 key norms; positions past the sequence length masked.
+//   by the fp16 key norms; positions past the sequence length masked. The
+//   reference of a head moves only when a score passes it (then to the
+//   tile's maximum plus a small headroom), so most tiles skip the maximum
+//   reduction and the rescaling of o.
 // * Values: P' = p * n^V (fp16) moves from the accumulator layout to the B
 //   operand with movmatrix; O^T(128 x G) += Vhat^T(128 x 16 tokens) P'^T with
 //   A registers holding one rotated coordinate of two tokens.
@@ -78,6 +81,7 @@ constexpr size_t kPairBlockBytes =
 static_assert(kPairBlockBytes % 128 == 0, "pair blocks keep the buckets 16-byte aligned");
 constexpr int kFallbackSlots = 1024;                  // CTA slots when no device answers
 constexpr int kMaxNew = 64;                           // tokens appended by a fused call
+constexpr float kHeadroom = 2.f;  // base-2 margin of a moved softmax reference
 constexpr int kScratch = 16640;  // q' staging; append: kz [32][129] fp32 + 64 fp16 norms
 
 struct DecodeParams {
@@ -97,6 +101,7 @@ struct DecodeParams {
   int64_t cap;
   int early;  // read lengths and stream tiles before waiting for the previous kernel
   int rope;   // appended keys are pre-RoPE: rotate each to its position first
+  long long stall_cycles;  // test hook (> 0): each warp first waits that long in vain
   double theta[64];
   uint8_t* pb_end;        // pair block of pair k at pb_end - (k + 1) * kPairBlockBytes
   float* part;            // [batch][n_kv][n_splits][G][132] = m, l, -, -, o[128]
@@ -112,6 +117,7 @@ struct alignas(128) Smem {
   float inv_scale[16];           // 2^-sigma of each head's q' scaling
   unsigned long long bar[kWarps][kStages];
   unsigned long long setup_bar;
+  unsigned long long stall_bar;  // nothing arrives on it (test hook of a wait that runs out)
   uint32_t cls_lane[8][32];      // per (class, lane): first K word << 8 | bit shift
   alignas(16) float thr[kThrPad];  // decision thresholds (fused append only)
   double theta[64];                // RoPE block frequencies (fused append of pre-RoPE keys)
@@ -310,6 +316,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   // ---- independent of earlier kernels: barriers, plan and lookup image
   if (tid == 0) {
     mbar_init(&sm.setup_bar, 1);
+    mbar_init(&sm.stall_bar, 1);
     for (int i = 0; i < kWarps * kStages; ++i) mbar_init(&sm.bar[i / kStages][i % kStages], 1);
     fence_proxy_async();
     const uint32_t thr_bytes = p.n_new > 0 ? (uint32_t)sizeof(g_thr) : 0u;
@@ -353,11 +360,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   const uint8_t* const cache0 = p.cm.table ? nullptr : p.cm.caches[b];  // contiguous base
   const int bk = sm.plan.bits_k;
   const int n_half = sm.plan.n_half;
-  const bool bad = !ok_setup || sm.plan.magic != KVQ_PLAN_MAGIC || sm.plan.bits_v != BV ||
-                   bk < 1 || bk > 8 || p.tile_bytes != tile_bytes(bk, BV) || n_half < 1 ||
-                   n_half > kMaxHalf || sm.plan.n_class < 1 || sm.plan.n_class > 8 ||
-                   sm.plan.n_ranks < 1 || sm.plan.n_ranks > 64 ||
-                   (reinterpret_cast<uintptr_t>(cache0) & 15) != 0;
+  bool bad = !ok_setup || sm.plan.magic != KVQ_PLAN_MAGIC || sm.plan.bits_v != BV ||
+             bk < 1 || bk > 8 || p.tile_bytes != tile_bytes(bk, BV) || n_half < 1 ||
+             n_half > kMaxHalf || sm.plan.n_class < 1 || sm.plan.n_class > 8 ||
+             sm.plan.n_ranks < 1 || sm.plan.n_ranks > 64 ||
+             (reinterpret_cast<uintptr_t>(cache0) & 15) != 0;
+  // width classes: every word a class reads must lie in the tile's key words
+  // plus the one half step of overrun a partial last half step allows
+  for (int ci = 0; !bad && ci < sm.plan.n_class; ++ci) {
+    const int W = sm.plan.cls_w[ci], hs0 = sm.plan.cls_hs0[ci], nhs = sm.plan.cls_nhs[ci];
+    bad = W < 1 || W > 8 || nhs < 1 || hs0 + nhs > n_half ||
+          sm.plan.cls_seg0[ci] + 8 * W * nhs > 128 * bk + 64;
+  }
   if (bad && tid == 0) atomicOr(p.status, ok_setup ? KVQ_FLAG_BAD_PLAN : KVQ_FLAG_TIMEOUT);
   const int len0 = sm.len0;
   int n_add = 0;
@@ -579,7 +593,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
     const int v_off = 4 * (g * BV + ((BV * c) >> 2));  // row g of each m-tile, lane's slots
     int consumed = 0;
     bool timed_out = false;
-    for (int i = 0; i < n_mine; ++i) {
+    if (p.stall_cycles > 0)  // test hook: a wait that runs out, then the timeout path
+      timed_out = !__all_sync(0xffffffffu, mbar_wait_bounded(&sm.stall_bar, 0u, p.stall_cycles));
+    for (int i = 0; i < n_mine && !timed_out; ++i) {
       const int s = i % kStages;
       const bool ok = mbar_wait_bounded(&sm.bar[warp][s], (uint32_t)((i / kStages) & 1));
       if (!__all_sync(0xffffffffu, ok)) {
@@ -613,46 +629,61 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
         nk[r] = val[r] ? __half2float(nrm[tok]) : 0.f;
         nv[r] = val[r] ? __half2float(nrm[kTile + tok]) : 0.f;
       }
+      // scores in base 2; a head's reference m_run only moves when a score
+      // passes it (lazy rescaling, warp-uniform test), and then to the
+      // tile's maximum plus kHeadroom, so 2^(s - m_run) <= 1 always and most
+      // tiles skip the maximum reduction and the rescale of o
+      float sv[NT][2][4];
+      bool up = false;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float isc = sm.inv_scale[8 * nt + 2 * c + e];
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const int mt = r >> 1, rr = r & 1;
+            sv[nt][e][r] = val[r] ? sacc[mt][nt][2 * rr + e] * (nk[r] * isc) : -INFINITY;
+            up |= sv[nt][e][r] > m_run[nt][e];
+          }
+        }
+      if (__any_sync(0xffffffffu, up)) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            float mx = fmaxf(fmaxf(sv[nt][e][0], sv[nt][e][1]), fmaxf(sv[nt][e][2], sv[nt][e][3]));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            if (mx > m_run[nt][e]) {
+              const float m_new = mx + kHeadroom;
+              const float alpha = ex2(m_run[nt][e] - m_new);  // 0 from -inf
+              l_run[nt][e] *= alpha;
+#pragma unroll
+              for (int mu = 0; mu < 8; ++mu) {
+                o[mu][nt][e] *= alpha;
+                o[mu][nt][2 + e] *= alpha;
+              }
+              m_run[nt][e] = m_new;
+            }
+          }
+      }
       uint32_t pb0[2][NT], pb1[2][NT];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         float pe[2][4];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const float isc = sm.inv_scale[8 * nt + 2 * c + e];
-          float sv[4];
+          // m_run is finite here: every processed tile holds a valid token
+          float lsum = 0.f;
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
-            const int mt = r >> 1, rr = r & 1;
-            sv[r] = val[r] ? sacc[mt][nt][2 * rr + e] * (nk[r] * isc) : -INFINITY;
+            const float pr = ex2(sv[nt][e][r] - m_run[nt][e]);  // 0 for masked tokens
+            lsum += pr;
+            pe[e][r] = pr * nv[r];
           }
-          float mx = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-          const float m_new = fmaxf(m_run[nt][e], mx);
-          float alpha = 1.f, lsum = 0.f;
-          if (m_new != -INFINITY) {
-            alpha = ex2(m_run[nt][e] - m_new);
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-              const float pr = ex2(sv[r] - m_new);
-              lsum += pr;
-              pe[e][r] = pr * nv[r];
-            }
-          } else {
-#pragma unroll
-            for (int r = 0; r < 4; ++r) pe[e][r] = 0.f;
-          }
-          l_run[nt][e] = l_run[nt][e] * alpha + lsum;
-          m_run[nt][e] = m_new;
-          if (alpha != 1.f) {
-#pragma unroll
-            for (int mu = 0; mu < 8; ++mu) {
-              o[mu][nt][e] *= alpha;
-              o[mu][nt][2 + e] *= alpha;
-            }
-          }
+          l_run[nt][e] += lsum;
         }
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt) {
@@ -1037,6 +1068,12 @@ static cudaError_t launch_decode_nt(const DecodeParams& p, int bits_v, int batch
 // ws: >= decode_workspace_bytes_for(...) bytes, zero-filled before its first
 // use; every completed call leaves its pair blocks (at the end of ws) zero.
 // n_new > 0 fuses the append of k_new / v_new ([batch][n_new][n_kv][128]).
+// Test hook: > 0 makes every later decode launch wait that many cycles on a
+// barrier nothing arrives on before its tiles (the wait runs out, the launch
+// flags TIMEOUT and skips its tiles).
+static std::atomic<long long> g_stall_cycles{0};
+void set_decode_stall(long long cycles) { g_stall_cycles.store(cycles > 0 ? cycles : 0); }
+
 cudaError_t launch_decode(const Plan* const* plans, const CacheMap& cm, int32_t* len,
                           int batch, int64_t max_len, const void* q, int q_dtype, int n_q, int n_kv,
                           int bits_k, int bits_v, float* out, void* ws, size_t ws_bytes,
@@ -1069,6 +1106,7 @@ cudaError_t launch_decode(const Plan* const* plans, const CacheMap& cm, int32_t*
   p.n_new = n_new;
   p.cap = cap;
   p.early = early;
+  p.stall_cycles = g_stall_cycles.load();
   p.rope = theta ? 1 : 0;
   for (int j = 0; j < 64; ++j) p.theta[j] = theta ? theta[j] : 0.0;
   p.part = reinterpret_cast<float*>(ws);
