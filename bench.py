@@ -70,6 +70,12 @@ def parse():
                     help="skip the timed oracle sample (sweep points)")
     ap.add_argument("--no-bf16", action="store_true",
                     help="skip the bf16 comparator (dense decode over an unquantized cache)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other workloads (llama8b layer, qwen7b serving step, context "
+                         "sweep with greedy and uniform plans, 512K x 36-layer prefill)")
+    ap.add_argument("--dist-steps", type=int, default=0,
+                    help="replays timed one by one for the step-time distribution "
+                         "(default: >= 100 and >= 1 s)")
     return ap.parse_args()
 
 
@@ -182,10 +188,29 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- CPU oracle
-def oracle_sample(wl, seconds_target=12.0, seed=0):
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def oracle_sample(wl, seconds_target=12.0, seed=0, threads=None):
     """Time the oracle's decode (unpack + dequantize + exact attention) on a
     bounded sample: one layer, one KV head and its G query heads, over
-    contexts of 8K tokens, repeated until ~seconds_target of CPU work."""
+    contexts of 8K tokens, repeated until ~seconds_target of CPU work.
+    threads: BLAS threads (None: as the process has them)."""
+    if threads is not None:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=threads):
+            r = oracle_sample(wl, seconds_target, seed, None)
+        r["cores"] = threads
+        return r
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     import oracle_pipeline as op  # noqa: F401
     from oracle import alloc, attn, energy, layout, quant
@@ -219,7 +244,15 @@ def oracle_sample(wl, seconds_target=12.0, seed=0):
     return {"value": bytes_done / el / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
             "sample": f"{reps} x (1 layer, 1 KV head + {G} query heads, {T} tokens, "
                       f"K{wl.bits_k}V{wl.bits_v}): unpack + dequantize + exact fp64 attention",
-            "seconds": el}
+            "seconds": el, "cpu_model": cpu_model(), "host_cpus": os.cpu_count()}
+
+
+def cpu_baselines(wl, seed):
+    """The oracle on all host cores (the line's cpu_baseline) and on one core."""
+    allc = oracle_sample(wl, seconds_target=8.0, seed=seed)
+    one = oracle_sample(wl, seconds_target=8.0, seed=seed, threads=1)
+    allc["one_core"] = {k: one[k] for k in ("value", "unit", "cores", "sample", "seconds")}
+    return allc
 
 
 # --------------------------------------------------------------- main paths
@@ -250,34 +283,24 @@ def run_reference(args, wl, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def run_kvq(args, wl, rank, world, dist):
+def build_stack(args, wl, T, n_layers, cfg, cap, rank, dev, dense, paged=0):
+    """Per layer: energies + greedy (or uniform) plans from the layer's own
+    keys and the bulk quantize-append of its T tokens (timed with events);
+    optionally the same keys / values as a bf16 cache for the comparator
+    ([batch][n_kv][cap][128] per layer). Returns the layers, the dense
+    caches, the seconds of plan building and of quantize-append."""
     import torch
 
-    from bit_kv_cache_19_b200 import kvq
     from bit_kv_cache_19_b200.runtime import PackedLayer, PagedLayer
 
-    dev = torch.device("cuda", torch.cuda.current_device())
-    n_layers, B, T = args.layers or wl.n_layers, wl.batch, args.context or wl.context
-    steps, warmup = args.steps, args.warmup
-    n_step = max(1, wl.n_new)  # tokens appended per sequence and layer in a step
-    cap = T + (steps + warmup + max(3, steps // 2) + 4) * n_step + 64
-    mode = kvq.ALLOC_UNIFORM if args.alloc == "uniform" else kvq.ALLOC_GREEDY
-    if args.rotate_keys:
-        mode |= kvq.ALLOC_ROTATE_KEYS
-    cfg = kvq.make_cfg(wl.n_kv_heads, wl.bits_k, wl.bits_v, v_seed=1234, alloc_mode=mode)
-    bpth = BYTES_PER_TOKEN_HEAD(wl.bits_k, wl.bits_v)
-
-    # ---- prefill: energies + greedy plans, bulk quantize-append (timed);
-    #      the same keys / values also fill the bf16 comparator's caches
-    #      ([batch][n_kv][cap][128] per layer)
-    layers = []
-    dense_k, dense_v = [], []
+    B = wl.batch
+    layers, dense_k, dense_v = [], [], []
     t_alloc = t_quant = 0.0
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for li in range(n_layers):
-        if args.paged:
-            per_seq = -(-cap // (32 * args.paged))
-            L = PagedLayer(cfg, B, B * per_seq, args.paged, per_seq, device=dev, layer=li)
+        if paged:
+            per_seq = -(-cap // (32 * paged))
+            L = PagedLayer(cfg, B, B * per_seq, paged, per_seq, device=dev, layer=li)
             order = [int(x) for x in np.random.default_rng(li).permutation(B * per_seq)]
             for b in range(B):
                 L.reserve(b, cap, order=order)
@@ -295,7 +318,7 @@ def run_kvq(args, wl, rank, world, dist):
         kall = torch.stack(ks)
         vall = torch.stack(vs)
         del ks, vs
-        if not args.no_bf16:
+        if dense:
             dk = torch.zeros(B, wl.n_kv_heads, cap, 128, dtype=torch.bfloat16, device=dev)
             dv = torch.zeros_like(dk)
             dk[:, :, :T].copy_(kall.permute(0, 2, 1, 3))
@@ -311,11 +334,16 @@ def run_kvq(args, wl, rank, world, dist):
         del kall, vall
         layers.append(L)
     torch.cuda.empty_cache()
+    return layers, dense_k, dense_v, t_alloc, t_quant
 
-    # ---- decode inputs (device resident) and static new-token buffers
-    # the step's inputs (q, new k, new v of every layer) live in one device
-    # buffer and its outputs in another, so that an end-to-end step moves
-    # them with one host-to-device and one device-to-host copy
+
+def step_buffers(wl, n_layers, n_step, T, seed, dev):
+    """The step's inputs (q, new k, new v of every layer) in one device
+    buffer and its outputs in another, so that an end-to-end step moves them
+    with one host-to-device and one device-to-host copy."""
+    import torch
+
+    B = wl.batch
     nq_el, nkv_el = B * wl.n_q_heads * 128, B * n_step * wl.n_kv_heads * 128
     per_layer = nq_el + 2 * nkv_el
     step_in = torch.empty(n_layers * per_layer, dtype=torch.bfloat16, device=dev)
@@ -326,17 +354,67 @@ def run_kvq(args, wl, rank, world, dist):
         q = step_in[base:base + nq_el].view(B, wl.n_q_heads, 128)
         k = step_in[base + nq_el:base + nq_el + nkv_el].view(B, n_step, wl.n_kv_heads, 128)
         v = step_in[base + nq_el + nkv_el:base + per_layer].view(B, n_step, wl.n_kv_heads, 128)
-        q.copy_(synth.queries_torch(wl, args.seed, li, B, T, dev))
+        q.copy_(synth.queries_torch(wl, seed, li, B, T, dev))
         k.copy_(torch.randn(B, n_step, wl.n_kv_heads, 128, device=dev).to(torch.bfloat16))
         v.copy_(torch.randn(B, n_step, wl.n_kv_heads, 128, device=dev).to(torch.bfloat16))
         qs.append(q)
         knew.append(k)
         vnew.append(v)
-    outs = [step_out[li] for li in range(n_layers)]
-    ws = layers[0].workspace(wl.n_q_heads, cap)
+    return step_in, step_out, qs, knew, vnew
 
+
+def time_replays(run, stream, steps, flush):
+    """Mean ms of `steps` runs on `stream`: two events around all of them, or,
+    with an L2 flush buffer, events around each run after its flush."""
+    import torch
+
+    if flush is None:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            run()
+        e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1) / steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for a, b_ in evs:
+        flush.add_(1)
+        a.record(stream)
+        run()
+        b_.record(stream)
+    stream.synchronize()
+    return sum(a.elapsed_time(b_) for a, b_ in evs) / steps
+
+
+def per_step_ms(run, stream, n, flush):
+    """Per-run ms of n runs, events around each (after the flush, if any)."""
+    import torch
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    for a, b_ in evs:
+        if flush is not None:
+            flush.add_(1)
+        a.record(stream)
+        run()
+        b_.record(stream)
+    stream.synchronize()
+    return [a.elapsed_time(b_) for a, b_ in evs]
+
+
+def percentiles(xs):
+    ys = sorted(xs)
+
+    def q(f):
+        return ys[min(len(ys) - 1, int(round(f * (len(ys) - 1))))]
+    return {"n": len(ys), "mean": statistics.mean(ys), "p10": q(0.1), "p50": q(0.5),
+            "p90": q(0.9), "min": ys[0], "max": ys[-1]}
+
+
+def fused_step_fn(kvq, args, cfg, layers, knew, vnew, qs, outs, ws, cap):
     def step():
-        # one launch per layer: quantize-append the new token, then decode
+        # one launch per layer: quantize-append the new token(s), then decode
         for li, L in enumerate(layers):
             if args.paged:
                 kvq.paged_append_decode(cfg, L.plan_ptrs, knew[li], vnew[li], L.pages, L.lens,
@@ -344,6 +422,36 @@ def run_kvq(args, wl, rank, world, dist):
             else:
                 kvq.append_decode(cfg, L.plan_ptrs, knew[li], vnew[li], L.cache_ptrs, L.lens,
                                   cap, cap, qs[li], outs[li], ws, L.status, kvq.STEP_EARLY)
+    return step
+
+
+def run_kvq(args, wl, rank, world, dist):
+    import torch
+
+    from bit_kv_cache_19_b200 import kvq
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    n_layers, B, T = args.layers or wl.n_layers, wl.batch, args.context or wl.context
+    steps, warmup = args.steps, args.warmup
+    n_step = max(1, wl.n_new)  # tokens appended per sequence and layer in a step
+    n_dist = args.dist_steps
+    n_dist_max = max(n_dist, 4000)
+    cap = T + (steps + warmup + max(3, steps // 2) + 4 + n_dist_max) * n_step + 64
+    mode = kvq.ALLOC_UNIFORM if args.alloc == "uniform" else kvq.ALLOC_GREEDY
+    if args.rotate_keys:
+        mode |= kvq.ALLOC_ROTATE_KEYS
+    cfg = kvq.make_cfg(wl.n_kv_heads, wl.bits_k, wl.bits_v, v_seed=1234, alloc_mode=mode)
+    bpth = BYTES_PER_TOKEN_HEAD(wl.bits_k, wl.bits_v)
+
+    # ---- prefill: energies + greedy plans, bulk quantize-append (timed)
+    layers, dense_k, dense_v, t_alloc, t_quant = build_stack(
+        args, wl, T, n_layers, cfg, cap, rank, dev, dense=not args.no_bf16, paged=args.paged)
+
+    # ---- decode inputs (device resident) and static new-token buffers
+    step_in, step_out, qs, knew, vnew = step_buffers(wl, n_layers, n_step, T, args.seed, dev)
+    outs = [step_out[li] for li in range(n_layers)]
+    ws = layers[0].workspace(wl.n_q_heads, cap)
+    step = fused_step_fn(kvq, args, cfg, layers, knew, vnew, qs, outs, ws, cap)
 
     stream = torch.cuda.Stream(device=dev)
     graph = None
@@ -355,6 +463,10 @@ def run_kvq(args, wl, rank, world, dist):
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph, stream=stream):
                 step()
+
+        def run():
+            graph.replay() if graph is not None else step()
+
         len_before = int(layers[0].lens[0].item())
         l2 = torch.cuda.get_device_properties(dev).L2_cache_size
         stack_bytes = n_layers * B * wl.n_kv_heads * bpth * T
@@ -366,28 +478,17 @@ def run_kvq(args, wl, rank, world, dist):
         torch.cuda.synchronize()
         sampler.start()
         time.sleep(0.3)
-        if flush is None:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(steps):
-                graph.replay() if graph is not None else step()
-            e1.record(stream)
-            e1.synchronize()
-            ms = e0.elapsed_time(e1) / steps
-        else:  # caches within 4x L2: flush it before each step, time the steps only
-            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in range(steps)]
-            for a, b_ in evs:
-                flush.add_(1)
-                a.record(stream)
-                graph.replay() if graph is not None else step()
-                b_.record(stream)
-            stream.synchronize()
-            ms = sum(a.elapsed_time(b_) for a, b_ in evs) / steps
+        ms = time_replays(run, stream, steps, flush)
+        torch.cuda.synchronize()
+        # the step-time distribution: >= 100 replays and >= 2 s (at most
+        # 4000), one by one (events between replays), inside the same clock
+        # record
+        n_d = n_dist or min(n_dist_max, max(100, int(2000.0 / max(ms, 1e-3)) + 1))
+        dist_ms = per_step_ms(run, stream, n_d, flush)
         torch.cuda.synchronize()
         clocks = sampler.stop()
     ms = rank_max(ms, dist, dev)
-    # packed bytes read per step: length grows by 1 per step
+    # packed bytes read per step: length grows by n_step per step
     lens_timed = [len_before + (i + 1) * n_step for i in range(steps)]
     bytes_step = n_layers * B * wl.n_kv_heads * bpth * statistics.mean(lens_timed)
     flags = 0
@@ -395,9 +496,14 @@ def run_kvq(args, wl, rank, world, dist):
         flags |= L.flags()
     assert flags == 0, f"status flags {flags}"
     value = job_rate(bytes_step, world, ms) / 1e9
+    stats = percentiles(dist_ms)
+    stats["unit"] = "ms per step"
+    stats["note"] = ("the step replayed one by one after the timed region (events around each, "
+                     "same clock record); the line's ms_per_step is the timed region's mean")
 
     # ---- bf16 comparator: the same decode over the unquantized caches (one
     #      dense launch per layer, lengths as in the packed step, graph)
+    peak, peak_kind = measured_peaks()
     bf16 = None
     if not args.no_bf16:
         dlen = torch.full((B,), int(layers[0].lens[0].item()), dtype=torch.int32, device=dev)
@@ -422,20 +528,22 @@ def run_kvq(args, wl, rank, world, dist):
                 dgraph = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(dgraph, stream=stream):
                     dense_step()
-            d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            d0.record(stream)
-            for _ in range(steps):
-                dgraph.replay() if dgraph is not None else dense_step()
-            d1.record(stream)
-            d1.synchronize()
-            dms = d0.elapsed_time(d1) / steps
+            dms = time_replays(lambda: dgraph.replay() if dgraph is not None else dense_step(),
+                               stream, steps, None)
         dms = rank_max(dms, dist, dev)
         assert int(dstatus.item()) == 0, "bf16 comparator status"
         dbytes = n_layers * B * wl.n_kv_heads * 512 * int(dlen[0].item())
+        dense_floor_ms = dbytes / (peak * 1e9) * 1e3
         bf16 = {"kernel": "dense_decode_kernel (kvq_bf16_decode_attn, one launch per layer)",
                 "ms_per_step": dms, "value": job_rate(dbytes, world, dms) / 1e9, "unit": "GB/s",
+                "frac": dbytes / (dms / 1e3) / 1e9 / peak,
                 "bytes_per_step": dbytes, "cache_bytes": "512 B per token-head (bf16 K + V)",
-                "packed_step_speedup": dms / ms, "note": "decode only (no append)"}
+                "packed_step_speedup": dms / ms,
+                "dense_step_at_copy_bw_ms": dense_floor_ms,
+                "packed_step_speedup_vs_dense_at_copy_bw": dense_floor_ms / ms,
+                "note": "decode only (no append); dense_step_at_copy_bw_ms = the bf16 cache "
+                        "bytes at the measured copy bandwidth, the time any dense decode of "
+                        "this step needs at least"}
         del dense_k, dense_v
         torch.cuda.empty_cache()
 
@@ -463,7 +571,6 @@ def run_kvq(args, wl, rank, world, dist):
     # (consecutive launches overlap by their prologue and merge tail)
     launch_ms = ms / n_layers
     bytes_launch = bytes_step / n_layers
-    peak, peak_kind = measured_peaks()
     achieved = bytes_launch / (launch_ms / 1e3) / 1e9
 
     # ---- e2e: host buffers, H2D of the step's inputs and D2H of its outputs
@@ -493,10 +600,20 @@ def run_kvq(args, wl, rank, world, dist):
     e2e_bytes = n_layers * B * wl.n_kv_heads * bpth * (e2e_len - n_step * (e2e_steps - 1) / 2)
     e2e_ms = rank_max(e2e_ms, dist, dev)
     e2e_val = job_rate(e2e_bytes, world, e2e_ms) / 1e9
+    graph = None
+    del layers, step_in, step_out, qs, knew, vnew, outs, ws
+    torch.cuda.empty_cache()
+
+    # ---- the other workloads (1 GPU, default workload only)
+    extras = None
+    if world == 1 and not args.no_extras and wl.name == "qwen3b_128k" and not args.layers \
+            and not args.context and not args.paged and args.alloc == "greedy" \
+            and not args.rotate_keys:
+        extras = run_extras(args, rank, dev, stream, peak)
 
     if rank != 0:
         return
-    cpu = (oracle_sample(wl, seconds_target=12.0, seed=args.seed)
+    cpu = (cpu_baselines(wl, seed=args.seed)
            if world == 1 and not args.no_cpu_baseline else None)
     n_tok_quant = n_layers * B * T
     line = {
@@ -520,9 +637,10 @@ def run_kvq(args, wl, rank, world, dist):
                           if flush is None else
                           f"L2 flushed before each timed step ({n_layers}-layer packed cache "
                           f"{stack_bytes / 1e6:.0f} MB < 4x L2)"),
-                   "graph": graph is not None},
+                   "graph": not args.no_graph},
         "pct_of_8TBs": value / 8000.0 * 100,
         "tokens_per_s": job_rate(B, world, ms),
+        "step_ms": stats,
         "quantize_prefill": {"layer_tokens_per_s": n_tok_quant / t_quant,
                              "token_heads_per_s": n_tok_quant * wl.n_kv_heads / t_quant,
                              "seconds": t_quant, "alloc_bits_seconds": t_alloc},
@@ -538,10 +656,108 @@ def run_kvq(args, wl, rank, world, dist):
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "bf16_comparator": bf16,
+        "workloads": extras,
         "gpu_launches": steps * n_layers,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
+
+
+def measure_point(args, wl, T, alloc, n_layers, rank, dev, stream, peak, steps):
+    """One workload point: build its stack (plans from its own keys, bulk
+    quantize-append, timed), then time `steps` graph replays of its fused
+    step (append n_new + decode per layer; L2 flushed before each step when
+    the stack is within 4x L2). Returns the point's numbers."""
+    import torch
+
+    from bit_kv_cache_19_b200 import kvq
+
+    B = wl.batch
+    n_step = max(1, wl.n_new)
+    warmup = 3
+    cap = T + (steps + warmup + 2) * n_step + 64
+    mode = kvq.ALLOC_UNIFORM if alloc == "uniform" else kvq.ALLOC_GREEDY
+    cfg = kvq.make_cfg(wl.n_kv_heads, wl.bits_k, wl.bits_v, v_seed=1234, alloc_mode=mode)
+    bpth = BYTES_PER_TOKEN_HEAD(wl.bits_k, wl.bits_v)
+    layers, _, _, _, t_quant = build_stack(args, wl, T, n_layers, cfg, cap, rank, dev, False)
+    _, _, qs, knew, vnew = step_buffers(wl, n_layers, n_step, T, args.seed, dev)
+    outs = [torch.empty(B, wl.n_q_heads, 128, dtype=torch.float32, device=dev)
+            for _ in range(n_layers)]
+    ws = layers[0].workspace(wl.n_q_heads, cap)
+
+    class _A:
+        paged = 0
+    step = fused_step_fn(kvq, _A, cfg, layers, knew, vnew, qs, outs, ws, cap)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            step()
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        len_before = int(layers[0].lens[0].item())
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        stack_bytes = n_layers * B * wl.n_kv_heads * bpth * T
+        flush = (torch.zeros(2 * l2 // 4, dtype=torch.int32, device=dev)
+                 if stack_bytes < 4 * l2 else None)
+        ms = time_replays(graph.replay, stream, steps, flush)
+        torch.cuda.synchronize()
+    flags = 0
+    for L in layers:
+        flags |= L.flags()
+    assert flags == 0, f"{wl.name} {T} {alloc}: status flags {flags}"
+    mean_len = len_before + n_step * (steps + 1) / 2
+    bytes_step = n_layers * B * wl.n_kv_heads * bpth * mean_len
+    gbs = bytes_step / (ms / 1e3) / 1e9
+    out = {"layers": n_layers, "batch": B, "context": T, "q_heads": wl.n_q_heads,
+           "kv_heads": wl.n_kv_heads, "budget": f"K{wl.bits_k}V{wl.bits_v}", "alloc": alloc,
+           "appended_per_step": n_step, "steps": steps, "ms_per_step": ms,
+           "launch_us": ms / n_layers * 1e3, "GB_per_s": gbs, "frac": gbs / peak,
+           "tokens_per_s": B / (ms / 1e3),
+           "l2": ("stack larger than 4x L2" if flush is None else "L2 flushed before each step"),
+           "prefill_seconds": t_quant,
+           "prefill_token_heads_per_s": n_layers * B * T * wl.n_kv_heads / t_quant}
+    graph = None
+    del layers, qs, knew, vnew, outs, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_extras(args, rank, dev, stream, peak):
+    """The other workloads of the build: one Llama-3.1-8B-shaped layer at 32K
+    (K2V2), the 7B-Qwen-shaped serving step (16 x 32K, append 16 + decode,
+    28 layers, K3V2), the Qwen2.5-3B-shaped context sweep 8K..512K with
+    Block-GTQ (greedy) and uniform plans of the same bytes, and the bulk
+    prefill of 512K tokens x 36 layers (its roofline: bf16 K/V in plus the
+    packed bytes out at the measured copy bandwidth)."""
+    steps = 20
+    out = {}
+    W = synth.WORKLOADS
+    t0 = time.perf_counter()
+    out["llama8b"] = measure_point(args, W["llama8b"], W["llama8b"].context, "greedy", 1, rank,
+                                   dev, stream, peak, steps)
+    sv = W["qwen7b_serve"]
+    out["qwen7b_serve"] = measure_point(args, sv, sv.context, "greedy", sv.n_layers, rank, dev,
+                                        stream, peak, steps)
+    sw = W["qwen3b_sweep"]
+    sweep = []
+    for T in sw.contexts:
+        for alloc in ("greedy", "uniform"):
+            sweep.append(measure_point(args, sw, T, alloc, sw.n_layers, rank, dev, stream, peak,
+                                       steps))
+    out["qwen3b_sweep"] = sweep
+    big = [p for p in sweep if p["context"] == max(sw.contexts) and p["alloc"] == "greedy"][0]
+    tok_heads = big["layers"] * big["context"] * sw.n_kv_heads
+    moved = tok_heads * (512 + BYTES_PER_TOKEN_HEAD(sw.bits_k, sw.bits_v))
+    floor_s = moved / (peak * 1e9)
+    out["prefill_512k_x36"] = {"seconds": big["prefill_seconds"],
+                               "token_heads_per_s": big["prefill_token_heads_per_s"],
+                               "bytes_moved": moved, "roofline_seconds": floor_s,
+                               "frac": floor_s / big["prefill_seconds"],
+                               "note": "bulk quantize-append, one launch per layer; bytes = "
+                                       "bf16 K + V in + packed codes and norms out"}
+    out["seconds"] = time.perf_counter() - t0
+    return out
 
 
 def issue_roofline(workload, launch_ms, clocks):
