@@ -387,13 +387,16 @@ def time_replays(run, stream, steps, flush):
     return sum(a.elapsed_time(b_) for a, b_ in evs) / steps
 
 
-def per_step_ms(run, stream, n, flush):
-    """Per-run ms of n runs, events around each (after the flush, if any)."""
+def per_step_ms(run, stream, n, flush, reset=None, every=0):
+    """Per-run ms of n runs, events around each (after the flush, if any);
+    reset() (outside the events) before every `every` runs."""
     import torch
 
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(n)]
-    for a, b_ in evs:
+    for i, (a, b_) in enumerate(evs):
+        if reset is not None and every and i % every == 0:
+            reset()
         if flush is not None:
             flush.add_(1)
         a.record(stream)
@@ -436,7 +439,7 @@ def run_kvq(args, wl, rank, world, dist):
     n_step = max(1, wl.n_new)  # tokens appended per sequence and layer in a step
     n_dist = args.dist_steps
     n_dist_max = max(n_dist, 4000)
-    cap = T + (steps + warmup + max(3, steps // 2) + 4 + n_dist_max) * n_step + 64
+    cap = T + (steps + warmup + max(3, steps // 2) + 4) * n_step + 64
     mode = kvq.ALLOC_UNIFORM if args.alloc == "uniform" else kvq.ALLOC_GREEDY
     if args.rotate_keys:
         mode |= kvq.ALLOC_ROTATE_KEYS
@@ -482,9 +485,18 @@ def run_kvq(args, wl, rank, world, dist):
         torch.cuda.synchronize()
         # the step-time distribution: >= 100 replays and >= 2 s (at most
         # 4000), one by one (events between replays), inside the same clock
-        # record
+        # record; every `steps` replays the lengths go back to where the
+        # timed region started, so the same lengths are replayed
         n_d = n_dist or min(n_dist_max, max(100, int(2000.0 / max(ms, 1e-3)) + 1))
-        dist_ms = per_step_ms(run, stream, n_d, flush)
+        lens_end = [L.lens.clone() for L in layers]
+        lens_start = [l1 - steps * n_step for l1 in lens_end]
+
+        def reset_lens():
+            for L, l0 in zip(layers, lens_start):
+                L.lens.copy_(l0)
+        dist_ms = per_step_ms(run, stream, n_d, flush, reset_lens, steps)
+        for L, l1 in zip(layers, lens_end):  # where the timed region ended
+            L.lens.copy_(l1)
         torch.cuda.synchronize()
         clocks = sampler.stop()
     ms = rank_max(ms, dist, dev)
