@@ -142,12 +142,111 @@ __device__ __forceinline__ int token_source(const QuantParams& p, const Item& it
   return p.dtype;
 }
 
+// Element i of a row of the input type DT (KVQ_BF16 / FP16 / FP32) as fp32.
+template <int DT>
+__device__ __forceinline__ float in_elem(const void* base, size_t i) {
+  if constexpr (DT == KVQ_BF16) return __bfloat162float(static_cast<const __nv_bfloat16*>(base)[i]);
+  else if constexpr (DT == KVQ_FP16) return __half2float(static_cast<const __half*>(base)[i]);
+  else return static_cast<const float*>(base)[i];
+}
+
+// Code of a width-W value from the thresholds held in registers (W <= 3):
+// the same binary search as code_of_w, its steps resolved by selects.
+template <int W>
+__device__ __forceinline__ uint32_t code_of_reg(const float (&t)[7], float z) {
+  if constexpr (W == 1) {
+    return t[0] < z ? 1u : 0u;
+  } else if constexpr (W == 2) {
+    const uint32_t c = t[1] < z ? 2u : 0u;
+    return c + ((c ? t[2] : t[0]) < z ? 1u : 0u);
+  } else {
+    const uint32_t c2 = t[3] < z ? 4u : 0u;
+    const uint32_t c1 = (c2 ? t[5] : t[1]) < z ? 2u : 0u;
+    const float tl = c2 ? (c1 ? t[6] : t[4]) : (c1 ? t[2] : t[0]);
+    return c2 + c1 + (tl < z ? 1u : 0u);
+  }
+}
+
+// Pass 1 of the bulk path for one token (one warp), input type DT known at
+// compile time: the arithmetic and decisions of warp_token_pass (fixed
+// sum-of-squares tree, IEEE norm and reciprocal, the same butterfly graph),
+// with the lane's value signs precomputed (bit q: coordinate lane + 32 q)
+// and, for value widths <= 3, the thresholds in registers.
+template <int BV, int DT>
+__device__ __forceinline__ void bulk_token_pass(const Plan& pl, const float* thr,
+                                                const float (&tv)[7], uint32_t vsgn,
+                                                const void* k, const void* v, size_t row,
+                                                int lane, int p, float* kz_row, uint32_t* words,
+                                                bool clear, __half& kn, __half& vn,
+                                                uint32_t& flags) {
+  float kx[4], vx[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    kx[q] = in_elem<DT>(k, row + lane + 32 * q);
+    vx[q] = in_elem<DT>(v, row + lane + 32 * q);
+  }
+  const bool kfin = __all_sync(0xffffffffu, isfinite(kx[0]) && isfinite(kx[1]) &&
+                                                isfinite(kx[2]) && isfinite(kx[3]));
+  const bool vfin = __all_sync(0xffffffffu, isfinite(vx[0]) && isfinite(vx[1]) &&
+                                                isfinite(vx[2]) && isfinite(vx[3]));
+  float kr;
+  norm_and_recip(kx, kfin, kn, kr, flags);
+  const bool klive = kfin && __half2float(kn) > 0.f;
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    kz_row[lane + 32 * q] = klive ? __fmul_rn(kx[q], kr) : __int_as_float(0x7fc00000);
+  float vr;
+  norm_and_recip(vx, vfin, vn, vr, flags);
+  const bool vlive = vfin && __half2float(vn) > 0.f;
+  float y[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float x = vfin ? vx[q] : 0.f;
+    y[q] = ((vsgn >> q) & 1u) ? -x : x;
+  }
+#pragma unroll
+  for (int hh = 1; hh < 32; hh <<= 1) {
+    const float sg = (lane & hh) ? -1.f : 1.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) y[q] = __fmaf_rn(y[q], sg, __shfl_xor_sync(0xffffffffu, y[q], hh));
+  }
+  {
+    const float a0 = __fadd_rn(y[0], y[1]), a1 = __fsub_rn(y[0], y[1]);
+    const float a2 = __fadd_rn(y[2], y[3]), a3 = __fsub_rn(y[2], y[3]);
+    y[0] = __fadd_rn(a0, a2);
+    y[2] = __fsub_rn(a0, a2);
+    y[1] = __fadd_rn(a1, a3);
+    y[3] = __fsub_rn(a1, a3);
+  }
+  uint32_t* vwords = words + kHeadDim * pl.bits_k + ((slot_v(p) * BV) >> 5) + BV * lane;
+  const int off = (slot_v(p) * BV) & 31;
+  const bool spill = off + BV > 32;
+  constexpr uint32_t mask = (1u << BV) - 1u;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t* w = vwords + BV * 32 * q;
+    const float z = __fmul_rn(y[q], vr);
+    uint32_t c = 0u;
+    if (vlive) {
+      if constexpr (BV <= 3) c = code_of_reg<BV>(tv, z);
+      else c = (uint32_t)code_of_w<BV>(thr, z);
+    }
+    if (clear) atomicAnd(w, ~(mask << off));
+    atomicOr(w, c << off);
+    if (spill) {
+      if (clear) atomicAnd(w + 1, ~(mask >> (32 - off)));
+      atomicOr(w + 1, c >> (32 - off));
+    }
+  }
+}
+
 // CTAs loop over the work items. A tile's words are assembled in shared
 // memory (from zero for a fresh tile, else from the record) by the two passes
 // of quant_dev.cuh and written back whole. The plan is reloaded only when
 // (b, h) changes. WIN: a window append (rows from the ring or the new tokens,
-// token by token); otherwise every row comes from the new tokens.
-template <int BV, bool WIN>
+// token by token); otherwise every row comes from the new tokens, of input
+// type DT (-1: any, as p.dtype says; pre-RoPE keys take that path).
+template <int BV, bool WIN, int DT>
 __global__ void __launch_bounds__(256, 4) quantize_append_kernel(QuantParams p) {
   __shared__ Plan s_plan;
   __shared__ float s_thr[KVQ_CB_N_THR];
@@ -160,6 +259,10 @@ __global__ void __launch_bounds__(256, 4) quantize_append_kernel(QuantParams p) 
   for (int i = threadIdx.x; i < KVQ_CB_N_THR; i += blockDim.x) s_thr[i] = c_thr[i];
   for (int i = threadIdx.x; i < 64; i += blockDim.x) s_theta[i] = p.theta[i];
   if (threadIdx.x == 0) s_flags = 0;
+  float tv[7];  // value thresholds in registers (widths <= 3)
+#pragma unroll
+  for (int i = 0; i < 7; ++i) tv[i] = c_thr[cb_t_off(BV) + min(i, (1 << BV) - 2)];
+  uint32_t vsgn = 0;  // value signs of this lane's coordinates lane + 32 q
   int cur = -1;  // (b, h) whose plan is in shared memory
   bool plan_ok = false;
   const int n_items = p.batch * p.n_kv * p.tiles_max;
@@ -194,6 +297,9 @@ __global__ void __launch_bounds__(256, 4) quantize_append_kernel(QuantParams p) 
                 s_plan.n_ranks >= 1 && s_plan.n_ranks <= 64 && s_plan.n_class >= 1 &&
                 s_plan.n_class <= 8;
       if (plan_ok && s_plan.k_rot) rot_tables(s_plan, s_rot, threadIdx.x);
+      vsgn = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) vsgn |= ((s_plan.v_sign[q] >> lane) & 1u) << q;
       __syncthreads();
     }
     if (!plan_ok) {
@@ -222,9 +328,13 @@ __global__ void __launch_bounds__(256, 4) quantize_append_kernel(QuantParams p) 
       } else {
         const size_t row =
             (((size_t)b * p.n_new + (tile * kTile + pp - len0)) * p.n_kv + h) * kHeadDim;
-        warp_token_pass<BV>(pl, s_thr, p.k, p.v, p.dtype, row, lane, pp, s_kz + pp * kKzStride,
-                            s_words, clear, kn, vn, flags, p.rope ? s_theta : nullptr,
-                            (int64_t)tile * kTile + pp);
+        if constexpr (DT >= 0)
+          bulk_token_pass<BV, DT>(pl, s_thr, tv, vsgn, p.k, p.v, row, lane, pp,
+                                  s_kz + pp * kKzStride, s_words, clear, kn, vn, flags);
+        else
+          warp_token_pass<BV>(pl, s_thr, p.k, p.v, p.dtype, row, lane, pp, s_kz + pp * kKzStride,
+                              s_words, clear, kn, vn, flags, p.rope ? s_theta : nullptr,
+                              (int64_t)tile * kTile + pp);
       }
       if (lane == 0) {
         norms[pp] = kn;
@@ -272,8 +382,11 @@ cudaError_t launch_energy(const void* k, int dtype, int64_t n_tokens, int n_kv,
 
 template <int BV>
 static void launch_quant_t(const QuantParams& p, bool win, unsigned grid, cudaStream_t st) {
-  if (win) quantize_append_kernel<BV, true><<<grid, 256, 0, st>>>(p);
-  else quantize_append_kernel<BV, false><<<grid, 256, 0, st>>>(p);
+  if (win) quantize_append_kernel<BV, true, -1><<<grid, 256, 0, st>>>(p);
+  else if (p.rope) quantize_append_kernel<BV, false, -1><<<grid, 256, 0, st>>>(p);
+  else if (p.dtype == KVQ_BF16) quantize_append_kernel<BV, false, KVQ_BF16><<<grid, 256, 0, st>>>(p);
+  else if (p.dtype == KVQ_FP16) quantize_append_kernel<BV, false, KVQ_FP16><<<grid, 256, 0, st>>>(p);
+  else quantize_append_kernel<BV, false, KVQ_FP32><<<grid, 256, 0, st>>>(p);
 }
 
 cudaError_t launch_quantize_append(const QuantParams& p_in, int bits_v, cudaStream_t st) {
