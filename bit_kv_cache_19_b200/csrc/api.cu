@@ -32,6 +32,7 @@ cudaError_t launch_dense_decode(const void* k, const void* v, const int32_t* len
 cudaError_t launch_combine(const Plan* const* plans, const float* recs, int n_parts, int batch,
                            int n_q, int n_kv, float* out, cudaStream_t st);
 void set_decode_stall(long long cycles);
+void set_decode_deterministic(int on);
 cudaError_t launch_window_push(const void* k, const void* v, int dtype, int n_new, int n_kv,
                                int32_t* len, int32_t* wlen, float* const* wins, int R,
                                int64_t cap, int batch, cudaStream_t st);
@@ -625,6 +626,11 @@ int kvq_combine_partials(const kvq_cfg* cfg, const void* const* plans_dev, int n
 int kvq_debug_decode_stall(long long cycles) {
   if (cycles < 0 || cycles > (1ll << 40)) return fail(KVQ_ERR_ARG, "stall cycles %lld", cycles);
   set_decode_stall(cycles);
+  return KVQ_OK;
+}
+
+int kvq_set_decode_deterministic(int on) {
+  set_decode_deterministic(on);
   return KVQ_OK;
 }
 

@@ -44,7 +44,8 @@
 //   rotation (inverse Walsh-Hadamard, signs) and writes o / l. A split max
 //   outside [-256, 256) makes the last split merge all records instead. The
 //   sum order of the atomics varies, so outputs agree run to run to fp32
-//   rounding, not bit for bit.
+//   rounding, not bit for bit; a process-wide deterministic mode makes the
+//   last split merge all records in split order instead.
 #include <algorithm>
 #include <cstddef>
 #include <atomic>
@@ -102,6 +103,7 @@ struct DecodeParams {
   int early;  // read lengths and stream tiles before waiting for the previous kernel
   int rope;   // appended keys are pre-RoPE: rotate each to its position first
   long long stall_cycles;  // test hook (> 0): each warp first waits that long in vain
+  int deterministic;       // merge the split records in split order (no L2 atomics)
   double theta[64];
   uint8_t* pb_end;        // pair block of pair k at pb_end - (k + 1) * kPairBlockBytes
   float* part;            // [batch][n_kv][n_splits][G][132] = m, l, -, -, o[128]
@@ -771,7 +773,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
       my_part[hd * kPartStride] = m;
       my_part[hd * kPartStride + 1] = l;
     }
-    if (m == -INFINITY) continue;  // no tokens in this split
+    if (m == -INFINITY || p.deterministic) continue;  // no tokens, or merged in order
     const float kf = floorf(m * (1.f / 32.f));
     if (!(kf >= -8.f && kf < 8.f)) {
       if (x4 == 0) atomicOr(ovf, 1u);
@@ -823,7 +825,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
       msk[it] = __ldcg(bmask + hd);
     }
   }
-  if (ovf_v == 0u) {
+  if (ovf_v == 0u && !p.deterministic) {
 #pragma unroll
     for (int it = 0; it < kItems; ++it) {
       const int item = tid + it * kThreads;
@@ -1073,6 +1075,11 @@ static cudaError_t launch_decode_nt(const DecodeParams& p, int bits_v, int batch
 // flags TIMEOUT and skips its tiles).
 static std::atomic<long long> g_stall_cycles{0};
 void set_decode_stall(long long cycles) { g_stall_cycles.store(cycles > 0 ? cycles : 0); }
+// Deterministic mode: the last split merges every split record in split
+// order instead of summing exponent buckets filled by L2 atomics in arrival
+// order, so outputs repeat bit for bit (slower: one CTA reads all records).
+static std::atomic<int> g_deterministic{0};
+void set_decode_deterministic(int on) { g_deterministic.store(on ? 1 : 0); }
 
 cudaError_t launch_decode(const Plan* const* plans, const CacheMap& cm, int32_t* len,
                           int batch, int64_t max_len, const void* q, int q_dtype, int n_q, int n_kv,
@@ -1107,6 +1114,7 @@ cudaError_t launch_decode(const Plan* const* plans, const CacheMap& cm, int32_t*
   p.cap = cap;
   p.early = early;
   p.stall_cycles = g_stall_cycles.load();
+  p.deterministic = g_deterministic.load();
   p.rope = theta ? 1 : 0;
   for (int j = 0; j < 64; ++j) p.theta[j] = theta ? theta[j] : 0.0;
   p.part = reinterpret_cast<float*>(ws);

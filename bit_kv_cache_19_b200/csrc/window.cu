@@ -46,8 +46,9 @@ __global__ void __launch_bounds__(kWinThreads) window_push_kernel(
   if (j0 < n_new) {
     float* wk = wins[b];
     float* wv = wk + (size_t)R * n_kv * kHeadDim;
-    for (int e = threadIdx.x; e < (n_new - j0) * per_tok; e += kWinThreads) {
-      const int j = j0 + e / per_tok, x = e - (e / per_tok) * per_tok;
+    const int64_t n_el = (int64_t)(n_new - j0) * per_tok;
+    for (int64_t e = threadIdx.x; e < n_el; e += kWinThreads) {
+      const int j = j0 + (int)(e / per_tok), x = (int)(e % per_tok);
       const int slot = (int)(((int64_t)len0 + w0 + j) % R);
       const size_t src = ((size_t)b * n_new + j) * per_tok + x;
       wk[(size_t)slot * per_tok + x] = load_as_float(k, dtype, src);

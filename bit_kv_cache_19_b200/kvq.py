@@ -114,6 +114,7 @@ _SIGS = {
                                        ctypes.POINTER(Pages), _vp, _i32, _i64, _vp, _i32, _i32,
                                        _vp, _vp, _sz, _i32, ctypes.c_double, _vp, _vp]),
     "kvq_debug_decode_stall": (_i32, [ctypes.c_longlong]),
+    "kvq_set_decode_deterministic": (_i32, [_i32]),
     "kvq_window_bytes": (_sz, [ctypes.POINTER(Cfg), _i32]),
     "kvq_window_append": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i32, _vp, _vp, _i64,
                                  _vp, _vp, _i32, _i32, _vp, _vp]),

@@ -28,7 +28,10 @@
  *   - Supported shapes: head_dim = 128; bits_k and bits_v in 1..8; b_max = 8;
  *     n_q_heads a multiple of n_kv_heads with G = n_q_heads / n_kv_heads <= 16.
  *   - Thread safety: calls on different streams may run concurrently; the
- *     library holds no mutable global state besides kvq_last_error().
+ *     library's mutable global state is kvq_last_error(), the two
+ *     process-wide decode modes (kvq_set_decode_deterministic,
+ *     kvq_debug_decode_stall) and the fixed scratch of
+ *     kvq_decode_attn_noalloc (whose calls must not overlap).
  */
 #ifndef KVQ_H_
 #define KVQ_H_
@@ -416,6 +419,18 @@ KVQ_API int kvq_combine_partials(const kvq_cfg* cfg, const void* const* plans_de
  * KVQ_ERR_ARG.
  */
 KVQ_API int kvq_debug_decode_stall(long long cycles);
+
+/*
+ * Deterministic decode (no counterpart in the paper; for reproducible
+ * debugging). on != 0: every later packed decode launch of the process
+ * (kvq_decode_attn, kvq_append_decode, the paged and partial forms) merges
+ * its split records in split order in the last split, instead of summing the
+ * splits in exponent buckets by L2 atomics whose order varies from run to
+ * run, so repeated calls on the same inputs give the same bits. It costs a
+ * few microseconds per launch (one CTA per sequence and KV head reads every
+ * split record). on = 0 restores the default. Returns KVQ_OK.
+ */
+KVQ_API int kvq_set_decode_deterministic(int on);
 
 /*
  * Recent-token window ("RoPE-Aware Bit Allocation for KV-Cache
