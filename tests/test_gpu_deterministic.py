@@ -46,3 +46,31 @@ def test_deterministic_decode_repeats_bit_for_bit():
     # the default mode after it, on the same workspace, still agrees to rounding
     o = L.decode(q, ws=ws).cpu().numpy()
     assert op.rel_err(o, outs[0]) <= 1e-5 and L.flags() == 0
+
+
+def test_deterministic_fused_step_repeats():
+    # the fused append + decode step in deterministic mode: two layers fed
+    # the same inputs end with the same records and the same outputs
+    rng = np.random.default_rng(30)
+    n_kv, T, G = 2, 9000, 8
+    cfg = kvq.make_cfg(n_kv, 3, 2, v_seed=4)
+    E = np.exp(rng.standard_normal((n_kv, 64)))
+    kb = synth.to_bf16_bits(rng.standard_normal((1, T, n_kv, 128)))
+    vb = synth.to_bf16_bits(rng.standard_normal((1, T, n_kv, 128)))
+    kn = dev_bf16(synth.to_bf16_bits(rng.standard_normal((1, 3, n_kv, 128))))
+    vn = dev_bf16(synth.to_bf16_bits(rng.standard_normal((1, 3, n_kv, 128))))
+    q = dev_bf16(synth.to_bf16_bits(rng.standard_normal((1, n_kv * G, 128))))
+    outs, layers = [], []
+    try:
+        kvq.lib().kvq_set_decode_deterministic(1)
+        for _ in range(2):
+            L = PackedLayer(cfg, 1, T + 64)
+            L.set_plans(kvq.plan_build(cfg, 0, E))
+            L.append(dev_bf16(kb), dev_bf16(vb))
+            outs.append(L.append_decode(kn, vn, q).cpu().numpy())
+            layers.append(L)
+    finally:
+        kvq.lib().kvq_set_decode_deterministic(0)
+    assert np.array_equal(outs[0], outs[1])
+    assert torch.equal(layers[0].caches[0], layers[1].caches[0])
+    assert all(L.flags() == 0 and int(L.lens.item()) == T + 3 for L in layers)

@@ -131,3 +131,49 @@ def test_window_evictions_past_capacity_flag_and_leave_state():
     torch.cuda.synchronize()
     assert L.flags() & kvq.FLAG_CAPACITY
     assert L.lens.item() == 54 and L.wlens.item() == 16
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "fp32"])
+def test_window_with_rotated_keys_and_other_input_types(dtype):
+    # plans with the width-group key rotation; fp16 / fp32 appends: the ring
+    # holds the values exactly and evicted tokens are quantized like any other
+    rng = np.random.default_rng(11 if dtype == "fp16" else 12)
+    n_kv, batch, R = 2, 2, 40
+    steps = [150, 3, 30, 1, 50]
+    T = sum(steps)
+    cfg = kvq.make_cfg(n_kv, 3, 3, v_seed=V_SEED, alloc_mode=kvq.ALLOC_GREEDY | kvq.ALLOC_ROTATE_KEYS)
+    L = PackedLayer(cfg, batch, T + 32, window=R)
+    E = np.exp(rng.standard_normal((n_kv, 64)) - np.arange(64) / 8.0)
+    L.set_plans(kvq.plan_build(cfg, 0, E))
+    # inputs exactly representable in bf16 (the oracle's input type) and in
+    # the append's type: bf16 values away from fp16's subnormal range are
+    # exact in fp16 (fewer mantissa bits, a wider exponent than needed)
+    kb, vb = _inputs(rng, batch, T, n_kv)
+    kf, vf = synth.bf16_bits_to_f64(kb), synth.bf16_bits_to_f64(vb)
+    kf[np.abs(kf) < 2.0 ** -14] = 0.0
+    vf[np.abs(vf) < 2.0 ** -14] = 0.0
+    kb, vb = synth.to_bf16_bits(kf), synth.to_bf16_bits(vf)
+    tdt = torch.float16 if dtype == "fp16" else torch.float32
+    kd = torch.from_numpy(kf).to(tdt).cuda()
+    vd = torch.from_numpy(vf).to(tdt).cuda()
+    assert np.array_equal(kd.double().cpu().numpy(), kf)
+    assert np.array_equal(vd.double().cpu().numpy(), vf)
+    t = 0
+    for n in steps:
+        L.append_window(kd[:, t:t + n].contiguous(), vd[:, t:t + n].contiguous())
+        t += n
+    torch.cuda.synchronize()
+    sp = window.split_point(T, R)
+    assert L.lens.cpu().tolist() == [sp] * batch and L.flags() == 0
+    qb = synth.to_bf16_bits(rng.standard_normal((batch, n_kv * 8, 128)))
+    out = L.decode_window(dev_bf16(qb)).cpu().numpy()
+    for s_ in range(batch):
+        kh, vh = op.bf16_heads(kb[s_], vb[s_])
+        heads = op.layer([x[:sp] for x in kh], [x[:sp] for x in vh], 3, 3, V_SEED, 0, E=E,
+                         rotate_keys=True)[1]
+        for h in range(n_kv):
+            check_records(L.head_records(s_, h, (sp + 31) // 32), heads[h]["rec"], sp, 3, 3)
+        ref = window.decode(synth.bf16_bits_to_f64(qb[s_]), [x["khat"] for x in heads],
+                            [x["vhat"] for x in heads], [x[sp:] for x in kh],
+                            [x[sp:] for x in vh])
+        assert op.rel_err(out[s_], ref) <= TOL
