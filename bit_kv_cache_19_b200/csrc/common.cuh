@@ -223,6 +223,72 @@ __device__ __forceinline__ uint32_t funnel_r(uint32_t lo, uint32_t hi, uint32_t 
   return __funnelshift_r(lo, hi, sh);
 }
 
+// Structural check of a plan (shared memory) by one whole warp; every lane
+// gets the answer. True iff the plan order, the K segment offsets, the half
+// steps and the width classes are exactly what the host's schedule builder
+// makes of the widths: order = the blocks of nonzero width, width
+// descending then block index ascending; seg_off[r + 1] = seg_off[r] + 2 W;
+// 128 bits_k K words in all; half steps = runs of one width cut into groups
+// of at most 4 ranks; classes = maximal runs of half steps of one width.
+// Every index the kernels derive from these fields then stays inside the
+// plan's arrays and the tile record, whatever the rest of the plan holds.
+constexpr int kMaxHalfSteps = 24;  // <= 64 / 4 + one partial group per width
+__device__ __forceinline__ bool plan_sched_ok(const Plan& pl, int lane) {
+  // scalar fields as lane 0 read them, so that the early exit is uniform
+  const int nr = __shfl_sync(0xffffffffu, pl.n_ranks, 0);
+  const int nh = __shfl_sync(0xffffffffu, (int)pl.n_half, 0);
+  const int nc = __shfl_sync(0xffffffffu, (int)pl.n_class, 0);
+  const int bk = __shfl_sync(0xffffffffu, pl.bits_k, 0);
+  if (nr < 1 || nr > 64 || bk < 1 || bk > 8 || nh < 1 || nh > kMaxHalfSteps || nc < 1 || nc > 8)
+    return false;
+  auto width_of_rank = [&](int r) { return (int)pl.width[pl.order[r] & 63]; };
+  bool ok = true;
+  uint32_t seen[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int r = lane + 32 * i;
+    if (r < nr) {
+      const int o = pl.order[r], w = width_of_rank(r);
+      ok &= o < 64 && w >= 1 && w <= 8;
+      ok &= pl.seg_off[r + 1] == pl.seg_off[r] + 2 * w;
+      if (r + 1 < nr) {
+        const int o2 = pl.order[r + 1], w2 = width_of_rank(r + 1);
+        ok &= w > w2 || (w == w2 && o < o2);
+      }
+      seen[(o >> 5) & 1] |= 1u << (o & 31);
+    }
+  }
+  ok &= pl.seg_off[0] == 0 && pl.seg_off[nr] == 128 * bk;
+  // the order holds each block of nonzero width once (with the strict
+  // ordering above, no block twice)
+  ok &= __reduce_or_sync(0xffffffffu, seen[0]) == __ballot_sync(0xffffffffu, pl.width[lane] != 0);
+  ok &= __reduce_or_sync(0xffffffffu, seen[1]) ==
+        __ballot_sync(0xffffffffu, pl.width[lane + 32] != 0);
+  if (lane < nh) {
+    const int r0 = pl.hs_rank0[lane], n = pl.hs_count[lane];
+    ok &= n >= 1 && n <= 4 && r0 + n <= nr && (lane > 0 || r0 == 0);
+    if (n >= 1 && r0 + n <= nr) {
+      const int w = width_of_rank(r0);
+      ok &= pl.hs_width[lane] == w && width_of_rank(r0 + n - 1) == w;
+      if (n < 4 && r0 + n < nr) ok &= width_of_rank(r0 + n) != w;  // a short group ends its run
+      ok &= lane + 1 < nh ? pl.hs_rank0[lane + 1] == r0 + n : r0 + n == nr;
+    }
+  }
+  if (lane < nc) {
+    const int h0 = pl.cls_hs0[lane], m = pl.cls_nhs[lane];
+    ok &= m >= 1 && h0 + m <= nh && (lane > 0 || h0 == 0);
+    if (m >= 1 && h0 + m <= nh) {
+      const int w = pl.hs_width[h0], r0 = pl.hs_rank0[h0];
+      ok &= pl.cls_w[lane] == w && pl.hs_width[h0 + m - 1] == w &&
+            pl.cls_last[lane] == pl.hs_count[h0 + m - 1] && r0 < nr &&
+            pl.cls_seg0[lane] == pl.seg_off[r0 & 63];
+      ok &= lane + 1 < nc ? pl.cls_hs0[lane + 1] == h0 + m && pl.hs_width[h0 + m] != w
+                          : h0 + m == nh;
+    }
+  }
+  return __all_sync(0xffffffffu, ok);
+}
+
 #endif  // __CUDACC__
 
 }  // namespace kvq

@@ -68,7 +68,7 @@ constexpr uint32_t kLutPair4 = 0x2800u, kLutPair5 = 0x2C00u, kLutSingle = 0x3C00
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kStages = 2;
-constexpr int kMaxHalf = 24;  // half steps of <= 4 blocks (<= 64/4 + 8)
+constexpr int kMaxHalf = kMaxHalfSteps;  // half steps of <= 4 blocks
 constexpr int kBuckets = 16;  // split maxima m in [32 (k - 8), 32 (k - 7)), k = 0..15
 // Per (sequence, KV head) "pair block" of the workspace, at a fixed distance
 // from its end: 32 counter words (0: arrivals, 1: range flag, 2..17: bucket
@@ -338,6 +338,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
     for (uintptr_t a = (q0 & ~(uintptr_t)127) + (uintptr_t)tid * 128; a < q1; a += kThreads * 128)
       prefetch_l2(reinterpret_cast<const void*>(a < q0 ? q0 : a));
   }
+  // ---- plan and lookup image (independent of the previous kernel): the
+  //      plan is checked before anything is derived from it
+  __syncthreads();  // the barriers are initialised
+  const bool ok_setup = mbar_wait_bounded(&sm.setup_bar, 0u);
+  const uint8_t* const cache0 = p.cm.table ? nullptr : p.cm.caches[b];  // contiguous base
+  const int bk = sm.plan.bits_k;
+  const int n_half = sm.plan.n_half;
+  bool bad = !plan_sched_ok(sm.plan, lane);  // the whole warp takes part
+  bad = bad || !ok_setup || sm.plan.magic != KVQ_PLAN_MAGIC || sm.plan.bits_v != BV ||
+        p.tile_bytes != tile_bytes(bk, BV) || (reinterpret_cast<uintptr_t>(cache0) & 15) != 0;
   // ---- with `early` the caller guarantees that the previous kernel on the
   //      stream writes neither these caches nor these lengths: the length is
   //      read and the first tiles are streamed before waiting for it
@@ -358,21 +368,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
     }
   }
   __syncthreads();
-  const bool ok_setup = mbar_wait_bounded(&sm.setup_bar, 0u);
-  const uint8_t* const cache0 = p.cm.table ? nullptr : p.cm.caches[b];  // contiguous base
-  const int bk = sm.plan.bits_k;
-  const int n_half = sm.plan.n_half;
-  bool bad = !ok_setup || sm.plan.magic != KVQ_PLAN_MAGIC || sm.plan.bits_v != BV ||
-             bk < 1 || bk > 8 || p.tile_bytes != tile_bytes(bk, BV) || n_half < 1 ||
-             n_half > kMaxHalf || sm.plan.n_class < 1 || sm.plan.n_class > 8 ||
-             sm.plan.n_ranks < 1 || sm.plan.n_ranks > 64 ||
-             (reinterpret_cast<uintptr_t>(cache0) & 15) != 0;
-  // width classes: every word a class reads must lie in the tile's key words
-  // plus the one half step of overrun a partial last half step allows
+  // width classes (consistent with the segments by the check above): every
+  // word a class reads lies in the tile's key words plus the one half step
+  // of overrun a partial last half step allows
   for (int ci = 0; !bad && ci < sm.plan.n_class; ++ci) {
-    const int W = sm.plan.cls_w[ci], hs0 = sm.plan.cls_hs0[ci], nhs = sm.plan.cls_nhs[ci];
-    bad = W < 1 || W > 8 || nhs < 1 || hs0 + nhs > n_half ||
-          sm.plan.cls_seg0[ci] + 8 * W * nhs > 128 * bk + 64;
+    const int W = sm.plan.cls_w[ci], nhs = sm.plan.cls_nhs[ci];
+    bad = sm.plan.cls_seg0[ci] + 8 * W * nhs > 128 * bk + 64;
   }
   if (bad && tid == 0) atomicOr(p.status, ok_setup ? KVQ_FLAG_BAD_PLAN : KVQ_FLAG_TIMEOUT);
   const int len0 = sm.len0;

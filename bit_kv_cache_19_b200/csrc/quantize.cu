@@ -294,8 +294,7 @@ __global__ void __launch_bounds__(256, 4) quantize_append_kernel(QuantParams p) 
       cur = bh;
       plan_ok = s_plan.magic == KVQ_PLAN_MAGIC && s_plan.bits_k >= 1 && s_plan.bits_k <= 8 &&
                 s_plan.bits_v == BV && p.tile_bytes == tile_bytes(s_plan.bits_k, BV) &&
-                s_plan.n_ranks >= 1 && s_plan.n_ranks <= 64 && s_plan.n_class >= 1 &&
-                s_plan.n_class <= 8;
+                plan_sched_ok(s_plan, lane);
       if (plan_ok && s_plan.k_rot) rot_tables(s_plan, s_rot, threadIdx.x);
       vsgn = 0;
 #pragma unroll

@@ -65,7 +65,9 @@ typedef struct CUstream_st* kvq_stream_t;
 #define KVQ_FLAG_NONFINITE 2u  /* a token had a NaN/Inf coordinate: stored as norm 0, codes 0 */
 #define KVQ_FLAG_NORM_SAT 4u   /* a norm overflowed fp16: stored as 65504 */
 #define KVQ_FLAG_TIMEOUT 8u    /* a bounded wait ran out: output invalid */
-#define KVQ_FLAG_BAD_PLAN 16u  /* a plan record failed its magic/shape check */
+#define KVQ_FLAG_BAD_PLAN 16u  /* a plan record failed its device check (magic, shape, or an
+                                  order / segment / schedule that does not follow from
+                                  its widths): nothing stored or read with it */
 #define KVQ_FLAG_BAD_PAGE 32u  /* paged cache: a tile past the block table or a page id outside
                                   the pool (appends skip it; decode output is invalid) */
 
@@ -345,7 +347,10 @@ KVQ_API int kvq_quantize_append_rope(const kvq_cfg* cfg, const void* const* plan
  * buckets and applies the inverse rotation. One kernel launch; fp32
  * accumulation; the atomic sum order varies, so repeated calls agree to fp32
  * rounding, not bit for bit.
- * plans_dev, cache_dev: as for kvq_quantize_append.
+ * plans_dev, cache_dev: as for kvq_quantize_append. The kernel uses
+ *        programmatic dependent launch and reads the plans (and their
+ *        pointer array) before the previous kernel on the stream has ended,
+ *        so that kernel must not write them.
  * len_dev: int32 [batch], each <= max_len (a larger value is clamped to
  *        max_len and flags CAPACITY). A sequence of length 0 gives o = 0.
  * q_dev: [batch][n_q_heads][128] of type q_dtype (post-RoPE queries).
