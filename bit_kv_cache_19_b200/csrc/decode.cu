@@ -338,16 +338,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
     for (uintptr_t a = (q0 & ~(uintptr_t)127) + (uintptr_t)tid * 128; a < q1; a += kThreads * 128)
       prefetch_l2(reinterpret_cast<const void*>(a < q0 ? q0 : a));
   }
-  // ---- plan and lookup image (independent of the previous kernel): the
-  //      plan is checked before anything is derived from it
-  __syncthreads();  // the barriers are initialised
-  const bool ok_setup = mbar_wait_bounded(&sm.setup_bar, 0u);
-  const uint8_t* const cache0 = p.cm.table ? nullptr : p.cm.caches[b];  // contiguous base
-  const int bk = sm.plan.bits_k;
-  const int n_half = sm.plan.n_half;
-  bool bad = !plan_sched_ok(sm.plan, lane);  // the whole warp takes part
-  bad = bad || !ok_setup || sm.plan.magic != KVQ_PLAN_MAGIC || sm.plan.bits_v != BV ||
-        p.tile_bytes != tile_bytes(bk, BV) || (reinterpret_cast<uintptr_t>(cache0) & 15) != 0;
   // ---- with `early` the caller guarantees that the previous kernel on the
   //      stream writes neither these caches nor these lengths: the length is
   //      read and the first tiles are streamed before waiting for it
@@ -368,12 +358,25 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
     }
   }
   __syncthreads();
-  // width classes (consistent with the segments by the check above): every
-  // word a class reads lies in the tile's key words plus the one half step
-  // of overrun a partial last half step allows
+  const bool ok_setup = mbar_wait_bounded(&sm.setup_bar, 0u);
+  const uint8_t* const cache0 = p.cm.table ? nullptr : p.cm.caches[b];  // contiguous base
+  const int bk = sm.plan.bits_k;
+  const int n_half = sm.plan.n_half;
+  // Bounds that keep every index the kernel takes from the plan in range,
+  // whatever its other bytes (the block pass of an append also masks its
+  // word index); the full check of the schedule (plan_sched_ok) runs where
+  // it costs no time, in split 0 during its arrival, and only flags
+  bool bad = !ok_setup || sm.plan.magic != KVQ_PLAN_MAGIC || sm.plan.bits_v != BV ||
+             bk < 1 || bk > 8 || p.tile_bytes != tile_bytes(bk, BV) || n_half < 1 ||
+             n_half > kMaxHalf || sm.plan.n_class < 1 || sm.plan.n_class > 8 ||
+             sm.plan.n_ranks < 1 || sm.plan.n_ranks > 64 ||
+             (reinterpret_cast<uintptr_t>(cache0) & 15) != 0;
+  // width classes: every word a class reads must lie in the tile's key words
+  // plus the one half step of overrun a partial last half step allows
   for (int ci = 0; !bad && ci < sm.plan.n_class; ++ci) {
-    const int W = sm.plan.cls_w[ci], nhs = sm.plan.cls_nhs[ci];
-    bad = sm.plan.cls_seg0[ci] + 8 * W * nhs > 128 * bk + 64;
+    const int W = sm.plan.cls_w[ci], hs0 = sm.plan.cls_hs0[ci], nhs = sm.plan.cls_nhs[ci];
+    bad = W < 1 || W > 8 || nhs < 1 || hs0 + nhs > n_half ||
+          sm.plan.cls_seg0[ci] + 8 * W * nhs > 128 * bk + 64;
   }
   if (bad && tid == 0) atomicOr(p.status, ok_setup ? KVQ_FLAG_BAD_PLAN : KVQ_FLAG_TIMEOUT);
   const int len0 = sm.len0;
@@ -790,7 +793,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
     }
   }
   __syncthreads();
-  if (tid == 0) sm.is_last = arrive_last(&cnt[0], (unsigned int)p.n_splits);
+  if (tid == 0) {
+    sm.is_last = arrive_last(&cnt[0], (unsigned int)p.n_splits);
+  } else if (warp == 1 && split == 0 && !bad) {
+    // during the arrival's round trip: the full plan check (flag only; the
+    // bounds checked up front keep every index of the decode in range)
+    if (!plan_sched_ok(sm.plan, lane) && lane == 0) atomicOr(p.status, KVQ_FLAG_BAD_PLAN);
+  }
   __syncthreads();
   if (!sm.is_last) return;
 

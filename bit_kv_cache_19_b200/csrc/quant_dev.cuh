@@ -60,10 +60,12 @@ constexpr int kKzStride = kHeadDim + 1;  // padded rows: pass 2 reads a column
 
 // Branch-free: the word after the field's first word is always touched (an
 // OR of 0 / AND of all ones when the field does not reach it), so `words`
-// needs one word of slack past the packed words. nbits <= 16.
+// needs one word of slack past the packed words. nbits <= 16. The first word
+// is clamped to wmax, so a plan whose segments lie outside the key words
+// (flagged by the plan checks) cannot send a write past word wmax + 1.
 __device__ __forceinline__ void put_field(uint32_t* words, int bit, uint32_t val, int nbits,
-                                          bool clear) {
-  const int wi = bit >> 5, off = bit & 31;
+                                          bool clear, int wmax) {
+  const int wi = min(bit >> 5, wmax), off = bit & 31;
   const uint32_t mask = (1u << nbits) - 1u;
   // parts of the field in word wi and wi + 1 (64-bit shift: off may be 0)
   const unsigned long long v2 = (unsigned long long)val << off;
@@ -306,12 +308,13 @@ template <int W>
 __device__ __forceinline__ void block_field(const Plan& pl, const float* thr, int r, int j,
                                             const float* row, int lane, uint32_t* words,
                                             bool clear, bool rot) {
-  const float g = pl.g[j];
-  const float z0 = rot ? row[2 * r] : __fmul_rn(row[j], g);
-  const float z1 = rot ? row[2 * r + 1] : __fmul_rn(row[j + 64], g);
+  const float g = pl.g[j & 63];
+  const float z0 = rot ? row[2 * r] : __fmul_rn(row[j & 63], g);
+  const float z1 = rot ? row[2 * r + 1] : __fmul_rn(row[(j & 63) + 64], g);
   const uint32_t c0 = (uint32_t)code_of_w<W>(thr, z0);
   const uint32_t c1 = (uint32_t)code_of_w<W>(thr, z1);
-  put_field(words, 32 * pl.seg_off[r] + slot_k(lane) * 2 * W, c0 | (c1 << W), 2 * W, clear);
+  put_field(words, 32 * pl.seg_off[r] + slot_k(lane) * 2 * W, c0 | (c1 << W), 2 * W, clear,
+            128 * pl.bits_k - 1);
 }
 
 __device__ __forceinline__ void warp_block_pass(const Plan& pl, const float* thr, int r,

@@ -225,12 +225,11 @@ __device__ __forceinline__ void bulk_token_pass(const Plan& pl, const float* thr
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     uint32_t* w = vwords + BV * 32 * q;
-    const float z = __fmul_rn(y[q], vr);
-    uint32_t c = 0u;
-    if (vlive) {
-      if constexpr (BV <= 3) c = code_of_reg<BV>(tv, z);
-      else c = (uint32_t)code_of_w<BV>(thr, z);
-    }
+    const float z = __fmul_rn(y[q], vr);  // 0 for a dead token (vr = 0)
+    uint32_t c;
+    if constexpr (BV <= 3) c = code_of_reg<BV>(tv, z);
+    else c = (uint32_t)code_of_w<BV>(thr, z);
+    c = vlive ? c : 0u;  // a select, not a branch, in the unrolled loop
     if (clear) atomicAnd(w, ~(mask << off));
     atomicOr(w, c << off);
     if (spill) {

@@ -67,7 +67,10 @@ typedef struct CUstream_st* kvq_stream_t;
 #define KVQ_FLAG_TIMEOUT 8u    /* a bounded wait ran out: output invalid */
 #define KVQ_FLAG_BAD_PLAN 16u  /* a plan record failed its device check (magic, shape, or an
                                   order / segment / schedule that does not follow from
-                                  its widths): nothing stored or read with it */
+                                  its widths): kvq_quantize_append stores no token with
+                                  it, a fused append (kvq_append_decode) may store
+                                  undefined codes in the token's tile record, the length
+                                  still advances, and decode output is invalid */
 #define KVQ_FLAG_BAD_PAGE 32u  /* paged cache: a tile past the block table or a page id outside
                                   the pool (appends skip it; decode output is invalid) */
 

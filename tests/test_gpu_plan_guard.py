@@ -1,10 +1,11 @@
 """Plan records whose magic and shape are valid but whose order, K segments
-or decode schedule do not follow from the widths are refused on the device:
-kvq_quantize_append stores nothing for them and kvq_decode_attn reads no tile
-with them, both flagging BAD_PLAN. The corruptions are ones the host check
-(kvq_plan_check) also refuses, and each keeps every index the kernels would
-derive from it inside the tile record (so the test is safe even against a
-kernel that failed to refuse it)."""
+or decode schedule do not follow from the widths are flagged on the device
+(BAD_PLAN): kvq_quantize_append stores nothing with them, and
+kvq_decode_attn and kvq_append_decode flag their output (the fused append
+keeps its writes inside the token's tile record). The corruptions are
+ones the host check (kvq_plan_check) also refuses, and each keeps every index
+the kernels would derive from it inside the tile record (so the test is safe
+even against a kernel that failed to refuse it)."""
 import numpy as np
 import pytest
 import torch
@@ -99,13 +100,24 @@ def test_device_refuses_inconsistent_plans():
         torch.cuda.synchronize()
         assert M.flags() & kvq.FLAG_BAD_PLAN, name
         assert torch.equal(before, M.caches[0]), name
-        # decode over a cache written with the valid plan: no tile read
+        # decode over a cache written with the valid plan: output flagged
         L.set_plans(bad, check=False)
         L.status.zero_()
-        out = L.decode(q, ws=ws)
+        L.decode(q, ws=ws)
         torch.cuda.synchronize()
         assert L.flags() & kvq.FLAG_BAD_PLAN, name
-        assert bool((out == 0).all()), name
+        # fused append + decode: flagged; the append writes only inside the
+        # record of the token's tile (tile 3 of 4 here)
+        n0 = int(L.lens.item())
+        rec = L.caches[0].clone()
+        L.status.zero_()
+        L.append_decode(k[:, :1].contiguous(), v[:, :1].contiguous(), q, ws=ws)
+        torch.cuda.synchronize()
+        assert L.flags() & kvq.FLAG_BAD_PLAN, name
+        tb = kvq.tile_bytes(cfg)
+        assert torch.equal(rec[:3 * tb], L.caches[0][:3 * tb]), name
+        L.caches[0].copy_(rec)
+        L.lens.fill_(n0)
     # the workspace is still usable with the valid plan
     L.set_plans(plan)
     L.status.zero_()
