@@ -735,13 +735,81 @@ def measure_point(args, wl, T, alloc, n_layers, rank, dev, stream, peak, steps):
     return out
 
 
+def measure_window(args, wl, T, R, n_layers, rank, dev, stream, peak, steps):
+    """The recent-token window on a workload point: per layer a cache whose R
+    most recent tokens stay exact (the prefill goes through the window, so
+    the oldest T - R tokens are packed), and a step of kvq_window_append (one
+    token: quantize the evicted token, push the new one) plus
+    kvq_decode_attn_window (partial decode over the packed tokens, the
+    window's record, combine) per layer; `steps` graph replays timed."""
+    import torch
+
+    from bit_kv_cache_19_b200 import kvq
+    from bit_kv_cache_19_b200.runtime import PackedLayer
+
+    B, n_step, warmup = wl.batch, max(1, wl.n_new), 3
+    cap = T + (steps + warmup + 2) * n_step + 64
+    cfg = kvq.make_cfg(wl.n_kv_heads, wl.bits_k, wl.bits_v, v_seed=1234)
+    bpth = BYTES_PER_TOKEN_HEAD(wl.bits_k, wl.bits_v)
+    layers = []
+    for li in range(n_layers):
+        L = PackedLayer(cfg, B, cap, device=dev, layer=li, window=R)
+        ks, vs = zip(*[synth.keys_values_torch(wl, rank_seed(args.seed, rank, b), li, T, dev)
+                       for b in range(B)])
+        L.alloc_bits(ks[0])
+        L.append_window(torch.stack(ks), torch.stack(vs))
+        del ks, vs
+        layers.append(L)
+    torch.cuda.synchronize()
+    _, _, qs, knew, vnew = step_buffers(wl, n_layers, n_step, T, args.seed, dev)
+    outs = [torch.empty(B, wl.n_q_heads, 128, dtype=torch.float32, device=dev)
+            for _ in range(n_layers)]
+    ws = torch.zeros(kvq.window_decode_workspace_bytes(cfg, B, wl.n_q_heads, cap),
+                     dtype=torch.uint8, device=dev)
+
+    def step():
+        for li, L in enumerate(layers):
+            L.append_window(knew[li], vnew[li])
+            L.decode_window(qs[li], out=outs[li], ws=ws)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            step()
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+        len_before = int(layers[0].lens[0].item())
+        ms = time_replays(graph.replay, stream, steps, None)
+        torch.cuda.synchronize()
+    flags = 0
+    for L in layers:
+        flags |= L.flags()
+    assert flags == 0, f"window {T} {R}: status flags {flags}"
+    mean_packed = len_before + n_step * (steps + 1) / 2
+    packed_bytes = n_layers * B * wl.n_kv_heads * bpth * mean_packed
+    ring_bytes = n_layers * B * wl.n_kv_heads * R * 2 * 128 * 4
+    out = {"layers": n_layers, "batch": B, "context": T, "window": R,
+           "budget": f"K{wl.bits_k}V{wl.bits_v}", "appended_per_step": n_step, "steps": steps,
+           "ms_per_step": ms, "GB_per_s": (packed_bytes + ring_bytes) / (ms / 1e3) / 1e9,
+           "frac": (packed_bytes + ring_bytes) / (ms / 1e3) / 1e9 / peak,
+           "launches_per_layer": 5,
+           "note": "bytes = packed tokens read by the partial decode + the fp32 window ring; "
+                   "the step is kvq_window_append + kvq_decode_attn_window per layer"}
+    graph = None
+    del layers, qs, knew, vnew, outs, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_extras(args, rank, dev, stream, peak):
     """The other workloads of the build: one Llama-3.1-8B-shaped layer at 32K
     (K2V2), the 7B-Qwen-shaped serving step (16 x 32K, append 16 + decode,
     28 layers, K3V2), the Qwen2.5-3B-shaped context sweep 8K..512K with
-    Block-GTQ (greedy) and uniform plans of the same bytes, and the bulk
-    prefill of 512K tokens x 36 layers (its roofline: bf16 K/V in plus the
-    packed bytes out at the measured copy bandwidth)."""
+    Block-GTQ (greedy) and uniform plans of the same bytes, the 36-layer
+    128K step with a 128-token recent-token window, and the bulk prefill of
+    512K tokens x 36 layers (its roofline: bf16 K/V in plus the packed bytes
+    out at the measured copy bandwidth)."""
     steps = 20
     out = {}
     W = synth.WORKLOADS
@@ -758,6 +826,9 @@ def run_extras(args, rank, dev, stream, peak):
             sweep.append(measure_point(args, sw, T, alloc, sw.n_layers, rank, dev, stream, peak,
                                        steps))
     out["qwen3b_sweep"] = sweep
+    wq = W["qwen3b_128k"]
+    out["qwen3b_128k_window128"] = measure_window(args, wq, wq.context, 128, wq.n_layers, rank,
+                                                  dev, stream, peak, steps)
     big = [p for p in sweep if p["context"] == max(sw.contexts) and p["alloc"] == "greedy"][0]
     tok_heads = big["layers"] * big["context"] * sw.n_kv_heads
     moved = tok_heads * (512 + BYTES_PER_TOKEN_HEAD(sw.bits_k, sw.bits_v))

@@ -40,6 +40,8 @@ cudaError_t launch_window_record(const Plan* const* plans, const float* const* w
                                  const int32_t* len, const int32_t* wlen, int R, const void* q,
                                  int q_dtype, int n_q, int n_kv, int batch, float* recs,
                                  cudaStream_t st);
+int window_parts(int R, int* tokens_per_part);
+constexpr int kWindowPartsMax = 32;  // window record parts per (KV head, sequence), at most
 
 namespace {
 
@@ -690,8 +692,10 @@ int kvq_window_append(const kvq_cfg* cfg, const void* const* plans_dev, const vo
   return KVQ_OK;
 }
 
+// The packed tokens' records, then up to kWindowPartsMax window record parts.
 static size_t window_records_bytes(int batch, int n_q_heads) {
-  return ((size_t)2 * batch * n_q_heads * kRecFloats * sizeof(float) + 255) / 256 * 256;
+  return ((size_t)(1 + kWindowPartsMax) * batch * n_q_heads * kRecFloats * sizeof(float) + 255) /
+         256 * 256;
 }
 
 size_t kvq_window_decode_workspace_bytes(const kvq_cfg* cfg, int batch, int n_q_heads,
@@ -731,8 +735,10 @@ int kvq_decode_attn_window(const kvq_cfg* cfg, const void* const* plans_dev,
                                        wlen_dev, R, q_dev, q_dtype, n_q_heads, cfg->n_kv_heads,
                                        batch, rec_win, st);
   if (e != cudaSuccess) return cuda_fail(e, "decode_attn_window (window)");
-  e = launch_combine(reinterpret_cast<const Plan* const*>(plans_dev), recs, 2, batch, n_q_heads,
-                     cfg->n_kv_heads, out_dev, st);
+  int per_part = 0;
+  const int parts = window_parts(R, &per_part);
+  e = launch_combine(reinterpret_cast<const Plan* const*>(plans_dev), recs, 1 + parts, batch,
+                     n_q_heads, cfg->n_kv_heads, out_dev, st);
   if (e != cudaSuccess) return cuda_fail(e, "decode_attn_window (combine)");
   return KVQ_OK;
 }

@@ -15,10 +15,11 @@
 //   ring or from the new rows), then window_push_kernel copies the remaining
 //   new tokens into the ring and updates both lengths.
 // * Decode: the packed tokens give one merged record per query head (the
-//   partial decode); window_record_kernel gives the window's record in the
+//   partial decode); window_record_kernel gives the window's records in the
 //   same form (base-2 maximum, sum, and o in the value-rotation domain: each
 //   window value enters as H (s . v), so the combine's inverse rotation
-//   returns it); the combine kernel merges the two records.
+//   returns it), one per part of the window (up to 32 CTAs per KV head and
+//   sequence); the combine kernel merges all of them.
 #include <algorithm>
 #include <atomic>
 
@@ -28,6 +29,7 @@ namespace kvq {
 
 constexpr int kWinThreads = 256;
 constexpr int kWinWarps = kWinThreads / 32;
+constexpr int kWinParts = 32;  // window record parts per (KV head, sequence), at most (api.cu)
 
 // One CTA per sequence: the new tokens that stay in the window go to their
 // ring slots (converted to fp32), then len += evicted, wlen = min(R, wlen +
@@ -62,101 +64,168 @@ __global__ void __launch_bounds__(kWinThreads) window_push_kernel(
   }
 }
 
-// One CTA per (KV head, sequence): the window's record of each of the G
-// query heads, (m, l, -, -, o[128]) with m the base-2 maximum logit, l =
-// sum 2^(s - m) and o = sum 2^(s - m) H (s . v) (value-rotation domain).
-// Warp w takes window tokens w, w + 8, ...; each keeps per head a running
-// maximum, sum and o (4 coordinates per lane); the warps merge in shared
-// memory. Logits in fp32: s = (q . k) log2(e) / sqrt(128).
+// Window records of the G query heads of a (KV head, sequence), split over
+// grid.z CTAs: CTA z takes window tokens [z C, z C + C) and writes record
+// part z, (m, l, -, -, o[128]) with m the base-2 maximum logit, l =
+// sum 2^(s - m) and o = sum 2^(s - m) H (s . v) (value-rotation domain);
+// the combine merges the parts with the packed tokens' record. A CTA takes
+// its tokens 16 at a time, staged in shared memory: the keys as read, the
+// values rotated (two tokens per warp, loads issued together; the fp32
+// butterflies of the value quantizer); then one thread per (token, head)
+// forms a logit (fp32, s = (q . k) log2(e) / sqrt(128)), one warp per head
+// updates the running maximum and sum, and one thread per (coordinate, head
+// set) updates o.
+constexpr int kWinSub = 16;                // tokens staged at a time
+constexpr int kWinKStride = kHeadDim + 1;  // padded key rows (a token per lane, no conflicts)
+
 __global__ void __launch_bounds__(kWinThreads) window_record_kernel(
     const Plan* const* plans, const float* const* wins, const int32_t* len,
-    const int32_t* wlen, int R, const void* __restrict__ q, int q_dtype, int n_q, int n_kv,
-    float* __restrict__ recs) {
-  extern __shared__ __align__(16) float wsm[];  // q' [G][128], then [warps][G][132]
-  const int h = blockIdx.x, b = blockIdx.y, G = n_q / n_kv;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* qs = wsm;
-  float* mg = wsm + G * kHeadDim;
+    const int32_t* wlen, int R, int C, const void* __restrict__ q, int q_dtype, int n_q,
+    int n_kv, int batch, float* __restrict__ recs) {
+  __shared__ __align__(16) float qs[16 * kHeadDim];           // q' [G][128]
+  __shared__ __align__(16) float ks[kWinSub * kWinKStride];    // staged keys
+  __shared__ __align__(16) float ys[kWinSub * kHeadDim];       // staged rotated values
+  __shared__ float ps[16 * kWinSub];                           // logits, then weights
+  __shared__ float st[48];                                     // max, sum, rescale per head
+  const int h = blockIdx.x, b = blockIdx.y, z = blockIdx.z, G = n_q / n_kv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const Plan& pl = plans[b][h];
-  for (int e = threadIdx.x; e < G * kHeadDim; e += kWinThreads)
+  for (int e = tid; e < G * kHeadDim; e += kWinThreads)
     qs[e] = load_as_float(q, q_dtype, ((size_t)b * n_q + (size_t)h * G) * kHeadDim + e) *
             0.12751743074f;  // log2(e) / sqrt(128)
-  __syncthreads();
+  if (tid < 16) {
+    st[tid] = -INFINITY;
+    st[16 + tid] = 0.f;
+  }
   const int w = R > 0 ? min(max(wlen[b], 0), R) : 0;
   const int len0 = max(len[b], 0);
-  const float* wk = w > 0 ? wins[b] : nullptr;
-  const float* wv = w > 0 ? wk + (size_t)R * n_kv * kHeadDim : nullptr;
-  float m[16], l[16], o[16][4];
+  const int t_lo = z * C, t_hi = min(w, t_lo + C);
+  const float* wk = t_lo < t_hi ? wins[b] : nullptr;
+  const float* wv = t_lo < t_hi ? wk + (size_t)R * n_kv * kHeadDim : nullptr;
+  const int ci = tid & (kHeadDim - 1), cg = tid >> 7;  // o: coordinate, first head
+  const int lt = tid & (kWinSub - 1), lg = tid >> 4;   // logit: token, head
+  float o[8];
 #pragma unroll
-  for (int g = 0; g < 16; ++g) {
-    m[g] = -INFINITY;
-    l[g] = 0.f;
+  for (int k = 0; k < 8; ++k) o[k] = 0.f;
+  uint32_t vsgn = 0;  // value signs of this lane's coordinates lane + 32 r
 #pragma unroll
-    for (int r = 0; r < 4; ++r) o[g][r] = 0.f;
-  }
-  for (int t = warp; t < w; t += kWinWarps) {
-    const int slot = (int)(((int64_t)len0 + t) % R);
-    const size_t row = ((size_t)slot * n_kv + h) * kHeadDim;
-    float kx[4], y[4];
+  for (int r = 0; r < 4; ++r) vsgn |= ((pl.v_sign[r] >> lane) & 1u) << r;
+  __syncthreads();
+  for (int c0 = t_lo; c0 < t_hi; c0 += kWinSub) {
+    const int n = min(kWinSub, t_hi - c0);
+    // ---- stage: tokens warp and warp + 8 of the sub-chunk
+    {
+      float kx[2][4], y[2][4];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int i = lane + 32 * r;
-      kx[r] = wk[row + i];
-      const float x = wv[row + i];
-      y[r] = ((pl.v_sign[i >> 5] >> (i & 31)) & 1u) ? -x : x;
-    }
-    // y = H (s . v): butterflies h = 1..16 across lanes, then 32 and 64
+      for (int u = 0; u < 2; ++u) {
+        const int t = warp + 8 * u;
+        if (t < n) {
+          const size_t row =
+              ((size_t)((int)(((int64_t)len0 + c0 + t) % R)) * n_kv + h) * kHeadDim;
 #pragma unroll
-    for (int hh = 1; hh < 32; hh <<= 1) {
-      const bool upper = (lane & hh) != 0;
+          for (int r = 0; r < 4; ++r) {
+            kx[u][r] = wk[row + lane + 32 * r];
+            const float x = wv[row + lane + 32 * r];
+            y[u][r] = ((vsgn >> r) & 1u) ? -x : x;
+          }
+        }
+      }
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const float x = __shfl_xor_sync(0xffffffffu, y[r], hh);
-        y[r] = upper ? x - y[r] : y[r] + x;
+      for (int u = 0; u < 2; ++u) {
+        const int t = warp + 8 * u;
+        if (t < n) {  // warp-uniform
+#pragma unroll
+          for (int r = 0; r < 4; ++r) ks[t * kWinKStride + lane + 32 * r] = kx[u][r];
+          // y = H (s . v): butterflies h = 1..16 across lanes, then 32 and 64
+#pragma unroll
+          for (int hh = 1; hh < 32; hh <<= 1) {
+            const bool upper = (lane & hh) != 0;
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+              const float x = __shfl_xor_sync(0xffffffffu, y[u][r], hh);
+              y[u][r] = upper ? x - y[u][r] : y[u][r] + x;
+            }
+          }
+          const float a0 = y[u][0] + y[u][1], a1 = y[u][0] - y[u][1];
+          const float a2 = y[u][2] + y[u][3], a3 = y[u][2] - y[u][3];
+          ys[t * kHeadDim + lane] = a0 + a2;
+          ys[t * kHeadDim + lane + 32] = a1 + a3;
+          ys[t * kHeadDim + lane + 64] = a0 - a2;
+          ys[t * kHeadDim + lane + 96] = a1 - a3;
+        }
       }
     }
-    {
-      const float a0 = y[0] + y[1], a1 = y[0] - y[1], a2 = y[2] + y[3], a3 = y[2] - y[3];
-      y[0] = a0 + a2;
-      y[2] = a0 - a2;
-      y[1] = a1 + a3;
-      y[3] = a1 - a3;
+    __syncthreads();
+    // ---- logit of token lt for head lg (four partial sums for latency)
+    if (lg < G) {
+      const float* kr = ks + lt * kWinKStride;
+      const float* qr = qs + lg * kHeadDim;
+      float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+      for (int i = 0; i < kHeadDim; i += 4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) a[u] = fmaf(qr[i + u], kr[i + u], a[u]);
+      }
+      ps[lg * kWinSub + lt] = lt < n ? (a[0] + a[1]) + (a[2] + a[3]) : -INFINITY;
     }
+    __syncthreads();
+    // ---- one warp per head: running maximum, weights 2^(s - m), sum
+    for (int g = warp; g < G; g += kWinWarps) {
+      const float s = lane < kWinSub ? ps[g * kWinSub + lane] : -INFINITY;
+      float mx = s;
 #pragma unroll
-    for (int g = 0; g < 16; ++g) {
-      if (g >= G) break;
-      float s = 0.f;
+      for (int mm = 16; mm; mm >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, mm));
+      const float m_old = st[g], m_new = fmaxf(m_old, mx);
+      const bool none = m_new == -INFINITY;  // no finite logit yet
+      const float pr = none ? 0.f : ex2(s - m_new);
+      float sum = pr;
 #pragma unroll
-      for (int r = 0; r < 4; ++r) s = fmaf(qs[g * kHeadDim + lane + 32 * r], kx[r], s);
-#pragma unroll
-      for (int mm = 16; mm; mm >>= 1) s += __shfl_xor_sync(0xffffffffu, s, mm);
-      const float mn = fmaxf(m[g], s);
-      const float a = ex2(m[g] - mn), pr = ex2(s - mn);
-      l[g] = l[g] * a + pr;
-#pragma unroll
-      for (int r = 0; r < 4; ++r) o[g][r] = o[g][r] * a + pr * y[r];
-      m[g] = mn;
+      for (int mm = 16; mm; mm >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, mm);
+      if (lane < kWinSub) ps[g * kWinSub + lane] = pr;
+      if (lane == 0) {
+        const float alpha = none ? 1.f : ex2(m_old - m_new);  // 0 from -inf
+        st[32 + g] = alpha;
+        st[16 + g] = st[16 + g] * alpha + sum;
+        st[g] = m_new;
+      }
     }
+    __syncthreads();
+    // ---- o of coordinate ci for heads cg, cg + 2, ...: rescale, add the sub-chunk
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int g = cg + 2 * k;
+      if (g < G) {
+        const float* pg = ps + g * kWinSub;
+        float acc = o[k] * st[32 + g];
+#pragma unroll
+        for (int t = 0; t < kWinSub; ++t)
+          if (t < n) acc = fmaf(pg[t], ys[t * kHeadDim + ci], acc);
+        o[k] = acc;
+      }
+    }
+    __syncthreads();  // the next sub-chunk overwrites the staged rows
   }
-  // warps -> shared records -> one merged record per head
+  float* dst = recs + ((size_t)z * batch * n_q + (size_t)b * n_q + (size_t)h * G) * kPartStride;
 #pragma unroll
-  for (int g = 0; g < 16; ++g) {
-    if (g >= G) break;
-    float* dst = mg + ((size_t)warp * G + g) * kPartStride;
-    if (lane == 0) {
-      dst[0] = m[g];
-      dst[1] = l[g];
-    }
-#pragma unroll
-    for (int r = 0; r < 4; ++r) dst[kRecO + lane + 32 * r] = o[g][r];
+  for (int k = 0; k < 8; ++k) {
+    const int g = cg + 2 * k;
+    if (g < G) dst[(size_t)g * kPartStride + kRecO + ci] = o[k];
   }
-  __syncthreads();
-  merge_records<kWinThreads, kWinWarps>(mg, kWinWarps, (size_t)G * kPartStride, G,
-                                        recs + ((size_t)b * n_q + (size_t)h * G) * kPartStride);
+  if (tid < G) {
+    dst[(size_t)tid * kPartStride] = st[tid];
+    dst[(size_t)tid * kPartStride + 1] = st[16 + tid];
+    dst[(size_t)tid * kPartStride + 2] = 0.f;
+    dst[(size_t)tid * kPartStride + 3] = 0.f;
+  }
 }
 
-size_t window_record_smem(int G) {
-  return ((size_t)G * kHeadDim + (size_t)kWinWarps * G * kPartStride) * sizeof(float);
+// Window record parts of a window of R tokens: at most kWinParts CTAs per
+// (KV head, sequence), each over a multiple of 16 tokens.
+int window_parts(int R, int* tokens_per_part) {
+  const int P = std::max(1, std::min(kWinParts, (R + kWinSub - 1) / kWinSub));
+  const int per = (R + P - 1) / P;
+  *tokens_per_part = std::max(kWinSub, (per + kWinSub - 1) / kWinSub * kWinSub);
+  return P;
 }
 
 cudaError_t launch_window_push(const void* k, const void* v, int dtype, int n_new, int n_kv,
@@ -171,19 +240,10 @@ cudaError_t launch_window_record(const Plan* const* plans, const float* const* w
                                  const int32_t* len, const int32_t* wlen, int R, const void* q,
                                  int q_dtype, int n_q, int n_kv, int batch, float* recs,
                                  cudaStream_t st) {
-  static std::atomic<unsigned long long> cap_set{0};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  const unsigned long long bit = 1ull << (dev & 63);
-  if (!(cap_set.load() & bit)) {  // once per device: the largest query group
-    e = cudaFuncSetAttribute(window_record_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)window_record_smem(16));
-    if (e != cudaSuccess) return e;
-    cap_set.fetch_or(bit);
-  }
-  window_record_kernel<<<dim3(n_kv, batch), kWinThreads, window_record_smem(n_q / n_kv), st>>>(
-      plans, wins, len, wlen, R, q, q_dtype, n_q, n_kv, recs);
+  int C = kWinSub;
+  const int P = window_parts(R, &C);
+  window_record_kernel<<<dim3(n_kv, batch, P), kWinThreads, 0, st>>>(
+      plans, wins, len, wlen, R, C, q, q_dtype, n_q, n_kv, batch, recs);
   return cudaGetLastError();
 }
 

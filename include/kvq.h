@@ -468,12 +468,13 @@ KVQ_API int kvq_set_decode_deterministic(int on);
  *   wlen untouched). Two launches; no workspace.
  * kvq_decode_attn_window: kvq_decode_attn over the packed tokens (len_dev,
  *   max_len >= every len) and the window tokens (wlen_dev) together: one
- *   partial decode of the packed tokens, one record of the window tokens
+ *   partial decode of the packed tokens, the records of the window tokens
  *   (fp32 logits q.k log2(e)/sqrt(128) and values rotated like the packed
- *   ones), one combine; three launches. ws_dev: >=
+ *   ones; up to 32 parts of the window per KV head and sequence, in
+ *   parallel), one combine; three launches. ws_dev: >=
  *   kvq_window_decode_workspace_bytes(...) bytes, 16-byte aligned,
  *   zero-filled once, reuse rules of kvq_decode_attn; its first
- *   2 batch n_q_heads 132 floats (rounded up to 256 bytes) hold the two
+ *   33 batch n_q_heads 132 floats (rounded up to 256 bytes) hold the
  *   records, the rest serves the partial decode.
  * Both return KVQ_OK or a negative code.
  */

@@ -58,8 +58,11 @@ def _check_state(L, kb, vb, T, E, bits_k, bits_v, R, rng, G):
         assert op.rel_err(out[s], ref) <= TOL, (s, T, sp)
 
 
+# R = 260: 17 window record parts of 16 tokens, with evictions; R = 700: 32
+# parts of 32 tokens (two staged sub-chunks each) over a window that holds
+# every token, so most parts are empty
 @pytest.mark.parametrize("R,bits_k,bits_v,G", [(48, 3, 2, 4), (32, 2, 3, 8), (100, 4, 4, 16),
-                                               (1, 3, 3, 7)])
+                                               (1, 3, 3, 7), (260, 3, 3, 8), (700, 2, 2, 5)])
 def test_window_appends_and_decode(R, bits_k, bits_v, G):
     rng = np.random.default_rng(R * 7 + bits_k)
     n_kv, batch = 2, 2

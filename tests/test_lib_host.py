@@ -176,7 +176,8 @@ def test_window_sizes_and_argument_errors_without_gpu():
     assert kvq.window_bytes(cfg, 48) == 2 * 48 * 2 * 128 * 4
     assert kvq.window_bytes(cfg, 0) == 0 and kvq.window_bytes(cfg, -1) == 0
     d = kvq.decode_workspace_bytes(cfg, 3, 8, 1000)
-    assert kvq.window_decode_workspace_bytes(cfg, 3, 8, 1000) == d + (2 * 3 * 8 * 528 + 255) // 256 * 256
+    # the packed tokens' records and up to 32 window record parts
+    assert kvq.window_decode_workspace_bytes(cfg, 3, 8, 1000) == d + (33 * 3 * 8 * 528 + 255) // 256 * 256
     p = ctypes.c_void_p(256)
     # negative R, a null length array, a window call without its ring
     assert L.kvq_window_append(ctypes.byref(cfg), p, p, p, 0, 1, p, p, 100, p, p, -1, 1, p,
