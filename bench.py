@@ -738,10 +738,11 @@ def measure_point(args, wl, T, alloc, n_layers, rank, dev, stream, peak, steps):
 def measure_window(args, wl, T, R, n_layers, rank, dev, stream, peak, steps):
     """The recent-token window on a workload point: per layer a cache whose R
     most recent tokens stay exact (the prefill goes through the window, so
-    the oldest T - R tokens are packed), and a step of kvq_window_append (one
-    token: quantize the evicted token, push the new one) plus
-    kvq_decode_attn_window (partial decode over the packed tokens, the
-    window's record, combine) per layer; `steps` graph replays timed."""
+    the oldest T - R tokens are packed), and a step of
+    kvq_append_decode_window per layer (one token: one launch that
+    quantize-appends the token leaving the window, writes the new one to the
+    ring and decodes over the packed and the window tokens); `steps` graph
+    replays timed."""
     import torch
 
     from bit_kv_cache_19_b200 import kvq
@@ -769,8 +770,8 @@ def measure_window(args, wl, T, R, n_layers, rank, dev, stream, peak, steps):
 
     def step():
         for li, L in enumerate(layers):
-            L.append_window(knew[li], vnew[li])
-            L.decode_window(qs[li], out=outs[li], ws=ws)
+            L.append_decode_window(knew[li], vnew[li], qs[li], out=outs[li], ws=ws,
+                                   step_flags=kvq.STEP_EARLY)
 
     with torch.cuda.stream(stream):
         for _ in range(warmup):
@@ -793,9 +794,9 @@ def measure_window(args, wl, T, R, n_layers, rank, dev, stream, peak, steps):
            "budget": f"K{wl.bits_k}V{wl.bits_v}", "appended_per_step": n_step, "steps": steps,
            "ms_per_step": ms, "GB_per_s": (packed_bytes + ring_bytes) / (ms / 1e3) / 1e9,
            "frac": (packed_bytes + ring_bytes) / (ms / 1e3) / 1e9 / peak,
-           "launches_per_layer": 5,
-           "note": "bytes = packed tokens read by the partial decode + the fp32 window ring; "
-                   "the step is kvq_window_append + kvq_decode_attn_window per layer"}
+           "launches_per_layer": 1,
+           "note": "bytes = packed tokens read by the decode + the fp32 window ring; the step "
+                   "is one kvq_append_decode_window launch per layer"}
     graph = None
     del layers, qs, knew, vnew, outs, ws
     torch.cuda.empty_cache()

@@ -41,6 +41,13 @@ cudaError_t launch_window_record(const Plan* const* plans, const float* const* w
                                  int q_dtype, int n_q, int n_kv, int batch, float* recs,
                                  cudaStream_t st);
 int window_parts(int R, int* tokens_per_part);
+cudaError_t launch_decode_window(const Plan* const* plans, const CacheMap& cm, int32_t* len,
+                                 int batch, int64_t max_len, const void* q, int q_dtype, int n_q,
+                                 int n_kv, int bits_k, int bits_v, float* out, void* ws,
+                                 size_t ws_bytes, uint32_t* status, cudaStream_t st,
+                                 const void* k_new, const void* v_new, int kv_dtype,
+                                 int64_t cap, int early, float* const* wins, int32_t* wlen,
+                                 int R);
 constexpr int kWindowPartsMax = 32;  // window record parts per (KV head, sequence), at most
 
 namespace {
@@ -740,6 +747,54 @@ int kvq_decode_attn_window(const kvq_cfg* cfg, const void* const* plans_dev,
   e = launch_combine(reinterpret_cast<const Plan* const*>(plans_dev), recs, 1 + parts, batch,
                      n_q_heads, cfg->n_kv_heads, out_dev, st);
   if (e != cudaSuccess) return cuda_fail(e, "decode_attn_window (combine)");
+  return KVQ_OK;
+}
+
+int kvq_append_decode_window(const kvq_cfg* cfg, const void* const* plans_dev, const void* k_dev,
+                             const void* v_dev, int kv_dtype, int n_new, void* const* cache_dev,
+                             int32_t* len_dev, int64_t cap_tokens, void* const* win_dev,
+                             int32_t* wlen_dev, int R, int batch, int64_t max_len,
+                             const void* q_dev, int q_dtype, int n_q_heads, float* out_dev,
+                             void* ws_dev, size_t ws_bytes, int step_flags, uint32_t* status_dev,
+                             kvq_stream_t stream) {
+  int rc = check_cfg(cfg);
+  if (rc) return rc;
+  if (step_flags & ~KVQ_STEP_EARLY) return fail(KVQ_ERR_ARG, "step_flags 0x%x", step_flags);
+  if (R < 0 || R > (1 << 20)) return fail(KVQ_ERR_ARG, "window R %d", R);
+  if (n_new != 1 || R == 0) {  // the two calls
+    rc = kvq_window_append(cfg, plans_dev, k_dev, v_dev, kv_dtype, n_new, cache_dev, len_dev,
+                           cap_tokens, win_dev, wlen_dev, R, batch, status_dev, stream);
+    if (rc) return rc;
+    return kvq_decode_attn_window(cfg, plans_dev, reinterpret_cast<const void* const*>(cache_dev),
+                                  len_dev, reinterpret_cast<const void* const*>(win_dev), wlen_dev,
+                                  R, batch, max_len, q_dev, q_dtype, n_q_heads, out_dev, ws_dev,
+                                  ws_bytes, status_dev, stream);
+  }
+  if (!plans_dev || !cache_dev || !len_dev || !win_dev || !wlen_dev || !q_dev || !out_dev ||
+      !ws_dev || !status_dev || !k_dev || !v_dev)
+    return fail(KVQ_ERR_ARG, "null device pointer");
+  if (!dtype_ok(kv_dtype) || !dtype_ok(q_dtype)) return fail(KVQ_ERR_ARG, "bad dtype");
+  if (batch < 1 || batch > 65535) return fail(KVQ_ERR_ARG, "batch %d", batch);
+  if (max_len < 1 || max_len > 0x7FFFFFFF || cap_tokens < 0 || cap_tokens > 0x7FFFFFFF)
+    return fail(KVQ_ERR_ARG, "max_len %lld / cap_tokens %lld", (long long)max_len,
+                (long long)cap_tokens);
+  if (n_q_heads < 1 || n_q_heads % cfg->n_kv_heads != 0 || n_q_heads / cfg->n_kv_heads > 16)
+    return fail(KVQ_ERR_ARG, "n_q_heads %d vs n_kv_heads %d", n_q_heads, cfg->n_kv_heads);
+  if (reinterpret_cast<uintptr_t>(ws_dev) & 15)
+    return fail(KVQ_ERR_ARG, "decode workspace not 16-byte aligned");
+  if (ws_bytes < kvq_window_decode_workspace_bytes(cfg, batch, n_q_heads, max_len))
+    return fail(KVQ_ERR_WORKSPACE, "window decode workspace %zu < %zu", ws_bytes,
+                kvq_window_decode_workspace_bytes(cfg, batch, n_q_heads, max_len));
+  // the fused step uses the decode part of the workspace (after the records)
+  const size_t rb = window_records_bytes(batch, n_q_heads);
+  cudaError_t e = launch_decode_window(
+      reinterpret_cast<const Plan* const*>(plans_dev), contiguous_map(cache_dev), len_dev, batch,
+      max_len, q_dev, q_dtype, n_q_heads, cfg->n_kv_heads, cfg->bits_k, cfg->bits_v, out_dev,
+      reinterpret_cast<uint8_t*>(ws_dev) + rb, ws_bytes - rb, status_dev,
+      reinterpret_cast<cudaStream_t>(stream), k_dev, v_dev, kv_dtype, cap_tokens,
+      (step_flags & KVQ_STEP_EARLY) ? 1 : 0, reinterpret_cast<float* const*>(win_dev), wlen_dev,
+      R);
+  if (e != cudaSuccess) return cuda_fail(e, "append_decode_window");
   return KVQ_OK;
 }
 

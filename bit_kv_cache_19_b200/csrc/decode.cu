@@ -104,6 +104,11 @@ struct DecodeParams {
   int rope;   // appended keys are pre-RoPE: rotate each to its position first
   long long stall_cycles;  // test hook (> 0): each warp first waits that long in vain
   int deterministic;       // merge the split records in split order (no L2 atomics)
+  // recent-token window step (window kernels only): per sequence a ring of R
+  // fp32 rows (keys, then values; token t in slot t mod R) and its length
+  float* const* wins;
+  int32_t* wlen;
+  int R;
   double theta[64];
   uint8_t* pb_end;        // pair block of pair k at pb_end - (k + 1) * kPairBlockBytes
   float* part;            // [batch][n_kv][n_splits][G][132] = m, l, -, -, o[128]
@@ -125,6 +130,7 @@ struct alignas(128) Smem {
   double theta[64];                // RoPE block frequencies (fused append of pre-RoPE keys)
   int8_t qj[kMaxHalf][4];        // per half step: block of MMA column c, or -1
   int len0, is_last;
+  int w0;  // window step: the window's length before the step
   uint32_t flags;
   RotTables rot;                   // key rotation tables (plans with k_rot)
 };
@@ -298,7 +304,146 @@ __device__ __forceinline__ void warp_unrotate_store(const float* src, const Plan
   }
 }
 
-template <int BV, int NT>
+// Window step (window kernels): the CTA's share of the window after the
+// step, positions [w_lo, w_lo + w_n) of the sequence in chunks of 8 (chunk c
+// to split c mod n_splits). A position below new_from is read from its ring
+// slot; from new_from on it is a token of this step, read from the new rows
+// (its ring slot is written in this launch by another CTA). Logits in fp32,
+// s = (q . k) log2(e) / sqrt(128); values enter as H (s . v), the packed
+// values' rotation. The CTA's record of its chunks (base-2 maximum, sum, o)
+// goes to rec (8 NT records of kPartStride floats); returns whether it has
+// chunks. qs: [G][128] floats; wsc: window scratch (kWinScratch floats).
+constexpr int kWinTok = 8;  // window tokens staged at a time (one per warp)
+constexpr int kWinScratch = kWinTok * (kHeadDim + 1) + kWinTok * kHeadDim + 16 * kWinTok + 48;
+
+template <int NT>
+__device__ __forceinline__ bool window_chunks(const DecodeParams& p, const Plan& pl, int b, int h,
+                                           int split, int w_lo, int w_n, int64_t new_from,
+                                           float* qs, float* wsc, float* rec, int tid) {
+  if (split * kWinTok >= w_n) return false;  // CTA-uniform
+  const int G = p.G, warp = tid >> 5, lane = tid & 31;
+  float* ks = wsc;                            // [8][129]
+  float* ys = ks + kWinTok * (kHeadDim + 1);  // [8][128]
+  float* ps = ys + kWinTok * kHeadDim;        // [16][8]
+  float* st = ps + 16 * kWinTok;              // max, sum, rescale per head
+  for (int e = tid; e < G * kHeadDim; e += kThreads)
+    qs[e] = load_as_float(p.q, p.q_dtype, ((size_t)b * p.n_q + (size_t)h * G) * kHeadDim + e) *
+            0.12751743074f;  // log2(e) / sqrt(128)
+  if (tid < 16) {
+    st[tid] = -INFINITY;
+    st[16 + tid] = 0.f;
+  }
+  uint32_t vsgn = 0;  // value signs of this lane's coordinates lane + 32 r
+#pragma unroll
+  for (int r = 0; r < 4; ++r) vsgn |= ((pl.v_sign[r] >> lane) & 1u) << r;
+  const float* wk = p.wins[b];
+  const float* wv = wk + (size_t)p.R * p.n_kv * kHeadDim;
+  const int ci = tid & (kHeadDim - 1), cg = tid >> 7;  // o: coordinate, first head
+  const int lt = tid & (kWinTok - 1), lg = tid >> 3;   // logit: token, head
+  float o[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) o[k] = 0.f;
+  __syncthreads();
+  for (int c = split; c * kWinTok < w_n; c += p.n_splits) {
+    const int c0 = w_lo + c * kWinTok, n = min(kWinTok, w_n - c * kWinTok);
+    if (warp < n) {  // stage token `warp` of the chunk
+      const int64_t pos = (int64_t)c0 + warp;
+      float kx[4], y[4];
+      if (pos >= new_from) {
+        const size_t row = (((size_t)b * p.n_new + (size_t)(pos - new_from)) * p.n_kv + h) * kHeadDim;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          kx[r] = load_as_float(p.k_new, p.kv_dtype, row + lane + 32 * r);
+          const float x = load_as_float(p.v_new, p.kv_dtype, row + lane + 32 * r);
+          y[r] = ((vsgn >> r) & 1u) ? -x : x;
+        }
+      } else {
+        const size_t row = ((size_t)(pos % p.R) * p.n_kv + h) * kHeadDim;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          kx[r] = wk[row + lane + 32 * r];
+          const float x = wv[row + lane + 32 * r];
+          y[r] = ((vsgn >> r) & 1u) ? -x : x;
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) ks[warp * (kHeadDim + 1) + lane + 32 * r] = kx[r];
+      // y = H (s . v): butterflies h = 1..16 across lanes, then 32 and 64
+#pragma unroll
+      for (int hh = 1; hh < 32; hh <<= 1) {
+        const bool upper = (lane & hh) != 0;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const float x = __shfl_xor_sync(0xffffffffu, y[r], hh);
+          y[r] = upper ? x - y[r] : y[r] + x;
+        }
+      }
+      const float a0 = y[0] + y[1], a1 = y[0] - y[1], a2 = y[2] + y[3], a3 = y[2] - y[3];
+      ys[warp * kHeadDim + lane] = a0 + a2;
+      ys[warp * kHeadDim + lane + 32] = a1 + a3;
+      ys[warp * kHeadDim + lane + 64] = a0 - a2;
+      ys[warp * kHeadDim + lane + 96] = a1 - a3;
+    }
+    __syncthreads();
+    if (lg < G) {  // logit of token lt for head lg (four partial sums)
+      const float* kr = ks + lt * (kHeadDim + 1);
+      const float* qr = qs + lg * kHeadDim;
+      float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+      for (int i = 0; i < kHeadDim; i += 4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) a[u] = fmaf(qr[i + u], kr[i + u], a[u]);
+      }
+      ps[lg * kWinTok + lt] = lt < n ? (a[0] + a[1]) + (a[2] + a[3]) : -INFINITY;
+    }
+    __syncthreads();
+    for (int g = warp; g < G; g += kWarps) {  // running maximum, weights, sum
+      const float sv = lane < kWinTok ? ps[g * kWinTok + lane] : -INFINITY;
+      float mx = sv;
+#pragma unroll
+      for (int mm = 16; mm; mm >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, mm));
+      const float m_old = st[g], m_new = fmaxf(m_old, mx);
+      const bool none = m_new == -INFINITY;
+      const float pr = none ? 0.f : ex2(sv - m_new);
+      float sum = pr;
+#pragma unroll
+      for (int mm = 16; mm; mm >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, mm);
+      if (lane < kWinTok) ps[g * kWinTok + lane] = pr;
+      if (lane == 0) {
+        const float alpha = none ? 1.f : ex2(m_old - m_new);  // 0 from -inf
+        st[32 + g] = alpha;
+        st[16 + g] = st[16 + g] * alpha + sum;
+        st[g] = m_new;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {  // o of coordinate ci for heads cg, cg + 2, ...
+      const int g = cg + 2 * k;
+      if (g < G) {
+        const float* pg = ps + g * kWinTok;
+        float acc = o[k] * st[32 + g];
+#pragma unroll
+        for (int t = 0; t < kWinTok; ++t)
+          if (t < n) acc = fmaf(pg[t], ys[t * kHeadDim + ci], acc);
+        o[k] = acc;
+      }
+    }
+    __syncthreads();  // the next chunk overwrites the staged rows
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int g = cg + 2 * k;
+    if (g < 8 * NT) rec[(size_t)g * kPartStride + kRecO + ci] = g < G ? o[k] : 0.f;
+  }
+  if (tid < 8 * NT) {
+    rec[(size_t)tid * kPartStride] = tid < G ? st[tid] : -INFINITY;
+    rec[(size_t)tid * kPartStride + 1] = tid < G ? st[16 + tid] : 0.f;
+  }
+  return true;
+}
+
+template <int BV, int NT, bool WIN>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
@@ -345,6 +490,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   if (tid == 0) {
     const int l0 = p.len[b];
     sm.len0 = l0;
+    int w0 = 0;
+    if constexpr (WIN) {
+      w0 = min(max(p.wlen[b], 0), p.R);
+      sm.w0 = w0;
+    }
     if (p.n_new > 0) {
       // the last CTA of the sequence to read its length writes the new one;
       // the counter wraps to zero in the same atomic, so a kernel that starts
@@ -353,7 +503,15 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
       const unsigned int total = (unsigned int)(p.n_kv * p.n_splits);
       if (atomicInc(seq_cnt, total - 1u) == total - 1u) {
         const int64_t lim = min((int64_t)p.max_len, p.cap);
-        if (l0 >= 0 && (int64_t)l0 + p.n_new <= lim) p.len[b] = l0 + p.n_new;
+        if constexpr (WIN) {  // the tokens leaving the window join the packed cache
+          const int e = max(0, w0 + p.n_new - p.R);
+          if (l0 >= 0 && (int64_t)l0 + e <= lim) {
+            p.len[b] = l0 + e;
+            p.wlen[b] = min(p.R, w0 + p.n_new);
+          }
+        } else {
+          if (l0 >= 0 && (int64_t)l0 + p.n_new <= lim) p.len[b] = l0 + p.n_new;
+        }
       }
     }
   }
@@ -381,10 +539,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   if (bad && tid == 0) atomicOr(p.status, ok_setup ? KVQ_FLAG_BAD_PLAN : KVQ_FLAG_TIMEOUT);
   const int len0 = sm.len0;
   int n_add = 0;
+  bool step_ok = false;  // the step's append fits (window: its evictions)
   if (p.n_new > 0) {
     const int64_t lim = min((int64_t)p.max_len, p.cap);
-    if (len0 >= 0 && (int64_t)len0 + p.n_new <= lim) {
-      n_add = p.n_new;
+    int want = p.n_new;
+    if constexpr (WIN) want = max(0, sm.w0 + p.n_new - p.R);
+    if (len0 >= 0 && (int64_t)len0 + want <= lim) {
+      n_add = want;
+      step_ok = true;
     } else if (tid == 0 && split == 0 && h == 0) {
       atomicOr(p.status, KVQ_FLAG_CAPACITY);
     }
@@ -431,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   const int a_lo = n_add > 0 ? max(len0 / kTile, tb) : 1;
   const int a_hi = n_add > 0 ? min((len0 + n_add - 1) / kTile, te - 1) : 0;
   const bool appends = has_work && a_lo <= a_hi;
-  if (appends) {  // the new tokens' rows into L2 (no value read before the wait)
+  if (!WIN && appends) {  // the new tokens' rows into L2 (no value read before the wait)
     const size_t esz = (p.kv_dtype == KVQ_BF16 || p.kv_dtype == KVQ_FP16) ? 2 : 4;
     const int lines = (int)(kHeadDim * esz / 128);
     const int j0 = max(len0, a_lo * kTile) - len0, j1 = min(len0 + n_add, a_hi * kTile + kTile) - len0;
@@ -486,10 +648,19 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
       // pass 1 (one warp per new token; the word after the packed words, the
       // first norm word of the copy, takes only no-op atomics), then pass 2
       for (int pp = p_lo + warp; pp < p_hi; pp += kWarps) {
-        const size_t row =
-            (((size_t)b * p.n_new + (tile * kTile + pp - len0)) * p.n_kv + h) * kHeadDim;
+        const int j = tile * kTile + pp - len0;  // j-th appended token
+        size_t row = (((size_t)b * p.n_new + j) * p.n_kv + h) * kHeadDim;
+        const void* ksrc = p.k_new;
+        const void* vsrc = p.v_new;
+        int dt = p.kv_dtype;
+        if constexpr (WIN) {  // a token leaving the window: its ring row (fp32)
+          row = ((size_t)(((int64_t)len0 + j) % p.R) * p.n_kv + h) * kHeadDim;
+          ksrc = p.wins[b];
+          vsrc = p.wins[b] + (size_t)p.R * p.n_kv * kHeadDim;
+          dt = KVQ_FP32;
+        }
         __half kn, vn;
-        warp_token_pass<BV>(sm.plan, sm.thr, p.k_new, p.v_new, p.kv_dtype, row, lane, pp,
+        warp_token_pass<BV>(sm.plan, sm.thr, ksrc, vsrc, dt, row, lane, pp,
                             kz + pp * kKzStride, sw, clear, kn, vn, flags,
                             p.rope ? sm.theta : nullptr, (int64_t)tile * kTile + pp);
         if (lane == 0) {
@@ -523,6 +694,24 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
     fence_proxy_async();  // patched stages are later overwritten by bulk copies
     __syncthreads();
     if (tid == 0 && sm.flags) atomicOr(p.status, sm.flags);
+  }
+  if constexpr (WIN) {
+    // the new tokens into their ring slots, by the CTA that owns the last
+    // packed tile: it has just read the slots of the tokens that left the
+    // window (the append above), and no other CTA reads them in this launch
+    const int ring_split = min(p.n_splits - 1, ((max(L, 1) - 1) / kTile) / p.tiles_per_split);
+    if (step_ok && !bad && split == ring_split) {
+      float* wk = p.wins[b];
+      float* wv = wk + (size_t)p.R * p.n_kv * kHeadDim;
+      for (int e = tid; e < p.n_new * kHeadDim; e += kThreads) {
+        const int j = e / kHeadDim, x = e % kHeadDim;
+        const size_t dst =
+            ((size_t)(((int64_t)len0 + sm.w0 + j) % p.R) * p.n_kv + h) * kHeadDim + x;
+        const size_t src = (((size_t)b * p.n_new + j) * p.n_kv + h) * kHeadDim + x;
+        wk[dst] = load_as_float(p.k_new, p.kv_dtype, src);
+        wv[dst] = load_as_float(p.v_new, p.kv_dtype, src);
+      }
+    }
   }
 
   float o[8][NT][4];
@@ -754,6 +943,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
       }
     }
   __syncthreads();
+  int n_rec = kWarps;  // records of the CTA merge
+  if constexpr (WIN) {
+    // the window after the step: [L, L + w_n) (the step's new token last)
+    const int w_n = bad ? 0 : (step_ok ? min(p.R, sm.w0 + p.n_new) : sm.w0);
+    if (window_chunks<NT>(p, sm.plan, b, h, split, L, w_n, (int64_t)len0 + sm.w0,
+                          reinterpret_cast<float*>(scratch), mg + (kWarps + 1) * 8 * NT * kPartStride,
+                          mg + kWarps * 8 * NT * kPartStride, tid))
+      n_rec = kWarps + 1;
+    __syncthreads();
+  }
   // ---- this split's record, then its contribution to the exponent buckets:
   //      head hd with max m adds 2^(m - 32 kk) (l, o), kk = floor(m / 32), to
   //      bucket kk by L2 atomics, so the splits are summed in L2 without a
@@ -768,7 +967,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
     const int hd = item >> 5, x4 = (item & 31) * 4;
     float m, l;
     float4 ov;
-    merge_item<kWarps>(mg + hd * kPartStride, kWarps, (size_t)8 * NT * kPartStride, x4, m, l, ov);
+    merge_item<kWarps>(mg + hd * kPartStride, n_rec, (size_t)8 * NT * kPartStride, x4, m, l, ov);
     *reinterpret_cast<float4*>(crec + hd * kPartStride + kRecO + x4) = ov;
     *reinterpret_cast<float4*>(my_part + hd * kPartStride + kRecO + x4) = ov;
     if (x4 == 0) {
@@ -930,11 +1129,15 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const Plan* const* pl
 }
 
 // ------------------------------------------------------------- launchers
-size_t decode_smem_bytes(int tile_bytes, int nt) {
+size_t decode_smem_bytes(int tile_bytes, int nt, bool win = false) {
   const size_t stages = (size_t)kWarps * kStages * tile_bytes;
   const size_t merge = (size_t)kWarps * 8 * nt * kPartStride * sizeof(float);
-  return sizeof(Smem) + kScratch + std::max(stages, merge);
+  // window step: one more record (the window's) and the window scratch
+  const size_t merge_win =
+      ((size_t)(kWarps + 1) * 8 * nt * kPartStride + kWinScratch) * sizeof(float);
+  return sizeof(Smem) + kScratch + std::max(stages, win ? merge_win : merge);
 }
+static_assert(16 * kHeadDim * sizeof(float) <= (size_t)kScratch, "window q' in the scratch");
 
 // CTAs per SM of one instantiation for tiles of (bits_k, BV), queried once per
 // device and bits_k. The first query also raises the dynamic shared-memory cap
@@ -950,13 +1153,13 @@ static int ctas_per_sm(int dev, int bits_k, cudaError_t* err) {
   cudaError_t e = cudaSuccess;
   const unsigned long long bit = 1ull << (dev & 63);
   if (!(cap_set.load() & bit)) {
-    e = cudaFuncSetAttribute(decode_kernel<BV, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(decode_kernel<BV, NT, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)decode_smem_bytes(tile_bytes(8, BV), NT));
     if (e == cudaSuccess) cap_set.fetch_or(bit);
   }
   if (e == cudaSuccess)
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-        &v, decode_kernel<BV, NT>, kThreads, decode_smem_bytes(tile_bytes(bits_k, BV), NT));
+        &v, decode_kernel<BV, NT, false>, kThreads, decode_smem_bytes(tile_bytes(bits_k, BV), NT));
   if (e != cudaSuccess) {
     *err = e;
     return 0;
@@ -1047,32 +1250,46 @@ size_t decode_workspace_bytes_for(int batch, int n_q, int n_kv, int bits_k, int 
   return decode_workspace_layout((size_t)batch * n_kv, sp.slots);
 }
 
-template <int BV, int NT>
+template <int BV, int NT, bool WIN>
 static cudaError_t launch_decode_t(const DecodeParams& p, int batch, cudaStream_t st) {
+  if constexpr (WIN) {  // once per device: the window instantiation's cap, for its largest tile
+    static std::atomic<unsigned long long> cap_set{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (!(cap_set.load() & bit)) {
+      e = cudaFuncSetAttribute(decode_kernel<BV, NT, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)decode_smem_bytes(tile_bytes(8, BV), NT, true));
+      if (e != cudaSuccess) return e;
+      cap_set.fetch_or(bit);
+    }
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.n_splits, p.n_kv, batch);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = decode_smem_bytes(p.tile_bytes, NT);
+  cfg.dynamicSmemBytes = decode_smem_bytes(p.tile_bytes, NT, WIN);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<BV, NT>, p);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<BV, NT, WIN>, p);
 }
 
-template <int NT>
+template <int NT, bool WIN>
 static cudaError_t launch_decode_nt(const DecodeParams& p, int bits_v, int batch, cudaStream_t st) {
   switch (bits_v) {
-    case 1: return launch_decode_t<1, NT>(p, batch, st);
-    case 2: return launch_decode_t<2, NT>(p, batch, st);
-    case 3: return launch_decode_t<3, NT>(p, batch, st);
-    case 4: return launch_decode_t<4, NT>(p, batch, st);
-    case 5: return launch_decode_t<5, NT>(p, batch, st);
-    case 6: return launch_decode_t<6, NT>(p, batch, st);
-    case 7: return launch_decode_t<7, NT>(p, batch, st);
-    case 8: return launch_decode_t<8, NT>(p, batch, st);
+    case 1: return launch_decode_t<1, NT, WIN>(p, batch, st);
+    case 2: return launch_decode_t<2, NT, WIN>(p, batch, st);
+    case 3: return launch_decode_t<3, NT, WIN>(p, batch, st);
+    case 4: return launch_decode_t<4, NT, WIN>(p, batch, st);
+    case 5: return launch_decode_t<5, NT, WIN>(p, batch, st);
+    case 6: return launch_decode_t<6, NT, WIN>(p, batch, st);
+    case 7: return launch_decode_t<7, NT, WIN>(p, batch, st);
+    case 8: return launch_decode_t<8, NT, WIN>(p, batch, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -1091,12 +1308,13 @@ void set_decode_stall(long long cycles) { g_stall_cycles.store(cycles > 0 ? cycl
 static std::atomic<int> g_deterministic{0};
 void set_decode_deterministic(int on) { g_deterministic.store(on ? 1 : 0); }
 
-cudaError_t launch_decode(const Plan* const* plans, const CacheMap& cm, int32_t* len,
-                          int batch, int64_t max_len, const void* q, int q_dtype, int n_q, int n_kv,
-                          int bits_k, int bits_v, float* out, void* ws, size_t ws_bytes,
-                          uint32_t* status, cudaStream_t st, const void* k_new,
-                          const void* v_new, int kv_dtype, int n_new, int64_t cap, int early,
-                          const double* theta, float* rec_out) {
+static cudaError_t launch_decode_any(const Plan* const* plans, const CacheMap& cm, int32_t* len,
+                                     int batch, int64_t max_len, const void* q, int q_dtype,
+                                     int n_q, int n_kv, int bits_k, int bits_v, float* out,
+                                     void* ws, size_t ws_bytes, uint32_t* status, cudaStream_t st,
+                                     const void* k_new, const void* v_new, int kv_dtype,
+                                     int n_new, int64_t cap, int early, const double* theta,
+                                     float* rec_out, float* const* wins, int32_t* wlen, int R) {
   cudaError_t err = cudaSuccess;
   const int G = n_q / n_kv;
   const SplitPlan sp = decode_split_plan(batch, n_kv, G, bits_k, bits_v, max_len, &err, false);
@@ -1133,8 +1351,41 @@ cudaError_t launch_decode(const Plan* const* plans, const CacheMap& cm, int32_t*
   p.out = out;
   p.rec_out = rec_out;
   p.status = status;
-  return G <= 8 ? launch_decode_nt<1>(p, bits_v, batch, st)
-                : launch_decode_nt<2>(p, bits_v, batch, st);
+  p.wins = wins;
+  p.wlen = wlen;
+  p.R = R;
+  if (wins)
+    return G <= 8 ? launch_decode_nt<1, true>(p, bits_v, batch, st)
+                  : launch_decode_nt<2, true>(p, bits_v, batch, st);
+  return G <= 8 ? launch_decode_nt<1, false>(p, bits_v, batch, st)
+                : launch_decode_nt<2, false>(p, bits_v, batch, st);
+}
+
+cudaError_t launch_decode(const Plan* const* plans, const CacheMap& cm, int32_t* len,
+                          int batch, int64_t max_len, const void* q, int q_dtype, int n_q, int n_kv,
+                          int bits_k, int bits_v, float* out, void* ws, size_t ws_bytes,
+                          uint32_t* status, cudaStream_t st, const void* k_new,
+                          const void* v_new, int kv_dtype, int n_new, int64_t cap, int early,
+                          const double* theta, float* rec_out) {
+  return launch_decode_any(plans, cm, len, batch, max_len, q, q_dtype, n_q, n_kv, bits_k, bits_v,
+                           out, ws, ws_bytes, status, st, k_new, v_new, kv_dtype, n_new, cap,
+                           early, theta, rec_out, nullptr, nullptr, 0);
+}
+
+// The window step in one launch: one new token per sequence (n_new = 1), the
+// token leaving a full window quantize-appended from its ring slot, the new
+// token written to the ring, decode over the packed tokens and the window.
+cudaError_t launch_decode_window(const Plan* const* plans, const CacheMap& cm, int32_t* len,
+                                 int batch, int64_t max_len, const void* q, int q_dtype, int n_q,
+                                 int n_kv, int bits_k, int bits_v, float* out, void* ws,
+                                 size_t ws_bytes, uint32_t* status, cudaStream_t st,
+                                 const void* k_new, const void* v_new, int kv_dtype,
+                                 int64_t cap, int early, float* const* wins, int32_t* wlen,
+                                 int R) {
+  if (!wins || !wlen || R < 1) return cudaErrorInvalidValue;
+  return launch_decode_any(plans, cm, len, batch, max_len, q, q_dtype, n_q, n_kv, bits_k, bits_v,
+                           out, ws, ws_bytes, status, st, k_new, v_new, kv_dtype, 1, cap, early,
+                           nullptr, nullptr, wins, wlen, R);
 }
 
 cudaError_t launch_combine(const Plan* const* plans, const float* recs, int n_parts, int batch,

@@ -121,6 +121,9 @@ _SIGS = {
     "kvq_window_decode_workspace_bytes": (_sz, [ctypes.POINTER(Cfg), _i32, _i32, _i64]),
     "kvq_decode_attn_window": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _vp, _vp, _i32, _i32,
                                       _i64, _vp, _i32, _i32, _vp, _vp, _sz, _vp, _vp]),
+    "kvq_append_decode_window": (_i32, [ctypes.POINTER(Cfg), _vp, _vp, _vp, _i32, _i32, _vp, _vp,
+                                        _i64, _vp, _vp, _i32, _i32, _i64, _vp, _i32, _i32, _vp,
+                                        _vp, _sz, _i32, _vp, _vp]),
 }
 EXPORTS = tuple(_SIGS)
 
@@ -424,6 +427,19 @@ def window_append(cfg, plan_ptrs, k, v, cache_ptrs, lens, cap_tokens, win_ptrs, 
                                    _dtype_code(k), n_new, _ptr(cache_ptrs), _ptr(lens),
                                    cap_tokens, _ptr(win_ptrs), _ptr(wlens), R, batch,
                                    _ptr(status), _stream()))
+
+
+def append_decode_window(cfg, plan_ptrs, k, v, cache_ptrs, lens, cap_tokens, win_ptrs, wlens, R,
+                         max_len, q, out, ws, status, step_flags=0):
+    """Window append of k, v [batch, n_new, n_kv, 128] then decode of q
+    [batch, n_q, 128]; one launch for n_new = 1."""
+    batch, n_new = k.shape[0], k.shape[1]
+    _check(lib().kvq_append_decode_window(ctypes.byref(cfg), _ptr(plan_ptrs), _ptr(k), _ptr(v),
+                                          _dtype_code(k), n_new, _ptr(cache_ptrs), _ptr(lens),
+                                          cap_tokens, _ptr(win_ptrs), _ptr(wlens), R, batch,
+                                          max_len, _ptr(q), _dtype_code(q), q.shape[1], _ptr(out),
+                                          _ptr(ws), ws.numel() * ws.element_size(), step_flags,
+                                          _ptr(status), _stream()))
 
 
 def decode_attn_window(cfg, plan_ptrs, cache_ptrs, lens, win_ptrs, wlens, R, max_len, q, out,

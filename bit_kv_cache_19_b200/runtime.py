@@ -107,6 +107,21 @@ class PackedLayer:
                                self.status)
         return out
 
+    def append_decode_window(self, k, v, q, out=None, ws=None, max_len=None, step_flags=0):
+        """One window step: append k, v [batch, n_new, n_kv, 128] through the
+        window and decode q [batch, n_q, 128] over packed + window tokens (one
+        launch for n_new = 1)."""
+        max_len = self.cap if max_len is None else max_len
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=self.device)
+        if ws is None:
+            n = kvq.window_decode_workspace_bytes(self.cfg, self.batch, q.shape[1], max_len)
+            ws = torch.zeros(n, dtype=torch.uint8, device=self.device)
+        kvq.append_decode_window(self.cfg, self.plan_ptrs, k, v, self.cache_ptrs, self.lens,
+                                 self.cap, self.win_ptrs, self.wlens, self.window, max_len, q, out,
+                                 ws, self.status, step_flags)
+        return out
+
     def window_rows(self, seq: int):
         """The window ring of one sequence on the host: keys, values fp32
         [R, n_kv, 128] (slot t mod R holds token t)."""

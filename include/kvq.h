@@ -494,6 +494,35 @@ KVQ_API int kvq_decode_attn_window(const kvq_cfg* cfg, const void* const* plans_
                                    uint32_t* status_dev, kvq_stream_t stream);
 
 /*
+ * A serving step with the recent-token window: kvq_window_append of n_new
+ * tokens per sequence, then kvq_decode_attn_window, with the same results
+ * (outputs to fp32 rounding). For n_new = 1 and R >= 1 it is one launch of
+ * the decode kernel: the CTA that owns the last packed tile quantize-appends
+ * the token leaving a full window (read from its ring slot) and then writes
+ * the new token into that slot; the window's other tokens (from the ring)
+ * and the new one (from k_dev, v_dev) are attended in chunks of 8 by a few
+ * CTAs after their tiles, each chunk's record merged with the CTA's own; the
+ * last CTA of the sequence to read the lengths writes len += evicted and
+ * wlen = min(R, wlen + 1). Other n_new (or R = 0) run the two calls.
+ * Arguments as for those calls; the evictions must fit min(cap_tokens,
+ * max_len) (else CAPACITY and the sequence's window is left as it was).
+ * step_flags: KVQ_STEP_EARLY as for kvq_append_decode (the previous kernel on
+ * the stream then writes neither the caches, the lengths nor the rings);
+ * KVQ_STEP_ROPE is refused (the window holds the keys as given).
+ * ws_dev: >= kvq_window_decode_workspace_bytes(...) bytes, rules as for
+ * kvq_decode_attn_window; the fused and the two-call forms may alternate
+ * on one workspace.
+ */
+KVQ_API int kvq_append_decode_window(const kvq_cfg* cfg, const void* const* plans_dev,
+                                     const void* k_dev, const void* v_dev, int kv_dtype,
+                                     int n_new, void* const* cache_dev, int32_t* len_dev,
+                                     int64_t cap_tokens, void* const* win_dev, int32_t* wlen_dev,
+                                     int R, int batch, int64_t max_len, const void* q_dev,
+                                     int q_dtype, int n_q_heads, float* out_dev, void* ws_dev,
+                                     size_t ws_bytes, int step_flags, uint32_t* status_dev,
+                                     kvq_stream_t stream);
+
+/*
  * One serving step in one launch: kvq_quantize_append of n_new tokens per
  * sequence followed by kvq_decode_attn over the grown caches (the pages'
  * packed-cache serving path: append the step's keys and values, then decode).

@@ -180,3 +180,83 @@ def test_window_with_rotated_keys_and_other_input_types(dtype):
                             [x["vhat"] for x in heads], [x[sp:] for x in kh],
                             [x[sp:] for x in vh])
         assert op.rel_err(out[s_], ref) <= TOL
+
+
+def _oracle_out(L, kb, vb, T, E, bits_k, bits_v, R, qb, s):
+    """fp64 oracle output of sequence s after T tokens (packed ones
+    dequantized, window ones exact) for queries qb (bf16 bits)."""
+    n_kv = L.cfg.n_kv_heads
+    sp = window.split_point(T, R)
+    kh, vh = op.bf16_heads(kb[s, :T], vb[s, :T])
+    heads = op.layer([x[:sp] for x in kh], [x[:sp] for x in vh], bits_k, bits_v, V_SEED, 0,
+                     E=E, pack=False)[1] if sp else None
+    empty = [np.zeros((0, 128))] * n_kv
+    return window.decode(synth.bf16_bits_to_f64(qb), [x["khat"] for x in heads] if sp else empty,
+                         [x["vhat"] for x in heads] if sp else empty, [x[sp:] for x in kh],
+                         [x[sp:] for x in vh])
+
+
+# one-token window steps in one launch (kvq_append_decode_window) against the
+# two calls (kvq_window_append + kvq_decode_attn_window) and the oracle: full
+# windows (an eviction every step), windows still filling (T0 < R), R = 1,
+# a 16-head query group (two MMA n-tiles) and a window of 17 tokens
+@pytest.mark.parametrize("R,T0,bits_k,bits_v,G", [(48, 300, 3, 3, 8), (64, 20, 3, 2, 4),
+                                                  (1, 100, 2, 2, 8), (100, 130, 4, 3, 16),
+                                                  (17, 64, 3, 3, 7)])
+def test_fused_window_steps(R, T0, bits_k, bits_v, G):
+    rng = np.random.default_rng(R * 13 + T0)
+    n_kv, batch, S = 2, 2, 40
+    T = T0 + S
+    cfg = kvq.make_cfg(n_kv, bits_k, bits_v, v_seed=V_SEED)
+    E = np.exp(rng.standard_normal((n_kv, 64)) - np.arange(64) / 8.0)
+    plans = kvq.plan_build(cfg, 0, E)
+    Lf = PackedLayer(cfg, batch, T + 32, window=R)  # fused steps
+    Lu = PackedLayer(cfg, batch, T + 32, window=R)  # the two calls
+    for L in (Lf, Lu):
+        L.set_plans(plans)
+    kb, vb = _inputs(rng, batch, T, n_kv)
+    for L in (Lf, Lu):
+        L.append_window(dev_bf16(kb[:, :T0]), dev_bf16(vb[:, :T0]))
+    nb = kvq.window_decode_workspace_bytes(cfg, batch, n_kv * G, T + 32)
+    wsf = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+    wsu = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+    qbs = synth.to_bf16_bits(rng.standard_normal((S, batch, n_kv * G, 128)))
+    for i in range(S):
+        t = T0 + i
+        k1, v1, q = dev_bf16(kb[:, t:t + 1]), dev_bf16(vb[:, t:t + 1]), dev_bf16(qbs[i])
+        out_f = Lf.append_decode_window(k1, v1, q, ws=wsf).cpu().numpy()
+        Lu.append_window(k1, v1)
+        out_u = Lu.decode_window(q, ws=wsu).cpu().numpy()
+        torch.cuda.synchronize()
+        assert Lf.flags() == 0 and Lu.flags() == 0, i
+        assert op.rel_err(out_f, out_u) <= 1e-5, i
+        if i in (0, 1, S // 2, S - 1):
+            for s in range(batch):
+                ref = _oracle_out(Lf, kb, vb, t + 1, E, bits_k, bits_v, R, qbs[i][s], s)
+                assert op.rel_err(out_f[s], ref) <= TOL, (i, s)
+    # the same packed caches, rings and lengths as the two calls
+    assert torch.equal(Lf.lens, Lu.lens) and torch.equal(Lf.wlens, Lu.wlens)
+    for s in range(batch):
+        assert torch.equal(Lf.caches[s], Lu.caches[s])
+        assert torch.equal(Lf.wins[s], Lu.wins[s])
+    _check_state(Lf, kb, vb, T, E, bits_k, bits_v, R, rng, G)
+
+
+def test_fused_window_step_capacity_leaves_sequence():
+    # an eviction that does not fit the capacity: CAPACITY, nothing moves
+    rng = np.random.default_rng(31)
+    n_kv, R, cap = 1, 8, 32
+    cfg = kvq.make_cfg(n_kv, 2, 2, v_seed=V_SEED)
+    L = PackedLayer(cfg, 1, cap, window=R)
+    L.set_plans(kvq.plan_build(cfg, 0, np.exp(rng.standard_normal((n_kv, 64)))))
+    kb, vb = _inputs(rng, 1, 41, n_kv)
+    L.append_window(dev_bf16(kb[:, :40]), dev_bf16(vb[:, :40]))  # 32 packed (full), 8 in the ring
+    torch.cuda.synchronize()
+    assert L.lens.item() == 32 and L.wlens.item() == 8 and L.flags() == 0
+    ring = L.wins[0].clone()
+    q = dev_bf16(synth.to_bf16_bits(rng.standard_normal((1, 4, 128))))
+    L.append_decode_window(dev_bf16(kb[:, 40:41]), dev_bf16(vb[:, 40:41]), q)
+    torch.cuda.synchronize()
+    assert L.flags() & kvq.FLAG_CAPACITY
+    assert L.lens.item() == 32 and L.wlens.item() == 8
+    assert torch.equal(ring, L.wins[0])
