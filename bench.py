@@ -517,6 +517,7 @@ def run_kvq(args, wl, rank, world, dist):
     #      dense launch per layer, lengths as in the packed step, graph)
     peak, peak_kind = measured_peaks()
     bf16 = None
+    fa2 = None
     if not args.no_bf16:
         dlen = torch.full((B,), int(layers[0].lens[0].item()), dtype=torch.int32, device=dev)
         dws = torch.zeros(kvq.bf16_decode_workspace_bytes(B, wl.n_kv_heads, wl.n_q_heads, cap),
@@ -556,6 +557,8 @@ def run_kvq(args, wl, rank, world, dist):
                 "note": "decode only (no append); dense_step_at_copy_bw_ms = the bf16 cache "
                         "bytes at the measured copy bandwidth, the time any dense decode of "
                         "this step needs at least"}
+        fa2 = fa2_comparator(dense_k, dense_v, dlen, cap, qs, n_layers, stream, steps, warmup,
+                             ms, peak, dist, dev, world, dout)
         del dense_k, dense_v
         torch.cuda.empty_cache()
 
@@ -668,11 +671,69 @@ def run_kvq(args, wl, rank, world, dist):
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "bf16_comparator": bf16,
+        "flash_attn_comparator": fa2,
         "workloads": extras,
         "gpu_launches": steps * n_layers,
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)
+
+
+def fa2_comparator(dense_k, dense_v, dlen, cap, qs, n_layers, stream, steps, warmup, packed_ms,
+                   peak, dist, dev, world, ref_out):
+    """The pages' own yardstick: FlashAttention-2 decode (flash_attn's
+    flash_attn_with_kvcache, library code) over the same unquantized caches,
+    bf16 (the pages name fp16; same bytes), one call per layer, graph-captured.
+    Its caches are [batch][cap][n_kv][128] copies of the comparator's. Returns
+    None if flash_attn is not importable, or an "unavailable" record if its
+    kernels do not run here."""
+    import torch
+
+    try:
+        from flash_attn import flash_attn_with_kvcache
+        import flash_attn
+    except Exception:
+        return None
+    try:
+        kf = [k.permute(0, 2, 1, 3).contiguous() for k in dense_k]
+        vf = [v.permute(0, 2, 1, 3).contiguous() for v in dense_v]
+        B, n_q = qs[0].shape[0], qs[0].shape[1]
+        fout = [None] * n_layers
+
+        def step():
+            for li in range(n_layers):
+                fout[li] = flash_attn_with_kvcache(qs[li].view(B, 1, n_q, 128), kf[li], vf[li],
+                                                   cache_seqlens=dlen,
+                                                   softmax_scale=128 ** -0.5)
+        with torch.cuda.stream(stream):
+            for _ in range(warmup):
+                step()
+            stream.synchronize()
+            if dist is not None:
+                dist.barrier()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                step()
+            fms = time_replays(graph.replay, stream, steps, None)
+            stream.synchronize()
+        fms = rank_max(fms, dist, dev)
+        # agreement with the bf16 comparator's output of the last layer
+        a = fout[n_layers - 1].float().view(B, n_q, 128)
+        b = ref_out[n_layers - 1]
+        rel = float(((a - b).abs().amax() / b.abs().amax()).item())
+        fbytes = n_layers * B * kf[0].shape[2] * 512 * int(dlen[0].item())
+        del kf, vf, graph
+        torch.cuda.empty_cache()
+        return {"kernel": f"flash_attn {flash_attn.__version__} flash_attn_with_kvcache (library)",
+                "ms_per_step": fms, "value": job_rate(fbytes, world, fms) / 1e9, "unit": "GB/s",
+                "frac": fbytes / (fms / 1e3) / 1e9 / peak, "bytes_per_step": fbytes,
+                "packed_step_speedup": fms / packed_ms,
+                "max_rel_diff_vs_bf16_comparator": rel,
+                "note": "bf16 K/V caches (the pages compare against fp16 FlashAttention-2 at "
+                        "128K); decode only, one call per layer, graph-captured"}
+    except Exception as e:  # e.g. no kernel image for this GPU
+        torch.cuda.synchronize()
+        return {"unavailable": str(e).splitlines()[0][:200]}
 
 
 def measure_point(args, wl, T, alloc, n_layers, rank, dev, stream, peak, steps):
