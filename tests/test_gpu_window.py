@@ -260,3 +260,29 @@ def test_fused_window_step_capacity_leaves_sequence():
     assert L.flags() & kvq.FLAG_CAPACITY
     assert L.lens.item() == 32 and L.wlens.item() == 8
     assert torch.equal(ring, L.wins[0])
+
+
+def test_window_step_of_several_tokens_is_the_two_calls():
+    # n_new > 1: kvq_append_decode_window runs kvq_window_append and
+    # kvq_decode_attn_window, so its state equals theirs and its output agrees
+    rng = np.random.default_rng(41)
+    n_kv, batch, R, G = 2, 2, 24, 8
+    cfg = kvq.make_cfg(n_kv, 3, 3, v_seed=V_SEED)
+    plans = kvq.plan_build(cfg, 0, np.exp(rng.standard_normal((n_kv, 64))))
+    La, Lb = PackedLayer(cfg, batch, 256, window=R), PackedLayer(cfg, batch, 256, window=R)
+    for L in (La, Lb):
+        L.set_plans(plans)
+    kb, vb = _inputs(rng, batch, 120, n_kv)
+    t = 0
+    for n in (50, 5, 17, 3):
+        k, v = dev_bf16(kb[:, t:t + n]), dev_bf16(vb[:, t:t + n])
+        q = dev_bf16(synth.to_bf16_bits(rng.standard_normal((batch, n_kv * G, 128))))
+        oa = La.append_decode_window(k, v, q).cpu().numpy()
+        Lb.append_window(k, v)
+        ob = Lb.decode_window(q).cpu().numpy()
+        t += n
+        torch.cuda.synchronize()
+        assert La.flags() == 0 and op.rel_err(oa, ob) <= 1e-5
+    assert torch.equal(La.lens, Lb.lens) and torch.equal(La.wlens, Lb.wlens)
+    for s in range(batch):
+        assert torch.equal(La.caches[s], Lb.caches[s]) and torch.equal(La.wins[s], Lb.wins[s])

@@ -192,6 +192,17 @@ def test_window_sizes_and_argument_errors_without_gpu():
     assert L.kvq_decode_attn_window(ctypes.byref(cfg), p, p, p, p, p, 8, 1, 100, p, 0, 8, p, p,
                                     kvq.decode_workspace_bytes(cfg, 1, 8, 100), p,
                                     None) == kvq.ERR_WORKSPACE
+    # the one-launch window step: no RoPE flag, R >= 0, the window decode workspace
+    ad = L.kvq_append_decode_window
+    wsb = kvq.window_decode_workspace_bytes(cfg, 1, 8, 100)
+    assert ad(ctypes.byref(cfg), p, p, p, 0, 1, p, p, 100, p, p, 8, 1, 100, p, 0, 8, p, p, wsb,
+              kvq.STEP_ROPE, p, None) == kvq.ERR_ARG
+    assert ad(ctypes.byref(cfg), p, p, p, 0, 1, p, p, 100, p, p, -1, 1, 100, p, 0, 8, p, p, wsb,
+              0, p, None) == kvq.ERR_ARG
+    assert ad(ctypes.byref(cfg), p, p, p, 0, 1, p, p, 100, None, p, 8, 1, 100, p, 0, 8, p, p, wsb,
+              0, p, None) == kvq.ERR_ARG
+    assert ad(ctypes.byref(cfg), p, p, p, 0, 1, p, p, 100, p, p, 8, 1, 100, p, 0, 8, p, p,
+              wsb - 256, 0, p, None) == kvq.ERR_WORKSPACE
 
 
 def test_argument_errors_without_gpu():
