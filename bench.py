@@ -113,11 +113,21 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def code_only(text):
+    """C++ source without comments and blank space: what the compiler sees,
+    so a comment edit does not retire counters taken on the same code."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def decode_source_hash():
+    """Hash of the decode kernel's code (its source files, comments left out)."""
     h = hashlib.sha256()
     for f in ("decode.cu", "common.cuh", "splitk.cuh", "quant_dev.cuh"):
-        with open(os.path.join(ROOT, "bit_kv_cache_19_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "bit_kv_cache_19_b200", "csrc", f)) as fh:
+            h.update(code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

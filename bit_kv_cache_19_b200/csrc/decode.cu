@@ -308,7 +308,7 @@ __device__ __forceinline__ void warp_unrotate_store(const float* src, const Plan
 // step, positions [w_lo, w_lo + w_n) of the sequence in chunks of 8 (chunk c
 // to split c mod n_splits). A position below new_from is read from its ring
 // slot; from new_from on it is a token of this step, read from the new rows
-// (its ring slot is written in this launch by another CTA). Logits in fp32,
+// (its ring slot is being written in this launch). Logits in fp32,
 // s = (q . k) log2(e) / sqrt(128); values enter as H (s . v), the packed
 // values' rotation. The CTA's record of its chunks (base-2 maximum, sum, o)
 // goes to rec (8 NT records of kPartStride floats); returns whether it has
