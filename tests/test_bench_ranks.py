@@ -67,3 +67,18 @@ def test_single_process_helpers():
 
     assert bench.rank_max(4.0, None) == 4.0
     assert bench.job_rate(10.0, 1, 1.0) == pytest.approx(1e4)
+
+
+def test_percentiles_and_code_hash():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    st = bench.percentiles([5.0, 1.0, 3.0, 2.0, 4.0])
+    assert (st["n"], st["min"], st["p50"], st["max"]) == (5, 1.0, 3.0, 5.0)
+    assert st["mean"] == pytest.approx(3.0)
+    # the traffic record is keyed by code, not comments or layout
+    a = "int f(int x) {  // one\n  /* two\n three */ return x + 1;\n}\n"
+    b = "int f(int x) {\n\n  return x + 1;   // other words\n}"
+    c = "int f(int x) { return x + 2; }"
+    assert bench.code_only(a) == bench.code_only(b) != bench.code_only(c)
+    assert len(bench.decode_source_hash()) == 16
