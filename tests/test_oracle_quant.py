@@ -125,6 +125,50 @@ def test_key_mse_matches_lloydmax(b):
     assert abs(rel - lloydmax.D(b)) / lloydmax.D(b) < 0.03
 
 
+def _sphere_distortion(b, d=128):
+    """E[(x - q_b(x))^2] for x = sqrt(d) u_1, u uniform on the unit sphere of
+    R^d (the coordinate a token's normalised vector presents to the
+    quantizer), q_b the frozen centroids and thresholds of width b. The
+    coordinate's density is C (1 - x^2 / d)^((d - 3) / 2) on [-sqrt(d),
+    sqrt(d)] with C = Gamma(d/2) / (Gamma((d-1)/2) sqrt(pi d)); integrated
+    cell by cell by quadrature."""
+    from scipy import integrate, special
+
+    logc = special.gammaln(d / 2) - special.gammaln((d - 1) / 2) - 0.5 * np.log(np.pi * d)
+
+    def dens(x):
+        return np.exp(logc + (d - 3) / 2 * np.log1p(-x * x / d))
+
+    c = lloydmax.centroids(b)
+    edges = np.concatenate([[-np.sqrt(d)], lloydmax.thresholds(b).astype(np.float64),
+                            [np.sqrt(d)]])
+    return sum(integrate.quad(lambda x: (x - c[k]) ** 2 * dens(x), edges[k], edges[k + 1],
+                              limit=200, epsabs=1e-15, epsrel=1e-12)[0] for k in range(len(c)))
+
+
+@pytest.mark.parametrize("b", range(1, 9))
+def test_mse_matches_sphere_quadrature_every_width(b):
+    # keys and values of isotropic Gaussian tokens: after the norm (and, for
+    # values, the rotation) each coordinate is sqrt(128) times a coordinate of
+    # a uniform unit vector, so the relative MSE is the quantizer's exact
+    # distortion under that density (a little below the Gaussian D(b)); 4000
+    # tokens give about 0.5 % of sampling spread
+    plan = _plan([b] * 64, b, b)
+    ds = _sphere_distortion(b)
+    rng = np.random.default_rng(300 + b)
+    k = rng.standard_normal((4000, 128)).astype(np.float32)
+    codes, n, _ = quant.quantize_keys(k, plan)
+    kh = attn.dequant_keys(codes, n, plan)
+    rel_k = np.sum((kh - k) ** 2) / np.sum(k.astype(np.float64) ** 2)
+    v = rng.standard_normal((4000, 128)).astype(np.float32)
+    codes, n, _ = quant.quantize_values(v, plan)
+    vh = attn.dequant_values(codes, n, plan)
+    rel_v = np.sum((vh - v) ** 2) / np.sum(v.astype(np.float64) ** 2)
+    assert abs(rel_k - ds) / ds < 0.02, (rel_k, ds)
+    assert abs(rel_v - ds) / ds < 0.02, (rel_v, ds)
+    assert ds < lloydmax.D(b)  # lighter tails than the Gaussian
+
+
 def test_key_block_widths_respected():
     w = np.zeros(64, dtype=int)
     w[[0, 1, 2]] = [8, 3, 1]
