@@ -41,6 +41,7 @@ cudaError_t launch_window_record(const Plan* const* plans, const float* const* w
                                  int q_dtype, int n_q, int n_kv, int batch, float* recs,
                                  cudaStream_t st);
 int window_parts(int R, int* tokens_per_part);
+int window_parts_max();
 cudaError_t launch_decode_window(const Plan* const* plans, const CacheMap& cm, int32_t* len,
                                  int batch, int64_t max_len, const void* q, int q_dtype, int n_q,
                                  int n_kv, int bits_k, int bits_v, float* out, void* ws,
@@ -48,7 +49,6 @@ cudaError_t launch_decode_window(const Plan* const* plans, const CacheMap& cm, i
                                  const void* k_new, const void* v_new, int kv_dtype,
                                  int64_t cap, int early, float* const* wins, int32_t* wlen,
                                  int R);
-constexpr int kWindowPartsMax = 32;  // window record parts per (KV head, sequence), at most
 
 namespace {
 
@@ -699,10 +699,10 @@ int kvq_window_append(const kvq_cfg* cfg, const void* const* plans_dev, const vo
   return KVQ_OK;
 }
 
-// The packed tokens' records, then up to kWindowPartsMax window record parts.
+// The packed tokens' records, then up to window_parts_max() window record parts.
 static size_t window_records_bytes(int batch, int n_q_heads) {
-  return ((size_t)(1 + kWindowPartsMax) * batch * n_q_heads * kRecFloats * sizeof(float) + 255) /
-         256 * 256;
+  return ((size_t)(1 + window_parts_max()) * batch * n_q_heads * kRecFloats * sizeof(float) +
+          255) / 256 * 256;
 }
 
 size_t kvq_window_decode_workspace_bytes(const kvq_cfg* cfg, int batch, int n_q_heads,

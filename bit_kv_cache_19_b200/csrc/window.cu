@@ -29,7 +29,7 @@ namespace kvq {
 
 constexpr int kWinThreads = 256;
 constexpr int kWinWarps = kWinThreads / 32;
-constexpr int kWinParts = 32;  // window record parts per (KV head, sequence), at most (api.cu)
+constexpr int kWinParts = 32;  // window record parts per (KV head, sequence), at most
 
 // One CTA per sequence: the new tokens that stay in the window go to their
 // ring slots (converted to fp32), then len += evicted, wlen = min(R, wlen +
@@ -218,6 +218,9 @@ __global__ void __launch_bounds__(kWinThreads) window_record_kernel(
     dst[(size_t)tid * kPartStride + 3] = 0.f;
   }
 }
+
+// The most window record parts of any call (the workspace is sized for it).
+int window_parts_max() { return kWinParts; }
 
 // Window record parts of a window of R tokens: at most kWinParts CTAs per
 // (KV head, sequence), each over a multiple of 16 tokens.
