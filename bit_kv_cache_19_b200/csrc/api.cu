@@ -47,8 +47,8 @@ cudaError_t launch_decode_window(const Plan* const* plans, const CacheMap& cm, i
                                  int n_kv, int bits_k, int bits_v, float* out, void* ws,
                                  size_t ws_bytes, uint32_t* status, cudaStream_t st,
                                  const void* k_new, const void* v_new, int kv_dtype,
-                                 int64_t cap, int early, float* const* wins, int32_t* wlen,
-                                 int R);
+                                 int n_new, int64_t cap, int early, float* const* wins,
+                                 int32_t* wlen, int R);
 
 namespace {
 
@@ -761,7 +761,7 @@ int kvq_append_decode_window(const kvq_cfg* cfg, const void* const* plans_dev, c
   if (rc) return rc;
   if (step_flags & ~KVQ_STEP_EARLY) return fail(KVQ_ERR_ARG, "step_flags 0x%x", step_flags);
   if (R < 0 || R > (1 << 20)) return fail(KVQ_ERR_ARG, "window R %d", R);
-  if (n_new != 1 || R == 0) {  // the two calls
+  if (R == 0 || n_new < 1 || n_new > std::min(R, 64)) {  // the two calls
     rc = kvq_window_append(cfg, plans_dev, k_dev, v_dev, kv_dtype, n_new, cache_dev, len_dev,
                            cap_tokens, win_dev, wlen_dev, R, batch, status_dev, stream);
     if (rc) return rc;
@@ -791,7 +791,7 @@ int kvq_append_decode_window(const kvq_cfg* cfg, const void* const* plans_dev, c
       reinterpret_cast<const Plan* const*>(plans_dev), contiguous_map(cache_dev), len_dev, batch,
       max_len, q_dev, q_dtype, n_q_heads, cfg->n_kv_heads, cfg->bits_k, cfg->bits_v, out_dev,
       reinterpret_cast<uint8_t*>(ws_dev) + rb, ws_bytes - rb, status_dev,
-      reinterpret_cast<cudaStream_t>(stream), k_dev, v_dev, kv_dtype, cap_tokens,
+      reinterpret_cast<cudaStream_t>(stream), k_dev, v_dev, kv_dtype, n_new, cap_tokens,
       (step_flags & KVQ_STEP_EARLY) ? 1 : 0, reinterpret_cast<float* const*>(win_dev), wlen_dev,
       R);
   if (e != cudaSuccess) return cuda_fail(e, "append_decode_window");

@@ -696,17 +696,21 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
     if (tid == 0 && sm.flags) atomicOr(p.status, sm.flags);
   }
   if constexpr (WIN) {
-    // the new tokens into their ring slots, by the CTA that owns the last
-    // packed tile: it has just read the slots of the tokens that left the
-    // window (the append above), and no other CTA reads them in this launch
-    const int ring_split = min(p.n_splits - 1, ((max(L, 1) - 1) / kTile) / p.tiles_per_split);
-    if (step_ok && !bad && split == ring_split) {
+    // the new tokens into their ring slots. New token j takes the slot of
+    // position len0 + w0 + j - R: a token that left the window in this
+    // launch (the CTA that appended it writes the slot, after reading it
+    // above) or one that left before (a free slot, written by the CTA that
+    // owns the last packed tile). No CTA reads those slots otherwise.
+    if (step_ok && !bad) {
+      const int ring_split = min(p.n_splits - 1, ((max(L, 1) - 1) / kTile) / p.tiles_per_split);
       float* wk = p.wins[b];
       float* wv = wk + (size_t)p.R * p.n_kv * kHeadDim;
       for (int e = tid; e < p.n_new * kHeadDim; e += kThreads) {
         const int j = e / kHeadDim, x = e % kHeadDim;
-        const size_t dst =
-            ((size_t)(((int64_t)len0 + sm.w0 + j) % p.R) * p.n_kv + h) * kHeadDim + x;
+        const int64_t pos = (int64_t)len0 + sm.w0 + j - p.R;  // the slot's previous token
+        const int owner = pos < len0 ? ring_split : (int)((pos / kTile) / p.tiles_per_split);
+        if (owner != split) continue;
+        const size_t dst = ((size_t)((pos + p.R) % p.R) * p.n_kv + h) * kHeadDim + x;
         const size_t src = (((size_t)b * p.n_new + j) * p.n_kv + h) * kHeadDim + x;
         wk[dst] = load_as_float(p.k_new, p.kv_dtype, src);
         wv[dst] = load_as_float(p.v_new, p.kv_dtype, src);
@@ -1372,20 +1376,22 @@ cudaError_t launch_decode(const Plan* const* plans, const CacheMap& cm, int32_t*
                            early, theta, rec_out, nullptr, nullptr, 0);
 }
 
-// The window step in one launch: one new token per sequence (n_new = 1), the
-// token leaving a full window quantize-appended from its ring slot, the new
-// token written to the ring, decode over the packed tokens and the window.
+// The window step in one launch: n_new (1..min(R, 64)) new tokens per
+// sequence, the tokens leaving the window quantize-appended from their ring
+// slots, the new tokens written to the ring, decode over the packed tokens
+// and the window.
 cudaError_t launch_decode_window(const Plan* const* plans, const CacheMap& cm, int32_t* len,
                                  int batch, int64_t max_len, const void* q, int q_dtype, int n_q,
                                  int n_kv, int bits_k, int bits_v, float* out, void* ws,
                                  size_t ws_bytes, uint32_t* status, cudaStream_t st,
                                  const void* k_new, const void* v_new, int kv_dtype,
-                                 int64_t cap, int early, float* const* wins, int32_t* wlen,
-                                 int R) {
-  if (!wins || !wlen || R < 1) return cudaErrorInvalidValue;
+                                 int n_new, int64_t cap, int early, float* const* wins,
+                                 int32_t* wlen, int R) {
+  if (!wins || !wlen || R < 1 || n_new < 1 || n_new > std::min(R, kMaxNew))
+    return cudaErrorInvalidValue;
   return launch_decode_any(plans, cm, len, batch, max_len, q, q_dtype, n_q, n_kv, bits_k, bits_v,
-                           out, ws, ws_bytes, status, st, k_new, v_new, kv_dtype, 1, cap, early,
-                           nullptr, nullptr, wins, wlen, R);
+                           out, ws, ws_bytes, status, st, k_new, v_new, kv_dtype, n_new, cap,
+                           early, nullptr, nullptr, wins, wlen, R);
 }
 
 cudaError_t launch_combine(const Plan* const* plans, const float* recs, int n_parts, int batch,

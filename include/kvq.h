@@ -496,14 +496,16 @@ KVQ_API int kvq_decode_attn_window(const kvq_cfg* cfg, const void* const* plans_
 /*
  * A serving step with the recent-token window: kvq_window_append of n_new
  * tokens per sequence, then kvq_decode_attn_window, with the same results
- * (outputs to fp32 rounding). For n_new = 1 and R >= 1 it is one launch of
- * the decode kernel: the CTA that owns the last packed tile quantize-appends
- * the token leaving a full window (read from its ring slot) and then writes
- * the new token into that slot; the window's other tokens (from the ring)
- * and the new one (from k_dev, v_dev) are attended in chunks of 8 by a few
- * CTAs after their tiles, each chunk's record merged with the CTA's own; the
- * last CTA of the sequence to read the lengths writes len += evicted and
- * wlen = min(R, wlen + 1). Other n_new (or R = 0) run the two calls.
+ * (outputs to fp32 rounding). For 1 <= n_new <= min(R, 64) it is one launch
+ * of the decode kernel: the CTAs that own the tiles of the tokens leaving
+ * the window quantize-append them (read from their ring slots) and then
+ * write the new tokens that take those slots; the CTA that owns the last
+ * packed tile writes the new tokens that take free slots; the window's
+ * older tokens (from the ring) and the new ones (from k_dev, v_dev) are
+ * attended in chunks of 8 by a few CTAs after their tiles, each chunk's
+ * record merged with the CTA's own; the last CTA of the sequence to read
+ * the lengths writes len += evicted and wlen = min(R, wlen + n_new). Other
+ * n_new (or R = 0) run the two calls.
  * Arguments as for those calls; the evictions must fit min(cap_tokens,
  * max_len) (else CAPACITY and the sequence's window is left as it was).
  * step_flags: KVQ_STEP_EARLY as for kvq_append_decode (the previous kernel on

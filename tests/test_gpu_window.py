@@ -204,9 +204,27 @@ def _oracle_out(L, kb, vb, T, E, bits_k, bits_v, R, qb, s):
                                                   (1, 100, 2, 2, 8), (100, 130, 4, 3, 16),
                                                   (17, 64, 3, 3, 7)])
 def test_fused_window_steps(R, T0, bits_k, bits_v, G):
-    rng = np.random.default_rng(R * 13 + T0)
-    n_kv, batch, S = 2, 2, 40
-    T = T0 + S
+    _fused_steps(R, T0, bits_k, bits_v, G, [1] * 40)
+
+
+# steps of several tokens in one launch: the tokens leaving the window span
+# tiles and, for the smaller caches, the boundary between two splits (so two
+# CTAs each append some of them and write the new tokens that take their
+# slots); step sizes up to min(R, 64)
+@pytest.mark.parametrize("R,T0,bits_k,bits_v,G,steps", [
+    (48, 300, 3, 3, 8, [5, 17, 32, 1, 48, 7, 3]),
+    (100, 230, 3, 2, 4, [64, 1, 33, 9, 64]),
+    (20, 40, 2, 2, 16, [20, 3, 19, 1, 7]),
+    (300, 100, 3, 3, 8, [64, 64, 50, 64, 2, 64])])
+def test_fused_window_steps_of_several_tokens(R, T0, bits_k, bits_v, G, steps):
+    _fused_steps(R, T0, bits_k, bits_v, G, steps)
+
+
+def _fused_steps(R, T0, bits_k, bits_v, G, steps):
+    rng = np.random.default_rng(R * 13 + T0 + len(steps))
+    n_kv, batch = 2, 2
+    S = len(steps)
+    T = T0 + sum(steps)
     cfg = kvq.make_cfg(n_kv, bits_k, bits_v, v_seed=V_SEED)
     E = np.exp(rng.standard_normal((n_kv, 64)) - np.arange(64) / 8.0)
     plans = kvq.plan_build(cfg, 0, E)
@@ -221,18 +239,19 @@ def test_fused_window_steps(R, T0, bits_k, bits_v, G):
     wsf = torch.zeros(nb, dtype=torch.uint8, device="cuda")
     wsu = torch.zeros(nb, dtype=torch.uint8, device="cuda")
     qbs = synth.to_bf16_bits(rng.standard_normal((S, batch, n_kv * G, 128)))
-    for i in range(S):
-        t = T0 + i
-        k1, v1, q = dev_bf16(kb[:, t:t + 1]), dev_bf16(vb[:, t:t + 1]), dev_bf16(qbs[i])
+    t = T0
+    for i, n in enumerate(steps):
+        k1, v1, q = dev_bf16(kb[:, t:t + n]), dev_bf16(vb[:, t:t + n]), dev_bf16(qbs[i])
         out_f = Lf.append_decode_window(k1, v1, q, ws=wsf).cpu().numpy()
         Lu.append_window(k1, v1)
         out_u = Lu.decode_window(q, ws=wsu).cpu().numpy()
+        t += n
         torch.cuda.synchronize()
         assert Lf.flags() == 0 and Lu.flags() == 0, i
         assert op.rel_err(out_f, out_u) <= 1e-5, i
         if i in (0, 1, S // 2, S - 1):
             for s in range(batch):
-                ref = _oracle_out(Lf, kb, vb, t + 1, E, bits_k, bits_v, R, qbs[i][s], s)
+                ref = _oracle_out(Lf, kb, vb, t, E, bits_k, bits_v, R, qbs[i][s], s)
                 assert op.rel_err(out_f[s], ref) <= TOL, (i, s)
     # the same packed caches, rings and lengths as the two calls
     assert torch.equal(Lf.lens, Lu.lens) and torch.equal(Lf.wlens, Lu.wlens)
